@@ -1,0 +1,434 @@
+"""FLARE forward throughput on B200 (tokens/s) with roofline and baselines.
+
+One step = one FLARE forward (encode partials -> combine -> decode) over the
+million-token workload: B=1, H=16, N=1,048,576, M=256, D=32, bf16 inputs,
+float32 accumulation, scale 1/sqrt(D), synthetic N(0,1) inputs (seed = rank).
+Inputs (3 GiB of K, V, Y) exceed the 126 MB L2, so no flush is needed.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 (torchrun, one process per GPU) each rank runs an independent
+problem of the same size (weak scaling, no data-path collective); rank 0
+prints one JSON line with the job-wide tokens/s over the max time across
+ranks.  ``--impl reference`` times the double-precision CPU oracle (the only
+reference available for this method) on a bounded sample of the workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from flare_inputs import WORKLOADS, make_inputs  # noqa: E402
+
+WORKLOAD = WORKLOADS["c3_fwd_bf16_1M"]
+METRIC = "FLARE fwd tokens/s at N=1M, M=256, H=16, D=32 bf16; % of roofline"
+
+# Nominal B200 unit counts used to derive the exp (MUFU) ceiling: 148 SMs,
+# 16 ex2 results per clock per SM (4 per SM sub-partition), max SM clock
+# 1965 MHz.  The HBM and tensor ceilings come from MEASURED_PEAKS.json.
+SMS = 148
+MUFU_PER_CLK_SM = 16
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0}
+
+THROTTLE_BAD = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, out_path: str | None = None):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.out_path = out_path
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        if self.out_path:
+            with open(self.out_path, "w") as f:
+                f.write(out)
+        return self.parse(out)
+
+    @staticmethod
+    def parse(text: str):
+        sms, maxes, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in text.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sms.append(float(parts[1]))
+                maxes.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sms:
+            return None
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxes),
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+# ------------------------------------------------------------- distributed
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return rank, world, local
+
+
+def dist_max(value: float, world: int, device) -> float:
+    """Max of a host float over ranks (one tiny all-reduce; no data path)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def dist_done(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# -------------------------------------------------------------- CPU oracle
+
+def oracle_sample_rate(target_s: float, w=WORKLOAD, seed: int = 0):
+    """Times the oracle's FLARE forward on a bounded sample of the workload:
+    one (b, h) head with n_s of its N tokens (same M, D, dtype rounding).
+    The sample size is calibrated so the timed run takes about target_s
+    seconds.  Returns (tokens/s of the full workload, description, cores).
+    A workload token carries H heads, so a head-token is 1/H of a token."""
+    import oracle
+    cores = oracle.num_threads()
+
+    def run(n_s):
+        x = make_inputs(1, 1, n_s, w.M, w.D, dtype=w.torch_dtype, seed=seed)
+        t0 = time.perf_counter()
+        oracle.flare_fwd(x["Q"], x["K"], x["V"], w.scale)
+        return time.perf_counter() - t0
+
+    n_cal = 4096
+    t_cal = max(run(n_cal), 1e-4)
+    n_s = int(min(w.N, max(n_cal, n_cal * target_s / t_cal)))
+    t = run(n_s)
+    rate = (n_s / w.H) / t
+    desc = (f"oracle FLARE fwd (double, OpenMP) on 1 of {w.B * w.H} heads, {n_s} of {w.N} "
+            f"tokens, M={w.M}, D={w.D}; {t:.2f} s; tokens/s scaled by 1/H per head-token")
+    return rate, desc, cores, n_s
+
+
+# ------------------------------------------------------------------ ours
+
+def roofline_entry(kernel_ms: dict, peaks: dict, peak_kind: str, w=WORKLOAD):
+    """Roofline of the dominant kernel (largest average duration).
+
+    Both forward kernels are bound by exponentials (MUFU ex2): each computes
+    B*H*N*M of them per launch (encode: softmax over tokens of every latent
+    row; decode: softmax over latents of every token).  Their other ceilings
+    (tensor-pipe FLOPs, HBM bytes) are reported alongside.
+    """
+    name = max(("encode", "decode"), key=lambda k: kernel_ms[k])
+    t = kernel_ms[name] / 1e3
+    exps = w.B * w.H * w.N * w.M
+    clk = float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
+    mufu_peak = SMS * MUFU_PER_CLK_SM * clk / 1e9  # Gexp/s
+    achieved = exps / t / 1e9
+    flops = 4 * w.B * w.H * w.N * w.M * w.D
+    if name == "encode":
+        hbm_bytes = 2 * w.B * w.H * w.N * w.D * 2          # K and V read once
+    else:
+        hbm_bytes = 2 * w.B * w.H * w.N * w.D * 2          # K read, Y written
+    traffic = read_traffic(name)
+    entry = {
+        "bound": "alu", "kernel": f"flare_{name}", "achieved": round(achieved, 1),
+        "peak": round(mufu_peak, 1), "unit": "Gexp/s", "frac": round(achieved / mufu_peak, 4),
+        "traffic": traffic,
+        "peak_basis": f"MUFU ex2: {MUFU_PER_CLK_SM}/clk/SM x {SMS} SMs x {clk / 1e6:.0f} MHz",
+        "algorithmic": {"exps": exps, "tensor_flops": flops, "hbm_bytes": hbm_bytes},
+        "other_ceilings": {
+            "tensor_frac": round(flops / t / 1e12 / float(peaks["bf16_tflops"]), 4),
+            "hbm_frac": round(hbm_bytes / t / 1e9 / float(peaks["hbm_gbs"]), 4),
+            "peaks": f"{peak_kind}: bf16 {peaks['bf16_tflops']} TFLOP/s, "
+                     f"HBM {peaks['hbm_gbs']} GB/s",
+        },
+    }
+    return entry
+
+
+def read_traffic(name: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        rec = d.get(name)
+        if not rec:
+            return None
+        src = os.path.join(ROOT, rec["source"])
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        if h != rec.get("source_sha256"):
+            return None
+        return rec["bytes_per_launch"]
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+def run_ours(args, rank, world, local):
+    import torch
+
+    import rank_latent_attention_flare_b200 as fl
+
+    w = WORKLOAD
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    x = make_inputs(w.B, w.H, w.N, w.M, w.D, dtype=w.torch_dtype, seed=rank)
+    g = {k: v.to(dev) for k, v in x.items()}
+    ws = fl.alloc_workspace(fl.FLARE_OP_FWD, w.B, w.H, w.N, w.M, w.D, w.torch_dtype, dev)
+    Y = torch.empty_like(g["K"])
+    st = torch.cuda.current_stream()
+
+    def step(events=None):
+        if events:
+            events[0].record(st)
+        fl.flare_encode(g["Q"], g["K"], g["V"], w.scale, workspace=ws)
+        if events:
+            events[1].record(st)
+        fl.flare_combine(w.B, w.H, w.N, w.M, w.D, w.torch_dtype, workspace=ws)
+        if events:
+            events[2].record(st)
+        fl.flare_decode(g["Q"], g["K"], w.scale, workspace=ws, out=Y)
+        if events:
+            events[3].record(st)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if fl.device_status(ws) != 0:
+        raise RuntimeError("device wait ran out during warm-up")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler = ClockSampler(local, os.path.join(args.out_dir, "clocks.csv") if args.out_dir else None) \
+        if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.5)
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(st)
+    for i in range(args.steps):
+        step(ev[i])
+    t_end.record(st)
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    clocks = sampler.stop() if sampler else None
+    if fl.device_status(ws) != 0:
+        raise RuntimeError("device wait ran out in the timed region")
+
+    ms_total = t_start.elapsed_time(t_end)
+    ms_total = dist_max(ms_total, world, dev)
+    kernel_ms = {
+        "encode": statistics.mean(e[0].elapsed_time(e[1]) for e in ev),
+        "combine": statistics.mean(e[1].elapsed_time(e[2]) for e in ev),
+        "decode": statistics.mean(e[2].elapsed_time(e[3]) for e in ev),
+    }
+    tokens_per_step = w.B * w.N
+    value = world * tokens_per_step * args.steps / (ms_total / 1e3)
+
+    # End to end through the public API: pinned host inputs -> device ->
+    # flare_fwd -> result back to pinned host memory, every step.
+    e2e = None
+    if not args.no_e2e:
+        hx = {k: v.pin_memory() for k, v in x.items()}
+        hY = torch.empty(Y.shape, dtype=Y.dtype, pin_memory=True)
+        dX = {k: torch.empty_like(v) for k, v in g.items()}
+        e2e_steps = max(1, min(args.steps, args.e2e_steps))
+
+        def e2e_step():
+            for k in ("Q", "K", "V"):
+                dX[k].copy_(hx[k], non_blocking=True)
+            fl.flare_fwd(dX["Q"], dX["K"], dX["V"], w.scale, workspace=ws, out=Y)
+            hY.copy_(Y, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        dist_barrier(world)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for _ in range(e2e_steps):
+            e2e_step()
+        b.record(st)
+        torch.cuda.synchronize()
+        e2e_ms = dist_max(a.elapsed_time(b), world, dev)
+        h2d = sum(hx[k].numel() * hx[k].element_size() for k in ("Q", "K", "V"))
+        e2e = {"value": world * tokens_per_step * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hY.numel() * hY.element_size(),
+               "steps": e2e_steps}
+        del hx, hY, dX
+
+    peaks, peak_kind = load_peaks()
+    roof = roofline_entry(kernel_ms, peaks, peak_kind)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        del g
+        rate, desc, cores, _ = oracle_sample_rate(args.cpu_seconds)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": desc}
+
+    path = fl.fwd_path(w.B, w.H, w.N, w.M, w.D, w.torch_dtype)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"FLARE fwd B={w.B} H={w.H} N={w.N} M={w.M} D={w.D} bf16, "
+                               "fp32 accumulate, scale 1/sqrt(D), i.i.d. N(0,1)",
+                   "global_batch": w.B * world, "seq_len": w.N, "heads": w.H, "latents": w.M,
+                   "head_dim": w.D, "parallelism": f"independent problems x{world}",
+                   "l2": "inputs 3 GiB > 126 MB L2: no flush",
+                   "kernels": "tcgen05" if path == 1 else "cuda-core"},
+        "kernel_ms": {k: round(v, 4) for k, v in kernel_ms.items()},
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 3 * args.steps * world,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------- reference
+
+def run_reference(args, rank, world):
+    """The oracle (double-precision CPU FLARE) timed per step on a bounded
+    sample; rank 0 only."""
+    if rank != 0:
+        return
+    w = WORKLOAD
+    import oracle
+    budget = max(30.0, args.ref_seconds)
+    per_step = budget / (args.steps + args.warmup)
+    _, _, cores, n_s = oracle_sample_rate(per_step)
+    x = make_inputs(1, 1, n_s, w.M, w.D, dtype=w.torch_dtype, seed=0)
+    for _ in range(args.warmup):
+        oracle.flare_fwd(x["Q"], x["K"], x["V"], w.scale)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.flare_fwd(x["Q"], x["K"], x["V"], w.scale)
+    t = time.perf_counter() - t0
+    value = args.steps * (n_s / w.H) / t
+    sample = (f"per step: oracle FLARE fwd on 1 of {w.B * w.H} heads, {n_s} of {w.N} tokens "
+              f"(M={w.M}, D={w.D}); tokens/s scaled by 1/H per head-token")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"FLARE fwd B={w.B} H={w.H} N={w.N} M={w.M} D={w.D} bf16-rounded "
+                               "inputs, scale 1/sqrt(D), i.i.d. N(0,1)",
+                   "global_batch": w.B, "seq_len": w.N, "parallelism": "cpu (OpenMP)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-seconds", type=float, default=120.0)
+    ap.add_argument("--out-dir", default=None, help="where to write the clock samples")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    rank, world, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        dist_done(world)
+
+
+if __name__ == "__main__":
+    main()

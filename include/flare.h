@@ -1,0 +1,184 @@
+/*
+ * flare.h -- C ABI of the FLARE / FLARE++ token-mixing library for B200
+ * (sm_100a).
+ *
+ * The operator (per batch b and head h, scale s, softmax in fp32):
+ *   encode  Z = softmax_N(s Q K^T) V      -- "Flare Fast Low Rank Attention"
+ *           skill page, section 2 "Implement Encode Stage" and section 4
+ *           (latents are the queries, the sequence gives keys and values);
+ *   decode  Y = softmax_M(s K Q^T) Z      -- FLARE arXiv 2508.12594 abstract:
+ *           the second of two SDPA calls, giving an input-input mixing matrix
+ *           W = softmax(s K Q^T) softmax(s Q K^T) of rank at most M;
+ *   FLARE++ Q_dyn = Q + encode(Q, K, V), then encode and decode with Q_dyn
+ *           -- FLARE++ arXiv 2608.11519 abstract (input-conditioned queries
+ *           that correct the learned ones);
+ *   backward: gradients of sum(Y * dY) with respect to Q, K, V.  The pages
+ *           give none; it is the chain rule through both softmax stages,
+ *           with the logits recomputed.
+ *
+ * Conventions shared by every entry point
+ *   - Every tensor pointer is a DEVICE pointer to contiguous row-major data,
+ *     16-byte aligned.  Shapes:
+ *       Q        [H,M,D] when q_batch_stride == 0 (learned latents shared by
+ *                the batch) or [B,H,M,D] when q_batch_stride == H*M*D;
+ *       K, V, Y, dY, dK, dV   [B,H,N,D];
+ *       Z_save   [B,H,M,D] float32;   lse_save  [B,H,M] float32 (natural log
+ *                of the encode softmax denominators, max included);
+ *       Q_dyn_out [B,H,M,D] in the input dtype.
+ *   - dtype: FLARE_F32 or FLARE_BF16 for Q, K, V, Y, dY, dQ, dK, dV.  All
+ *     arithmetic accumulates in float32; bf16 operands feed the tensor cores.
+ *   - Supported sizes: B, H >= 1; N >= 1; D in {16, 32}; M a multiple of 16
+ *     in [16, 256]; B*H*N*D < 2^40.  scale must be finite and > 0.
+ *   - The caller owns every buffer.  The library never allocates or frees
+ *     memory and never synchronises the device (flare_device_status is the
+ *     one exception and says so).  Work is enqueued on `stream` (a
+ *     cudaStream_t; NULL = legacy default stream).
+ *   - `workspace` is caller-allocated device memory of at least
+ *     flare_workspace_size(op, ...) bytes, 256-byte aligned.  Its contents
+ *     need no initialisation and are scratch between calls, except that
+ *     flare_encode -> flare_combine -> flare_decode pass their intermediate
+ *     results through it.  Two calls that run concurrently must not share a
+ *     workspace.
+ *   - Errors are returned, never thrown.  All arguments are validated
+ *     before anything is enqueued, so a call that returns an error other
+ *     than FLARE_ERR_CUDA has no side effect.  FLARE_ERR_CUDA means a launch
+ *     failed; the CUDA error is left for cudaGetLastError.
+ *   - Every wait inside a kernel is bounded.  A wait that runs out sets an
+ *     error word in the workspace header instead of hanging; read it with
+ *     flare_device_status after the stream has been synchronised.
+ *   - The library holds no mutable global state and is thread-safe.
+ */
+#ifndef FLARE_H_
+#define FLARE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FLARE_API __attribute__((visibility("default")))
+#else
+#define FLARE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { FLARE_F32 = 0, FLARE_BF16 = 1 } flare_dtype_t;
+
+typedef enum {
+  FLARE_OK = 0,
+  FLARE_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or scale */
+  FLARE_ERR_UNSUPPORTED = 2,   /* valid but unsupported D, M or stride      */
+  FLARE_ERR_WORKSPACE = 3,     /* workspace missing, misaligned or too small */
+  FLARE_ERR_CUDA = 4,          /* a kernel launch failed                    */
+  FLARE_ERR_DEVICE_TIMEOUT = 5 /* a kernel's bounded wait ran out           */
+} flare_status_t;
+
+typedef enum { FLARE_OP_FWD = 0, FLARE_OP_PP_FWD = 1, FLARE_OP_BWD = 2 } flare_op_t;
+
+/* Library ABI version (major*10000 + minor*100 + patch). */
+FLARE_API int flare_version(void);
+
+/* Human-readable text for a status code (static storage, never NULL). */
+FLARE_API const char* flare_status_string(flare_status_t status);
+
+/*
+ * Bytes of workspace needed by `op` for these sizes on the current device,
+ * or 0 when the sizes are invalid or unsupported.  The stage calls
+ * flare_encode / flare_combine / flare_decode use FLARE_OP_FWD's size.
+ */
+FLARE_API size_t flare_workspace_size(flare_op_t op, int64_t B, int64_t H, int64_t N, int64_t M,
+                            int64_t D, flare_dtype_t dtype);
+
+/*
+ * FLARE forward: Y = decode(Q, K, encode(Q, K, V)).
+ * Q, K, V in; Y out.  Z_save / lse_save are optional (NULL for inference)
+ * and are what flare_bwd needs.  Equivalent to flare_encode, flare_combine
+ * and flare_decode in sequence on the same workspace.
+ */
+FLARE_API flare_status_t flare_fwd(const void* Q, int64_t q_batch_stride, const void* K, const void* V,
+                         void* Y, int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
+                         flare_dtype_t dtype, float scale, float* Z_save, float* lse_save,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * FLARE++ forward with learned latents Q [H,M,D] (FLARE++ abstract):
+ *   Q_dyn = Q + encode(Q, K, V);  Z = encode(Q_dyn, K, V);  Y = decode(Q_dyn, K, Z).
+ * Q_dyn is rounded to the input dtype before it is used (it is the operand
+ * of both later stages).  Q_dyn_out (optional) receives it; Z_save and
+ * lse_save (optional) receive the second encode's Z and lse.
+ */
+FLARE_API flare_status_t flare_pp_fwd(const void* Q, const void* K, const void* V, void* Y,
+                            void* Q_dyn_out, int64_t B, int64_t H, int64_t N, int64_t M,
+                            int64_t D, flare_dtype_t dtype, float scale, float* Z_save,
+                            float* lse_save, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/*
+ * FLARE backward (fixed latents): gradients of sum(Y * dY).
+ * Inputs: Q, K, V, dY and the forward's Z_save, lse_save (both required).
+ * Outputs in the input dtype: dQ ([H,M,D] summed over the batch when
+ * q_batch_stride == 0, else [B,H,M,D]), dK, dV.  The logits of both stages
+ * are recomputed; every reduction is in a fixed order, so results are
+ * bitwise reproducible run to run.
+ */
+FLARE_API flare_status_t flare_bwd(const void* Q, int64_t q_batch_stride, const void* K, const void* V,
+                         const void* dY, const float* Z_save, const float* lse_save, void* dQ,
+                         void* dK, void* dV, int64_t B, int64_t H, int64_t N, int64_t M,
+                         int64_t D, flare_dtype_t dtype, float scale, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/*
+ * Stage 1 of the forward -- encode partials.  For each (b, h) and each
+ * chunk of tokens, the running softmax max m, denominator l and weighted
+ * value sum acc of every latent row (skill page section 2; online softmax
+ * across token tiles).  Results stay in the workspace.
+ */
+FLARE_API flare_status_t flare_encode(const void* Q, int64_t q_batch_stride, const void* K, const void* V,
+                            int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
+                            flare_dtype_t dtype, float scale, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/*
+ * Stage 2 -- merge the chunk partials of flare_encode (log-sum-exp merge):
+ * Z = sum_c acc_c 2^(m_c - m*) / sum_c l_c 2^(m_c - m*).  Writes Z to the
+ * workspace (float32 and the bf16 operand copy used by the decode) and, when
+ * non-NULL, to Z_save and lse_save.  Must follow flare_encode with the same
+ * sizes, dtype and workspace.
+ */
+FLARE_API flare_status_t flare_combine(int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
+                             flare_dtype_t dtype, float* Z_save, float* lse_save,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Stage 3 -- decode: Y = softmax_M(s K Q^T) Z with the Z that flare_combine
+ * left in the workspace (FLARE abstract, second SDPA call).  The N x M
+ * logits never leave the chip.
+ */
+FLARE_API flare_status_t flare_decode(const void* Q, int64_t q_batch_stride, const void* K, void* Y,
+                            int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
+                            flare_dtype_t dtype, float scale, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/*
+ * Reads and clears the device error word in the workspace header.  This
+ * call SYNCHRONISES `stream`.  Returns FLARE_OK, FLARE_ERR_DEVICE_TIMEOUT
+ * (a bounded wait ran out; *detail receives the site code) or
+ * FLARE_ERR_CUDA.  detail may be NULL.
+ */
+FLARE_API flare_status_t flare_device_status(void* workspace, size_t workspace_bytes, uint32_t* detail,
+                                   void* stream);
+
+/*
+ * Which kernel family a forward call with these sizes uses:
+ * 1 = tcgen05/TMEM/TMA tensor-core kernels, 0 = CUDA-core kernels.
+ * Returns -1 for invalid or unsupported sizes.
+ */
+FLARE_API int flare_fwd_path(int64_t B, int64_t H, int64_t N, int64_t M, int64_t D, flare_dtype_t dtype);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLARE_H_ */

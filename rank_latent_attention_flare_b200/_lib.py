@@ -1,0 +1,86 @@
+"""ctypes declarations of the C ABI in include/flare.h.
+
+Loads the in-tree ``libflare.so``.  There is no fallback: if the library is
+missing or does not load, importing the binding raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libflare.so")
+
+FLARE_F32 = 0
+FLARE_BF16 = 1
+
+FLARE_OP_FWD = 0
+FLARE_OP_PP_FWD = 1
+FLARE_OP_BWD = 2
+
+STATUS_NAMES = {
+    0: "FLARE_OK",
+    1: "FLARE_ERR_INVALID_ARG",
+    2: "FLARE_ERR_UNSUPPORTED",
+    3: "FLARE_ERR_WORKSPACE",
+    4: "FLARE_ERR_CUDA",
+    5: "FLARE_ERR_DEVICE_TIMEOUT",
+}
+
+# Every symbol include/flare.h declares, with (restype, argtypes).
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int
+_f32 = ctypes.c_float
+_sz = ctypes.c_size_t
+_u32p = ctypes.POINTER(ctypes.c_uint32)
+
+SIGNATURES = {
+    "flare_version": (_i32, []),
+    "flare_status_string": (ctypes.c_char_p, [_i32]),
+    "flare_workspace_size": (_sz, [_i32, _i64, _i64, _i64, _i64, _i64, _i32]),
+    "flare_fwd": (_i32, [_vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i32, _f32,
+                         _vp, _vp, _vp, _sz, _vp]),
+    "flare_pp_fwd": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i32, _f32,
+                            _vp, _vp, _vp, _sz, _vp]),
+    "flare_bwd": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                         _i64, _i64, _i32, _f32, _vp, _sz, _vp]),
+    "flare_encode": (_i32, [_vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i32, _f32, _vp,
+                            _sz, _vp]),
+    "flare_combine": (_i32, [_i64, _i64, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "flare_decode": (_i32, [_vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i32, _f32, _vp,
+                            _sz, _vp]),
+    "flare_device_status": (_i32, [_vp, _sz, _u32p, _vp]),
+    "flare_fwd_path": (_i32, [_i64, _i64, _i64, _i64, _i64, _i32]),
+}
+
+_lib = None
+
+
+class FlareError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        text = STATUS_NAMES.get(status, f"status {status}")
+        super().__init__(f"{where}: {text}")
+
+
+def load() -> ctypes.CDLL:
+    """Load libflare.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m rank_latent_attention_flare_b200.build` (nvcc, sm_100a)")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def check(status: int, where: str) -> None:
+    if status != 0:
+        raise FlareError(status, where)

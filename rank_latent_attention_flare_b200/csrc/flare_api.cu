@@ -1,0 +1,287 @@
+// C ABI of the FLARE library: argument validation, workspace carving and
+// launch orchestration on the caller's stream.  No allocation, no
+// synchronisation (except flare_device_status, documented as such), no
+// global mutable state.
+#include <string.h>
+
+#include "flare_internal.cuh"
+
+using namespace flare;
+
+namespace {
+
+int current_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 148;  // B200
+  }
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return n;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+flare_status_t check_sizes(int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
+                           flare_dtype_t dt) {
+  if (B < 1 || H < 1 || N < 1 || M < 1 || D < 1) return FLARE_ERR_INVALID_ARG;
+  if (dt != FLARE_F32 && dt != FLARE_BF16) return FLARE_ERR_INVALID_ARG;
+  if (B > (1LL << 20) || H > (1LL << 16) || N > (1LL << 34)) return FLARE_ERR_INVALID_ARG;
+  if (D != 16 && D != 32) return FLARE_ERR_UNSUPPORTED;
+  if (M < 16 || M > 256 || (M % 16) != 0) return FLARE_ERR_UNSUPPORTED;
+  const double elems = (double)B * (double)H * (double)N * (double)D;
+  if (elems >= 1099511627776.0) return FLARE_ERR_INVALID_ARG;  // 2^40
+  if (B * H > 65535) return FLARE_ERR_UNSUPPORTED;               // grid.y limit
+  return FLARE_OK;
+}
+
+flare_status_t check_scale(float scale) {
+  return (std::isfinite(scale) && scale > 0.f) ? FLARE_OK : FLARE_ERR_INVALID_ARG;
+}
+
+flare_status_t check_ptr(const void* p) {
+  return (p != nullptr && aligned16(p)) ? FLARE_OK : FLARE_ERR_INVALID_ARG;
+}
+
+flare_status_t check_opt_ptr(const void* p) {
+  return (p == nullptr || aligned16(p)) ? FLARE_OK : FLARE_ERR_INVALID_ARG;
+}
+
+flare_status_t check_qbs(int64_t qbs, int64_t H, int64_t M, int64_t D) {
+  return (qbs == 0 || qbs == H * M * D) ? FLARE_OK : FLARE_ERR_UNSUPPORTED;
+}
+
+flare_status_t check_ws(const void* ws, size_t bytes, size_t need) {
+  if (ws == nullptr || ((uintptr_t)ws & 255u) != 0) return FLARE_ERR_WORKSPACE;
+  return bytes >= need ? FLARE_OK : FLARE_ERR_WORKSPACE;
+}
+
+#define FLARE_TRY(x)                    \
+  do {                                  \
+    flare_status_t s_ = (x);            \
+    if (s_ != FLARE_OK) return s_;      \
+  } while (0)
+
+#define FLARE_CUDA(x)                                 \
+  do {                                                \
+    if ((x) != cudaSuccess) return FLARE_ERR_CUDA;    \
+  } while (0)
+
+flare_status_t reset_error_word(char* ws, cudaStream_t st) {
+  FLARE_CUDA(cudaMemsetAsync(ws, 0, 4, st));
+  return FLARE_OK;
+}
+
+// Stage launchers shared by the public entry points (arguments validated).
+flare_status_t run_encode(const void* Q, int64_t qbs, const void* K, const void* V,
+                          const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,
+                          char* ws, cudaStream_t st) {
+  const Path path = choose_path(d.M, d.D, dt);
+  float* pml = (float*)(ws + L.part_ml);
+  float* pacc = (float*)(ws + L.part_acc);
+  if (path.tc_fwd)
+    FLARE_CUDA(launch_tc_encode(Q, qbs, K, V, d, scale, L.enc, pml, pacc, (uint32_t*)(ws + L.hdr),
+                                st));
+  else
+    FLARE_CUDA(launch_simt_encode(Q, qbs, K, V, d, dt, scale, L.enc, pml, pacc, st));
+  return FLARE_OK;
+}
+
+flare_status_t run_combine(const Dims& d, flare_dtype_t dt, float* Z_save, float* lse_save,
+                           const void* Qpp, void* Qdyn, const WsLayout& L, char* ws,
+                           cudaStream_t st) {
+  FLARE_CUDA(launch_combine(d, dt, L.enc.slots_per_bh(), (const float*)(ws + L.part_ml),
+                            (const float*)(ws + L.part_acc), (float*)(ws + L.zf),
+                            (__nv_bfloat16*)(ws + L.zb), Z_save, lse_save, Qpp, Qdyn, st));
+  return FLARE_OK;
+}
+
+flare_status_t run_decode(const void* Q, int64_t qbs, const void* K, void* Y, const Dims& d,
+                          flare_dtype_t dt, float scale, const WsLayout& L, char* ws,
+                          cudaStream_t st, int sms) {
+  const Path path = choose_path(d.M, d.D, dt);
+  if (path.tc_fwd)
+    FLARE_CUDA(launch_tc_decode(Q, qbs, K, (const __nv_bfloat16*)(ws + L.zb), Y, d, scale,
+                                decode_plan(d.BH(), d.N, sms), (uint32_t*)(ws + L.hdr), st));
+  else
+    FLARE_CUDA(launch_simt_decode(Q, qbs, K, (const float*)(ws + L.zf), Y, d, dt, scale, st));
+  return FLARE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int flare_version(void) { return 100; }
+
+const char* flare_status_string(flare_status_t s) {
+  switch (s) {
+    case FLARE_OK: return "FLARE_OK";
+    case FLARE_ERR_INVALID_ARG: return "FLARE_ERR_INVALID_ARG: invalid pointer, size or scale";
+    case FLARE_ERR_UNSUPPORTED: return "FLARE_ERR_UNSUPPORTED: unsupported D, M or Q stride";
+    case FLARE_ERR_WORKSPACE: return "FLARE_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case FLARE_ERR_CUDA: return "FLARE_ERR_CUDA: a CUDA launch failed";
+    case FLARE_ERR_DEVICE_TIMEOUT: return "FLARE_ERR_DEVICE_TIMEOUT: a bounded device wait ran out";
+  }
+  return "FLARE: unknown status";
+}
+
+size_t flare_workspace_size(flare_op_t op, int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
+                            flare_dtype_t dt) {
+  if (op != FLARE_OP_FWD && op != FLARE_OP_PP_FWD && op != FLARE_OP_BWD) return 0;
+  if (check_sizes(B, H, N, M, D, dt) != FLARE_OK) return 0;
+  return ws_layout(op, B, H, N, M, D, dt, current_sm_count()).total;
+}
+
+int flare_fwd_path(int64_t B, int64_t H, int64_t N, int64_t M, int64_t D, flare_dtype_t dt) {
+  if (check_sizes(B, H, N, M, D, dt) != FLARE_OK) return -1;
+  return choose_path(M, D, dt).tc_fwd ? 1 : 0;
+}
+
+flare_status_t flare_encode(const void* Q, int64_t qbs, const void* K, const void* V, int64_t B,
+                            int64_t H, int64_t N, int64_t M, int64_t D, flare_dtype_t dt,
+                            float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  FLARE_TRY(check_sizes(B, H, N, M, D, dt));
+  FLARE_TRY(check_scale(scale));
+  FLARE_TRY(check_ptr(Q));
+  FLARE_TRY(check_ptr(K));
+  FLARE_TRY(check_ptr(V));
+  FLARE_TRY(check_qbs(qbs, H, M, D));
+  const WsLayout L = ws_layout(FLARE_OP_FWD, B, H, N, M, D, dt, current_sm_count());
+  FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  char* ws = (char*)workspace;
+  cudaStream_t st = (cudaStream_t)stream;
+  FLARE_TRY(reset_error_word(ws, st));
+  return run_encode(Q, qbs, K, V, Dims{B, H, N, M, D}, dt, scale, L, ws, st);
+}
+
+flare_status_t flare_combine(int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
+                             flare_dtype_t dt, float* Z_save, float* lse_save, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  FLARE_TRY(check_sizes(B, H, N, M, D, dt));
+  FLARE_TRY(check_opt_ptr(Z_save));
+  FLARE_TRY(check_opt_ptr(lse_save));
+  const WsLayout L = ws_layout(FLARE_OP_FWD, B, H, N, M, D, dt, current_sm_count());
+  FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  return run_combine(Dims{B, H, N, M, D}, dt, Z_save, lse_save, nullptr, nullptr, L,
+                     (char*)workspace, (cudaStream_t)stream);
+}
+
+flare_status_t flare_decode(const void* Q, int64_t qbs, const void* K, void* Y, int64_t B,
+                            int64_t H, int64_t N, int64_t M, int64_t D, flare_dtype_t dt,
+                            float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  FLARE_TRY(check_sizes(B, H, N, M, D, dt));
+  FLARE_TRY(check_scale(scale));
+  FLARE_TRY(check_ptr(Q));
+  FLARE_TRY(check_ptr(K));
+  FLARE_TRY(check_ptr(Y));
+  FLARE_TRY(check_qbs(qbs, H, M, D));
+  const int sms = current_sm_count();
+  const WsLayout L = ws_layout(FLARE_OP_FWD, B, H, N, M, D, dt, sms);
+  FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  return run_decode(Q, qbs, K, Y, Dims{B, H, N, M, D}, dt, scale, L, (char*)workspace,
+                    (cudaStream_t)stream, sms);
+}
+
+flare_status_t flare_fwd(const void* Q, int64_t qbs, const void* K, const void* V, void* Y,
+                         int64_t B, int64_t H, int64_t N, int64_t M, int64_t D, flare_dtype_t dt,
+                         float scale, float* Z_save, float* lse_save, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  FLARE_TRY(check_sizes(B, H, N, M, D, dt));
+  FLARE_TRY(check_scale(scale));
+  FLARE_TRY(check_ptr(Q));
+  FLARE_TRY(check_ptr(K));
+  FLARE_TRY(check_ptr(V));
+  FLARE_TRY(check_ptr(Y));
+  FLARE_TRY(check_opt_ptr(Z_save));
+  FLARE_TRY(check_opt_ptr(lse_save));
+  FLARE_TRY(check_qbs(qbs, H, M, D));
+  const int sms = current_sm_count();
+  const WsLayout L = ws_layout(FLARE_OP_FWD, B, H, N, M, D, dt, sms);
+  FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  char* ws = (char*)workspace;
+  cudaStream_t st = (cudaStream_t)stream;
+  const Dims d{B, H, N, M, D};
+  FLARE_TRY(reset_error_word(ws, st));
+  FLARE_TRY(run_encode(Q, qbs, K, V, d, dt, scale, L, ws, st));
+  FLARE_TRY(run_combine(d, dt, Z_save, lse_save, nullptr, nullptr, L, ws, st));
+  return run_decode(Q, qbs, K, Y, d, dt, scale, L, ws, st, sms);
+}
+
+flare_status_t flare_pp_fwd(const void* Q, const void* K, const void* V, void* Y,
+                            void* Q_dyn_out, int64_t B, int64_t H, int64_t N, int64_t M,
+                            int64_t D, flare_dtype_t dt, float scale, float* Z_save,
+                            float* lse_save, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  FLARE_TRY(check_sizes(B, H, N, M, D, dt));
+  FLARE_TRY(check_scale(scale));
+  FLARE_TRY(check_ptr(Q));
+  FLARE_TRY(check_ptr(K));
+  FLARE_TRY(check_ptr(V));
+  FLARE_TRY(check_ptr(Y));
+  FLARE_TRY(check_opt_ptr(Q_dyn_out));
+  FLARE_TRY(check_opt_ptr(Z_save));
+  FLARE_TRY(check_opt_ptr(lse_save));
+  const int sms = current_sm_count();
+  const WsLayout L = ws_layout(FLARE_OP_PP_FWD, B, H, N, M, D, dt, sms);
+  FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  char* ws = (char*)workspace;
+  cudaStream_t st = (cudaStream_t)stream;
+  const Dims d{B, H, N, M, D};
+  void* qdyn = Q_dyn_out ? Q_dyn_out : (void*)(ws + L.qdyn);
+  const int64_t qdyn_bs = H * M * D;
+  FLARE_TRY(reset_error_word(ws, st));
+  // Z1 = encode(Q, K, V); Q_dyn = Q + Z1 (written by the combine)
+  FLARE_TRY(run_encode(Q, 0, K, V, d, dt, scale, L, ws, st));
+  FLARE_TRY(run_combine(d, dt, nullptr, nullptr, Q, qdyn, L, ws, st));
+  // Z = encode(Q_dyn, K, V); Y = decode(Q_dyn, K, Z)
+  FLARE_TRY(run_encode(qdyn, qdyn_bs, K, V, d, dt, scale, L, ws, st));
+  FLARE_TRY(run_combine(d, dt, Z_save, lse_save, nullptr, nullptr, L, ws, st));
+  return run_decode(qdyn, qdyn_bs, K, Y, d, dt, scale, L, ws, st, sms);
+}
+
+flare_status_t flare_bwd(const void* Q, int64_t qbs, const void* K, const void* V,
+                         const void* dY, const float* Z_save, const float* lse_save, void* dQ,
+                         void* dK, void* dV, int64_t B, int64_t H, int64_t N, int64_t M,
+                         int64_t D, flare_dtype_t dt, float scale, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  FLARE_TRY(check_sizes(B, H, N, M, D, dt));
+  FLARE_TRY(check_scale(scale));
+  FLARE_TRY(check_ptr(Q));
+  FLARE_TRY(check_ptr(K));
+  FLARE_TRY(check_ptr(V));
+  FLARE_TRY(check_ptr(dY));
+  FLARE_TRY(check_ptr(Z_save));
+  FLARE_TRY(check_ptr(lse_save));
+  FLARE_TRY(check_ptr(dQ));
+  FLARE_TRY(check_ptr(dK));
+  FLARE_TRY(check_ptr(dV));
+  FLARE_TRY(check_qbs(qbs, H, M, D));
+  const WsLayout L = ws_layout(FLARE_OP_BWD, B, H, N, M, D, dt, current_sm_count());
+  FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  char* ws = (char*)workspace;
+  cudaStream_t st = (cudaStream_t)stream;
+  FLARE_TRY(reset_error_word(ws, st));
+  FLARE_CUDA(launch_bwd(Q, qbs, K, V, dY, Z_save, lse_save, dQ, dK, dV, Dims{B, H, N, M, D}, dt,
+                        scale, L, ws, st));
+  return FLARE_OK;
+}
+
+flare_status_t flare_device_status(void* workspace, size_t workspace_bytes, uint32_t* detail,
+                                   void* stream) {
+  if (workspace == nullptr || workspace_bytes < 256 || ((uintptr_t)workspace & 255u) != 0)
+    return FLARE_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, workspace, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return FLARE_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return FLARE_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, 4, st) != cudaSuccess) return FLARE_ERR_CUDA;
+  if (detail) *detail = word;
+  return word == 0 ? FLARE_OK : FLARE_ERR_DEVICE_TIMEOUT;
+}
+
+}  // extern "C"

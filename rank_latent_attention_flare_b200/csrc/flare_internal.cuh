@@ -1,0 +1,217 @@
+// Internal declarations shared by the FLARE CUDA sources: workspace layout,
+// work partitioning, device helpers and kernel launchers.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cmath>
+
+#include "flare.h"
+
+namespace flare {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// Error sites recorded in the workspace header when a bounded wait runs out.
+enum ErrorSite : uint32_t {
+  kErrNone = 0,
+  kErrEncTmaWait = 0x101,
+  kErrEncMmaWait = 0x102,
+  kErrEncSoftmaxWait = 0x103,
+  kErrDecTmaWait = 0x201,
+  kErrDecMmaWait = 0x202,
+  kErrDecSoftmaxWait = 0x203,
+  kErrTmemAlloc = 0x301,
+};
+
+// ------------------------------------------------------------------ planning
+
+// Split of one (b, h) token range into `chunks` contiguous chunks of
+// `chunk_tiles` tiles of `tile` tokens (the last chunk may be shorter).
+struct ChunkPlan {
+  int tile = 0;
+  int64_t tiles_per_bh = 0;
+  int chunks = 0;
+  int64_t chunk_tiles = 0;
+  int sub = 1;  // partial records per chunk (tensor-core encode with M=128: 2)
+  int64_t chunk_tokens() const { return chunk_tiles * tile; }
+  int slots_per_bh() const { return chunks * sub; }
+};
+
+// Picks the chunk count that minimises (waves x tiles per chunk), where a
+// wave is `cta_slots` concurrently resident CTAs and each CTA pays
+// `overhead_tiles` of set-up.  Deterministic for given arguments.
+inline ChunkPlan plan_chunks(int64_t BH, int64_t N, int tile, int64_t cta_slots,
+                             double overhead_tiles, int64_t max_chunks) {
+  ChunkPlan p;
+  p.tile = tile;
+  p.tiles_per_bh = (N + tile - 1) / tile;
+  int64_t hi = p.tiles_per_bh;
+  if (hi > max_chunks) hi = max_chunks;
+  double best = 1e300;
+  int64_t best_c = 1, best_per = p.tiles_per_bh;
+  for (int64_t c = 1; c <= hi; ++c) {
+    int64_t per = (p.tiles_per_bh + c - 1) / c;
+    int64_t ceff = (p.tiles_per_bh + per - 1) / per;
+    if (ceff != c) continue;
+    int64_t waves = (BH * ceff + cta_slots - 1) / cta_slots;
+    double cost = (double)waves * ((double)per + overhead_tiles);
+    if (cost < best - 1e-9) {
+      best = cost;
+      best_c = ceff;
+      best_per = per;
+    }
+  }
+  p.chunks = (int)best_c;
+  p.chunk_tiles = best_per;
+  return p;
+}
+
+// Which kernels a call uses.
+struct Path {
+  bool tc_fwd = false;  // tcgen05 encode + decode
+};
+
+inline Path choose_path(int64_t M, int64_t D, flare_dtype_t dt) {
+  Path p;
+  p.tc_fwd = false && (dt == FLARE_BF16) && (M == 128 || M == 256) && (D == 16 || D == 32);
+  return p;
+}
+
+constexpr int kSimtEncTile = 64;
+constexpr int kSimtEncThreads = 256;
+constexpr int kSimtDecThreads = 128;
+constexpr int kTcTile = 128;
+constexpr int kBwdTile = 256;
+
+inline ChunkPlan encode_plan(int64_t BH, int64_t N, int64_t M, int64_t D, flare_dtype_t dt,
+                             int sms) {
+  Path path = choose_path(M, D, dt);
+  if (path.tc_fwd) {
+    ChunkPlan p = plan_chunks(BH, N, kTcTile, sms, 6.0, 16 * (int64_t)sms);
+    p.sub = (M == 128) ? 2 : 1;
+    return p;
+  }
+  return plan_chunks(BH, N, kSimtEncTile, 4LL * sms, 2.0, 64 * (int64_t)sms);
+}
+
+inline ChunkPlan decode_plan(int64_t BH, int64_t N, int sms) {
+  return plan_chunks(BH, N, kTcTile, sms, 6.0, 16 * (int64_t)sms);
+}
+
+inline ChunkPlan bwd_plan(int64_t BH, int64_t N, int sms) {
+  return plan_chunks(BH, N, kBwdTile, 2LL * sms, 1.0, 16 * (int64_t)sms);
+}
+
+// ------------------------------------------------------------- workspace
+
+struct WsLayout {
+  size_t hdr = 0;       // uint32 error word (256 bytes reserved)
+  size_t part_ml = 0;   // [BH*slots][M][2] float: running max (log2 units), sum
+  size_t part_acc = 0;  // [BH*slots][M][D] float
+  size_t zf = 0;        // [BH][M][D] float  Z
+  size_t zb = 0;        // [BH][M][D] bf16   Z operand copy for the decode
+  size_t qdyn = 0;      // [BH][M][D] dtype  FLARE++ corrected queries
+  size_t dkf = 0;       // [BH][N][D] float  decode-stage part of dK
+  size_t dqp = 0;       // [2][BH*chunks][M][D] float dQ partials (decode, encode)
+  size_t dzp = 0;       // [BH*chunks][M][D] float  dZ partials
+  size_t dz = 0;        // [BH][M][D] float
+  size_t delta = 0;     // [BH][M] float  rowsum(dZ * Z)
+  size_t total = 0;
+  ChunkPlan enc, bwd;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+inline WsLayout ws_layout(flare_op_t op, int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
+                          flare_dtype_t dt, int sms) {
+  WsLayout L;
+  const int64_t BH = B * H;
+  const size_t esz = (dt == FLARE_F32) ? 4 : 2;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L.enc = encode_plan(BH, N, M, D, dt, sms);
+  const int64_t slots = BH * L.enc.slots_per_bh();
+  L.hdr = take(256);
+  L.part_ml = take((size_t)slots * M * 2 * 4);
+  L.part_acc = take((size_t)slots * M * D * 4);
+  L.zf = take((size_t)BH * M * D * 4);
+  L.zb = take((size_t)BH * M * D * 2);
+  if (op == FLARE_OP_PP_FWD) L.qdyn = take((size_t)BH * M * D * esz);
+  if (op == FLARE_OP_BWD) {
+    L.bwd = bwd_plan(BH, N, sms);
+    const int64_t bslots = BH * L.bwd.chunks;
+    L.dkf = take((size_t)BH * N * D * 4);
+    L.dqp = take((size_t)2 * bslots * M * D * 4);
+    L.dzp = take((size_t)bslots * M * D * 4);
+    L.dz = take((size_t)BH * M * D * 4);
+    L.delta = take((size_t)BH * M * 4);
+  }
+  L.total = off;
+  return L;
+}
+
+// ------------------------------------------------------------ device helpers
+
+template <typename T>
+__device__ __forceinline__ float to_f(T x);
+template <>
+__device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+
+template <typename T>
+__device__ __forceinline__ T from_f(float x);
+template <>
+__device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+__host__ __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+__device__ __forceinline__ void record_error(uint32_t* err, uint32_t site) {
+  if (err) atomicCAS(err, 0u, site);
+}
+
+// ------------------------------------------------------------ launchers
+// Each returns cudaSuccess or the launch error.
+
+struct Dims {
+  int64_t B, H, N, M, D;
+  int64_t BH() const { return B * H; }
+};
+
+cudaError_t launch_simt_encode(const void* Q, int64_t qbs, const void* K, const void* V,
+                               const Dims& d, flare_dtype_t dt, float scale,
+                               const ChunkPlan& plan, float* part_ml, float* part_acc,
+                               cudaStream_t st);
+cudaError_t launch_simt_decode(const void* Q, int64_t qbs, const void* K, const float* Zf,
+                               void* Y, const Dims& d, flare_dtype_t dt, float scale,
+                               cudaStream_t st);
+cudaError_t launch_combine(const Dims& d, flare_dtype_t dt, int slots_per_bh,
+                           const float* part_ml, const float* part_acc, float* Zf,
+                           __nv_bfloat16* Zb, float* Z_save, float* lse_save, const void* Qpp,
+                           void* Qdyn, cudaStream_t st);
+cudaError_t launch_tc_encode(const void* Q, int64_t qbs, const void* K, const void* V,
+                             const Dims& d, float scale, const ChunkPlan& plan,
+                             float* part_ml, float* part_acc, uint32_t* err, cudaStream_t st);
+cudaError_t launch_tc_decode(const void* Q, int64_t qbs, const void* K,
+                             const __nv_bfloat16* Zb, void* Y, const Dims& d, float scale,
+                             const ChunkPlan& plan, uint32_t* err, cudaStream_t st);
+cudaError_t launch_bwd(const void* Q, int64_t qbs, const void* K, const void* V, const void* dY,
+                       const float* Z, const float* lse, void* dQ, void* dK, void* dV,
+                       const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,
+                       char* ws, cudaStream_t st);
+
+}  // namespace flare

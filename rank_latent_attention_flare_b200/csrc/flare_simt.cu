@@ -1,0 +1,249 @@
+// CUDA-core (FFMA + exp2f) kernels of the FLARE forward: encode partials,
+// partial combine and decode.  They serve float32 inputs (where the
+// tensor-core path's bf16 operand rounding would break a 1e-5 tolerance)
+// and bf16 shapes the tensor-core kernels do not cover.
+//
+// Encode, per (b, h) and latent m ("Flare Fast Low Rank Attention" skill
+// page, section 2): Z[m] = sum_n softmax_n(s Q[m].K[n]) V[n], evaluated as an
+// online softmax over token tiles.  Logits are kept in log2 units
+// (s * log2(e) folded into Q) so every exponential is one exp2.
+// Decode (FLARE arXiv abstract, second SDPA call): Y[n] = softmax_m(s K[n].Q[m]) Z.
+#include "flare_internal.cuh"
+
+namespace flare {
+namespace {
+
+// One CTA = one chunk of tokens of one (b, h); thread m owns latent row m.
+template <typename T, int D>
+__global__ void __launch_bounds__(kSimtEncThreads)
+    simt_encode_kernel(const T* __restrict__ Q, int64_t q_bstride, const T* __restrict__ K,
+                       const T* __restrict__ V, int H, int64_t N, int M, float c,
+                       int64_t chunk_tokens, float* __restrict__ part_ml,
+                       float* __restrict__ part_acc) {
+  __shared__ float ks[kSimtEncTile][D];
+  __shared__ float vs[kSimtEncTile][D];
+  const int chunk = blockIdx.x;
+  const int chunks = gridDim.x;
+  const int64_t bh = blockIdx.y;
+  const int64_t b = bh / H, h = bh % H;
+  const int64_t n0 = (int64_t)chunk * chunk_tokens;
+  const int64_t n1 = min(N, n0 + chunk_tokens);
+  const T* Kb = K + bh * N * D;
+  const T* Vb = V + bh * N * D;
+  const int m = threadIdx.x;
+  const bool active = m < M;
+
+  float q[D];
+#pragma unroll
+  for (int d = 0; d < D; ++d)
+    q[d] = active ? to_f(Q[b * q_bstride + ((int64_t)h * M + m) * D + d]) * c : 0.f;
+  float mref = -INFINITY, l = 0.f;
+  float acc[D];
+#pragma unroll
+  for (int d = 0; d < D; ++d) acc[d] = 0.f;
+
+  for (int64_t t0 = n0; t0 < n1; t0 += kSimtEncTile) {
+    const int nt = (int)imin64(kSimtEncTile, n1 - t0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < kSimtEncTile * D; i += blockDim.x) {
+      const int j = i / D, d = i % D;
+      float kv = 0.f, vv = 0.f;
+      if (j < nt) {
+        kv = to_f(Kb[(t0 + j) * D + d]);
+        vv = to_f(Vb[(t0 + j) * D + d]);
+      }
+      ks[j][d] = kv;
+      vs[j][d] = vv;
+    }
+    __syncthreads();
+    if (active) {
+      float s[kSimtEncTile];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < kSimtEncTile; ++j) {
+        float a = 0.f;
+#pragma unroll
+        for (int d = 0; d < D; ++d) a = fmaf(q[d], ks[j][d], a);
+        s[j] = (j < nt) ? a : -INFINITY;
+        mx = fmaxf(mx, s[j]);
+      }
+      if (mx > mref) {  // rescale the running sums to the new maximum
+        const float f = exp2f(mref - mx);
+        l *= f;
+#pragma unroll
+        for (int d = 0; d < D; ++d) acc[d] *= f;
+        mref = mx;
+      }
+#pragma unroll
+      for (int j = 0; j < kSimtEncTile; ++j) {
+        const float p = exp2f(s[j] - mref);
+        l += p;
+#pragma unroll
+        for (int d = 0; d < D; ++d) acc[d] = fmaf(p, vs[j][d], acc[d]);
+      }
+    }
+  }
+  if (active) {
+    const int64_t row = (bh * chunks + chunk) * M + m;
+    part_ml[row * 2 + 0] = mref;
+    part_ml[row * 2 + 1] = l;
+#pragma unroll
+    for (int d = 0; d < D; ++d) part_acc[row * D + d] = acc[d];
+  }
+}
+
+// One thread per token; Q (pre-scaled to log2 units) and Z staged in smem.
+template <typename T, int D>
+__global__ void __launch_bounds__(kSimtDecThreads)
+    simt_decode_kernel(const T* __restrict__ Q, int64_t q_bstride, const T* __restrict__ K,
+                       const float* __restrict__ Zf, T* __restrict__ Y, int H, int64_t N, int M,
+                       float c) {
+  extern __shared__ float sm[];
+  float* qs = sm;
+  float* zs = sm + M * D;
+  const int64_t bh = blockIdx.y;
+  const int64_t b = bh / H, h = bh % H;
+  for (int i = threadIdx.x; i < M * D; i += blockDim.x) {
+    qs[i] = to_f(Q[b * q_bstride + h * (int64_t)M * D + i]) * c;
+    zs[i] = Zf[bh * M * D + i];
+  }
+  __syncthreads();
+  const int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  const T* kr = K + (bh * N + n) * D;
+  float k[D];
+#pragma unroll
+  for (int d = 0; d < D; ++d) k[d] = to_f(kr[d]);
+  float mx = -INFINITY;
+  for (int m = 0; m < M; ++m) {
+    float a = 0.f;
+#pragma unroll
+    for (int d = 0; d < D; ++d) a = fmaf(k[d], qs[m * D + d], a);
+    mx = fmaxf(mx, a);
+  }
+  float sum = 0.f, y[D];
+#pragma unroll
+  for (int d = 0; d < D; ++d) y[d] = 0.f;
+  for (int m = 0; m < M; ++m) {
+    float a = 0.f;
+#pragma unroll
+    for (int d = 0; d < D; ++d) a = fmaf(k[d], qs[m * D + d], a);
+    const float p = exp2f(a - mx);
+    sum += p;
+#pragma unroll
+    for (int d = 0; d < D; ++d) y[d] = fmaf(p, zs[m * D + d], y[d]);
+  }
+  const float inv = 1.f / sum;
+  T* yr = Y + (bh * N + n) * D;
+#pragma unroll
+  for (int d = 0; d < D; ++d) yr[d] = from_f<T>(y[d] * inv);
+}
+
+// One warp per (b, h, m); lane d < D owns Z[m][d].  Merges the per-chunk
+// (max, sum, acc) records with the log-sum-exp rule and, for FLARE++,
+// writes Q_dyn = Q + Z in the input dtype.
+template <typename T>
+__global__ void combine_kernel(const float* __restrict__ part_ml,
+                               const float* __restrict__ part_acc, int64_t BH, int H, int M,
+                               int D, int slots, float* __restrict__ Zf,
+                               __nv_bfloat16* __restrict__ Zb, float* __restrict__ Z_save,
+                               float* __restrict__ lse_save, const T* __restrict__ Qpp,
+                               T* __restrict__ Qdyn) {
+  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= BH * M) return;
+  const int64_t bh = w / M;
+  const int m = (int)(w % M);
+  float mstar = -INFINITY;
+  for (int s = 0; s < slots; ++s)
+    mstar = fmaxf(mstar, part_ml[((bh * slots + s) * M + m) * 2]);
+  float l = 0.f, acc = 0.f;
+  for (int s = 0; s < slots; ++s) {
+    const int64_t row = (bh * slots + s) * M + m;
+    const float ms = part_ml[row * 2];
+    if (ms == -INFINITY) continue;  // empty record
+    const float f = exp2f(ms - mstar);
+    l = fmaf(f, part_ml[row * 2 + 1], l);
+    if (lane < D) acc = fmaf(f, part_acc[row * D + lane], acc);
+  }
+  if (lane < D) {
+    const float z = acc / l;
+    const int64_t o = w * D + lane;
+    Zf[o] = z;
+    Zb[o] = __float2bfloat16_rn(z);
+    if (Z_save) Z_save[o] = z;
+    if (Qdyn) {
+      const int64_t h = bh % H;
+      Qdyn[o] = from_f<T>(to_f(Qpp[(h * M + m) * D + lane]) + z);
+    }
+  }
+  if (lane == 0 && lse_save) lse_save[w] = (mstar + log2f(l)) * kLn2;
+}
+
+template <typename T, int D>
+cudaError_t simt_encode_t(const void* Q, int64_t qbs, const void* K, const void* V,
+                          const Dims& d, float scale, const ChunkPlan& plan, float* part_ml,
+                          float* part_acc, cudaStream_t st) {
+  dim3 grid(plan.chunks, (unsigned)d.BH());
+  simt_encode_kernel<T, D><<<grid, kSimtEncThreads, 0, st>>>(
+      (const T*)Q, qbs, (const T*)K, (const T*)V, (int)d.H, d.N, (int)d.M, scale * kLog2e,
+      plan.chunk_tokens(), part_ml, part_acc);
+  return cudaPeekAtLastError();
+}
+
+template <typename T, int D>
+cudaError_t simt_decode_t(const void* Q, int64_t qbs, const void* K, const float* Zf, void* Y,
+                          const Dims& d, float scale, cudaStream_t st) {
+  const size_t smem = (size_t)2 * d.M * D * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(simt_decode_kernel<T, D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((d.N + kSimtDecThreads - 1) / kSimtDecThreads), (unsigned)d.BH());
+  simt_decode_kernel<T, D><<<grid, kSimtDecThreads, smem, st>>>(
+      (const T*)Q, qbs, (const T*)K, Zf, (T*)Y, (int)d.H, d.N, (int)d.M, scale * kLog2e);
+  return cudaPeekAtLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_simt_encode(const void* Q, int64_t qbs, const void* K, const void* V,
+                               const Dims& d, flare_dtype_t dt, float scale,
+                               const ChunkPlan& plan, float* part_ml, float* part_acc,
+                               cudaStream_t st) {
+  if (dt == FLARE_F32)
+    return d.D == 16 ? simt_encode_t<float, 16>(Q, qbs, K, V, d, scale, plan, part_ml, part_acc, st)
+                     : simt_encode_t<float, 32>(Q, qbs, K, V, d, scale, plan, part_ml, part_acc, st);
+  return d.D == 16
+             ? simt_encode_t<__nv_bfloat16, 16>(Q, qbs, K, V, d, scale, plan, part_ml, part_acc, st)
+             : simt_encode_t<__nv_bfloat16, 32>(Q, qbs, K, V, d, scale, plan, part_ml, part_acc, st);
+}
+
+cudaError_t launch_simt_decode(const void* Q, int64_t qbs, const void* K, const float* Zf,
+                               void* Y, const Dims& d, flare_dtype_t dt, float scale,
+                               cudaStream_t st) {
+  if (dt == FLARE_F32)
+    return d.D == 16 ? simt_decode_t<float, 16>(Q, qbs, K, Zf, Y, d, scale, st)
+                     : simt_decode_t<float, 32>(Q, qbs, K, Zf, Y, d, scale, st);
+  return d.D == 16 ? simt_decode_t<__nv_bfloat16, 16>(Q, qbs, K, Zf, Y, d, scale, st)
+                   : simt_decode_t<__nv_bfloat16, 32>(Q, qbs, K, Zf, Y, d, scale, st);
+}
+
+cudaError_t launch_combine(const Dims& d, flare_dtype_t dt, int slots_per_bh,
+                           const float* part_ml, const float* part_acc, float* Zf,
+                           __nv_bfloat16* Zb, float* Z_save, float* lse_save, const void* Qpp,
+                           void* Qdyn, cudaStream_t st) {
+  const int64_t warps = d.BH() * d.M;
+  const int threads = 256;
+  const unsigned blocks = (unsigned)((warps * 32 + threads - 1) / threads);
+  if (dt == FLARE_F32)
+    combine_kernel<float><<<blocks, threads, 0, st>>>(
+        part_ml, part_acc, d.BH(), (int)d.H, (int)d.M, (int)d.D, slots_per_bh, Zf, Zb, Z_save,
+        lse_save, (const float*)Qpp, (float*)Qdyn);
+  else
+    combine_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(
+        part_ml, part_acc, d.BH(), (int)d.H, (int)d.M, (int)d.D, slots_per_bh, Zf, Zb, Z_save,
+        lse_save, (const __nv_bfloat16*)Qpp, (__nv_bfloat16*)Qdyn);
+  return cudaPeekAtLastError();
+}
+
+}  // namespace flare

@@ -1,0 +1,186 @@
+"""Thin PyTorch binding over the C ABI (argument marshalling only).
+
+Every function here allocates outputs and the workspace with torch (the
+library never allocates), passes raw device pointers and the current CUDA
+stream to ``libflare.so``, and raises :class:`FlareError` on a non-OK status.
+All computation happens in the library's CUDA kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import FlareError  # noqa: F401  (re-export)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return _lib.FLARE_F32
+    if t.dtype == torch.bfloat16:
+        return _lib.FLARE_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("FLARE tensors must live on a CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("FLARE tensors must be contiguous")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dims(Q: torch.Tensor, K: torch.Tensor):
+    if K.dim() != 4:
+        raise ValueError("K must be [B,H,N,D]")
+    B, H, N, D = K.shape
+    M = Q.shape[-2]
+    if Q.dim() == 3:
+        qbs = 0
+    elif Q.dim() == 4:
+        qbs = H * M * D
+    else:
+        raise ValueError("Q must be [H,M,D] or [B,H,M,D]")
+    return B, H, N, M, D, qbs
+
+
+def default_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)
+
+
+def workspace_size(op: int, B: int, H: int, N: int, M: int, D: int, dtype: torch.dtype) -> int:
+    code = _lib.FLARE_F32 if dtype == torch.float32 else _lib.FLARE_BF16
+    return int(_lib.load().flare_workspace_size(op, B, H, N, M, D, code))
+
+
+def fwd_path(B: int, H: int, N: int, M: int, D: int, dtype: torch.dtype) -> int:
+    """1 = tcgen05 tensor-core kernels, 0 = CUDA-core kernels, -1 = unsupported."""
+    code = _lib.FLARE_F32 if dtype == torch.float32 else _lib.FLARE_BF16
+    return int(_lib.load().flare_fwd_path(B, H, N, M, D, code))
+
+
+def alloc_workspace(op: int, B, H, N, M, D, dtype, device) -> torch.Tensor:
+    n = workspace_size(op, B, H, N, M, D, dtype)
+    if n == 0:
+        raise FlareError(2, "flare_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def device_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronises the stream; returns the device error site (0 = none)."""
+    detail = ctypes.c_uint32(0)
+    st = _lib.load().flare_device_status(_ptr(workspace), workspace.numel(),
+                                         ctypes.byref(detail), _stream(stream))
+    if st not in (0, 5):
+        _lib.check(st, "flare_device_status")
+    return int(detail.value)
+
+
+def flare_fwd(Q, K, V, scale: Optional[float] = None, *, save: bool = False,
+              workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+              stream=None):
+    """FLARE forward.  Returns Y, or (Y, Z, lse) when ``save``."""
+    _need_cuda(Q, K, V, workspace, out)
+    B, H, N, M, D, qbs = _dims(Q, K)
+    dt = _dtype_code(K)
+    s = default_scale(D) if scale is None else float(scale)
+    Y = torch.empty_like(K) if out is None else out
+    Z = torch.empty((B, H, M, D), dtype=torch.float32, device=K.device) if save else None
+    lse = torch.empty((B, H, M), dtype=torch.float32, device=K.device) if save else None
+    ws = workspace if workspace is not None else alloc_workspace(
+        _lib.FLARE_OP_FWD, B, H, N, M, D, K.dtype, K.device)
+    st = _lib.load().flare_fwd(_ptr(Q), qbs, _ptr(K), _ptr(V), _ptr(Y), B, H, N, M, D, dt, s,
+                               _ptr(Z), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream))
+    _lib.check(st, "flare_fwd")
+    return (Y, Z, lse) if save else Y
+
+
+def flare_pp_fwd(Q, K, V, scale: Optional[float] = None, *, save: bool = False,
+                 workspace: Optional[torch.Tensor] = None, stream=None):
+    """FLARE++ forward with learned Q [H,M,D].  Returns (Y, Q_dyn) or
+    (Y, Q_dyn, Z, lse) when ``save``."""
+    _need_cuda(Q, K, V, workspace)
+    B, H, N, M, D, qbs = _dims(Q, K)
+    if qbs != 0:
+        raise ValueError("FLARE++ takes learned latents Q of shape [H,M,D]")
+    dt = _dtype_code(K)
+    s = default_scale(D) if scale is None else float(scale)
+    Y = torch.empty_like(K)
+    Qd = torch.empty((B, H, M, D), dtype=K.dtype, device=K.device)
+    Z = torch.empty((B, H, M, D), dtype=torch.float32, device=K.device) if save else None
+    lse = torch.empty((B, H, M), dtype=torch.float32, device=K.device) if save else None
+    ws = workspace if workspace is not None else alloc_workspace(
+        _lib.FLARE_OP_PP_FWD, B, H, N, M, D, K.dtype, K.device)
+    st = _lib.load().flare_pp_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(Y), _ptr(Qd), B, H, N, M, D,
+                                  dt, s, _ptr(Z), _ptr(lse), _ptr(ws), ws.numel(),
+                                  _stream(stream))
+    _lib.check(st, "flare_pp_fwd")
+    return (Y, Qd, Z, lse) if save else (Y, Qd)
+
+
+def flare_bwd(Q, K, V, dY, Z, lse, scale: Optional[float] = None, *,
+              workspace: Optional[torch.Tensor] = None, stream=None):
+    """FLARE backward.  Returns (dQ, dK, dV)."""
+    _need_cuda(Q, K, V, dY, Z, lse, workspace)
+    B, H, N, M, D, qbs = _dims(Q, K)
+    dt = _dtype_code(K)
+    s = default_scale(D) if scale is None else float(scale)
+    dQ = torch.empty_like(Q)
+    dK = torch.empty_like(K)
+    dV = torch.empty_like(V)
+    ws = workspace if workspace is not None else alloc_workspace(
+        _lib.FLARE_OP_BWD, B, H, N, M, D, K.dtype, K.device)
+    st = _lib.load().flare_bwd(_ptr(Q), qbs, _ptr(K), _ptr(V), _ptr(dY), _ptr(Z), _ptr(lse),
+                               _ptr(dQ), _ptr(dK), _ptr(dV), B, H, N, M, D, dt, s, _ptr(ws),
+                               ws.numel(), _stream(stream))
+    _lib.check(st, "flare_bwd")
+    return dQ, dK, dV
+
+
+def flare_encode(Q, K, V, scale: Optional[float] = None, *, workspace: torch.Tensor,
+                 stream=None) -> None:
+    """Stage 1: encode partials into ``workspace`` (FLARE_OP_FWD size)."""
+    _need_cuda(Q, K, V, workspace)
+    B, H, N, M, D, qbs = _dims(Q, K)
+    s = default_scale(D) if scale is None else float(scale)
+    st = _lib.load().flare_encode(_ptr(Q), qbs, _ptr(K), _ptr(V), B, H, N, M, D, _dtype_code(K),
+                                  s, _ptr(workspace), workspace.numel(), _stream(stream))
+    _lib.check(st, "flare_encode")
+
+
+def flare_combine(B, H, N, M, D, dtype: torch.dtype, *, workspace: torch.Tensor,
+                  Z_save: Optional[torch.Tensor] = None, lse_save: Optional[torch.Tensor] = None,
+                  stream=None) -> None:
+    """Stage 2: merge the encode partials in ``workspace``."""
+    _need_cuda(workspace, Z_save, lse_save)
+    code = _lib.FLARE_F32 if dtype == torch.float32 else _lib.FLARE_BF16
+    st = _lib.load().flare_combine(B, H, N, M, D, code, _ptr(Z_save), _ptr(lse_save),
+                                   _ptr(workspace), workspace.numel(), _stream(stream))
+    _lib.check(st, "flare_combine")
+
+
+def flare_decode(Q, K, scale: Optional[float] = None, *, workspace: torch.Tensor,
+                 out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Stage 3: decode with the Z left in ``workspace`` by flare_combine."""
+    _need_cuda(Q, K, workspace, out)
+    B, H, N, M, D, qbs = _dims(Q, K)
+    s = default_scale(D) if scale is None else float(scale)
+    Y = torch.empty_like(K) if out is None else out
+    st = _lib.load().flare_decode(_ptr(Q), qbs, _ptr(K), _ptr(Y), B, H, N, M, D, _dtype_code(K),
+                                  s, _ptr(workspace), workspace.numel(), _stream(stream))
+    _lib.check(st, "flare_decode")
+    return Y

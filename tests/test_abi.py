@@ -1,0 +1,189 @@
+"""The C ABI library loads, exports every symbol include/flare.h declares, and
+rejects invalid arguments with status codes before touching the device.
+
+These run without a GPU.  The argument-validation tests pass fake
+(never dereferenced) device addresses, so they are skipped when a CUDA
+device is present: on a GPU machine the same checks run in the gpu tests with
+real buffers.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+import rank_latent_attention_flare_b200 as fl
+from rank_latent_attention_flare_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "flare.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE, CUDA = 0, 1, 2, 3, 4
+
+no_gpu_only = pytest.mark.skipif(torch.cuda.is_available(),
+                                 reason="fake-pointer validation tests run on CPU-only hosts")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from rank_latent_attention_flare_b200 import build
+    build.build()
+    return fl.load()
+
+
+def header_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"FLARE_API\s+[\w\s\*]+?\b(flare_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    syms = header_symbols()
+    for name in ("flare_fwd", "flare_pp_fwd", "flare_bwd", "flare_workspace_size",
+                 "flare_status_string", "flare_encode", "flare_combine", "flare_decode"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    syms = header_symbols()
+    assert set(syms) == set(_lib.SIGNATURES), "binding signatures out of sync with flare.h"
+    out = subprocess.run(["nm", "-D", "--defined-only", fl.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(flare_\w+)", out))
+    missing = set(syms) - exported
+    assert not missing, missing
+    for s in syms:
+        assert getattr(lib, s) is not None
+
+
+def test_library_targets_sm100a_only(lib):
+    out = subprocess.run(["/usr/local/cuda/bin/cuobjdump", "--list-elf", fl.LIB_PATH],
+                         capture_output=True, text=True)
+    if out.returncode != 0:
+        pytest.skip("cuobjdump unavailable")
+    archs = set(re.findall(r"sm_(\d+a?)", out.stdout))
+    assert archs == {"100a"}, archs
+
+
+def test_version_and_status_strings(lib):
+    assert lib.flare_version() >= 100
+    for code in range(6):
+        s = lib.flare_status_string(code).decode()
+        assert s.startswith("FLARE"), s
+    assert b"unknown" in lib.flare_status_string(99)
+
+
+def test_workspace_size(lib):
+    ws = lib.flare_workspace_size
+    assert ws(0, 1, 16, 1 << 20, 256, 32, 1) > 0
+    assert ws(1, 2, 8, 1 << 18, 256, 32, 1) > ws(0, 2, 8, 1 << 18, 256, 32, 1)
+    assert ws(2, 8, 8, 16384, 128, 32, 1) > 8 * 8 * 16384 * 32 * 4  # holds the fp32 dK
+    assert ws(0, 1, 1, 1, 16, 16, 0) > 0
+    # invalid or unsupported sizes -> 0
+    assert ws(0, 0, 1, 100, 16, 16, 0) == 0
+    assert ws(0, 1, 1, 0, 16, 16, 0) == 0
+    assert ws(0, 1, 1, 100, 24, 16, 0) == 0
+    assert ws(0, 1, 1, 100, 16, 64, 0) == 0
+    assert ws(0, 1, 1, 100, 512, 16, 0) == 0
+    assert ws(7, 1, 1, 100, 16, 16, 0) == 0
+    assert ws(0, 1, 1, 100, 16, 16, 5) == 0
+
+
+def test_fwd_path_selection(lib):
+    assert lib.flare_fwd_path(1, 4, 1024, 32, 16, 0) == 0        # fp32 -> CUDA cores
+    assert lib.flare_fwd_path(1, 16, 1 << 20, 256, 32, 1) in (0, 1)
+    assert lib.flare_fwd_path(1, 4, 1024, 40, 16, 1) == -1
+
+
+# ------------------------------------------------ validation before launch ---
+
+FAKE = 0x7F0000000000       # 16- and 256-byte aligned, never dereferenced
+
+
+def _p(x):
+    return ctypes.c_void_p(x)
+
+
+def _fwd(lib, Q=FAKE, qbs=0, K=FAKE + 0x100000, V=FAKE + 0x200000, Y=FAKE + 0x300000,
+         B=1, H=2, N=100, M=32, D=16, dt=0, scale=0.25, Z=None, lse=None,
+         ws=FAKE + 0x400000, wsb=None):
+    if wsb is None:
+        wsb = lib.flare_workspace_size(0, B, H, N, M, D, dt) or (1 << 30)
+    return lib.flare_fwd(_p(Q), qbs, _p(K), _p(V), _p(Y), B, H, N, M, D, dt, scale,
+                         _p(Z) if Z else None, _p(lse) if lse else None, _p(ws), wsb, None)
+
+
+@no_gpu_only
+def test_fwd_rejects_bad_pointers(lib):
+    assert _fwd(lib, Q=0) == INVALID
+    assert _fwd(lib, K=0) == INVALID
+    assert _fwd(lib, V=0) == INVALID
+    assert _fwd(lib, Y=0) == INVALID
+    assert _fwd(lib, Q=FAKE + 8) == INVALID          # misaligned
+    assert _fwd(lib, Y=FAKE + 0x300002) == INVALID
+    assert _fwd(lib, Z=FAKE + 0x500004) == INVALID   # optional but misaligned
+
+
+@no_gpu_only
+def test_fwd_rejects_bad_sizes_and_scale(lib):
+    assert _fwd(lib, N=0) == INVALID
+    assert _fwd(lib, B=0) == INVALID
+    assert _fwd(lib, H=-1) == INVALID
+    assert _fwd(lib, dt=3) == INVALID
+    for s in (0.0, -1.0, float("nan"), float("inf")):
+        assert _fwd(lib, scale=s) == INVALID
+    assert _fwd(lib, D=24) == UNSUPPORTED
+    assert _fwd(lib, D=64) == UNSUPPORTED
+    assert _fwd(lib, M=8) == UNSUPPORTED
+    assert _fwd(lib, M=100) == UNSUPPORTED
+    assert _fwd(lib, M=272) == UNSUPPORTED
+    assert _fwd(lib, qbs=7) == UNSUPPORTED
+    assert _fwd(lib, B=1 << 21) == INVALID
+
+
+@no_gpu_only
+def test_fwd_rejects_bad_workspace(lib):
+    need = lib.flare_workspace_size(0, 1, 2, 100, 32, 16, 0)
+    assert _fwd(lib, wsb=need - 1) == WORKSPACE
+    assert _fwd(lib, ws=0) == WORKSPACE
+    assert _fwd(lib, ws=FAKE + 0x400010) == WORKSPACE   # not 256-byte aligned
+
+
+@no_gpu_only
+def test_other_entry_points_validate(lib):
+    F = FAKE
+    ws_pp = lib.flare_workspace_size(1, 1, 2, 100, 32, 16, 0)
+    assert lib.flare_pp_fwd(None, _p(F), _p(F), _p(F), None, 1, 2, 100, 32, 16, 0, 0.25, None,
+                            None, _p(F), ws_pp, None) == INVALID
+    assert lib.flare_pp_fwd(_p(F), _p(F), _p(F), _p(F), None, 1, 2, 100, 32, 16, 0, 0.25, None,
+                            None, _p(F), ws_pp - 1, None) == WORKSPACE
+    ws_b = lib.flare_workspace_size(2, 1, 2, 100, 32, 16, 0)
+    # Z_save and lse_save are required by the backward
+    assert lib.flare_bwd(_p(F), 0, _p(F), _p(F), _p(F), None, _p(F), _p(F), _p(F), _p(F),
+                         1, 2, 100, 32, 16, 0, 0.25, _p(F), ws_b, None) == INVALID
+    assert lib.flare_bwd(_p(F), 0, _p(F), _p(F), _p(F), _p(F), None, _p(F), _p(F), _p(F),
+                         1, 2, 100, 32, 16, 0, 0.25, _p(F), ws_b, None) == INVALID
+    assert lib.flare_bwd(_p(F), 0, _p(F), _p(F), _p(F), _p(F), _p(F), _p(F), _p(F), _p(F),
+                         1, 2, 100, 32, 16, 0, 0.25, _p(F), ws_b - 1, None) == WORKSPACE
+    ws_f = lib.flare_workspace_size(0, 1, 2, 100, 32, 16, 0)
+    assert lib.flare_encode(None, 0, _p(F), _p(F), 1, 2, 100, 32, 16, 0, 0.25, _p(F), ws_f,
+                            None) == INVALID
+    assert lib.flare_combine(1, 2, 100, 32, 16, 0, None, None, _p(F), ws_f - 1,
+                             None) == WORKSPACE
+    assert lib.flare_decode(_p(F), 0, _p(F), None, 1, 2, 100, 32, 16, 0, 0.25, _p(F), ws_f,
+                            None) == INVALID
+    assert lib.flare_device_status(None, 256, None, None) == WORKSPACE
+
+
+@no_gpu_only
+def test_valid_call_without_device_reports_cuda_error(lib):
+    # Arguments pass validation; the first enqueue fails because there is no
+    # device, which must surface as FLARE_ERR_CUDA (not a crash).
+    assert _fwd(lib) == CUDA
+
+
+def test_binding_fails_loudly_without_cuda_tensors():
+    x = torch.zeros(1, 2, 8, 16)
+    with pytest.raises(ValueError):
+        fl.flare_fwd(torch.zeros(2, 16, 16), x, x)

@@ -1,0 +1,134 @@
+"""GPU parity of the FLARE forward (through the C ABI) against the oracle.
+
+Shapes span several 128-token tiles with a ragged tail, single-token and
+single-tile heads, every supported M class and both D, shared and per-batch
+latents, float32 (CUDA-core kernels) and bf16 (tensor-core kernels where the
+shape is covered).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rank_latent_attention_flare_b200 as fl
+from flare_inputs import make_inputs
+from gpu_util import assert_close, rel_fro
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+SHAPES = [
+    # B, H, N, M, D
+    (1, 1, 1, 16, 16),
+    (1, 2, 7, 32, 16),
+    (2, 3, 129, 64, 32),
+    (1, 2, 1000, 128, 16),
+    (2, 2, 1000, 128, 32),
+    (1, 2, 1000, 256, 32),
+    (1, 1, 4097, 256, 16),
+    (3, 1, 385, 256, 32),
+    (1, 2, 300, 48, 32),
+    (2, 1, 2049, 128, 32),
+]
+
+
+def _run(x, s, dtype, per_batch_q=False, save=True):
+    g = {k: v.to(DEV) for k, v in x.items()}
+    return fl.flare_fwd(g["Q"], g["K"], g["V"], s, save=save)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("B,H,N,M,D", SHAPES)
+def test_fwd_matches_oracle(B, H, N, M, D, dtype):
+    s = 1.0 / math.sqrt(D)
+    x = make_inputs(B, H, N, M, D, dtype=dtype, seed=N + M + D)
+    Y, Z, lse = _run(x, s, dtype)
+    torch.cuda.synchronize()
+    Yo, Zo, lo = oracle.flare_fwd(x["Q"], x["K"], x["V"], s)
+    assert_close(Z, Zo, dtype, "Z")
+    assert_close(Y, Yo, dtype, "Y")
+    assert_close(lse, lo, torch.float32 if dtype == torch.float32 else dtype, "lse")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("M,D", [(128, 16), (256, 32), (32, 16)])
+def test_fwd_per_batch_latents(M, D, dtype):
+    B, H, N = 3, 2, 700
+    s = 1.0 / math.sqrt(D)
+    x = make_inputs(B, H, N, M, D, dtype=dtype, seed=77, per_batch_q=True)
+    Y, Z, lse = _run(x, s, dtype)
+    torch.cuda.synchronize()
+    Yo, Zo, _ = oracle.flare_fwd(x["Q"], x["K"], x["V"], s)
+    assert_close(Z, Zo, dtype, "Z")
+    assert_close(Y, Yo, dtype, "Y")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_fwd_large_scale_stable(dtype):
+    # scale 100x the usual 1/sqrt(D): softmaxes are sharply peaked, the
+    # running max must keep every exponential finite.
+    B, H, N, M, D = 1, 2, 900, 128, 32
+    s = 100.0 / math.sqrt(D)
+    x = make_inputs(B, H, N, M, D, dtype=dtype, seed=5)
+    Y, Z, lse = _run(x, s, dtype)
+    torch.cuda.synchronize()
+    assert torch.isfinite(Y.float()).all() and torch.isfinite(Z).all()
+    Yo, Zo, _ = oracle.flare_fwd(x["Q"], x["K"], x["V"], s)
+    # Peaked softmaxes amplify the bf16 rounding of the logits; compare with
+    # the float32 bar on the fp32 path and a looser relative bar on bf16.
+    if dtype == torch.float32:
+        assert rel_fro(Z, Zo) <= 1e-4 and rel_fro(Y, Yo) <= 1e-4
+    else:
+        assert rel_fro(Z, Zo) <= 5e-2 and rel_fro(Y, Yo) <= 5e-2
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_fwd_writes_every_output_and_is_deterministic(dtype):
+    B, H, N, M, D = 2, 2, 1537, 256, 32
+    s = 1.0 / math.sqrt(D)
+    x = make_inputs(B, H, N, M, D, dtype=dtype, seed=9)
+    g = {k: v.to(DEV) for k, v in x.items()}
+    ws = fl.alloc_workspace(fl.FLARE_OP_FWD, B, H, N, M, D, dtype, DEV)
+    ws.fill_(0xFF)  # poison: NaN bit patterns everywhere in the workspace
+    Y1 = torch.full_like(g["K"], float("nan"))
+    fl.flare_fwd(g["Q"], g["K"], g["V"], s, workspace=ws, out=Y1)
+    Y2 = torch.full_like(g["K"], float("nan"))
+    fl.flare_fwd(g["Q"], g["K"], g["V"], s, workspace=ws, out=Y2)
+    assert fl.device_status(ws) == 0
+    assert not torch.isnan(Y1.float()).any()
+    assert torch.equal(Y1, Y2)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_stage_calls_equal_fused_call(dtype):
+    B, H, N, M, D = 1, 3, 2000, 128, 16
+    s = 1.0 / math.sqrt(D)
+    x = make_inputs(B, H, N, M, D, dtype=dtype, seed=10)
+    g = {k: v.to(DEV) for k, v in x.items()}
+    ws = fl.alloc_workspace(fl.FLARE_OP_FWD, B, H, N, M, D, dtype, DEV)
+    Y1, Z1, l1 = fl.flare_fwd(g["Q"], g["K"], g["V"], s, save=True, workspace=ws)
+    Z2 = torch.empty_like(Z1)
+    l2 = torch.empty_like(l1)
+    fl.flare_encode(g["Q"], g["K"], g["V"], s, workspace=ws)
+    fl.flare_combine(B, H, N, M, D, dtype, workspace=ws, Z_save=Z2, lse_save=l2)
+    Y2 = fl.flare_decode(g["Q"], g["K"], s, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(Y1, Y2) and torch.equal(Z1, Z2) and torch.equal(l1, l2)
+
+
+def test_gpu_rejects_invalid_arguments_without_side_effects():
+    B, H, N, M, D = 1, 2, 100, 32, 16
+    x = {k: v.to(DEV) for k, v in make_inputs(B, H, N, M, D, dtype=torch.float32).items()}
+    Y = torch.zeros_like(x["K"])
+    with pytest.raises(fl.FlareError) as e:
+        fl.flare_fwd(x["Q"], x["K"], x["V"], scale=-1.0, out=Y)
+    assert e.value.status == 1
+    small = torch.empty(64, dtype=torch.uint8, device=DEV)
+    with pytest.raises(fl.FlareError) as e:
+        fl.flare_fwd(x["Q"], x["K"], x["V"], workspace=small, out=Y)
+    assert e.value.status == 3
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(Y) == 0
