@@ -80,6 +80,13 @@ typedef enum { FLARE_OP_FWD = 0, FLARE_OP_PP_FWD = 1, FLARE_OP_BWD = 2 } flare_o
 /* Library ABI version (major*10000 + minor*100 + patch). */
 FLARE_API int flare_version(void);
 
+/*
+ * Description of the last FLARE_ERR_CUDA returned on the calling host thread
+ * (the failing call and the CUDA error name), or "" if none.  Thread-local
+ * storage, valid until the next FLARE call on this thread.
+ */
+FLARE_API const char* flare_last_error_detail(void);
+
 /* Human-readable text for a status code (static storage, never NULL). */
 FLARE_API const char* flare_status_string(flare_status_t status);
 

@@ -37,6 +37,7 @@ _u32p = ctypes.POINTER(ctypes.c_uint32)
 
 SIGNATURES = {
     "flare_version": (_i32, []),
+    "flare_last_error_detail": (ctypes.c_char_p, []),
     "flare_status_string": (ctypes.c_char_p, [_i32]),
     "flare_workspace_size": (_sz, [_i32, _i64, _i64, _i64, _i64, _i64, _i32]),
     "flare_fwd": (_i32, [_vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i32, _f32,
@@ -83,4 +84,7 @@ def load() -> ctypes.CDLL:
 
 def check(status: int, where: str) -> None:
     if status != 0:
-        raise FlareError(status, where)
+        detail = ""
+        if status == 4 and _lib is not None:
+            detail = (_lib.flare_last_error_detail() or b"").decode(errors="replace")
+        raise FlareError(status, where + (f" [{detail}]" if detail else ""))

@@ -2,11 +2,26 @@
 // launch orchestration on the caller's stream.  No allocation, no
 // synchronisation (except flare_device_status, documented as such), no
 // global mutable state.
+#include <stdarg.h>
+#include <stdio.h>
 #include <string.h>
 
 #include "flare_internal.cuh"
 
 using namespace flare;
+
+namespace flare {
+namespace {
+thread_local char g_error_detail[512];
+}
+
+void note_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_error_detail, sizeof(g_error_detail), fmt, ap);
+  va_end(ap);
+}
+}  // namespace flare
 
 namespace {
 
@@ -65,12 +80,18 @@ flare_status_t check_ws(const void* ws, size_t bytes, size_t need) {
     if (s_ != FLARE_OK) return s_;      \
   } while (0)
 
-#define FLARE_CUDA(x)                                 \
-  do {                                                \
-    if ((x) != cudaSuccess) return FLARE_ERR_CUDA;    \
+#define FLARE_CUDA(x)                                                               \
+  do {                                                                              \
+    cudaError_t e_ = (x);                                                           \
+    if (e_ != cudaSuccess) {                                                        \
+      if (g_error_detail[0] == 0)                                                   \
+        note_error("%s: %s (%s)", #x, cudaGetErrorName(e_), cudaGetErrorString(e_)); \
+      return FLARE_ERR_CUDA;                                                        \
+    }                                                                               \
   } while (0)
 
 flare_status_t reset_error_word(char* ws, cudaStream_t st) {
+  g_error_detail[0] = 0;
   FLARE_CUDA(cudaMemsetAsync(ws, 0, 4, st));
   return FLARE_OK;
 }
@@ -79,7 +100,7 @@ flare_status_t reset_error_word(char* ws, cudaStream_t st) {
 flare_status_t run_encode(const void* Q, int64_t qbs, const void* K, const void* V,
                           const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,
                           char* ws, cudaStream_t st) {
-  const Path path = choose_path(d.M, d.D, dt);
+  const Path path = choose_path(d.N, d.M, d.D, dt);
   float* pml = (float*)(ws + L.part_ml);
   float* pacc = (float*)(ws + L.part_acc);
   if (path.tc_fwd)
@@ -102,7 +123,7 @@ flare_status_t run_combine(const Dims& d, flare_dtype_t dt, float* Z_save, float
 flare_status_t run_decode(const void* Q, int64_t qbs, const void* K, void* Y, const Dims& d,
                           flare_dtype_t dt, float scale, const WsLayout& L, char* ws,
                           cudaStream_t st, int sms) {
-  const Path path = choose_path(d.M, d.D, dt);
+  const Path path = choose_path(d.N, d.M, d.D, dt);
   if (path.tc_fwd)
     FLARE_CUDA(launch_tc_decode(Q, qbs, K, (const __nv_bfloat16*)(ws + L.zb), Y, d, scale,
                                 decode_plan(d.BH(), d.N, sms), (uint32_t*)(ws + L.hdr), st));
@@ -116,6 +137,8 @@ flare_status_t run_decode(const void* Q, int64_t qbs, const void* K, void* Y, co
 extern "C" {
 
 int flare_version(void) { return 100; }
+
+const char* flare_last_error_detail(void) { return g_error_detail; }
 
 const char* flare_status_string(flare_status_t s) {
   switch (s) {
@@ -138,7 +161,7 @@ size_t flare_workspace_size(flare_op_t op, int64_t B, int64_t H, int64_t N, int6
 
 int flare_fwd_path(int64_t B, int64_t H, int64_t N, int64_t M, int64_t D, flare_dtype_t dt) {
   if (check_sizes(B, H, N, M, D, dt) != FLARE_OK) return -1;
-  return choose_path(M, D, dt).tc_fwd ? 1 : 0;
+  return choose_path(N, M, D, dt).tc_fwd ? 1 : 0;
 }
 
 flare_status_t flare_encode(const void* Q, int64_t qbs, const void* K, const void* V, int64_t B,
@@ -166,6 +189,7 @@ flare_status_t flare_combine(int64_t B, int64_t H, int64_t N, int64_t M, int64_t
   FLARE_TRY(check_opt_ptr(lse_save));
   const WsLayout L = ws_layout(FLARE_OP_FWD, B, H, N, M, D, dt, current_sm_count());
   FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  g_error_detail[0] = 0;
   return run_combine(Dims{B, H, N, M, D}, dt, Z_save, lse_save, nullptr, nullptr, L,
                      (char*)workspace, (cudaStream_t)stream);
 }
@@ -182,6 +206,7 @@ flare_status_t flare_decode(const void* Q, int64_t qbs, const void* K, void* Y, 
   const int sms = current_sm_count();
   const WsLayout L = ws_layout(FLARE_OP_FWD, B, H, N, M, D, dt, sms);
   FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  g_error_detail[0] = 0;
   return run_decode(Q, qbs, K, Y, Dims{B, H, N, M, D}, dt, scale, L, (char*)workspace,
                     (cudaStream_t)stream, sms);
 }

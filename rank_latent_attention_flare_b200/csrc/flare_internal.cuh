@@ -75,23 +75,27 @@ struct Path {
   bool tc_fwd = false;  // tcgen05 encode + decode
 };
 
-inline Path choose_path(int64_t M, int64_t D, flare_dtype_t dt) {
+// The tcgen05 kernels cover bf16 with M in {128, 256} (one or two 128-row
+// MMA tiles of latents), D in {16, 32} and N addressable by a TMA coordinate.
+inline Path choose_path(int64_t N, int64_t M, int64_t D, flare_dtype_t dt) {
   Path p;
-  p.tc_fwd = false && (dt == FLARE_BF16) && (M == 128 || M == 256) && (D == 16 || D == 32);
+  p.tc_fwd = (dt == FLARE_BF16) && (M == 128 || M == 256) && (D == 16 || D == 32) &&
+             (N < (1LL << 31) - 256);
   return p;
 }
 
 constexpr int kSimtEncTile = 64;
 constexpr int kSimtEncThreads = 256;
 constexpr int kSimtDecThreads = 128;
-constexpr int kTcTile = 128;
+constexpr int kTcTile = 128;     // decode tile (tokens)
+constexpr int kTcEncTile = 64;   // tensor-core encode tile (tokens)
 constexpr int kBwdTile = 256;
 
 inline ChunkPlan encode_plan(int64_t BH, int64_t N, int64_t M, int64_t D, flare_dtype_t dt,
                              int sms) {
-  Path path = choose_path(M, D, dt);
+  Path path = choose_path(N, M, D, dt);
   if (path.tc_fwd) {
-    ChunkPlan p = plan_chunks(BH, N, kTcTile, sms, 6.0, 16 * (int64_t)sms);
+    ChunkPlan p = plan_chunks(BH, N, kTcEncTile, sms, 12.0, 16 * (int64_t)sms);
     p.sub = (M == 128) ? 2 : 1;
     return p;
   }
@@ -183,6 +187,10 @@ __host__ __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { retur
 __device__ __forceinline__ void record_error(uint32_t* err, uint32_t site) {
   if (err) atomicCAS(err, 0u, site);
 }
+
+// Records a description of the last launch-time failure on this host thread
+// (read back through flare_last_error_detail).
+void note_error(const char* fmt, ...);
 
 // ------------------------------------------------------------ launchers
 // Each returns cudaSuccess or the launch error.

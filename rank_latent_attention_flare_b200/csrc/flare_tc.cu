@@ -1,16 +1,746 @@
-// Tensor-core (tcgen05 / TMEM / TMA) encode and decode kernels: placeholder
-// until the sm_100a kernels land; the dispatcher does not select them yet.
+// Tensor-core FLARE forward for sm_100a: tcgen05.mma with TMEM accumulators,
+// operands staged in shared memory by TMA, softmax on the CUDA cores with one
+// TMEM lane (one row) per thread.
+//
+// Encode, per (b, h) and chunk of tokens ("Flare Fast Low Rank Attention"
+// skill page, section 2, latents as queries): for every 128-token tile
+//   S = Q K_tile^T            (tcgen05, M=128 latents x N=128 tokens x K=D)
+//   P = 2^(c S - m_ref)       (row = latent, online max with lazy rescale)
+//   O += P V_tile             (tcgen05, A = P from TMEM, B = V from smem)
+// and at the end of the chunk the record (m_ref, l = row sum of P, O) goes to
+// the workspace for the log-sum-exp combine.
+// Decode (FLARE arXiv abstract, second SDPA call): for every 128-token tile
+//   S = K_tile Q^T            (M=128 tokens x N=M latents x K=D)
+//   P = 2^(c S - rowmax)      (row = token, whole row in one thread)
+//   Y = (P Z) / rowsum(P)     (A = P from TMEM, B = Z from smem)
+// so the N x M logits never leave the SM.
+//
+// Roles per CTA (384 threads, three warpgroups): warps 0-3 and 4-7 are two
+// softmax warpgroups, warp 8 issues TMA loads, warp 9 owns TMEM and issues
+// the MMAs, warps 10-11 only lend their registers.  The CTA launches at 168
+// registers per thread; the producer warpgroup drops to 56 and the softmax
+// warpgroups rise to 224 (2 x 128 x 224 + 128 x 56 = 384 x 168, and each SM
+// sub-partition keeps 2 x 224 + 56 registers x 32 lanes <= 16384).
+// Exponentials use ex2.approx (MUFU); c = scale * log2(e) is folded in.
+#include <cudaTypedefs.h>
+
 #include "flare_internal.cuh"
+#include "tc_primitives.cuh"
 
 namespace flare {
+namespace {
 
-cudaError_t launch_tc_encode(const void*, int64_t, const void*, const void*, const Dims&, float,
-                             const ChunkPlan&, float*, float*, uint32_t*, cudaStream_t) {
+using namespace tc;
+
+constexpr int kTile = 128;        // tokens per tile (MMA M or N)
+constexpr int kThreads = 384;
+constexpr int kRegsSoftmax = 224;
+constexpr int kRegsProducer = 56;
+constexpr int kWarpTma = 8;
+constexpr int kWarpMma = 9;
+constexpr int kEncStages = 8;
+constexpr int kDecStages = 6;
+constexpr float kRescaleTau = 8.0f;   // log2 units: rescale only when the max grows by > 2^8
+constexpr int kMinSmemBytes = 120 * 1024;  // keeps one CTA (and its TMEM) per SM
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return (uint8_t*)(((uintptr_t)p + 1023) & ~(uintptr_t)1023);
+}
+
+// ============================================================== encode
+//
+// Tiles of kEncTile = 64 tokens.  TMEM (512 columns): S[w][b] at w*128 + b*64
+// (two 64-column S buffers per warpgroup, so the MMA computes the next tile's
+// logits while the softmax works on this one), P[w][b] at 256 + w*64 + b*32
+// (bf16 pairs), O[w] at 384 + w*32.  With M = 256 warpgroup w owns latent
+// rows [128w, 128w+128) of every tile; with M = 128 the warpgroups take
+// alternate tiles and each keeps its own running record.
+
+constexpr int kEncTile = 64;
+
+template <int D, int M>
+struct EncLayout {
+  static constexpr int RB = 2 * D;                  // bytes per row (one token or latent)
+  static constexpr int TILE = kEncTile * RB;        // one K or V tile
+  static constexpr int Q_OFF = 0;
+  static constexpr int KV_OFF = M * RB;
+  static constexpr int BAR_OFF = KV_OFF + kEncStages * 2 * TILE;
+  static constexpr int NBARS = 2 * kEncStages + 1 + 4 + 4 + 2 + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+  static constexpr int BYTES = MISC_OFF + 16;
+};
+
+template <int D, int M>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_encode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, int H, int64_t N, int q_per_batch,
+                     float c, int64_t tiles_per_bh, int64_t chunk_tiles, int slots_per_bh,
+                     float* __restrict__ part_ml, float* __restrict__ part_acc,
+                     uint32_t* __restrict__ err) {
+  using L = EncLayout<D, M>;
+  constexpr int NH = M / 128;        // latent halves; M=128 -> the two warpgroups split tiles
+  constexpr int SUB = (NH == 1) ? 2 : 1;
+  constexpr int RB = L::RB;
+  constexpr uint32_t SW = umma_swizzle_code(RB);
+  constexpr uint32_t TM_S = 0, TM_P = 256, TM_O = 384;   // TMEM column bases
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* Qs = smem + L::Q_OFF;
+  uint64_t* bars = (uint64_t*)(smem + L::BAR_OFF);
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = bars + kEncStages;
+  uint64_t* q_full = bars + 2 * kEncStages;
+  uint64_t* s_full = q_full + 1;      // [w*2 + b]
+  uint64_t* sp_done = s_full + 4;     // [w*2 + b]: S read and P written
+  uint64_t* pv_done = sp_done + 4;    // [w]
+  uint64_t* drain = pv_done + 2;
+  uint32_t* tmem_slot = (uint32_t*)(smem + L::MISC_OFF);
+  volatile int* abort_flag = (volatile int*)(smem + L::MISC_OFF + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x;
+  const int64_t bh = blockIdx.y;
+  const int64_t h = bh % H;
+  const int64_t tile0 = (int64_t)chunk * chunk_tiles;
+  const int64_t ntiles = imin64(chunk_tiles, tiles_per_bh - tile0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kEncStages; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    mbar_init(q_full, 1);
+    for (int k = 0; k < 4; ++k) {
+      mbar_init(&s_full[k], 1);
+      mbar_init(&sp_done[k], 128);
+    }
+    mbar_init(&pv_done[0], 1);
+    mbar_init(&pv_done[1], 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kWarpMma) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp >= 8) {
+    regs_release<kRegsProducer>();
+    if (warp == kWarpTma) {
+      // ---------------------------------------------------- TMA producer
+      if (lane == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        mbar_arrive_expect_tx(q_full, M * RB);
+        const int32_t qz = (int32_t)(q_per_batch ? bh : h);
+        for (int half = 0; half < NH; ++half)
+          tma_load_3d(Qs + half * 128 * RB, &tmQ, q_full, 0, half * 128, qz);
+        int64_t issued = 0;
+        for (int64_t i = 0; i < ntiles; ++i) {
+          const int s = (int)(i % kEncStages);
+          const uint32_t ph = (uint32_t)((i / kEncStages) & 1);
+          if (i >= kEncStages && !mbar_wait(&kv_empty[s], ph ^ 1)) {
+            record_error(err, kErrEncTmaWait);
+            *abort_flag = 1;
+            break;
+          }
+          if (*abort_flag) break;
+          uint8_t* kt = smem + L::KV_OFF + s * 2 * L::TILE;
+          mbar_arrive_expect_tx(&kv_full[s], 2 * L::TILE);
+          const int32_t tok = (int32_t)((tile0 + i) * kEncTile);
+          tma_load_3d(kt, &tmK, &kv_full[s], 0, tok, (int32_t)bh);
+          tma_load_3d(kt + L::TILE, &tmV, &kv_full[s], 0, tok, (int32_t)bh);
+          issued = i + 1;
+        }
+        // let every load still in flight land before the CTA can exit
+        for (int64_t i = (issued > kEncStages ? issued - kEncStages : 0); i < issued; ++i)
+          mbar_wait(&kv_full[i % kEncStages], (uint32_t)((i / kEncStages) & 1));
+        mbar_wait(q_full, 0);
+      }
+    } else if (warp == kWarpMma) {
+      // ---------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t idS = idesc_bf16_f32(128, kEncTile, 0, 0);
+        constexpr uint32_t idPV = idesc_bf16_f32(128, D, 0, 1);
+        const uint32_t q_addr = smem_u32(Qs);
+        bool ok = mbar_wait(q_full, 0);
+        auto wg_count = [&](int64_t) { return NH == 2 ? 2 : 1; };
+        auto wg_of = [&](int64_t i, int k) { return NH == 2 ? k : (int)(i & 1); };
+        auto wg_tile = [&](int64_t i) { return NH == 2 ? i : (i >> 1); };
+        auto issue_S = [&](int64_t i) -> bool {
+          const int s = (int)(i % kEncStages);
+          if (!mbar_wait(&kv_full[s], (uint32_t)((i / kEncStages) & 1))) return false;
+          const uint32_t k_addr = smem_u32(smem + L::KV_OFF + s * 2 * L::TILE);
+          for (int k = 0; k < wg_count(i); ++k) {
+            const int w = wg_of(i, k);
+            const int64_t j = wg_tile(i);
+            const int b = (int)(j & 1);
+            if (j >= 2 && !mbar_wait(&sp_done[w * 2 + b], (uint32_t)(((j >> 1) - 1) & 1)))
+              return false;
+            tc_fence_after();
+            const uint32_t qa = q_addr + (NH == 2 ? w * 128 * RB : 0);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tmem + TM_S + w * 128 + b * 64, smem_desc(qa + 32 * kk, 16, 8 * RB, SW),
+                     smem_desc(k_addr + 32 * kk, 16, 8 * RB, SW), idS, kk > 0);
+            mma_commit(&s_full[w * 2 + b]);
+          }
+          return true;
+        };
+        auto issue_PV = [&](int64_t i) -> bool {
+          const int s = (int)(i % kEncStages);
+          const uint32_t v_addr = smem_u32(smem + L::KV_OFF + s * 2 * L::TILE + L::TILE);
+          for (int k = 0; k < wg_count(i); ++k) {
+            const int w = wg_of(i, k);
+            const int64_t j = wg_tile(i);
+            const int b = (int)(j & 1);
+            if (!mbar_wait(&sp_done[w * 2 + b], (uint32_t)((j >> 1) & 1))) return false;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kEncTile / 16; ++kk)
+              mma_ts(tmem + TM_O + w * 32, tmem + TM_P + w * 64 + b * 32 + 8 * kk,
+                     smem_desc(v_addr + kk * 16 * RB, L::TILE, 8 * RB, SW), idPV,
+                     (j > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&pv_done[w]);
+          }
+          mma_commit(&kv_empty[s]);
+          return true;
+        };
+        if (ok && ntiles > 0) ok = issue_S(0);
+        if (ok && ntiles > 1) ok = issue_S(1);
+        if (NH == 1 && ok && ntiles > 2) ok = issue_S(2);
+        if (NH == 1 && ok && ntiles > 3) ok = issue_S(3);
+        const int ahead = (NH == 2) ? 2 : 4;   // S tiles in flight beyond the PV being issued
+        for (int64_t i = 0; ok && i < ntiles; ++i) {
+          ok = issue_PV(i);
+          if (ok && i + ahead < ntiles) ok = issue_S(i + ahead);
+          if (*abort_flag) ok = false;
+        }
+        if (!ok) {
+          record_error(err, kErrEncMmaWait);
+          *abort_flag = 1;
+        }
+        mma_commit(drain);
+        mbar_wait(drain, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------ softmax warpgroups
+    regs_acquire<kRegsSoftmax>();
+    const int w = warp >> 2, q = warp & 3;
+    const int r = q * 32 + lane;                     // TMEM lane = latent row in the half
+    const uint32_t lb = (uint32_t)(q * 32) << 16;
+    const uint32_t tO = tmem + lb + TM_O + w * 32;
+    const int64_t nW = (NH == 2) ? ntiles : (ntiles - w + 1) / 2;
+    float mref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int64_t j = 0; j < nW; ++j) {
+      const int64_t i = (NH == 2) ? j : 2 * j + w;
+      const int b = (int)(j & 1);
+      const int nvalid = (int)imin64(kEncTile, N - (tile0 + i) * kEncTile);
+      const uint32_t tS = tmem + lb + TM_S + w * 128 + b * 64;
+      const uint32_t tP = tmem + lb + TM_P + w * 64 + b * 32;
+      if (!mbar_wait(&s_full[w * 2 + b], (uint32_t)((j >> 1) & 1)) || *abort_flag) {
+        ok = false;
+        break;
+      }
+      __syncwarp();
+      tc_fence_after();
+      // pass 1: tile max of the raw logits (masked past the end of the head)
+      float mx = -INFINITY;
+#pragma unroll
+      for (int cc = 0; cc < kEncTile / 32; ++cc) {
+        uint32_t a[32];
+        tmem_ld32(tS + 32 * cc, a);
+        tmem_wait_ld();
+#pragma unroll
+        for (int t = 0; t < 32; ++t)
+          if (32 * cc + t < nvalid) mx = fmaxf(mx, __uint_as_float(a[t]));
+      }
+      const float mx2 = mx * c;
+      float factor = 1.f;
+      bool rescale = false;
+      if (mx2 > mref + kRescaleTau) {
+        rescale = (mref != -INFINITY);
+        factor = ex2(mref - mx2);
+        mref = mx2;
+      }
+      if (j > 0) {   // previous P.V done: O is stable and this P buffer is free
+        if (!mbar_wait(&pv_done[w], (uint32_t)((j - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        __syncwarp();
+        tc_fence_after();
+      }
+      if (rescale) {
+        l *= factor;
+        if (D == 32) {
+          uint32_t o[32];
+          tmem_ld32(tO, o);
+          tmem_wait_ld();
+          uint32_t lo[16], hi[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            lo[t] = __float_as_uint(__uint_as_float(o[t]) * factor);
+            hi[t] = __float_as_uint(__uint_as_float(o[16 + t]) * factor);
+          }
+          tmem_st16(tO, lo);
+          tmem_st16(tO + 16, hi);
+        } else {
+          uint32_t o[16];
+          tmem_ld16(tO, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 16; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * factor);
+          tmem_st16(tO, o);
+        }
+      }
+      // pass 2: P = 2^(c S - m_ref) as bf16 pairs, and its row sum
+      const float neg = -mref;
+      float sum = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < kEncTile / 32; ++cc) {
+        uint32_t a[32];
+        tmem_ld32(tS + 32 * cc, a);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          const int n0 = 32 * cc + 2 * t;
+          const float p0 = (n0 < nvalid) ? ex2(fmaf(__uint_as_float(a[2 * t]), c, neg)) : 0.f;
+          const float p1 =
+              (n0 + 1 < nvalid) ? ex2(fmaf(__uint_as_float(a[2 * t + 1]), c, neg)) : 0.f;
+          sum += p0 + p1;
+          pk[t] = pack_bf16(p0, p1);
+        }
+        tmem_st16(tP + 16 * cc, pk);
+      }
+      tmem_wait_st();
+      l += sum;
+      tc_fence_before();
+      mbar_arrive(&sp_done[w * 2 + b]);
+    }
+    float acc[D];
+#pragma unroll
+    for (int d = 0; d < D; ++d) acc[d] = 0.f;
+    if (ok && nW > 0) {
+      ok = mbar_wait(&pv_done[w], (uint32_t)((nW - 1) & 1));
+      __syncwarp();
+      tc_fence_after();
+      if (ok) {
+        if (D == 32) {
+          uint32_t o[32];
+          tmem_ld32(tO, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int d = 0; d < D; ++d) acc[d] = __uint_as_float(o[d]);
+        } else {
+          uint32_t o[16];
+          tmem_ld16(tO, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int d = 0; d < D; ++d) acc[d] = __uint_as_float(o[d & 15]);
+        }
+      }
+    }
+    if (!ok) {
+      record_error(err, kErrEncSoftmaxWait);
+      *abort_flag = 1;
+    } else {
+      const int64_t slot = bh * slots_per_bh + (int64_t)chunk * SUB + (NH == 1 ? w : 0);
+      const int64_t row = slot * M + (NH == 2 ? w * 128 : 0) + r;
+      part_ml[row * 2 + 0] = (nW > 0) ? mref : -INFINITY;
+      part_ml[row * 2 + 1] = l;
+      float4* dst = reinterpret_cast<float4*>(part_acc + row * D);
+#pragma unroll
+      for (int d = 0; d < D / 4; ++d)
+        dst[d] = make_float4(acc[4 * d], acc[4 * d + 1], acc[4 * d + 2], acc[4 * d + 3]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kWarpMma) tmem_dealloc(tmem, 512);
+}
+
+// ============================================================== decode
+
+template <int D, int M>
+struct DecLayout {
+  static constexpr int RB = 2 * D;
+  static constexpr int TILE = kTile * RB;
+  static constexpr int Q_OFF = 0;
+  static constexpr int Z_OFF = M * RB;
+  static constexpr int K_OFF = 2 * M * RB;
+  static constexpr int BAR_OFF = K_OFF + kDecStages * TILE;
+  static constexpr int NBARS = 2 * kDecStages + 1 + 4 * 2 + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+  static constexpr int BYTES = MISC_OFF + 16;
+};
+
+template <int D, int M>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmZ, int H, int64_t N, int q_per_batch,
+                     float c, int64_t tiles_per_bh, int64_t chunk_tiles,
+                     __nv_bfloat16* __restrict__ Y, uint32_t* __restrict__ err) {
+  using L = DecLayout<D, M>;
+  constexpr int RB = L::RB;
+  constexpr uint32_t SW = umma_swizzle_code(RB);
+  constexpr int R = M;                 // TMEM columns per warpgroup
+  constexpr uint32_t NCOLS = 2 * R;    // 256 or 512
+  constexpr int TY = M / 2;            // Y accumulator column inside a warpgroup's region
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* Qs = smem + L::Q_OFF;
+  uint8_t* Zs = smem + L::Z_OFF;
+  uint64_t* bars = (uint64_t*)(smem + L::BAR_OFF);
+  uint64_t* k_full = bars;
+  uint64_t* k_empty = bars + kDecStages;
+  uint64_t* qz_full = bars + 2 * kDecStages;
+  uint64_t* s_full = qz_full + 1;
+  uint64_t* s_empty = s_full + 2;
+  uint64_t* p_full = s_empty + 2;
+  uint64_t* y_full = p_full + 2;
+  uint64_t* drain = y_full + 2;
+  uint32_t* tmem_slot = (uint32_t*)(smem + L::MISC_OFF);
+  volatile int* abort_flag = (volatile int*)(smem + L::MISC_OFF + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x;
+  const int64_t bh = blockIdx.y;
+  const int64_t h = bh % H;
+  const int64_t tile0 = (int64_t)chunk * chunk_tiles;
+  const int64_t ntiles = imin64(chunk_tiles, tiles_per_bh - tile0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    mbar_init(qz_full, 1);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&s_full[w], 1);
+      mbar_init(&s_empty[w], 128);
+      mbar_init(&p_full[w], 128);
+      mbar_init(&y_full[w], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kWarpMma) tmem_alloc(tmem_slot, NCOLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp >= 8) {
+    regs_release<kRegsProducer>();
+    if (warp == kWarpTma) {
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmZ);
+      mbar_arrive_expect_tx(qz_full, 2 * M * RB);
+      tma_load_3d(Qs, &tmQ, qz_full, 0, 0, (int32_t)(q_per_batch ? bh : h));
+      tma_load_3d(Zs, &tmZ, qz_full, 0, 0, (int32_t)bh);
+      int64_t issued = 0;
+      for (int64_t i = 0; i < ntiles; ++i) {
+        const int s = (int)(i % kDecStages);
+        const uint32_t ph = (uint32_t)((i / kDecStages) & 1);
+        if (i >= kDecStages && !mbar_wait(&k_empty[s], ph ^ 1)) {
+          record_error(err, kErrDecTmaWait);
+          *abort_flag = 1;
+          break;
+        }
+        if (*abort_flag) break;
+        mbar_arrive_expect_tx(&k_full[s], L::TILE);
+        tma_load_3d(smem + L::K_OFF + s * L::TILE, &tmK, &k_full[s], 0,
+                    (int32_t)((tile0 + i) * kTile), (int32_t)bh);
+        issued = i + 1;
+      }
+      for (int64_t i = (issued > kDecStages ? issued - kDecStages : 0); i < issued; ++i)
+        mbar_wait(&k_full[i % kDecStages], (uint32_t)((i / kDecStages) & 1));
+      mbar_wait(qz_full, 0);
+    }
+  } else if (warp == kWarpMma) {
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, M, 0, 0);
+      constexpr uint32_t idY = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t q_addr = smem_u32(Qs);
+      const uint32_t z_addr = smem_u32(Zs);
+      bool ok = mbar_wait(qz_full, 0);
+      auto issue_S = [&](int64_t i) -> bool {
+        const int w = (int)(i & 1);
+        const int64_t j = i >> 1;
+        const int s = (int)(i % kDecStages);
+        if (!mbar_wait(&k_full[s], (uint32_t)((i / kDecStages) & 1))) return false;
+        if (j > 0 && !mbar_wait(&s_empty[w], (uint32_t)((j - 1) & 1))) return false;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(smem + L::K_OFF + s * L::TILE);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + w * R, smem_desc(k_addr + 32 * kk, 16, 8 * RB, SW),
+                 smem_desc(q_addr + 32 * kk, 16, 8 * RB, SW), idS, kk > 0);
+        mma_commit(&s_full[w]);
+        mma_commit(&k_empty[s]);
+        return true;
+      };
+      auto issue_Y = [&](int64_t i) -> bool {
+        const int w = (int)(i & 1);
+        const int64_t j = i >> 1;
+        if (!mbar_wait(&p_full[w], (uint32_t)(j & 1))) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < M / 16; ++kk) {
+          const uint32_t acol = (kk < M / 32) ? 8 * kk : M / 2 + 8 * kk;
+          mma_ts(tmem + w * R + TY, tmem + w * R + acol,
+                 smem_desc(z_addr + kk * 16 * RB, M * RB, 8 * RB, SW), idY, kk > 0);
+        }
+        mma_commit(&y_full[w]);
+        return true;
+      };
+      if (ok && ntiles > 0) ok = issue_S(0);
+      if (ok && ntiles > 1) ok = issue_S(1);
+      for (int64_t i = 0; ok && i < ntiles; ++i) {
+        ok = issue_Y(i);
+        if (ok && i + 2 < ntiles) ok = issue_S(i + 2);
+        if (*abort_flag) ok = false;
+      }
+      if (!ok) {
+        record_error(err, kErrDecMmaWait);
+        *abort_flag = 1;
+      }
+      mma_commit(drain);
+      mbar_wait(drain, 0);
+    }
+    }
+  } else {
+    regs_acquire<kRegsSoftmax>();
+    const int w = warp >> 2, q = warp & 3;
+    const int r = q * 32 + lane;                     // TMEM lane = token row in the tile
+    const uint32_t lb = (uint32_t)(q * 32) << 16;
+    const uint32_t tR = tmem + lb + w * R;
+    const int64_t nW = (ntiles - w + 1) / 2;
+    bool ok = true;
+    for (int64_t j = 0; j < nW; ++j) {
+      const int64_t i = 2 * j + w;
+      const int64_t tok = (tile0 + i) * kTile + r;
+      if (!mbar_wait(&s_full[w], (uint32_t)(j & 1)) || *abort_flag) {
+        ok = false;
+        break;
+      }
+      __syncwarp();
+      tc_fence_after();
+      // pass 1: row max over all M logits
+      float mx = -INFINITY;
+#pragma unroll
+      for (int cc = 0; cc < M / 32; ++cc) {
+        uint32_t a[32];
+        tmem_ld32(tR + 32 * cc, a);
+        tmem_wait_ld();
+#pragma unroll
+        for (int t = 0; t < 32; ++t) mx = fmaxf(mx, __uint_as_float(a[t]));
+      }
+      const float neg = -mx * c;
+      float sum = 0.f;
+      // pass 2, upper half of the latents, last chunk first: P of S columns
+      // [M/2 + 32cc, +32) goes to columns [3M/4 + 16cc, +16), which hold
+      // S chunks already read (chunk index M/128 + cc/2 >= cc).
+#pragma unroll
+      for (int cc = M / 64 - 1; cc >= 0; --cc) {
+        uint32_t a[32];
+        tmem_ld32(tR + M / 2 + 32 * cc, a);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          const float p0 = ex2(fmaf(__uint_as_float(a[2 * t]), c, neg));
+          const float p1 = ex2(fmaf(__uint_as_float(a[2 * t + 1]), c, neg));
+          sum += p0 + p1;
+          pk[t] = pack_bf16(p0, p1);
+        }
+        tmem_st16(tR + 3 * M / 4 + 16 * cc, pk);
+      }
+      // pass 2, lower half, first chunk first: P of S columns [32cc, +32)
+      // goes to columns [16cc, +16), inside chunks already read.
+#pragma unroll
+      for (int cc = 0; cc < M / 64; ++cc) {
+        uint32_t a[32];
+        tmem_ld32(tR + 32 * cc, a);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          const float p0 = ex2(fmaf(__uint_as_float(a[2 * t]), c, neg));
+          const float p1 = ex2(fmaf(__uint_as_float(a[2 * t + 1]), c, neg));
+          sum += p0 + p1;
+          pk[t] = pack_bf16(p0, p1);
+        }
+        tmem_st16(tR + 16 * cc, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[w]);
+      if (!mbar_wait(&y_full[w], (uint32_t)(j & 1))) {
+        ok = false;
+        break;
+      }
+      __syncwarp();
+      tc_fence_after();
+      float y[D];
+      if (D == 32) {
+        uint32_t o[32];
+        tmem_ld32(tR + TY, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int d = 0; d < D; ++d) y[d] = __uint_as_float(o[d]);
+      } else {
+        uint32_t o[16];
+        tmem_ld16(tR + TY, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int d = 0; d < D; ++d) y[d] = __uint_as_float(o[d & 15]);
+      }
+      tc_fence_before();
+      mbar_arrive(&s_empty[w]);
+      if (tok < N) {
+        const float inv = 1.f / sum;
+        uint4* dst = reinterpret_cast<uint4*>(Y + (bh * N + tok) * D);
+#pragma unroll
+        for (int v = 0; v < D / 8; ++v) {
+          uint4 u;
+          u.x = pack_bf16(y[8 * v + 0] * inv, y[8 * v + 1] * inv);
+          u.y = pack_bf16(y[8 * v + 2] * inv, y[8 * v + 3] * inv);
+          u.z = pack_bf16(y[8 * v + 4] * inv, y[8 * v + 5] * inv);
+          u.w = pack_bf16(y[8 * v + 6] * inv, y[8 * v + 7] * inv);
+          dst[v] = u;
+        }
+      }
+    }
+    if (!ok) {
+      record_error(err, kErrDecSoftmaxWait);
+      *abort_flag = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kWarpMma) tmem_dealloc(tmem, NCOLS);
+}
+
+// ============================================================== host side
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return (PFN_cuTensorMapEncodeTiled_v12000)p;
+  }();
+  return fn;
+}
+
+// 3-D map over a bf16 tensor [depth][rows][D] with boxes of box_rows rows,
+// swizzled to match the UMMA descriptors (row = whole head dimension).
+cudaError_t make_map(CUtensorMap* m, const void* base, int D, int64_t rows, int64_t depth,
+                     int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) {
+    note_error("cuTensorMapEncodeTiled entry point unavailable");
+    return cudaErrorNotSupported;
+  }
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)depth};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
+  cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  const CUtensorMapSwizzle sw = (D == 32) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    note_error("cuTensorMapEncodeTiled failed (CUresult %d): D=%d rows=%lld depth=%lld box=%d",
+               (int)r, D, (long long)rows, (long long)depth, box_rows);
+    return cudaErrorInvalidValue;
+  }
+  return cudaSuccess;
+}
+
+template <int D, int M>
+cudaError_t tc_encode_t(const void* Q, int64_t qbs, const void* K, const void* V, const Dims& d,
+                        float scale, const ChunkPlan& plan, float* pml, float* pacc,
+                        uint32_t* err, cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  const int q_per_batch = qbs != 0;
+  cudaError_t e;
+  if ((e = make_map(&mq, Q, D, M, q_per_batch ? d.BH() : d.H, 128)) != cudaSuccess) return e;
+  if ((e = make_map(&mk, K, D, d.N, d.BH(), kEncTile)) != cudaSuccess) return e;
+  if ((e = make_map(&mv, V, D, d.N, d.BH(), kEncTile)) != cudaSuccess) return e;
+  const int smem = (EncLayout<D, M>::BYTES + 1024 > kMinSmemBytes) ? EncLayout<D, M>::BYTES + 1024
+                                                                   : kMinSmemBytes;
+  e = cudaFuncSetAttribute(tc_encode_kernel<D, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(plan.chunks, (unsigned)d.BH());
+  tc_encode_kernel<D, M><<<grid, kThreads, smem, st>>>(
+      mq, mk, mv, (int)d.H, d.N, q_per_batch, scale * kLog2e, plan.tiles_per_bh, plan.chunk_tiles,
+      plan.slots_per_bh(), pml, pacc, err);
+  return cudaPeekAtLastError();
+}
+
+template <int D, int M>
+cudaError_t tc_decode_t(const void* Q, int64_t qbs, const void* K, const __nv_bfloat16* Zb,
+                        void* Y, const Dims& d, float scale, const ChunkPlan& plan, uint32_t* err,
+                        cudaStream_t st) {
+  CUtensorMap mq, mk, mz;
+  const int q_per_batch = qbs != 0;
+  cudaError_t e;
+  if ((e = make_map(&mq, Q, D, M, q_per_batch ? d.BH() : d.H, M)) != cudaSuccess) return e;
+  if ((e = make_map(&mk, K, D, d.N, d.BH(), kTile)) != cudaSuccess) return e;
+  if ((e = make_map(&mz, Zb, D, M, d.BH(), M)) != cudaSuccess) return e;
+  const int smem = (DecLayout<D, M>::BYTES + 1024 > kMinSmemBytes) ? DecLayout<D, M>::BYTES + 1024
+                                                                   : kMinSmemBytes;
+  e = cudaFuncSetAttribute(tc_decode_kernel<D, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(plan.chunks, (unsigned)d.BH());
+  tc_decode_kernel<D, M><<<grid, kThreads, smem, st>>>(mq, mk, mz, (int)d.H, d.N, q_per_batch,
+                                                       scale * kLog2e, plan.tiles_per_bh,
+                                                       plan.chunk_tiles, (__nv_bfloat16*)Y, err);
+  return cudaPeekAtLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_tc_encode(const void* Q, int64_t qbs, const void* K, const void* V,
+                             const Dims& d, float scale, const ChunkPlan& plan, float* pml,
+                             float* pacc, uint32_t* err, cudaStream_t st) {
+  if (d.D == 32 && d.M == 256) return tc_encode_t<32, 256>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
+  if (d.D == 32 && d.M == 128) return tc_encode_t<32, 128>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
+  if (d.D == 16 && d.M == 256) return tc_encode_t<16, 256>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
+  if (d.D == 16 && d.M == 128) return tc_encode_t<16, 128>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
   return cudaErrorNotSupported;
 }
 
-cudaError_t launch_tc_decode(const void*, int64_t, const void*, const __nv_bfloat16*, void*,
-                             const Dims&, float, const ChunkPlan&, uint32_t*, cudaStream_t) {
+cudaError_t launch_tc_decode(const void* Q, int64_t qbs, const void* K, const __nv_bfloat16* Zb,
+                             void* Y, const Dims& d, float scale, const ChunkPlan& plan,
+                             uint32_t* err, cudaStream_t st) {
+  if (d.D == 32 && d.M == 256) return tc_decode_t<32, 256>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
+  if (d.D == 32 && d.M == 128) return tc_decode_t<32, 128>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
+  if (d.D == 16 && d.M == 256) return tc_decode_t<16, 256>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
+  if (d.D == 16 && d.M == 128) return tc_decode_t<16, 128>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
   return cudaErrorNotSupported;
 }
 
