@@ -182,6 +182,16 @@ def oracle_sample_rate(target_s: float, w=WORKLOAD, seed: int = 0):
 
 # ------------------------------------------------------------------ ours
 
+def workload_from_args(args):
+    """The headline workload, or a smaller one of the same per-head shape for
+    profiling captures (--heads / --seq)."""
+    import dataclasses
+    w = WORKLOAD
+    if args.heads or args.seq:
+        w = dataclasses.replace(w, name=w.name + "_reduced", H=args.heads or w.H, N=args.seq or w.N)
+    return w
+
+
 def roofline_entry(kernel_ms: dict, peaks: dict, peak_kind: str, w=WORKLOAD):
     """Roofline of the dominant kernel (largest average duration).
 
@@ -244,7 +254,7 @@ def run_ours(args, rank, world, local):
 
     import rank_latent_attention_flare_b200 as fl
 
-    w = WORKLOAD
+    w = workload_from_args(args)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     x = make_inputs(w.B, w.H, w.N, w.M, w.D, dtype=w.torch_dtype, seed=rank)
@@ -335,7 +345,7 @@ def run_ours(args, rank, world, local):
         del hx, hY, dX
 
     peaks, peak_kind = load_peaks()
-    roof = roofline_entry(kernel_ms, peaks, peak_kind)
+    roof = roofline_entry(kernel_ms, peaks, peak_kind, w)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -417,6 +427,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=120.0)
     ap.add_argument("--out-dir", default=None, help="where to write the clock samples")
+    ap.add_argument("--heads", type=int, default=0, help="override H (profiling captures only)")
+    ap.add_argument("--seq", type=int, default=0, help="override N (profiling captures only)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")

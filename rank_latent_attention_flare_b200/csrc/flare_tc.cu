@@ -250,17 +250,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       tc_fence_after();
+      const bool full = (nvalid == kEncTile);   // warp-uniform: only a head's last tile is partial
       // pass 1: tile max of the raw logits (masked past the end of the head)
-      float mx = -INFINITY;
+      float mf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int cc = 0; cc < kEncTile / 32; ++cc) {
         uint32_t a[32];
         tmem_ld32(tS + 32 * cc, a);
         tmem_wait_ld();
+        if (full) {
+          max_fold32(a, mf);
+        } else {
 #pragma unroll
-        for (int t = 0; t < 32; ++t)
-          if (32 * cc + t < nvalid) mx = fmaxf(mx, __uint_as_float(a[t]));
+          for (int t = 0; t < 32; ++t)
+            if (32 * cc + t < nvalid) mf[t & 3] = fmaxf(mf[t & 3], __uint_as_float(a[t]));
+        }
       }
+      const float mx = fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3]));
       const float mx2 = mx * c;
       float factor = 1.f;
       bool rescale = false;
@@ -302,26 +308,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // pass 2: P = 2^(c S - m_ref) as bf16 pairs, and its row sum
       const float neg = -mref;
-      float sum = 0.f;
+      float sf[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int cc = 0; cc < kEncTile / 32; ++cc) {
         uint32_t a[32];
         tmem_ld32(tS + 32 * cc, a);
         tmem_wait_ld();
-        uint32_t pk[16];
+        if (!full) {   // tokens past the end of the head get weight 0
 #pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          const int n0 = 32 * cc + 2 * t;
-          const float p0 = (n0 < nvalid) ? ex2(fmaf(__uint_as_float(a[2 * t]), c, neg)) : 0.f;
-          const float p1 =
-              (n0 + 1 < nvalid) ? ex2(fmaf(__uint_as_float(a[2 * t + 1]), c, neg)) : 0.f;
-          sum += p0 + p1;
-          pk[t] = pack_bf16(p0, p1);
+          for (int t = 0; t < 32; ++t)
+            if (32 * cc + t >= nvalid) a[t] = __float_as_uint(-INFINITY);
         }
+        uint32_t pk[16];
+        exp_pack32(a, c, neg, pk, sf);
         tmem_st16(tP + 16 * cc, pk);
       }
       tmem_wait_st();
-      l += sum;
+      l += (sf[0] + sf[1]) + (sf[2] + sf[3]);
       tc_fence_before();
       mbar_arrive(&sp_done[w * 2 + b]);
     }
@@ -541,17 +544,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       tc_fence_after();
       // pass 1: row max over all M logits
-      float mx = -INFINITY;
+      float mf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int cc = 0; cc < M / 32; ++cc) {
         uint32_t a[32];
         tmem_ld32(tR + 32 * cc, a);
         tmem_wait_ld();
-#pragma unroll
-        for (int t = 0; t < 32; ++t) mx = fmaxf(mx, __uint_as_float(a[t]));
+        max_fold32(a, mf);
       }
+      const float mx = fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3]));
       const float neg = -mx * c;
-      float sum = 0.f;
+      float sf[4] = {0.f, 0.f, 0.f, 0.f};
       // pass 2, upper half of the latents, last chunk first: P of S columns
       // [M/2 + 32cc, +32) goes to columns [3M/4 + 16cc, +16), which hold
       // S chunks already read (chunk index M/128 + cc/2 >= cc).
@@ -561,13 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tR + M / 2 + 32 * cc, a);
         tmem_wait_ld();
         uint32_t pk[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          const float p0 = ex2(fmaf(__uint_as_float(a[2 * t]), c, neg));
-          const float p1 = ex2(fmaf(__uint_as_float(a[2 * t + 1]), c, neg));
-          sum += p0 + p1;
-          pk[t] = pack_bf16(p0, p1);
-        }
+        exp_pack32(a, c, neg, pk, sf);
         tmem_st16(tR + 3 * M / 4 + 16 * cc, pk);
       }
       // pass 2, lower half, first chunk first: P of S columns [32cc, +32)
@@ -578,13 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tR + 32 * cc, a);
         tmem_wait_ld();
         uint32_t pk[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          const float p0 = ex2(fmaf(__uint_as_float(a[2 * t]), c, neg));
-          const float p1 = ex2(fmaf(__uint_as_float(a[2 * t + 1]), c, neg));
-          sum += p0 + p1;
-          pk[t] = pack_bf16(p0, p1);
-        }
+        exp_pack32(a, c, neg, pk, sf);
         tmem_st16(tR + 16 * cc, pk);
       }
       tmem_wait_st();
@@ -613,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&s_empty[w]);
       if (tok < N) {
-        const float inv = 1.f / sum;
+        const float inv = 1.f / ((sf[0] + sf[1]) + (sf[2] + sf[3]));
         uint4* dst = reinterpret_cast<uint4*>(Y + (bh * N + tok) * D);
 #pragma unroll
         for (int v = 0; v < D / 8; ++v) {

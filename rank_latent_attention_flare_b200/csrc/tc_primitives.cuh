@@ -233,9 +233,43 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Max of 32 values folded into four independent accumulators.
+__device__ __forceinline__ void max_fold32(const uint32_t (&a)[32], float (&m)[4]) {
+#pragma unroll
+  for (int t = 0; t < 32; t += 8) {
+    m[0] = max3(m[0], __uint_as_float(a[t + 0]), __uint_as_float(a[t + 1]));
+    m[1] = max3(m[1], __uint_as_float(a[t + 2]), __uint_as_float(a[t + 3]));
+    m[2] = max3(m[2], __uint_as_float(a[t + 4]), __uint_as_float(a[t + 5]));
+    m[3] = max3(m[3], __uint_as_float(a[t + 6]), __uint_as_float(a[t + 7]));
+  }
+}
+
+// p = 2^(a*c + neg) for 32 logits: packed into 16 bf16 pairs, sums folded
+// into four independent accumulators.
+__device__ __forceinline__ void exp_pack32(const uint32_t (&a)[32], float c, float neg,
+                                           uint32_t (&pk)[16], float (&s)[4]);
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void exp_pack32(const uint32_t (&a)[32], float c, float neg,
+                                           uint32_t (&pk)[16], float (&s)[4]) {
+#pragma unroll
+  for (int t = 0; t < 16; ++t) {
+    const float p0 = ex2(fmaf(__uint_as_float(a[2 * t]), c, neg));
+    const float p1 = ex2(fmaf(__uint_as_float(a[2 * t + 1]), c, neg));
+    s[t & 3] += p0 + p1;
+    pk[t] = pack_bf16(p0, p1);
+  }
 }
 
 }  // namespace tc
