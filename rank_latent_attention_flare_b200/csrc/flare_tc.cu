@@ -253,17 +253,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool full = (nvalid == kEncTile);   // warp-uniform: only a head's last tile is partial
       // pass 1: tile max of the raw logits (masked past the end of the head)
       float mf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      uint32_t a[2][32];
+      tmem_ld32(tS, a[0]);
 #pragma unroll
       for (int cc = 0; cc < kEncTile / 32; ++cc) {
-        uint32_t a[32];
-        tmem_ld32(tS + 32 * cc, a);
-        tmem_wait_ld();
+        tmem_wait_ld_dep(a[cc & 1]);
+        if (cc + 1 < kEncTile / 32) tmem_ld32(tS + 32 * (cc + 1), a[(cc + 1) & 1]);
         if (full) {
-          max_fold32(a, mf);
+          max_fold32(a[cc & 1], mf);
         } else {
 #pragma unroll
           for (int t = 0; t < 32; ++t)
-            if (32 * cc + t < nvalid) mf[t & 3] = fmaxf(mf[t & 3], __uint_as_float(a[t]));
+            if (32 * cc + t < nvalid) mf[t & 3] = fmaxf(mf[t & 3], __uint_as_float(a[cc & 1][t]));
         }
       }
       const float mx = fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3]));
@@ -309,18 +310,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       // pass 2: P = 2^(c S - m_ref) as bf16 pairs, and its row sum
       const float neg = -mref;
       float sf[4] = {0.f, 0.f, 0.f, 0.f};
+      tmem_ld32(tS, a[0]);
 #pragma unroll
       for (int cc = 0; cc < kEncTile / 32; ++cc) {
-        uint32_t a[32];
-        tmem_ld32(tS + 32 * cc, a);
-        tmem_wait_ld();
+        tmem_wait_ld_dep(a[cc & 1]);
+        if (cc + 1 < kEncTile / 32) tmem_ld32(tS + 32 * (cc + 1), a[(cc + 1) & 1]);
         if (!full) {   // tokens past the end of the head get weight 0
 #pragma unroll
           for (int t = 0; t < 32; ++t)
-            if (32 * cc + t >= nvalid) a[t] = __float_as_uint(-INFINITY);
+            if (32 * cc + t >= nvalid) a[cc & 1][t] = __float_as_uint(-INFINITY);
         }
         uint32_t pk[16];
-        exp_pack32(a, c, neg, pk, sf);
+        exp_pack32(a[cc & 1], c, neg, pk, sf);
         tmem_st16(tP + 16 * cc, pk);
       }
       tmem_wait_st();
@@ -544,39 +545,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       tc_fence_after();
       // pass 1: row max over all M logits
+      // Chunks of 32 columns are double-buffered: the load of the next chunk
+      // is in flight while the current one is processed.
+      constexpr int NC = M / 32;
+      uint32_t a[2][32];
       float mf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      tmem_ld32(tR, a[0]);
 #pragma unroll
-      for (int cc = 0; cc < M / 32; ++cc) {
-        uint32_t a[32];
-        tmem_ld32(tR + 32 * cc, a);
-        tmem_wait_ld();
-        max_fold32(a, mf);
+      for (int cc = 0; cc < NC; ++cc) {
+        tmem_wait_ld_dep(a[cc & 1]);
+        if (cc + 1 < NC) tmem_ld32(tR + 32 * (cc + 1), a[(cc + 1) & 1]);
+        max_fold32(a[cc & 1], mf);
       }
       const float mx = fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3]));
       const float neg = -mx * c;
       float sf[4] = {0.f, 0.f, 0.f, 0.f};
-      // pass 2, upper half of the latents, last chunk first: P of S columns
-      // [M/2 + 32cc, +32) goes to columns [3M/4 + 16cc, +16), which hold
-      // S chunks already read (chunk index M/128 + cc/2 >= cc).
+      // pass 2 visits the chunks in the order: upper half last chunk first,
+      // then lower half first chunk first.  The P of upper chunk u (S columns
+      // [M/2 + 32u, +32)) goes to columns [3M/4 + 16u, +16), inside upper
+      // chunks already read; the P of lower chunk u goes to [16u, +16),
+      // inside lower chunks already read.  No store touches a chunk that is
+      // still to be loaded.
+      auto chunk_col = [](int k) { return k < NC / 2 ? M / 2 + 32 * (NC / 2 - 1 - k) : 32 * (k - NC / 2); };
+      auto p_col = [](int k) { return k < NC / 2 ? 3 * M / 4 + 16 * (NC / 2 - 1 - k) : 16 * (k - NC / 2); };
+      tmem_ld32(tR + chunk_col(0), a[0]);
 #pragma unroll
-      for (int cc = M / 64 - 1; cc >= 0; --cc) {
-        uint32_t a[32];
-        tmem_ld32(tR + M / 2 + 32 * cc, a);
-        tmem_wait_ld();
+      for (int k = 0; k < NC; ++k) {
+        tmem_wait_ld_dep(a[k & 1]);
+        if (k + 1 < NC) tmem_ld32(tR + chunk_col(k + 1), a[(k + 1) & 1]);
         uint32_t pk[16];
-        exp_pack32(a, c, neg, pk, sf);
-        tmem_st16(tR + 3 * M / 4 + 16 * cc, pk);
-      }
-      // pass 2, lower half, first chunk first: P of S columns [32cc, +32)
-      // goes to columns [16cc, +16), inside chunks already read.
-#pragma unroll
-      for (int cc = 0; cc < M / 64; ++cc) {
-        uint32_t a[32];
-        tmem_ld32(tR + 32 * cc, a);
-        tmem_wait_ld();
-        uint32_t pk[16];
-        exp_pack32(a, c, neg, pk, sf);
-        tmem_st16(tR + 16 * cc, pk);
+        exp_pack32(a[k & 1], c, neg, pk, sf);
+        tmem_st16(tR + p_col(k), pk);
       }
       tmem_wait_st();
       tc_fence_before();
