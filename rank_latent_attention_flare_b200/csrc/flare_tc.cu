@@ -18,9 +18,9 @@
 // Roles per CTA (384 threads, three warpgroups): warps 0-3 and 4-7 are two
 // softmax warpgroups, warp 8 issues TMA loads, warp 9 owns TMEM and issues
 // the MMAs, warps 10-11 only lend their registers.  The CTA launches at 168
-// registers per thread; the producer warpgroup drops to 56 and the softmax
-// warpgroups rise to 224 (2 x 128 x 224 + 128 x 56 = 384 x 168, and each SM
-// sub-partition keeps 2 x 224 + 56 registers x 32 lanes <= 16384).
+// registers per thread; the producer warpgroup moves to 104 and the softmax
+// warpgroups to 200 (2 x 128 x 200 + 128 x 104 = 384 x 168, and each SM
+// sub-partition holds 2 x 200 + 104 <= 512 registers per lane).
 // Exponentials use ex2.approx (MUFU); c = scale * log2(e) is folded in.
 #include <cudaTypedefs.h>
 
@@ -34,8 +34,8 @@ using namespace tc;
 
 constexpr int kTile = 128;        // tokens per tile (MMA M or N)
 constexpr int kThreads = 384;
-constexpr int kRegsSoftmax = 224;
-constexpr int kRegsProducer = 56;
+constexpr int kRegsSoftmax = 200;
+constexpr int kRegsProducer = 104;
 constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
 constexpr int kEncStages = 8;
