@@ -82,7 +82,8 @@ FLARE_API int flare_version(void);
 
 /*
  * Description of the last FLARE_ERR_CUDA returned on the calling host thread
- * (the failing call and the CUDA error name), or "" if none.  Thread-local
+ * (the failing call and the CUDA error name), or of a size rejection by
+ * flare_fwd_noalloc, or "" if none.  Thread-local
  * storage, valid until the next FLARE call on this thread.
  */
 FLARE_API const char* flare_last_error_detail(void);
@@ -167,6 +168,38 @@ FLARE_API flare_status_t flare_decode(const void* Q, int64_t q_batch_stride, con
                             int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
                             flare_dtype_t dtype, float scale, void* workspace,
                             size_t workspace_bytes, void* stream);
+
+/*
+ * Size of the fixed scratch array behind flare_fwd_noalloc (32 MiB).  Every
+ * GPU that loads this library holds one such array until the process exits.
+ */
+#define FLARE_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * FLARE forward for callers that cannot allocate device memory -- a plugin
+ * inside a framework that owns every device allocation and passes its
+ * plugins no workspace, or a running latency-critical loop where cudaMalloc
+ * (which can synchronise the device) is not allowed.  The papers have no
+ * counterpart to this call; it is an interface convenience.
+ *
+ * Same arguments, layouts and results as flare_fwd, minus the workspace:
+ * the scratch lives in a file-scope device array of
+ * FLARE_NOALLOC_SCRATCH_BYTES bytes.  The call allocates and frees nothing.
+ * Sizes whose flare_workspace_size(FLARE_OP_FWD, ...) exceeds that limit
+ * are rejected with FLARE_ERR_WORKSPACE before anything is enqueued
+ * (flare_last_error_detail says why); use flare_fwd for them.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture.  All calls on a device share the
+ * array: calls whose work overlaps on the GPU (other streams or host
+ * threads, same device) race on it and must be serialised by the caller.
+ */
+FLARE_API flare_status_t flare_fwd_noalloc(const void* Q, int64_t q_batch_stride, const void* K,
+                                           const void* V, void* Y, int64_t B, int64_t H,
+                                           int64_t N, int64_t M, int64_t D, flare_dtype_t dtype,
+                                           float scale, float* Z_save, float* lse_save,
+                                           void* stream);
 
 /*
  * Reads and clears the device error word in the workspace header.  This

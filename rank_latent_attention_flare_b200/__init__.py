@@ -5,14 +5,15 @@ tensor-core kernels and CUDA-core kernels) behind the C ABI declared in
 ``include/flare.h``.  This package is a thin ctypes binding over it.
 """
 from ._lib import (FLARE_BF16, FLARE_F32, FLARE_OP_BWD, FLARE_OP_FWD, FLARE_OP_PP_FWD,
-                   FlareError, LIB_PATH, SIGNATURES, load)
+                   NOALLOC_SCRATCH_BYTES, FlareError, LIB_PATH, SIGNATURES, load)
 from .flare import (alloc_workspace, default_scale, device_status, flare_bwd, flare_combine,
-                    flare_decode, flare_encode, flare_fwd, flare_pp_fwd, fwd_path,
-                    workspace_size)
+                    flare_decode, flare_encode, flare_fwd, flare_fwd_noalloc, flare_pp_fwd,
+                    fwd_path, workspace_size)
 
 __all__ = [
     "FLARE_BF16", "FLARE_F32", "FLARE_OP_BWD", "FLARE_OP_FWD", "FLARE_OP_PP_FWD", "FlareError",
     "LIB_PATH", "SIGNATURES", "load", "alloc_workspace", "default_scale", "device_status",
-    "flare_bwd", "flare_combine", "flare_decode", "flare_encode", "flare_fwd", "flare_pp_fwd",
+    "flare_bwd", "flare_combine", "flare_decode", "flare_encode", "flare_fwd", "flare_fwd_noalloc",
+    "flare_pp_fwd", "NOALLOC_SCRATCH_BYTES",
     "fwd_path", "workspace_size",
 ]

@@ -18,6 +18,9 @@ FLARE_OP_FWD = 0
 FLARE_OP_PP_FWD = 1
 FLARE_OP_BWD = 2
 
+# Size of the fixed device scratch array behind flare_fwd_noalloc.
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
 STATUS_NAMES = {
     0: "FLARE_OK",
     1: "FLARE_ERR_INVALID_ARG",
@@ -53,6 +56,8 @@ SIGNATURES = {
                             _sz, _vp]),
     "flare_device_status": (_i32, [_vp, _sz, _u32p, _vp]),
     "flare_fwd_path": (_i32, [_i64, _i64, _i64, _i64, _i64, _i32]),
+    "flare_fwd_noalloc": (_i32, [_vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i32,
+                                 _f32, _vp, _vp, _vp]),
 }
 
 _lib = None

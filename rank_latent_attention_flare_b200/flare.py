@@ -184,3 +184,30 @@ def flare_decode(Q, K, scale: Optional[float] = None, *, workspace: torch.Tensor
                                   s, _ptr(workspace), workspace.numel(), _stream(stream))
     _lib.check(st, "flare_decode")
     return Y
+
+
+def flare_fwd_noalloc(Q, K, V, scale: Optional[float] = None, *, save: bool = False,
+                      out: Optional[torch.Tensor] = None, stream=None):
+    """FLARE forward without a workspace, for callers that cannot allocate.
+
+    The library keeps the scratch in a fixed device array of
+    ``NOALLOC_SCRATCH_BYTES`` bytes shared by every call on the device, so
+    calls that overlap on the GPU race; sizes that need more scratch raise
+    FlareError(FLARE_ERR_WORKSPACE).  This wrapper still allocates the
+    outputs with torch for convenience; the C entry point allocates nothing.
+    """
+    _need_cuda(Q, K, V, out)
+    B, H, N, M, D, qbs = _dims(Q, K)
+    dt = _dtype_code(K)
+    s = default_scale(D) if scale is None else float(scale)
+    Y = torch.empty_like(K) if out is None else out
+    Z = torch.empty((B, H, M, D), dtype=torch.float32, device=K.device) if save else None
+    lse = torch.empty((B, H, M), dtype=torch.float32, device=K.device) if save else None
+    lib = _lib.load()
+    st = lib.flare_fwd_noalloc(_ptr(Q), qbs, _ptr(K), _ptr(V), _ptr(Y), B, H, N, M, D, dt, s,
+                               _ptr(Z), _ptr(lse), _stream(stream))
+    if st == 3:
+        detail = (lib.flare_last_error_detail() or b"").decode(errors="replace")
+        raise FlareError(st, "flare_fwd_noalloc" + (f" [{detail}]" if detail else ""))
+    _lib.check(st, "flare_fwd_noalloc")
+    return (Y, Z, lse) if save else Y
