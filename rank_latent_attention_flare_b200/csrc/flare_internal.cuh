@@ -95,7 +95,8 @@ inline ChunkPlan encode_plan(int64_t BH, int64_t N, int64_t M, int64_t D, flare_
                              int sms) {
   Path path = choose_path(N, M, D, dt);
   if (path.tc_fwd) {
-    ChunkPlan p = plan_chunks(BH, N, kTcEncTile, sms, 12.0, 16 * (int64_t)sms);
+    // two encode CTAs are resident per SM
+    ChunkPlan p = plan_chunks(BH, N, kTcEncTile, 2LL * sms, 12.0, 32 * (int64_t)sms);
     p.sub = (M == 128) ? 2 : 1;
     return p;
   }

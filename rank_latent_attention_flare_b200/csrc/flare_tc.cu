@@ -49,12 +49,15 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 
 // ============================================================== encode
 //
-// Tiles of kEncTile = 64 tokens.  TMEM (512 columns): S[w][b] at w*128 + b*64
-// (two 64-column S buffers per warpgroup, so the MMA computes the next tile's
-// logits while the softmax works on this one), P[w][b] at 256 + w*64 + b*32
-// (bf16 pairs), O[w] at 384 + w*32.  With M = 256 warpgroup w owns latent
-// rows [128w, 128w+128) of every tile; with M = 128 the warpgroups take
-// alternate tiles and each keeps its own running record.
+// Tiles of kEncTile = 64 tokens.  Each softmax warpgroup w has SB S buffers
+// of 64 TMEM columns, SB P buffers of 32 columns (bf16 pairs) and an O
+// accumulator of 32 columns: S[w][b] at (w*SB + b)*64, P[w][b] at
+// 128*SB + (w*SB + b)*32, O[w] at 192*SB + 32w.  SB = 1 needs 256 columns,
+// so two CTAs share an SM and their four softmax warpgroups hide each
+// other's latencies; SB = 2 (448 columns, one CTA per SM) lets the MMA fill
+// the next S buffer while the softmax works on this one.  With M = 256
+// warpgroup w owns latent rows [128w, 128w+128) of every tile; with M = 128
+// the warpgroups take alternate tiles and each keeps its own running record.
 
 constexpr int kEncTile = 64;
 
@@ -65,13 +68,19 @@ struct EncLayout {
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = M * RB;
   static constexpr int BAR_OFF = KV_OFF + kEncStages * 2 * TILE;
-  static constexpr int NBARS = 2 * kEncStages + 1 + 4 + 4 + 2 + 1;
+  static constexpr int NBARS = 2 * kEncStages + 1 + 4 + 4 + 2 + 1;   // sized for SB <= 2
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
 };
 
-template <int D, int M>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int SB>
+struct EncRegs {   // setmaxnreg split; launch cap is 168 (SB = 2) or 80 (SB = 1)
+  static constexpr int kSoftmax = (SB == 2) ? kRegsSoftmax : 88;
+  static constexpr int kProducer = (SB == 2) ? kRegsProducer : 56;
+};
+
+template <int D, int M, int SB>
+__global__ void __launch_bounds__(kThreads, (SB == 1) ? 2 : 1)
     tc_encode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, int H, int64_t N, int q_per_batch,
                      float c, int64_t tiles_per_bh, int64_t chunk_tiles, int slots_per_bh,
@@ -82,7 +91,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int SUB = (NH == 1) ? 2 : 1;
   constexpr int RB = L::RB;
   constexpr uint32_t SW = umma_swizzle_code(RB);
-  constexpr uint32_t TM_S = 0, TM_P = 256, TM_O = 384;   // TMEM column bases
+  constexpr uint32_t TM_S = 0, TM_P = 128 * SB, TM_O = 192 * SB;   // TMEM column bases
+  constexpr uint32_t TM_COLS = (SB == 1) ? 256 : 512;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -91,8 +101,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = bars + kEncStages;
   uint64_t* q_full = bars + 2 * kEncStages;
-  uint64_t* s_full = q_full + 1;      // [w*2 + b]
-  uint64_t* sp_done = s_full + 4;     // [w*2 + b]: S read and P written
+  uint64_t* s_full = q_full + 1;      // [w*SB + b]
+  uint64_t* sp_done = s_full + 4;     // [w*SB + b]: S read and P written
   uint64_t* pv_done = sp_done + 4;    // [w]
   uint64_t* drain = pv_done + 2;
   uint32_t* tmem_slot = (uint32_t*)(smem + L::MISC_OFF);
@@ -121,14 +131,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kWarpMma) tmem_alloc(tmem_slot, 512);
+  if (warp == kWarpMma) tmem_alloc(tmem_slot, TM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= 8) {
-    regs_release<kRegsProducer>();
+    regs_release<EncRegs<SB>::kProducer>();
     if (warp == kWarpTma) {
       // ---------------------------------------------------- TMA producer
       if (lane == 0) {
@@ -178,16 +188,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < wg_count(i); ++k) {
             const int w = wg_of(i, k);
             const int64_t j = wg_tile(i);
-            const int b = (int)(j & 1);
-            if (j >= 2 && !mbar_wait(&sp_done[w * 2 + b], (uint32_t)(((j >> 1) - 1) & 1)))
+            const int b = (int)(j % SB);
+            if (j >= SB && !mbar_wait(&sp_done[w * SB + b], (uint32_t)(((j / SB) - 1) & 1)))
               return false;
             tc_fence_after();
             const uint32_t qa = q_addr + (NH == 2 ? w * 128 * RB : 0);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
-              mma_ss(tmem + TM_S + w * 128 + b * 64, smem_desc(qa + 32 * kk, 16, 8 * RB, SW),
+              mma_ss(tmem + TM_S + (w * SB + b) * 64, smem_desc(qa + 32 * kk, 16, 8 * RB, SW),
                      smem_desc(k_addr + 32 * kk, 16, 8 * RB, SW), idS, kk > 0);
-            mma_commit(&s_full[w * 2 + b]);
+            mma_commit(&s_full[w * SB + b]);
           }
           return true;
         };
@@ -197,12 +207,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < wg_count(i); ++k) {
             const int w = wg_of(i, k);
             const int64_t j = wg_tile(i);
-            const int b = (int)(j & 1);
-            if (!mbar_wait(&sp_done[w * 2 + b], (uint32_t)((j >> 1) & 1))) return false;
+            const int b = (int)(j % SB);
+            if (!mbar_wait(&sp_done[w * SB + b], (uint32_t)((j / SB) & 1))) return false;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < kEncTile / 16; ++kk)
-              mma_ts(tmem + TM_O + w * 32, tmem + TM_P + w * 64 + b * 32 + 8 * kk,
+              mma_ts(tmem + TM_O + w * 32, tmem + TM_P + (w * SB + b) * 32 + 8 * kk,
                      smem_desc(v_addr + kk * 16 * RB, L::TILE, 8 * RB, SW), idPV,
                      (j > 0 || kk > 0) ? 1u : 0u);
             mma_commit(&pv_done[w]);
@@ -210,11 +220,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&kv_empty[s]);
           return true;
         };
-        if (ok && ntiles > 0) ok = issue_S(0);
-        if (ok && ntiles > 1) ok = issue_S(1);
-        if (NH == 1 && ok && ntiles > 2) ok = issue_S(2);
-        if (NH == 1 && ok && ntiles > 3) ok = issue_S(3);
-        const int ahead = (NH == 2) ? 2 : 4;   // S tiles in flight beyond the PV being issued
+        // S tiles in flight beyond the P.V being issued: every S buffer of
+        // every warpgroup.
+        const int ahead = (NH == 2) ? SB : 2 * SB;
+        for (int64_t i = 0; ok && i < ahead && i < ntiles; ++i) ok = issue_S(i);
         for (int64_t i = 0; ok && i < ntiles; ++i) {
           ok = issue_PV(i);
           if (ok && i + ahead < ntiles) ok = issue_S(i + ahead);
@@ -230,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------ softmax warpgroups
-    regs_acquire<kRegsSoftmax>();
+    regs_acquire<EncRegs<SB>::kSoftmax>();
     const int w = warp >> 2, q = warp & 3;
     const int r = q * 32 + lane;                     // TMEM lane = latent row in the half
     const uint32_t lb = (uint32_t)(q * 32) << 16;
@@ -240,11 +249,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int64_t j = 0; j < nW; ++j) {
       const int64_t i = (NH == 2) ? j : 2 * j + w;
-      const int b = (int)(j & 1);
+      const int b = (int)(j % SB);
       const int nvalid = (int)imin64(kEncTile, N - (tile0 + i) * kEncTile);
-      const uint32_t tS = tmem + lb + TM_S + w * 128 + b * 64;
-      const uint32_t tP = tmem + lb + TM_P + w * 64 + b * 32;
-      if (!mbar_wait(&s_full[w * 2 + b], (uint32_t)((j >> 1) & 1)) || *abort_flag) {
+      const uint32_t tS = tmem + lb + TM_S + (w * SB + b) * 64;
+      const uint32_t tP = tmem + lb + TM_P + (w * SB + b) * 32;
+      if (!mbar_wait(&s_full[w * SB + b], (uint32_t)((j / SB) & 1)) || *abort_flag) {
         ok = false;
         break;
       }
@@ -253,18 +262,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool full = (nvalid == kEncTile);   // warp-uniform: only a head's last tile is partial
       // pass 1: tile max of the raw logits (masked past the end of the head)
       float mf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      uint32_t a[2][32];
-      tmem_ld32(tS, a[0]);
 #pragma unroll
       for (int cc = 0; cc < kEncTile / 32; ++cc) {
-        tmem_wait_ld_dep(a[cc & 1]);
-        if (cc + 1 < kEncTile / 32) tmem_ld32(tS + 32 * (cc + 1), a[(cc + 1) & 1]);
+        uint32_t a[32];
+        tmem_ld32(tS + 32 * cc, a);
+        tmem_wait_ld_dep(a);
         if (full) {
-          max_fold32(a[cc & 1], mf);
+          max_fold32(a, mf);
         } else {
 #pragma unroll
           for (int t = 0; t < 32; ++t)
-            if (32 * cc + t < nvalid) mf[t & 3] = fmaxf(mf[t & 3], __uint_as_float(a[cc & 1][t]));
+            if (32 * cc + t < nvalid) mf[t & 3] = fmaxf(mf[t & 3], __uint_as_float(a[t]));
         }
       }
       const float mx = fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3]));
@@ -310,24 +318,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       // pass 2: P = 2^(c S - m_ref) as bf16 pairs, and its row sum
       const float neg = -mref;
       float sf[4] = {0.f, 0.f, 0.f, 0.f};
-      tmem_ld32(tS, a[0]);
 #pragma unroll
       for (int cc = 0; cc < kEncTile / 32; ++cc) {
-        tmem_wait_ld_dep(a[cc & 1]);
-        if (cc + 1 < kEncTile / 32) tmem_ld32(tS + 32 * (cc + 1), a[(cc + 1) & 1]);
+        uint32_t a[32];
+        tmem_ld32(tS + 32 * cc, a);
+        tmem_wait_ld_dep(a);
         if (!full) {   // tokens past the end of the head get weight 0
 #pragma unroll
           for (int t = 0; t < 32; ++t)
-            if (32 * cc + t >= nvalid) a[cc & 1][t] = __float_as_uint(-INFINITY);
+            if (32 * cc + t >= nvalid) a[t] = __float_as_uint(-INFINITY);
         }
         uint32_t pk[16];
-        exp_pack32(a[cc & 1], c, neg, pk, sf);
+        exp_pack32(a, c, neg, pk, sf);
         tmem_st16(tP + 16 * cc, pk);
       }
       tmem_wait_st();
       l += (sf[0] + sf[1]) + (sf[2] + sf[3]);
       tc_fence_before();
-      mbar_arrive(&sp_done[w * 2 + b]);
+      mbar_arrive(&sp_done[w * SB + b]);
     }
     float acc[D];
 #pragma unroll
@@ -370,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kWarpMma) tmem_dealloc(tmem, 512);
+  if (warp == kWarpMma) tmem_dealloc(tmem, TM_COLS);
 }
 
 // ============================================================== decode
@@ -668,6 +676,8 @@ cudaError_t make_map(CUtensorMap* m, const void* base, int D, int64_t rows, int6
   return cudaSuccess;
 }
 
+constexpr int kEncSB = 1;   // S buffers per softmax warpgroup (1: two CTAs per SM)
+
 template <int D, int M>
 cudaError_t tc_encode_t(const void* Q, int64_t qbs, const void* K, const void* V, const Dims& d,
                         float scale, const ChunkPlan& plan, float* pml, float* pacc,
@@ -678,13 +688,15 @@ cudaError_t tc_encode_t(const void* Q, int64_t qbs, const void* K, const void* V
   if ((e = make_map(&mq, Q, D, M, q_per_batch ? d.BH() : d.H, 128)) != cudaSuccess) return e;
   if ((e = make_map(&mk, K, D, d.N, d.BH(), kEncTile)) != cudaSuccess) return e;
   if ((e = make_map(&mv, V, D, d.N, d.BH(), kEncTile)) != cudaSuccess) return e;
-  const int smem = (EncLayout<D, M>::BYTES + 1024 > kMinSmemBytes) ? EncLayout<D, M>::BYTES + 1024
-                                                                   : kMinSmemBytes;
-  e = cudaFuncSetAttribute(tc_encode_kernel<D, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           smem);
+  // SB = 1: two CTAs per SM (their TMEM, 2 x 256 columns, fits exactly);
+  // SB = 2: the smem request keeps one CTA (and its 512 columns) per SM.
+  const int need = EncLayout<D, M>::BYTES + 1024;
+  const int smem = (kEncSB == 1 || need > kMinSmemBytes) ? need : kMinSmemBytes;
+  e = cudaFuncSetAttribute(tc_encode_kernel<D, M, kEncSB>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(plan.chunks, (unsigned)d.BH());
-  tc_encode_kernel<D, M><<<grid, kThreads, smem, st>>>(
+  tc_encode_kernel<D, M, kEncSB><<<grid, kThreads, smem, st>>>(
       mq, mk, mv, (int)d.H, d.N, q_per_batch, scale * kLog2e, plan.tiles_per_bh, plan.chunk_tiles,
       plan.slots_per_bh(), pml, pacc, err);
   return cudaPeekAtLastError();
