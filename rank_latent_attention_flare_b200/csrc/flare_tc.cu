@@ -41,10 +41,36 @@ constexpr int kWarpMma = 9;
 constexpr int kEncStages = 8;
 constexpr int kDecStages = 6;
 constexpr float kRescaleTau = 8.0f;   // log2 units: rescale only when the max grows by > 2^8
+constexpr float kRedoTau = 64.0f;     // log2 units: past 2^64 above m_ref a tile is recomputed
 constexpr int kMinSmemBytes = 120 * 1024;  // keeps one CTA (and its TMEM) per SM
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return (uint8_t*)(((uintptr_t)p + 1023) & ~(uintptr_t)1023);
+}
+
+// Multiplies this thread's row of a D-column fp32 TMEM accumulator by f.
+template <int D>
+__device__ __forceinline__ void scale_tmem_row(uint32_t taddr, float f) {
+  if (D == 32) {
+    uint32_t o[32];
+    tmem_ld32(taddr, o);
+    tmem_wait_ld_dep(o);
+    uint32_t lo[16], hi[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      lo[t] = __float_as_uint(__uint_as_float(o[t]) * f);
+      hi[t] = __float_as_uint(__uint_as_float(o[16 + t]) * f);
+    }
+    tmem_st16(taddr, lo);
+    tmem_st16(taddr + 16, hi);
+  } else {
+    uint32_t o[16];
+    tmem_ld16(taddr, o);
+    tmem_wait_ld();
+#pragma unroll
+    for (int t = 0; t < 16; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * f);
+    tmem_st16(taddr, o);
+  }
 }
 
 // ============================================================== encode
@@ -246,6 +272,7 @@ __global__ void __launch_bounds__(kThreads, (SB == 1) ? 2 : 1)
     const uint32_t tO = tmem + lb + TM_O + w * 32;
     const int64_t nW = (NH == 2) ? ntiles : (ntiles - w + 1) / 2;
     float mref = -INFINITY, l = 0.f;
+    float pend = 1.f;   // factor O still owes to a move of m_ref
     bool ok = true;
     for (int64_t j = 0; j < nW; ++j) {
       const int64_t i = (NH == 2) ? j : 2 * j + w;
@@ -253,87 +280,123 @@ __global__ void __launch_bounds__(kThreads, (SB == 1) ? 2 : 1)
       const int nvalid = (int)imin64(kEncTile, N - (tile0 + i) * kEncTile);
       const uint32_t tS = tmem + lb + TM_S + (w * SB + b) * 64;
       const uint32_t tP = tmem + lb + TM_P + (w * SB + b) * 32;
-      if (!mbar_wait(&s_full[w * SB + b], (uint32_t)((j / SB) & 1)) || *abort_flag) {
+      if (!warp_all(mbar_wait(&s_full[w * SB + b], (uint32_t)((j / SB) & 1)) && !*abort_flag)) {
         ok = false;
         break;
       }
       __syncwarp();
       tc_fence_after();
       const bool full = (nvalid == kEncTile);   // warp-uniform: only a head's last tile is partial
-      // pass 1: tile max of the raw logits (masked past the end of the head)
-      float mf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      // Before the first P store: the previous P.V must be done (P buffer
+      // free, O stable) and O must pay any rescale decided after that tile.
+      bool ready = (j == 0);
+      auto make_ready = [&]() -> bool {
+        if (ready) return true;
+        ready = true;
+        if (!warp_all(mbar_wait(&pv_done[w], (uint32_t)((j - 1) & 1)))) return false;
+        __syncwarp();
+        tc_fence_after();
+        if (warp_any(pend != 1.f)) scale_tmem_row<D>(tO, pend);   // rows without a rescale x 1
+        pend = 1.f;
+        return true;
+      };
+      // Optimistic single pass (every tile after a warpgroup's first): P is
+      // taken against the running reference m_ref while the tile max is
+      // folded in.  A max above m_ref + kRescaleTau moves m_ref after the
+      // tile (l now, O before the next P.V); a max above m_ref + kRedoTau,
+      // where P could overflow, makes the whole warp recompute the tile with
+      // the exact max.
+      bool exact = warp_any(mref == -INFINITY);
+      if (!exact) {
+        const float neg = -mref;
+        float mf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float sf[4] = {0.f, 0.f, 0.f, 0.f};
+        bool good = true;
 #pragma unroll
-      for (int cc = 0; cc < kEncTile / 32; ++cc) {
-        uint32_t a[32];
-        tmem_ld32(tS + 32 * cc, a);
-        tmem_wait_ld_dep(a);
-        if (full) {
+        for (int cc = 0; cc < kEncTile / 32; ++cc) {
+          uint32_t a[32];
+          tmem_ld32(tS + 32 * cc, a);
+          tmem_wait_ld_dep(a);
+          if (!full) {   // tokens past the end of the head get weight 0
+#pragma unroll
+            for (int t = 0; t < 32; ++t)
+              if (32 * cc + t >= nvalid) a[t] = __float_as_uint(-INFINITY);
+          }
           max_fold32(a, mf);
-        } else {
-#pragma unroll
-          for (int t = 0; t < 32; ++t)
-            if (32 * cc + t < nvalid) mf[t & 3] = fmaxf(mf[t & 3], __uint_as_float(a[t]));
+          uint32_t pk[16];
+          exp_pack32(a, c, neg, pk, sf);
+          if (cc == 0 && !make_ready()) {   // overlap the P.V wait with chunk 0's exponentials
+            good = false;
+            break;
+          }
+          tmem_st16(tP + 16 * cc, pk);
         }
-      }
-      const float mx = fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3]));
-      const float mx2 = mx * c;
-      float factor = 1.f;
-      bool rescale = false;
-      if (mx2 > mref + kRescaleTau) {
-        rescale = (mref != -INFINITY);
-        factor = ex2(mref - mx2);
-        mref = mx2;
-      }
-      if (j > 0) {   // previous P.V done: O is stable and this P buffer is free
-        if (!mbar_wait(&pv_done[w], (uint32_t)((j - 1) & 1))) {
+        if (!good) {
           ok = false;
           break;
         }
-        __syncwarp();
-        tc_fence_after();
-      }
-      if (rescale) {
-        l *= factor;
-        if (D == 32) {
-          uint32_t o[32];
-          tmem_ld32(tO, o);
-          tmem_wait_ld();
-          uint32_t lo[16], hi[16];
-#pragma unroll
-          for (int t = 0; t < 16; ++t) {
-            lo[t] = __float_as_uint(__uint_as_float(o[t]) * factor);
-            hi[t] = __float_as_uint(__uint_as_float(o[16 + t]) * factor);
-          }
-          tmem_st16(tO, lo);
-          tmem_st16(tO + 16, hi);
+        const float mx2 = fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3])) * c;
+        if (warp_any(mx2 > mref + kRedoTau)) {
+          exact = true;
         } else {
-          uint32_t o[16];
-          tmem_ld16(tO, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int t = 0; t < 16; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * factor);
-          tmem_st16(tO, o);
+          const float sum = (sf[0] + sf[1]) + (sf[2] + sf[3]);
+          if (mx2 > mref + kRescaleTau) {
+            pend = ex2(mref - mx2);
+            l = (l + sum) * pend;
+            mref = mx2;
+          } else {
+            l += sum;
+          }
         }
       }
-      // pass 2: P = 2^(c S - m_ref) as bf16 pairs, and its row sum
-      const float neg = -mref;
-      float sf[4] = {0.f, 0.f, 0.f, 0.f};
+      if (exact) {
+        // pass 1: exact tile max of the raw logits (masked past the end of the head)
+        float mf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int cc = 0; cc < kEncTile / 32; ++cc) {
-        uint32_t a[32];
-        tmem_ld32(tS + 32 * cc, a);
-        tmem_wait_ld_dep(a);
-        if (!full) {   // tokens past the end of the head get weight 0
+        for (int cc = 0; cc < kEncTile / 32; ++cc) {
+          uint32_t a[32];
+          tmem_ld32(tS + 32 * cc, a);
+          tmem_wait_ld_dep(a);
+          if (full) {
+            max_fold32(a, mf);
+          } else {
 #pragma unroll
-          for (int t = 0; t < 32; ++t)
-            if (32 * cc + t >= nvalid) a[t] = __float_as_uint(-INFINITY);
+            for (int t = 0; t < 32; ++t)
+              if (32 * cc + t < nvalid) mf[t & 3] = fmaxf(mf[t & 3], __uint_as_float(a[t]));
+          }
         }
-        uint32_t pk[16];
-        exp_pack32(a, c, neg, pk, sf);
-        tmem_st16(tP + 16 * cc, pk);
+        const float mx2 = fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3])) * c;
+        if (!make_ready()) {
+          ok = false;
+          break;
+        }
+        float f = 1.f;   // rescale of this row's earlier tiles (1 when the max did not move)
+        if (mx2 > mref) {
+          if (mref != -INFINITY) f = ex2(mref - mx2);
+          mref = mx2;
+        }
+        l *= f;
+        if (warp_any(f != 1.f)) scale_tmem_row<D>(tO, f);
+        // pass 2: P = 2^(c S - m_ref) as bf16 pairs, and its row sum
+        const float neg = -mref;
+        float sf[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int cc = 0; cc < kEncTile / 32; ++cc) {
+          uint32_t a[32];
+          tmem_ld32(tS + 32 * cc, a);
+          tmem_wait_ld_dep(a);
+          if (!full) {
+#pragma unroll
+            for (int t = 0; t < 32; ++t)
+              if (32 * cc + t >= nvalid) a[t] = __float_as_uint(-INFINITY);
+          }
+          uint32_t pk[16];
+          exp_pack32(a, c, neg, pk, sf);
+          tmem_st16(tP + 16 * cc, pk);
+        }
+        l += (sf[0] + sf[1]) + (sf[2] + sf[3]);
       }
       tmem_wait_st();
-      l += (sf[0] + sf[1]) + (sf[2] + sf[3]);
       tc_fence_before();
       mbar_arrive(&sp_done[w * SB + b]);
     }
@@ -341,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, (SB == 1) ? 2 : 1)
 #pragma unroll
     for (int d = 0; d < D; ++d) acc[d] = 0.f;
     if (ok && nW > 0) {
-      ok = mbar_wait(&pv_done[w], (uint32_t)((nW - 1) & 1));
+      ok = warp_all(mbar_wait(&pv_done[w], (uint32_t)((nW - 1) & 1)));
       __syncwarp();
       tc_fence_after();
       if (ok) {
@@ -350,13 +413,13 @@ __global__ void __launch_bounds__(kThreads, (SB == 1) ? 2 : 1)
           tmem_ld32(tO, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int d = 0; d < D; ++d) acc[d] = __uint_as_float(o[d]);
+          for (int d = 0; d < D; ++d) acc[d] = __uint_as_float(o[d]) * pend;
         } else {
           uint32_t o[16];
           tmem_ld16(tO, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int d = 0; d < D; ++d) acc[d] = __uint_as_float(o[d & 15]);
+          for (int d = 0; d < D; ++d) acc[d] = __uint_as_float(o[d & 15]) * pend;
         }
       }
     }
@@ -546,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int64_t j = 0; j < nW; ++j) {
       const int64_t i = 2 * j + w;
       const int64_t tok = (tile0 + i) * kTile + r;
-      if (!mbar_wait(&s_full[w], (uint32_t)(j & 1)) || *abort_flag) {
+      if (!warp_all(mbar_wait(&s_full[w], (uint32_t)(j & 1)) && !*abort_flag)) {
         ok = false;
         break;
       }
@@ -588,7 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[w]);
-      if (!mbar_wait(&y_full[w], (uint32_t)(j & 1))) {
+      if (!warp_all(mbar_wait(&y_full[w], (uint32_t)(j & 1)))) {
         ok = false;
         break;
       }

@@ -132,3 +132,36 @@ def test_gpu_rejects_invalid_arguments_without_side_effects():
     assert e.value.status == 3
     torch.cuda.synchronize()
     assert torch.count_nonzero(Y) == 0
+
+
+@pytest.mark.parametrize("M", [128, 256])
+@pytest.mark.parametrize("regime", ["spiky", "growing"])
+def test_encode_running_max_over_many_tiles(M, regime):
+    # One head of 262,144 tokens: every encode CTA walks many 64-token tiles,
+    # so the running-max machinery is exercised.  "spiky": scale x100 makes
+    # tile maxima jump by far more than 2^64 (tiles recomputed with the exact
+    # max); "growing": keys grow steadily along the sequence, so the running
+    # max keeps rising by more than 2^8 (deferred rescales).
+    B, H, N, D = 1, 1, 262144, 32
+    x = make_inputs(B, H, N, M, D, dtype=torch.bfloat16, seed=21 + M)
+    if regime == "spiky":
+        s = 100.0 / math.sqrt(D)
+    else:
+        s = 1.0 / math.sqrt(D)
+        ramp = torch.linspace(0.25, 4.0, N).view(1, 1, N, 1)
+        x["K"] = (x["K"].float() * ramp).to(torch.bfloat16)
+    g = {k: v.to(DEV) for k, v in x.items()}
+    ws = fl.alloc_workspace(fl.FLARE_OP_FWD, B, H, N, M, D, torch.bfloat16, DEV)
+    Y, Z, lse = fl.flare_fwd(g["Q"], g["K"], g["V"], s, save=True, workspace=ws)
+    assert fl.device_status(ws) == 0
+    assert torch.isfinite(Z).all() and torch.isfinite(Y.float()).all()
+    Zo, lo = oracle.encode(x["Q"], x["K"], x["V"], s)
+    rows = np.unique(np.concatenate([np.arange(64), np.arange(N - 64, N),
+                                     np.random.default_rng(0).integers(0, N, 2048)]))
+    Yo = oracle.decode_rows(x["Q"], x["K"], Zo, s, rows)
+    if regime == "spiky":   # peaked softmaxes amplify bf16 logit rounding
+        assert rel_fro(Z, Zo) <= 5e-2 and rel_fro(Y.float().cpu().reshape(-1, D)[rows], Yo) <= 5e-2
+    else:
+        assert_close(Z, Zo, torch.bfloat16, "Z")
+        assert_close(lse, lo, torch.bfloat16, "lse")
+        assert_close(Y.float().cpu().reshape(-1, D)[rows], Yo, torch.bfloat16, "Y")
