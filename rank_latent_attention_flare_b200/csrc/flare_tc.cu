@@ -42,6 +42,9 @@ constexpr int kEncStages = 8;
 constexpr int kDecStages = 6;
 constexpr float kRescaleTau = 8.0f;   // log2 units: rescale only when the max grows by > 2^8
 constexpr float kRedoTau = 64.0f;     // log2 units: past 2^64 above m_ref a tile is recomputed
+// Every kPolyEvery-th pair of exponentials is computed on the FMA pipe
+// (exp2_fma) instead of the MUFU, which is the unit that bounds both kernels.
+constexpr int kPolyEvery = 0;
 constexpr int kMinSmemBytes = 120 * 1024;  // keeps one CTA (and its TMEM) per SM
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -94,7 +97,7 @@ struct EncLayout {
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = M * RB;
   static constexpr int BAR_OFF = KV_OFF + kEncStages * 2 * TILE;
-  static constexpr int NBARS = 2 * kEncStages + 1 + 4 + 4 + 2 + 1;   // sized for SB <= 2
+  static constexpr int NBARS = 2 * kEncStages + 1 + 4 + 4 + 2 + 2;   // sized for SB <= 2
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
 };
@@ -144,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, (SB == 1) ? 2 : 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kEncStages; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_empty[s], NH == 2 ? 2 : 1);   // one release per warpgroup reading the tile
     }
     mbar_init(q_full, 1);
     for (int k = 0; k < 4; ++k) {
@@ -153,7 +156,8 @@ __global__ void __launch_bounds__(kThreads, (SB == 1) ? 2 : 1)
     }
     mbar_init(&pv_done[0], 1);
     mbar_init(&pv_done[1], 1);
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -197,70 +201,67 @@ __global__ void __launch_bounds__(kThreads, (SB == 1) ? 2 : 1)
           mbar_wait(&kv_full[i % kEncStages], (uint32_t)((i / kEncStages) & 1));
         mbar_wait(q_full, 0);
       }
-    } else if (warp == kWarpMma) {
-      // ---------------------------------------------------- MMA issuer
+    } else if (warp == kWarpMma || warp == kWarpMma + 1) {
+      // ------------------------------------------- MMA issuers, one per warpgroup
+      // Warp 9 serves softmax warpgroup 0 and warp 10 warpgroup 1, so neither
+      // issue stream waits for the other warpgroup.  For warpgroup w's j-th
+      // tile: S into buffer j % SB once that buffer is free (the softmax has
+      // finished tile j - SB) and the K tile has landed; P.V once the softmax
+      // has finished tile j, after the S that reuses its buffer.
       if (lane == 0) {
+        const int w = warp - kWarpMma;
         constexpr uint32_t idS = idesc_bf16_f32(128, kEncTile, 0, 0);
         constexpr uint32_t idPV = idesc_bf16_f32(128, D, 0, 1);
-        const uint32_t q_addr = smem_u32(Qs);
+        const int nw = (NH == 2) ? (int)ntiles : (int)((ntiles - w + 1) / 2);
+        const int first = (NH == 2) ? 0 : w;
+        constexpr int stride = (NH == 2) ? 1 : 2;
+        // descriptors built once; per stage / k-step only the address field moves
+        const uint32_t kv0 = smem_u32(smem + L::KV_OFF);
+        const uint64_t dQ = smem_desc(smem_u32(Qs) + (NH == 2 ? w * 128 * RB : 0), 16, 8 * RB, SW);
+        const uint64_t dK = smem_desc(kv0, 16, 8 * RB, SW);
+        const uint64_t dV = smem_desc(kv0 + L::TILE, L::TILE, 8 * RB, SW);
+        const uint32_t tS0 = tmem + TM_S + (w * SB) * 64;
+        const uint32_t tP0 = tmem + TM_P + (w * SB) * 32;
+        const uint32_t tO = tmem + TM_O + w * 32;
         bool ok = mbar_wait(q_full, 0);
-        auto wg_count = [&](int64_t) { return NH == 2 ? 2 : 1; };
-        auto wg_of = [&](int64_t i, int k) { return NH == 2 ? k : (int)(i & 1); };
-        auto wg_tile = [&](int64_t i) { return NH == 2 ? i : (i >> 1); };
-        auto issue_S = [&](int64_t i) -> bool {
-          const int s = (int)(i % kEncStages);
+        auto issue_S = [&](int j) -> bool {
+          const int i = first + stride * j;
+          const int s = i % kEncStages;
           if (!mbar_wait(&kv_full[s], (uint32_t)((i / kEncStages) & 1))) return false;
-          const uint32_t k_addr = smem_u32(smem + L::KV_OFF + s * 2 * L::TILE);
-          for (int k = 0; k < wg_count(i); ++k) {
-            const int w = wg_of(i, k);
-            const int64_t j = wg_tile(i);
-            const int b = (int)(j % SB);
-            if (j >= SB && !mbar_wait(&sp_done[w * SB + b], (uint32_t)(((j / SB) - 1) & 1)))
-              return false;
-            tc_fence_after();
-            const uint32_t qa = q_addr + (NH == 2 ? w * 128 * RB : 0);
+          tc_fence_after();
+          const uint32_t koff = (uint32_t)(s * 2 * L::TILE) >> 4;
+          const int b = j % SB;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-              mma_ss(tmem + TM_S + (w * SB + b) * 64, smem_desc(qa + 32 * kk, 16, 8 * RB, SW),
-                     smem_desc(k_addr + 32 * kk, 16, 8 * RB, SW), idS, kk > 0);
-            mma_commit(&s_full[w * SB + b]);
-          }
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tS0 + b * 64, dQ + 2 * kk, dK + koff + 2 * kk, idS, kk > 0);
+          mma_commit(&s_full[w * SB + b]);
           return true;
         };
-        auto issue_PV = [&](int64_t i) -> bool {
-          const int s = (int)(i % kEncStages);
-          const uint32_t v_addr = smem_u32(smem + L::KV_OFF + s * 2 * L::TILE + L::TILE);
-          for (int k = 0; k < wg_count(i); ++k) {
-            const int w = wg_of(i, k);
-            const int64_t j = wg_tile(i);
-            const int b = (int)(j % SB);
-            if (!mbar_wait(&sp_done[w * SB + b], (uint32_t)((j / SB) & 1))) return false;
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < kEncTile / 16; ++kk)
-              mma_ts(tmem + TM_O + w * 32, tmem + TM_P + (w * SB + b) * 32 + 8 * kk,
-                     smem_desc(v_addr + kk * 16 * RB, L::TILE, 8 * RB, SW), idPV,
-                     (j > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(&pv_done[w]);
+        for (int j = 0; ok && j < SB && j < nw; ++j) ok = issue_S(j);
+        for (int j = 0; ok && j < nw; ++j) {
+          const int b = j % SB;
+          if (!mbar_wait(&sp_done[w * SB + b], (uint32_t)((j / SB) & 1))) {
+            ok = false;
+            break;
           }
-          mma_commit(&kv_empty[s]);
-          return true;
-        };
-        // S tiles in flight beyond the P.V being issued: every S buffer of
-        // every warpgroup.
-        const int ahead = (NH == 2) ? SB : 2 * SB;
-        for (int64_t i = 0; ok && i < ahead && i < ntiles; ++i) ok = issue_S(i);
-        for (int64_t i = 0; ok && i < ntiles; ++i) {
-          ok = issue_PV(i);
-          if (ok && i + ahead < ntiles) ok = issue_S(i + ahead);
+          tc_fence_after();
+          if (j + SB < nw && !(ok = issue_S(j + SB))) break;
+          const int i = first + stride * j;
+          const uint32_t voff = (uint32_t)((i % kEncStages) * 2 * L::TILE) >> 4;
+#pragma unroll
+          for (int kk = 0; kk < kEncTile / 16; ++kk)
+            mma_ts(tO, tP0 + b * 32 + 8 * kk, dV + voff + ((uint32_t)(kk * 16 * RB) >> 4), idPV,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&pv_done[w]);
+          mma_commit(&kv_empty[i % kEncStages]);
           if (*abort_flag) ok = false;
         }
         if (!ok) {
           record_error(err, kErrEncMmaWait);
           *abort_flag = 1;
         }
-        mma_commit(drain);
-        mbar_wait(drain, 0);
+        mma_commit(drain + w);
+        mbar_wait(drain + w, 0);
       }
     }
   } else {
@@ -324,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, (SB == 1) ? 2 : 1)
           }
           max_fold32(a, mf);
           uint32_t pk[16];
-          exp_pack32(a, c, neg, pk, sf);
+          exp_pack32<kPolyEvery>(a, c, neg, pk, sf);
           if (cc == 0 && !make_ready()) {   // overlap the P.V wait with chunk 0's exponentials
             good = false;
             break;
@@ -391,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, (SB == 1) ? 2 : 1)
               if (32 * cc + t >= nvalid) a[t] = __float_as_uint(-INFINITY);
           }
           uint32_t pk[16];
-          exp_pack32(a, c, neg, pk, sf);
+          exp_pack32<kPolyEvery>(a, c, neg, pk, sf);
           tmem_st16(tP + 16 * cc, pk);
         }
         l += (sf[0] + sf[1]) + (sf[2] + sf[3]);
@@ -645,7 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld_dep(a[k & 1]);
         if (k + 1 < NC) tmem_ld32(tR + chunk_col(k + 1), a[(k + 1) & 1]);
         uint32_t pk[16];
-        exp_pack32(a[k & 1], c, neg, pk, sf);
+        exp_pack32<kPolyEvery>(a[k & 1], c, neg, pk, sf);
         tmem_st16(tR + p_col(k), pk);
       }
       tmem_wait_st();

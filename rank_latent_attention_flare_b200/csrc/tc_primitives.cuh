@@ -58,6 +58,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking: true once the phase with the given parity has completed.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete; false on timeout.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -289,8 +302,30 @@ __device__ __forceinline__ void max_fold32(const uint32_t (&a)[32], float (&m)[4
   }
 }
 
+// 2^x on the FMA pipe, leaving the MUFU free for other exponentials.
+// Single-split range reduction x = j + f with j = round(x) (the 1.5 * 2^23
+// add puts round(x) in the low mantissa bits), f in [-1/2, 1/2]; 2^f by a
+// degree-3 polynomial fitted by Remez exchange for minimum relative error
+// (7.5e-5, see fit_exp2_poly.py); j is added to the result's exponent field.
+// Exact enough for values that are rounded to bf16 next.  Valid for
+// x <= 126; x below -125 is clamped (result 2^-125 instead of smaller).
+__device__ __forceinline__ float exp2_fma(float x) {
+  constexpr float kE0 = 0.9999280571937561f, kE1 = 0.6932609677314758f;
+  constexpr float kE2 = 0.2426111251115799f, kE3 = 0.0551716685295105f;
+  constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
+  x = fmaxf(x, -125.0f);
+  const float t = x + kRound;
+  const float f = x - (t - kRound);
+  float p = fmaf(kE3, f, kE2);
+  p = fmaf(p, f, kE1);
+  p = fmaf(p, f, kE0);
+  return __uint_as_float((__float_as_uint(t) << 23) + __float_as_uint(p));
+}
+
 // p = 2^(a*c + neg) for 32 logits: packed into 16 bf16 pairs, sums folded
-// into four independent accumulators.
+// into four independent accumulators.  With POLY_EVERY = k > 0, every k-th
+// pair is computed on the FMA pipe (exp2_fma) instead of the MUFU.
+template <int POLY_EVERY = 0>
 __device__ __forceinline__ void exp_pack32(const uint32_t (&a)[32], float c, float neg,
                                            uint32_t (&pk)[16], float (&s)[4]);
 
@@ -299,12 +334,16 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+template <int POLY_EVERY>
 __device__ __forceinline__ void exp_pack32(const uint32_t (&a)[32], float c, float neg,
                                            uint32_t (&pk)[16], float (&s)[4]) {
 #pragma unroll
   for (int t = 0; t < 16; ++t) {
-    const float p0 = ex2(fmaf(__uint_as_float(a[2 * t]), c, neg));
-    const float p1 = ex2(fmaf(__uint_as_float(a[2 * t + 1]), c, neg));
+    const float x0 = fmaf(__uint_as_float(a[2 * t]), c, neg);
+    const float x1 = fmaf(__uint_as_float(a[2 * t + 1]), c, neg);
+    const bool poly = POLY_EVERY > 0 && (t % (POLY_EVERY > 0 ? POLY_EVERY : 1)) == POLY_EVERY - 1;
+    const float p0 = poly ? exp2_fma(x0) : ex2(x0);
+    const float p1 = poly ? exp2_fma(x1) : ex2(x1);
     s[t & 3] += p0 + p1;
     pk[t] = pack_bf16(p0, p1);
   }
