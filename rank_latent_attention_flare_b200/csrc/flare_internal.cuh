@@ -88,7 +88,7 @@ constexpr int kSimtEncTile = 64;
 constexpr int kSimtEncThreads = 256;
 constexpr int kSimtDecThreads = 128;
 constexpr int kTcTile = 128;     // decode tile (tokens)
-constexpr int kTcEncTile = 64;   // tensor-core encode tile (tokens)
+constexpr int kTcEncTile = 48;   // tensor-core encode tile (tokens)
 constexpr int kBwdTile = 256;
 
 inline ChunkPlan encode_plan(int64_t BH, int64_t N, int64_t M, int64_t D, flare_dtype_t dt,

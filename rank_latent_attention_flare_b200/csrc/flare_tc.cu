@@ -78,17 +78,19 @@ __device__ __forceinline__ void scale_tmem_row(uint32_t taddr, float f) {
 
 // ============================================================== encode
 //
-// Tiles of kEncTile = 64 tokens.  Each softmax warpgroup w has SB S buffers
-// of 64 TMEM columns, SB P buffers of 32 columns (bf16 pairs) and an O
-// accumulator of 32 columns: S[w][b] at (w*SB + b)*64, P[w][b] at
-// 128*SB + (w*SB + b)*32, O[w] at 192*SB + 32w.  SB = 1 needs 256 columns,
-// so two CTAs share an SM and their four softmax warpgroups hide each
-// other's latencies; SB = 2 (448 columns, one CTA per SM) lets the MMA fill
-// the next S buffer while the softmax works on this one.  With M = 256
-// warpgroup w owns latent rows [128w, 128w+128) of every tile; with M = 128
-// the warpgroups take alternate tiles and each keeps its own running record.
+// Tiles of kEncTile = 48 tokens; two CTAs share an SM (256 TMEM columns and
+// an 80-register launch each), so four softmax warpgroups per SM hide each
+// other's latencies.  Softmax warpgroup w owns TMEM columns
+// [128w, 128w + 128): two 48-column S buffers at 128w + 48b (b = 0, 1), whose
+// first 24 columns receive the tile's P (bf16 pairs) once S has been read,
+// and the O accumulator at 128w + 96.  While the softmax works on one
+// buffer, the MMA fills the other with the next tile's logits.  With M = 256
+// warpgroup w owns latent rows [128w, 128w + 128) of every tile; with M = 128
+// the warpgroups take alternate tiles, each with its own running record.
 
-constexpr int kEncTile = 64;
+constexpr int kEncTile = 48;
+constexpr int kEncP = kEncTile / 2;   // P columns (bf16 pairs) per tile
+constexpr int kEncRegsSoftmax = 88, kEncRegsProducer = 56;   // 256 x 88 + 128 x 56 <= 384 x 80
 
 template <int D, int M>
 struct EncLayout {
@@ -97,19 +99,13 @@ struct EncLayout {
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = M * RB;
   static constexpr int BAR_OFF = KV_OFF + kEncStages * 2 * TILE;
-  static constexpr int NBARS = 2 * kEncStages + 1 + 4 + 4 + 2 + 2;   // sized for SB <= 2
+  static constexpr int NBARS = 2 * kEncStages + 1 + 4 + 4 + 4 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
 };
 
-template <int SB>
-struct EncRegs {   // setmaxnreg split; launch cap is 168 (SB = 2) or 80 (SB = 1)
-  static constexpr int kSoftmax = (SB == 2) ? kRegsSoftmax : 88;
-  static constexpr int kProducer = (SB == 2) ? kRegsProducer : 56;
-};
-
-template <int D, int M, int SB>
-__global__ void __launch_bounds__(kThreads, (SB == 1) ? 2 : 1)
+template <int D, int M>
+__global__ void __launch_bounds__(kThreads, 2)
     tc_encode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, int H, int64_t N, int q_per_batch,
                      float c, int64_t tiles_per_bh, int64_t chunk_tiles, int slots_per_bh,
@@ -120,8 +116,8 @@ __global__ void __launch_bounds__(kThreads, (SB == 1) ? 2 : 1)
   constexpr int SUB = (NH == 1) ? 2 : 1;
   constexpr int RB = L::RB;
   constexpr uint32_t SW = umma_swizzle_code(RB);
-  constexpr uint32_t TM_S = 0, TM_P = 128 * SB, TM_O = 192 * SB;   // TMEM column bases
-  constexpr uint32_t TM_COLS = (SB == 1) ? 256 : 512;
+  constexpr uint32_t TM_COLS = 256;
+  constexpr int stride = (NH == 2) ? 1 : 2;   // tile step of one warpgroup
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -130,10 +126,10 @@ __global__ void __launch_bounds__(kThreads, (SB == 1) ? 2 : 1)
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = bars + kEncStages;
   uint64_t* q_full = bars + 2 * kEncStages;
-  uint64_t* s_full = q_full + 1;      // [w*SB + b]
-  uint64_t* sp_done = s_full + 4;     // [w*SB + b]: S read and P written
-  uint64_t* pv_done = sp_done + 4;    // [w]
-  uint64_t* drain = pv_done + 2;
+  uint64_t* s_full = q_full + 1;      // [2w + b]: S written by the MMA
+  uint64_t* sp_done = s_full + 4;     // [2w + b]: S read and P written by the softmax
+  uint64_t* pv_done = sp_done + 4;    // [2w + b]: P.V of a tile from buffer b complete
+  uint64_t* drain = pv_done + 4;      // [w]
   uint32_t* tmem_slot = (uint32_t*)(smem + L::MISC_OFF);
   volatile int* abort_flag = (volatile int*)(smem + L::MISC_OFF + 4);
 
@@ -153,11 +149,9 @@ __global__ void __launch_bounds__(kThreads, (SB == 1) ? 2 : 1)
     for (int k = 0; k < 4; ++k) {
       mbar_init(&s_full[k], 1);
       mbar_init(&sp_done[k], 128);
+      mbar_init(&pv_done[k], 1);
     }
-    mbar_init(&pv_done[0], 1);
-    mbar_init(&pv_done[1], 1);
-    mbar_init(&drain[0], 1);
-    mbar_init(&drain[1], 1);
+    for (int k = 0; k < 2; ++k) mbar_init(&drain[k], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -168,7 +162,7 @@ __global__ void __launch_bounds__(kThreads, (SB == 1) ? 2 : 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= 8) {
-    regs_release<EncRegs<SB>::kProducer>();
+    regs_release<kEncRegsProducer>();
     if (warp == kWarpTma) {
       // ---------------------------------------------------- TMA producer
       if (lane == 0) {
@@ -179,9 +173,9 @@ __global__ void __launch_bounds__(kThreads, (SB == 1) ? 2 : 1)
         const int32_t qz = (int32_t)(q_per_batch ? bh : h);
         for (int half = 0; half < NH; ++half)
           tma_load_3d(Qs + half * 128 * RB, &tmQ, q_full, 0, half * 128, qz);
-        int64_t issued = 0;
-        for (int64_t i = 0; i < ntiles; ++i) {
-          const int s = (int)(i % kEncStages);
+        int issued = 0;
+        for (int i = 0; i < (int)ntiles; ++i) {
+          const int s = i % kEncStages;
           const uint32_t ph = (uint32_t)((i / kEncStages) & 1);
           if (i >= kEncStages && !mbar_wait(&kv_empty[s], ph ^ 1)) {
             record_error(err, kErrEncTmaWait);
@@ -197,32 +191,28 @@ __global__ void __launch_bounds__(kThreads, (SB == 1) ? 2 : 1)
           issued = i + 1;
         }
         // let every load still in flight land before the CTA can exit
-        for (int64_t i = (issued > kEncStages ? issued - kEncStages : 0); i < issued; ++i)
+        for (int i = (issued > kEncStages ? issued - kEncStages : 0); i < issued; ++i)
           mbar_wait(&kv_full[i % kEncStages], (uint32_t)((i / kEncStages) & 1));
         mbar_wait(q_full, 0);
       }
     } else if (warp == kWarpMma || warp == kWarpMma + 1) {
-      // ------------------------------------------- MMA issuers, one per warpgroup
-      // Warp 9 serves softmax warpgroup 0 and warp 10 warpgroup 1, so neither
-      // issue stream waits for the other warpgroup.  For warpgroup w's j-th
-      // tile: S into buffer j % SB once that buffer is free (the softmax has
-      // finished tile j - SB) and the K tile has landed; P.V once the softmax
-      // has finished tile j, after the S that reuses its buffer.
+      // -------------------------------------- MMA issuers, one per warpgroup
+      // Warp 9 serves softmax warpgroup 0 and warp 10 warpgroup 1.  For the
+      // warpgroup's j-th tile (buffer b = j % 2): P.V once the softmax has
+      // finished it; then, once that P.V has completed (it reads P from
+      // buffer b), the S of tile j + 2 into the same buffer.
       if (lane == 0) {
         const int w = warp - kWarpMma;
         constexpr uint32_t idS = idesc_bf16_f32(128, kEncTile, 0, 0);
         constexpr uint32_t idPV = idesc_bf16_f32(128, D, 0, 1);
         const int nw = (NH == 2) ? (int)ntiles : (int)((ntiles - w + 1) / 2);
         const int first = (NH == 2) ? 0 : w;
-        constexpr int stride = (NH == 2) ? 1 : 2;
         // descriptors built once; per stage / k-step only the address field moves
         const uint32_t kv0 = smem_u32(smem + L::KV_OFF);
         const uint64_t dQ = smem_desc(smem_u32(Qs) + (NH == 2 ? w * 128 * RB : 0), 16, 8 * RB, SW);
         const uint64_t dK = smem_desc(kv0, 16, 8 * RB, SW);
         const uint64_t dV = smem_desc(kv0 + L::TILE, L::TILE, 8 * RB, SW);
-        const uint32_t tS0 = tmem + TM_S + (w * SB) * 64;
-        const uint32_t tP0 = tmem + TM_P + (w * SB) * 32;
-        const uint32_t tO = tmem + TM_O + w * 32;
+        const uint32_t tW = tmem + 128 * w;
         bool ok = mbar_wait(q_full, 0);
         auto issue_S = [&](int j) -> bool {
           const int i = first + stride * j;
@@ -230,30 +220,38 @@ __global__ void __launch_bounds__(kThreads, (SB == 1) ? 2 : 1)
           if (!mbar_wait(&kv_full[s], (uint32_t)((i / kEncStages) & 1))) return false;
           tc_fence_after();
           const uint32_t koff = (uint32_t)(s * 2 * L::TILE) >> 4;
-          const int b = j % SB;
+          const int b = j & 1;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tS0 + b * 64, dQ + 2 * kk, dK + koff + 2 * kk, idS, kk > 0);
-          mma_commit(&s_full[w * SB + b]);
+            mma_ss(tW + 48 * b, dQ + 2 * kk, dK + koff + 2 * kk, idS, kk > 0);
+          mma_commit(&s_full[2 * w + b]);
           return true;
         };
-        for (int j = 0; ok && j < SB && j < nw; ++j) ok = issue_S(j);
+        for (int j = 0; ok && j < 2 && j < nw; ++j) ok = issue_S(j);
         for (int j = 0; ok && j < nw; ++j) {
-          const int b = j % SB;
-          if (!mbar_wait(&sp_done[w * SB + b], (uint32_t)((j / SB) & 1))) {
+          const int b = j & 1;
+          if (!mbar_wait(&sp_done[2 * w + b], (uint32_t)((j >> 1) & 1))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          if (j + SB < nw && !(ok = issue_S(j + SB))) break;
           const int i = first + stride * j;
           const uint32_t voff = (uint32_t)((i % kEncStages) * 2 * L::TILE) >> 4;
 #pragma unroll
           for (int kk = 0; kk < kEncTile / 16; ++kk)
-            mma_ts(tO, tP0 + b * 32 + 8 * kk, dV + voff + ((uint32_t)(kk * 16 * RB) >> 4), idPV,
-                   (j > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&pv_done[w]);
+            mma_ts(tW + 96, tW + 48 * b + 8 * kk, dV + voff + ((uint32_t)(kk * 16 * RB) >> 4),
+                   idPV, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&pv_done[2 * w + b]);
           mma_commit(&kv_empty[i % kEncStages]);
+          if (j + 2 < nw) {
+            // buffer b still holds the P this P.V reads: wait for it to finish
+            if (!mbar_wait(&pv_done[2 * w + b], (uint32_t)((j >> 1) & 1))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            if (!(ok = issue_S(j + 2))) break;
+          }
           if (*abort_flag) ok = false;
         }
         if (!ok) {
@@ -266,80 +264,94 @@ __global__ void __launch_bounds__(kThreads, (SB == 1) ? 2 : 1)
     }
   } else {
     // ------------------------------------------------------ softmax warpgroups
-    regs_acquire<EncRegs<SB>::kSoftmax>();
+    regs_acquire<kEncRegsSoftmax>();
     const int w = warp >> 2, q = warp & 3;
     const int r = q * 32 + lane;                     // TMEM lane = latent row in the half
     const uint32_t lb = (uint32_t)(q * 32) << 16;
-    const uint32_t tO = tmem + lb + TM_O + w * 32;
-    const int64_t nW = (NH == 2) ? ntiles : (ntiles - w + 1) / 2;
+    const uint32_t tW = tmem + lb + 128 * w;
+    const uint32_t tO = tW + 96;
+    const int nW = (NH == 2) ? (int)ntiles : (int)((ntiles - w + 1) / 2);
+    const int first = (NH == 2) ? 0 : w;
     float mref = -INFINITY, l = 0.f;
     float pend = 1.f;   // factor O still owes to a move of m_ref
     bool ok = true;
-    for (int64_t j = 0; j < nW; ++j) {
-      const int64_t i = (NH == 2) ? j : 2 * j + w;
-      const int b = (int)(j % SB);
+    // P.V of this warpgroup's tile jj (and, by issue order, of every earlier
+    // one) has completed.  Each S buffer has its own barrier: with one
+    // barrier per warpgroup a waiter two phases behind would read the
+    // wrong parity as complete.
+    auto pv_wait = [&](int jj) -> bool {
+      return mbar_wait(&pv_done[2 * w + (jj & 1)], (uint32_t)((jj >> 1) & 1));
+    };
+    // Waits for the previous tile's P.V (O stable) and multiplies O by g.
+    auto scale_O = [&](int j, float g) -> bool {
+      if (!warp_any(g != 1.f)) return true;
+      if (j > 0) {
+        if (!warp_all(pv_wait(j - 1))) return false;
+        __syncwarp();
+        tc_fence_after();
+      }
+      scale_tmem_row<D>(tO, g);   // rows without a rescale multiply by 1
+      return true;
+    };
+    for (int j = 0; j < nW; ++j) {
+      const int64_t i = first + (int64_t)stride * j;
+      const int b = j & 1;
       const int nvalid = (int)imin64(kEncTile, N - (tile0 + i) * kEncTile);
-      const uint32_t tS = tmem + lb + TM_S + (w * SB + b) * 64;
-      const uint32_t tP = tmem + lb + TM_P + (w * SB + b) * 32;
-      if (!warp_all(mbar_wait(&s_full[w * SB + b], (uint32_t)((j / SB) & 1)) && !*abort_flag)) {
+      const bool full = (nvalid == kEncTile);   // warp-uniform: only a head's last tile is partial
+      const uint32_t tS = tW + 48 * b;
+      if (!warp_all(mbar_wait(&s_full[2 * w + b], (uint32_t)((j >> 1) & 1)) && !*abort_flag)) {
         ok = false;
         break;
       }
       __syncwarp();
       tc_fence_after();
-      const bool full = (nvalid == kEncTile);   // warp-uniform: only a head's last tile is partial
-      // Before the first P store: the previous P.V must be done (P buffer
-      // free, O stable) and O must pay any rescale decided after that tile.
-      bool ready = (j == 0);
-      auto make_ready = [&]() -> bool {
-        if (ready) return true;
-        ready = true;
-        if (!warp_all(mbar_wait(&pv_done[w], (uint32_t)((j - 1) & 1)))) return false;
-        __syncwarp();
-        tc_fence_after();
-        if (warp_any(pend != 1.f)) scale_tmem_row<D>(tO, pend);   // rows without a rescale x 1
-        pend = 1.f;
-        return true;
-      };
       // Optimistic single pass (every tile after a warpgroup's first): P is
       // taken against the running reference m_ref while the tile max is
       // folded in.  A max above m_ref + kRescaleTau moves m_ref after the
       // tile (l now, O before the next P.V); a max above m_ref + kRedoTau,
-      // where P could overflow, makes the whole warp recompute the tile with
-      // the exact max.
+      // where P could overflow, makes the whole warp recompute the tile
+      // with the exact max.  P stays in registers until that check passes.
       bool exact = warp_any(mref == -INFINITY);
       if (!exact) {
         const float neg = -mref;
         float mf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         float sf[4] = {0.f, 0.f, 0.f, 0.f};
-        bool good = true;
-#pragma unroll
-        for (int cc = 0; cc < kEncTile / 32; ++cc) {
+        uint32_t pa[16], pb[8];
+        {
           uint32_t a[32];
-          tmem_ld32(tS + 32 * cc, a);
+          tmem_ld32(tS, a);
           tmem_wait_ld_dep(a);
           if (!full) {   // tokens past the end of the head get weight 0
 #pragma unroll
             for (int t = 0; t < 32; ++t)
-              if (32 * cc + t >= nvalid) a[t] = __float_as_uint(-INFINITY);
+              if (t >= nvalid) a[t] = __float_as_uint(-INFINITY);
           }
           max_fold32(a, mf);
-          uint32_t pk[16];
-          exp_pack32<kPolyEvery>(a, c, neg, pk, sf);
-          if (cc == 0 && !make_ready()) {   // overlap the P.V wait with chunk 0's exponentials
-            good = false;
-            break;
-          }
-          tmem_st16(tP + 16 * cc, pk);
+          exp_pack32<kPolyEvery>(a, c, neg, pa, sf);
         }
-        if (!good) {
-          ok = false;
-          break;
+        {
+          uint32_t a[16];
+          tmem_ld16(tS + 32, a);
+          tmem_wait_ld_dep16(a);
+          if (!full) {
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+              if (32 + t >= nvalid) a[t] = __float_as_uint(-INFINITY);
+          }
+          max_fold16(a, mf);
+          exp_pack16(a, c, neg, pb, sf);
         }
         const float mx2 = fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3])) * c;
         if (warp_any(mx2 > mref + kRedoTau)) {
           exact = true;
         } else {
+          if (!scale_O(j, pend)) {   // a rescale decided after the previous tile
+            ok = false;
+            break;
+          }
+          pend = 1.f;
+          tmem_st16(tS, pa);          // P over S columns already read
+          tmem_st8(tS + 16, pb);
           const float sum = (sf[0] + sf[1]) + (sf[2] + sf[3]);
           if (mx2 > mref + kRescaleTau) {
             pend = ex2(mref - mx2);
@@ -353,72 +365,89 @@ __global__ void __launch_bounds__(kThreads, (SB == 1) ? 2 : 1)
       if (exact) {
         // pass 1: exact tile max of the raw logits (masked past the end of the head)
         float mf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int cc = 0; cc < kEncTile / 32; ++cc) {
+        {
           uint32_t a[32];
-          tmem_ld32(tS + 32 * cc, a);
+          tmem_ld32(tS, a);
           tmem_wait_ld_dep(a);
-          if (full) {
-            max_fold32(a, mf);
-          } else {
 #pragma unroll
-            for (int t = 0; t < 32; ++t)
-              if (32 * cc + t < nvalid) mf[t & 3] = fmaxf(mf[t & 3], __uint_as_float(a[t]));
-          }
+          for (int t = 0; t < 32; ++t)
+            if (t < nvalid) mf[t & 3] = fmaxf(mf[t & 3], __uint_as_float(a[t]));
+        }
+        {
+          uint32_t a[16];
+          tmem_ld16(tS + 32, a);
+          tmem_wait_ld_dep16(a);
+#pragma unroll
+          for (int t = 0; t < 16; ++t)
+            if (32 + t < nvalid) mf[t & 3] = fmaxf(mf[t & 3], __uint_as_float(a[t]));
         }
         const float mx2 = fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3])) * c;
-        if (!make_ready()) {
-          ok = false;
-          break;
-        }
         float f = 1.f;   // rescale of this row's earlier tiles (1 when the max did not move)
         if (mx2 > mref) {
           if (mref != -INFINITY) f = ex2(mref - mx2);
           mref = mx2;
         }
         l *= f;
-        if (warp_any(f != 1.f)) scale_tmem_row<D>(tO, f);
-        // pass 2: P = 2^(c S - m_ref) as bf16 pairs, and its row sum
+        if (!scale_O(j, pend * f)) {
+          ok = false;
+          break;
+        }
+        pend = 1.f;
+        // pass 2: P = 2^(c S - m_ref) as bf16 pairs, and its row sum; chunk
+        // 0's P lands on S columns [0, 16) and chunk 1's on [16, 24), both
+        // already read.
         const float neg = -mref;
         float sf[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int cc = 0; cc < kEncTile / 32; ++cc) {
+        {
           uint32_t a[32];
-          tmem_ld32(tS + 32 * cc, a);
+          tmem_ld32(tS, a);
           tmem_wait_ld_dep(a);
           if (!full) {
 #pragma unroll
             for (int t = 0; t < 32; ++t)
-              if (32 * cc + t >= nvalid) a[t] = __float_as_uint(-INFINITY);
+              if (t >= nvalid) a[t] = __float_as_uint(-INFINITY);
           }
           uint32_t pk[16];
           exp_pack32<kPolyEvery>(a, c, neg, pk, sf);
-          tmem_st16(tP + 16 * cc, pk);
+          tmem_st16(tS, pk);
+        }
+        {
+          uint32_t a[16];
+          tmem_ld16(tS + 32, a);
+          tmem_wait_ld_dep16(a);
+          if (!full) {
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+              if (32 + t >= nvalid) a[t] = __float_as_uint(-INFINITY);
+          }
+          uint32_t pk[8];
+          exp_pack16(a, c, neg, pk, sf);
+          tmem_st8(tS + 16, pk);
         }
         l += (sf[0] + sf[1]) + (sf[2] + sf[3]);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sp_done[w * SB + b]);
+      mbar_arrive(&sp_done[2 * w + b]);
     }
     float acc[D];
 #pragma unroll
     for (int d = 0; d < D; ++d) acc[d] = 0.f;
     if (ok && nW > 0) {
-      ok = warp_all(mbar_wait(&pv_done[w], (uint32_t)((nW - 1) & 1)));
+      ok = warp_all(pv_wait(nW - 1));
       __syncwarp();
       tc_fence_after();
       if (ok) {
         if (D == 32) {
           uint32_t o[32];
           tmem_ld32(tO, o);
-          tmem_wait_ld();
+          tmem_wait_ld_dep(o);
 #pragma unroll
           for (int d = 0; d < D; ++d) acc[d] = __uint_as_float(o[d]) * pend;
         } else {
           uint32_t o[16];
           tmem_ld16(tO, o);
-          tmem_wait_ld();
+          tmem_wait_ld_dep16(o);
 #pragma unroll
           for (int d = 0; d < D; ++d) acc[d] = __uint_as_float(o[d & 15]) * pend;
         }
@@ -740,8 +769,6 @@ cudaError_t make_map(CUtensorMap* m, const void* base, int D, int64_t rows, int6
   return cudaSuccess;
 }
 
-constexpr int kEncSB = 1;   // S buffers per softmax warpgroup (1: two CTAs per SM)
-
 template <int D, int M>
 cudaError_t tc_encode_t(const void* Q, int64_t qbs, const void* K, const void* V, const Dims& d,
                         float scale, const ChunkPlan& plan, float* pml, float* pacc,
@@ -752,15 +779,13 @@ cudaError_t tc_encode_t(const void* Q, int64_t qbs, const void* K, const void* V
   if ((e = make_map(&mq, Q, D, M, q_per_batch ? d.BH() : d.H, 128)) != cudaSuccess) return e;
   if ((e = make_map(&mk, K, D, d.N, d.BH(), kEncTile)) != cudaSuccess) return e;
   if ((e = make_map(&mv, V, D, d.N, d.BH(), kEncTile)) != cudaSuccess) return e;
-  // SB = 1: two CTAs per SM (their TMEM, 2 x 256 columns, fits exactly);
-  // SB = 2: the smem request keeps one CTA (and its 512 columns) per SM.
-  const int need = EncLayout<D, M>::BYTES + 1024;
-  const int smem = (kEncSB == 1 || need > kMinSmemBytes) ? need : kMinSmemBytes;
-  e = cudaFuncSetAttribute(tc_encode_kernel<D, M, kEncSB>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  // two CTAs per SM: their TMEM (2 x 256 columns) fits exactly
+  const int smem = EncLayout<D, M>::BYTES + 1024;
+  e = cudaFuncSetAttribute(tc_encode_kernel<D, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem);
   if (e != cudaSuccess) return e;
   dim3 grid(plan.chunks, (unsigned)d.BH());
-  tc_encode_kernel<D, M, kEncSB><<<grid, kThreads, smem, st>>>(
+  tc_encode_kernel<D, M><<<grid, kThreads, smem, st>>>(
       mq, mk, mv, (int)d.H, d.N, q_per_batch, scale * kLog2e, plan.tiles_per_bh, plan.chunk_tiles,
       plan.slots_per_bh(), pml, pacc, err);
   return cudaPeekAtLastError();

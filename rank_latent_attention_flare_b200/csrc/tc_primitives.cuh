@@ -171,6 +171,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
+// tcgen05.wait::ld that names 16 loaded registers as in/out operands.
+__device__ __forceinline__ void tmem_wait_ld_dep16(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
+}
+
 // 32 lanes x 64 consecutive 32-bit columns in one load.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
   asm volatile(
@@ -205,6 +215,13 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
       "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
       : "memory");
 }
 
@@ -322,6 +339,17 @@ __device__ __forceinline__ float exp2_fma(float x) {
   return __uint_as_float((__float_as_uint(t) << 23) + __float_as_uint(p));
 }
 
+// Max of 16 values folded into four independent accumulators.
+__device__ __forceinline__ void max_fold16(const uint32_t (&a)[16], float (&m)[4]) {
+#pragma unroll
+  for (int t = 0; t < 16; t += 8) {
+    m[0] = max3(m[0], __uint_as_float(a[t + 0]), __uint_as_float(a[t + 1]));
+    m[1] = max3(m[1], __uint_as_float(a[t + 2]), __uint_as_float(a[t + 3]));
+    m[2] = max3(m[2], __uint_as_float(a[t + 4]), __uint_as_float(a[t + 5]));
+    m[3] = max3(m[3], __uint_as_float(a[t + 6]), __uint_as_float(a[t + 7]));
+  }
+}
+
 // p = 2^(a*c + neg) for 32 logits: packed into 16 bf16 pairs, sums folded
 // into four independent accumulators.  With POLY_EVERY = k > 0, every k-th
 // pair is computed on the FMA pipe (exp2_fma) instead of the MUFU.
@@ -344,6 +372,18 @@ __device__ __forceinline__ void exp_pack32(const uint32_t (&a)[32], float c, flo
     const bool poly = POLY_EVERY > 0 && (t % (POLY_EVERY > 0 ? POLY_EVERY : 1)) == POLY_EVERY - 1;
     const float p0 = poly ? exp2_fma(x0) : ex2(x0);
     const float p1 = poly ? exp2_fma(x1) : ex2(x1);
+    s[t & 3] += p0 + p1;
+    pk[t] = pack_bf16(p0, p1);
+  }
+}
+
+// p = 2^(a*c + neg) for 16 logits: 8 bf16 pairs, sums into four accumulators.
+__device__ __forceinline__ void exp_pack16(const uint32_t (&a)[16], float c, float neg,
+                                           uint32_t (&pk)[8], float (&s)[4]) {
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    const float p0 = ex2(fmaf(__uint_as_float(a[2 * t]), c, neg));
+    const float p1 = ex2(fmaf(__uint_as_float(a[2 * t + 1]), c, neg));
     s[t & 3] += p0 + p1;
     pk[t] = pack_bf16(p0, p1);
   }

@@ -137,7 +137,7 @@ def test_gpu_rejects_invalid_arguments_without_side_effects():
 @pytest.mark.parametrize("M", [128, 256])
 @pytest.mark.parametrize("regime", ["spiky", "growing"])
 def test_encode_running_max_over_many_tiles(M, regime):
-    # One head of 262,144 tokens: every encode CTA walks many 64-token tiles,
+    # One head of 262,144 tokens: every encode CTA walks many 48-token tiles,
     # so the running-max machinery is exercised.  "spiky": scale x100 makes
     # tile maxima jump by far more than 2^64 (tiles recomputed with the exact
     # max); "growing": keys grow steadily along the sequence, so the running
