@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int i = 0; i < (int)ntiles; ++i) {
           const int s = i % kEncStages;
           const uint32_t ph = (uint32_t)((i / kEncStages) & 1);
-          if (i >= kEncStages && !mbar_wait(&kv_empty[s], ph ^ 1)) {
+          if (i >= kEncStages && !mbar_wait_sleep(&kv_empty[s], ph ^ 1)) {
             record_error(err, kErrEncTmaWait);
             *abort_flag = 1;
             break;
@@ -192,8 +192,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         // let every load still in flight land before the CTA can exit
         for (int i = (issued > kEncStages ? issued - kEncStages : 0); i < issued; ++i)
-          mbar_wait(&kv_full[i % kEncStages], (uint32_t)((i / kEncStages) & 1));
-        mbar_wait(q_full, 0);
+          mbar_wait_sleep(&kv_full[i % kEncStages], (uint32_t)((i / kEncStages) & 1));
+        mbar_wait_sleep(q_full, 0);
       }
     } else if (warp == kWarpMma || warp == kWarpMma + 1) {
       // -------------------------------------- MMA issuers, one per warpgroup
@@ -213,11 +213,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint64_t dK = smem_desc(kv0, 16, 8 * RB, SW);
         const uint64_t dV = smem_desc(kv0 + L::TILE, L::TILE, 8 * RB, SW);
         const uint32_t tW = tmem + 128 * w;
-        bool ok = mbar_wait(q_full, 0);
+        bool ok = mbar_wait_sleep(q_full, 0);
         auto issue_S = [&](int j) -> bool {
           const int i = first + stride * j;
           const int s = i % kEncStages;
-          if (!mbar_wait(&kv_full[s], (uint32_t)((i / kEncStages) & 1))) return false;
+          if (!mbar_wait_sleep(&kv_full[s], (uint32_t)((i / kEncStages) & 1))) return false;
           tc_fence_after();
           const uint32_t koff = (uint32_t)(s * 2 * L::TILE) >> 4;
           const int b = j & 1;
@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int j = 0; ok && j < 2 && j < nw; ++j) ok = issue_S(j);
         for (int j = 0; ok && j < nw; ++j) {
           const int b = j & 1;
-          if (!mbar_wait(&sp_done[2 * w + b], (uint32_t)((j >> 1) & 1))) {
+          if (!mbar_wait_sleep(&sp_done[2 * w + b], (uint32_t)((j >> 1) & 1))) {
             ok = false;
             break;
           }
@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           mma_commit(&kv_empty[i % kEncStages]);
           if (j + 2 < nw) {
             // buffer b still holds the P this P.V reads: wait for it to finish
-            if (!mbar_wait(&pv_done[2 * w + b], (uint32_t)((j >> 1) & 1))) {
+            if (!mbar_wait_sleep(&pv_done[2 * w + b], (uint32_t)((j >> 1) & 1))) {
               ok = false;
               break;
             }
@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           *abort_flag = 1;
         }
         mma_commit(drain + w);
-        mbar_wait(drain + w, 0);
+        mbar_wait_sleep(drain + w, 0);
       }
     }
   } else {
@@ -561,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int64_t i = 0; i < ntiles; ++i) {
         const int s = (int)(i % kDecStages);
         const uint32_t ph = (uint32_t)((i / kDecStages) & 1);
-        if (i >= kDecStages && !mbar_wait(&k_empty[s], ph ^ 1)) {
+        if (i >= kDecStages && !mbar_wait_sleep(&k_empty[s], ph ^ 1)) {
           record_error(err, kErrDecTmaWait);
           *abort_flag = 1;
           break;
@@ -573,8 +573,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         issued = i + 1;
       }
       for (int64_t i = (issued > kDecStages ? issued - kDecStages : 0); i < issued; ++i)
-        mbar_wait(&k_full[i % kDecStages], (uint32_t)((i / kDecStages) & 1));
-      mbar_wait(qz_full, 0);
+        mbar_wait_sleep(&k_full[i % kDecStages], (uint32_t)((i / kDecStages) & 1));
+      mbar_wait_sleep(qz_full, 0);
     }
   } else if (warp == kWarpMma) {
     if (lane == 0) {
@@ -582,13 +582,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idY = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t q_addr = smem_u32(Qs);
       const uint32_t z_addr = smem_u32(Zs);
-      bool ok = mbar_wait(qz_full, 0);
+      bool ok = mbar_wait_sleep(qz_full, 0);
       auto issue_S = [&](int64_t i) -> bool {
         const int w = (int)(i & 1);
         const int64_t j = i >> 1;
         const int s = (int)(i % kDecStages);
-        if (!mbar_wait(&k_full[s], (uint32_t)((i / kDecStages) & 1))) return false;
-        if (j > 0 && !mbar_wait(&s_empty[w], (uint32_t)((j - 1) & 1))) return false;
+        if (!mbar_wait_sleep(&k_full[s], (uint32_t)((i / kDecStages) & 1))) return false;
+        if (j > 0 && !mbar_wait_sleep(&s_empty[w], (uint32_t)((j - 1) & 1))) return false;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(smem + L::K_OFF + s * L::TILE);
 #pragma unroll
@@ -602,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_Y = [&](int64_t i) -> bool {
         const int w = (int)(i & 1);
         const int64_t j = i >> 1;
-        if (!mbar_wait(&p_full[w], (uint32_t)(j & 1))) return false;
+        if (!mbar_wait_sleep(&p_full[w], (uint32_t)(j & 1))) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < M / 16; ++kk) {
@@ -625,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 1;
       }
       mma_commit(drain);
-      mbar_wait(drain, 0);
+      mbar_wait_sleep(drain, 0);
     }
     }
   } else {
@@ -639,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int64_t j = 0; j < nW; ++j) {
       const int64_t i = 2 * j + w;
       const int64_t tok = (tile0 + i) * kTile + r;
-      if (!warp_all(mbar_wait(&s_full[w], (uint32_t)(j & 1)) && !*abort_flag)) {
+      if (!warp_all(mbar_wait_sleep(&s_full[w], (uint32_t)(j & 1)) && !*abort_flag)) {
         ok = false;
         break;
       }
@@ -681,7 +681,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[w]);
-      if (!warp_all(mbar_wait(&y_full[w], (uint32_t)(j & 1)))) {
+      if (!warp_all(mbar_wait_sleep(&y_full[w], (uint32_t)(j & 1)))) {
         ok = false;
         break;
       }

@@ -14,6 +14,7 @@ namespace flare {
 namespace tc {
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
+constexpr uint32_t kSuspendHintNs = 100000u;       // per poll; far below the bound
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -69,6 +70,34 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
       : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
+}
+
+// try_wait with a suspend-time hint: the thread sleeps in hardware until the
+// phase completes (or the hint expires) instead of re-issuing the poll.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
+  return ok != 0;
+}
+
+// As mbar_wait, but suspended between polls: for waits whose spinning would
+// take issue slots from the exponential-bound softmax warps on the same SM
+// sub-partition.  Same bound; false on timeout.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait_sleep(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait_sleep(bar, parity)) return true;
+    if (globaltimer() - t0 > kWaitLimitNs) return false;
+  }
 }
 
 // Waits for the phase with the given parity to complete; false on timeout.
@@ -362,31 +391,59 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int POLY_EVERY>
-__device__ __forceinline__ void exp_pack32(const uint32_t (&a)[32], float c, float neg,
-                                           uint32_t (&pk)[16], float (&s)[4]) {
+// Packed fp32x2 arithmetic (sm_100): one instruction for two lanes of
+// float work, halving the issue slots of the scale-shift and the row sums.
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void split_f32x2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// 2^(a*c + neg) for NP consecutive pairs of logits: bf16 pairs into pk, the
+// values summed into s (s[0], s[2] collect even lanes, s[1], s[3] odd ones).
+template <int NP, int POLY_EVERY>
+__device__ __forceinline__ void exp_pack_pairs(const uint32_t* a, float c, float neg,
+                                               uint32_t* pk, float (&s)[4]) {
+  const uint64_t c2 = f32x2(c, c), n2 = f32x2(neg, neg);
+  uint64_t acc[2] = {f32x2(s[0], s[1]), f32x2(s[2], s[3])};
 #pragma unroll
-  for (int t = 0; t < 16; ++t) {
-    const float x0 = fmaf(__uint_as_float(a[2 * t]), c, neg);
-    const float x1 = fmaf(__uint_as_float(a[2 * t + 1]), c, neg);
+  for (int t = 0; t < NP; ++t) {
+    float x0, x1;
+    split_f32x2(fma_f32x2(f32x2(__uint_as_float(a[2 * t]), __uint_as_float(a[2 * t + 1])), c2, n2),
+                x0, x1);
     const bool poly = POLY_EVERY > 0 && (t % (POLY_EVERY > 0 ? POLY_EVERY : 1)) == POLY_EVERY - 1;
     const float p0 = poly ? exp2_fma(x0) : ex2(x0);
     const float p1 = poly ? exp2_fma(x1) : ex2(x1);
-    s[t & 3] += p0 + p1;
+    acc[t & 1] = add_f32x2(acc[t & 1], f32x2(p0, p1));
     pk[t] = pack_bf16(p0, p1);
   }
+  split_f32x2(acc[0], s[0], s[1]);
+  split_f32x2(acc[1], s[2], s[3]);
+}
+
+template <int POLY_EVERY>
+__device__ __forceinline__ void exp_pack32(const uint32_t (&a)[32], float c, float neg,
+                                           uint32_t (&pk)[16], float (&s)[4]) {
+  exp_pack_pairs<16, POLY_EVERY>(a, c, neg, pk, s);
 }
 
 // p = 2^(a*c + neg) for 16 logits: 8 bf16 pairs, sums into four accumulators.
 __device__ __forceinline__ void exp_pack16(const uint32_t (&a)[16], float c, float neg,
                                            uint32_t (&pk)[8], float (&s)[4]) {
-#pragma unroll
-  for (int t = 0; t < 8; ++t) {
-    const float p0 = ex2(fmaf(__uint_as_float(a[2 * t]), c, neg));
-    const float p1 = ex2(fmaf(__uint_as_float(a[2 * t + 1]), c, neg));
-    s[t & 3] += p0 + p1;
-    pk[t] = pack_bf16(p0, p1);
-  }
+  exp_pack_pairs<8, 0>(a, c, neg, pk, s);
 }
 
 }  // namespace tc
