@@ -157,27 +157,32 @@ def dist_done(world: int):
 
 def oracle_sample_rate(target_s: float, w=WORKLOAD, seed: int = 0):
     """Times the oracle's FLARE forward on a bounded sample of the workload:
-    one (b, h) head with n_s of its N tokens (same M, D, dtype rounding).
-    The sample size is calibrated so the timed run takes about target_s
-    seconds.  Returns (tokens/s of the full workload, description, cores).
-    A workload token carries H heads, so a head-token is 1/H of a token."""
+    h_s of its heads with n_s of their N tokens each (same M, D, dtype
+    rounding), sized so the timed run takes about target_s seconds (a whole
+    head first, then more heads).  Returns (tokens/s of the full workload,
+    description, cores, n_s, h_s).  A workload token carries H heads, so one
+    head-token is 1/H of a token."""
     import oracle
     cores = oracle.num_threads()
 
-    def run(n_s):
-        x = make_inputs(1, 1, n_s, w.M, w.D, dtype=w.torch_dtype, seed=seed)
+    def run(h_s, n_s):
+        x = make_inputs(1, h_s, n_s, w.M, w.D, dtype=w.torch_dtype, seed=seed)
         t0 = time.perf_counter()
         oracle.flare_fwd(x["Q"], x["K"], x["V"], w.scale)
         return time.perf_counter() - t0
 
     n_cal = 4096
-    t_cal = max(run(n_cal), 1e-4)
+    t_cal = max(run(1, n_cal), 1e-4)
     n_s = int(min(w.N, max(n_cal, n_cal * target_s / t_cal)))
-    t = run(n_s)
-    rate = (n_s / w.H) / t
-    desc = (f"oracle FLARE fwd (double, OpenMP) on 1 of {w.B * w.H} heads, {n_s} of {w.N} "
-            f"tokens, M={w.M}, D={w.D}; {t:.2f} s; tokens/s scaled by 1/H per head-token")
-    return rate, desc, cores, n_s
+    h_s = 1
+    if n_s == w.N:
+        h_s = int(max(1, min(w.B * w.H, target_s / (t_cal * w.N / n_cal))))
+    t = run(h_s, n_s)
+    rate = (h_s * n_s / w.H) / t
+    desc = (f"oracle FLARE fwd (double, OpenMP) on {h_s} of {w.B * w.H} heads x {n_s} of "
+            f"{w.N} tokens, M={w.M}, D={w.D}; {t:.2f} s; tokens/s counts 1/H token per "
+            f"head-token")
+    return rate, desc, cores, n_s, h_s
 
 
 # ------------------------------------------------------------------ ours
@@ -347,10 +352,16 @@ def run_ours(args, rank, world, local):
     peaks, peak_kind = load_peaks()
     roof = roofline_entry(kernel_ms, peaks, peak_kind, w)
 
+    rows = None
+    if not args.no_rows:
+        del Y, ws
+        g.clear()
+        torch.cuda.empty_cache()
+        rows = time_other_rows(dev, peaks, peak_kind, seed=rank)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        del g
-        rate, desc, cores, _ = oracle_sample_rate(args.cpu_seconds)
+        rate, desc, cores, _, _ = oracle_sample_rate(args.cpu_seconds)
         cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": desc}
 
@@ -368,6 +379,7 @@ def run_ours(args, rank, world, local):
                    "kernels": "tcgen05" if path == 1 else "cuda-core"},
         "kernel_ms": {k: round(v, 4) for k, v in kernel_ms.items()},
         "roofline": roof,
+        "rows": rows,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": 3 * args.steps * world,
@@ -375,6 +387,101 @@ def run_ours(args, rank, world, local):
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------- the other rows
+
+def _row_roofline(t_ms: float, exps: float, flops: float, hbm_bytes: float, peaks: dict,
+                  peak_kind: str):
+    """Roofline of a whole row: the slowest of the exponential, tensor and
+    HBM limits (each at its peak) over the measured time."""
+    clk = float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
+    mufu = SMS * MUFU_PER_CLK_SM * clk            # exp/s
+    lim = {"exp": exps / mufu, "tensor": flops / (float(peaks["bf16_tflops"]) * 1e12),
+           "hbm": hbm_bytes / (float(peaks["hbm_gbs"]) * 1e9)}
+    bound = max(lim, key=lim.get)
+    t = t_ms / 1e3
+    return {"bound": bound, "t_roof_ms": round(lim[bound] * 1e3, 4),
+            "frac": round(lim[bound] / t, 4),
+            "exp_frac": round(lim["exp"] / t, 4), "tensor_frac": round(lim["tensor"] / t, 4),
+            "hbm_frac": round(lim["hbm"] / t, 4),
+            "algorithmic": {"exps": exps, "tensor_flops": flops, "hbm_bytes": hbm_bytes},
+            "peaks": f"MUFU {mufu / 1e9:.0f} Gexp/s (derived), {peak_kind} bf16 "
+                     f"{peaks['bf16_tflops']} TFLOP/s, {peak_kind} HBM {peaks['hbm_gbs']} GB/s"}
+
+
+def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0):
+    """Times the FLARE++ forward (B=2 H=8 N=262,144 M=256 D=32) and the
+    forward + backward of B=8 H=8 N=16,384 M=128 D=32, both bf16, on the
+    same device with CUDA events (median of `iters` launches after 3
+    warm-ups, L2 flushed before each by writing 256 MB)."""
+    import torch
+
+    import rank_latent_attention_flare_b200 as fl
+
+    st = torch.cuda.current_stream()
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        pairs = []
+        for _ in range(iters):
+            flush_buf.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            fn()
+            b.record(st)
+            pairs.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in pairs)
+
+    rows = {}
+    w = WORKLOADS["c4_ppfwd_bf16_256k"]
+    x = make_inputs(w.B, w.H, w.N, w.M, w.D, dtype=w.torch_dtype, seed=seed)
+    g = {k: v.to(dev) for k, v in x.items()}
+    ws = fl.alloc_workspace(fl.FLARE_OP_PP_FWD, w.B, w.H, w.N, w.M, w.D, w.torch_dtype, dev)
+    ms = timed(lambda: fl.flare_pp_fwd(g["Q"], g["K"], g["V"], w.scale, workspace=ws))
+    if fl.device_status(ws) != 0:
+        raise RuntimeError("device wait ran out in the FLARE++ forward")
+    u = w.B * w.H * w.N
+    rows["flare_pp_fwd"] = {
+        "workload": f"FLARE++ fwd B={w.B} H={w.H} N={w.N} M={w.M} D={w.D} bf16",
+        "ms": round(ms, 4), "tokens_per_s": w.B * w.N / (ms / 1e3),
+        "roofline": _row_roofline(ms, 3.0 * u * w.M, 12.0 * u * w.M * w.D,
+                                  6.0 * u * w.D * 2, peaks, peak_kind)}
+    del g, ws
+
+    w = WORKLOADS["c5_fwdbwd_bf16_16k"]
+    x = make_inputs(w.B, w.H, w.N, w.M, w.D, dtype=w.torch_dtype, seed=seed, with_dy=True)
+    g = {k: v.to(dev) for k, v in x.items()}
+    wsf = fl.alloc_workspace(fl.FLARE_OP_FWD, w.B, w.H, w.N, w.M, w.D, w.torch_dtype, dev)
+    wsb = fl.alloc_workspace(fl.FLARE_OP_BWD, w.B, w.H, w.N, w.M, w.D, w.torch_dtype, dev)
+    saved = {}
+
+    def fwd():
+        saved["out"] = fl.flare_fwd(g["Q"], g["K"], g["V"], w.scale, save=True, workspace=wsf)
+
+    ms_f = timed(fwd)
+    _, Z, lse = saved["out"]
+    ms_b = timed(lambda: fl.flare_bwd(g["Q"], g["K"], g["V"], g["dY"], Z, lse, w.scale,
+                                      workspace=wsb))
+    if fl.device_status(wsf) != 0 or fl.device_status(wsb) != 0:
+        raise RuntimeError("device wait ran out in the forward + backward")
+    u = w.B * w.H * w.N
+    ms = ms_f + ms_b
+    rows["flare_fwd_bwd"] = {
+        "workload": f"FLARE fwd+bwd B={w.B} H={w.H} N={w.N} M={w.M} D={w.D} bf16",
+        "ms": round(ms, 4), "fwd_ms": round(ms_f, 4), "bwd_ms": round(ms_b, 4),
+        "tokens_per_s": w.B * w.N / (ms / 1e3),
+        "roofline": _row_roofline(ms, 4.0 * u * w.M, 28.0 * u * w.M * w.D,
+                                  9.0 * u * w.D * 2, peaks, peak_kind),
+        "bwd_roofline": _row_roofline(ms_b, 2.0 * u * w.M, 20.0 * u * w.M * w.D,
+                                      5.0 * u * w.D * 2, peaks, peak_kind)}
+    del g, wsf, wsb, flush_buf
+    torch.cuda.empty_cache()
+    return rows
 
 
 # ------------------------------------------------------------- reference
@@ -388,17 +495,17 @@ def run_reference(args, rank, world):
     import oracle
     budget = max(30.0, args.ref_seconds)
     per_step = budget / (args.steps + args.warmup)
-    _, _, cores, n_s = oracle_sample_rate(per_step)
-    x = make_inputs(1, 1, n_s, w.M, w.D, dtype=w.torch_dtype, seed=0)
+    _, _, cores, n_s, h_s = oracle_sample_rate(per_step)
+    x = make_inputs(1, h_s, n_s, w.M, w.D, dtype=w.torch_dtype, seed=0)
     for _ in range(args.warmup):
         oracle.flare_fwd(x["Q"], x["K"], x["V"], w.scale)
     t0 = time.perf_counter()
     for _ in range(args.steps):
         oracle.flare_fwd(x["Q"], x["K"], x["V"], w.scale)
     t = time.perf_counter() - t0
-    value = args.steps * (n_s / w.H) / t
-    sample = (f"per step: oracle FLARE fwd on 1 of {w.B * w.H} heads, {n_s} of {w.N} tokens "
-              f"(M={w.M}, D={w.D}); tokens/s scaled by 1/H per head-token")
+    value = args.steps * (h_s * n_s / w.H) / t
+    sample = (f"per step: oracle FLARE fwd on {h_s} of {w.B * w.H} heads x {n_s} of {w.N} "
+              f"tokens (M={w.M}, D={w.D}); tokens/s counts 1/H token per head-token")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -424,6 +531,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rows", action="store_true",
+                    help="skip the FLARE++ and forward+backward timings")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=120.0)
     ap.add_argument("--out-dir", default=None, help="where to write the clock samples")
