@@ -6,7 +6,7 @@ tensor-core kernels and CUDA-core kernels) behind the C ABI declared in
 """
 from ._lib import (FLARE_BF16, FLARE_F32, FLARE_OP_BWD, FLARE_OP_FWD, FLARE_OP_PP_FWD,
                    NOALLOC_SCRATCH_BYTES, FlareError, LIB_PATH, SIGNATURES, load)
-from .flare import (alloc_workspace, default_scale, device_status, flare_bwd, flare_combine,
+from .flare import (alloc_workspace, bwd_path, default_scale, device_status, flare_bwd, flare_combine,
                     flare_decode, flare_encode, flare_fwd, flare_fwd_noalloc, flare_pp_fwd,
                     fwd_path, workspace_size)
 
@@ -15,5 +15,5 @@ __all__ = [
     "LIB_PATH", "SIGNATURES", "load", "alloc_workspace", "default_scale", "device_status",
     "flare_bwd", "flare_combine", "flare_decode", "flare_encode", "flare_fwd", "flare_fwd_noalloc",
     "flare_pp_fwd", "NOALLOC_SCRATCH_BYTES",
-    "fwd_path", "workspace_size",
+    "bwd_path", "fwd_path", "workspace_size",
 ]

@@ -56,6 +56,7 @@ SIGNATURES = {
                             _sz, _vp]),
     "flare_device_status": (_i32, [_vp, _sz, _u32p, _vp]),
     "flare_fwd_path": (_i32, [_i64, _i64, _i64, _i64, _i64, _i32]),
+    "flare_bwd_path": (_i32, [_i64, _i64, _i64, _i64, _i64, _i32]),
     "flare_fwd_noalloc": (_i32, [_vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i32,
                                  _f32, _vp, _vp, _vp]),
 }

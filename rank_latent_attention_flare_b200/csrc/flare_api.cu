@@ -164,6 +164,11 @@ int flare_fwd_path(int64_t B, int64_t H, int64_t N, int64_t M, int64_t D, flare_
   return choose_path(N, M, D, dt).tc_fwd ? 1 : 0;
 }
 
+int flare_bwd_path(int64_t B, int64_t H, int64_t N, int64_t M, int64_t D, flare_dtype_t dt) {
+  if (check_sizes(B, H, N, M, D, dt) != FLARE_OK) return -1;
+  return choose_path(N, M, D, dt).tc_bwd ? 1 : 0;
+}
+
 flare_status_t flare_encode(const void* Q, int64_t qbs, const void* K, const void* V, int64_t B,
                             int64_t H, int64_t N, int64_t M, int64_t D, flare_dtype_t dt,
                             float scale, void* workspace, size_t workspace_bytes, void* stream) {

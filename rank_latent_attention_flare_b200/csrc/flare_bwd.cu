@@ -346,6 +346,8 @@ cudaError_t launch_bwd(const void* Q, int64_t qbs, const void* K, const void* V,
                        const float* Z, const float* lse, void* dQ, void* dK, void* dV,
                        const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,
                        char* ws, cudaStream_t st) {
+  if (choose_path(d.N, d.M, d.D, dt).tc_bwd)
+    return launch_tc_bwd(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
   if (dt == FLARE_F32)
     return d.D == 16 ? bwd_t<float, 16>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st)
                      : bwd_t<float, 32>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);

@@ -2,6 +2,7 @@
 // work partitioning, device helpers and kernel launchers.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -25,6 +26,12 @@ enum ErrorSite : uint32_t {
   kErrDecMmaWait = 0x202,
   kErrDecSoftmaxWait = 0x203,
   kErrTmemAlloc = 0x301,
+  kErrBwdATmaWait = 0x401,
+  kErrBwdAMmaWait = 0x402,
+  kErrBwdARowWait = 0x403,
+  kErrBwdBTmaWait = 0x501,
+  kErrBwdBMmaWait = 0x502,
+  kErrBwdBRowWait = 0x503,
 };
 
 // ------------------------------------------------------------------ planning
@@ -73,6 +80,7 @@ inline ChunkPlan plan_chunks(int64_t BH, int64_t N, int tile, int64_t cta_slots,
 // Which kernels a call uses.
 struct Path {
   bool tc_fwd = false;  // tcgen05 encode + decode
+  bool tc_bwd = false;  // tcgen05 backward (two passes over the tokens)
 };
 
 // The tcgen05 kernels cover bf16 with M in {128, 256} (one or two 128-row
@@ -80,6 +88,8 @@ struct Path {
 inline Path choose_path(int64_t N, int64_t M, int64_t D, flare_dtype_t dt) {
   Path p;
   p.tc_fwd = (dt == FLARE_BF16) && (M == 128 || M == 256) && (D == 16 || D == 32) &&
+             (N < (1LL << 31) - 256);
+  p.tc_bwd = (dt == FLARE_BF16) && (M == 128) && (D == 16 || D == 32) &&
              (N < (1LL << 31) - 256);
   return p;
 }
@@ -111,6 +121,11 @@ inline ChunkPlan bwd_plan(int64_t BH, int64_t N, int sms) {
   return plan_chunks(BH, N, kBwdTile, 2LL * sms, 1.0, 16 * (int64_t)sms);
 }
 
+// Both passes of the tensor-core backward: 128-token tiles, one CTA per SM.
+inline ChunkPlan tc_bwd_plan(int64_t BH, int64_t N, int sms) {
+  return plan_chunks(BH, N, kTcTile, sms, 6.0, 16 * (int64_t)sms);
+}
+
 // ------------------------------------------------------------- workspace
 
 struct WsLayout {
@@ -125,6 +140,12 @@ struct WsLayout {
   size_t dzp = 0;       // [BH*chunks][M][D] float  dZ partials
   size_t dz = 0;        // [BH][M][D] float
   size_t delta = 0;     // [BH][M] float  rowsum(dZ * Z)
+  // tensor-core backward (the dZ / dQ partials use dzp / dqp, one set each)
+  size_t stats = 0;     // [BH][N] float2  decode log-sum-exp (log2 units), delta_d
+  size_t dzs = 0;       // [BH][M][D] bf16  f * dZ
+  size_t aug = 0;       // [BH][M][16] bf16 extra K-step row (-f delta_e in three terms)
+  size_t params = 0;    // [BH] float2  R, fast-form flag
+  size_t lse2 = 0;      // [BH][M] float  lse in log2 units
   size_t total = 0;
   ChunkPlan enc, bwd;
 };
@@ -150,7 +171,17 @@ inline WsLayout ws_layout(flare_op_t op, int64_t B, int64_t H, int64_t N, int64_
   L.zf = take((size_t)BH * M * D * 4);
   L.zb = take((size_t)BH * M * D * 2);
   if (op == FLARE_OP_PP_FWD) L.qdyn = take((size_t)BH * M * D * esz);
-  if (op == FLARE_OP_BWD) {
+  if (op == FLARE_OP_BWD && choose_path(N, M, D, dt).tc_bwd) {
+    L.bwd = tc_bwd_plan(BH, N, sms);
+    const int64_t bslots = BH * L.bwd.chunks;
+    L.stats = take((size_t)BH * N * 8);
+    L.dzp = take((size_t)bslots * M * D * 4);
+    L.dqp = take((size_t)bslots * M * D * 4);
+    L.dzs = take((size_t)BH * M * D * 2);
+    L.aug = take((size_t)BH * M * 16 * 2);
+    L.params = take((size_t)BH * 8);
+    L.lse2 = take((size_t)BH * M * 4);
+  } else if (op == FLARE_OP_BWD) {
     L.bwd = bwd_plan(BH, N, sms);
     const int64_t bslots = BH * L.bwd.chunks;
     L.dkf = take((size_t)BH * N * D * 4);
@@ -218,6 +249,16 @@ cudaError_t launch_tc_encode(const void* Q, int64_t qbs, const void* K, const vo
 cudaError_t launch_tc_decode(const void* Q, int64_t qbs, const void* K,
                              const __nv_bfloat16* Zb, void* Y, const Dims& d, float scale,
                              const ChunkPlan& plan, uint32_t* err, cudaStream_t st);
+// 3-D TMA map over a bf16 tensor [depth][rows][D] (D in {16, 32}) with
+// boxes of box_rows whole rows, swizzled to match the UMMA descriptors
+// (64-byte swizzle for 64-byte rows, 32-byte for 32-byte rows).
+cudaError_t make_map(CUtensorMap* m, const void* base, int D, int64_t rows, int64_t depth,
+                     int box_rows);
+
+cudaError_t launch_tc_bwd(const void* Q, int64_t qbs, const void* K, const void* V,
+                          const void* dY, const float* Z, const float* lse, void* dQ, void* dK,
+                          void* dV, const Dims& d, float scale, const WsLayout& L, char* ws,
+                          cudaStream_t st);
 cudaError_t launch_bwd(const void* Q, int64_t qbs, const void* K, const void* V, const void* dY,
                        const float* Z, const float* lse, void* dQ, void* dK, void* dV,
                        const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,

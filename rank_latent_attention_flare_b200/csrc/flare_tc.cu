@@ -731,6 +731,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ============================================================== host side
 
+}  // namespace
+
+
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
     void* p = nullptr;
@@ -768,6 +771,8 @@ cudaError_t make_map(CUtensorMap* m, const void* base, int D, int64_t rows, int6
   }
   return cudaSuccess;
 }
+
+namespace {
 
 template <int D, int M>
 cudaError_t tc_encode_t(const void* Q, int64_t qbs, const void* K, const void* V, const Dims& d,

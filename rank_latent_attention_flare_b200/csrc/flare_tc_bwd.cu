@@ -1,0 +1,1060 @@
+// Tensor-core FLARE backward for sm_100a: bf16 inputs, M = 128 latents,
+// D in {16, 32}.  Gradients of sum(Y * dY) with respect to Q, K and V with
+// the logits of both stages recomputed on the tensor cores (tcgen05.mma,
+// TMEM accumulators, TMA-fed operands).  The pages give no backward; this is
+// the chain rule through the encode (skill page section 2: softmax over the
+// tokens of every latent row) and the decode (FLARE abstract: softmax over
+// the latents of every token), as in flare_bwd.cu.
+//
+// Token-major notation per (b, h), c = scale * log2(e), all exponentials in
+// base 2 ("log2 units"):
+//   S[n,m]   = K[n] . Q[m]                        (both stages' logits / scale)
+//   P_d[n,m] = 2^(c S - mx'[n])                   decode softmax over m;
+//              mx'[n] = c max_m S + log2(row sum) (its log-sum-exp)
+//   P_e[n,m] = 2^(c S - lse2[m])                  encode softmax over n;
+//              lse2 = forward lse * log2(e)
+//   dPd = dY Z^T, delta_d[n] = sum_m P_d dPd = dY[n] . Y[n]
+//   dPe = V dZ^T, delta_e[m] = dZ[m] . Z[m],  dZ = P_d^T dY
+//   G   = P_d (dPd - delta_d) + P_e (dPe - delta_e)   (the logit gradient / scale)
+//   dK = s G Q,  dQ = s G^T K,  dV = P_e^T... = sum_m P_e[n,m] dZ[m]
+//
+// Pass A (tc_bwd_a_kernel, per 128-token tile, one thread per token row):
+// S = K Q^T into TMEM; row max and P = 2^(c S - c max) as in the forward's
+// decode; P (bf16) into TMEM for Y = P Z and into shared memory for
+// dZ += P^T dY' with dY' = dY / rowsum written over the dY tile; the row's
+// mx' and delta_d = dY . Y go to the workspace.
+//
+// Between the passes (bwd_mid_kernel): dZ = sum of the chunk partials,
+// delta_e, and the split of the encode weights
+//   P_e[n,m] = P_d[n,m] * g[n] * f[m],  g[n] = 2^(mx'[n] - R), f[m] = 2^(R - lse2[m])
+// with R = max_m lse2[m].  f goes into the operand dZ'' = f dZ (bf16) and into
+// an extra K-step of the dPe'' = V dZ''^T - f delta_e product (three bf16
+// terms of -f delta_e against a tile of ones), so
+//   G = P_d (dPd - delta_d + g dPe''),   dV[n] = g[n] sum_m P_d[n,m] dZ''[m]
+// and pass B needs ONE exponential per token-latent pair.  When the lse2 of
+// a head spread over more than 64 (f or g could leave the float range) the
+// head takes the exact form instead: f = 1, P_e = 2^(c S - lse2[m]) per
+// element.
+//
+// Pass B (tc_bwd_b_kernel, per 128-token tile, latents in quarters of 32):
+// S, dPd and dPe'' of a quarter into TMEM; G and the dV weights (bf16) back
+// into TMEM for dK += G Q and dV += P dZ'' (tensor cores, token rows), and G
+// into shared memory for dQ += G^T K (latent rows, accumulated over the
+// chunk's tiles).  dK and dV are final per tile; dQ partials per chunk are
+// summed in a fixed order afterwards, so results are reproducible bitwise.
+//
+// Roles per CTA (384 threads): warps 0-3 and 4-7 are the row warpgroups,
+// warp 8 issues TMA loads, warp 9 issues the MMAs, warps 10-11 only lend
+// registers (as in the forward's decode kernel).
+#include <cudaTypedefs.h>
+
+#include "flare_internal.cuh"
+#include "tc_primitives.cuh"
+
+namespace flare {
+namespace {
+
+using namespace tc;
+
+constexpr int kT = 128;          // tokens per tile
+constexpr int kM = 128;          // latents
+constexpr int kThr = 384;
+constexpr int kRegsRow = 200;
+constexpr int kRegsPro = 104;
+constexpr int kWTma = 8;
+constexpr int kWMma = 9;
+constexpr int kAStages = 4;
+constexpr int kBStages = 3;
+constexpr uint32_t kSw128 = 2u;  // UMMA descriptor code of the 128-byte swizzle
+constexpr uint32_t kSw32 = 6u;   // ... and of the 32-byte swizzle
+constexpr float kSpreadMax = 64.f;  // log2 units: beyond, a head takes the exact form
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return (uint8_t*)(((uintptr_t)p + 1023) & ~(uintptr_t)1023);
+}
+
+// A [128 tokens x 128 latents] bf16 tile stored latent-contiguous, i.e. as
+// the MN-major A operand of a [latents x tokens] x [tokens x D] product:
+// 128-byte swizzle atoms of 64 latents x 8 tokens, consecutive atoms along
+// the tokens 1 KB apart, the second 64 latents 16 KB further.  Offset of the
+// 16-byte group of latents [8 grp, 8 grp + 8) in token row n.
+constexpr uint32_t kMnLbo = 16384, kMnSbo = 1024, kMnKStep = 2048;  // K step = 16 tokens
+__device__ __forceinline__ uint32_t mn_off(int n, int grp) {
+  return (uint32_t)((grp >> 3) * 16384 + (n >> 3) * 1024 + (n & 7) * 128 +
+                    (((grp & 7) ^ (n & 7)) << 4));
+}
+
+// Offset of 16-byte chunk ch of row r in a tile written by TMA with the
+// swizzle make_map uses for rows of 2D bytes (64B for D = 32, 32B for 16).
+template <int D>
+__device__ __forceinline__ uint32_t tma_row_chunk(int r, int ch) {
+  if (D == 32) return (uint32_t)(r * 64 + ((ch ^ ((r >> 1) & 3)) << 4));
+  return (uint32_t)(r * 32 + ((ch ^ ((r >> 2) & 1)) << 4));
+}
+
+// Empty asm that names 16 registers as in/out operands: placed after a
+// tcgen05.wait::ld it keeps every use of them behind the wait.
+__device__ __forceinline__ void reg_fence16(uint32_t (&r)[16]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]));
+}
+
+__device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+// ============================================================== pass A
+
+template <int D>
+struct ALayout {
+  static constexpr int M = kM;
+  static constexpr int RB = 2 * D;
+  static constexpr int TILE = kT * RB;        // one K or dY tile
+  static constexpr int PBUF = kT * M * 2;     // one P tile, MN-major
+  static constexpr int P_OFF = 0;             // one P buffer per row warpgroup
+  static constexpr int Q_OFF = 2 * PBUF;
+  static constexpr int Z_OFF = Q_OFF + M * RB;
+  static constexpr int ONE_OFF = Z_OFF + M * RB;  // second N block of Y's B operand
+  static constexpr int ST_OFF = ONE_OFF + M * RB;   // stages: K tile, dY tile
+  static constexpr int BAR_OFF = ST_OFF + kAStages * 2 * TILE;
+  static constexpr int NBARS = 2 * kAStages + 1 + 8 + 2;
+  static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+  static constexpr int BYTES = MISC_OFF + 16;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThr, 1)
+    tc_bwd_a_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmdY, const __grid_constant__ CUtensorMap tmZ,
+                    int H, int64_t N, int q_per_batch, float c, int64_t tiles_per_bh,
+                    int64_t chunk_tiles, float2* __restrict__ stats, float* __restrict__ dz_part,
+                    uint32_t* __restrict__ err) {
+  using L = ALayout<D>;
+  constexpr int M = L::M;
+  constexpr int RB = L::RB;
+  constexpr uint32_t SW = umma_swizzle_code(RB);
+  constexpr int R = M;          // TMEM columns per row warpgroup: S, then P and Y inside
+  constexpr int TY = M / 4;     // [Y | row sum of bf16 P] inside the warpgroup's columns
+  static_assert(TY + D + 16 <= 3 * M / 4, "Y must sit between the two P halves");
+  constexpr int TDZ = 2 * M;    // dZ accumulator (latent lanes)
+  constexpr uint32_t NCOLS = 512;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* bars = (uint64_t*)(smem + L::BAR_OFF);
+  uint64_t* st_full = bars;
+  uint64_t* st_empty = bars + kAStages;
+  uint64_t* qz_full = bars + 2 * kAStages;
+  uint64_t* s_full = qz_full + 1;   // [w] S of the warpgroup's tile in TMEM
+  uint64_t* p_full = s_full + 2;    // [w] P written (TMEM and shared memory)
+  uint64_t* y_full = p_full + 2;    // [w] Y = P Z complete
+  uint64_t* a_done = y_full + 2;    // [w] Y read, dY' written: TMEM columns free
+  uint64_t* dz_final = a_done + 2;
+  uint64_t* drain = dz_final + 1;
+  uint32_t* tmem_slot = (uint32_t*)(smem + L::MISC_OFF);
+  volatile int* abort_flag = (volatile int*)(smem + L::MISC_OFF + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x, chunks = gridDim.x;
+  const int64_t bh = blockIdx.y;
+  const int64_t h = bh % H;
+  const int64_t tile0 = (int64_t)chunk * chunk_tiles;
+  const int64_t ntiles = imin64(chunk_tiles, tiles_per_bh - tile0);
+
+  // Y = P [Z | e0]: the second N block of the B operand holds a one in
+  // column 0 of every latent row (same swizzled layout as the Z rows), so
+  // the accumulator's column D is the row sum of the bf16 P the MMA uses.
+  for (int m = threadIdx.x; m < M; m += blockDim.x) {
+#pragma unroll
+    for (int ch = 0; ch < D / 8; ++ch)
+      *reinterpret_cast<uint4*>(smem + L::ONE_OFF + tma_row_chunk<D>(m, ch)) =
+          make_uint4(ch == 0 ? 0x3F80u : 0u, 0u, 0u, 0u);
+  }
+  fence_proxy_async_smem();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kAStages; ++s) {
+      mbar_init(&st_full[s], 1);
+      mbar_init(&st_empty[s], 1);
+    }
+    mbar_init(qz_full, 1);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&s_full[w], 1);
+      mbar_init(&p_full[w], 128);
+      mbar_init(&y_full[w], 1);
+      mbar_init(&a_done[w], 128);
+    }
+    mbar_init(dz_final, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kWMma) tmem_alloc(tmem_slot, NCOLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp >= 8) {
+    regs_release<kRegsPro>();
+    if (warp == kWTma) {
+      if (lane == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmdY);
+        prefetch_tmap(&tmZ);
+        mbar_arrive_expect_tx(qz_full, 2 * M * RB);
+        tma_load_3d(smem + L::Q_OFF, &tmQ, qz_full, 0, 0, (int32_t)(q_per_batch ? bh : h));
+        tma_load_3d(smem + L::Z_OFF, &tmZ, qz_full, 0, 0, (int32_t)bh);
+        int64_t issued = 0;
+        for (int64_t i = 0; i < ntiles; ++i) {
+          const int s = (int)(i % kAStages);
+          const uint32_t ph = (uint32_t)((i / kAStages) & 1);
+          if (i >= kAStages && !mbar_wait_sleep(&st_empty[s], ph ^ 1)) {
+            record_error(err, kErrBwdATmaWait);
+            *abort_flag = 1;
+            break;
+          }
+          if (*abort_flag) break;
+          uint8_t* dst = smem + L::ST_OFF + s * 2 * L::TILE;
+          mbar_arrive_expect_tx(&st_full[s], 2 * L::TILE);
+          const int32_t tok = (int32_t)((tile0 + i) * kT);
+          tma_load_3d(dst, &tmK, &st_full[s], 0, tok, (int32_t)bh);
+          tma_load_3d(dst + L::TILE, &tmdY, &st_full[s], 0, tok, (int32_t)bh);
+          issued = i + 1;
+        }
+        for (int64_t i = (issued > kAStages ? issued - kAStages : 0); i < issued; ++i)
+          mbar_wait_sleep(&st_full[i % kAStages], (uint32_t)((i / kAStages) & 1));
+        mbar_wait_sleep(qz_full, 0);
+      }
+    } else if (warp == kWMma) {
+      if (lane == 0) {
+        constexpr uint32_t idS = idesc_bf16_f32(128, M, 0, 0);
+        constexpr uint32_t idY = idesc_bf16_f32(128, D + 16, 0, 1);   // N = [Z | e0]
+        constexpr uint32_t idZ = idesc_bf16_f32(128, D, 1, 1);
+        const uint32_t q_addr = smem_u32(smem + L::Q_OFF);
+        const uint32_t z_addr = smem_u32(smem + L::Z_OFF);
+        const uint32_t st0 = smem_u32(smem + L::ST_OFF);
+        const uint32_t p0 = smem_u32(smem + L::P_OFF);
+        bool ok = mbar_wait_sleep(qz_full, 0);
+        auto issue_S = [&](int64_t i) -> bool {
+          const int w = (int)(i & 1);
+          const int s = (int)(i % kAStages);
+          if (!mbar_wait_sleep(&st_full[s], (uint32_t)((i / kAStages) & 1))) return false;
+          tc_fence_after();
+          const uint32_t k_addr = st0 + s * 2 * L::TILE;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tmem + w * R, smem_desc(k_addr + 32 * kk, 16, 8 * RB, SW),
+                   smem_desc(q_addr + 32 * kk, 16, 8 * RB, SW), idS, kk > 0);
+          mma_commit(&s_full[w]);
+          return true;
+        };
+        auto issue_Y = [&](int64_t i) -> bool {
+          const int w = (int)(i & 1);
+          const int64_t j = i >> 1;
+          if (!mbar_wait_sleep(&p_full[w], (uint32_t)(j & 1))) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < M / 16; ++kk) {
+            const uint32_t acol = (kk < M / 32) ? 8 * kk : M / 2 + 8 * kk;
+            mma_ts(tmem + w * R + TY, tmem + w * R + acol,
+                   smem_desc(z_addr + kk * 16 * RB, M * RB, 8 * RB, SW), idY, kk > 0);
+          }
+          mma_commit(&y_full[w]);
+          return true;
+        };
+        auto issue_dZ = [&](int64_t i) -> bool {
+          const int w = (int)(i & 1);
+          const int64_t j = i >> 1;
+          const int s = (int)(i % kAStages);
+          if (!mbar_wait_sleep(&a_done[w], (uint32_t)(j & 1))) return false;
+          tc_fence_after();
+          const uint32_t pa = p0 + w * L::PBUF;
+          const uint32_t dy_addr = st0 + s * 2 * L::TILE + L::TILE;
+#pragma unroll
+          for (int kk = 0; kk < kT / 16; ++kk)
+            mma_ss(tmem + TDZ, smem_desc(pa + kk * kMnKStep, kMnLbo, kMnSbo, kSw128),
+                   smem_desc(dy_addr + kk * 16 * RB, L::TILE, 8 * RB, SW), idZ,
+                   (i > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&st_empty[s]);
+          return true;
+        };
+        if (ok && ntiles > 0) ok = issue_S(0);
+        if (ok && ntiles > 1) ok = issue_S(1);
+        for (int64_t i = 0; ok && i < ntiles; ++i) {
+          ok = issue_Y(i);
+          if (ok) ok = issue_dZ(i);
+          // the warpgroup's columns are free (a_done) and, by issue order,
+          // the dZ MMA that reads its P buffer completes before this S does
+          if (ok && i + 2 < ntiles) ok = issue_S(i + 2);
+          if (*abort_flag) ok = false;
+        }
+        if (!ok) {
+          record_error(err, kErrBwdAMmaWait);
+          *abort_flag = 1;
+        }
+        mma_commit(dz_final);
+        mma_commit(drain);
+        mbar_wait_sleep(drain, 0);
+      }
+    }
+  } else {
+    regs_acquire<kRegsRow>();
+    const int w = warp >> 2, qw = warp & 3;
+    const int r = qw * 32 + lane;                    // TMEM lane = token row of the tile
+    const uint32_t lb = (uint32_t)(qw * 32) << 16;
+    const uint32_t tR = tmem + lb + w * R;
+    uint8_t* pbuf = smem + L::P_OFF + w * L::PBUF;
+    const int64_t nW = (ntiles - w + 1) / 2;
+    bool ok = true;
+    for (int64_t j = 0; j < nW; ++j) {
+      const int64_t i = 2 * j + w;
+      const int s = (int)(i % kAStages);
+      const int64_t tok = (tile0 + i) * kT + r;
+      if (!warp_all(mbar_wait_sleep(&s_full[w], (uint32_t)(j & 1)) && !*abort_flag)) {
+        ok = false;
+        break;
+      }
+      __syncwarp();
+      tc_fence_after();
+      // pass 1: row max over the M logits (32-column chunks, double-buffered loads)
+      constexpr int NC = M / 32;
+      uint32_t a[2][32];
+      float mf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      tmem_ld32(tR, a[0]);
+#pragma unroll
+      for (int cc = 0; cc < NC; ++cc) {
+        tmem_wait_ld_dep(a[cc & 1]);
+        if (cc + 1 < NC) tmem_ld32(tR + 32 * (cc + 1), a[(cc + 1) & 1]);
+        max_fold32(a[cc & 1], mf);
+      }
+      const float mx = fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3]));
+      const float neg = -mx * c;
+      float sf[4] = {0.f, 0.f, 0.f, 0.f};
+      // pass 2: P = 2^(c S - c mx) as bf16 pairs.  TMEM copy for Y = P Z,
+      // placed as in the forward's decode (upper-half chunks last-first so
+      // no store lands on a chunk still to be read); shared-memory copy for
+      // dZ += P^T dY'.
+      auto chunk_col = [](int k) { return k < NC / 2 ? M / 2 + 32 * (NC / 2 - 1 - k) : 32 * (k - NC / 2); };
+      auto p_col = [](int k) { return k < NC / 2 ? 3 * M / 4 + 16 * (NC / 2 - 1 - k) : 16 * (k - NC / 2); };
+      tmem_ld32(tR + chunk_col(0), a[0]);
+#pragma unroll
+      for (int k = 0; k < NC; ++k) {
+        tmem_wait_ld_dep(a[k & 1]);
+        if (k + 1 < NC) tmem_ld32(tR + chunk_col(k + 1), a[(k + 1) & 1]);
+        uint32_t pk[16];
+        exp_pack32<0>(a[k & 1], c, neg, pk, sf);
+        tmem_st16(tR + p_col(k), pk);
+        const int g0 = chunk_col(k) >> 3;
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          *reinterpret_cast<uint4*>(pbuf + mn_off(r, g0 + v)) =
+              make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[w]);
+      // Y = P Z (unnormalised); delta_d = dY . Y / l; dY' = dY / l in place
+      if (!warp_all(mbar_wait_sleep(&y_full[w], (uint32_t)(j & 1)) &&
+                    mbar_wait(&st_full[s], (uint32_t)((i / kAStages) & 1)))) {
+        ok = false;
+        break;
+      }
+      __syncwarp();
+      tc_fence_after();
+      float y[D];
+      float lb;   // row sum of the bf16 P (the weights the tensor cores used)
+      if (D == 32) {
+        uint32_t o[32], o2[16];
+        tmem_ld32(tR + TY, o);
+        tmem_ld16(tR + TY + 32, o2);
+        tmem_wait_ld_dep(o);
+        reg_fence16(o2);
+#pragma unroll
+        for (int d = 0; d < D; ++d) y[d] = __uint_as_float(o[d]);
+        lb = __uint_as_float(o2[0]);
+      } else {
+        uint32_t o[32];
+        tmem_ld32(tR + TY, o);
+        tmem_wait_ld_dep(o);
+#pragma unroll
+        for (int d = 0; d < D; ++d) y[d] = __uint_as_float(o[d]);
+        lb = __uint_as_float(o[D]);
+      }
+      const float l = (sf[0] + sf[1]) + (sf[2] + sf[3]);
+      const float inv = 1.f / lb;
+      uint8_t* dyt = smem + L::ST_OFF + s * 2 * L::TILE + L::TILE;
+      float dot = 0.f;
+#pragma unroll
+      for (int ch = 0; ch < D / 8; ++ch) {
+        uint4* p = reinterpret_cast<uint4*>(dyt + tma_row_chunk<D>(r, ch));
+        uint4 u = *p;
+        const float* yy = y + 8 * ch;
+        dot = fmaf(bf_lo(u.x), yy[0], dot);
+        dot = fmaf(bf_hi(u.x), yy[1], dot);
+        dot = fmaf(bf_lo(u.y), yy[2], dot);
+        dot = fmaf(bf_hi(u.y), yy[3], dot);
+        dot = fmaf(bf_lo(u.z), yy[4], dot);
+        dot = fmaf(bf_hi(u.z), yy[5], dot);
+        dot = fmaf(bf_lo(u.w), yy[6], dot);
+        dot = fmaf(bf_hi(u.w), yy[7], dot);
+        u.x = pack_bf16(bf_lo(u.x) * inv, bf_hi(u.x) * inv);
+        u.y = pack_bf16(bf_lo(u.y) * inv, bf_hi(u.y) * inv);
+        u.z = pack_bf16(bf_lo(u.z) * inv, bf_hi(u.z) * inv);
+        u.w = pack_bf16(bf_lo(u.w) * inv, bf_hi(u.w) * inv);
+        *p = u;
+      }
+      if (tok < N) stats[bh * N + tok] = make_float2(fmaf(mx, c, log2f(l)), dot * inv);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&a_done[w]);
+    }
+    if (!ok) {
+      record_error(err, kErrBwdARowWait);
+      *abort_flag = 1;
+    }
+    // dZ partial of this chunk: warpgroup 0, thread r = latent r
+    if (w == 0) {
+      float acc[D];
+#pragma unroll
+      for (int d = 0; d < D; ++d) acc[d] = 0.f;
+      if (ok && ntiles > 0) {
+        ok = warp_all(mbar_wait_sleep(dz_final, 0));
+        __syncwarp();
+        tc_fence_after();
+        if (ok) {
+          if (D == 32) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lb + TDZ, o);
+            tmem_wait_ld_dep(o);
+#pragma unroll
+            for (int d = 0; d < D; ++d) acc[d] = __uint_as_float(o[d]);
+          } else {
+            uint32_t o[16];
+            tmem_ld16(tmem + lb + TDZ, o);
+            tmem_wait_ld_dep16(o);
+#pragma unroll
+            for (int d = 0; d < D; ++d) acc[d] = __uint_as_float(o[d & 15]);
+          }
+        } else {
+          record_error(err, kErrBwdARowWait);
+          *abort_flag = 1;
+        }
+      }
+      float4* dst = reinterpret_cast<float4*>(dz_part + (((int64_t)bh * chunks + chunk) * M + r) * D);
+#pragma unroll
+      for (int d = 0; d < D / 4; ++d)
+        dst[d] = make_float4(acc[4 * d], acc[4 * d + 1], acc[4 * d + 2], acc[4 * d + 3]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kWMma) tmem_dealloc(tmem, NCOLS);
+}
+
+// ======================================================= between passes
+
+// Z (float) -> bf16 copy, the operand of Y = P Z and dPd = dY Z^T.
+__global__ void bwd_zbf16_kernel(const float4* __restrict__ z, uint2* __restrict__ zb, int64_t n4) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  const float4 v = z[i];
+  zb[i] = make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
+}
+
+// One block per (b, h), one thread per latent m.  dZ = sum of the chunk
+// partials (fixed order), lse2 = lse log2(e); R = max lse2 over the head;
+// f = 2^(R - lse2) when the head's lse2 spread is at most kSpreadMax (else
+// f = 1 and the exact form); the bf16 operand dZ'' = f dZ; the extra K-step
+// row: -dZ'' . Z (= -f delta_e) as three bf16 terms, then zeros.
+template <int D>
+__global__ void __launch_bounds__(kM)
+    bwd_mid_kernel(const float* __restrict__ dz_part, int chunks, const float* __restrict__ Z,
+                   const float* __restrict__ lse, __nv_bfloat16* __restrict__ dzs,
+                   uint32_t* __restrict__ aug, float2* __restrict__ params,
+                   float* __restrict__ lse2_out) {
+  __shared__ float red_max[kM / 32], red_min[kM / 32];
+  const int64_t bh = blockIdx.x;
+  const int m = threadIdx.x;
+  const int64_t row = bh * kM + m;
+  float dz[D];
+#pragma unroll
+  for (int d = 0; d < D; ++d) dz[d] = 0.f;
+  for (int k = 0; k < chunks; ++k) {
+    const float4* p = reinterpret_cast<const float4*>(dz_part + ((bh * chunks + k) * kM + m) * D);
+#pragma unroll
+    for (int d = 0; d < D / 4; ++d) {
+      const float4 v = p[d];
+      dz[4 * d] += v.x;
+      dz[4 * d + 1] += v.y;
+      dz[4 * d + 2] += v.z;
+      dz[4 * d + 3] += v.w;
+    }
+  }
+  const float l2 = lse[row] * kLog2e;
+  float mx = l2, mn = l2;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+  }
+  if ((m & 31) == 0) {
+    red_max[m >> 5] = mx;
+    red_min[m >> 5] = mn;
+  }
+  __syncthreads();
+  float R = red_max[0], lo = red_min[0];
+#pragma unroll
+  for (int k = 1; k < kM / 32; ++k) {
+    R = fmaxf(R, red_max[k]);
+    lo = fminf(lo, red_min[k]);
+  }
+  const bool fast = (R - lo) <= kSpreadMax;
+  const float f = fast ? exp2f(R - l2) : 1.f;
+  // delta_e is taken with the bf16 operand dZ'' that the tensor cores use,
+  // so dPe'' = V dZ''^T - dZ'' . Z vanishes exactly where V = Z.
+  float de = 0.f;
+#pragma unroll
+  for (int d = 0; d < D; d += 2) {
+    const uint32_t pr = pack_bf16(f * dz[d], f * dz[d + 1]);
+    *reinterpret_cast<uint32_t*>(dzs + row * D + d) = pr;
+    de = fmaf(bf_lo(pr), Z[row * D + d], de);
+    de = fmaf(bf_hi(pr), Z[row * D + d + 1], de);
+  }
+  const float x = -de;
+  const __nv_bfloat16 b0 = __float2bfloat16_rn(x);
+  const float r1 = x - __bfloat162float(b0);
+  const __nv_bfloat16 b1 = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(b1);
+  const __nv_bfloat16 b2 = __float2bfloat16_rn(r2);
+  uint32_t* a = aug + row * 8;   // 16 bf16
+  a[0] = (uint32_t)__bfloat16_as_ushort(b0) | ((uint32_t)__bfloat16_as_ushort(b1) << 16);
+  a[1] = (uint32_t)__bfloat16_as_ushort(b2);
+#pragma unroll
+  for (int k = 2; k < 8; ++k) a[k] = 0u;
+  lse2_out[row] = l2;
+  if (m == 0) params[bh] = make_float2(R, fast ? 1.f : 0.f);
+}
+
+// ============================================================== pass B
+
+template <int D>
+struct BLayout {
+  static constexpr int M = kM;
+  static constexpr int NQ = M / 32;           // latent quarters per tile
+  static constexpr int RB = 2 * D;
+  static constexpr int TILE = kT * RB;
+  static constexpr int GBUF = kT * M * 2;     // one G tile, MN-major
+  static constexpr int G_OFF = 0;             // two G buffers (tile parity)
+  static constexpr int Q_OFF = 2 * GBUF;
+  static constexpr int Z_OFF = Q_OFF + M * RB;
+  static constexpr int DZ_OFF = Z_OFF + M * RB;
+  static constexpr int AUG_OFF = DZ_OFF + M * RB;     // [M][16] bf16, 32-byte rows
+  static constexpr int ONES_OFF = AUG_OFF + M * 32;   // [128][16] bf16
+  static constexpr int ST_OFF = ONES_OFF + kT * 32;   // stages: K, V, dY tiles
+  static constexpr int LSE_OFF = ST_OFF + kBStages * 3 * TILE;
+  static constexpr int BAR_OFF = LSE_OFF + M * 4;
+  static constexpr int NBARS = 2 * kBStages + 1 + 12 + 4;
+  static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+  static constexpr int BYTES = MISC_OFF + 16;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThr, 1)
+    tc_bwd_b_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdY,
+                    const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmDZ,
+                    const __grid_constant__ CUtensorMap tmAug, int H, int64_t N, int q_per_batch,
+                    float c, float s, int64_t tiles_per_bh, int64_t chunk_tiles,
+                    const float2* __restrict__ stats, const float2* __restrict__ params,
+                    const float* __restrict__ lse2, __nv_bfloat16* __restrict__ dK,
+                    __nv_bfloat16* __restrict__ dV, float* __restrict__ dq_part,
+                    uint32_t* __restrict__ err) {
+  using L = BLayout<D>;
+  constexpr int M = L::M;
+  constexpr int NQ = L::NQ;
+  constexpr int RB = L::RB;
+  constexpr uint32_t SW = umma_swizzle_code(RB);
+  constexpr int QC = 96;          // TMEM columns of one quarter: S | dPd | dPe''
+  constexpr int TDK = 4 * QC;     // dK accumulator (token lanes)
+  constexpr int TDV = TDK + D;    // dV accumulator (token lanes)
+  constexpr int TDQ = TDV + D;    // dQ accumulator (latent lanes)
+  constexpr uint32_t NCOLS = 512;
+  static_assert(TDQ + D <= 512, "TMEM budget");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* bars = (uint64_t*)(smem + L::BAR_OFF);
+  uint64_t* st_full = bars;
+  uint64_t* st_empty = bars + kBStages;
+  uint64_t* c_full = bars + 2 * kBStages;
+  uint64_t* q_full = c_full + 1;     // [slot] a quarter's S, dPd, dPe'' in TMEM
+  uint64_t* q_done = q_full + 4;     // [slot] G and the dV weights written
+  uint64_t* r_free = q_done + 4;     // [slot] dK/dV MMAs of the quarter complete
+  uint64_t* tile_done = r_free + 4;  // dK/dV of a tile final, dQ MMA of the tile complete
+  uint64_t* acc_empty = tile_done + 1;
+  uint64_t* dq_final = acc_empty + 1;
+  uint64_t* drain = dq_final + 1;
+  uint32_t* tmem_slot = (uint32_t*)(smem + L::MISC_OFF);
+  volatile int* abort_flag = (volatile int*)(smem + L::MISC_OFF + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x, chunks = gridDim.x;
+  const int64_t bh = blockIdx.y;
+  const int64_t h = bh % H;
+  const int64_t tile0 = (int64_t)chunk * chunk_tiles;
+  const int64_t ntiles = imin64(chunk_tiles, tiles_per_bh - tile0);
+  const int64_t KQ = ntiles * NQ;   // quarters of this chunk
+
+  // the constant A operand of the extra K-step: ones in columns 0-2 of
+  // every row, 32-byte swizzle (row t at 32 t, 16-byte chunk x at x ^ bit 2 of t)
+  {
+    uint8_t* ones = smem + L::ONES_OFF;
+    for (int t = threadIdx.x; t < kT; t += blockDim.x) {
+      const uint4 one3 = make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u);
+      const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+      const int x0 = 0 ^ ((t >> 2) & 1), x1 = 1 ^ ((t >> 2) & 1);
+      *reinterpret_cast<uint4*>(ones + t * 32 + x0 * 16) = one3;
+      *reinterpret_cast<uint4*>(ones + t * 32 + x1 * 16) = zero;
+    }
+    float* ls = (float*)(smem + L::LSE_OFF);
+    for (int m = threadIdx.x; m < M; m += blockDim.x) ls[m] = lse2[bh * M + m];
+  }
+  fence_proxy_async_smem();
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < kBStages; ++k) {
+      mbar_init(&st_full[k], 1);
+      mbar_init(&st_empty[k], 1);
+    }
+    mbar_init(c_full, 1);
+    for (int k = 0; k < 4; ++k) {
+      mbar_init(&q_full[k], 1);
+      mbar_init(&q_done[k], 128);
+      mbar_init(&r_free[k], 1);
+    }
+    mbar_init(tile_done, 1);
+    mbar_init(acc_empty, 256);
+    mbar_init(dq_final, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kWMma) tmem_alloc(tmem_slot, NCOLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // slot of quarter k: warpgroup k & 1, and each warpgroup alternates two slots
+  auto slot_of = [](int64_t k) { return (int)(((k & 1) << 1) | ((k >> 1) & 1)); };
+
+  if (warp >= 8) {
+    regs_release<kRegsPro>();
+    if (warp == kWTma) {
+      if (lane == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        prefetch_tmap(&tmdY);
+        prefetch_tmap(&tmZ);
+        prefetch_tmap(&tmDZ);
+        prefetch_tmap(&tmAug);
+        mbar_arrive_expect_tx(c_full, 3 * M * RB + M * 32);
+        tma_load_3d(smem + L::Q_OFF, &tmQ, c_full, 0, 0, (int32_t)(q_per_batch ? bh : h));
+        tma_load_3d(smem + L::Z_OFF, &tmZ, c_full, 0, 0, (int32_t)bh);
+        tma_load_3d(smem + L::DZ_OFF, &tmDZ, c_full, 0, 0, (int32_t)bh);
+        tma_load_3d(smem + L::AUG_OFF, &tmAug, c_full, 0, 0, (int32_t)bh);
+        int64_t issued = 0;
+        for (int64_t t = 0; t < ntiles; ++t) {
+          const int k = (int)(t % kBStages);
+          const uint32_t ph = (uint32_t)((t / kBStages) & 1);
+          if (t >= kBStages && !mbar_wait_sleep(&st_empty[k], ph ^ 1)) {
+            record_error(err, kErrBwdBTmaWait);
+            *abort_flag = 1;
+            break;
+          }
+          if (*abort_flag) break;
+          uint8_t* dst = smem + L::ST_OFF + k * 3 * L::TILE;
+          mbar_arrive_expect_tx(&st_full[k], 3 * L::TILE);
+          const int32_t tok = (int32_t)((tile0 + t) * kT);
+          tma_load_3d(dst, &tmK, &st_full[k], 0, tok, (int32_t)bh);
+          tma_load_3d(dst + L::TILE, &tmV, &st_full[k], 0, tok, (int32_t)bh);
+          tma_load_3d(dst + 2 * L::TILE, &tmdY, &st_full[k], 0, tok, (int32_t)bh);
+          issued = t + 1;
+        }
+        for (int64_t t = (issued > kBStages ? issued - kBStages : 0); t < issued; ++t)
+          mbar_wait_sleep(&st_full[t % kBStages], (uint32_t)((t / kBStages) & 1));
+        mbar_wait_sleep(c_full, 0);
+      }
+    } else if (warp == kWMma) {
+      if (lane == 0) {
+        constexpr uint32_t idL = idesc_bf16_f32(128, 32, 0, 0);   // quarter logits
+        constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);    // dK, dV (A in TMEM)
+        constexpr uint32_t idQ = idesc_bf16_f32(128, D, 1, 1);    // dQ (A MN-major)
+        const uint32_t q_addr = smem_u32(smem + L::Q_OFF);
+        const uint32_t z_addr = smem_u32(smem + L::Z_OFF);
+        const uint32_t dz_addr = smem_u32(smem + L::DZ_OFF);
+        const uint32_t aug_addr = smem_u32(smem + L::AUG_OFF);
+        const uint32_t ones_addr = smem_u32(smem + L::ONES_OFF);
+        const uint32_t st0 = smem_u32(smem + L::ST_OFF);
+        const uint32_t g0 = smem_u32(smem + L::G_OFF);
+        bool ok = mbar_wait_sleep(c_full, 0);
+        auto issue_L = [&](int64_t k) -> bool {
+          const int64_t t = k / NQ;
+          const int qq = (int)(k % NQ);
+          const int st = (int)(t % kBStages);
+          if (qq == 0 && !mbar_wait_sleep(&st_full[st], (uint32_t)((t / kBStages) & 1)))
+            return false;
+          tc_fence_after();
+          const uint32_t base = tmem + QC * slot_of(k);
+          const uint32_t k_addr = st0 + st * 3 * L::TILE;
+          const uint32_t v_addr = k_addr + L::TILE;
+          const uint32_t dy_addr = k_addr + 2 * L::TILE;
+          const uint32_t roff = (uint32_t)(32 * qq * RB);   // latent rows [32 qq, 32 qq + 32)
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(base, smem_desc(k_addr + 32 * kk, 16, 8 * RB, SW),
+                   smem_desc(q_addr + roff + 32 * kk, 16, 8 * RB, SW), idL, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(base + 32, smem_desc(dy_addr + 32 * kk, 16, 8 * RB, SW),
+                   smem_desc(z_addr + roff + 32 * kk, 16, 8 * RB, SW), idL, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(base + 64, smem_desc(v_addr + 32 * kk, 16, 8 * RB, SW),
+                   smem_desc(dz_addr + roff + 32 * kk, 16, 8 * RB, SW), idL, kk > 0);
+          mma_ss(base + 64, smem_desc(ones_addr, 16, 256, kSw32),
+                 smem_desc(aug_addr + 32 * qq * 32, 16, 256, kSw32), idL, 1u);
+          mma_commit(&q_full[slot_of(k)]);
+          return true;
+        };
+        for (int64_t k = 0; ok && k < 4 && k < KQ; ++k) ok = issue_L(k);
+        for (int64_t k = 0; ok && k < KQ; ++k) {
+          const int slot = slot_of(k);
+          const int64_t t = k / NQ;
+          const int qq = (int)(k % NQ);
+          const uint32_t use = (uint32_t)((k >> 2) & 1);
+          if (!mbar_wait_sleep(&q_done[slot], use)) {
+            ok = false;
+            break;
+          }
+          if (qq == 0 && t > 0 && !mbar_wait_sleep(acc_empty, (uint32_t)((t - 1) & 1))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t base = tmem + QC * slot;
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            const uint32_t rows = (uint32_t)((32 * qq + 16 * kk) * RB);
+            const uint32_t acc = (qq > 0 || kk > 0) ? 1u : 0u;
+            mma_ts(tmem + TDK, base + 8 * kk, smem_desc(q_addr + rows, M * RB, 8 * RB, SW), idO,
+                   acc);
+            mma_ts(tmem + TDV, base + 32 + 8 * kk, smem_desc(dz_addr + rows, M * RB, 8 * RB, SW),
+                   idO, acc);
+          }
+          mma_commit(&r_free[slot]);
+          if (qq == NQ - 1) {
+            const int st = (int)(t % kBStages);
+            const uint32_t gb = g0 + (uint32_t)((t & 1) * L::GBUF);
+            const uint32_t k_addr = st0 + st * 3 * L::TILE;
+#pragma unroll
+            for (int kk = 0; kk < kT / 16; ++kk)
+              mma_ss(tmem + TDQ, smem_desc(gb + kk * kMnKStep, kMnLbo, kMnSbo, kSw128),
+                     smem_desc(k_addr + kk * 16 * RB, L::TILE, 8 * RB, SW), idQ,
+                     (t > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(tile_done);
+            mma_commit(&st_empty[st]);
+          }
+          if (k + 4 < KQ) {
+            if (!mbar_wait_sleep(&r_free[slot], use)) {
+              ok = false;
+              break;
+            }
+            if (!(ok = issue_L(k + 4))) break;
+          }
+          if (*abort_flag) ok = false;
+        }
+        if (!ok) {
+          record_error(err, kErrBwdBMmaWait);
+          *abort_flag = 1;
+        }
+        mma_commit(dq_final);
+        mma_commit(drain);
+        mbar_wait_sleep(drain, 0);
+      }
+    }
+  } else {
+    regs_acquire<kRegsRow>();
+    const int w = warp >> 2, qw = warp & 3;
+    const int r = qw * 32 + lane;                    // TMEM lane = token row of the tile
+    const uint32_t lb = (uint32_t)(qw * 32) << 16;
+    const float2 prm = params[bh];
+    const float Rref = prm.x;
+    const bool fast = prm.y != 0.f;
+    const float* ls = (const float*)(smem + L::LSE_OFF);
+    const uint64_t c2 = f32x2(c, c);
+    float mxp = 0.f, dd = 0.f, g = 0.f, gprev = 0.f;
+    bool valid = false;
+    bool ok = true;
+
+    // dK (warpgroup 0) or dV (warpgroup 1) of tile tt: wait for the tile's
+    // accumulators, release them, scale and store the rows.
+    auto finish = [&](int64_t tt, float gv) -> bool {
+      if (!warp_all(mbar_wait_sleep(tile_done, (uint32_t)(tt & 1)) && !*abort_flag)) return false;
+      __syncwarp();
+      tc_fence_after();
+      float o[D];
+      if (D == 32) {
+        uint32_t u[32];
+        tmem_ld32(tmem + lb + (w == 0 ? TDK : TDV), u);
+        tmem_wait_ld_dep(u);
+#pragma unroll
+        for (int d = 0; d < D; ++d) o[d] = __uint_as_float(u[d]);
+      } else {
+        uint32_t u[16];
+        tmem_ld16(tmem + lb + (w == 0 ? TDK : TDV), u);
+        tmem_wait_ld_dep16(u);
+#pragma unroll
+        for (int d = 0; d < D; ++d) o[d] = __uint_as_float(u[d & 15]);
+      }
+      tc_fence_before();
+      mbar_arrive(acc_empty);
+      const int64_t tok = (tile0 + tt) * kT + r;
+      if (tok < N) {
+        const float f = (w == 0) ? s : gv;
+        uint4* dst = reinterpret_cast<uint4*>((w == 0 ? dK : dV) + (bh * N + tok) * D);
+#pragma unroll
+        for (int v = 0; v < D / 8; ++v)
+          dst[v] = make_uint4(pack_bf16(o[8 * v] * f, o[8 * v + 1] * f),
+                              pack_bf16(o[8 * v + 2] * f, o[8 * v + 3] * f),
+                              pack_bf16(o[8 * v + 4] * f, o[8 * v + 5] * f),
+                              pack_bf16(o[8 * v + 6] * f, o[8 * v + 7] * f));
+      }
+      return true;
+    };
+
+    for (int64_t k = w; k < KQ; k += 2) {
+      const int64_t t = k / NQ;
+      const int qq = (int)(k % NQ);
+      const int slot = slot_of(k);
+      if (qq == w) {   // this warpgroup's first quarter of tile t: the row's statistics
+        gprev = g;
+        const int64_t tok = (tile0 + t) * kT + r;
+        valid = tok < N;
+        if (valid) {
+          const float2 st = stats[bh * N + tok];
+          mxp = st.x;
+          dd = st.y;
+          g = fast ? exp2f(mxp - Rref) : 1.f;
+        } else {
+          mxp = 0.f;
+          dd = 0.f;
+          g = 0.f;
+        }
+      }
+      if (!warp_all(mbar_wait_sleep(&q_full[slot], (uint32_t)((k >> 2) & 1)) && !*abort_flag)) {
+        ok = false;
+        break;
+      }
+      __syncwarp();
+      tc_fence_after();
+      const uint32_t tq = tmem + lb + QC * slot;
+      uint8_t* gsm = smem + L::G_OFF + (t & 1) * L::GBUF;
+      const uint64_t nm2 = f32x2(-mxp, -mxp), nd2 = f32x2(-dd, -dd), g2 = f32x2(g, g);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t a[16], b[16], e[16];
+        tmem_ld16(tq + 16 * hh, a);
+        tmem_ld16(tq + 32 + 16 * hh, b);
+        tmem_ld16(tq + 64 + 16 * hh, e);
+        tmem_wait_ld_dep16(a);
+        reg_fence16(b);
+        reg_fence16(e);
+        uint32_t gk[8], vk[8];
+        const int m0 = 32 * qq + 16 * hh;
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+          const uint64_t S2 = f32x2(__uint_as_float(a[2 * p]), __uint_as_float(a[2 * p + 1]));
+          const uint64_t P2 = f32x2(__uint_as_float(b[2 * p]), __uint_as_float(b[2 * p + 1]));
+          const uint64_t E2 = f32x2(__uint_as_float(e[2 * p]), __uint_as_float(e[2 * p + 1]));
+          float x0, x1;
+          split_f32x2(fma_f32x2(S2, c2, nm2), x0, x1);
+          const float p0 = ex2(x0), p1 = ex2(x1);
+          float g0v, g1v, w0, w1;
+          if (fast) {
+            // G = P_d (dPd - delta_d + g dPe'');  dV weights P_d
+            split_f32x2(mul_f32x2(f32x2(p0, p1), add_f32x2(fma_f32x2(E2, g2, P2), nd2)), g0v,
+                        g1v);
+            w0 = p0;
+            w1 = p1;
+          } else {
+            // exact form: P_e = 2^(c S - lse2[m]); G = P_d (dPd - delta_d) + P_e dPe'
+            float s0, s1, e0, e1;
+            split_f32x2(S2, s0, s1);
+            split_f32x2(E2, e0, e1);
+            w0 = valid ? ex2(fmaf(s0, c, -ls[m0 + 2 * p])) : 0.f;
+            w1 = valid ? ex2(fmaf(s1, c, -ls[m0 + 2 * p + 1])) : 0.f;
+            float d0, d1;
+            split_f32x2(add_f32x2(P2, nd2), d0, d1);
+            g0v = fmaf(w0, e0, p0 * d0);
+            g1v = fmaf(w1, e1, p1 * d1);
+          }
+          gk[p] = pack_bf16(g0v, g1v);
+          vk[p] = pack_bf16(w0, w1);
+        }
+        tmem_st8(tq + 8 * hh, gk);        // over S columns already read
+        tmem_st8(tq + 32 + 8 * hh, vk);   // over dPd columns already read
+        const int grp = m0 >> 3;
+        *reinterpret_cast<uint4*>(gsm + mn_off(r, grp)) = make_uint4(gk[0], gk[1], gk[2], gk[3]);
+        *reinterpret_cast<uint4*>(gsm + mn_off(r, grp + 1)) = make_uint4(gk[4], gk[5], gk[6], gk[7]);
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&q_done[slot]);
+      if (qq == w && t > 0 && !(ok = finish(t - 1, gprev))) break;
+    }
+    if (ok && KQ > 0) ok = finish(ntiles - 1, g);
+    if (!ok) {
+      record_error(err, kErrBwdBRowWait);
+      *abort_flag = 1;
+    }
+    // dQ partial of this chunk (scaled): warpgroup 0, thread r = latent r
+    if (w == 0) {
+      float acc[D];
+#pragma unroll
+      for (int d = 0; d < D; ++d) acc[d] = 0.f;
+      if (ok && KQ > 0) {
+        ok = warp_all(mbar_wait_sleep(dq_final, 0));
+        __syncwarp();
+        tc_fence_after();
+        if (ok) {
+          if (D == 32) {
+            uint32_t u[32];
+            tmem_ld32(tmem + lb + TDQ, u);
+            tmem_wait_ld_dep(u);
+#pragma unroll
+            for (int d = 0; d < D; ++d) acc[d] = __uint_as_float(u[d]) * s;
+          } else {
+            uint32_t u[16];
+            tmem_ld16(tmem + lb + TDQ, u);
+            tmem_wait_ld_dep16(u);
+#pragma unroll
+            for (int d = 0; d < D; ++d) acc[d] = __uint_as_float(u[d & 15]) * s;
+          }
+        } else {
+          record_error(err, kErrBwdBRowWait);
+          *abort_flag = 1;
+        }
+      }
+      float4* dst = reinterpret_cast<float4*>(dq_part + (((int64_t)bh * chunks + chunk) * M + r) * D);
+#pragma unroll
+      for (int d = 0; d < D / 4; ++d)
+        dst[d] = make_float4(acc[4 * d], acc[4 * d + 1], acc[4 * d + 2], acc[4 * d + 3]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kWMma) tmem_dealloc(tmem, NCOLS);
+}
+
+// dQ = sum over (batch when Q is shared) x chunks of the scaled partials,
+// in a fixed order.  One thread per output element.
+__global__ void bwd_dq_sum_kernel(const float* __restrict__ dq_part, int B, int H, int M, int D,
+                                  int chunks, bool shared_q, __nv_bfloat16* __restrict__ dQ) {
+  const int64_t per = (int64_t)H * M * D;
+  const int64_t total = shared_q ? per : (int64_t)B * per;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= total) return;
+  const int64_t b0 = shared_q ? 0 : i / per;
+  const int64_t b1 = shared_q ? B : b0 + 1;
+  const int64_t rr = i % per;
+  const int64_t h = rr / ((int64_t)M * D);
+  const int64_t md = rr % ((int64_t)M * D);
+  float acc = 0.f;
+  for (int64_t b = b0; b < b1; ++b) {
+    const int64_t bh = b * H + h;
+    for (int k = 0; k < chunks; ++k) acc += dq_part[(bh * chunks + k) * (int64_t)M * D + md];
+  }
+  dQ[i] = __float2bfloat16_rn(acc);
+}
+
+template <int D>
+cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, const void* dY,
+                     const float* Z, const float* lse, void* dQ, void* dK, void* dV, const Dims& d,
+                     float scale, const WsLayout& L, char* ws, cudaStream_t st) {
+  const ChunkPlan& p = L.bwd;
+  const int64_t BH = d.BH();
+  const int q_per_batch = qbs != 0;
+  const float c = scale * kLog2e;
+  uint32_t* err = (uint32_t*)(ws + L.hdr);
+  __nv_bfloat16* zb = (__nv_bfloat16*)(ws + L.zb);
+  float2* stats = (float2*)(ws + L.stats);
+  float* dzp = (float*)(ws + L.dzp);
+  __nv_bfloat16* dzs = (__nv_bfloat16*)(ws + L.dzs);
+  __nv_bfloat16* aug = (__nv_bfloat16*)(ws + L.aug);
+  float2* params = (float2*)(ws + L.params);
+  float* lse2 = (float*)(ws + L.lse2);
+  float* dqp = (float*)(ws + L.dqp);
+  cudaError_t e;
+
+  const int64_t n4 = BH * kM * D / 4;
+  bwd_zbf16_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>((const float4*)Z, (uint2*)zb, n4);
+  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+
+  CUtensorMap mq, mk, mv, mdy, mz, mdz, maug;
+  if ((e = make_map(&mq, Q, D, kM, q_per_batch ? BH : d.H, kM)) != cudaSuccess) return e;
+  if ((e = make_map(&mk, K, D, d.N, BH, kT)) != cudaSuccess) return e;
+  if ((e = make_map(&mv, V, D, d.N, BH, kT)) != cudaSuccess) return e;
+  if ((e = make_map(&mdy, dY, D, d.N, BH, kT)) != cudaSuccess) return e;
+  if ((e = make_map(&mz, zb, D, kM, BH, kM)) != cudaSuccess) return e;
+  if ((e = make_map(&mdz, dzs, D, kM, BH, kM)) != cudaSuccess) return e;
+  if ((e = make_map(&maug, aug, 16, kM, BH, kM)) != cudaSuccess) return e;
+
+  dim3 grid(p.chunks, (unsigned)BH);
+  const int smemA = ALayout<D>::BYTES + 1024;
+  e = cudaFuncSetAttribute(tc_bwd_a_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemA);
+  if (e != cudaSuccess) return e;
+  tc_bwd_a_kernel<D><<<grid, kThr, smemA, st>>>(mq, mk, mdy, mz, (int)d.H, d.N, q_per_batch, c,
+                                                p.tiles_per_bh, p.chunk_tiles, stats, dzp, err);
+  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+
+  bwd_mid_kernel<D><<<(unsigned)BH, kM, 0, st>>>(dzp, p.chunks, Z, lse, dzs, (uint32_t*)aug,
+                                                 params, lse2);
+  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+
+  const int smemB = BLayout<D>::BYTES + 1024;
+  e = cudaFuncSetAttribute(tc_bwd_b_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemB);
+  if (e != cudaSuccess) return e;
+  tc_bwd_b_kernel<D><<<grid, kThr, smemB, st>>>(
+      mq, mk, mv, mdy, mz, mdz, maug, (int)d.H, d.N, q_per_batch, c, scale, p.tiles_per_bh,
+      p.chunk_tiles, stats, params, lse2, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, dqp, err);
+  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+
+  const bool shared_q = (qbs == 0);
+  const int64_t total = shared_q ? d.H * kM * D : BH * kM * D;
+  bwd_dq_sum_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
+      dqp, (int)d.B, (int)d.H, kM, D, p.chunks, shared_q, (__nv_bfloat16*)dQ);
+  return cudaPeekAtLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_tc_bwd(const void* Q, int64_t qbs, const void* K, const void* V,
+                          const void* dY, const float* Z, const float* lse, void* dQ, void* dK,
+                          void* dV, const Dims& d, float scale, const WsLayout& L, char* ws,
+                          cudaStream_t st) {
+  if (d.M != kM) return cudaErrorNotSupported;
+  if (d.D == 32) return tc_bwd_t<32>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
+  if (d.D == 16) return tc_bwd_t<16>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
+  return cudaErrorNotSupported;
+}
+
+}  // namespace flare

@@ -73,6 +73,12 @@ def fwd_path(B: int, H: int, N: int, M: int, D: int, dtype: torch.dtype) -> int:
     return int(_lib.load().flare_fwd_path(B, H, N, M, D, code))
 
 
+def bwd_path(B: int, H: int, N: int, M: int, D: int, dtype: torch.dtype) -> int:
+    """1 = tcgen05 tensor-core backward, 0 = CUDA-core kernels, -1 = unsupported."""
+    code = _lib.FLARE_F32 if dtype == torch.float32 else _lib.FLARE_BF16
+    return int(_lib.load().flare_bwd_path(B, H, N, M, D, code))
+
+
 def alloc_workspace(op: int, B, H, N, M, D, dtype, device) -> torch.Tensor:
     n = workspace_size(op, B, H, N, M, D, dtype)
     if n == 0:

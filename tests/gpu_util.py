@@ -38,3 +38,17 @@ def assert_close(got, ref, dtype, what="", rel_f32=TOL_F32_REL):
         assert r <= TOL_BF16_REL and m <= TOL_BF16_ABS, \
             f"{what}: rel_fro {r:.3e} (<= {TOL_BF16_REL}), max_abs {m:.3e} (<= {TOL_BF16_ABS})"
     return r
+
+
+def assert_close_scaled(got, ref, what=""):
+    """bf16 parity for outputs that are not of unit scale: relative Frobenius
+    error <= 1e-2 and max-abs error <= 3e-2 x max(1, max |ref|).  A bf16
+    number of magnitude >= 8 has a rounding step of 1/16 or more, so an
+    absolute 3e-2 bound cannot hold for it even after one correct rounding."""
+    r = rel_fro(got, ref)
+    m = max_abs(got, ref)
+    big = float(np.abs(to64(ref)).max()) if to64(ref).size else 0.0
+    bound = TOL_BF16_ABS * max(1.0, big)
+    assert r <= TOL_BF16_REL and m <= bound, \
+        f"{what}: rel_fro {r:.3e} (<= {TOL_BF16_REL}), max_abs {m:.3e} (<= {bound:.3e}, max|ref| {big:.3e})"
+    return r

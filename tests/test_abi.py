@@ -78,7 +78,10 @@ def test_workspace_size(lib):
     ws = lib.flare_workspace_size
     assert ws(0, 1, 16, 1 << 20, 256, 32, 1) > 0
     assert ws(1, 2, 8, 1 << 18, 256, 32, 1) > ws(0, 2, 8, 1 << 18, 256, 32, 1)
-    assert ws(2, 8, 8, 16384, 128, 32, 1) > 8 * 8 * 16384 * 32 * 4  # holds the fp32 dK
+    # the tensor-core backward keeps two floats of statistics per token
+    assert ws(2, 8, 8, 16384, 128, 32, 1) > 8 * 8 * 16384 * 8
+    # the CUDA-core backward (fp32) holds the fp32 decode-stage dK
+    assert ws(2, 8, 8, 16384, 128, 32, 0) > 8 * 8 * 16384 * 32 * 4
     assert ws(0, 1, 1, 1, 16, 16, 0) > 0
     # invalid or unsupported sizes -> 0
     assert ws(0, 0, 1, 100, 16, 16, 0) == 0
@@ -96,6 +99,11 @@ def test_fwd_path_selection(lib):
     assert lib.flare_fwd_path(4, 8, 1 << 16, 128, 16, 1) == 1
     assert lib.flare_fwd_path(1, 4, 1000, 64, 32, 1) == 0         # bf16, M=64 -> CUDA cores
     assert lib.flare_fwd_path(1, 4, 1024, 40, 16, 1) == -1
+    assert lib.flare_bwd_path(8, 8, 16384, 128, 32, 1) == 1      # bf16, M=128 -> tcgen05
+    assert lib.flare_bwd_path(1, 2, 300, 128, 16, 1) == 1
+    assert lib.flare_bwd_path(1, 2, 300, 256, 32, 1) == 0        # bf16, M=256 -> CUDA cores
+    assert lib.flare_bwd_path(1, 2, 300, 128, 32, 0) == 0        # fp32 -> CUDA cores
+    assert lib.flare_bwd_path(1, 2, 300, 40, 32, 1) == -1
 
 
 # ------------------------------------------------ validation before launch ---
