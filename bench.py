@@ -410,7 +410,8 @@ def _row_roofline(t_ms: float, exps: float, flops: float, hbm_bytes: float, peak
                      f"{peaks['bf16_tflops']} TFLOP/s, {peak_kind} HBM {peaks['hbm_gbs']} GB/s"}
 
 
-def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0):
+def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0,
+                    which=("flare_pp_fwd", "flare_fwd_bwd")):
     """Times the FLARE++ forward (B=2 H=8 N=262,144 M=256 D=32) and the
     forward + backward of B=8 H=8 N=16,384 M=128 D=32, both bf16, on the
     same device with CUDA events (median of `iters` launches after 3
@@ -438,6 +439,18 @@ def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0):
         return statistics.median(a.elapsed_time(b) for a, b in pairs)
 
     rows = {}
+    if "flare_pp_fwd" in which:
+        rows.update(_time_pp(dev, peaks, peak_kind, timed, seed))
+    if "flare_fwd_bwd" in which:
+        rows.update(_time_fwd_bwd(dev, peaks, peak_kind, timed, seed))
+    del flush_buf
+    torch.cuda.empty_cache()
+    return rows
+
+
+def _time_pp(dev, peaks, peak_kind, timed, seed):
+    import rank_latent_attention_flare_b200 as fl
+    rows = {}
     w = WORKLOADS["c4_ppfwd_bf16_256k"]
     x = make_inputs(w.B, w.H, w.N, w.M, w.D, dtype=w.torch_dtype, seed=seed)
     g = {k: v.to(dev) for k, v in x.items()}
@@ -451,8 +464,12 @@ def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0):
         "ms": round(ms, 4), "tokens_per_s": w.B * w.N / (ms / 1e3),
         "roofline": _row_roofline(ms, 3.0 * u * w.M, 12.0 * u * w.M * w.D,
                                   6.0 * u * w.D * 2, peaks, peak_kind)}
-    del g, ws
+    return rows
 
+
+def _time_fwd_bwd(dev, peaks, peak_kind, timed, seed):
+    import rank_latent_attention_flare_b200 as fl
+    rows = {}
     w = WORKLOADS["c5_fwdbwd_bf16_16k"]
     x = make_inputs(w.B, w.H, w.N, w.M, w.D, dtype=w.torch_dtype, seed=seed, with_dy=True)
     g = {k: v.to(dev) for k, v in x.items()}
@@ -479,9 +496,20 @@ def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0):
                                   9.0 * u * w.D * 2, peaks, peak_kind),
         "bwd_roofline": _row_roofline(ms_b, 2.0 * u * w.M, 20.0 * u * w.M * w.D,
                                       5.0 * u * w.D * 2, peaks, peak_kind)}
-    del g, wsf, wsb, flush_buf
-    torch.cuda.empty_cache()
     return rows
+
+
+def run_row(args, rank, local):
+    """One of the other workloads alone (FLARE++ forward, or forward +
+    backward), e.g. for a profiler capture."""
+    import torch
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_kind = load_peaks()
+    rows = time_other_rows(dev, peaks, peak_kind, iters=max(1, args.steps), seed=rank,
+                           which=(args.row,))
+    if rank == 0:
+        print(json.dumps({"row": args.row, **rows[args.row]}), flush=True)
 
 
 # ------------------------------------------------------------- reference
@@ -533,6 +561,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true",
                     help="skip the FLARE++ and forward+backward timings")
+    ap.add_argument("--row", choices=["flare_pp_fwd", "flare_fwd_bwd"], default=None,
+                    help="time only this workload (one JSON line with its timing and roofline)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=120.0)
     ap.add_argument("--out-dir", default=None, help="where to write the clock samples")
@@ -545,6 +575,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
+        elif args.row:
+            run_row(args, rank, local)
         else:
             run_ours(args, rank, world, local)
     finally:

@@ -141,7 +141,10 @@ struct WsLayout {
   size_t dz = 0;        // [BH][M][D] float
   size_t delta = 0;     // [BH][M] float  rowsum(dZ * Z)
   // tensor-core backward (the dZ / dQ partials use dzp / dqp, one set each)
-  size_t stats = 0;     // [BH][N] float2  decode log-sum-exp (log2 units), delta_d
+  size_t stats = 0;     // [BH][N] float4  decode log-sum-exp (log2 units), delta_d, delta''
+  size_t dy2 = 0;       // [BH][N][D] bf16  dY / g
+  size_t rref = 0;      // [BH] float  R = max lse2
+  size_t flags = 0;     // [BH] uint32  a token out of the range of the one-exponential form
   size_t dzs = 0;       // [BH][M][D] bf16  f * dZ
   size_t aug = 0;       // [BH][M][16] bf16 extra K-step row (-f delta_e in three terms)
   size_t params = 0;    // [BH] float2  R, fast-form flag
@@ -174,7 +177,10 @@ inline WsLayout ws_layout(flare_op_t op, int64_t B, int64_t H, int64_t N, int64_
   if (op == FLARE_OP_BWD && choose_path(N, M, D, dt).tc_bwd) {
     L.bwd = tc_bwd_plan(BH, N, sms);
     const int64_t bslots = BH * L.bwd.chunks;
-    L.stats = take((size_t)BH * N * 8);
+    L.stats = take((size_t)BH * N * 16);
+    L.dy2 = take((size_t)BH * N * D * 2);
+    L.rref = take((size_t)BH * 4);
+    L.flags = take((size_t)BH * 4);
     L.dzp = take((size_t)bslots * M * D * 4);
     L.dqp = take((size_t)bslots * M * D * 4);
     L.dzs = take((size_t)BH * M * D * 2);

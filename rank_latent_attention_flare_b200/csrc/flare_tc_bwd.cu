@@ -67,7 +67,8 @@ constexpr int kAStages = 4;
 constexpr int kBStages = 3;
 constexpr uint32_t kSw128 = 2u;  // UMMA descriptor code of the 128-byte swizzle
 constexpr uint32_t kSw32 = 6u;   // ... and of the 32-byte swizzle
-constexpr float kSpreadMax = 64.f;  // log2 units: beyond, a head takes the exact form
+constexpr float kSpreadMax = 64.f;     // log2 units: lse spread beyond which a head takes the exact form
+constexpr float kRowRangeMax = 100.f;  // log2 units: a token this far below R flags its head
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return (uint8_t*)(((uintptr_t)p + 1023) & ~(uintptr_t)1023);
@@ -111,9 +112,9 @@ struct ALayout {
   static constexpr int M = kM;
   static constexpr int RB = 2 * D;
   static constexpr int TILE = kT * RB;        // one K or dY tile
-  static constexpr int PBUF = kT * M * 2;     // one P tile, MN-major
-  static constexpr int P_OFF = 0;             // one P buffer per row warpgroup
-  static constexpr int Q_OFF = 2 * PBUF;
+  static constexpr int PBUF = kT * M * 2;     // one P tile (swizzled, latent-contiguous rows)
+  static constexpr int P_OFF = 0;             // two P buffers per row warpgroup
+  static constexpr int Q_OFF = 4 * PBUF;
   static constexpr int Z_OFF = Q_OFF + M * RB;
   static constexpr int ONE_OFF = Z_OFF + M * RB;  // second N block of Y's B operand
   static constexpr int ST_OFF = ONE_OFF + M * RB;   // stages: K tile, dY tile
@@ -128,16 +129,19 @@ __global__ void __launch_bounds__(kThr, 1)
     tc_bwd_a_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmdY, const __grid_constant__ CUtensorMap tmZ,
                     int H, int64_t N, int q_per_batch, float c, int64_t tiles_per_bh,
-                    int64_t chunk_tiles, float2* __restrict__ stats, float* __restrict__ dz_part,
+                    int64_t chunk_tiles, const float* __restrict__ rref,
+                    float4* __restrict__ stats, __nv_bfloat16* __restrict__ dy2,
+                    uint32_t* __restrict__ flags, float* __restrict__ dz_part,
                     uint32_t* __restrict__ err) {
   using L = ALayout<D>;
   constexpr int M = L::M;
   constexpr int RB = L::RB;
   constexpr uint32_t SW = umma_swizzle_code(RB);
-  constexpr int R = M;          // TMEM columns per row warpgroup: S, then P and Y inside
-  constexpr int TY = M / 4;     // [Y | row sum of bf16 P] inside the warpgroup's columns
-  static_assert(TY + D + 16 <= 3 * M / 4, "Y must sit between the two P halves");
-  constexpr int TDZ = 2 * M;    // dZ accumulator (latent lanes)
+  constexpr int R = M;          // TMEM columns of a row warpgroup's S
+  constexpr int TY = 2 * M;     // [Y | row sum of bf16 P] of warpgroup w at TY + YC w
+  constexpr int YC = D + 16;
+  constexpr int TDZ = TY + 2 * YC;   // dZ accumulator (latent lanes)
+  static_assert(TDZ + D <= 512, "TMEM budget");
   constexpr uint32_t NCOLS = 512;
 
   extern __shared__ uint8_t smem_raw[];
@@ -236,60 +240,75 @@ __global__ void __launch_bounds__(kThr, 1)
         const uint32_t z_addr = smem_u32(smem + L::Z_OFF);
         const uint32_t st0 = smem_u32(smem + L::ST_OFF);
         const uint32_t p0 = smem_u32(smem + L::P_OFF);
+        // descriptors built once; per MMA only the address field moves
+        const uint64_t dSt = smem_desc(st0, 16, 8 * RB, SW);          // K tile rows, K-major
+        const uint64_t dQk = smem_desc(q_addr, 16, 8 * RB, SW);
+        const uint64_t dPk = smem_desc(p0, 16, kMnSbo, kSw128);       // P, K-major (Y = P Z)
+        const uint64_t dPm = smem_desc(p0, kMnLbo, kMnSbo, kSw128);   // P, MN-major (dZ)
+        const uint64_t dZm = smem_desc(z_addr, M * RB, 8 * RB, SW);   // [Z | e0], MN-major
+        const uint64_t dStm = smem_desc(st0, L::TILE, 8 * RB, SW);    // dY tile, MN-major
+        constexpr uint32_t kTile16 = (uint32_t)L::TILE >> 4;
+        constexpr uint32_t kRow16 = (uint32_t)RB;                     // 16 rows >> 4
+        constexpr uint32_t kP16 = (uint32_t)L::PBUF >> 4;
+        const int nt = (int)ntiles;
         bool ok = mbar_wait_sleep(qz_full, 0);
-        auto issue_S = [&](int64_t i) -> bool {
-          const int w = (int)(i & 1);
-          const int s = (int)(i % kAStages);
+        auto issue_S = [&](int i) -> bool {
+          const int w = i & 1;
+          const int s = i % kAStages;
           if (!mbar_wait_sleep(&st_full[s], (uint32_t)((i / kAStages) & 1))) return false;
           tc_fence_after();
-          const uint32_t k_addr = st0 + s * 2 * L::TILE;
+          const uint32_t so = (uint32_t)(s * 2) * kTile16;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + w * R, smem_desc(k_addr + 32 * kk, 16, 8 * RB, SW),
-                   smem_desc(q_addr + 32 * kk, 16, 8 * RB, SW), idS, kk > 0);
+            mma_ss(tmem + w * R, dSt + so + 2 * kk, dQk + 2 * kk, idS, kk > 0);
           mma_commit(&s_full[w]);
           return true;
         };
-        auto issue_Y = [&](int64_t i) -> bool {
-          const int w = (int)(i & 1);
-          const int64_t j = i >> 1;
+        // Y = P [Z | e0] with P read from shared memory as a K-major operand
+        // (token rows, latents contiguous: the same bytes dZ reads MN-major)
+        auto issue_Y = [&](int i) -> bool {
+          const int w = i & 1;
+          const int j = i >> 1;
           if (!mbar_wait_sleep(&p_full[w], (uint32_t)(j & 1))) return false;
           tc_fence_after();
+          const uint32_t po = (uint32_t)(2 * w + (j & 1)) * kP16;
 #pragma unroll
-          for (int kk = 0; kk < M / 16; ++kk) {
-            const uint32_t acol = (kk < M / 32) ? 8 * kk : M / 2 + 8 * kk;
-            mma_ts(tmem + w * R + TY, tmem + w * R + acol,
-                   smem_desc(z_addr + kk * 16 * RB, M * RB, 8 * RB, SW), idY, kk > 0);
-          }
+          for (int kk = 0; kk < M / 16; ++kk)
+            mma_ss(tmem + TY + YC * w, dPk + po + (kk >> 2) * (kMnLbo >> 4) + (kk & 3) * 2,
+                   dZm + kk * kRow16, idY, kk > 0);
           mma_commit(&y_full[w]);
           return true;
         };
-        auto issue_dZ = [&](int64_t i) -> bool {
-          const int w = (int)(i & 1);
-          const int64_t j = i >> 1;
-          const int s = (int)(i % kAStages);
+        auto issue_dZ = [&](int i) -> bool {
+          const int w = i & 1;
+          const int j = i >> 1;
+          const int s = i % kAStages;
           if (!mbar_wait_sleep(&a_done[w], (uint32_t)(j & 1))) return false;
           tc_fence_after();
-          const uint32_t pa = p0 + w * L::PBUF;
-          const uint32_t dy_addr = st0 + s * 2 * L::TILE + L::TILE;
+          const uint32_t po = (uint32_t)(2 * w + (j & 1)) * kP16;
+          const uint32_t so = (uint32_t)(s * 2 + 1) * kTile16;
 #pragma unroll
           for (int kk = 0; kk < kT / 16; ++kk)
-            mma_ss(tmem + TDZ, smem_desc(pa + kk * kMnKStep, kMnLbo, kMnSbo, kSw128),
-                   smem_desc(dy_addr + kk * 16 * RB, L::TILE, 8 * RB, SW), idZ,
+            mma_ss(tmem + TDZ, dPm + po + kk * (kMnKStep >> 4), dStm + so + kk * kRow16, idZ,
                    (i > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&st_empty[s]);
           return true;
         };
-        if (ok && ntiles > 0) ok = issue_S(0);
-        if (ok && ntiles > 1) ok = issue_S(1);
-        for (int64_t i = 0; ok && i < ntiles; ++i) {
+        // S of tile i + 2 goes into warpgroup (i & 1)'s S columns as soon as
+        // its P is written; dZ of a tile is issued one tile later, so the
+        // issuer never waits on one warpgroup while the other has work ready.
+        // P buffers alternate per warpgroup: dZ(i) is issued before S(i + 4),
+        // so S(i + 4) completing implies dZ(i), and with it the last read of
+        // the buffer P(i + 4) reuses.
+        if (ok && nt > 0) ok = issue_S(0);
+        if (ok && nt > 1) ok = issue_S(1);
+        for (int i = 0; ok && i < nt; ++i) {
           ok = issue_Y(i);
-          if (ok) ok = issue_dZ(i);
-          // the warpgroup's columns are free (a_done) and, by issue order,
-          // the dZ MMA that reads its P buffer completes before this S does
-          if (ok && i + 2 < ntiles) ok = issue_S(i + 2);
+          if (ok && i + 2 < nt) ok = issue_S(i + 2);
+          if (ok && i >= 1) ok = issue_dZ(i - 1);
           if (*abort_flag) ok = false;
         }
+        if (ok && nt > 0) ok = issue_dZ(nt - 1);
         if (!ok) {
           record_error(err, kErrBwdAMmaWait);
           *abort_flag = 1;
@@ -305,13 +324,14 @@ __global__ void __launch_bounds__(kThr, 1)
     const int r = qw * 32 + lane;                    // TMEM lane = token row of the tile
     const uint32_t lb = (uint32_t)(qw * 32) << 16;
     const uint32_t tR = tmem + lb + w * R;
-    uint8_t* pbuf = smem + L::P_OFF + w * L::PBUF;
+    const float Rh = rref[bh];
     const int64_t nW = (ntiles - w + 1) / 2;
     bool ok = true;
     for (int64_t j = 0; j < nW; ++j) {
       const int64_t i = 2 * j + w;
       const int s = (int)(i % kAStages);
       const int64_t tok = (tile0 + i) * kT + r;
+      uint8_t* pbuf = smem + L::P_OFF + (2 * w + (j & 1)) * L::PBUF;
       if (!warp_all(mbar_wait_sleep(&s_full[w], (uint32_t)(j & 1)) && !*abort_flag)) {
         ok = false;
         break;
@@ -332,27 +352,20 @@ __global__ void __launch_bounds__(kThr, 1)
       const float mx = fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3]));
       const float neg = -mx * c;
       float sf[4] = {0.f, 0.f, 0.f, 0.f};
-      // pass 2: P = 2^(c S - c mx) as bf16 pairs.  TMEM copy for Y = P Z,
-      // placed as in the forward's decode (upper-half chunks last-first so
-      // no store lands on a chunk still to be read); shared-memory copy for
-      // dZ += P^T dY'.
-      auto chunk_col = [](int k) { return k < NC / 2 ? M / 2 + 32 * (NC / 2 - 1 - k) : 32 * (k - NC / 2); };
-      auto p_col = [](int k) { return k < NC / 2 ? 3 * M / 4 + 16 * (NC / 2 - 1 - k) : 16 * (k - NC / 2); };
-      tmem_ld32(tR + chunk_col(0), a[0]);
+      // pass 2: P = 2^(c S - c mx) as bf16 pairs into shared memory (the
+      // operand of Y = P [Z | e0] and of dZ += P^T dY')
+      tmem_ld32(tR, a[0]);
 #pragma unroll
       for (int k = 0; k < NC; ++k) {
         tmem_wait_ld_dep(a[k & 1]);
-        if (k + 1 < NC) tmem_ld32(tR + chunk_col(k + 1), a[(k + 1) & 1]);
+        if (k + 1 < NC) tmem_ld32(tR + 32 * (k + 1), a[(k + 1) & 1]);
         uint32_t pk[16];
         exp_pack32<0>(a[k & 1], c, neg, pk, sf);
-        tmem_st16(tR + p_col(k), pk);
-        const int g0 = chunk_col(k) >> 3;
 #pragma unroll
         for (int v = 0; v < 4; ++v)
-          *reinterpret_cast<uint4*>(pbuf + mn_off(r, g0 + v)) =
+          *reinterpret_cast<uint4*>(pbuf + mn_off(r, 4 * k + v)) =
               make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
       }
-      tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&p_full[w]);
@@ -365,48 +378,59 @@ __global__ void __launch_bounds__(kThr, 1)
       __syncwarp();
       tc_fence_after();
       float y[D];
-      float lb;   // row sum of the bf16 P (the weights the tensor cores used)
+      float lsum;   // row sum of the bf16 P (the weights the tensor cores used)
       if (D == 32) {
         uint32_t o[32], o2[16];
-        tmem_ld32(tR + TY, o);
-        tmem_ld16(tR + TY + 32, o2);
+        tmem_ld32(tmem + lb + TY + YC * w, o);
+        tmem_ld16(tmem + lb + TY + YC * w + 32, o2);
         tmem_wait_ld_dep(o);
         reg_fence16(o2);
 #pragma unroll
         for (int d = 0; d < D; ++d) y[d] = __uint_as_float(o[d]);
-        lb = __uint_as_float(o2[0]);
+        lsum = __uint_as_float(o2[0]);
       } else {
         uint32_t o[32];
-        tmem_ld32(tR + TY, o);
+        tmem_ld32(tmem + lb + TY + YC * w, o);
         tmem_wait_ld_dep(o);
 #pragma unroll
         for (int d = 0; d < D; ++d) y[d] = __uint_as_float(o[d]);
-        lb = __uint_as_float(o[D]);
+        lsum = __uint_as_float(o[D]);
       }
       const float l = (sf[0] + sf[1]) + (sf[2] + sf[3]);
-      const float inv = 1.f / lb;
+      const float inv = 1.f / lsum;
+      const float mxp = fmaf(mx, c, log2f(l));   // row log-sum-exp, log2 units
+      const float lg = mxp - Rh;                  // log2 of g[n]
+      const bool bad = lg < -kRowRangeMax;        // g[n] would leave the float range
+      const float ginv = bad ? 0.f : ex2(-lg);    // 1 / g[n]
       uint8_t* dyt = smem + L::ST_OFF + s * 2 * L::TILE + L::TILE;
-      float dot = 0.f;
+      float dot = 0.f, dot2 = 0.f;
+      uint4 o2[D / 8];
 #pragma unroll
       for (int ch = 0; ch < D / 8; ++ch) {
         uint4* p = reinterpret_cast<uint4*>(dyt + tma_row_chunk<D>(r, ch));
-        uint4 u = *p;
-        const float* yy = y + 8 * ch;
-        dot = fmaf(bf_lo(u.x), yy[0], dot);
-        dot = fmaf(bf_hi(u.x), yy[1], dot);
-        dot = fmaf(bf_lo(u.y), yy[2], dot);
-        dot = fmaf(bf_hi(u.y), yy[3], dot);
-        dot = fmaf(bf_lo(u.z), yy[4], dot);
-        dot = fmaf(bf_hi(u.z), yy[5], dot);
-        dot = fmaf(bf_lo(u.w), yy[6], dot);
-        dot = fmaf(bf_hi(u.w), yy[7], dot);
-        u.x = pack_bf16(bf_lo(u.x) * inv, bf_hi(u.x) * inv);
-        u.y = pack_bf16(bf_lo(u.y) * inv, bf_hi(u.y) * inv);
-        u.z = pack_bf16(bf_lo(u.z) * inv, bf_hi(u.z) * inv);
-        u.w = pack_bf16(bf_lo(u.w) * inv, bf_hi(u.w) * inv);
-        *p = u;
+        const uint4 u = *p;
+        const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
+        uint32_t wv[4], w2[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float a0 = bf_lo(uu[j]), a1 = bf_hi(uu[j]);
+          const float y0 = y[8 * ch + 2 * j], y1 = y[8 * ch + 2 * j + 1];
+          dot = fmaf(a0, y0, fmaf(a1, y1, dot));
+          w2[j] = pack_bf16(a0 * ginv, a1 * ginv);           // dY'' = dY / g
+          dot2 = fmaf(bf_lo(w2[j]), y0, fmaf(bf_hi(w2[j]), y1, dot2));
+          wv[j] = pack_bf16(a0 * inv, a1 * inv);             // dY' = dY / rowsum
+        }
+        *p = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        o2[ch] = make_uint4(w2[0], w2[1], w2[2], w2[3]);
       }
-      if (tok < N) stats[bh * N + tok] = make_float2(fmaf(mx, c, log2f(l)), dot * inv);
+      if (tok < N) {
+        // delta_d = dY . Y and its counterpart with the rounded dY'' (= delta_d / g)
+        stats[bh * N + tok] = make_float4(mxp, dot * inv, dot2 * inv, 0.f);
+        uint4* dst = reinterpret_cast<uint4*>(dy2 + (bh * N + tok) * D);
+#pragma unroll
+        for (int ch = 0; ch < D / 8; ++ch) dst[ch] = o2[ch];
+      }
+      if (warp_any(bad && tok < N) && lane == 0) atomicOr(flags + bh, 1u);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&a_done[w]);
@@ -458,25 +482,49 @@ __global__ void __launch_bounds__(kThr, 1)
 
 // ======================================================= between passes
 
-// Z (float) -> bf16 copy, the operand of Y = P Z and dPd = dY Z^T.
-__global__ void bwd_zbf16_kernel(const float4* __restrict__ z, uint2* __restrict__ zb, int64_t n4) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n4) return;
-  const float4 v = z[i];
-  zb[i] = make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
+// One block per (b, h), one thread per latent m: the bf16 copy of Z (the
+// operand of Y = P Z and of dY'' Z^T) and R = max_m lse2[m], the reference
+// of the split of the encode weights; clears the head's range flag.
+template <int D>
+__global__ void __launch_bounds__(kM)
+    bwd_prep_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
+                    __nv_bfloat16* __restrict__ zb, float* __restrict__ rref,
+                    uint32_t* __restrict__ flags) {
+  __shared__ float red[kM / 32];
+  const int64_t bh = blockIdx.x;
+  const int m = threadIdx.x;
+  const int64_t row = bh * kM + m;
+#pragma unroll
+  for (int d = 0; d < D; d += 4) {
+    const float4 v = *reinterpret_cast<const float4*>(Z + row * D + d);
+    *reinterpret_cast<uint2*>(zb + row * D + d) = make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
+  }
+  float mx = lse[row] * kLog2e;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((m & 31) == 0) red[m >> 5] = mx;
+  __syncthreads();
+  if (m == 0) {
+    float R = red[0];
+#pragma unroll
+    for (int k = 1; k < kM / 32; ++k) R = fmaxf(R, red[k]);
+    rref[bh] = R;
+    flags[bh] = 0u;
+  }
 }
 
 // One block per (b, h), one thread per latent m.  dZ = sum of the chunk
 // partials (fixed order), lse2 = lse log2(e); R = max lse2 over the head;
-// f = 2^(R - lse2) when the head's lse2 spread is at most kSpreadMax (else
-// f = 1 and the exact form); the bf16 operand dZ'' = f dZ; the extra K-step
-// row: -dZ'' . Z (= -f delta_e) as three bf16 terms, then zeros.
+// f = 2^(R - lse2) when the head's lse2 spread is at most kSpreadMax and no
+// token of it lies more than kRowRangeMax below R (else f = 1 and the exact
+// form); the bf16 operand dZ'' = f dZ; the extra K-step row: -dZ'' . Z
+// (= -f delta_e) as three bf16 terms, then zeros.
 template <int D>
 __global__ void __launch_bounds__(kM)
     bwd_mid_kernel(const float* __restrict__ dz_part, int chunks, const float* __restrict__ Z,
                    const float* __restrict__ lse, __nv_bfloat16* __restrict__ dzs,
-                   uint32_t* __restrict__ aug, float2* __restrict__ params,
-                   float* __restrict__ lse2_out) {
+                   uint32_t* __restrict__ aug, const uint32_t* __restrict__ flags,
+                   float2* __restrict__ params, float* __restrict__ lse2_out) {
   __shared__ float red_max[kM / 32], red_min[kM / 32];
   const int64_t bh = blockIdx.x;
   const int m = threadIdx.x;
@@ -513,7 +561,7 @@ __global__ void __launch_bounds__(kM)
     R = fmaxf(R, red_max[k]);
     lo = fminf(lo, red_min[k]);
   }
-  const bool fast = (R - lo) <= kSpreadMax;
+  const bool fast = (R - lo) <= kSpreadMax && flags[bh] == 0u;
   const float f = fast ? exp2f(R - l2) : 1.f;
   // delta_e is taken with the bf16 operand dZ'' that the tensor cores use,
   // so dPe'' = V dZ''^T - dZ'' . Z vanishes exactly where V = Z.
@@ -565,12 +613,12 @@ struct BLayout {
 
 template <int D>
 __global__ void __launch_bounds__(kThr, 1)
-    tc_bwd_b_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+    tc_bwd_b_exact_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdY,
                     const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmDZ,
                     const __grid_constant__ CUtensorMap tmAug, int H, int64_t N, int q_per_batch,
                     float c, float s, int64_t tiles_per_bh, int64_t chunk_tiles,
-                    const float2* __restrict__ stats, const float2* __restrict__ params,
+                    const float4* __restrict__ stats, const float2* __restrict__ params,
                     const float* __restrict__ lse2, __nv_bfloat16* __restrict__ dK,
                     __nv_bfloat16* __restrict__ dV, float* __restrict__ dq_part,
                     uint32_t* __restrict__ err) {
@@ -609,6 +657,7 @@ __global__ void __launch_bounds__(kThr, 1)
   const int64_t tile0 = (int64_t)chunk * chunk_tiles;
   const int64_t ntiles = imin64(chunk_tiles, tiles_per_bh - tile0);
   const int64_t KQ = ntiles * NQ;   // quarters of this chunk
+  if (params[bh].y != 0.f) return;  // head served by tc_bwd_b_fast_kernel
 
   // the constant A operand of the extra K-step: ones in columns 0-2 of
   // every row, 32-byte swizzle (row t at 32 t, 16-byte chunk x at x ^ bit 2 of t)
@@ -793,9 +842,6 @@ __global__ void __launch_bounds__(kThr, 1)
     const int w = warp >> 2, qw = warp & 3;
     const int r = qw * 32 + lane;                    // TMEM lane = token row of the tile
     const uint32_t lb = (uint32_t)(qw * 32) << 16;
-    const float2 prm = params[bh];
-    const float Rref = prm.x;
-    const bool fast = prm.y != 0.f;
     const float* ls = (const float*)(smem + L::LSE_OFF);
     const uint64_t c2 = f32x2(c, c);
     float mxp = 0.f, dd = 0.f, g = 0.f, gprev = 0.f;
@@ -847,10 +893,10 @@ __global__ void __launch_bounds__(kThr, 1)
         const int64_t tok = (tile0 + t) * kT + r;
         valid = tok < N;
         if (valid) {
-          const float2 st = stats[bh * N + tok];
+          const float4 st = stats[bh * N + tok];
           mxp = st.x;
           dd = st.y;
-          g = fast ? exp2f(mxp - Rref) : 1.f;
+          g = 1.f;
         } else {
           mxp = 0.f;
           dd = 0.f;
@@ -865,7 +911,7 @@ __global__ void __launch_bounds__(kThr, 1)
       tc_fence_after();
       const uint32_t tq = tmem + lb + QC * slot;
       uint8_t* gsm = smem + L::G_OFF + (t & 1) * L::GBUF;
-      const uint64_t nm2 = f32x2(-mxp, -mxp), nd2 = f32x2(-dd, -dd), g2 = f32x2(g, g);
+      const uint64_t nm2 = f32x2(-mxp, -mxp), nd2 = f32x2(-dd, -dd);
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t a[16], b[16], e[16];
@@ -885,25 +931,16 @@ __global__ void __launch_bounds__(kThr, 1)
           float x0, x1;
           split_f32x2(fma_f32x2(S2, c2, nm2), x0, x1);
           const float p0 = ex2(x0), p1 = ex2(x1);
-          float g0v, g1v, w0, w1;
-          if (fast) {
-            // G = P_d (dPd - delta_d + g dPe'');  dV weights P_d
-            split_f32x2(mul_f32x2(f32x2(p0, p1), add_f32x2(fma_f32x2(E2, g2, P2), nd2)), g0v,
-                        g1v);
-            w0 = p0;
-            w1 = p1;
-          } else {
-            // exact form: P_e = 2^(c S - lse2[m]); G = P_d (dPd - delta_d) + P_e dPe'
-            float s0, s1, e0, e1;
-            split_f32x2(S2, s0, s1);
-            split_f32x2(E2, e0, e1);
-            w0 = valid ? ex2(fmaf(s0, c, -ls[m0 + 2 * p])) : 0.f;
-            w1 = valid ? ex2(fmaf(s1, c, -ls[m0 + 2 * p + 1])) : 0.f;
-            float d0, d1;
-            split_f32x2(add_f32x2(P2, nd2), d0, d1);
-            g0v = fmaf(w0, e0, p0 * d0);
-            g1v = fmaf(w1, e1, p1 * d1);
-          }
+          // exact form: P_e = 2^(c S - lse2[m]); G = P_d (dPd - delta_d) + P_e dPe'
+          float s0, s1, e0, e1;
+          split_f32x2(S2, s0, s1);
+          split_f32x2(E2, e0, e1);
+          const float w0 = valid ? ex2(fmaf(s0, c, -ls[m0 + 2 * p])) : 0.f;
+          const float w1 = valid ? ex2(fmaf(s1, c, -ls[m0 + 2 * p + 1])) : 0.f;
+          float d0, d1;
+          split_f32x2(add_f32x2(P2, nd2), d0, d1);
+          const float g0v = fmaf(w0, e0, p0 * d0);
+          const float g1v = fmaf(w1, e1, p1 * d1);
           gk[p] = pack_bf16(g0v, g1v);
           vk[p] = pack_bf16(w0, w1);
         }
@@ -930,6 +967,432 @@ __global__ void __launch_bounds__(kThr, 1)
 #pragma unroll
       for (int d = 0; d < D; ++d) acc[d] = 0.f;
       if (ok && KQ > 0) {
+        ok = warp_all(mbar_wait_sleep(dq_final, 0));
+        __syncwarp();
+        tc_fence_after();
+        if (ok) {
+          if (D == 32) {
+            uint32_t u[32];
+            tmem_ld32(tmem + lb + TDQ, u);
+            tmem_wait_ld_dep(u);
+#pragma unroll
+            for (int d = 0; d < D; ++d) acc[d] = __uint_as_float(u[d]) * s;
+          } else {
+            uint32_t u[16];
+            tmem_ld16(tmem + lb + TDQ, u);
+            tmem_wait_ld_dep16(u);
+#pragma unroll
+            for (int d = 0; d < D; ++d) acc[d] = __uint_as_float(u[d & 15]) * s;
+          }
+        } else {
+          record_error(err, kErrBwdBRowWait);
+          *abort_flag = 1;
+        }
+      }
+      float4* dst = reinterpret_cast<float4*>(dq_part + (((int64_t)bh * chunks + chunk) * M + r) * D);
+#pragma unroll
+      for (int d = 0; d < D / 4; ++d)
+        dst[d] = make_float4(acc[4 * d], acc[4 * d + 1], acc[4 * d + 2], acc[4 * d + 3]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kWMma) tmem_dealloc(tmem, NCOLS);
+}
+
+// ------------------------------------------------- pass B, one-exponential form
+//
+// For heads whose ranges allow it (params.y = 1): with e = 2^(c S - R),
+//   P_d = e / g[n],  P_e = e f[m],
+//   G   = e U,  U[n,m] = dY''[n] . Z[m] + V[n] . dZ''[m] - dZ''[m] . Z[m] - delta''[n]
+// where dY'' = dY / g (written by pass A), delta'' = dY'' . Y, dZ'' = f dZ.
+// The first three terms of U are ONE tensor-core product over a K of
+// 2 D + 16 (dY'' | V | ones against Z | dZ'' | -dZ''.Z split in three bf16).
+//   dK = s G Q,  dV = e dZ'',  dQ = s G^T K.
+// Work unit: half a tile (128 tokens x 64 latents; warpgroup w takes latent
+// half w of every tile).  S and U of a half go to one of three TMEM slots;
+// the row warps write G and e only to shared memory (128-byte swizzled,
+// token rows, latents contiguous), from where dK = G Q and dV = e dZ'' read
+// them as K-major operands and dQ = G^T K as an MN-major one.  A slot is
+// therefore free as soon as its rows are read, and the output products of a
+// tile are issued once both halves are in.
+
+template <int D>
+struct BFLayout {
+  static constexpr int M = kM;
+  static constexpr int NSLOT = 3;
+  static constexpr int KST = 4;                       // K tiles: held until the tile's dQ
+  static constexpr int VST = 2;                       // V, dY'' tiles: until its U products
+  static constexpr int RB = 2 * D;
+  static constexpr int TILE = kT * RB;
+  static constexpr int GBUF = kT * M * 2;              // 32 KB
+  static constexpr int G_OFF = 0;                      // two G buffers (tile parity)
+  static constexpr int E_OFF = 2 * GBUF;               // two e buffers (tile parity)
+  static constexpr int Q_OFF = 4 * GBUF;
+  static constexpr int Z_OFF = Q_OFF + M * RB;
+  static constexpr int DZ_OFF = Z_OFF + M * RB;
+  static constexpr int AUG_OFF = DZ_OFF + M * RB;      // [M][16] bf16, 32-byte rows
+  static constexpr int ONES_OFF = AUG_OFF + M * 32;    // [128][16] bf16
+  static constexpr int K_OFF = ONES_OFF + kT * 32;     // K ring
+  static constexpr int VD_OFF = K_OFF + KST * TILE;    // (V, dY'') ring
+  static constexpr int BAR_OFF = VD_OFF + VST * 2 * TILE;
+  static constexpr int NBARS = 2 * KST + 2 * VST + 1 + 2 * NSLOT + 1 + 1 + 1 + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+  static constexpr int BYTES = MISC_OFF + 16;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThr, 1)
+    tc_bwd_b_fast_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdY2,
+                         const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmDZ,
+                         const __grid_constant__ CUtensorMap tmAug, int H, int64_t N, int q_per_batch,
+                         float c, float s, int64_t tiles_per_bh, int64_t chunk_tiles,
+                         const float4* __restrict__ stats, const float2* __restrict__ params,
+                         __nv_bfloat16* __restrict__ dK, __nv_bfloat16* __restrict__ dV,
+                         float* __restrict__ dq_part, uint32_t* __restrict__ err) {
+  using L = BFLayout<D>;
+  constexpr int M = L::M;
+  constexpr int NS = L::NSLOT;
+  constexpr int KST = L::KST;
+  constexpr int VST = L::VST;
+  constexpr int RB = L::RB;
+  constexpr uint32_t SW = umma_swizzle_code(RB);
+  constexpr int HC = 128;              // TMEM columns of one half slot: S (64) | U (64)
+  constexpr int TDK = NS * HC;         // dK accumulator (token lanes)
+  constexpr int TDV = TDK + D;         // dV accumulator (token lanes)
+  constexpr int TDQ = TDV + D;         // dQ accumulator (latent lanes)
+  constexpr uint32_t NCOLS = 512;
+  static_assert(TDQ + D <= 512, "TMEM budget");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* bars = (uint64_t*)(smem + L::BAR_OFF);
+  uint64_t* k_full = bars;
+  uint64_t* k_empty = k_full + KST;
+  uint64_t* v_full = k_empty + KST;
+  uint64_t* v_empty = v_full + VST;
+  uint64_t* c_full = v_empty + VST;
+  uint64_t* h_full = c_full + 1;        // [slot] S and U of a half in TMEM
+  uint64_t* h_done = h_full + NS;       // [slot] the half's rows read, G and e in shared memory
+  uint64_t* tile_done = h_done + NS;    // dK, dV of a tile final; its G, e buffers free
+  uint64_t* acc_empty = tile_done + 1;  // dK, dV accumulators read back
+  uint64_t* dq_final = acc_empty + 1;
+  uint64_t* drain = dq_final + 1;
+  uint32_t* tmem_slot = (uint32_t*)(smem + L::MISC_OFF);
+  volatile int* abort_flag = (volatile int*)(smem + L::MISC_OFF + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x, chunks = gridDim.x;
+  const int64_t bh = blockIdx.y;
+  const int64_t h = bh % H;
+  const int64_t tile0 = (int64_t)chunk * chunk_tiles;
+  const int nt = (int)imin64(chunk_tiles, tiles_per_bh - tile0);
+  const float2 prm = params[bh];
+  if (prm.y == 0.f) return;   // head served by tc_bwd_b_exact_kernel
+
+  for (int t = threadIdx.x; t < kT; t += blockDim.x) {
+    // ones in columns 0-2 of every row of the extra K-step's A operand (32-byte swizzle)
+    uint8_t* ones = smem + L::ONES_OFF;
+    const int x0 = (t >> 2) & 1;
+    *reinterpret_cast<uint4*>(ones + t * 32 + x0 * 16) = make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u);
+    *reinterpret_cast<uint4*>(ones + t * 32 + (x0 ^ 1) * 16) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  fence_proxy_async_smem();
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < KST; ++k) {
+      mbar_init(&k_full[k], 1);
+      mbar_init(&k_empty[k], 1);
+    }
+    for (int k = 0; k < VST; ++k) {
+      mbar_init(&v_full[k], 1);
+      mbar_init(&v_empty[k], 1);
+    }
+    mbar_init(c_full, 1);
+    for (int k = 0; k < NS; ++k) {
+      mbar_init(&h_full[k], 1);
+      mbar_init(&h_done[k], 128);
+    }
+    mbar_init(tile_done, 1);
+    mbar_init(acc_empty, 256);
+    mbar_init(dq_final, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kWMma) tmem_alloc(tmem_slot, NCOLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp >= 8) {
+    regs_release<kRegsPro>();
+    if (warp == kWTma) {
+      if (lane == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        prefetch_tmap(&tmdY2);
+        prefetch_tmap(&tmZ);
+        prefetch_tmap(&tmDZ);
+        prefetch_tmap(&tmAug);
+        mbar_arrive_expect_tx(c_full, 3 * M * RB + M * 32);
+        tma_load_3d(smem + L::Q_OFF, &tmQ, c_full, 0, 0, (int32_t)(q_per_batch ? bh : h));
+        tma_load_3d(smem + L::Z_OFF, &tmZ, c_full, 0, 0, (int32_t)bh);
+        tma_load_3d(smem + L::DZ_OFF, &tmDZ, c_full, 0, 0, (int32_t)bh);
+        tma_load_3d(smem + L::AUG_OFF, &tmAug, c_full, 0, 0, (int32_t)bh);
+        int issued = 0;
+        for (int t = 0; t < nt; ++t) {
+          const int32_t tok = (int32_t)((tile0 + t) * kT);
+          const int kb = t % KST, vb = t % VST;
+          if (t >= KST && !mbar_wait_sleep(&k_empty[kb], (uint32_t)(((t / KST) & 1) ^ 1))) {
+            record_error(err, kErrBwdBTmaWait);
+            *abort_flag = 1;
+            break;
+          }
+          if (*abort_flag) break;
+          mbar_arrive_expect_tx(&k_full[kb], L::TILE);
+          tma_load_3d(smem + L::K_OFF + kb * L::TILE, &tmK, &k_full[kb], 0, tok, (int32_t)bh);
+          if (t >= VST && !mbar_wait_sleep(&v_empty[vb], (uint32_t)(((t / VST) & 1) ^ 1))) {
+            record_error(err, kErrBwdBTmaWait);
+            *abort_flag = 1;
+            mbar_wait_sleep(&k_full[kb], (uint32_t)((t / KST) & 1));
+            break;
+          }
+          uint8_t* dst = smem + L::VD_OFF + vb * 2 * L::TILE;
+          mbar_arrive_expect_tx(&v_full[vb], 2 * L::TILE);
+          tma_load_3d(dst, &tmV, &v_full[vb], 0, tok, (int32_t)bh);
+          tma_load_3d(dst + L::TILE, &tmdY2, &v_full[vb], 0, tok, (int32_t)bh);
+          issued = t + 1;
+        }
+        // let every load still in flight land before the CTA can exit
+        for (int t = (issued > KST ? issued - KST : 0); t < issued; ++t)
+          mbar_wait_sleep(&k_full[t % KST], (uint32_t)((t / KST) & 1));
+        for (int t = (issued > VST ? issued - VST : 0); t < issued; ++t)
+          mbar_wait_sleep(&v_full[t % VST], (uint32_t)((t / VST) & 1));
+        mbar_wait_sleep(c_full, 0);
+      }
+    } else if (warp == kWMma) {
+      if (lane == 0) {
+        constexpr uint32_t idH = idesc_bf16_f32(128, 64, 0, 0);   // a half's S or U
+        constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);    // dK, dV (A K-major)
+        constexpr uint32_t idQ = idesc_bf16_f32(128, D, 1, 1);    // dQ (A MN-major)
+        const uint32_t q_addr = smem_u32(smem + L::Q_OFF);
+        const uint32_t z_addr = smem_u32(smem + L::Z_OFF);
+        const uint32_t dz_addr = smem_u32(smem + L::DZ_OFF);
+        const uint32_t aug_addr = smem_u32(smem + L::AUG_OFF);
+        const uint32_t ones_addr = smem_u32(smem + L::ONES_OFF);
+        const uint32_t k0 = smem_u32(smem + L::K_OFF);
+        const uint32_t v0 = smem_u32(smem + L::VD_OFF);
+        const uint32_t g0 = smem_u32(smem + L::G_OFF);
+        // descriptors built once; per MMA only the 14-bit address field
+        // moves (offsets >> 4 added; shared addresses stay below 256 KB)
+        const uint64_t dK0 = smem_desc(k0, 16, 8 * RB, SW);           // K tile rows, K-major
+        const uint64_t dV0 = smem_desc(v0, 16, 8 * RB, SW);           // V / dY'' tile rows
+        const uint64_t dQk = smem_desc(q_addr, 16, 8 * RB, SW);       // latent rows, K-major
+        const uint64_t dZk = smem_desc(z_addr, 16, 8 * RB, SW);
+        const uint64_t dDZk = smem_desc(dz_addr, 16, 8 * RB, SW);
+        const uint64_t dOnes = smem_desc(ones_addr, 16, 256, kSw32);
+        const uint64_t dAug = smem_desc(aug_addr, 16, 256, kSw32);
+        const uint64_t dQm = smem_desc(q_addr, M * RB, 8 * RB, SW);   // latent rows, MN-major
+        const uint64_t dDZm = smem_desc(dz_addr, M * RB, 8 * RB, SW);
+        const uint64_t dKm = smem_desc(k0, L::TILE, 8 * RB, SW);      // K tile, MN-major
+        const uint64_t dGk = smem_desc(g0, 16, kMnSbo, kSw128);       // G or e, K-major
+        const uint64_t dGm = smem_desc(g0, kMnLbo, kMnSbo, kSw128);   // G, MN-major
+        constexpr uint32_t kTile16 = (uint32_t)L::TILE >> 4;
+        constexpr uint32_t kRow16 = (uint32_t)RB;                     // 16 rows >> 4
+        constexpr uint32_t kBuf16 = (uint32_t)L::GBUF >> 4;
+        const int nh = 2 * nt;
+        bool ok = mbar_wait_sleep(c_full, 0);
+        // S and U of half k (tile k / 2, latents [64 (k & 1), +64)) into slot k % 3
+        auto issue_H = [&](int k) -> bool {
+          const int t = k >> 1;
+          const int hf = k & 1;
+          const int kb = t % KST, vb = t % VST;
+          if (hf == 0 && !(mbar_wait_sleep(&k_full[kb], (uint32_t)((t / KST) & 1)) &&
+                           mbar_wait_sleep(&v_full[vb], (uint32_t)((t / VST) & 1))))
+            return false;
+          tc_fence_after();
+          const uint32_t base = tmem + HC * (uint32_t)(k % NS);
+          const uint32_t ko = (uint32_t)kb * kTile16;
+          const uint32_t vo = (uint32_t)(2 * vb) * kTile16;     // V at vo, dY'' at vo + kTile16
+          const uint32_t ro = (uint32_t)(64 * hf * RB) >> 4;   // latent rows [64 hf, +64)
+          // the S and U chains interleaved, so consecutive MMAs are independent
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            mma_ss(base, dK0 + ko + 2 * kk, dQk + ro + 2 * kk, idH, kk > 0);
+            mma_ss(base + 64, dV0 + vo + kTile16 + 2 * kk, dZk + ro + 2 * kk, idH, kk > 0);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(base + 64, dV0 + vo + 2 * kk, dDZk + ro + 2 * kk, idH, 1u);
+          mma_ss(base + 64, dOnes, dAug + (uint32_t)(2 * 64 * hf), idH, 1u);
+          mma_commit(&h_full[k % NS]);
+          if (hf == 1) mma_commit(&v_empty[vb]);   // V and dY'' of tile t read by both halves
+          return true;
+        };
+        for (int k = 0; ok && k < NS && k < nh; ++k) ok = issue_H(k);
+        for (int k = 0; ok && k < nh; ++k) {
+          // half k read: its slot takes half k + 3 at once (no MMA reads TMEM slots)
+          if (!mbar_wait_sleep(&h_done[k % NS], (uint32_t)((k / NS) & 1))) {
+            ok = false;
+            break;
+          }
+          if (k + NS < nh && !(ok = issue_H(k + NS))) break;
+          if ((k & 1) == 0) continue;
+          // both halves of tile t in shared memory: dK, dV, dQ of the tile
+          const int t = k >> 1;
+          if (t > 0 && !mbar_wait_sleep(acc_empty, (uint32_t)((t - 1) & 1))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t go = (uint32_t)(t & 1) * kBuf16;
+          const uint32_t eo = go + 2 * kBuf16;
+          const uint32_t ko = (uint32_t)(t % KST) * kTile16;
+          // three independent accumulator chains, interleaved
+          static_assert(M == kT, "dK/dV and dQ take the same number of K-steps");
+#pragma unroll
+          for (int kk = 0; kk < M / 16; ++kk) {
+            const uint32_t ak = (kk >> 2) * (kMnLbo >> 4) + (kk & 3) * 2;   // 16 latents
+            mma_ss(tmem + TDK, dGk + go + ak, dQm + kk * kRow16, idO, kk > 0);
+            mma_ss(tmem + TDV, dGk + eo + ak, dDZm + kk * kRow16, idO, kk > 0);
+            mma_ss(tmem + TDQ, dGm + go + kk * (kMnKStep >> 4), dKm + ko + kk * kRow16, idQ,
+                   (t > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(tile_done);
+          mma_commit(&k_empty[t % KST]);
+          if (*abort_flag) ok = false;
+        }
+        if (!ok) {
+          record_error(err, kErrBwdBMmaWait);
+          *abort_flag = 1;
+        }
+        mma_commit(dq_final);
+        mma_commit(drain);
+        mbar_wait_sleep(drain, 0);
+      }
+    }
+  } else {
+    regs_acquire<kRegsRow>();
+    const int w = warp >> 2, qw = warp & 3;
+    const int r = qw * 32 + lane;                    // TMEM lane = token row of the tile
+    const uint32_t lb = (uint32_t)(qw * 32) << 16;
+    const float Rh = prm.x;
+    const uint64_t c2 = f32x2(c, c);
+    bool ok = true;
+    // delta'' of this thread's row in tile tt, loaded one tile ahead of use
+    auto load_dpp = [&](int tt) -> float {
+      const int64_t tok = (tile0 + tt) * kT + r;
+      return (tt < nt && tok < N) ? stats[bh * N + tok].z : 0.f;
+    };
+    float dpp_next = load_dpp(0);
+
+    // dK (warpgroup 0) or dV (warpgroup 1) of tile tt: wait for the tile's
+    // products, read and release the accumulator, scale and store the rows.
+    auto finish = [&](int tt) -> bool {
+      if (!warp_all(mbar_wait_sleep(tile_done, (uint32_t)(tt & 1)) && !*abort_flag)) return false;
+      __syncwarp();
+      tc_fence_after();
+      float o[D];
+      const uint32_t col = (w == 0) ? TDK : TDV;
+      if (D == 32) {
+        uint32_t u[32];
+        tmem_ld32(tmem + lb + col, u);
+        tmem_wait_ld_dep(u);
+#pragma unroll
+        for (int d = 0; d < D; ++d) o[d] = __uint_as_float(u[d]);
+      } else {
+        uint32_t u[16];
+        tmem_ld16(tmem + lb + col, u);
+        tmem_wait_ld_dep16(u);
+#pragma unroll
+        for (int d = 0; d < D; ++d) o[d] = __uint_as_float(u[d & 15]);
+      }
+      tc_fence_before();
+      mbar_arrive(acc_empty);
+      const int64_t tok = (tile0 + tt) * kT + r;
+      if (tok < N) {
+        const float f = (w == 0) ? s : 1.f;
+        uint4* dst = reinterpret_cast<uint4*>((w == 0 ? dK : dV) + (bh * N + tok) * D);
+#pragma unroll
+        for (int v = 0; v < D / 8; ++v)
+          dst[v] = make_uint4(pack_bf16(o[8 * v] * f, o[8 * v + 1] * f),
+                              pack_bf16(o[8 * v + 2] * f, o[8 * v + 3] * f),
+                              pack_bf16(o[8 * v + 4] * f, o[8 * v + 5] * f),
+                              pack_bf16(o[8 * v + 6] * f, o[8 * v + 7] * f));
+      }
+      return true;
+    };
+
+    for (int t = 0; t < nt; ++t) {
+      const int k = 2 * t + w;          // this warpgroup's half of tile t
+      const int slot = k % NS;
+      const int64_t tok = (tile0 + t) * kT + r;
+      const float ndd = -dpp_next;
+      const float nR = (tok < N) ? -Rh : -INFINITY;   // past the end of the head: e = 0, G = 0
+      dpp_next = load_dpp(t + 1);
+      if (!warp_all(mbar_wait_sleep(&h_full[slot], (uint32_t)((k / NS) & 1)) && !*abort_flag)) {
+        ok = false;
+        break;
+      }
+      __syncwarp();
+      tc_fence_after();
+      // the G / e buffers of tile t were last read by tile t - 2's products,
+      // which completed before this warpgroup's finish(t - 2) returned
+      const uint32_t tq = tmem + lb + HC * slot;
+      uint8_t* gsm = smem + L::G_OFF + (t & 1) * L::GBUF;
+      uint8_t* esm = smem + L::E_OFF + (t & 1) * L::GBUF;
+      const uint64_t nR2 = f32x2(nR, nR), nd2 = f32x2(ndd, ndd);
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t a[32], u[32];
+        tmem_ld32(tq + 32 * cc, a);
+        tmem_ld32(tq + 64 + 32 * cc, u);
+        tmem_wait_ld_dep(a);
+        tmem_wait_ld_dep(u);
+        uint32_t gk[16], ek[16];
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+          float x0, x1, g0v, g1v;
+          split_f32x2(fma_f32x2(f32x2(__uint_as_float(a[2 * p]), __uint_as_float(a[2 * p + 1])), c2,
+                                nR2), x0, x1);
+          const float e0 = ex2(x0), e1 = ex2(x1);
+          split_f32x2(mul_f32x2(f32x2(e0, e1),
+                                add_f32x2(f32x2(__uint_as_float(u[2 * p]), __uint_as_float(u[2 * p + 1])),
+                                          nd2)),
+                      g0v, g1v);
+          gk[p] = pack_bf16(g0v, g1v);
+          ek[p] = pack_bf16(e0, e1);
+        }
+        const int grp = 8 * w + 4 * cc;   // latents 64 w + 32 cc, in groups of 8
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          *reinterpret_cast<uint4*>(gsm + mn_off(r, grp + v)) =
+              make_uint4(gk[4 * v], gk[4 * v + 1], gk[4 * v + 2], gk[4 * v + 3]);
+          *reinterpret_cast<uint4*>(esm + mn_off(r, grp + v)) =
+              make_uint4(ek[4 * v], ek[4 * v + 1], ek[4 * v + 2], ek[4 * v + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&h_done[slot]);
+      if (t > 0 && !(ok = finish(t - 1))) break;
+    }
+    if (ok && nt > 0) ok = finish(nt - 1);
+    if (!ok) {
+      record_error(err, kErrBwdBRowWait);
+      *abort_flag = 1;
+    }
+    // dQ partial of this chunk (scaled): warpgroup 0, thread r = latent r
+    if (w == 0) {
+      float acc[D];
+#pragma unroll
+      for (int d = 0; d < D; ++d) acc[d] = 0.f;
+      if (ok && nt > 0) {
         ok = warp_all(mbar_wait_sleep(dq_final, 0));
         __syncwarp();
         tc_fence_after();
@@ -996,7 +1459,10 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
   const float c = scale * kLog2e;
   uint32_t* err = (uint32_t*)(ws + L.hdr);
   __nv_bfloat16* zb = (__nv_bfloat16*)(ws + L.zb);
-  float2* stats = (float2*)(ws + L.stats);
+  float4* stats = (float4*)(ws + L.stats);
+  __nv_bfloat16* dy2 = (__nv_bfloat16*)(ws + L.dy2);
+  float* rref = (float*)(ws + L.rref);
+  uint32_t* flags = (uint32_t*)(ws + L.flags);
   float* dzp = (float*)(ws + L.dzp);
   __nv_bfloat16* dzs = (__nv_bfloat16*)(ws + L.dzs);
   __nv_bfloat16* aug = (__nv_bfloat16*)(ws + L.aug);
@@ -1005,15 +1471,15 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
   float* dqp = (float*)(ws + L.dqp);
   cudaError_t e;
 
-  const int64_t n4 = BH * kM * D / 4;
-  bwd_zbf16_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>((const float4*)Z, (uint2*)zb, n4);
+  bwd_prep_kernel<D><<<(unsigned)BH, kM, 0, st>>>(Z, lse, zb, rref, flags);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
-  CUtensorMap mq, mk, mv, mdy, mz, mdz, maug;
+  CUtensorMap mq, mk, mv, mdy, mdy2, mz, mdz, maug;
   if ((e = make_map(&mq, Q, D, kM, q_per_batch ? BH : d.H, kM)) != cudaSuccess) return e;
   if ((e = make_map(&mk, K, D, d.N, BH, kT)) != cudaSuccess) return e;
   if ((e = make_map(&mv, V, D, d.N, BH, kT)) != cudaSuccess) return e;
   if ((e = make_map(&mdy, dY, D, d.N, BH, kT)) != cudaSuccess) return e;
+  if ((e = make_map(&mdy2, dy2, D, d.N, BH, kT)) != cudaSuccess) return e;
   if ((e = make_map(&mz, zb, D, kM, BH, kM)) != cudaSuccess) return e;
   if ((e = make_map(&mdz, dzs, D, kM, BH, kM)) != cudaSuccess) return e;
   if ((e = make_map(&maug, aug, 16, kM, BH, kM)) != cudaSuccess) return e;
@@ -1023,17 +1489,28 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
   e = cudaFuncSetAttribute(tc_bwd_a_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemA);
   if (e != cudaSuccess) return e;
   tc_bwd_a_kernel<D><<<grid, kThr, smemA, st>>>(mq, mk, mdy, mz, (int)d.H, d.N, q_per_batch, c,
-                                                p.tiles_per_bh, p.chunk_tiles, stats, dzp, err);
+                                                p.tiles_per_bh, p.chunk_tiles, rref, stats, dy2,
+                                                flags, dzp, err);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
   bwd_mid_kernel<D><<<(unsigned)BH, kM, 0, st>>>(dzp, p.chunks, Z, lse, dzs, (uint32_t*)aug,
-                                                 params, lse2);
+                                                 flags, params, lse2);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
-  const int smemB = BLayout<D>::BYTES + 1024;
-  e = cudaFuncSetAttribute(tc_bwd_b_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemB);
+  // each head runs in exactly one of the two pass-B kernels (params.y)
+  const int smemF = BFLayout<D>::BYTES + 1024;
+  e = cudaFuncSetAttribute(tc_bwd_b_fast_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smemF);
   if (e != cudaSuccess) return e;
-  tc_bwd_b_kernel<D><<<grid, kThr, smemB, st>>>(
+  tc_bwd_b_fast_kernel<D><<<grid, kThr, smemF, st>>>(
+      mq, mk, mv, mdy2, mz, mdz, maug, (int)d.H, d.N, q_per_batch, c, scale, p.tiles_per_bh,
+      p.chunk_tiles, stats, params, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, dqp, err);
+  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+  const int smemB = BLayout<D>::BYTES + 1024;
+  e = cudaFuncSetAttribute(tc_bwd_b_exact_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smemB);
+  if (e != cudaSuccess) return e;
+  tc_bwd_b_exact_kernel<D><<<grid, kThr, smemB, st>>>(
       mq, mk, mv, mdy, mz, mdz, maug, (int)d.H, d.N, q_per_batch, c, scale, p.tiles_per_bh,
       p.chunk_tiles, stats, params, lse2, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, dqp, err);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;

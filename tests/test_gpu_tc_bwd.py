@@ -107,3 +107,26 @@ def test_tc_bwd_bitwise_reproducible():
     torch.cuda.synchronize()
     for u, v in zip(a, b):
         assert torch.equal(u, v)
+
+
+def test_tc_bwd_mixed_heads_fast_and_exact():
+    # Head 1's latents are scaled up so its lse spreads far beyond 64 (log2
+    # units) and it takes the exact form, while head 0 takes the
+    # one-exponential form, in the same launch.
+    B, H, N, M, D = 2, 2, 1500, 128, 32
+    s = 1.0 / math.sqrt(D)
+    x = make_inputs(B, H, N, M, D, dtype=BF16, seed=15, with_dy=True)
+    x["Q"][1] = (x["Q"][1].float() * 40.0).to(BF16)
+    g = {k: v.to(DEV) for k, v in x.items()}
+    Y, Z, lse = fl.flare_fwd(g["Q"], g["K"], g["V"], s, save=True)
+    spread = (lse.float().amax(-1) - lse.float().amin(-1)) * math.log2(math.e)
+    assert float(spread[:, 1].min()) > 64.0 and float(spread[:, 0].max()) < 64.0
+    ws = fl.alloc_workspace(fl.FLARE_OP_BWD, B, H, N, M, D, BF16, DEV)
+    dQ, dK, dV = fl.flare_bwd(g["Q"], g["K"], g["V"], g["dY"], Z, lse, s, workspace=ws)
+    assert fl.device_status(ws) == 0
+    dQo, dKo, dVo = oracle.flare_bwd(x["Q"], x["K"], x["V"], x["dY"], s)
+    for hh in (0, 1):
+        chk = assert_close if hh == 0 else (lambda a, b, dt, w: assert_close_scaled(a, b, w))
+        chk(dV[:, hh], dVo[:, hh], BF16, f"dV head {hh}")
+        chk(dK[:, hh], dKo[:, hh], BF16, f"dK head {hh}")
+        chk(dQ[hh], dQo[hh], BF16, f"dQ head {hh}")
