@@ -42,9 +42,14 @@ constexpr int kEncStages = 8;
 constexpr int kDecStages = 6;
 constexpr float kRescaleTau = 8.0f;   // log2 units: rescale only when the max grows by > 2^8
 constexpr float kRedoTau = 64.0f;     // log2 units: past 2^64 above m_ref a tile is recomputed
-// Every kPolyEvery-th pair of exponentials is computed on the FMA pipe
-// (exp2_fma) instead of the MUFU, which is the unit that bounds both kernels.
-constexpr int kPolyEvery = 0;
+// Every k-th pair of exponentials is computed on the FMA pipe (exp2_fma)
+// instead of the MUFU, which is the unit that bounds both kernels.  The
+// encode (four softmax warps per SM sub-partition) gains from moving every
+// fourth pair (1.44 -> 1.36 ms on the million-token workload); the decode
+// (two per sub-partition, close to its register budget) loses, so it keeps
+// every exponential on the MUFU.
+constexpr int kEncPolyEvery = 4;
+constexpr int kDecPolyEvery = 0;
 constexpr int kMinSmemBytes = 120 * 1024;  // keeps one CTA (and its TMEM) per SM
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -327,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 2)
               if (t >= nvalid) a[t] = __float_as_uint(-INFINITY);
           }
           max_fold32(a, mf);
-          exp_pack32<kPolyEvery>(a, c, neg, pa, sf);
+          exp_pack32<kEncPolyEvery>(a, c, neg, pa, sf);
         }
         {
           uint32_t a[16];
@@ -408,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 2)
               if (t >= nvalid) a[t] = __float_as_uint(-INFINITY);
           }
           uint32_t pk[16];
-          exp_pack32<kPolyEvery>(a, c, neg, pk, sf);
+          exp_pack32<kEncPolyEvery>(a, c, neg, pk, sf);
           tmem_st16(tS, pk);
         }
         {
@@ -675,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld_dep(a[k & 1]);
         if (k + 1 < NC) tmem_ld32(tR + chunk_col(k + 1), a[(k + 1) & 1]);
         uint32_t pk[16];
-        exp_pack32<kPolyEvery>(a[k & 1], c, neg, pk, sf);
+        exp_pack32<kDecPolyEvery>(a[k & 1], c, neg, pk, sf);
         tmem_st16(tR + p_col(k), pk);
       }
       tmem_wait_st();
