@@ -119,7 +119,7 @@ struct ALayout {
   static constexpr int ONE_OFF = Z_OFF + M * RB;  // second N block of Y's B operand
   static constexpr int ST_OFF = ONE_OFF + M * RB;   // stages: K tile, dY tile
   static constexpr int BAR_OFF = ST_OFF + kAStages * 2 * TILE;
-  static constexpr int NBARS = 2 * kAStages + 1 + 8 + 2;
+  static constexpr int NBARS = 2 * kAStages + 1 + 8 + 4 + 1 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
 };
@@ -154,8 +154,9 @@ __global__ void __launch_bounds__(kThr, 1)
   uint64_t* p_full = s_full + 2;    // [w] P written (TMEM and shared memory)
   uint64_t* y_full = p_full + 2;    // [w] Y = P Z complete
   uint64_t* a_done = y_full + 2;    // [w] Y read, dY' written: TMEM columns free
-  uint64_t* dz_final = a_done + 2;
-  uint64_t* drain = dz_final + 1;
+  uint64_t* dz_done = a_done + 2;   // [2 w + b] dZ of warpgroup w's tile in P buffer b complete
+  uint64_t* dz_final = dz_done + 4;
+  uint64_t* drain = dz_final + 1;   // [2]: one per issuing thread
   uint32_t* tmem_slot = (uint32_t*)(smem + L::MISC_OFF);
   volatile int* abort_flag = (volatile int*)(smem + L::MISC_OFF + 4);
 
@@ -179,7 +180,7 @@ __global__ void __launch_bounds__(kThr, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kAStages; ++s) {
       mbar_init(&st_full[s], 1);
-      mbar_init(&st_empty[s], 1);
+      mbar_init(&st_empty[s], 2);   // K read by S (warp 9), dY' by dZ (warp 10)
     }
     mbar_init(qz_full, 1);
     for (int w = 0; w < 2; ++w) {
@@ -188,8 +189,10 @@ __global__ void __launch_bounds__(kThr, 1)
       mbar_init(&y_full[w], 1);
       mbar_init(&a_done[w], 128);
     }
+    for (int k = 0; k < 4; ++k) mbar_init(&dz_done[k], 1);
     mbar_init(dz_final, 1);
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -231,7 +234,10 @@ __global__ void __launch_bounds__(kThr, 1)
           mbar_wait_sleep(&st_full[i % kAStages], (uint32_t)((i / kAStages) & 1));
         mbar_wait_sleep(qz_full, 0);
       }
-    } else if (warp == kWMma) {
+    } else if (warp == kWMma || warp == kWMma + 1) {
+      // Two issuing threads: warp 9 issues S (it waits on TMA tiles), warp
+      // 10 issues Y and dZ (they wait on the row warps), so neither kind of
+      // wait delays the other kind of product.
       if (lane == 0) {
         constexpr uint32_t idS = idesc_bf16_f32(128, M, 0, 0);
         constexpr uint32_t idY = idesc_bf16_f32(128, D + 16, 0, 1);   // N = [Z | e0]
@@ -252,70 +258,76 @@ __global__ void __launch_bounds__(kThr, 1)
         constexpr uint32_t kP16 = (uint32_t)L::PBUF >> 4;
         const int nt = (int)ntiles;
         bool ok = mbar_wait_sleep(qz_full, 0);
-        auto issue_S = [&](int i) -> bool {
-          const int w = i & 1;
-          const int s = i % kAStages;
-          if (!mbar_wait_sleep(&st_full[s], (uint32_t)((i / kAStages) & 1))) return false;
-          tc_fence_after();
-          const uint32_t so = (uint32_t)(s * 2) * kTile16;
+        if (warp == kWMma) {
+          // S(i) into warpgroup (i & 1)'s S columns once its tile i - 2 has
+          // been read (p_full) and tile i's K is in shared memory
+          for (int i = 0; ok && i < nt; ++i) {
+            const int w = i & 1;
+            const int s = i % kAStages;
+            if (i >= 2 && !mbar_wait_sleep(&p_full[w], (uint32_t)(((i - 2) >> 1) & 1))) {
+              ok = false;
+              break;
+            }
+            if (!mbar_wait_sleep(&st_full[s], (uint32_t)((i / kAStages) & 1))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t so = (uint32_t)(s * 2) * kTile16;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + w * R, dSt + so + 2 * kk, dQk + 2 * kk, idS, kk > 0);
-          mma_commit(&s_full[w]);
-          return true;
-        };
-        // Y = P [Z | e0] with P read from shared memory as a K-major operand
-        // (token rows, latents contiguous: the same bytes dZ reads MN-major)
-        auto issue_Y = [&](int i) -> bool {
-          const int w = i & 1;
-          const int j = i >> 1;
-          if (!mbar_wait_sleep(&p_full[w], (uint32_t)(j & 1))) return false;
-          tc_fence_after();
-          const uint32_t po = (uint32_t)(2 * w + (j & 1)) * kP16;
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tmem + w * R, dSt + so + 2 * kk, dQk + 2 * kk, idS, kk > 0);
+            mma_commit(&s_full[w]);
+            mma_commit(&st_empty[s]);
+            if (*abort_flag) ok = false;
+          }
+        } else {
+          // Y = P [Z | e0] with P read from shared memory as a K-major
+          // operand (token rows, latents contiguous: the same bytes dZ reads
+          // MN-major); dZ of a tile is issued one tile later, so a warpgroup
+          // waiting for its Y never waits behind the other one's dY work.
+          auto issue_dZ = [&](int i) -> bool {
+            const int w = i & 1;
+            const int j = i >> 1;
+            const int s = i % kAStages;
+            if (!mbar_wait_sleep(&a_done[w], (uint32_t)(j & 1))) return false;
+            tc_fence_after();
+            const uint32_t po = (uint32_t)(2 * w + (j & 1)) * kP16;
+            const uint32_t so = (uint32_t)(s * 2 + 1) * kTile16;
 #pragma unroll
-          for (int kk = 0; kk < M / 16; ++kk)
-            mma_ss(tmem + TY + YC * w, dPk + po + (kk >> 2) * (kMnLbo >> 4) + (kk & 3) * 2,
-                   dZm + kk * kRow16, idY, kk > 0);
-          mma_commit(&y_full[w]);
-          return true;
-        };
-        auto issue_dZ = [&](int i) -> bool {
-          const int w = i & 1;
-          const int j = i >> 1;
-          const int s = i % kAStages;
-          if (!mbar_wait_sleep(&a_done[w], (uint32_t)(j & 1))) return false;
-          tc_fence_after();
-          const uint32_t po = (uint32_t)(2 * w + (j & 1)) * kP16;
-          const uint32_t so = (uint32_t)(s * 2 + 1) * kTile16;
+            for (int kk = 0; kk < kT / 16; ++kk)
+              mma_ss(tmem + TDZ, dPm + po + kk * (kMnKStep >> 4), dStm + so + kk * kRow16, idZ,
+                     (i > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&st_empty[s]);
+            mma_commit(&dz_done[2 * w + (j & 1)]);
+            return true;
+          };
+          for (int i = 0; ok && i < nt; ++i) {
+            const int w = i & 1;
+            const int j = i >> 1;
+            if (!mbar_wait_sleep(&p_full[w], (uint32_t)(j & 1))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t po = (uint32_t)(2 * w + (j & 1)) * kP16;
 #pragma unroll
-          for (int kk = 0; kk < kT / 16; ++kk)
-            mma_ss(tmem + TDZ, dPm + po + kk * (kMnKStep >> 4), dStm + so + kk * kRow16, idZ,
-                   (i > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&st_empty[s]);
-          return true;
-        };
-        // S of tile i + 2 goes into warpgroup (i & 1)'s S columns as soon as
-        // its P is written; dZ of a tile is issued one tile later, so the
-        // issuer never waits on one warpgroup while the other has work ready.
-        // P buffers alternate per warpgroup: dZ(i) is issued before S(i + 4),
-        // so S(i + 4) completing implies dZ(i), and with it the last read of
-        // the buffer P(i + 4) reuses.
-        if (ok && nt > 0) ok = issue_S(0);
-        if (ok && nt > 1) ok = issue_S(1);
-        for (int i = 0; ok && i < nt; ++i) {
-          ok = issue_Y(i);
-          if (ok && i + 2 < nt) ok = issue_S(i + 2);
-          if (ok && i >= 1) ok = issue_dZ(i - 1);
-          if (*abort_flag) ok = false;
+            for (int kk = 0; kk < M / 16; ++kk)
+              mma_ss(tmem + TY + YC * w, dPk + po + (kk >> 2) * (kMnLbo >> 4) + (kk & 3) * 2,
+                     dZm + kk * kRow16, idY, kk > 0);
+            mma_commit(&y_full[w]);
+            if (i >= 1) ok = issue_dZ(i - 1);
+            if (*abort_flag) ok = false;
+          }
+          if (ok && nt > 0) ok = issue_dZ(nt - 1);
+          mma_commit(dz_final);
         }
-        if (ok && nt > 0) ok = issue_dZ(nt - 1);
         if (!ok) {
           record_error(err, kErrBwdAMmaWait);
           *abort_flag = 1;
         }
-        mma_commit(dz_final);
-        mma_commit(drain);
-        mbar_wait_sleep(drain, 0);
+        mma_commit(drain + (warp - kWMma));
+        mbar_wait_sleep(drain + (warp - kWMma), 0);
       }
     }
   } else {
@@ -332,7 +344,10 @@ __global__ void __launch_bounds__(kThr, 1)
       const int s = (int)(i % kAStages);
       const int64_t tok = (tile0 + i) * kT + r;
       uint8_t* pbuf = smem + L::P_OFF + (2 * w + (j & 1)) * L::PBUF;
-      if (!warp_all(mbar_wait_sleep(&s_full[w], (uint32_t)(j & 1)) && !*abort_flag)) {
+      // the P buffer of tile j was last read by the dZ of tile j - 2
+      if (!warp_all(mbar_wait_sleep(&s_full[w], (uint32_t)(j & 1)) &&
+                    (j < 2 || mbar_wait_sleep(&dz_done[2 * w + (j & 1)], (uint32_t)(((j - 2) >> 1) & 1))) &&
+                    !*abort_flag)) {
         ok = false;
         break;
       }
@@ -1038,7 +1053,7 @@ struct BFLayout {
   static constexpr int K_OFF = ONES_OFF + kT * 32;     // K ring
   static constexpr int VD_OFF = K_OFF + KST * TILE;    // (V, dY'') ring
   static constexpr int BAR_OFF = VD_OFF + VST * 2 * TILE;
-  static constexpr int NBARS = 2 * KST + 2 * VST + 1 + 2 * NSLOT + 1 + 1 + 1 + 1;
+  static constexpr int NBARS = 2 * KST + 2 * VST + 1 + 2 * NSLOT + 2 + 1 + 1 + 1 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
 };
@@ -1077,10 +1092,11 @@ __global__ void __launch_bounds__(kThr, 1)
   uint64_t* c_full = v_empty + VST;
   uint64_t* h_full = c_full + 1;        // [slot] S and U of a half in TMEM
   uint64_t* h_done = h_full + NS;       // [slot] the half's rows read, G and e in shared memory
-  uint64_t* tile_done = h_done + NS;    // dK, dV of a tile final; its G, e buffers free
+  uint64_t* t_ready = h_done + NS;      // [t & 1] both halves of tile t in shared memory
+  uint64_t* tile_done = t_ready + 2;    // dK, dV of a tile final; its G, e buffers free
   uint64_t* acc_empty = tile_done + 1;  // dK, dV accumulators read back
   uint64_t* dq_final = acc_empty + 1;
-  uint64_t* drain = dq_final + 1;
+  uint64_t* drain = dq_final + 1;       // [2]: one per issuing thread
   uint32_t* tmem_slot = (uint32_t*)(smem + L::MISC_OFF);
   volatile int* abort_flag = (volatile int*)(smem + L::MISC_OFF + 4);
 
@@ -1115,10 +1131,13 @@ __global__ void __launch_bounds__(kThr, 1)
       mbar_init(&h_full[k], 1);
       mbar_init(&h_done[k], 128);
     }
+    mbar_init(&t_ready[0], 1);
+    mbar_init(&t_ready[1], 1);
     mbar_init(tile_done, 1);
     mbar_init(acc_empty, 256);
     mbar_init(dq_final, 1);
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -1175,7 +1194,10 @@ __global__ void __launch_bounds__(kThr, 1)
           mbar_wait_sleep(&v_full[t % VST], (uint32_t)((t / VST) & 1));
         mbar_wait_sleep(c_full, 0);
       }
-    } else if (warp == kWMma) {
+    } else if (warp == kWMma || warp == kWMma + 1) {
+      // Two issuing threads: warp 9 keeps the slot ring full (S and U of
+      // each half; it waits on TMA tiles), warp 10 issues each tile's output
+      // products (they wait on the row warps and the accumulators).
       if (lane == 0) {
         constexpr uint32_t idH = idesc_bf16_f32(128, 64, 0, 0);   // a half's S or U
         constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);    // dK, dV (A K-major)
@@ -1234,46 +1256,53 @@ __global__ void __launch_bounds__(kThr, 1)
           if (hf == 1) mma_commit(&v_empty[vb]);   // V and dY'' of tile t read by both halves
           return true;
         };
-        for (int k = 0; ok && k < NS && k < nh; ++k) ok = issue_H(k);
-        for (int k = 0; ok && k < nh; ++k) {
-          // half k read: its slot takes half k + 3 at once (no MMA reads TMEM slots)
-          if (!mbar_wait_sleep(&h_done[k % NS], (uint32_t)((k / NS) & 1))) {
-            ok = false;
-            break;
+        if (warp == kWMma) {
+          for (int k = 0; ok && k < NS && k < nh; ++k) ok = issue_H(k);
+          for (int k = 0; ok && k < nh; ++k) {
+            // half k read: its slot takes half k + 3 at once (no MMA reads TMEM slots)
+            if (!mbar_wait_sleep(&h_done[k % NS], (uint32_t)((k / NS) & 1))) {
+              ok = false;
+              break;
+            }
+            if (k & 1) mbar_arrive(&t_ready[(k >> 1) & 1]);   // tile k / 2 in shared memory
+            if (k + NS < nh && !(ok = issue_H(k + NS))) break;
+            if (*abort_flag) ok = false;
           }
-          if (k + NS < nh && !(ok = issue_H(k + NS))) break;
-          if ((k & 1) == 0) continue;
-          // both halves of tile t in shared memory: dK, dV, dQ of the tile
-          const int t = k >> 1;
-          if (t > 0 && !mbar_wait_sleep(acc_empty, (uint32_t)((t - 1) & 1))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t go = (uint32_t)(t & 1) * kBuf16;
-          const uint32_t eo = go + 2 * kBuf16;
-          const uint32_t ko = (uint32_t)(t % KST) * kTile16;
-          // three independent accumulator chains, interleaved
-          static_assert(M == kT, "dK/dV and dQ take the same number of K-steps");
+        } else {
+          for (int t = 0; ok && t < nt; ++t) {
+            // both halves of tile t in shared memory and the accumulators free:
+            // dK, dV, dQ of the tile
+            if (!mbar_wait_sleep(&t_ready[t & 1], (uint32_t)((t >> 1) & 1)) ||
+                (t > 0 && !mbar_wait_sleep(acc_empty, (uint32_t)((t - 1) & 1)))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t go = (uint32_t)(t & 1) * kBuf16;
+            const uint32_t eo = go + 2 * kBuf16;
+            const uint32_t ko = (uint32_t)(t % KST) * kTile16;
+            // three independent accumulator chains, interleaved
+            static_assert(M == kT, "dK/dV and dQ take the same number of K-steps");
 #pragma unroll
-          for (int kk = 0; kk < M / 16; ++kk) {
-            const uint32_t ak = (kk >> 2) * (kMnLbo >> 4) + (kk & 3) * 2;   // 16 latents
-            mma_ss(tmem + TDK, dGk + go + ak, dQm + kk * kRow16, idO, kk > 0);
-            mma_ss(tmem + TDV, dGk + eo + ak, dDZm + kk * kRow16, idO, kk > 0);
-            mma_ss(tmem + TDQ, dGm + go + kk * (kMnKStep >> 4), dKm + ko + kk * kRow16, idQ,
-                   (t > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < M / 16; ++kk) {
+              const uint32_t ak = (kk >> 2) * (kMnLbo >> 4) + (kk & 3) * 2;   // 16 latents
+              mma_ss(tmem + TDK, dGk + go + ak, dQm + kk * kRow16, idO, kk > 0);
+              mma_ss(tmem + TDV, dGk + eo + ak, dDZm + kk * kRow16, idO, kk > 0);
+              mma_ss(tmem + TDQ, dGm + go + kk * (kMnKStep >> 4), dKm + ko + kk * kRow16, idQ,
+                     (t > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(tile_done);
+            mma_commit(&k_empty[t % KST]);
+            if (*abort_flag) ok = false;
           }
-          mma_commit(tile_done);
-          mma_commit(&k_empty[t % KST]);
-          if (*abort_flag) ok = false;
+          mma_commit(dq_final);
         }
         if (!ok) {
           record_error(err, kErrBwdBMmaWait);
           *abort_flag = 1;
         }
-        mma_commit(dq_final);
-        mma_commit(drain);
-        mbar_wait_sleep(drain, 0);
+        mma_commit(drain + (warp - kWMma));
+        mbar_wait_sleep(drain + (warp - kWMma), 0);
       }
     }
   } else {
