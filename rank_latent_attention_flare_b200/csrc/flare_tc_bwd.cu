@@ -1028,32 +1028,32 @@ __global__ void __launch_bounds__(kThr, 1)
 //   dK = s G Q,  dV = e dZ'',  dQ = s G^T K.
 // Work unit: half a tile (128 tokens x 64 latents; warpgroup w takes latent
 // half w of every tile).  S and U of a half go to one of three TMEM slots;
-// the row warps write G and e only to shared memory (128-byte swizzled,
-// token rows, latents contiguous), from where dK = G Q and dV = e dZ'' read
-// them as K-major operands and dQ = G^T K as an MN-major one.  A slot is
-// therefore free as soon as its rows are read, and the output products of a
-// tile are issued once both halves are in.
+// the row warps write G and e (bf16) back over the slot's S and U columns,
+// where dK += G Q and dV += e dZ'' read them, and G also to shared memory
+// (128-byte swizzled, token rows, latents contiguous) for dQ += G^T K.  The
+// tensor cores' shared-memory operand traffic bounds this kernel, so every
+// operand that can come from TMEM does (G and e for dK / dV, the ones of the
+// extra K-step).  Warp 9 keeps the slot ring full; warp 10 issues dK / dV of
+// each half (then the slot is refilled) and dQ of each tile.
 
 template <int D>
 struct BFLayout {
   static constexpr int M = kM;
   static constexpr int NSLOT = 3;
-  static constexpr int KST = 4;                       // K tiles: held until the tile's dQ
-  static constexpr int VST = 2;                       // V, dY'' tiles: until its U products
+  static constexpr int KST = 6;                       // K tiles: held until the tile's dQ
+  static constexpr int VST = 4;                       // V, dY'' tiles: until its U products
   static constexpr int RB = 2 * D;
   static constexpr int TILE = kT * RB;
   static constexpr int GBUF = kT * M * 2;              // 32 KB
   static constexpr int G_OFF = 0;                      // two G buffers (tile parity)
-  static constexpr int E_OFF = 2 * GBUF;               // two e buffers (tile parity)
-  static constexpr int Q_OFF = 4 * GBUF;
+  static constexpr int Q_OFF = 2 * GBUF;
   static constexpr int Z_OFF = Q_OFF + M * RB;
   static constexpr int DZ_OFF = Z_OFF + M * RB;
   static constexpr int AUG_OFF = DZ_OFF + M * RB;      // [M][16] bf16, 32-byte rows
-  static constexpr int ONES_OFF = AUG_OFF + M * 32;    // [128][16] bf16
-  static constexpr int K_OFF = ONES_OFF + kT * 32;     // K ring
+  static constexpr int K_OFF = AUG_OFF + M * 32;       // K ring
   static constexpr int VD_OFF = K_OFF + KST * TILE;    // (V, dY'') ring
   static constexpr int BAR_OFF = VD_OFF + VST * 2 * TILE;
-  static constexpr int NBARS = 2 * KST + 2 * VST + 1 + 2 * NSLOT + 2 + 1 + 1 + 1 + 2;
+  static constexpr int NBARS = 2 * KST + 2 * VST + 1 + 3 * NSLOT + 1 + 1 + 1 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
 };
@@ -1079,8 +1079,9 @@ __global__ void __launch_bounds__(kThr, 1)
   constexpr int TDK = NS * HC;         // dK accumulator (token lanes)
   constexpr int TDV = TDK + D;         // dV accumulator (token lanes)
   constexpr int TDQ = TDV + D;         // dQ accumulator (latent lanes)
+  constexpr int TONE = TDQ + D;        // ones of the extra K-step (8 columns of bf16 pairs)
   constexpr uint32_t NCOLS = 512;
-  static_assert(TDQ + D <= 512, "TMEM budget");
+  static_assert(TONE + 8 <= 512, "TMEM budget");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -1091,9 +1092,9 @@ __global__ void __launch_bounds__(kThr, 1)
   uint64_t* v_empty = v_full + VST;
   uint64_t* c_full = v_empty + VST;
   uint64_t* h_full = c_full + 1;        // [slot] S and U of a half in TMEM
-  uint64_t* h_done = h_full + NS;       // [slot] the half's rows read, G and e in shared memory
-  uint64_t* t_ready = h_done + NS;      // [t & 1] both halves of tile t in shared memory
-  uint64_t* tile_done = t_ready + 2;    // dK, dV of a tile final; its G, e buffers free
+  uint64_t* h_done = h_full + NS;       // [slot] the half's rows read; G, e written back
+  uint64_t* r_free = h_done + NS;       // [slot] dK / dV of the half complete: slot free
+  uint64_t* tile_done = r_free + NS;    // dK, dV of a tile final; its G buffer free
   uint64_t* acc_empty = tile_done + 1;  // dK, dV accumulators read back
   uint64_t* dq_final = acc_empty + 1;
   uint64_t* drain = dq_final + 1;       // [2]: one per issuing thread
@@ -1109,14 +1110,6 @@ __global__ void __launch_bounds__(kThr, 1)
   const float2 prm = params[bh];
   if (prm.y == 0.f) return;   // head served by tc_bwd_b_exact_kernel
 
-  for (int t = threadIdx.x; t < kT; t += blockDim.x) {
-    // ones in columns 0-2 of every row of the extra K-step's A operand (32-byte swizzle)
-    uint8_t* ones = smem + L::ONES_OFF;
-    const int x0 = (t >> 2) & 1;
-    *reinterpret_cast<uint4*>(ones + t * 32 + x0 * 16) = make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u);
-    *reinterpret_cast<uint4*>(ones + t * 32 + (x0 ^ 1) * 16) = make_uint4(0u, 0u, 0u, 0u);
-  }
-  fence_proxy_async_smem();
   if (threadIdx.x == 0) {
     for (int k = 0; k < KST; ++k) {
       mbar_init(&k_full[k], 1);
@@ -1130,9 +1123,8 @@ __global__ void __launch_bounds__(kThr, 1)
     for (int k = 0; k < NS; ++k) {
       mbar_init(&h_full[k], 1);
       mbar_init(&h_done[k], 128);
+      mbar_init(&r_free[k], 1);
     }
-    mbar_init(&t_ready[0], 1);
-    mbar_init(&t_ready[1], 1);
     mbar_init(tile_done, 1);
     mbar_init(acc_empty, 256);
     mbar_init(dq_final, 1);
@@ -1146,6 +1138,15 @@ __global__ void __launch_bounds__(kThr, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (warp < 4) {
+    // the A operand of the extra K-step: ones in columns 0-2 of every row
+    uint32_t one[8] = {0x3F803F80u, 0x00003F80u, 0u, 0u, 0u, 0u, 0u, 0u};
+    tmem_st8(tmem + ((uint32_t)(warp * 32) << 16) + TONE, one);
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
 
   if (warp >= 8) {
     regs_release<kRegsPro>();
@@ -1196,17 +1197,16 @@ __global__ void __launch_bounds__(kThr, 1)
       }
     } else if (warp == kWMma || warp == kWMma + 1) {
       // Two issuing threads: warp 9 keeps the slot ring full (S and U of
-      // each half; it waits on TMA tiles), warp 10 issues each tile's output
-      // products (they wait on the row warps and the accumulators).
+      // each half; it waits on TMA tiles), warp 10 issues dK / dV of each
+      // half and dQ of each tile (they wait on the row warps).
       if (lane == 0) {
         constexpr uint32_t idH = idesc_bf16_f32(128, 64, 0, 0);   // a half's S or U
-        constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);    // dK, dV (A K-major)
+        constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);    // dK, dV (A in TMEM)
         constexpr uint32_t idQ = idesc_bf16_f32(128, D, 1, 1);    // dQ (A MN-major)
         const uint32_t q_addr = smem_u32(smem + L::Q_OFF);
         const uint32_t z_addr = smem_u32(smem + L::Z_OFF);
         const uint32_t dz_addr = smem_u32(smem + L::DZ_OFF);
         const uint32_t aug_addr = smem_u32(smem + L::AUG_OFF);
-        const uint32_t ones_addr = smem_u32(smem + L::ONES_OFF);
         const uint32_t k0 = smem_u32(smem + L::K_OFF);
         const uint32_t v0 = smem_u32(smem + L::VD_OFF);
         const uint32_t g0 = smem_u32(smem + L::G_OFF);
@@ -1217,12 +1217,10 @@ __global__ void __launch_bounds__(kThr, 1)
         const uint64_t dQk = smem_desc(q_addr, 16, 8 * RB, SW);       // latent rows, K-major
         const uint64_t dZk = smem_desc(z_addr, 16, 8 * RB, SW);
         const uint64_t dDZk = smem_desc(dz_addr, 16, 8 * RB, SW);
-        const uint64_t dOnes = smem_desc(ones_addr, 16, 256, kSw32);
         const uint64_t dAug = smem_desc(aug_addr, 16, 256, kSw32);
         const uint64_t dQm = smem_desc(q_addr, M * RB, 8 * RB, SW);   // latent rows, MN-major
         const uint64_t dDZm = smem_desc(dz_addr, M * RB, 8 * RB, SW);
         const uint64_t dKm = smem_desc(k0, L::TILE, 8 * RB, SW);      // K tile, MN-major
-        const uint64_t dGk = smem_desc(g0, 16, kMnSbo, kSw128);       // G or e, K-major
         const uint64_t dGm = smem_desc(g0, kMnLbo, kMnSbo, kSw128);   // G, MN-major
         constexpr uint32_t kTile16 = (uint32_t)L::TILE >> 4;
         constexpr uint32_t kRow16 = (uint32_t)RB;                     // 16 rows >> 4
@@ -1251,48 +1249,54 @@ __global__ void __launch_bounds__(kThr, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             mma_ss(base + 64, dV0 + vo + 2 * kk, dDZk + ro + 2 * kk, idH, 1u);
-          mma_ss(base + 64, dOnes, dAug + (uint32_t)(2 * 64 * hf), idH, 1u);
+          mma_ts(base + 64, tmem + TONE, dAug + (uint32_t)(2 * 64 * hf), idH, 1u);
           mma_commit(&h_full[k % NS]);
           if (hf == 1) mma_commit(&v_empty[vb]);   // V and dY'' of tile t read by both halves
           return true;
         };
         if (warp == kWMma) {
           for (int k = 0; ok && k < NS && k < nh; ++k) ok = issue_H(k);
-          for (int k = 0; ok && k < nh; ++k) {
-            // half k read: its slot takes half k + 3 at once (no MMA reads TMEM slots)
-            if (!mbar_wait_sleep(&h_done[k % NS], (uint32_t)((k / NS) & 1))) {
+          for (int k = 0; ok && k + NS < nh; ++k) {
+            // dK / dV of half k done: its slot takes half k + 3
+            if (!mbar_wait_sleep(&r_free[k % NS], (uint32_t)((k / NS) & 1))) {
               ok = false;
               break;
             }
-            if (k & 1) mbar_arrive(&t_ready[(k >> 1) & 1]);   // tile k / 2 in shared memory
-            if (k + NS < nh && !(ok = issue_H(k + NS))) break;
+            if (!(ok = issue_H(k + NS))) break;
             if (*abort_flag) ok = false;
           }
         } else {
-          for (int t = 0; ok && t < nt; ++t) {
-            // both halves of tile t in shared memory and the accumulators free:
-            // dK, dV, dQ of the tile
-            if (!mbar_wait_sleep(&t_ready[t & 1], (uint32_t)((t >> 1) & 1)) ||
-                (t > 0 && !mbar_wait_sleep(acc_empty, (uint32_t)((t - 1) & 1)))) {
+          for (int k = 0; ok && k < nh; ++k) {
+            const int slot = k % NS;
+            const int t = k >> 1;
+            const int hf = k & 1;
+            if (!mbar_wait_sleep(&h_done[slot], (uint32_t)((k / NS) & 1)) ||
+                (hf == 0 && t > 0 && !mbar_wait_sleep(acc_empty, (uint32_t)((t - 1) & 1)))) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t go = (uint32_t)(t & 1) * kBuf16;
-            const uint32_t eo = go + 2 * kBuf16;
-            const uint32_t ko = (uint32_t)(t % KST) * kTile16;
-            // three independent accumulator chains, interleaved
-            static_assert(M == kT, "dK/dV and dQ take the same number of K-steps");
+            // dK += G Q, dV += e dZ'' over the half's 64 latents (A from TMEM)
+            const uint32_t base = tmem + HC * (uint32_t)slot;
 #pragma unroll
-            for (int kk = 0; kk < M / 16; ++kk) {
-              const uint32_t ak = (kk >> 2) * (kMnLbo >> 4) + (kk & 3) * 2;   // 16 latents
-              mma_ss(tmem + TDK, dGk + go + ak, dQm + kk * kRow16, idO, kk > 0);
-              mma_ss(tmem + TDV, dGk + eo + ak, dDZm + kk * kRow16, idO, kk > 0);
-              mma_ss(tmem + TDQ, dGm + go + kk * (kMnKStep >> 4), dKm + ko + kk * kRow16, idQ,
-                     (t > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t rows = (uint32_t)(4 * hf + kk) * kRow16;   // latents 64 hf + 16 kk
+              const uint32_t acc = (hf > 0 || kk > 0) ? 1u : 0u;
+              mma_ts(tmem + TDK, base + 8 * kk, dQm + rows, idO, acc);
+              mma_ts(tmem + TDV, base + 64 + 8 * kk, dDZm + rows, idO, acc);
             }
-            mma_commit(tile_done);
-            mma_commit(&k_empty[t % KST]);
+            mma_commit(&r_free[slot]);
+            if (hf == 1) {
+              // dQ += G^T K over the tile's 128 tokens (G of both halves)
+              const uint32_t go = (uint32_t)(t & 1) * kBuf16;
+              const uint32_t ko = (uint32_t)(t % KST) * kTile16;
+#pragma unroll
+              for (int kk = 0; kk < kT / 16; ++kk)
+                mma_ss(tmem + TDQ, dGm + go + kk * (kMnKStep >> 4), dKm + ko + kk * kRow16, idQ,
+                       (t > 0 || kk > 0) ? 1u : 0u);
+              mma_commit(tile_done);
+              mma_commit(&k_empty[t % KST]);
+            }
             if (*abort_flag) ok = false;
           }
           mma_commit(dq_final);
@@ -1370,11 +1374,10 @@ __global__ void __launch_bounds__(kThr, 1)
       }
       __syncwarp();
       tc_fence_after();
-      // the G / e buffers of tile t were last read by tile t - 2's products,
-      // which completed before this warpgroup's finish(t - 2) returned
+      // the G buffer of tile t was last read by tile t - 2's dQ, which
+      // completed before this warpgroup's finish(t - 2) returned
       const uint32_t tq = tmem + lb + HC * slot;
       uint8_t* gsm = smem + L::G_OFF + (t & 1) * L::GBUF;
-      uint8_t* esm = smem + L::E_OFF + (t & 1) * L::GBUF;
       const uint64_t nR2 = f32x2(nR, nR), nd2 = f32x2(ndd, ndd);
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
@@ -1397,15 +1400,17 @@ __global__ void __launch_bounds__(kThr, 1)
           gk[p] = pack_bf16(g0v, g1v);
           ek[p] = pack_bf16(e0, e1);
         }
+        // G over S columns [16 cc, +16) and e over U columns [64 + 16 cc,
+        // +16), both already read; G also to shared memory for dQ
+        tmem_st16(tq + 16 * cc, gk);
+        tmem_st16(tq + 64 + 16 * cc, ek);
         const int grp = 8 * w + 4 * cc;   // latents 64 w + 32 cc, in groups of 8
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
+        for (int v = 0; v < 4; ++v)
           *reinterpret_cast<uint4*>(gsm + mn_off(r, grp + v)) =
               make_uint4(gk[4 * v], gk[4 * v + 1], gk[4 * v + 2], gk[4 * v + 3]);
-          *reinterpret_cast<uint4*>(esm + mn_off(r, grp + v)) =
-              make_uint4(ek[4 * v], ek[4 * v + 1], ek[4 * v + 2], ek[4 * v + 3]);
-        }
       }
+      tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&h_done[slot]);
