@@ -46,10 +46,11 @@ constexpr float kRedoTau = 64.0f;     // log2 units: past 2^64 above m_ref a til
 // instead of the MUFU, which is the unit that bounds both kernels.  The
 // encode (four softmax warps per SM sub-partition) gains from moving every
 // fourth pair (1.44 -> 1.36 ms on the million-token workload); the decode
-// (two per sub-partition, close to its register budget) loses, so it keeps
-// every exponential on the MUFU.
+// (two per sub-partition, close to its register budget) gains only from the
+// last pair of each 32-column chunk (1.40 -> 1.38 ms; every 4th, 8th, 10th
+// or 12th pair is slower).
 constexpr int kEncPolyEvery = 4;
-constexpr int kDecPolyEvery = 0;
+constexpr int kDecPolyEvery = 16;
 constexpr int kMinSmemBytes = 120 * 1024;  // keeps one CTA (and its TMEM) per SM
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -644,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int64_t j = 0; j < nW; ++j) {
       const int64_t i = 2 * j + w;
       const int64_t tok = (tile0 + i) * kTile + r;
-      if (!warp_all(mbar_wait_sleep(&s_full[w], (uint32_t)(j & 1)) && !*abort_flag)) {
+      if (!warp_all(mbar_wait(&s_full[w], (uint32_t)(j & 1)) && !*abort_flag)) {
         ok = false;
         break;
       }
@@ -686,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[w]);
-      if (!warp_all(mbar_wait_sleep(&y_full[w], (uint32_t)(j & 1)))) {
+      if (!warp_all(mbar_wait(&y_full[w], (uint32_t)(j & 1)))) {
         ok = false;
         break;
       }
