@@ -521,7 +521,7 @@ def run_reference(args, rank, world):
         return
     w = WORKLOAD
     import oracle
-    budget = max(30.0, args.ref_seconds)
+    budget = max(1.0, args.ref_seconds)
     per_step = budget / (args.steps + args.warmup)
     _, _, cores, n_s, h_s = oracle_sample_rate(per_step)
     x = make_inputs(1, h_s, n_s, w.M, w.D, dtype=w.torch_dtype, seed=0)
