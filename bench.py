@@ -71,7 +71,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
@@ -353,11 +353,16 @@ def run_ours(args, rank, world, local):
     roof = roofline_entry(kernel_ms, peaks, peak_kind, w)
 
     rows = None
+    context = None
     if not args.no_rows:
         del Y, ws
         g.clear()
         torch.cuda.empty_cache()
         rows = time_other_rows(dev, peaks, peak_kind, seed=rank)
+        try:
+            context = time_sdpa_context(dev, seed=rank)
+        except (RuntimeError, ValueError) as e:   # a torch build without a kernel for this shape
+            context = {"what": "two torch scaled_dot_product_attention calls", "error": str(e)[:200]}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -380,6 +385,7 @@ def run_ours(args, rank, world, local):
         "kernel_ms": {k: round(v, 4) for k, v in kernel_ms.items()},
         "roofline": roof,
         "rows": rows,
+        "context_sdpa": context,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": 3 * args.steps * world,
@@ -497,6 +503,41 @@ def _time_fwd_bwd(dev, peaks, peak_kind, timed, seed):
         "bwd_roofline": _row_roofline(ms_b, 2.0 * u * w.M, 20.0 * u * w.M * w.D,
                                       5.0 * u * w.D * 2, peaks, peak_kind)}
     return rows
+
+
+def time_sdpa_context(dev, w=WORKLOAD, iters: int = 5, seed: int = 0):
+    """Prior-art context, not a target: the pages' expression of FLARE as two
+    stock attention calls (encode SDPA(Q, K, V), decode SDPA(K, Q, Z)) with
+    torch.nn.functional.scaled_dot_product_attention on the same device and
+    workload, CUDA-event timed (median of `iters` after 2 warm-ups)."""
+    import torch
+    import torch.nn.functional as F
+    x = make_inputs(w.B, w.H, w.N, w.M, w.D, dtype=w.torch_dtype, seed=seed)
+    Q = x["Q"].to(dev).unsqueeze(0).expand(w.B, w.H, w.M, w.D).contiguous()
+    K = x["K"].to(dev)
+    V = x["V"].to(dev)
+    st = torch.cuda.current_stream()
+
+    def two_calls():
+        Z = F.scaled_dot_product_attention(Q, K, V, scale=w.scale)
+        return F.scaled_dot_product_attention(K, Q, Z, scale=w.scale)
+
+    for _ in range(2):
+        two_calls()
+    times = []
+    for _ in range(iters):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        two_calls()
+        b.record(st)
+        times.append((a, b))
+    torch.cuda.synchronize()
+    ms = statistics.median(a.elapsed_time(b) for a, b in times)
+    del Q, K, V
+    torch.cuda.empty_cache()
+    return {"what": "two torch scaled_dot_product_attention calls (prior art, context only)",
+            "ms": round(ms, 4), "tokens_per_s": w.B * w.N / (ms / 1e3)}
 
 
 def run_row(args, rank, local):
