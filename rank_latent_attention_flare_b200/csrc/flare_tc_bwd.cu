@@ -63,7 +63,6 @@ constexpr int kRegsRow = 200;
 constexpr int kRegsPro = 104;
 constexpr int kWTma = 8;
 constexpr int kWMma = 9;
-constexpr int kAStages = 4;
 constexpr int kBStages = 3;
 constexpr uint32_t kSw128 = 2u;  // UMMA descriptor code of the 128-byte swizzle
 constexpr uint32_t kSw32 = 6u;   // ... and of the 32-byte swizzle
@@ -110,6 +109,8 @@ __device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 
 template <int D>
 struct ALayout {
   static constexpr int M = kM;
+  static constexpr int KST = 4;               // K tiles: held until their S product
+  static constexpr int DST = 4;               // dY tiles: held until their dZ product
   static constexpr int RB = 2 * D;
   static constexpr int TILE = kT * RB;        // one K or dY tile
   static constexpr int PBUF = kT * M * 2;     // one P tile (swizzled, latent-contiguous rows)
@@ -117,13 +118,19 @@ struct ALayout {
   static constexpr int Q_OFF = 4 * PBUF;
   static constexpr int Z_OFF = Q_OFF + M * RB;
   static constexpr int ONE_OFF = Z_OFF + M * RB;  // second N block of Y's B operand
-  static constexpr int ST_OFF = ONE_OFF + M * RB;   // stages: K tile, dY tile
-  static constexpr int BAR_OFF = ST_OFF + kAStages * 2 * TILE;
-  static constexpr int NBARS = 2 * kAStages + 1 + 8 + 4 + 1 + 2;
+  static constexpr int K_OFF = ONE_OFF + M * RB;  // K ring
+  static constexpr int DY_OFF = K_OFF + KST * TILE;   // dY ring
+  static constexpr int BAR_OFF = DY_OFF + DST * TILE;
+  static constexpr int NBARS = 2 * KST + 2 * DST + 1 + 2 + 2 + 4 + 2 + 4 + 1 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
 };
 
+// Per 128-token tile (the two row warpgroups alternate tiles), software
+// pipelined: a warpgroup writes P of its tile j, starts the softmax of its
+// tile j + 1 while Y = P [Z | e0] of tile j runs on the tensor cores, and
+// then finishes tile j (delta_d, dY', dY'', statistics).  Each warpgroup has
+// two Y accumulators in TMEM for that overlap.
 template <int D>
 __global__ void __launch_bounds__(kThr, 1)
     tc_bwd_a_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -136,24 +143,28 @@ __global__ void __launch_bounds__(kThr, 1)
   using L = ALayout<D>;
   constexpr int M = L::M;
   constexpr int RB = L::RB;
+  constexpr int KST = L::KST;
+  constexpr int DST = L::DST;
   constexpr uint32_t SW = umma_swizzle_code(RB);
   constexpr int R = M;          // TMEM columns of a row warpgroup's S
-  constexpr int TY = 2 * M;     // [Y | row sum of bf16 P] of warpgroup w at TY + YC w
-  constexpr int YC = D + 16;
-  constexpr int TDZ = TY + 2 * YC;   // dZ accumulator (latent lanes)
-  static_assert(TDZ + D <= 512, "TMEM budget");
+  constexpr int YC = D + 16;    // one [Y | row sum of bf16 P] accumulator
+  constexpr int TY = 2 * M;     // Y accumulators: warpgroup w, buffer b at TY + YC (2 w + b)
+  constexpr int TDZ = TY + 4 * YC;   // dZ accumulator (latent lanes)
   constexpr uint32_t NCOLS = 512;
+  static_assert(TDZ + D <= 512, "TMEM budget");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* bars = (uint64_t*)(smem + L::BAR_OFF);
-  uint64_t* st_full = bars;
-  uint64_t* st_empty = bars + kAStages;
-  uint64_t* qz_full = bars + 2 * kAStages;
+  uint64_t* k_full = bars;
+  uint64_t* k_empty = k_full + KST;
+  uint64_t* d_full = k_empty + KST;
+  uint64_t* d_empty = d_full + DST;
+  uint64_t* qz_full = d_empty + DST;
   uint64_t* s_full = qz_full + 1;   // [w] S of the warpgroup's tile in TMEM
-  uint64_t* p_full = s_full + 2;    // [w] P written (TMEM and shared memory)
-  uint64_t* y_full = p_full + 2;    // [w] Y = P Z complete
-  uint64_t* a_done = y_full + 2;    // [w] Y read, dY' written: TMEM columns free
+  uint64_t* p_full = s_full + 2;    // [w] P in shared memory, S columns read
+  uint64_t* y_full = p_full + 2;    // [2 w + b] Y of the warpgroup's tile in buffer b complete
+  uint64_t* a_done = y_full + 4;    // [w] Y read, dY' written
   uint64_t* dz_done = a_done + 2;   // [2 w + b] dZ of warpgroup w's tile in P buffer b complete
   uint64_t* dz_final = dz_done + 4;
   uint64_t* drain = dz_final + 1;   // [2]: one per issuing thread
@@ -165,7 +176,7 @@ __global__ void __launch_bounds__(kThr, 1)
   const int64_t bh = blockIdx.y;
   const int64_t h = bh % H;
   const int64_t tile0 = (int64_t)chunk * chunk_tiles;
-  const int64_t ntiles = imin64(chunk_tiles, tiles_per_bh - tile0);
+  const int nt = (int)imin64(chunk_tiles, tiles_per_bh - tile0);
 
   // Y = P [Z | e0]: the second N block of the B operand holds a one in
   // column 0 of every latent row (same swizzled layout as the Z rows), so
@@ -178,18 +189,24 @@ __global__ void __launch_bounds__(kThr, 1)
   }
   fence_proxy_async_smem();
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kAStages; ++s) {
-      mbar_init(&st_full[s], 1);
-      mbar_init(&st_empty[s], 2);   // K read by S (warp 9), dY' by dZ (warp 10)
+    for (int s = 0; s < KST; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < DST; ++s) {
+      mbar_init(&d_full[s], 1);
+      mbar_init(&d_empty[s], 1);
     }
     mbar_init(qz_full, 1);
     for (int w = 0; w < 2; ++w) {
       mbar_init(&s_full[w], 1);
       mbar_init(&p_full[w], 128);
-      mbar_init(&y_full[w], 1);
       mbar_init(&a_done[w], 128);
     }
-    for (int k = 0; k < 4; ++k) mbar_init(&dz_done[k], 1);
+    for (int k = 0; k < 4; ++k) {
+      mbar_init(&y_full[k], 1);
+      mbar_init(&dz_done[k], 1);
+    }
     mbar_init(dz_final, 1);
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
@@ -204,101 +221,104 @@ __global__ void __launch_bounds__(kThr, 1)
 
   if (warp >= 8) {
     regs_release<kRegsPro>();
-    if (warp == kWTma) {
+    if (warp == kWTma || warp == kWMma + 2) {
+      // two producers, one per ring, so a dY tile that waits for its slot
+      // never holds back the K tile the next S needs
       if (lane == 0) {
-        prefetch_tmap(&tmQ);
-        prefetch_tmap(&tmK);
-        prefetch_tmap(&tmdY);
-        prefetch_tmap(&tmZ);
-        mbar_arrive_expect_tx(qz_full, 2 * M * RB);
-        tma_load_3d(smem + L::Q_OFF, &tmQ, qz_full, 0, 0, (int32_t)(q_per_batch ? bh : h));
-        tma_load_3d(smem + L::Z_OFF, &tmZ, qz_full, 0, 0, (int32_t)bh);
-        int64_t issued = 0;
-        for (int64_t i = 0; i < ntiles; ++i) {
-          const int s = (int)(i % kAStages);
-          const uint32_t ph = (uint32_t)((i / kAStages) & 1);
-          if (i >= kAStages && !mbar_wait_sleep(&st_empty[s], ph ^ 1)) {
+        const bool kq = (warp == kWTma);
+        uint64_t* full = kq ? k_full : d_full;
+        uint64_t* empty = kq ? k_empty : d_empty;
+        const int nst = kq ? KST : DST;
+        uint8_t* ring = smem + (kq ? L::K_OFF : L::DY_OFF);
+        const CUtensorMap* map = kq ? &tmK : &tmdY;
+        prefetch_tmap(map);
+        if (kq) {
+          prefetch_tmap(&tmQ);
+          prefetch_tmap(&tmZ);
+          mbar_arrive_expect_tx(qz_full, 2 * M * RB);
+          tma_load_3d(smem + L::Q_OFF, &tmQ, qz_full, 0, 0, (int32_t)(q_per_batch ? bh : h));
+          tma_load_3d(smem + L::Z_OFF, &tmZ, qz_full, 0, 0, (int32_t)bh);
+        }
+        int issued = 0;
+        for (int i = 0; i < nt; ++i) {
+          const int s = i % nst;
+          if (i >= nst && !mbar_wait_sleep(&empty[s], (uint32_t)(((i / nst) & 1) ^ 1))) {
             record_error(err, kErrBwdATmaWait);
             *abort_flag = 1;
             break;
           }
           if (*abort_flag) break;
-          uint8_t* dst = smem + L::ST_OFF + s * 2 * L::TILE;
-          mbar_arrive_expect_tx(&st_full[s], 2 * L::TILE);
-          const int32_t tok = (int32_t)((tile0 + i) * kT);
-          tma_load_3d(dst, &tmK, &st_full[s], 0, tok, (int32_t)bh);
-          tma_load_3d(dst + L::TILE, &tmdY, &st_full[s], 0, tok, (int32_t)bh);
+          mbar_arrive_expect_tx(&full[s], L::TILE);
+          tma_load_3d(ring + s * L::TILE, map, &full[s], 0, (int32_t)((tile0 + i) * kT), (int32_t)bh);
           issued = i + 1;
         }
-        for (int64_t i = (issued > kAStages ? issued - kAStages : 0); i < issued; ++i)
-          mbar_wait_sleep(&st_full[i % kAStages], (uint32_t)((i / kAStages) & 1));
-        mbar_wait_sleep(qz_full, 0);
+        // let every load still in flight land before the CTA can exit
+        for (int i = (issued > nst ? issued - nst : 0); i < issued; ++i)
+          mbar_wait_sleep(&full[i % nst], (uint32_t)((i / nst) & 1));
+        if (kq) mbar_wait_sleep(qz_full, 0);
       }
     } else if (warp == kWMma || warp == kWMma + 1) {
       // Two issuing threads: warp 9 issues S (it waits on TMA tiles), warp
-      // 10 issues Y and dZ (they wait on the row warps), so neither kind of
-      // wait delays the other kind of product.
+      // 10 issues Y and dZ (they wait on the row warps).
       if (lane == 0) {
         constexpr uint32_t idS = idesc_bf16_f32(128, M, 0, 0);
         constexpr uint32_t idY = idesc_bf16_f32(128, D + 16, 0, 1);   // N = [Z | e0]
         constexpr uint32_t idZ = idesc_bf16_f32(128, D, 1, 1);
         const uint32_t q_addr = smem_u32(smem + L::Q_OFF);
         const uint32_t z_addr = smem_u32(smem + L::Z_OFF);
-        const uint32_t st0 = smem_u32(smem + L::ST_OFF);
+        const uint32_t k0 = smem_u32(smem + L::K_OFF);
+        const uint32_t dy0 = smem_u32(smem + L::DY_OFF);
         const uint32_t p0 = smem_u32(smem + L::P_OFF);
         // descriptors built once; per MMA only the address field moves
-        const uint64_t dSt = smem_desc(st0, 16, 8 * RB, SW);          // K tile rows, K-major
+        const uint64_t dKk = smem_desc(k0, 16, 8 * RB, SW);           // K tile rows, K-major
         const uint64_t dQk = smem_desc(q_addr, 16, 8 * RB, SW);
         const uint64_t dPk = smem_desc(p0, 16, kMnSbo, kSw128);       // P, K-major (Y = P Z)
         const uint64_t dPm = smem_desc(p0, kMnLbo, kMnSbo, kSw128);   // P, MN-major (dZ)
         const uint64_t dZm = smem_desc(z_addr, M * RB, 8 * RB, SW);   // [Z | e0], MN-major
-        const uint64_t dStm = smem_desc(st0, L::TILE, 8 * RB, SW);    // dY tile, MN-major
+        const uint64_t dDYm = smem_desc(dy0, L::TILE, 8 * RB, SW);    // dY tile, MN-major
         constexpr uint32_t kTile16 = (uint32_t)L::TILE >> 4;
         constexpr uint32_t kRow16 = (uint32_t)RB;                     // 16 rows >> 4
         constexpr uint32_t kP16 = (uint32_t)L::PBUF >> 4;
-        const int nt = (int)ntiles;
         bool ok = mbar_wait_sleep(qz_full, 0);
         if (warp == kWMma) {
           // S(i) into warpgroup (i & 1)'s S columns once its tile i - 2 has
           // been read (p_full) and tile i's K is in shared memory
           for (int i = 0; ok && i < nt; ++i) {
             const int w = i & 1;
-            const int s = i % kAStages;
+            const int s = i % KST;
             if (i >= 2 && !mbar_wait_sleep(&p_full[w], (uint32_t)(((i - 2) >> 1) & 1))) {
               ok = false;
               break;
             }
-            if (!mbar_wait_sleep(&st_full[s], (uint32_t)((i / kAStages) & 1))) {
+            if (!mbar_wait_sleep(&k_full[s], (uint32_t)((i / KST) & 1))) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t so = (uint32_t)(s * 2) * kTile16;
+            const uint32_t ko = (uint32_t)s * kTile16;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
-              mma_ss(tmem + w * R, dSt + so + 2 * kk, dQk + 2 * kk, idS, kk > 0);
+              mma_ss(tmem + w * R, dKk + ko + 2 * kk, dQk + 2 * kk, idS, kk > 0);
             mma_commit(&s_full[w]);
-            mma_commit(&st_empty[s]);
+            mma_commit(&k_empty[s]);
             if (*abort_flag) ok = false;
           }
         } else {
-          // Y = P [Z | e0] with P read from shared memory as a K-major
-          // operand (token rows, latents contiguous: the same bytes dZ reads
-          // MN-major); dZ of a tile is issued one tile later, so a warpgroup
-          // waiting for its Y never waits behind the other one's dY work.
+          // Y(i) as soon as P(i) is written; dZ(i) once its warpgroup has
+          // finished tile i (after the softmax of its next tile)
           auto issue_dZ = [&](int i) -> bool {
             const int w = i & 1;
             const int j = i >> 1;
-            const int s = i % kAStages;
+            const int s = i % DST;
             if (!mbar_wait_sleep(&a_done[w], (uint32_t)(j & 1))) return false;
             tc_fence_after();
             const uint32_t po = (uint32_t)(2 * w + (j & 1)) * kP16;
-            const uint32_t so = (uint32_t)(s * 2 + 1) * kTile16;
+            const uint32_t so = (uint32_t)s * kTile16;
 #pragma unroll
             for (int kk = 0; kk < kT / 16; ++kk)
-              mma_ss(tmem + TDZ, dPm + po + kk * (kMnKStep >> 4), dStm + so + kk * kRow16, idZ,
+              mma_ss(tmem + TDZ, dPm + po + kk * (kMnKStep >> 4), dDYm + so + kk * kRow16, idZ,
                      (i > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(&st_empty[s]);
+            mma_commit(&d_empty[s]);
             mma_commit(&dz_done[2 * w + (j & 1)]);
             return true;
           };
@@ -313,13 +333,14 @@ __global__ void __launch_bounds__(kThr, 1)
             const uint32_t po = (uint32_t)(2 * w + (j & 1)) * kP16;
 #pragma unroll
             for (int kk = 0; kk < M / 16; ++kk)
-              mma_ss(tmem + TY + YC * w, dPk + po + (kk >> 2) * (kMnLbo >> 4) + (kk & 3) * 2,
-                     dZm + kk * kRow16, idY, kk > 0);
-            mma_commit(&y_full[w]);
-            if (i >= 1) ok = issue_dZ(i - 1);
+              mma_ss(tmem + TY + YC * (2 * w + (j & 1)),
+                     dPk + po + (kk >> 2) * (kMnLbo >> 4) + (kk & 3) * 2, dZm + kk * kRow16, idY,
+                     kk > 0);
+            mma_commit(&y_full[2 * w + (j & 1)]);
+            if (i >= 2) ok = issue_dZ(i - 2);
             if (*abort_flag) ok = false;
           }
-          if (ok && nt > 0) ok = issue_dZ(nt - 1);
+          for (int i = (nt > 2 ? nt - 2 : 0); ok && i < nt; ++i) ok = issue_dZ(i);
           mma_commit(dz_final);
         }
         if (!ok) {
@@ -337,16 +358,86 @@ __global__ void __launch_bounds__(kThr, 1)
     const uint32_t lb = (uint32_t)(qw * 32) << 16;
     const uint32_t tR = tmem + lb + w * R;
     const float Rh = rref[bh];
-    const int64_t nW = (ntiles - w + 1) / 2;
+    const int nW = (nt - w + 1) / 2;
     bool ok = true;
-    for (int64_t j = 0; j < nW; ++j) {
-      const int64_t i = 2 * j + w;
-      const int s = (int)(i % kAStages);
+    float mx_prev = 0.f, l_prev = 0.f;   // statistics of the tile whose finish is pending
+
+    // the second half of tile j: Y (with the row sum of the bf16 P),
+    // delta_d = dY . Y, dY' = dY / rowsum in place, dY'' = dY / g, statistics
+    auto finish = [&](int j, float mx, float l) -> bool {
+      const int i = 2 * j + w;
+      const int s = i % DST;
       const int64_t tok = (tile0 + i) * kT + r;
+      if (!warp_all(mbar_wait(&y_full[2 * w + (j & 1)], (uint32_t)((j >> 1) & 1)) &&
+                    mbar_wait(&d_full[s], (uint32_t)((i / DST) & 1)) && !*abort_flag))
+        return false;
+      __syncwarp();
+      tc_fence_after();
+      float y[D];
+      float lsum;   // row sum of the bf16 P (the weights the tensor cores used)
+      const uint32_t ty = tmem + lb + TY + YC * (2 * w + (j & 1));
+      if (D == 32) {
+        uint32_t o[32], o2[16];
+        tmem_ld32(ty, o);
+        tmem_ld16(ty + 32, o2);
+        tmem_wait_ld_dep(o);
+        reg_fence16(o2);
+#pragma unroll
+        for (int d = 0; d < D; ++d) y[d] = __uint_as_float(o[d]);
+        lsum = __uint_as_float(o2[0]);
+      } else {
+        uint32_t o[32];
+        tmem_ld32(ty, o);
+        tmem_wait_ld_dep(o);
+#pragma unroll
+        for (int d = 0; d < D; ++d) y[d] = __uint_as_float(o[d]);
+        lsum = __uint_as_float(o[D]);
+      }
+      const float inv = 1.f / lsum;
+      const float mxp = fmaf(mx, c, log2f(l));   // row log-sum-exp, log2 units
+      const float lg = mxp - Rh;                  // log2 of g[n]
+      const bool bad = lg < -kRowRangeMax;        // g[n] would leave the float range
+      const float ginv = bad ? 0.f : ex2(-lg);    // 1 / g[n]
+      uint8_t* dyt = smem + L::DY_OFF + s * L::TILE;
+      float dot = 0.f, dot2 = 0.f;
+      uint4 o2v[D / 8];
+#pragma unroll
+      for (int ch = 0; ch < D / 8; ++ch) {
+        uint4* p = reinterpret_cast<uint4*>(dyt + tma_row_chunk<D>(r, ch));
+        const uint4 u = *p;
+        const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
+        uint32_t wv[4], w2[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const float a0 = bf_lo(uu[jj]), a1 = bf_hi(uu[jj]);
+          const float y0 = y[8 * ch + 2 * jj], y1 = y[8 * ch + 2 * jj + 1];
+          dot = fmaf(a0, y0, fmaf(a1, y1, dot));
+          w2[jj] = pack_bf16(a0 * ginv, a1 * ginv);           // dY'' = dY / g
+          dot2 = fmaf(bf_lo(w2[jj]), y0, fmaf(bf_hi(w2[jj]), y1, dot2));
+          wv[jj] = pack_bf16(a0 * inv, a1 * inv);             // dY' = dY / rowsum
+        }
+        *p = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        o2v[ch] = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+      }
+      if (tok < N) {
+        // delta_d = dY . Y and its counterpart with the rounded dY'' (= delta_d / g)
+        stats[bh * N + tok] = make_float4(mxp, dot * inv, dot2 * inv, 0.f);
+        uint4* dst = reinterpret_cast<uint4*>(dy2 + (bh * N + tok) * D);
+#pragma unroll
+        for (int ch = 0; ch < D / 8; ++ch) dst[ch] = o2v[ch];
+      }
+      if (warp_any(bad && tok < N) && lane == 0) atomicOr(flags + bh, 1u);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&a_done[w]);
+      return true;
+    };
+
+    for (int j = 0; j < nW; ++j) {
       uint8_t* pbuf = smem + L::P_OFF + (2 * w + (j & 1)) * L::PBUF;
       // the P buffer of tile j was last read by the dZ of tile j - 2
-      if (!warp_all(mbar_wait_sleep(&s_full[w], (uint32_t)(j & 1)) &&
-                    (j < 2 || mbar_wait_sleep(&dz_done[2 * w + (j & 1)], (uint32_t)(((j - 2) >> 1) & 1))) &&
+      if (!warp_all(mbar_wait(&s_full[w], (uint32_t)(j & 1)) &&
+                    (j < 2 || mbar_wait(&dz_done[2 * w + (j & 1)], (uint32_t)(((j - 2) >> 1) & 1))) &&
                     !*abort_flag)) {
         ok = false;
         break;
@@ -384,72 +475,12 @@ __global__ void __launch_bounds__(kThr, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&p_full[w]);
-      // Y = P Z (unnormalised); delta_d = dY . Y / l; dY' = dY / l in place
-      if (!warp_all(mbar_wait_sleep(&y_full[w], (uint32_t)(j & 1)) &&
-                    mbar_wait(&st_full[s], (uint32_t)((i / kAStages) & 1)))) {
-        ok = false;
-        break;
-      }
-      __syncwarp();
-      tc_fence_after();
-      float y[D];
-      float lsum;   // row sum of the bf16 P (the weights the tensor cores used)
-      if (D == 32) {
-        uint32_t o[32], o2[16];
-        tmem_ld32(tmem + lb + TY + YC * w, o);
-        tmem_ld16(tmem + lb + TY + YC * w + 32, o2);
-        tmem_wait_ld_dep(o);
-        reg_fence16(o2);
-#pragma unroll
-        for (int d = 0; d < D; ++d) y[d] = __uint_as_float(o[d]);
-        lsum = __uint_as_float(o2[0]);
-      } else {
-        uint32_t o[32];
-        tmem_ld32(tmem + lb + TY + YC * w, o);
-        tmem_wait_ld_dep(o);
-#pragma unroll
-        for (int d = 0; d < D; ++d) y[d] = __uint_as_float(o[d]);
-        lsum = __uint_as_float(o[D]);
-      }
-      const float l = (sf[0] + sf[1]) + (sf[2] + sf[3]);
-      const float inv = 1.f / lsum;
-      const float mxp = fmaf(mx, c, log2f(l));   // row log-sum-exp, log2 units
-      const float lg = mxp - Rh;                  // log2 of g[n]
-      const bool bad = lg < -kRowRangeMax;        // g[n] would leave the float range
-      const float ginv = bad ? 0.f : ex2(-lg);    // 1 / g[n]
-      uint8_t* dyt = smem + L::ST_OFF + s * 2 * L::TILE + L::TILE;
-      float dot = 0.f, dot2 = 0.f;
-      uint4 o2[D / 8];
-#pragma unroll
-      for (int ch = 0; ch < D / 8; ++ch) {
-        uint4* p = reinterpret_cast<uint4*>(dyt + tma_row_chunk<D>(r, ch));
-        const uint4 u = *p;
-        const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
-        uint32_t wv[4], w2[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float a0 = bf_lo(uu[j]), a1 = bf_hi(uu[j]);
-          const float y0 = y[8 * ch + 2 * j], y1 = y[8 * ch + 2 * j + 1];
-          dot = fmaf(a0, y0, fmaf(a1, y1, dot));
-          w2[j] = pack_bf16(a0 * ginv, a1 * ginv);           // dY'' = dY / g
-          dot2 = fmaf(bf_lo(w2[j]), y0, fmaf(bf_hi(w2[j]), y1, dot2));
-          wv[j] = pack_bf16(a0 * inv, a1 * inv);             // dY' = dY / rowsum
-        }
-        *p = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-        o2[ch] = make_uint4(w2[0], w2[1], w2[2], w2[3]);
-      }
-      if (tok < N) {
-        // delta_d = dY . Y and its counterpart with the rounded dY'' (= delta_d / g)
-        stats[bh * N + tok] = make_float4(mxp, dot * inv, dot2 * inv, 0.f);
-        uint4* dst = reinterpret_cast<uint4*>(dy2 + (bh * N + tok) * D);
-#pragma unroll
-        for (int ch = 0; ch < D / 8; ++ch) dst[ch] = o2[ch];
-      }
-      if (warp_any(bad && tok < N) && lane == 0) atomicOr(flags + bh, 1u);
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&a_done[w]);
+      // while Y of tile j runs, finish tile j - 1
+      if (j > 0 && !(ok = finish(j - 1, mx_prev, l_prev))) break;
+      mx_prev = mx;
+      l_prev = (sf[0] + sf[1]) + (sf[2] + sf[3]);
     }
+    if (ok && nW > 0) ok = finish(nW - 1, mx_prev, l_prev);
     if (!ok) {
       record_error(err, kErrBwdARowWait);
       *abort_flag = 1;
@@ -459,7 +490,7 @@ __global__ void __launch_bounds__(kThr, 1)
       float acc[D];
 #pragma unroll
       for (int d = 0; d < D; ++d) acc[d] = 0.f;
-      if (ok && ntiles > 0) {
+      if (ok && nt > 0) {
         ok = warp_all(mbar_wait_sleep(dz_final, 0));
         __syncwarp();
         tc_fence_after();
@@ -580,13 +611,22 @@ __global__ void __launch_bounds__(kM)
   const float f = fast ? exp2f(R - l2) : 1.f;
   // delta_e is taken with the bf16 operand dZ'' that the tensor cores use,
   // so dPe'' = V dZ''^T - dZ'' . Z vanishes exactly where V = Z.
+  float zr[D];
+#pragma unroll
+  for (int d = 0; d < D; d += 4) {
+    const float4 zv = *reinterpret_cast<const float4*>(Z + row * D + d);
+    zr[d] = zv.x;
+    zr[d + 1] = zv.y;
+    zr[d + 2] = zv.z;
+    zr[d + 3] = zv.w;
+  }
   float de = 0.f;
 #pragma unroll
   for (int d = 0; d < D; d += 2) {
     const uint32_t pr = pack_bf16(f * dz[d], f * dz[d + 1]);
     *reinterpret_cast<uint32_t*>(dzs + row * D + d) = pr;
-    de = fmaf(bf_lo(pr), Z[row * D + d], de);
-    de = fmaf(bf_hi(pr), Z[row * D + d + 1], de);
+    de = fmaf(bf_lo(pr), zr[d], de);
+    de = fmaf(bf_hi(pr), zr[d + 1], de);
   }
   const float x = -de;
   const __nv_bfloat16 b0 = __float2bfloat16_rn(x);
@@ -1463,24 +1503,43 @@ __global__ void __launch_bounds__(kThr, 1)
 }
 
 // dQ = sum over (batch when Q is shared) x chunks of the scaled partials,
-// in a fixed order.  One thread per output element.
-__global__ void bwd_dq_sum_kernel(const float* __restrict__ dq_part, int B, int H, int M, int D,
+// in a fixed order (batch outer, chunk inner).  One thread per 4 output
+// elements; the partials' loads are issued in groups of 8 before they are
+// added, so their latencies overlap.
+__global__ void bwd_dq_sum_kernel(const float4* __restrict__ dq_part, int B, int H, int M, int D,
                                   int chunks, bool shared_q, __nv_bfloat16* __restrict__ dQ) {
-  const int64_t per = (int64_t)H * M * D;
-  const int64_t total = shared_q ? per : (int64_t)B * per;
+  const int64_t md4 = (int64_t)M * D / 4;
+  const int64_t per4 = (int64_t)H * md4;
+  const int64_t total4 = shared_q ? per4 : (int64_t)B * per4;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= total) return;
-  const int64_t b0 = shared_q ? 0 : i / per;
-  const int64_t b1 = shared_q ? B : b0 + 1;
-  const int64_t rr = i % per;
-  const int64_t h = rr / ((int64_t)M * D);
-  const int64_t md = rr % ((int64_t)M * D);
-  float acc = 0.f;
-  for (int64_t b = b0; b < b1; ++b) {
-    const int64_t bh = b * H + h;
-    for (int k = 0; k < chunks; ++k) acc += dq_part[(bh * chunks + k) * (int64_t)M * D + md];
+  if (i >= total4) return;
+  const int64_t b0 = shared_q ? 0 : i / per4;
+  const int64_t rr = i % per4;
+  const int64_t h = rr / md4;
+  const int64_t e = rr % md4;
+  const int n = (shared_q ? B : 1) * chunks;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int q0 = 0; q0 < n; q0 += 8) {
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int q = q0 + u;
+      if (q < n) {
+        const int64_t bh = (b0 + q / chunks) * H + h;
+        v[u] = dq_part[(bh * chunks + q % chunks) * md4 + e];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (q0 + u < n) {
+        acc.x += v[u].x;
+        acc.y += v[u].y;
+        acc.z += v[u].z;
+        acc.w += v[u].w;
+      }
+    }
   }
-  dQ[i] = __float2bfloat16_rn(acc);
+  *reinterpret_cast<uint2*>(dQ + i * 4) = make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
 }
 
 template <int D>
@@ -1551,8 +1610,8 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
 
   const bool shared_q = (qbs == 0);
   const int64_t total = shared_q ? d.H * kM * D : BH * kM * D;
-  bwd_dq_sum_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
-      dqp, (int)d.B, (int)d.H, kM, D, p.chunks, shared_q, (__nv_bfloat16*)dQ);
+  bwd_dq_sum_kernel<<<(unsigned)((total / 4 + 127) / 128), 128, 0, st>>>(
+      (const float4*)dqp, (int)d.B, (int)d.H, kM, D, p.chunks, shared_q, (__nv_bfloat16*)dQ);
   return cudaPeekAtLastError();
 }
 
