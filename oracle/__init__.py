@@ -61,8 +61,10 @@ def _load():
                                             ctypes.c_double, _c_dp, _c_dp, _c_dp, _c_dp]
         lib.oracle_flare_bwd.argtypes = [_c_dp, _i64, _c_dp, _c_dp, _c_dp, _i64, _i64, _i64,
                                          _i64, _i64, ctypes.c_double, _c_dp, _c_dp, _c_dp]
+        lib.oracle_flare_pp_bwd.argtypes = [_c_dp, _c_dp, _c_dp, _c_dp, _i64, _i64, _i64, _i64,
+                                            _i64, ctypes.c_double, _c_dp, _c_dp, _c_dp]
         for f in ("oracle_encode", "oracle_decode", "oracle_decode_rows", "oracle_flare_fwd",
-                  "oracle_flare_pp_fwd", "oracle_flare_bwd"):
+                  "oracle_flare_pp_fwd", "oracle_flare_bwd", "oracle_flare_pp_bwd"):
             getattr(lib, f).restype = None
         _lib = lib
     return _lib
@@ -167,4 +169,19 @@ def flare_bwd(Q, K, V, dY, scale: float):
     dV = np.empty((B, H, N, D))
     _load().oracle_flare_bwd(_p(Q), qbs, _p(K), _p(V), _p(dY), B, H, N, M, D, float(scale),
                              _p(dQ), _p(dK), _p(dV))
+    return dQ, dK, dV
+
+
+def flare_pp_bwd(Q, K, V, dY, scale: float):
+    """Gradients (dQ [H,M,D], dK, dV) of sum(Y * dY) for FLARE++ with learned
+    Q [H,M,D] (FLARE++ abstract: the encoder's outputs correct the learned
+    queries; the chain rule runs through both uses of Q_dyn and through the
+    first encode)."""
+    Q, K, V, dY = _f64(Q), _f64(K), _f64(V), _f64(dY)
+    B, H, N, M, D, _ = _shapes(Q, K, True)
+    dQ = np.empty(Q.shape)
+    dK = np.empty((B, H, N, D))
+    dV = np.empty((B, H, N, D))
+    _load().oracle_flare_pp_bwd(_p(Q), _p(K), _p(V), _p(dY), B, H, N, M, D, float(scale),
+                                _p(dQ), _p(dK), _p(dV))
     return dQ, dK, dV

@@ -32,7 +32,9 @@
  *   - FLARE++: Q_dyn = Q + encode(Q, K, V) (plain sum, per batch), then
  *     Z = encode(Q_dyn, K, V) and Y = decode(Q_dyn, Z) [P5];
  *   - the pages give no backward pass; the gradient below is the chain rule
- *     of the two softmax-attention stages applied to L = sum(Y * dY).
+ *     of the two softmax-attention stages applied to L = sum(Y * dY);
+ *   - FLARE++ gradient: the same chain rule through Q_dyn = Q + encode(Q, K,
+ *     V), with Q shared over the batch (its gradient summed over b).
  *
  * Layouts: Q is [H,M,D] when q_bstride == 0 (shared over the batch) or
  * [B,H,M,D] when q_bstride == H*M*D; K, V, Y, dY are [B,H,N,D]; Z is
@@ -301,4 +303,89 @@ void oracle_flare_bwd(const double* Q, int64_t q_bstride, const double* K,
     memcpy(dQ, dQbh, (size_t)(BH * M * D) * sizeof(double));
   }
   free(dQbh);
+}
+
+/*
+ * Adds the gradient of L = sum(Z1 * dZ1) for the encode Z1 = softmax_n(s Q K^T) V
+ * with Q [H,M,D] shared over the batch: for one (b, h),
+ *   P = softmax over n of s Q K^T [M,N],   dP = dZ1 V^T,
+ *   dA = P * (dP - rowsum(P * dP)),
+ *   dV += P^T dZ1,   dK += s dA^T Q,   dQ += s dA K (summed over b).
+ */
+static void encode_bwd_add(const double* Q, const double* K, const double* V,
+                           const double* dZ1, int64_t B, int64_t H, int64_t N,
+                           int64_t M, int64_t D, double scale, double* dQ,
+                           double* dK, double* dV) {
+  int64_t BH = B * H;
+  double* dQbh = (double*)calloc((size_t)(BH * M * D), sizeof(double));
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t bh = 0; bh < BH; ++bh) {
+    int64_t h = bh % H;
+    const double* q = Q + h * M * D;
+    const double* k = K + bh * N * D;
+    const double* v = V + bh * N * D;
+    const double* dz = dZ1 + bh * M * D;
+    double* dk = dK + bh * N * D;
+    double* dv = dV + bh * N * D;
+    double* dq = dQbh + bh * M * D;
+    double* P = (double*)malloc((size_t)N * sizeof(double));
+    for (int64_t m = 0; m < M; ++m) {
+      double mu = -INFINITY;
+      for (int64_t n = 0; n < N; ++n) {
+        P[n] = scale * dotd(q + m * D, k + n * D, D);
+        if (P[n] > mu) mu = P[n];
+      }
+      double den = 0.0;
+      for (int64_t n = 0; n < N; ++n) {
+        P[n] = exp(P[n] - mu);
+        den += P[n];
+      }
+      double delta = 0.0;
+      for (int64_t n = 0; n < N; ++n) {
+        P[n] /= den;
+        delta += P[n] * dotd(dz + m * D, v + n * D, D);
+      }
+      for (int64_t n = 0; n < N; ++n) {
+        double dA = P[n] * (dotd(dz + m * D, v + n * D, D) - delta);
+        for (int64_t d = 0; d < D; ++d) {
+          dv[n * D + d] += P[n] * dz[m * D + d];
+          dk[n * D + d] += scale * dA * q[m * D + d];
+          dq[m * D + d] += scale * dA * k[n * D + d];
+        }
+      }
+    }
+    free(P);
+  }
+  for (int64_t b = 0; b < B; ++b)
+    for (int64_t i = 0; i < H * M * D; ++i) dQ[i] += dQbh[b * H * M * D + i];
+  free(dQbh);
+}
+
+/*
+ * Gradient of L = sum(Y * dY) for FLARE++ with learned Q [H,M,D]:
+ *   Q_dyn = Q + Z1, Z1 = encode(Q, K, V)      (per batch)
+ *   Y = FLARE(Q_dyn, K, V)                     (per-batch latents)
+ * FLARE's gradient with per-batch latents gives dQ_dyn, dK, dV; Q_dyn's
+ * gradient then reaches Q directly (summed over b) and through Z1 (the
+ * encode's gradient with upstream dZ1 = dQ_dyn), which also adds to dK, dV.
+ */
+void oracle_flare_pp_bwd(const double* Q, const double* K, const double* V,
+                         const double* dY, int64_t B, int64_t H, int64_t N,
+                         int64_t M, int64_t D, double scale, double* dQ,
+                         double* dK, double* dV) {
+  int64_t per_b = H * M * D;
+  double* Z1 = (double*)malloc((size_t)(B * per_b) * sizeof(double));
+  double* Qdyn = (double*)malloc((size_t)(B * per_b) * sizeof(double));
+  double* dQd = (double*)malloc((size_t)(B * per_b) * sizeof(double));
+  oracle_encode(Q, 0, K, V, B, H, N, M, D, scale, Z1, NULL);
+  for (int64_t b = 0; b < B; ++b)
+    for (int64_t i = 0; i < per_b; ++i) Qdyn[b * per_b + i] = Q[i] + Z1[b * per_b + i];
+  oracle_flare_bwd(Qdyn, per_b, K, V, dY, B, H, N, M, D, scale, dQd, dK, dV);
+  memset(dQ, 0, (size_t)per_b * sizeof(double));
+  for (int64_t b = 0; b < B; ++b)
+    for (int64_t i = 0; i < per_b; ++i) dQ[i] += dQd[b * per_b + i];
+  encode_bwd_add(Q, K, V, dQd, B, H, N, M, D, scale, dQ, dK, dV);
+  free(Z1);
+  free(Qdyn);
+  free(dQd);
 }

@@ -297,3 +297,67 @@ def test_bwd_value_gradient_sums_to_output_gradient():
     x = _x(2, 2, 300, 16, 8, seed=21, with_dy=True)
     _, _, dV = oracle.flare_bwd(x["Q"], x["K"], x["V"], x["dY"], 0.3)
     np.testing.assert_allclose(dV.sum(axis=2), x["dY"].sum(axis=2), rtol=1e-11, atol=1e-11)
+
+
+# ------------------------------------------------------- FLARE++ gradient ---
+
+def _pp_loss(Q, K, V, dY, s):
+    Y, _, _, _ = oracle.flare_pp_fwd(Q, K, V, s)
+    return float((Y * dY).sum())
+
+
+def test_pp_bwd_central_finite_differences():
+    # Every element of the learned latents Q, of K and of V; the chain runs
+    # through both uses of Q_dyn and through the first encode.
+    B, H, N, M, D = 2, 1, 40, 4, 4
+    x = _x(B, H, N, M, D, seed=23, with_dy=True)
+    s = 1.0 / math.sqrt(D)
+    dQ, dK, dV = oracle.flare_pp_bwd(x["Q"], x["K"], x["V"], x["dY"], s)
+    eps = 1e-5
+    for name, grad in (("Q", dQ), ("K", dK), ("V", dV)):
+        base = x[name]
+        fd = np.empty_like(base)
+        flat = base.reshape(-1)
+        for i in range(flat.size):
+            old = flat[i]
+            flat[i] = old + eps
+            lp = _pp_loss(x["Q"], x["K"], x["V"], x["dY"], s)
+            flat[i] = old - eps
+            lm = _pp_loss(x["Q"], x["K"], x["V"], x["dY"], s)
+            flat[i] = old
+            fd.reshape(-1)[i] = (lp - lm) / (2 * eps)
+        scale_ref = np.abs(fd).max()
+        assert np.abs(grad - fd).max() <= 1e-7 * max(scale_ref, 1.0), name
+
+
+def test_pp_bwd_float64_autograd_crosscheck():
+    # The abstracts' form written with torch SDPA in float64: Q_dyn = Q +
+    # SDPA(Q, K, V), then the two-call FLARE with Q_dyn; autograd's gradients.
+    x = _x(2, 2, 130, 16, 8, seed=24, with_dy=True)
+    s = 0.3
+    dQ, dK, dV = oracle.flare_pp_bwd(x["Q"], x["K"], x["V"], x["dY"], s)
+    t = {k: torch.from_numpy(v.copy()).requires_grad_(k != "dY") for k, v in x.items()}
+    Qb = t["Q"].unsqueeze(0).expand(t["K"].shape[0], -1, -1, -1)
+    Qd = Qb + F.scaled_dot_product_attention(Qb, t["K"], t["V"], scale=s)
+    Yt, _ = _sdpa_flare(Qd, t["K"], t["V"], s)
+    (Yt * t["dY"]).sum().backward()
+    np.testing.assert_allclose(dQ, t["Q"].grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dK, t["K"].grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dV, t["V"].grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_pp_bwd_reduces_to_flare_when_the_correction_is_removed():
+    # With V = 0 the first encode returns Z1 = 0, so Q_dyn = Q and the FLARE++
+    # forward equals FLARE's; the gradients w.r.t. Q and K then equal FLARE's
+    # (Z1 = P V is linear in V, so no dQ or dK flows through it at V = 0),
+    # and dV gains only the first encode's P^T dQ_dyn term.
+    B, H, N, M, D = 2, 2, 70, 8, 8
+    x = _x(B, H, N, M, D, seed=25, with_dy=True)
+    x["V"][:] = 0.0
+    s = 0.4
+    dQ, dK, dV = oracle.flare_pp_bwd(x["Q"], x["K"], x["V"], x["dY"], s)
+    dQf, dKf, dVf = oracle.flare_bwd(x["Q"], x["K"], x["V"], x["dY"], s)
+    np.testing.assert_allclose(dK, dKf, rtol=1e-11, atol=1e-12)
+    # dQ: FLARE's dQ with per-batch Q_dyn = Q, summed over the batch, is
+    # FLARE's shared-Q dQ
+    np.testing.assert_allclose(dQ, dQf, rtol=1e-11, atol=1e-12)
