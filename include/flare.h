@@ -75,7 +75,12 @@ typedef enum {
   FLARE_ERR_DEVICE_TIMEOUT = 5 /* a kernel's bounded wait ran out           */
 } flare_status_t;
 
-typedef enum { FLARE_OP_FWD = 0, FLARE_OP_PP_FWD = 1, FLARE_OP_BWD = 2 } flare_op_t;
+typedef enum {
+  FLARE_OP_FWD = 0,
+  FLARE_OP_PP_FWD = 1,
+  FLARE_OP_BWD = 2,
+  FLARE_OP_PP_BWD = 3
+} flare_op_t;
 
 /* Library ABI version (major*10000 + minor*100 + patch). */
 FLARE_API int flare_version(void);
@@ -139,6 +144,26 @@ FLARE_API flare_status_t flare_bwd(const void* Q, int64_t q_batch_stride, const 
                          void* dK, void* dV, int64_t B, int64_t H, int64_t N, int64_t M,
                          int64_t D, flare_dtype_t dtype, float scale, void* workspace,
                          size_t workspace_bytes, void* stream);
+
+/*
+ * FLARE++ backward with learned latents Q [H,M,D] (FLARE++ abstract: the
+ * encoder's M outputs correct the learned queries, and the corrected
+ * queries drive both compression and redistribution):
+ *   Q_dyn = Q + encode(Q, K, V),  Y = FLARE(Q_dyn, K, V).
+ * Gradients of sum(Y * dY): FLARE's backward with the per-batch latents
+ * Q_dyn, then the first encode's backward with upstream gradient dQ_dyn;
+ * dQ [H,M,D] is summed over the batch.  Inputs: Q, K, V, dY, the forward's
+ * Q_dyn ([B,H,M,D], input dtype) and its Z_save / lse_save (the second
+ * encode's).  The first encode is recomputed; Q_dyn's rounding to the
+ * input dtype is treated as the identity.  Outputs dQ, dK, dV in the input
+ * dtype.  Workspace: flare_workspace_size(FLARE_OP_PP_BWD, ...).  Every
+ * reduction is in a fixed order (bitwise reproducible).
+ */
+FLARE_API flare_status_t flare_pp_bwd(const void* Q, const void* K, const void* V, const void* dY,
+                            const void* Q_dyn, const float* Z_save, const float* lse_save,
+                            void* dQ, void* dK, void* dV, int64_t B, int64_t H, int64_t N,
+                            int64_t M, int64_t D, flare_dtype_t dtype, float scale,
+                            void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Stage 1 of the forward -- encode partials.  For each (b, h) and each

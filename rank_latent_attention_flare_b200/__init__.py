@@ -4,16 +4,18 @@ The compute lives in ``libflare.so`` (hand-written CUDA: tcgen05/TMEM/TMA
 tensor-core kernels and CUDA-core kernels) behind the C ABI declared in
 ``include/flare.h``.  This package is a thin ctypes binding over it.
 """
-from ._lib import (FLARE_BF16, FLARE_F32, FLARE_OP_BWD, FLARE_OP_FWD, FLARE_OP_PP_FWD,
+from ._lib import (FLARE_BF16, FLARE_F32, FLARE_OP_BWD, FLARE_OP_FWD, FLARE_OP_PP_BWD,
+                   FLARE_OP_PP_FWD,
                    NOALLOC_SCRATCH_BYTES, FlareError, LIB_PATH, SIGNATURES, load)
 from .flare import (alloc_workspace, bwd_path, default_scale, device_status, flare_bwd, flare_combine,
-                    flare_decode, flare_encode, flare_fwd, flare_fwd_noalloc, flare_pp_fwd,
+                    flare_decode, flare_encode, flare_fwd, flare_fwd_noalloc, flare_pp_bwd, flare_pp_fwd,
                     fwd_path, workspace_size)
 
 __all__ = [
-    "FLARE_BF16", "FLARE_F32", "FLARE_OP_BWD", "FLARE_OP_FWD", "FLARE_OP_PP_FWD", "FlareError",
+    "FLARE_BF16", "FLARE_F32", "FLARE_OP_BWD", "FLARE_OP_FWD", "FLARE_OP_PP_BWD",
+    "FLARE_OP_PP_FWD", "FlareError",
     "LIB_PATH", "SIGNATURES", "load", "alloc_workspace", "default_scale", "device_status",
     "flare_bwd", "flare_combine", "flare_decode", "flare_encode", "flare_fwd", "flare_fwd_noalloc",
-    "flare_pp_fwd", "NOALLOC_SCRATCH_BYTES",
+    "flare_pp_bwd", "flare_pp_fwd", "NOALLOC_SCRATCH_BYTES",
     "bwd_path", "fwd_path", "workspace_size",
 ]

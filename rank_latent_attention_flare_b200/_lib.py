@@ -17,6 +17,7 @@ FLARE_BF16 = 1
 FLARE_OP_FWD = 0
 FLARE_OP_PP_FWD = 1
 FLARE_OP_BWD = 2
+FLARE_OP_PP_BWD = 3
 
 # Size of the fixed device scratch array behind flare_fwd_noalloc.
 NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -49,6 +50,8 @@ SIGNATURES = {
                             _vp, _vp, _vp, _sz, _vp]),
     "flare_bwd": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
                          _i64, _i64, _i32, _f32, _vp, _sz, _vp]),
+    "flare_pp_bwd": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                            _i64, _i64, _i32, _f32, _vp, _sz, _vp]),
     "flare_encode": (_i32, [_vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i32, _f32, _vp,
                             _sz, _vp]),
     "flare_combine": (_i32, [_i64, _i64, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _sz, _vp]),

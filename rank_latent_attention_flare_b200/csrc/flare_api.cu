@@ -154,7 +154,8 @@ const char* flare_status_string(flare_status_t s) {
 
 size_t flare_workspace_size(flare_op_t op, int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
                             flare_dtype_t dt) {
-  if (op != FLARE_OP_FWD && op != FLARE_OP_PP_FWD && op != FLARE_OP_BWD) return 0;
+  if (op != FLARE_OP_FWD && op != FLARE_OP_PP_FWD && op != FLARE_OP_BWD && op != FLARE_OP_PP_BWD)
+    return 0;
   if (check_sizes(B, H, N, M, D, dt) != FLARE_OK) return 0;
   return ws_layout(op, B, H, N, M, D, dt, current_sm_count()).total;
 }
@@ -297,6 +298,42 @@ flare_status_t flare_bwd(const void* Q, int64_t qbs, const void* K, const void* 
   FLARE_TRY(reset_error_word(ws, st));
   FLARE_CUDA(launch_bwd(Q, qbs, K, V, dY, Z_save, lse_save, dQ, dK, dV, Dims{B, H, N, M, D}, dt,
                         scale, L, ws, st));
+  return FLARE_OK;
+}
+
+flare_status_t flare_pp_bwd(const void* Q, const void* K, const void* V, const void* dY,
+                            const void* Q_dyn, const float* Z_save, const float* lse_save,
+                            void* dQ, void* dK, void* dV, int64_t B, int64_t H, int64_t N,
+                            int64_t M, int64_t D, flare_dtype_t dt, float scale, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  FLARE_TRY(check_sizes(B, H, N, M, D, dt));
+  FLARE_TRY(check_scale(scale));
+  FLARE_TRY(check_ptr(Q));
+  FLARE_TRY(check_ptr(K));
+  FLARE_TRY(check_ptr(V));
+  FLARE_TRY(check_ptr(dY));
+  FLARE_TRY(check_ptr(Q_dyn));
+  FLARE_TRY(check_ptr(Z_save));
+  FLARE_TRY(check_ptr(lse_save));
+  FLARE_TRY(check_ptr(dQ));
+  FLARE_TRY(check_ptr(dK));
+  FLARE_TRY(check_ptr(dV));
+  const WsLayout L = ws_layout(FLARE_OP_PP_BWD, B, H, N, M, D, dt, current_sm_count());
+  FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  char* ws = (char*)workspace;
+  cudaStream_t st = (cudaStream_t)stream;
+  const Dims d{B, H, N, M, D};
+  float* z1 = (float*)(ws + L.z1);
+  float* lse1 = (float*)(ws + L.lse1);
+  FLARE_TRY(reset_error_word(ws, st));
+  // the first encode, recomputed: Z1 and its lse
+  FLARE_TRY(run_encode(Q, 0, K, V, d, dt, scale, L, ws, st));
+  FLARE_TRY(run_combine(d, dt, z1, lse1, nullptr, nullptr, L, ws, st));
+  // FLARE's backward with the per-batch latents Q_dyn: dQ_dyn, dK, dV
+  FLARE_CUDA(launch_bwd(Q_dyn, H * M * D, K, V, dY, Z_save, lse_save, ws + L.dqd, dK, dV, d, dt,
+                        scale, L, ws, st));
+  // the first encode's gradient with upstream dQ_dyn, and dQ
+  FLARE_CUDA(launch_pp_bwd_tail(Q, K, V, z1, lse1, ws + L.dqd, dQ, dK, dV, d, dt, scale, L, ws, st));
   return FLARE_OK;
 }
 

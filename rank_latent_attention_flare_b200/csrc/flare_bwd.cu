@@ -357,3 +357,207 @@ cudaError_t launch_bwd(const void* Q, int64_t qbs, const void* K, const void* V,
 }
 
 }  // namespace flare
+
+// ============================================================ FLARE++ backward
+//
+// Q_dyn = Q + Z1, Z1 = encode(Q, K, V) with learned Q [H,M,D] shared over the
+// batch (FLARE++ abstract), and Y = FLARE(Q_dyn, K, V).  After FLARE's
+// backward with per-batch latents Q_dyn has produced dQ_dyn, dK and dV, the
+// first encode's gradient with upstream dZ1 = dQ_dyn is added here:
+//   P1 = exp(s Q K^T - lse1), dP1 = dZ1 V^T, delta1 = rowsum(dZ1 * Z1),
+//   dA1 = P1 * (dP1 - delta1), dV += P1^T dZ1, dK += s dA1^T Q,
+//   dQ = sum over b of (dQ_dyn + s dA1 K).
+
+namespace flare {
+namespace {
+
+// dZ1 = dQ_dyn (widened to float) and delta1 = rowsum(dZ1 * Z1); one warp per
+// latent row.
+template <typename T>
+__global__ void pp_dz1_kernel(const T* __restrict__ dqd, const float* __restrict__ z1,
+                              int64_t rows, int D, float* __restrict__ dz1,
+                              float* __restrict__ delta1) {
+  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= rows) return;
+  float v = 0.f, prod = 0.f;
+  if (lane < D) {
+    v = to_f(dqd[w * D + lane]);
+    prod = v * z1[w * D + lane];
+    dz1[w * D + lane] = v;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) prod += __shfl_xor_sync(0xffffffffu, prod, o);
+  if (lane == 0) delta1[w] = prod;
+}
+
+// The first encode's gradient, added into dK and dV (read-modify-write of
+// each thread's own token rows), with per-chunk partials of its dQ part.
+template <typename T, int D>
+__global__ void __launch_bounds__(kT)
+    pp_encode_bwd_kernel(const T* __restrict__ Q, const T* __restrict__ K,
+                         const T* __restrict__ V, const float* __restrict__ lse1,
+                         const float* __restrict__ dz1, const float* __restrict__ delta1, int H,
+                         int64_t N, int M, float c, float s, int64_t chunk_tokens,
+                         T* __restrict__ dK, T* __restrict__ dV, float* __restrict__ dq_part) {
+  extern __shared__ float sm[];
+  float* qs = sm;                 // [M][D]
+  float* dzs = qs + M * D;        // [M][D]
+  float* ls = dzs + M * D;        // [M] lse1 in log2 units
+  float* des = ls + M;            // [M] delta1
+  float* ks = des + M;            // [kT][D]
+  float* vs = ks + kT * D;        // [kT][D]
+  const int chunk = blockIdx.x, chunks = gridDim.x;
+  const int64_t bh = blockIdx.y, h = bh % H;
+  const int64_t n0 = (int64_t)chunk * chunk_tokens, n1 = min(N, n0 + chunk_tokens);
+  for (int i = threadIdx.x; i < M * D; i += blockDim.x) {
+    qs[i] = to_f(Q[h * (int64_t)M * D + i]);
+    dzs[i] = dz1[bh * M * D + i];
+  }
+  for (int i = threadIdx.x; i < M; i += blockDim.x) {
+    ls[i] = lse1[bh * M + i] * kLog2e;
+    des[i] = delta1[bh * M + i];
+  }
+  const int tid = threadIdx.x;
+  const bool active_m = tid < M;
+  float dq[D];
+#pragma unroll
+  for (int d = 0; d < D; ++d) dq[d] = 0.f;
+
+  for (int64_t t0 = n0; t0 < n1; t0 += kT) {
+    const int nt = (int)imin64(kT, n1 - t0);
+    __syncthreads();
+    for (int i = tid; i < kT * D; i += blockDim.x) {
+      const int j = i / D;
+      const int64_t g = (bh * N + t0) * D + i;
+      ks[i] = (j < nt) ? to_f(K[g]) : 0.f;
+      vs[i] = (j < nt) ? to_f(V[g]) : 0.f;
+    }
+    __syncthreads();
+    // one thread per token: the encode's dV and dK parts, added to the rows
+    if (tid < nt) {
+      const int64_t n = t0 + tid;
+      float k[D], v[D], dk[D], dv[D];
+#pragma unroll
+      for (int d = 0; d < D; ++d) {
+        k[d] = ks[tid * D + d];
+        v[d] = vs[tid * D + d];
+        dk[d] = 0.f;
+        dv[d] = 0.f;
+      }
+      for (int m = 0; m < M; ++m) {
+        float a = 0.f, dp = 0.f;
+#pragma unroll
+        for (int d = 0; d < D; ++d) {
+          a = fmaf(k[d], qs[m * D + d], a);
+          dp = fmaf(dzs[m * D + d], v[d], dp);
+        }
+        const float p = exp2f(a * c - ls[m]);
+        const float dA = s * p * (dp - des[m]);
+#pragma unroll
+        for (int d = 0; d < D; ++d) {
+          dv[d] = fmaf(p, dzs[m * D + d], dv[d]);
+          dk[d] = fmaf(dA, qs[m * D + d], dk[d]);
+        }
+      }
+#pragma unroll
+      for (int d = 0; d < D; ++d) {
+        const int64_t o = (bh * N + n) * D + d;
+        dK[o] = from_f<T>(to_f(dK[o]) + dk[d]);
+        dV[o] = from_f<T>(to_f(dV[o]) + dv[d]);
+      }
+    }
+    // one thread per latent: the encode's part of dQ over this tile
+    if (active_m) {
+      float q[D], dzr[D];
+#pragma unroll
+      for (int d = 0; d < D; ++d) {
+        q[d] = qs[tid * D + d];
+        dzr[d] = dzs[tid * D + d];
+      }
+      const float lm = ls[tid], dm = des[tid];
+      for (int j = 0; j < nt; ++j) {
+        float a = 0.f, dp = 0.f;
+#pragma unroll
+        for (int d = 0; d < D; ++d) {
+          a = fmaf(ks[j * D + d], q[d], a);
+          dp = fmaf(dzr[d], vs[j * D + d], dp);
+        }
+        const float dA = s * exp2f(a * c - lm) * (dp - dm);
+#pragma unroll
+        for (int d = 0; d < D; ++d) dq[d] = fmaf(dA, ks[j * D + d], dq[d]);
+      }
+    }
+  }
+  if (active_m) {
+    const int64_t row = (bh * chunks + chunk) * M + tid;
+#pragma unroll
+    for (int d = 0; d < D; ++d) dq_part[row * D + d] = dq[d];
+  }
+}
+
+// dQ[h] = sum over b of (dQ_dyn[b, h] + sum over chunks of the encode
+// partials), in a fixed order.  One thread per output element.
+template <typename T>
+__global__ void pp_dq_kernel(const T* __restrict__ dqd, const float* __restrict__ dq_part, int B,
+                             int H, int M, int D, int chunks, T* __restrict__ dQ) {
+  const int64_t per = (int64_t)H * M * D;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= per) return;
+  const int64_t h = i / ((int64_t)M * D);
+  const int64_t md = i % ((int64_t)M * D);
+  float acc = 0.f;
+  for (int b = 0; b < B; ++b) {
+    const int64_t bh = (int64_t)b * H + h;
+    acc += to_f(dqd[(int64_t)b * per + i]);
+    for (int k = 0; k < chunks; ++k) acc += dq_part[(bh * chunks + k) * (int64_t)M * D + md];
+  }
+  dQ[i] = from_f<T>(acc);
+}
+
+template <typename T, int D>
+cudaError_t pp_tail_t(const void* Q, const void* K, const void* V, const float* z1,
+                      const float* lse1, const void* dqd, void* dQ, void* dK, void* dV,
+                      const Dims& d, float scale, const WsLayout& L, char* ws, cudaStream_t st) {
+  const ChunkPlan& p = L.ppe;
+  const int M = (int)d.M;
+  const int64_t BH = d.BH();
+  float* dz1 = (float*)(ws + L.dz1);
+  float* delta1 = (float*)(ws + L.delta1);
+  float* dqe = (float*)(ws + L.dqe);
+  cudaError_t e;
+  const int64_t rows = BH * M;
+  pp_dz1_kernel<T><<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>((const T*)dqd, z1, rows,
+                                                                        D, dz1, delta1);
+  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+  const size_t smem = (size_t)(2 * M * D + 2 * M + 2 * kT * D) * sizeof(float);
+  e = cudaFuncSetAttribute(pp_encode_bwd_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.chunks, (unsigned)BH);
+  pp_encode_bwd_kernel<T, D><<<grid, kT, smem, st>>>(
+      (const T*)Q, (const T*)K, (const T*)V, lse1, dz1, delta1, (int)d.H, d.N, M,
+      scale * kLog2e, scale, p.chunk_tokens(), (T*)dK, (T*)dV, dqe);
+  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+  const int64_t per = d.H * M * D;
+  pp_dq_kernel<T><<<(unsigned)((per + 255) / 256), 256, 0, st>>>((const T*)dqd, dqe, (int)d.B,
+                                                                 (int)d.H, M, D, p.chunks,
+                                                                 (T*)dQ);
+  return cudaPeekAtLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_pp_bwd_tail(const void* Q, const void* K, const void* V, const float* z1,
+                               const float* lse1, const void* dqd, void* dQ, void* dK, void* dV,
+                               const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,
+                               char* ws, cudaStream_t st) {
+  if (dt == FLARE_F32)
+    return d.D == 16 ? pp_tail_t<float, 16>(Q, K, V, z1, lse1, dqd, dQ, dK, dV, d, scale, L, ws, st)
+                     : pp_tail_t<float, 32>(Q, K, V, z1, lse1, dqd, dQ, dK, dV, d, scale, L, ws, st);
+  return d.D == 16
+             ? pp_tail_t<__nv_bfloat16, 16>(Q, K, V, z1, lse1, dqd, dQ, dK, dV, d, scale, L, ws, st)
+             : pp_tail_t<__nv_bfloat16, 32>(Q, K, V, z1, lse1, dqd, dQ, dK, dV, d, scale, L, ws, st);
+}
+
+}  // namespace flare

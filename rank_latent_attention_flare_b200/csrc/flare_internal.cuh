@@ -149,8 +149,15 @@ struct WsLayout {
   size_t aug = 0;       // [BH][M][16] bf16 extra K-step row (-f delta_e in three terms)
   size_t params = 0;    // [BH] float2  R, fast-form flag
   size_t lse2 = 0;      // [BH][M] float  lse in log2 units
+  // FLARE++ backward, in addition to the FLARE backward's buffers
+  size_t z1 = 0;        // [BH][M][D] float  first encode's Z1 (recomputed)
+  size_t lse1 = 0;      // [BH][M] float  its lse
+  size_t dqd = 0;       // [BH][M][D] dtype  dQ_dyn
+  size_t dz1 = 0;       // [BH][M][D] float  dQ_dyn widened
+  size_t delta1 = 0;    // [BH][M] float  rowsum(dZ1 * Z1)
+  size_t dqe = 0;       // [BH*chunks][M][D] float  first encode's dQ partials
   size_t total = 0;
-  ChunkPlan enc, bwd;
+  ChunkPlan enc, bwd, ppe;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -174,7 +181,8 @@ inline WsLayout ws_layout(flare_op_t op, int64_t B, int64_t H, int64_t N, int64_
   L.zf = take((size_t)BH * M * D * 4);
   L.zb = take((size_t)BH * M * D * 2);
   if (op == FLARE_OP_PP_FWD) L.qdyn = take((size_t)BH * M * D * esz);
-  if (op == FLARE_OP_BWD && choose_path(N, M, D, dt).tc_bwd) {
+  const bool bwd_like = (op == FLARE_OP_BWD || op == FLARE_OP_PP_BWD);
+  if (bwd_like && choose_path(N, M, D, dt).tc_bwd) {
     L.bwd = tc_bwd_plan(BH, N, sms);
     const int64_t bslots = BH * L.bwd.chunks;
     L.stats = take((size_t)BH * N * 16);
@@ -187,7 +195,7 @@ inline WsLayout ws_layout(flare_op_t op, int64_t B, int64_t H, int64_t N, int64_
     L.aug = take((size_t)BH * M * 16 * 2);
     L.params = take((size_t)BH * 8);
     L.lse2 = take((size_t)BH * M * 4);
-  } else if (op == FLARE_OP_BWD) {
+  } else if (bwd_like) {
     L.bwd = bwd_plan(BH, N, sms);
     const int64_t bslots = BH * L.bwd.chunks;
     L.dkf = take((size_t)BH * N * D * 4);
@@ -195,6 +203,15 @@ inline WsLayout ws_layout(flare_op_t op, int64_t B, int64_t H, int64_t N, int64_
     L.dzp = take((size_t)bslots * M * D * 4);
     L.dz = take((size_t)BH * M * D * 4);
     L.delta = take((size_t)BH * M * 4);
+  }
+  if (op == FLARE_OP_PP_BWD) {
+    L.ppe = bwd_plan(BH, N, sms);
+    L.z1 = take((size_t)BH * M * D * 4);
+    L.lse1 = take((size_t)BH * M * 4);
+    L.dqd = take((size_t)BH * M * D * esz);
+    L.dz1 = take((size_t)BH * M * D * 4);
+    L.delta1 = take((size_t)BH * M * 4);
+    L.dqe = take((size_t)BH * L.ppe.chunks * M * D * 4);
   }
   L.total = off;
   return L;
@@ -265,6 +282,10 @@ cudaError_t launch_tc_bwd(const void* Q, int64_t qbs, const void* K, const void*
                           const void* dY, const float* Z, const float* lse, void* dQ, void* dK,
                           void* dV, const Dims& d, float scale, const WsLayout& L, char* ws,
                           cudaStream_t st);
+cudaError_t launch_pp_bwd_tail(const void* Q, const void* K, const void* V, const float* z1,
+                               const float* lse1, const void* dqd, void* dQ, void* dK, void* dV,
+                               const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,
+                               char* ws, cudaStream_t st);
 cudaError_t launch_bwd(const void* Q, int64_t qbs, const void* K, const void* V, const void* dY,
                        const float* Z, const float* lse, void* dQ, void* dK, void* dV,
                        const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,

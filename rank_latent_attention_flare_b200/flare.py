@@ -157,6 +157,28 @@ def flare_bwd(Q, K, V, dY, Z, lse, scale: Optional[float] = None, *,
     return dQ, dK, dV
 
 
+def flare_pp_bwd(Q, K, V, dY, Q_dyn, Z, lse, scale: Optional[float] = None, *,
+                 workspace: Optional[torch.Tensor] = None, stream=None):
+    """FLARE++ backward with learned Q [H,M,D] (Q_dyn, Z, lse from
+    flare_pp_fwd(..., save=True)).  Returns (dQ [H,M,D], dK, dV)."""
+    _need_cuda(Q, K, V, dY, Q_dyn, Z, lse, workspace)
+    B, H, N, M, D, qbs = _dims(Q, K)
+    if qbs != 0:
+        raise ValueError("FLARE++ takes learned latents Q of shape [H,M,D]")
+    dt = _dtype_code(K)
+    s = default_scale(D) if scale is None else float(scale)
+    dQ = torch.empty_like(Q)
+    dK = torch.empty_like(K)
+    dV = torch.empty_like(V)
+    ws = workspace if workspace is not None else alloc_workspace(
+        _lib.FLARE_OP_PP_BWD, B, H, N, M, D, K.dtype, K.device)
+    st = _lib.load().flare_pp_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(dY), _ptr(Q_dyn), _ptr(Z),
+                                  _ptr(lse), _ptr(dQ), _ptr(dK), _ptr(dV), B, H, N, M, D, dt, s,
+                                  _ptr(ws), ws.numel(), _stream(stream))
+    _lib.check(st, "flare_pp_bwd")
+    return dQ, dK, dV
+
+
 def flare_encode(Q, K, V, scale: Optional[float] = None, *, workspace: torch.Tensor,
                  stream=None) -> None:
     """Stage 1: encode partials into ``workspace`` (FLARE_OP_FWD size)."""

@@ -176,6 +176,15 @@ def test_other_entry_points_validate(lib):
                          1, 2, 100, 32, 16, 0, 0.25, _p(F), ws_b, None) == INVALID
     assert lib.flare_bwd(_p(F), 0, _p(F), _p(F), _p(F), _p(F), _p(F), _p(F), _p(F), _p(F),
                          1, 2, 100, 32, 16, 0, 0.25, _p(F), ws_b - 1, None) == WORKSPACE
+    ws_ppb = lib.flare_workspace_size(3, 1, 2, 100, 32, 16, 0)
+    assert ws_ppb > ws_b
+    # FLARE++ backward: Q_dyn, Z_save and lse_save are required
+    assert lib.flare_pp_bwd(_p(F), _p(F), _p(F), _p(F), None, _p(F), _p(F), _p(F), _p(F), _p(F),
+                            1, 2, 100, 32, 16, 0, 0.25, _p(F), ws_ppb, None) == INVALID
+    assert lib.flare_pp_bwd(_p(F), _p(F), _p(F), _p(F), _p(F), _p(F), None, _p(F), _p(F), _p(F),
+                            1, 2, 100, 32, 16, 0, 0.25, _p(F), ws_ppb, None) == INVALID
+    assert lib.flare_pp_bwd(_p(F), _p(F), _p(F), _p(F), _p(F), _p(F), _p(F), _p(F), _p(F), _p(F),
+                            1, 2, 100, 32, 16, 0, 0.25, _p(F), ws_ppb - 1, None) == WORKSPACE
     ws_f = lib.flare_workspace_size(0, 1, 2, 100, 32, 16, 0)
     assert lib.flare_encode(None, 0, _p(F), _p(F), 1, 2, 100, 32, 16, 0, 0.25, _p(F), ws_f,
                             None) == INVALID

@@ -75,3 +75,51 @@ def test_bwd_single_token_closed_form(dtype):
     assert float(dQ.float().abs().max()) <= tol
     assert float(dK.float().abs().max()) <= tol
     assert float((dV.float() - g["dY"].float()).abs().max()) <= tol
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("B,H,N,M,D", [(2, 2, 600, 128, 32), (1, 2, 257, 256, 16),
+                                       (2, 1, 300, 32, 16), (2, 2, 1000, 128, 16)])
+def test_pp_bwd_matches_oracle(B, H, N, M, D, dtype):
+    s = 1.0 / math.sqrt(D)
+    x = make_inputs(B, H, N, M, D, dtype=dtype, seed=51 + N, with_dy=True)
+    g = {k: v.to(DEV) for k, v in x.items()}
+    Y, Qd, Z, lse = fl.flare_pp_fwd(g["Q"], g["K"], g["V"], s, save=True)
+    ws = fl.alloc_workspace(fl.FLARE_OP_PP_BWD, B, H, N, M, D, dtype, DEV)
+    ws.fill_(0xFF)   # NaN in every float the kernels might read unwritten
+    dQ, dK, dV = fl.flare_pp_bwd(g["Q"], g["K"], g["V"], g["dY"], Qd, Z, lse, s, workspace=ws)
+    assert fl.device_status(ws) == 0
+    dQo, dKo, dVo = oracle.flare_pp_bwd(x["Q"], x["K"], x["V"], x["dY"], s)
+    assert_close(dV, dVo, dtype, "dV", rel_f32=TOL_F32_GRAD_REL)
+    assert_close(dK, dKo, dtype, "dK", rel_f32=TOL_F32_GRAD_REL)
+    assert_close(dQ, dQo, dtype, "dQ", rel_f32=TOL_F32_GRAD_REL)
+
+
+def test_pp_bwd_is_bitwise_deterministic():
+    B, H, N, M, D = 2, 2, 2000, 128, 32
+    s = 1.0 / math.sqrt(D)
+    x = make_inputs(B, H, N, M, D, dtype=torch.bfloat16, seed=52, with_dy=True)
+    g = {k: v.to(DEV) for k, v in x.items()}
+    Y, Qd, Z, lse = fl.flare_pp_fwd(g["Q"], g["K"], g["V"], s, save=True)
+    a = fl.flare_pp_bwd(g["Q"], g["K"], g["V"], g["dY"], Qd, Z, lse, s)
+    b = fl.flare_pp_bwd(g["Q"], g["K"], g["V"], g["dY"], Qd, Z, lse, s)
+    torch.cuda.synchronize()
+    for u, v in zip(a, b):
+        assert torch.equal(u, v)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_pp_bwd_single_token_closed_form(dtype):
+    # One token: both encodes return V[0] for every latent and the decode
+    # returns Y = V[0] whatever Q and K are, so dQ = dK = 0 and dV = dY.
+    B, H, N, M, D = 1, 3, 1, 16, 32
+    s = 1.0 / math.sqrt(D)
+    x = make_inputs(B, H, N, M, D, dtype=dtype, seed=53, with_dy=True)
+    g = {k: v.to(DEV) for k, v in x.items()}
+    Y, Qd, Z, lse = fl.flare_pp_fwd(g["Q"], g["K"], g["V"], s, save=True)
+    dQ, dK, dV = fl.flare_pp_bwd(g["Q"], g["K"], g["V"], g["dY"], Qd, Z, lse, s)
+    torch.cuda.synchronize()
+    tol = 1e-5 if dtype == torch.float32 else 3e-2
+    assert float(dQ.float().abs().max()) <= tol
+    assert float(dK.float().abs().max()) <= tol
+    assert float((dV.float() - g["dY"].float()).abs().max()) <= tol
