@@ -417,7 +417,7 @@ def _row_roofline(t_ms: float, exps: float, flops: float, hbm_bytes: float, peak
 
 
 def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0,
-                    which=("flare_pp_fwd", "flare_fwd_bwd")):
+                    which=("flare_pp_fwd", "flare_fwd_bwd", "flare_pp_fwd_bwd")):
     """Times the FLARE++ forward (B=2 H=8 N=262,144 M=256 D=32) and the
     forward + backward of B=8 H=8 N=16,384 M=128 D=32, both bf16, on the
     same device with CUDA events (median of `iters` launches after 3
@@ -449,6 +449,8 @@ def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0,
         rows.update(_time_pp(dev, peaks, peak_kind, timed, seed))
     if "flare_fwd_bwd" in which:
         rows.update(_time_fwd_bwd(dev, peaks, peak_kind, timed, seed))
+    if "flare_pp_fwd_bwd" in which:
+        rows.update(_time_pp_fwd_bwd(dev, peaks, peak_kind, timed, seed))
     del flush_buf
     torch.cuda.empty_cache()
     return rows
@@ -540,6 +542,41 @@ def time_sdpa_context(dev, w=WORKLOAD, iters: int = 5, seed: int = 0):
             "ms": round(ms, 4), "tokens_per_s": w.B * w.N / (ms / 1e3)}
 
 
+def _time_pp_fwd_bwd(dev, peaks, peak_kind, timed, seed):
+    """FLARE++ forward + backward on the forward + backward workload's shape
+    (B=8 H=8 N=16,384 M=128 D=32 bf16).  Algorithmic work per token-head:
+    forward 3 M exponentials, 12 M D tensor FLOPs, K read 3x, V 2x, Y written;
+    backward 3 M exponentials (P_d, P_e of the second encode, P of the first),
+    30 M D tensor FLOPs, K, V, dY read and dK, dV written once."""
+    import rank_latent_attention_flare_b200 as fl
+    w = WORKLOADS["c5_fwdbwd_bf16_16k"]
+    x = make_inputs(w.B, w.H, w.N, w.M, w.D, dtype=w.torch_dtype, seed=seed, with_dy=True)
+    g = {k: v.to(dev) for k, v in x.items()}
+    wsf = fl.alloc_workspace(fl.FLARE_OP_PP_FWD, w.B, w.H, w.N, w.M, w.D, w.torch_dtype, dev)
+    wsb = fl.alloc_workspace(fl.FLARE_OP_PP_BWD, w.B, w.H, w.N, w.M, w.D, w.torch_dtype, dev)
+    saved = {}
+
+    def fwd():
+        saved["out"] = fl.flare_pp_fwd(g["Q"], g["K"], g["V"], w.scale, save=True, workspace=wsf)
+
+    ms_f = timed(fwd)
+    _, Qd, Z, lse = saved["out"]
+    ms_b = timed(lambda: fl.flare_pp_bwd(g["Q"], g["K"], g["V"], g["dY"], Qd, Z, lse, w.scale,
+                                         workspace=wsb))
+    if fl.device_status(wsf) != 0 or fl.device_status(wsb) != 0:
+        raise RuntimeError("device wait ran out in the FLARE++ forward + backward")
+    u = w.B * w.H * w.N
+    ms = ms_f + ms_b
+    return {"flare_pp_fwd_bwd": {
+        "workload": f"FLARE++ fwd+bwd B={w.B} H={w.H} N={w.N} M={w.M} D={w.D} bf16",
+        "ms": round(ms, 4), "fwd_ms": round(ms_f, 4), "bwd_ms": round(ms_b, 4),
+        "tokens_per_s": w.B * w.N / (ms / 1e3),
+        "roofline": _row_roofline(ms, 6.0 * u * w.M, 42.0 * u * w.M * w.D,
+                                  11.0 * u * w.D * 2, peaks, peak_kind),
+        "bwd_roofline": _row_roofline(ms_b, 3.0 * u * w.M, 30.0 * u * w.M * w.D,
+                                      5.0 * u * w.D * 2, peaks, peak_kind)}}
+
+
 def run_row(args, rank, local):
     """One of the other workloads alone (FLARE++ forward, or forward +
     backward), e.g. for a profiler capture."""
@@ -602,7 +639,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true",
                     help="skip the FLARE++ and forward+backward timings")
-    ap.add_argument("--row", choices=["flare_pp_fwd", "flare_fwd_bwd"], default=None,
+    ap.add_argument("--row", choices=["flare_pp_fwd", "flare_fwd_bwd", "flare_pp_fwd_bwd"],
+                    default=None,
                     help="time only this workload (one JSON line with its timing and roofline)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=120.0)

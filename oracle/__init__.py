@@ -63,8 +63,10 @@ def _load():
                                          _i64, _i64, ctypes.c_double, _c_dp, _c_dp, _c_dp]
         lib.oracle_flare_pp_bwd.argtypes = [_c_dp, _c_dp, _c_dp, _c_dp, _i64, _i64, _i64, _i64,
                                             _i64, ctypes.c_double, _c_dp, _c_dp, _c_dp]
+        lib.oracle_encode_bwd.argtypes = lib.oracle_flare_pp_bwd.argtypes
         for f in ("oracle_encode", "oracle_decode", "oracle_decode_rows", "oracle_flare_fwd",
-                  "oracle_flare_pp_fwd", "oracle_flare_bwd", "oracle_flare_pp_bwd"):
+                  "oracle_flare_pp_fwd", "oracle_flare_bwd", "oracle_flare_pp_bwd",
+                  "oracle_encode_bwd"):
             getattr(lib, f).restype = None
         _lib = lib
     return _lib
@@ -169,6 +171,21 @@ def flare_bwd(Q, K, V, dY, scale: float):
     dV = np.empty((B, H, N, D))
     _load().oracle_flare_bwd(_p(Q), qbs, _p(K), _p(V), _p(dY), B, H, N, M, D, float(scale),
                              _p(dQ), _p(dK), _p(dV))
+    return dQ, dK, dV
+
+
+def encode_bwd(Q, K, V, dZ, scale: float):
+    """Gradients (dQ [H,M,D] summed over the batch, dK, dV) of sum(Z * dZ) for
+    the encode Z = softmax_N(s Q K^T) V with Q [H,M,D] shared over the batch
+    (the FLARE paper's encode step; FLARE++ uses it for the first encode)."""
+    Q, K, V, dZ = _f64(Q), _f64(K), _f64(V), _f64(dZ)
+    B, H, N, M, D, _ = _shapes(Q, K, True)
+    assert dZ.shape == (B, H, M, D), dZ.shape
+    dQ = np.empty(Q.shape)
+    dK = np.empty((B, H, N, D))
+    dV = np.empty((B, H, N, D))
+    _load().oracle_encode_bwd(_p(Q), _p(K), _p(V), _p(dZ), B, H, N, M, D, float(scale),
+                              _p(dQ), _p(dK), _p(dV))
     return dQ, dK, dV
 
 

@@ -361,6 +361,18 @@ static void encode_bwd_add(const double* Q, const double* K, const double* V,
   free(dQbh);
 }
 
+/* The encode's gradient alone (outputs overwritten): dQ [H,M,D] summed over
+ * the batch, dK, dV [B,H,N,D]. */
+void oracle_encode_bwd(const double* Q, const double* K, const double* V,
+                       const double* dZ1, int64_t B, int64_t H, int64_t N,
+                       int64_t M, int64_t D, double scale, double* dQ,
+                       double* dK, double* dV) {
+  memset(dQ, 0, (size_t)(H * M * D) * sizeof(double));
+  memset(dK, 0, (size_t)(B * H * N * D) * sizeof(double));
+  memset(dV, 0, (size_t)(B * H * N * D) * sizeof(double));
+  encode_bwd_add(Q, K, V, dZ1, B, H, N, M, D, scale, dQ, dK, dV);
+}
+
 /*
  * Gradient of L = sum(Y * dY) for FLARE++ with learned Q [H,M,D]:
  *   Q_dyn = Q + Z1, Z1 = encode(Q, K, V)      (per batch)

@@ -552,6 +552,8 @@ cudaError_t launch_pp_bwd_tail(const void* Q, const void* K, const void* V, cons
                                const float* lse1, const void* dqd, void* dQ, void* dK, void* dV,
                                const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,
                                char* ws, cudaStream_t st) {
+  if (choose_path(d.N, d.M, d.D, dt).tc_bwd)
+    return launch_tc_enc_bwd(Q, K, V, z1, lse1, dqd, dQ, dK, dV, d, scale, L, ws, st);
   if (dt == FLARE_F32)
     return d.D == 16 ? pp_tail_t<float, 16>(Q, K, V, z1, lse1, dqd, dQ, dK, dV, d, scale, L, ws, st)
                      : pp_tail_t<float, 32>(Q, K, V, z1, lse1, dqd, dQ, dK, dV, d, scale, L, ws, st);

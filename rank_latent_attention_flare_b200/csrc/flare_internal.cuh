@@ -205,10 +205,13 @@ inline WsLayout ws_layout(flare_op_t op, int64_t B, int64_t H, int64_t N, int64_
     L.delta = take((size_t)BH * M * 4);
   }
   if (op == FLARE_OP_PP_BWD) {
-    L.ppe = bwd_plan(BH, N, sms);
     L.z1 = take((size_t)BH * M * D * 4);
     L.lse1 = take((size_t)BH * M * 4);
     L.dqd = take((size_t)BH * M * D * esz);
+  }
+  if (op == FLARE_OP_PP_BWD && !choose_path(N, M, D, dt).tc_bwd) {
+    // the first encode's gradient on CUDA cores
+    L.ppe = bwd_plan(BH, N, sms);
     L.dz1 = take((size_t)BH * M * D * 4);
     L.delta1 = take((size_t)BH * M * 4);
     L.dqe = take((size_t)BH * L.ppe.chunks * M * D * 4);
@@ -282,6 +285,13 @@ cudaError_t launch_tc_bwd(const void* Q, int64_t qbs, const void* K, const void*
                           const void* dY, const float* Z, const float* lse, void* dQ, void* dK,
                           void* dV, const Dims& d, float scale, const WsLayout& L, char* ws,
                           cudaStream_t st);
+// FLARE++'s first-encode gradient on the tensor cores (bf16, M = 128,
+// D in {16, 32}): adds into dK, dV and writes dQ (sum over the batch of dZ1
+// and the encode's dQ); reuses the tensor-core backward's workspace.
+cudaError_t launch_tc_enc_bwd(const void* Q, const void* K, const void* V, const float* Z1,
+                              const float* lse1, const void* dZ1, void* dQ, void* dK, void* dV,
+                              const Dims& d, float scale, const WsLayout& L, char* ws,
+                              cudaStream_t st);
 cudaError_t launch_pp_bwd_tail(const void* Q, const void* K, const void* V, const float* z1,
                                const float* lse1, const void* dqd, void* dQ, void* dK, void* dV,
                                const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,

@@ -567,7 +567,8 @@ __global__ void __launch_bounds__(kM)
 // (= -f delta_e) as three bf16 terms, then zeros.
 template <int D>
 __global__ void __launch_bounds__(kM)
-    bwd_mid_kernel(const float* __restrict__ dz_part, int chunks, const float* __restrict__ Z,
+    bwd_mid_kernel(const float* __restrict__ dz_part, int chunks,
+                   const __nv_bfloat16* __restrict__ dz_direct, const float* __restrict__ Z,
                    const float* __restrict__ lse, __nv_bfloat16* __restrict__ dzs,
                    uint32_t* __restrict__ aug, const uint32_t* __restrict__ flags,
                    float2* __restrict__ params, float* __restrict__ lse2_out) {
@@ -578,6 +579,10 @@ __global__ void __launch_bounds__(kM)
   float dz[D];
 #pragma unroll
   for (int d = 0; d < D; ++d) dz[d] = 0.f;
+  if (dz_direct) {   // FLARE++'s first encode: dZ1 = dQ_dyn
+#pragma unroll
+    for (int d = 0; d < D; ++d) dz[d] = __bfloat162float(dz_direct[row * D + d]);
+  }
   for (int k = 0; k < chunks; ++k) {
     const float4* p = reinterpret_cast<const float4*>(dz_part + ((bh * chunks + k) * kM + m) * D);
 #pragma unroll
@@ -674,7 +679,7 @@ __global__ void __launch_bounds__(kThr, 1)
                     const __grid_constant__ CUtensorMap tmAug, int H, int64_t N, int q_per_batch,
                     float c, float s, int64_t tiles_per_bh, int64_t chunk_tiles,
                     const float4* __restrict__ stats, const float2* __restrict__ params,
-                    const float* __restrict__ lse2, __nv_bfloat16* __restrict__ dK,
+                    const float* __restrict__ lse2, int enc_only, __nv_bfloat16* __restrict__ dK,
                     __nv_bfloat16* __restrict__ dV, float* __restrict__ dq_part,
                     uint32_t* __restrict__ err) {
   using L = BLayout<D>;
@@ -929,12 +934,26 @@ __global__ void __launch_bounds__(kThr, 1)
       if (tok < N) {
         const float f = (w == 0) ? s : gv;
         uint4* dst = reinterpret_cast<uint4*>((w == 0 ? dK : dV) + (bh * N + tok) * D);
+        if (enc_only) {   // added to the gradient already in the rows
+#pragma unroll
+          for (int v = 0; v < D / 8; ++v) {
+            const uint4 q4 = dst[v];
+            const uint32_t qq[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              o[8 * v + 2 * jj] = fmaf(o[8 * v + 2 * jj], f, bf_lo(qq[jj]));
+              o[8 * v + 2 * jj + 1] = fmaf(o[8 * v + 2 * jj + 1], f, bf_hi(qq[jj]));
+            }
+          }
+        } else {
+#pragma unroll
+          for (int d = 0; d < D; ++d) o[d] *= f;
+        }
 #pragma unroll
         for (int v = 0; v < D / 8; ++v)
-          dst[v] = make_uint4(pack_bf16(o[8 * v] * f, o[8 * v + 1] * f),
-                              pack_bf16(o[8 * v + 2] * f, o[8 * v + 3] * f),
-                              pack_bf16(o[8 * v + 4] * f, o[8 * v + 5] * f),
-                              pack_bf16(o[8 * v + 6] * f, o[8 * v + 7] * f));
+          dst[v] = make_uint4(pack_bf16(o[8 * v], o[8 * v + 1]), pack_bf16(o[8 * v + 2], o[8 * v + 3]),
+                              pack_bf16(o[8 * v + 4], o[8 * v + 5]),
+                              pack_bf16(o[8 * v + 6], o[8 * v + 7]));
       }
       return true;
     };
@@ -948,7 +967,7 @@ __global__ void __launch_bounds__(kThr, 1)
         const int64_t tok = (tile0 + t) * kT + r;
         valid = tok < N;
         if (valid) {
-          const float4 st = stats[bh * N + tok];
+          const float4 st = enc_only ? make_float4(0.f, 0.f, 0.f, 0.f) : stats[bh * N + tok];
           mxp = st.x;
           dd = st.y;
           g = 1.f;
@@ -985,7 +1004,8 @@ __global__ void __launch_bounds__(kThr, 1)
           const uint64_t E2 = f32x2(__uint_as_float(e[2 * p]), __uint_as_float(e[2 * p + 1]));
           float x0, x1;
           split_f32x2(fma_f32x2(S2, c2, nm2), x0, x1);
-          const float p0 = ex2(x0), p1 = ex2(x1);
+          // an encode-only gradient has no decode term: P_d = 0
+          const float p0 = enc_only ? 0.f : ex2(x0), p1 = enc_only ? 0.f : ex2(x1);
           // exact form: P_e = 2^(c S - lse2[m]); G = P_d (dPd - delta_d) + P_e dPe'
           float s0, s1, e0, e1;
           split_f32x2(S2, s0, s1);
@@ -1106,8 +1126,9 @@ __global__ void __launch_bounds__(kThr, 1)
                          const __grid_constant__ CUtensorMap tmAug, int H, int64_t N, int q_per_batch,
                          float c, float s, int64_t tiles_per_bh, int64_t chunk_tiles,
                          const float4* __restrict__ stats, const float2* __restrict__ params,
-                         __nv_bfloat16* __restrict__ dK, __nv_bfloat16* __restrict__ dV,
-                         float* __restrict__ dq_part, uint32_t* __restrict__ err) {
+                         int enc_only, __nv_bfloat16* __restrict__ dK,
+                         __nv_bfloat16* __restrict__ dV, float* __restrict__ dq_part,
+                         uint32_t* __restrict__ err) {
   using L = BFLayout<D>;
   constexpr int M = L::M;
   constexpr int NS = L::NSLOT;
@@ -1223,9 +1244,9 @@ __global__ void __launch_bounds__(kThr, 1)
             break;
           }
           uint8_t* dst = smem + L::VD_OFF + vb * 2 * L::TILE;
-          mbar_arrive_expect_tx(&v_full[vb], 2 * L::TILE);
+          mbar_arrive_expect_tx(&v_full[vb], (enc_only ? 1 : 2) * L::TILE);
           tma_load_3d(dst, &tmV, &v_full[vb], 0, tok, (int32_t)bh);
-          tma_load_3d(dst + L::TILE, &tmdY2, &v_full[vb], 0, tok, (int32_t)bh);
+          if (!enc_only) tma_load_3d(dst + L::TILE, &tmdY2, &v_full[vb], 0, tok, (int32_t)bh);
           issued = t + 1;
         }
         // let every load still in flight land before the CTA can exit
@@ -1281,14 +1302,17 @@ __global__ void __launch_bounds__(kThr, 1)
           const uint32_t vo = (uint32_t)(2 * vb) * kTile16;     // V at vo, dY'' at vo + kTile16
           const uint32_t ro = (uint32_t)(64 * hf * RB) >> 4;   // latent rows [64 hf, +64)
           // the S and U chains interleaved, so consecutive MMAs are independent
+          // (an encode-only gradient has no dY'' Z^T term)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             mma_ss(base, dK0 + ko + 2 * kk, dQk + ro + 2 * kk, idH, kk > 0);
-            mma_ss(base + 64, dV0 + vo + kTile16 + 2 * kk, dZk + ro + 2 * kk, idH, kk > 0);
+            if (!enc_only)
+              mma_ss(base + 64, dV0 + vo + kTile16 + 2 * kk, dZk + ro + 2 * kk, idH, kk > 0);
           }
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(base + 64, dV0 + vo + 2 * kk, dDZk + ro + 2 * kk, idH, 1u);
+            mma_ss(base + 64, dV0 + vo + 2 * kk, dDZk + ro + 2 * kk, idH,
+                   (!enc_only || kk > 0) ? 1u : 0u);
           mma_ts(base + 64, tmem + TONE, dAug + (uint32_t)(2 * 64 * hf), idH, 1u);
           mma_commit(&h_full[k % NS]);
           if (hf == 1) mma_commit(&v_empty[vb]);   // V and dY'' of tile t read by both halves
@@ -1360,7 +1384,7 @@ __global__ void __launch_bounds__(kThr, 1)
     // delta'' of this thread's row in tile tt, loaded one tile ahead of use
     auto load_dpp = [&](int tt) -> float {
       const int64_t tok = (tile0 + tt) * kT + r;
-      return (tt < nt && tok < N) ? stats[bh * N + tok].z : 0.f;
+      return (!enc_only && tt < nt && tok < N) ? stats[bh * N + tok].z : 0.f;
     };
     float dpp_next = load_dpp(0);
 
@@ -1391,12 +1415,26 @@ __global__ void __launch_bounds__(kThr, 1)
       if (tok < N) {
         const float f = (w == 0) ? s : 1.f;
         uint4* dst = reinterpret_cast<uint4*>((w == 0 ? dK : dV) + (bh * N + tok) * D);
+        if (enc_only) {   // added to the gradient already in the rows
+#pragma unroll
+          for (int v = 0; v < D / 8; ++v) {
+            const uint4 q4 = dst[v];
+            const uint32_t qq[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              o[8 * v + 2 * jj] = fmaf(o[8 * v + 2 * jj], f, bf_lo(qq[jj]));
+              o[8 * v + 2 * jj + 1] = fmaf(o[8 * v + 2 * jj + 1], f, bf_hi(qq[jj]));
+            }
+          }
+        } else {
+#pragma unroll
+          for (int d = 0; d < D; ++d) o[d] *= f;
+        }
 #pragma unroll
         for (int v = 0; v < D / 8; ++v)
-          dst[v] = make_uint4(pack_bf16(o[8 * v] * f, o[8 * v + 1] * f),
-                              pack_bf16(o[8 * v + 2] * f, o[8 * v + 3] * f),
-                              pack_bf16(o[8 * v + 4] * f, o[8 * v + 5] * f),
-                              pack_bf16(o[8 * v + 6] * f, o[8 * v + 7] * f));
+          dst[v] = make_uint4(pack_bf16(o[8 * v], o[8 * v + 1]), pack_bf16(o[8 * v + 2], o[8 * v + 3]),
+                              pack_bf16(o[8 * v + 4], o[8 * v + 5]),
+                              pack_bf16(o[8 * v + 6], o[8 * v + 7]));
       }
       return true;
     };
@@ -1505,9 +1543,11 @@ __global__ void __launch_bounds__(kThr, 1)
 // dQ = sum over (batch when Q is shared) x chunks of the scaled partials,
 // in a fixed order (batch outer, chunk inner).  One thread per 4 output
 // elements; the partials' loads are issued in groups of 8 before they are
-// added, so their latencies overlap.
+// added, so their latencies overlap.  With Q shared, `extra` (if given,
+// [B][H][M][D] bf16) is summed over the batch first: FLARE++'s dQ_dyn.
 __global__ void bwd_dq_sum_kernel(const float4* __restrict__ dq_part, int B, int H, int M, int D,
-                                  int chunks, bool shared_q, __nv_bfloat16* __restrict__ dQ) {
+                                  int chunks, bool shared_q, const __nv_bfloat16* __restrict__ extra,
+                                  __nv_bfloat16* __restrict__ dQ) {
   const int64_t md4 = (int64_t)M * D / 4;
   const int64_t per4 = (int64_t)H * md4;
   const int64_t total4 = shared_q ? per4 : (int64_t)B * per4;
@@ -1519,6 +1559,15 @@ __global__ void bwd_dq_sum_kernel(const float4* __restrict__ dq_part, int B, int
   const int64_t e = rr % md4;
   const int n = (shared_q ? B : 1) * chunks;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (extra && shared_q) {
+    for (int b = 0; b < B; ++b) {
+      const uint2 x = *reinterpret_cast<const uint2*>(extra + (b * per4 + i) * 4);
+      acc.x += bf_lo(x.x);
+      acc.y += bf_hi(x.x);
+      acc.z += bf_lo(x.y);
+      acc.w += bf_hi(x.y);
+    }
+  }
   for (int q0 = 0; q0 < n; q0 += 8) {
     float4 v[8];
 #pragma unroll
@@ -1586,8 +1635,8 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
                                                 flags, dzp, err);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
-  bwd_mid_kernel<D><<<(unsigned)BH, kM, 0, st>>>(dzp, p.chunks, Z, lse, dzs, (uint32_t*)aug,
-                                                 flags, params, lse2);
+  bwd_mid_kernel<D><<<(unsigned)BH, kM, 0, st>>>(dzp, p.chunks, nullptr, Z, lse, dzs,
+                                                 (uint32_t*)aug, flags, params, lse2);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
   // each head runs in exactly one of the two pass-B kernels (params.y)
@@ -1597,7 +1646,7 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
   if (e != cudaSuccess) return e;
   tc_bwd_b_fast_kernel<D><<<grid, kThr, smemF, st>>>(
       mq, mk, mv, mdy2, mz, mdz, maug, (int)d.H, d.N, q_per_batch, c, scale, p.tiles_per_bh,
-      p.chunk_tiles, stats, params, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, dqp, err);
+      p.chunk_tiles, stats, params, 0, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, dqp, err);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   const int smemB = BLayout<D>::BYTES + 1024;
   e = cudaFuncSetAttribute(tc_bwd_b_exact_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1605,13 +1654,80 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
   if (e != cudaSuccess) return e;
   tc_bwd_b_exact_kernel<D><<<grid, kThr, smemB, st>>>(
       mq, mk, mv, mdy, mz, mdz, maug, (int)d.H, d.N, q_per_batch, c, scale, p.tiles_per_bh,
-      p.chunk_tiles, stats, params, lse2, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, dqp, err);
+      p.chunk_tiles, stats, params, lse2, 0, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, dqp, err);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
   const bool shared_q = (qbs == 0);
   const int64_t total = shared_q ? d.H * kM * D : BH * kM * D;
   bwd_dq_sum_kernel<<<(unsigned)((total / 4 + 127) / 128), 128, 0, st>>>(
-      (const float4*)dqp, (int)d.B, (int)d.H, kM, D, p.chunks, shared_q, (__nv_bfloat16*)dQ);
+      (const float4*)dqp, (int)d.B, (int)d.H, kM, D, p.chunks, shared_q, nullptr,
+      (__nv_bfloat16*)dQ);
+  return cudaPeekAtLastError();
+}
+
+// FLARE++'s first encode, Z1 = softmax_N(s Q K^T) V with Q shared over the
+// batch, differentiated with upstream dZ1 = dQ_dyn: the pass-B kernels in
+// their encode-only form (no decode term; dK, dV added to the rows that
+// FLARE's backward wrote), then dQ = sum over b of (dQ_dyn + the encode's
+// partials).  Runs after FLARE's backward on the same stream and reuses its
+// workspace.
+template <int D>
+cudaError_t tc_enc_bwd_t(const void* Q, const void* K, const void* V, const float* Z1,
+                         const float* lse1, const void* dZ1, void* dQ, void* dK, void* dV,
+                         const Dims& d, float scale, const WsLayout& L, char* ws, cudaStream_t st) {
+  const ChunkPlan& p = L.bwd;
+  const int64_t BH = d.BH();
+  const float c = scale * kLog2e;
+  uint32_t* err = (uint32_t*)(ws + L.hdr);
+  __nv_bfloat16* zb = (__nv_bfloat16*)(ws + L.zb);
+  float4* stats = (float4*)(ws + L.stats);
+  float* rref = (float*)(ws + L.rref);
+  uint32_t* flags = (uint32_t*)(ws + L.flags);
+  __nv_bfloat16* dzs = (__nv_bfloat16*)(ws + L.dzs);
+  __nv_bfloat16* aug = (__nv_bfloat16*)(ws + L.aug);
+  float2* params = (float2*)(ws + L.params);
+  float* lse2 = (float*)(ws + L.lse2);
+  float* dqp = (float*)(ws + L.dqp);
+  cudaError_t e;
+
+  // bf16 Z1 and a cleared range flag (no decode, so no token can raise it)
+  bwd_prep_kernel<D><<<(unsigned)BH, kM, 0, st>>>(Z1, lse1, zb, rref, flags);
+  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+  bwd_mid_kernel<D><<<(unsigned)BH, kM, 0, st>>>(nullptr, 0, (const __nv_bfloat16*)dZ1, Z1, lse1,
+                                                 dzs, (uint32_t*)aug, flags, params, lse2);
+  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+
+  // the decode operands' maps point at V: valid tiles that are never used
+  CUtensorMap mq, mk, mv, mz, mdz, maug;
+  if ((e = make_map(&mq, Q, D, kM, d.H, kM)) != cudaSuccess) return e;
+  if ((e = make_map(&mk, K, D, d.N, BH, kT)) != cudaSuccess) return e;
+  if ((e = make_map(&mv, V, D, d.N, BH, kT)) != cudaSuccess) return e;
+  if ((e = make_map(&mz, zb, D, kM, BH, kM)) != cudaSuccess) return e;
+  if ((e = make_map(&mdz, dzs, D, kM, BH, kM)) != cudaSuccess) return e;
+  if ((e = make_map(&maug, aug, 16, kM, BH, kM)) != cudaSuccess) return e;
+
+  dim3 grid(p.chunks, (unsigned)BH);
+  const int smemF = BFLayout<D>::BYTES + 1024;
+  e = cudaFuncSetAttribute(tc_bwd_b_fast_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smemF);
+  if (e != cudaSuccess) return e;
+  tc_bwd_b_fast_kernel<D><<<grid, kThr, smemF, st>>>(
+      mq, mk, mv, mv, mz, mdz, maug, (int)d.H, d.N, 0, c, scale, p.tiles_per_bh, p.chunk_tiles,
+      stats, params, 1, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, dqp, err);
+  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+  const int smemB = BLayout<D>::BYTES + 1024;
+  e = cudaFuncSetAttribute(tc_bwd_b_exact_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smemB);
+  if (e != cudaSuccess) return e;
+  tc_bwd_b_exact_kernel<D><<<grid, kThr, smemB, st>>>(
+      mq, mk, mv, mv, mz, mdz, maug, (int)d.H, d.N, 0, c, scale, p.tiles_per_bh, p.chunk_tiles,
+      stats, params, lse2, 1, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, dqp, err);
+  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+
+  const int64_t total = d.H * kM * D;
+  bwd_dq_sum_kernel<<<(unsigned)((total / 4 + 127) / 128), 128, 0, st>>>(
+      (const float4*)dqp, (int)d.B, (int)d.H, kM, D, p.chunks, true,
+      (const __nv_bfloat16*)dZ1, (__nv_bfloat16*)dQ);
   return cudaPeekAtLastError();
 }
 
@@ -1624,6 +1740,16 @@ cudaError_t launch_tc_bwd(const void* Q, int64_t qbs, const void* K, const void*
   if (d.M != kM) return cudaErrorNotSupported;
   if (d.D == 32) return tc_bwd_t<32>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
   if (d.D == 16) return tc_bwd_t<16>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
+  return cudaErrorNotSupported;
+}
+
+cudaError_t launch_tc_enc_bwd(const void* Q, const void* K, const void* V, const float* Z1,
+                              const float* lse1, const void* dZ1, void* dQ, void* dK, void* dV,
+                              const Dims& d, float scale, const WsLayout& L, char* ws,
+                              cudaStream_t st) {
+  if (d.M != kM) return cudaErrorNotSupported;
+  if (d.D == 32) return tc_enc_bwd_t<32>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st);
+  if (d.D == 16) return tc_enc_bwd_t<16>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st);
   return cudaErrorNotSupported;
 }
 

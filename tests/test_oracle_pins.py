@@ -361,3 +361,47 @@ def test_pp_bwd_reduces_to_flare_when_the_correction_is_removed():
     # dQ: FLARE's dQ with per-batch Q_dyn = Q, summed over the batch, is
     # FLARE's shared-Q dQ
     np.testing.assert_allclose(dQ, dQf, rtol=1e-11, atol=1e-12)
+
+
+def test_encode_bwd_central_finite_differences():
+    # The encode's gradient alone: d/dX of sum(Z * dZ), Z = softmax_N(s Q K^T) V
+    # with Q shared over the batch; every element of Q, K and V.
+    B, H, N, M, D = 2, 1, 30, 5, 4
+    x = _x(B, H, N, M, D, seed=26)
+    dZ = np.random.default_rng(27).standard_normal((B, H, M, D))
+    s = 0.7
+    dQ, dK, dV = oracle.encode_bwd(x["Q"], x["K"], x["V"], dZ, s)
+
+    def loss():
+        Z, _ = oracle.encode(x["Q"], x["K"], x["V"], s)
+        return float((Z * dZ).sum())
+
+    eps = 1e-5
+    for name, grad in (("Q", dQ), ("K", dK), ("V", dV)):
+        flat = x[name].reshape(-1)
+        fd = np.empty(flat.size)
+        for i in range(flat.size):
+            old = flat[i]
+            flat[i] = old + eps
+            lp = loss()
+            flat[i] = old - eps
+            lm = loss()
+            flat[i] = old
+            fd[i] = (lp - lm) / (2 * eps)
+        assert np.abs(grad.reshape(-1) - fd).max() <= 1e-7 * max(np.abs(fd).max(), 1.0), name
+
+
+def test_encode_bwd_is_the_part_of_the_flare_pp_gradient_through_z1():
+    # FLARE++'s gradient = FLARE's gradient at Q_dyn (per-batch latents) plus
+    # the encode's gradient with upstream dQ_dyn; dQ also collects dQ_dyn
+    # summed over the batch.
+    B, H, N, M, D = 2, 2, 50, 6, 4
+    x = _x(B, H, N, M, D, seed=28, with_dy=True)
+    s = 0.5
+    dQ, dK, dV = oracle.flare_pp_bwd(x["Q"], x["K"], x["V"], x["dY"], s)
+    _, Qd, _, _ = oracle.flare_pp_fwd(x["Q"], x["K"], x["V"], s)
+    dQd, dKa, dVa = oracle.flare_bwd(Qd, x["K"], x["V"], x["dY"], s)
+    dQe, dKe, dVe = oracle.encode_bwd(x["Q"], x["K"], x["V"], dQd, s)
+    np.testing.assert_allclose(dK, dKa + dKe, rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(dV, dVa + dVe, rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(dQ, dQd.sum(0) + dQe, rtol=1e-11, atol=1e-13)
