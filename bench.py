@@ -281,6 +281,13 @@ def run_ours(args, rank, world, local):
         if events:
             events[3].record(st)
 
+    # the clock sampler starts before the warm-up, so that no idle gap (while
+    # nvidia-smi starts) separates the warm-up from the timed steps
+    sampler = ClockSampler(local, os.path.join(args.out_dir, "clocks.csv") if args.out_dir else None) \
+        if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.5)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -288,11 +295,6 @@ def run_ours(args, rank, world, local):
         raise RuntimeError("device wait ran out during warm-up")
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    sampler = ClockSampler(local, os.path.join(args.out_dir, "clocks.csv") if args.out_dir else None) \
-        if rank == 0 else None
-    if sampler:
-        sampler.start()
-        time.sleep(0.5)
     dist_barrier(world)
     torch.cuda.synchronize()
     t_start = torch.cuda.Event(enable_timing=True)

@@ -17,8 +17,9 @@
  *           with the logits recomputed.
  *
  * Conventions shared by every entry point
- *   - Every tensor pointer is a DEVICE pointer to contiguous row-major data,
- *     16-byte aligned.  Shapes:
+ *   - Every tensor pointer is a DEVICE pointer to contiguous row-major data
+ *     (token tensors may instead be strided: the *_strided calls), 16-byte
+ *     aligned.  Shapes:
  *       Q        [H,M,D] when q_batch_stride == 0 (learned latents shared by
  *                the batch) or [B,H,M,D] when q_batch_stride == H*M*D;
  *       K, V, Y, dY, dK, dV   [B,H,N,D];
@@ -81,6 +82,23 @@ typedef enum {
   FLARE_OP_BWD = 2,
   FLARE_OP_PP_BWD = 3
 } flare_op_t;
+
+/*
+ * Layout of one token tensor (K, V, Y, dY, dK or dV) of logical shape
+ * [B,H,N,D] whose head dimension D is contiguous: element (b, h, n, d) sits
+ * at element offset b*b_stride + h*h_stride + n*n_stride + d from the base
+ * pointer.  Contiguous [B,H,N,D] is {H*N*D, N*D, D}; the layout of a fused
+ * projection's output [B,N,H,D] is {N*H*D, D, H*D}.  Used by the *_strided
+ * entry points.  Every stride must be >= 1, a multiple of 16 bytes and
+ * below 2^40 bytes (else FLARE_ERR_INVALID_ARG, or FLARE_ERR_UNSUPPORTED for
+ * a stride that is not a multiple of 16 bytes).  The rows of an output
+ * tensor must not overlap (checked: in order of stride, each dimension with
+ * more than one index must step over all rows of the dimensions inside it;
+ * else FLARE_ERR_INVALID_ARG); inputs may share or overlap rows.
+ */
+typedef struct {
+  int64_t b_stride, h_stride, n_stride;
+} flare_strides_t;
 
 /* Library ABI version (major*10000 + minor*100 + patch). */
 FLARE_API int flare_version(void);
@@ -164,6 +182,48 @@ FLARE_API flare_status_t flare_pp_bwd(const void* Q, const void* K, const void* 
                             void* dQ, void* dK, void* dV, int64_t B, int64_t H, int64_t N,
                             int64_t M, int64_t D, flare_dtype_t dtype, float scale,
                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The four entry points above with token tensors in any layout that
+ * flare_strides_t describes (for example [B,N,H,D] straight from a fused
+ * QKV projection, with no transpose).  `strides` points to one
+ * flare_strides_t per token tensor, in this order:
+ *   flare_fwd_strided, flare_pp_fwd_strided:  K, V, Y;
+ *   flare_bwd_strided, flare_pp_bwd_strided:  K, V, dY, dK, dV.
+ * NULL means every token tensor is contiguous [B,H,N,D] (the plain entry
+ * points are these calls with NULL).  Latent tensors (Q, Q_dyn, dQ, Z_save,
+ * lse_save) stay contiguous.  Results are identical to the plain calls on
+ * the same values; outputs must not alias inputs.
+ */
+FLARE_API flare_status_t flare_fwd_strided(const void* Q, int64_t q_batch_stride, const void* K,
+                                           const void* V, void* Y,
+                                           const flare_strides_t* strides, int64_t B, int64_t H,
+                                           int64_t N, int64_t M, int64_t D, flare_dtype_t dtype,
+                                           float scale, float* Z_save, float* lse_save,
+                                           void* workspace, size_t workspace_bytes,
+                                           void* stream);
+FLARE_API flare_status_t flare_pp_fwd_strided(const void* Q, const void* K, const void* V,
+                                              void* Y, void* Q_dyn_out,
+                                              const flare_strides_t* strides, int64_t B,
+                                              int64_t H, int64_t N, int64_t M, int64_t D,
+                                              flare_dtype_t dtype, float scale, float* Z_save,
+                                              float* lse_save, void* workspace,
+                                              size_t workspace_bytes, void* stream);
+FLARE_API flare_status_t flare_bwd_strided(const void* Q, int64_t q_batch_stride, const void* K,
+                                           const void* V, const void* dY, const float* Z_save,
+                                           const float* lse_save, void* dQ, void* dK, void* dV,
+                                           const flare_strides_t* strides, int64_t B, int64_t H,
+                                           int64_t N, int64_t M, int64_t D, flare_dtype_t dtype,
+                                           float scale, void* workspace, size_t workspace_bytes,
+                                           void* stream);
+FLARE_API flare_status_t flare_pp_bwd_strided(const void* Q, const void* K, const void* V,
+                                              const void* dY, const void* Q_dyn,
+                                              const float* Z_save, const float* lse_save,
+                                              void* dQ, void* dK, void* dV,
+                                              const flare_strides_t* strides, int64_t B,
+                                              int64_t H, int64_t N, int64_t M, int64_t D,
+                                              flare_dtype_t dtype, float scale, void* workspace,
+                                              size_t workspace_bytes, void* stream);
 
 /*
  * Stage 1 of the forward -- encode partials.  For each (b, h) and each

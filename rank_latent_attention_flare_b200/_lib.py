@@ -39,6 +39,15 @@ _f32 = ctypes.c_float
 _sz = ctypes.c_size_t
 _u32p = ctypes.POINTER(ctypes.c_uint32)
 
+
+class FlareStrides(ctypes.Structure):
+    """flare_strides_t: element strides of a [B,H,N,D] token tensor."""
+    _fields_ = [("b_stride", ctypes.c_int64), ("h_stride", ctypes.c_int64),
+                ("n_stride", ctypes.c_int64)]
+
+
+_stp = ctypes.POINTER(FlareStrides)
+
 SIGNATURES = {
     "flare_version": (_i32, []),
     "flare_last_error_detail": (ctypes.c_char_p, []),
@@ -52,6 +61,14 @@ SIGNATURES = {
                          _i64, _i64, _i32, _f32, _vp, _sz, _vp]),
     "flare_pp_bwd": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
                             _i64, _i64, _i32, _f32, _vp, _sz, _vp]),
+    "flare_fwd_strided": (_i32, [_vp, _i64, _vp, _vp, _vp, _stp, _i64, _i64, _i64, _i64, _i64,
+                                 _i32, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "flare_pp_fwd_strided": (_i32, [_vp, _vp, _vp, _vp, _vp, _stp, _i64, _i64, _i64, _i64, _i64,
+                                    _i32, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "flare_bwd_strided": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _stp, _i64,
+                                 _i64, _i64, _i64, _i64, _i32, _f32, _vp, _sz, _vp]),
+    "flare_pp_bwd_strided": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _stp, _i64,
+                                    _i64, _i64, _i64, _i64, _i32, _f32, _vp, _sz, _vp]),
     "flare_encode": (_i32, [_vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i32, _f32, _vp,
                             _sz, _vp]),
     "flare_combine": (_i32, [_i64, _i64, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _sz, _vp]),

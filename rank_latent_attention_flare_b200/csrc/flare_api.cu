@@ -38,6 +38,12 @@ int current_sm_count() {
   return n;
 }
 
+#define FLARE_TRY(x)                    \
+  do {                                  \
+    flare_status_t s_ = (x);            \
+    if (s_ != FLARE_OK) return s_;      \
+  } while (0)
+
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 flare_status_t check_sizes(int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
@@ -69,16 +75,55 @@ flare_status_t check_qbs(int64_t qbs, int64_t H, int64_t M, int64_t D) {
   return (qbs == 0 || qbs == H * M * D) ? FLARE_OK : FLARE_ERR_UNSUPPORTED;
 }
 
+// One token tensor's strides: each positive, a multiple of 16 bytes and
+// below 2^40 bytes (the TMA limits).  The rows of an output may not overlap:
+// taken in order of stride, every dimension with more than one index must
+// step over all the rows of the dimensions inside it.
+flare_status_t tok_from(const flare_strides_t& st, const Dims& d, flare_dtype_t dt,
+                        bool output, Tok* out) {
+  const int64_t esz = (dt == FLARE_F32) ? 4 : 2;
+  const int64_t v[3] = {st.b_stride, st.h_stride, st.n_stride};
+  for (int i = 0; i < 3; ++i) {
+    if (v[i] < 1 || v[i] >= (1LL << 40) / esz) return FLARE_ERR_INVALID_ARG;
+    if ((v[i] * esz) % 16 != 0) return FLARE_ERR_UNSUPPORTED;
+  }
+  if (output) {
+    int64_t s3[3] = {st.b_stride, st.h_stride, st.n_stride}, e3[3] = {d.B, d.H, d.N};
+    for (int i = 0; i < 3; ++i)
+      for (int j = i + 1; j < 3; ++j)
+        if (s3[j] < s3[i]) {
+          const int64_t ts = s3[i], te = e3[i];
+          s3[i] = s3[j];
+          e3[i] = e3[j];
+          s3[j] = ts;
+          e3[j] = te;
+        }
+    int64_t span = d.D;   // elements spanned by the dimensions inside
+    for (int i = 0; i < 3; ++i) {
+      if (e3[i] == 1) continue;
+      if (s3[i] < span) return FLARE_ERR_INVALID_ARG;
+      span += s3[i] * (e3[i] - 1);
+    }
+  }
+  *out = Tok{st.b_stride, st.h_stride, st.n_stride};
+  return FLARE_OK;
+}
+
+// The token tensors' layouts: NULL = contiguous; else one flare_strides_t
+// per tensor in the order given by `which` (entries of Dims), the last
+// `n_out` of them outputs.
+flare_status_t apply_strides(const flare_strides_t* st, Tok Dims::* const* which, int n,
+                             int n_out, flare_dtype_t dt, Dims* d) {
+  if (st == nullptr) return FLARE_OK;
+  for (int i = 0; i < n; ++i) FLARE_TRY(tok_from(st[i], *d, dt, i >= n - n_out, &(d->*which[i])));
+  return FLARE_OK;
+}
+
 flare_status_t check_ws(const void* ws, size_t bytes, size_t need) {
   if (ws == nullptr || ((uintptr_t)ws & 255u) != 0) return FLARE_ERR_WORKSPACE;
   return bytes >= need ? FLARE_OK : FLARE_ERR_WORKSPACE;
 }
 
-#define FLARE_TRY(x)                    \
-  do {                                  \
-    flare_status_t s_ = (x);            \
-    if (s_ != FLARE_OK) return s_;      \
-  } while (0)
 
 #define FLARE_CUDA(x)                                                               \
   do {                                                                              \
@@ -131,6 +176,11 @@ flare_status_t run_decode(const void* Q, int64_t qbs, const void* K, void* Y, co
     FLARE_CUDA(launch_simt_decode(Q, qbs, K, (const float*)(ws + L.zf), Y, d, dt, scale, st));
   return FLARE_OK;
 }
+
+// Order of the flare_strides_t entries: forward K, V, Y; backward K, V,
+// dY, dK, dV.
+Tok Dims::* const kFwdTensors[3] = {&Dims::k, &Dims::v, &Dims::y};
+Tok Dims::* const kBwdTensors[5] = {&Dims::k, &Dims::v, &Dims::dy, &Dims::dk, &Dims::dv};
 
 }  // namespace
 
@@ -217,10 +267,11 @@ flare_status_t flare_decode(const void* Q, int64_t qbs, const void* K, void* Y, 
                     (cudaStream_t)stream, sms);
 }
 
-flare_status_t flare_fwd(const void* Q, int64_t qbs, const void* K, const void* V, void* Y,
-                         int64_t B, int64_t H, int64_t N, int64_t M, int64_t D, flare_dtype_t dt,
-                         float scale, float* Z_save, float* lse_save, void* workspace,
-                         size_t workspace_bytes, void* stream) {
+flare_status_t flare_fwd_strided(const void* Q, int64_t qbs, const void* K, const void* V,
+                                 void* Y, const flare_strides_t* strides, int64_t B, int64_t H,
+                                 int64_t N, int64_t M, int64_t D, flare_dtype_t dt, float scale,
+                                 float* Z_save, float* lse_save, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
   FLARE_TRY(check_sizes(B, H, N, M, D, dt));
   FLARE_TRY(check_scale(scale));
   FLARE_TRY(check_ptr(Q));
@@ -233,20 +284,21 @@ flare_status_t flare_fwd(const void* Q, int64_t qbs, const void* K, const void* 
   const int sms = current_sm_count();
   const WsLayout L = ws_layout(FLARE_OP_FWD, B, H, N, M, D, dt, sms);
   FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  Dims d{B, H, N, M, D};
+  FLARE_TRY(apply_strides(strides, kFwdTensors, 3, 1, dt, &d));
   char* ws = (char*)workspace;
   cudaStream_t st = (cudaStream_t)stream;
-  const Dims d{B, H, N, M, D};
   FLARE_TRY(reset_error_word(ws, st));
   FLARE_TRY(run_encode(Q, qbs, K, V, d, dt, scale, L, ws, st));
   FLARE_TRY(run_combine(d, dt, Z_save, lse_save, nullptr, nullptr, L, ws, st));
   return run_decode(Q, qbs, K, Y, d, dt, scale, L, ws, st, sms);
 }
 
-flare_status_t flare_pp_fwd(const void* Q, const void* K, const void* V, void* Y,
-                            void* Q_dyn_out, int64_t B, int64_t H, int64_t N, int64_t M,
-                            int64_t D, flare_dtype_t dt, float scale, float* Z_save,
-                            float* lse_save, void* workspace, size_t workspace_bytes,
-                            void* stream) {
+flare_status_t flare_pp_fwd_strided(const void* Q, const void* K, const void* V, void* Y,
+                                    void* Q_dyn_out, const flare_strides_t* strides, int64_t B,
+                                    int64_t H, int64_t N, int64_t M, int64_t D, flare_dtype_t dt,
+                                    float scale, float* Z_save, float* lse_save, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
   FLARE_TRY(check_sizes(B, H, N, M, D, dt));
   FLARE_TRY(check_scale(scale));
   FLARE_TRY(check_ptr(Q));
@@ -259,9 +311,10 @@ flare_status_t flare_pp_fwd(const void* Q, const void* K, const void* V, void* Y
   const int sms = current_sm_count();
   const WsLayout L = ws_layout(FLARE_OP_PP_FWD, B, H, N, M, D, dt, sms);
   FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  Dims d{B, H, N, M, D};
+  FLARE_TRY(apply_strides(strides, kFwdTensors, 3, 1, dt, &d));
   char* ws = (char*)workspace;
   cudaStream_t st = (cudaStream_t)stream;
-  const Dims d{B, H, N, M, D};
   void* qdyn = Q_dyn_out ? Q_dyn_out : (void*)(ws + L.qdyn);
   const int64_t qdyn_bs = H * M * D;
   FLARE_TRY(reset_error_word(ws, st));
@@ -274,11 +327,12 @@ flare_status_t flare_pp_fwd(const void* Q, const void* K, const void* V, void* Y
   return run_decode(qdyn, qdyn_bs, K, Y, d, dt, scale, L, ws, st, sms);
 }
 
-flare_status_t flare_bwd(const void* Q, int64_t qbs, const void* K, const void* V,
-                         const void* dY, const float* Z_save, const float* lse_save, void* dQ,
-                         void* dK, void* dV, int64_t B, int64_t H, int64_t N, int64_t M,
-                         int64_t D, flare_dtype_t dt, float scale, void* workspace,
-                         size_t workspace_bytes, void* stream) {
+flare_status_t flare_bwd_strided(const void* Q, int64_t qbs, const void* K, const void* V,
+                                 const void* dY, const float* Z_save, const float* lse_save,
+                                 void* dQ, void* dK, void* dV, const flare_strides_t* strides,
+                                 int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
+                                 flare_dtype_t dt, float scale, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
   FLARE_TRY(check_sizes(B, H, N, M, D, dt));
   FLARE_TRY(check_scale(scale));
   FLARE_TRY(check_ptr(Q));
@@ -293,19 +347,21 @@ flare_status_t flare_bwd(const void* Q, int64_t qbs, const void* K, const void* 
   FLARE_TRY(check_qbs(qbs, H, M, D));
   const WsLayout L = ws_layout(FLARE_OP_BWD, B, H, N, M, D, dt, current_sm_count());
   FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  Dims d{B, H, N, M, D};
+  FLARE_TRY(apply_strides(strides, kBwdTensors, 5, 2, dt, &d));
   char* ws = (char*)workspace;
   cudaStream_t st = (cudaStream_t)stream;
   FLARE_TRY(reset_error_word(ws, st));
-  FLARE_CUDA(launch_bwd(Q, qbs, K, V, dY, Z_save, lse_save, dQ, dK, dV, Dims{B, H, N, M, D}, dt,
-                        scale, L, ws, st));
+  FLARE_CUDA(launch_bwd(Q, qbs, K, V, dY, Z_save, lse_save, dQ, dK, dV, d, dt, scale, L, ws, st));
   return FLARE_OK;
 }
 
-flare_status_t flare_pp_bwd(const void* Q, const void* K, const void* V, const void* dY,
-                            const void* Q_dyn, const float* Z_save, const float* lse_save,
-                            void* dQ, void* dK, void* dV, int64_t B, int64_t H, int64_t N,
-                            int64_t M, int64_t D, flare_dtype_t dt, float scale, void* workspace,
-                            size_t workspace_bytes, void* stream) {
+flare_status_t flare_pp_bwd_strided(const void* Q, const void* K, const void* V, const void* dY,
+                                    const void* Q_dyn, const float* Z_save, const float* lse_save,
+                                    void* dQ, void* dK, void* dV, const flare_strides_t* strides,
+                                    int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
+                                    flare_dtype_t dt, float scale, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
   FLARE_TRY(check_sizes(B, H, N, M, D, dt));
   FLARE_TRY(check_scale(scale));
   FLARE_TRY(check_ptr(Q));
@@ -320,9 +376,10 @@ flare_status_t flare_pp_bwd(const void* Q, const void* K, const void* V, const v
   FLARE_TRY(check_ptr(dV));
   const WsLayout L = ws_layout(FLARE_OP_PP_BWD, B, H, N, M, D, dt, current_sm_count());
   FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  Dims d{B, H, N, M, D};
+  FLARE_TRY(apply_strides(strides, kBwdTensors, 5, 2, dt, &d));
   char* ws = (char*)workspace;
   cudaStream_t st = (cudaStream_t)stream;
-  const Dims d{B, H, N, M, D};
   float* z1 = (float*)(ws + L.z1);
   float* lse1 = (float*)(ws + L.lse1);
   FLARE_TRY(reset_error_word(ws, st));
@@ -335,6 +392,41 @@ flare_status_t flare_pp_bwd(const void* Q, const void* K, const void* V, const v
   // the first encode's gradient with upstream dQ_dyn, and dQ
   FLARE_CUDA(launch_pp_bwd_tail(Q, K, V, z1, lse1, ws + L.dqd, dQ, dK, dV, d, dt, scale, L, ws, st));
   return FLARE_OK;
+}
+
+flare_status_t flare_fwd(const void* Q, int64_t qbs, const void* K, const void* V, void* Y,
+                         int64_t B, int64_t H, int64_t N, int64_t M, int64_t D, flare_dtype_t dt,
+                         float scale, float* Z_save, float* lse_save, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  return flare_fwd_strided(Q, qbs, K, V, Y, nullptr, B, H, N, M, D, dt, scale, Z_save, lse_save,
+                           workspace, workspace_bytes, stream);
+}
+
+flare_status_t flare_pp_fwd(const void* Q, const void* K, const void* V, void* Y,
+                            void* Q_dyn_out, int64_t B, int64_t H, int64_t N, int64_t M,
+                            int64_t D, flare_dtype_t dt, float scale, float* Z_save,
+                            float* lse_save, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  return flare_pp_fwd_strided(Q, K, V, Y, Q_dyn_out, nullptr, B, H, N, M, D, dt, scale, Z_save,
+                              lse_save, workspace, workspace_bytes, stream);
+}
+
+flare_status_t flare_bwd(const void* Q, int64_t qbs, const void* K, const void* V,
+                         const void* dY, const float* Z_save, const float* lse_save, void* dQ,
+                         void* dK, void* dV, int64_t B, int64_t H, int64_t N, int64_t M,
+                         int64_t D, flare_dtype_t dt, float scale, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  return flare_bwd_strided(Q, qbs, K, V, dY, Z_save, lse_save, dQ, dK, dV, nullptr, B, H, N, M,
+                           D, dt, scale, workspace, workspace_bytes, stream);
+}
+
+flare_status_t flare_pp_bwd(const void* Q, const void* K, const void* V, const void* dY,
+                            const void* Q_dyn, const float* Z_save, const float* lse_save,
+                            void* dQ, void* dK, void* dV, int64_t B, int64_t H, int64_t N,
+                            int64_t M, int64_t D, flare_dtype_t dt, float scale, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  return flare_pp_bwd_strided(Q, K, V, dY, Q_dyn, Z_save, lse_save, dQ, dK, dV, nullptr, B, H, N,
+                              M, D, dt, scale, workspace, workspace_bytes, stream);
 }
 
 flare_status_t flare_device_status(void* workspace, size_t workspace_bytes, uint32_t* detail,

@@ -24,8 +24,9 @@ constexpr int kT = kBwdTile;  // tokens per tile (= threads per CTA)
 template <typename T, int D>
 __global__ void __launch_bounds__(kT)
     bwd_decode_kernel(const T* __restrict__ Q, int64_t q_bstride, const T* __restrict__ K,
-                      const T* __restrict__ dY, const float* __restrict__ Z, int H, int64_t N,
-                      int M, float c, float s, int64_t chunk_tokens, float* __restrict__ dkf,
+                      const T* __restrict__ dY, Tok tk, Tok tdy, const float* __restrict__ Z,
+                      int H, int64_t N, int M, float c, float s, int64_t chunk_tokens,
+                      float* __restrict__ dkf,
                       float* __restrict__ dq_part, float* __restrict__ dz_part) {
   extern __shared__ float sm[];
   float* qs = sm;                 // [M][D] raw latents
@@ -38,6 +39,7 @@ __global__ void __launch_bounds__(kT)
   const int chunk = blockIdx.x, chunks = gridDim.x;
   const int64_t bh = blockIdx.y, b = bh / H, h = bh % H;
   const int64_t n0 = (int64_t)chunk * chunk_tokens, n1 = min(N, n0 + chunk_tokens);
+  const int64_t kh = tk.head(bh, H), dyh = tdy.head(bh, H);
   for (int i = threadIdx.x; i < M * D; i += blockDim.x) {
     qs[i] = to_f(Q[b * q_bstride + h * (int64_t)M * D + i]);
     zs[i] = Z[bh * M * D + i];
@@ -52,10 +54,9 @@ __global__ void __launch_bounds__(kT)
     const int nt = (int)imin64(kT, n1 - t0);
     __syncthreads();
     for (int i = tid; i < kT * D; i += blockDim.x) {
-      const int j = i / D;
-      const int64_t g = (bh * N + t0) * D + i;
-      ks[i] = (j < nt) ? to_f(K[g]) : 0.f;
-      dys[i] = (j < nt) ? to_f(dY[g]) : 0.f;
+      const int j = i / D, d = i % D;
+      ks[i] = (j < nt) ? to_f(K[kh + (t0 + j) * tk.sn + d]) : 0.f;
+      dys[i] = (j < nt) ? to_f(dY[dyh + (t0 + j) * tdy.sn + d]) : 0.f;
     }
     __syncthreads();
     // phase 1: one thread per token -> softmax statistics, delta_d and dK
@@ -168,9 +169,9 @@ __global__ void __launch_bounds__(kT)
     bwd_encode_kernel(const T* __restrict__ Q, int64_t q_bstride, const T* __restrict__ K,
                       const T* __restrict__ V, const float* __restrict__ dkf,
                       const float* __restrict__ lse, const float* __restrict__ dzg,
-                      const float* __restrict__ delta, int H, int64_t N, int M, float c, float s,
-                      int64_t chunk_tokens, T* __restrict__ dK, T* __restrict__ dV,
-                      float* __restrict__ dq_part) {
+                      const float* __restrict__ delta, Tok tk, Tok tv, Tok tdk, Tok tdv, int H,
+                      int64_t N, int M, float c, float s, int64_t chunk_tokens,
+                      T* __restrict__ dK, T* __restrict__ dV, float* __restrict__ dq_part) {
   extern __shared__ float sm[];
   float* qs = sm;                 // [M][D]
   float* dzs = qs + M * D;        // [M][D]
@@ -181,6 +182,8 @@ __global__ void __launch_bounds__(kT)
   const int chunk = blockIdx.x, chunks = gridDim.x;
   const int64_t bh = blockIdx.y, b = bh / H, h = bh % H;
   const int64_t n0 = (int64_t)chunk * chunk_tokens, n1 = min(N, n0 + chunk_tokens);
+  const int64_t kh = tk.head(bh, H), vh = tv.head(bh, H);
+  const int64_t dkh = tdk.head(bh, H), dvh = tdv.head(bh, H);
   for (int i = threadIdx.x; i < M * D; i += blockDim.x) {
     qs[i] = to_f(Q[b * q_bstride + h * (int64_t)M * D + i]);
     dzs[i] = dzg[bh * M * D + i];
@@ -199,10 +202,9 @@ __global__ void __launch_bounds__(kT)
     const int nt = (int)imin64(kT, n1 - t0);
     __syncthreads();
     for (int i = tid; i < kT * D; i += blockDim.x) {
-      const int j = i / D;
-      const int64_t g = (bh * N + t0) * D + i;
-      ks[i] = (j < nt) ? to_f(K[g]) : 0.f;
-      vs[i] = (j < nt) ? to_f(V[g]) : 0.f;
+      const int j = i / D, d = i % D;
+      ks[i] = (j < nt) ? to_f(K[kh + (t0 + j) * tk.sn + d]) : 0.f;
+      vs[i] = (j < nt) ? to_f(V[vh + (t0 + j) * tv.sn + d]) : 0.f;
     }
     __syncthreads();
     // phase 1: one thread per token -> dV and the encode part of dK
@@ -233,8 +235,8 @@ __global__ void __launch_bounds__(kT)
       }
 #pragma unroll
       for (int d = 0; d < D; ++d) {
-        dK[(bh * N + n) * D + d] = from_f<T>(dk[d]);
-        dV[(bh * N + n) * D + d] = from_f<T>(dv[d]);
+        dK[dkh + n * tdk.sn + d] = from_f<T>(dk[d]);
+        dV[dvh + n * tdv.sn + d] = from_f<T>(dv[d]);
       }
     }
     // phase 2: one thread per latent -> partial dQ (encode part)
@@ -314,9 +316,9 @@ cudaError_t bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, cons
   cudaError_t e = cudaFuncSetAttribute(bwd_decode_kernel<T, D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemA);
   if (e != cudaSuccess) return e;
-  bwd_decode_kernel<T, D><<<grid, kT, smemA, st>>>((const T*)Q, qbs, (const T*)K, (const T*)dY, Z,
-                                                   (int)d.H, d.N, M, c, scale, p.chunk_tokens(),
-                                                   dkf, dq_dec, dzp);
+  bwd_decode_kernel<T, D><<<grid, kT, smemA, st>>>((const T*)Q, qbs, (const T*)K, (const T*)dY, d.k,
+                                                   d.dy, Z, (int)d.H, d.N, M, c, scale,
+                                                   p.chunk_tokens(), dkf, dq_dec, dzp);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
   const int64_t warps = d.BH() * M;
@@ -329,8 +331,9 @@ cudaError_t bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, cons
                            (int)smemB);
   if (e != cudaSuccess) return e;
   bwd_encode_kernel<T, D><<<grid, kT, smemB, st>>>((const T*)Q, qbs, (const T*)K, (const T*)V, dkf,
-                                                   lse, dz, delta, (int)d.H, d.N, M, c, scale,
-                                                   p.chunk_tokens(), (T*)dK, (T*)dV, dq_enc);
+                                                   lse, dz, delta, d.k, d.v, d.dk, d.dv, (int)d.H,
+                                                   d.N, M, c, scale, p.chunk_tokens(), (T*)dK,
+                                                   (T*)dV, dq_enc);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
   const bool shared_q = (qbs == 0);
@@ -397,8 +400,9 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kT)
     pp_encode_bwd_kernel(const T* __restrict__ Q, const T* __restrict__ K,
                          const T* __restrict__ V, const float* __restrict__ lse1,
-                         const float* __restrict__ dz1, const float* __restrict__ delta1, int H,
-                         int64_t N, int M, float c, float s, int64_t chunk_tokens,
+                         const float* __restrict__ dz1, const float* __restrict__ delta1, Tok tk,
+                         Tok tv, Tok tdk, Tok tdv, int H, int64_t N, int M, float c, float s,
+                         int64_t chunk_tokens,
                          T* __restrict__ dK, T* __restrict__ dV, float* __restrict__ dq_part) {
   extern __shared__ float sm[];
   float* qs = sm;                 // [M][D]
@@ -410,6 +414,8 @@ __global__ void __launch_bounds__(kT)
   const int chunk = blockIdx.x, chunks = gridDim.x;
   const int64_t bh = blockIdx.y, h = bh % H;
   const int64_t n0 = (int64_t)chunk * chunk_tokens, n1 = min(N, n0 + chunk_tokens);
+  const int64_t kh = tk.head(bh, H), vh = tv.head(bh, H);
+  const int64_t dkh = tdk.head(bh, H), dvh = tdv.head(bh, H);
   for (int i = threadIdx.x; i < M * D; i += blockDim.x) {
     qs[i] = to_f(Q[h * (int64_t)M * D + i]);
     dzs[i] = dz1[bh * M * D + i];
@@ -428,10 +434,9 @@ __global__ void __launch_bounds__(kT)
     const int nt = (int)imin64(kT, n1 - t0);
     __syncthreads();
     for (int i = tid; i < kT * D; i += blockDim.x) {
-      const int j = i / D;
-      const int64_t g = (bh * N + t0) * D + i;
-      ks[i] = (j < nt) ? to_f(K[g]) : 0.f;
-      vs[i] = (j < nt) ? to_f(V[g]) : 0.f;
+      const int j = i / D, d = i % D;
+      ks[i] = (j < nt) ? to_f(K[kh + (t0 + j) * tk.sn + d]) : 0.f;
+      vs[i] = (j < nt) ? to_f(V[vh + (t0 + j) * tv.sn + d]) : 0.f;
     }
     __syncthreads();
     // one thread per token: the encode's dV and dK parts, added to the rows
@@ -462,9 +467,9 @@ __global__ void __launch_bounds__(kT)
       }
 #pragma unroll
       for (int d = 0; d < D; ++d) {
-        const int64_t o = (bh * N + n) * D + d;
-        dK[o] = from_f<T>(to_f(dK[o]) + dk[d]);
-        dV[o] = from_f<T>(to_f(dV[o]) + dv[d]);
+        const int64_t ok = dkh + n * tdk.sn + d, ov = dvh + n * tdv.sn + d;
+        dK[ok] = from_f<T>(to_f(dK[ok]) + dk[d]);
+        dV[ov] = from_f<T>(to_f(dV[ov]) + dv[d]);
       }
     }
     // one thread per latent: the encode's part of dQ over this tile
@@ -536,8 +541,8 @@ cudaError_t pp_tail_t(const void* Q, const void* K, const void* V, const float* 
   if (e != cudaSuccess) return e;
   dim3 grid(p.chunks, (unsigned)BH);
   pp_encode_bwd_kernel<T, D><<<grid, kT, smem, st>>>(
-      (const T*)Q, (const T*)K, (const T*)V, lse1, dz1, delta1, (int)d.H, d.N, M,
-      scale * kLog2e, scale, p.chunk_tokens(), (T*)dK, (T*)dV, dqe);
+      (const T*)Q, (const T*)K, (const T*)V, lse1, dz1, delta1, d.k, d.v, d.dk, d.dv, (int)d.H,
+      d.N, M, scale * kLog2e, scale, p.chunk_tokens(), (T*)dK, (T*)dV, dqe);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   const int64_t per = d.H * M * D;
   pp_dq_kernel<T><<<(unsigned)((per + 255) / 256), 256, 0, st>>>((const T*)dqd, dqe, (int)d.B,

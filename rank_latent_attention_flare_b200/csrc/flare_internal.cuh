@@ -253,9 +253,24 @@ void note_error(const char* fmt, ...);
 // ------------------------------------------------------------ launchers
 // Each returns cudaSuccess or the launch error.
 
+// Element strides of a token tensor [B,H,N,D] whose head dimension D is
+// contiguous: element (b, h, n, d) sits at b sb + h sh + n sn + d.
+struct Tok {
+  int64_t sb, sh, sn;
+  // offset of row 0 of head bh = b H + h
+  __host__ __device__ __forceinline__ int64_t head(int64_t bh, int64_t H) const {
+    return (bh / H) * sb + (bh % H) * sh;
+  }
+};
+
+// Problem sizes and the layouts of the token tensors (contiguous [B,H,N,D]
+// unless the caller gave strides).
 struct Dims {
   int64_t B, H, N, M, D;
+  Tok k = contig(), v = contig(), y = contig();     // K, V, the forward's Y
+  Tok dy = contig(), dk = contig(), dv = contig();  // dY, dK, dV
   int64_t BH() const { return B * H; }
+  Tok contig() const { return Tok{H * N * D, N * D, D}; }
 };
 
 cudaError_t launch_simt_encode(const void* Q, int64_t qbs, const void* K, const void* V,
@@ -280,6 +295,23 @@ cudaError_t launch_tc_decode(const void* Q, int64_t qbs, const void* K,
 // (64-byte swizzle for 64-byte rows, 32-byte for 32-byte rows).
 cudaError_t make_map(CUtensorMap* m, const void* base, int D, int64_t rows, int64_t depth,
                      int box_rows);
+// Stride of the flattened head index bh = b H + h of a token tensor, or -1
+// when its batch and head dimensions do not flatten into one.
+inline int64_t flat_stride(const Tok& t, const Dims& d) {
+  if (d.B == 1) return t.sh;
+  if (d.H == 1) return t.sb;
+  return t.sb == d.H * t.sh ? t.sh : -1;
+}
+// True when K, V and dY all flatten (contiguous tensors do): the tensor-core
+// kernels then take 3-D maps {D, N, B*H}, else 4-D maps {D, N, H, B}.
+inline bool tok_flat(const Dims& d) {
+  return flat_stride(d.k, d) > 0 && flat_stride(d.v, d) > 0 && flat_stride(d.dy, d) > 0;
+}
+// TMA map over a bf16 token tensor [B,H,N,D] with strides t: 3-D
+// {D, N, B*H} when `flat`, else 4-D {D, N, H, B}; boxes of box_rows tokens
+// of one head, swizzled as make_map.
+cudaError_t make_tok_map(CUtensorMap* m, const void* base, const Dims& d, const Tok& t,
+                         int box_rows, bool flat);
 
 cudaError_t launch_tc_bwd(const void* Q, int64_t qbs, const void* K, const void* V,
                           const void* dY, const float* Z, const float* lse, void* dQ, void* dK,

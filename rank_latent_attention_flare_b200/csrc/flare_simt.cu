@@ -17,8 +17,8 @@ namespace {
 template <typename T, int D>
 __global__ void __launch_bounds__(kSimtEncThreads)
     simt_encode_kernel(const T* __restrict__ Q, int64_t q_bstride, const T* __restrict__ K,
-                       const T* __restrict__ V, int H, int64_t N, int M, float c,
-                       int64_t chunk_tokens, float* __restrict__ part_ml,
+                       const T* __restrict__ V, Tok tk, Tok tv, int H, int64_t N, int M,
+                       float c, int64_t chunk_tokens, float* __restrict__ part_ml,
                        float* __restrict__ part_acc) {
   __shared__ float ks[kSimtEncTile][D];
   __shared__ float vs[kSimtEncTile][D];
@@ -28,8 +28,8 @@ __global__ void __launch_bounds__(kSimtEncThreads)
   const int64_t b = bh / H, h = bh % H;
   const int64_t n0 = (int64_t)chunk * chunk_tokens;
   const int64_t n1 = min(N, n0 + chunk_tokens);
-  const T* Kb = K + bh * N * D;
-  const T* Vb = V + bh * N * D;
+  const T* Kb = K + tk.head(bh, H);
+  const T* Vb = V + tv.head(bh, H);
   const int m = threadIdx.x;
   const bool active = m < M;
 
@@ -49,8 +49,8 @@ __global__ void __launch_bounds__(kSimtEncThreads)
       const int j = i / D, d = i % D;
       float kv = 0.f, vv = 0.f;
       if (j < nt) {
-        kv = to_f(Kb[(t0 + j) * D + d]);
-        vv = to_f(Vb[(t0 + j) * D + d]);
+        kv = to_f(Kb[(t0 + j) * tk.sn + d]);
+        vv = to_f(Vb[(t0 + j) * tv.sn + d]);
       }
       ks[j][d] = kv;
       vs[j][d] = vv;
@@ -96,8 +96,8 @@ __global__ void __launch_bounds__(kSimtEncThreads)
 template <typename T, int D>
 __global__ void __launch_bounds__(kSimtDecThreads)
     simt_decode_kernel(const T* __restrict__ Q, int64_t q_bstride, const T* __restrict__ K,
-                       const float* __restrict__ Zf, T* __restrict__ Y, int H, int64_t N, int M,
-                       float c) {
+                       const float* __restrict__ Zf, T* __restrict__ Y, Tok tk, Tok ty, int H,
+                       int64_t N, int M, float c) {
   extern __shared__ float sm[];
   float* qs = sm;
   float* zs = sm + M * D;
@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(kSimtDecThreads)
   __syncthreads();
   const int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (n >= N) return;
-  const T* kr = K + (bh * N + n) * D;
+  const T* kr = K + tk.head(bh, H) + n * tk.sn;
   float k[D];
 #pragma unroll
   for (int d = 0; d < D; ++d) k[d] = to_f(kr[d]);
@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(kSimtDecThreads)
     for (int d = 0; d < D; ++d) y[d] = fmaf(p, zs[m * D + d], y[d]);
   }
   const float inv = 1.f / sum;
-  T* yr = Y + (bh * N + n) * D;
+  T* yr = Y + ty.head(bh, H) + n * ty.sn;
 #pragma unroll
   for (int d = 0; d < D; ++d) yr[d] = from_f<T>(y[d] * inv);
 }
@@ -186,8 +186,8 @@ cudaError_t simt_encode_t(const void* Q, int64_t qbs, const void* K, const void*
                           float* part_acc, cudaStream_t st) {
   dim3 grid(plan.chunks, (unsigned)d.BH());
   simt_encode_kernel<T, D><<<grid, kSimtEncThreads, 0, st>>>(
-      (const T*)Q, qbs, (const T*)K, (const T*)V, (int)d.H, d.N, (int)d.M, scale * kLog2e,
-      plan.chunk_tokens(), part_ml, part_acc);
+      (const T*)Q, qbs, (const T*)K, (const T*)V, d.k, d.v, (int)d.H, d.N, (int)d.M,
+      scale * kLog2e, plan.chunk_tokens(), part_ml, part_acc);
   return cudaPeekAtLastError();
 }
 
@@ -200,7 +200,8 @@ cudaError_t simt_decode_t(const void* Q, int64_t qbs, const void* K, const float
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((d.N + kSimtDecThreads - 1) / kSimtDecThreads), (unsigned)d.BH());
   simt_decode_kernel<T, D><<<grid, kSimtDecThreads, smem, st>>>(
-      (const T*)Q, qbs, (const T*)K, Zf, (T*)Y, (int)d.H, d.N, (int)d.M, scale * kLog2e);
+      (const T*)Q, qbs, (const T*)K, Zf, (T*)Y, d.k, d.y, (int)d.H, d.N, (int)d.M,
+      scale * kLog2e);
   return cudaPeekAtLastError();
 }
 

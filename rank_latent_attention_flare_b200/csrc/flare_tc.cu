@@ -95,7 +95,6 @@ __device__ __forceinline__ void scale_tmem_row(uint32_t taddr, float f) {
 // the warpgroups take alternate tiles, each with its own running record.
 
 constexpr int kEncTile = 48;
-constexpr int kEncP = kEncTile / 2;   // P columns (bf16 pairs) per tile
 constexpr int kEncRegsSoftmax = 88, kEncRegsProducer = 56;   // 256 x 88 + 128 x 56 <= 384 x 80
 
 template <int D, int M>
@@ -110,7 +109,7 @@ struct EncLayout {
   static constexpr int BYTES = MISC_OFF + 16;
 };
 
-template <int D, int M>
+template <int D, int M, bool FLAT>
 __global__ void __launch_bounds__(kThreads, 2)
     tc_encode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, int H, int64_t N, int q_per_batch,
@@ -192,8 +191,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           uint8_t* kt = smem + L::KV_OFF + s * 2 * L::TILE;
           mbar_arrive_expect_tx(&kv_full[s], 2 * L::TILE);
           const int32_t tok = (int32_t)((tile0 + i) * kEncTile);
-          tma_load_3d(kt, &tmK, &kv_full[s], 0, tok, (int32_t)bh);
-          tma_load_3d(kt + L::TILE, &tmV, &kv_full[s], 0, tok, (int32_t)bh);
+          tma_load_tok<FLAT>(kt, &tmK, &kv_full[s], tok, bh, H);
+          tma_load_tok<FLAT>(kt + L::TILE, &tmV, &kv_full[s], tok, bh, H);
           issued = i + 1;
         }
         // let every load still in flight land before the CTA can exit
@@ -495,12 +494,12 @@ struct DecLayout {
   static constexpr int BYTES = MISC_OFF + 16;
 };
 
-template <int D, int M>
+template <int D, int M, bool FLAT>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmZ, int H, int64_t N, int q_per_batch,
                      float c, int64_t tiles_per_bh, int64_t chunk_tiles,
-                     __nv_bfloat16* __restrict__ Y, uint32_t* __restrict__ err) {
+                     __nv_bfloat16* __restrict__ Y, Tok ty, uint32_t* __restrict__ err) {
   using L = DecLayout<D, M>;
   constexpr int RB = L::RB;
   constexpr uint32_t SW = umma_swizzle_code(RB);
@@ -528,6 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int chunk = blockIdx.x;
   const int64_t bh = blockIdx.y;
   const int64_t h = bh % H;
+  const int64_t yhead = ty.head(bh, H);   // row 0 of this head in Y
   const int64_t tile0 = (int64_t)chunk * chunk_tiles;
   const int64_t ntiles = imin64(chunk_tiles, tiles_per_bh - tile0);
 
@@ -574,8 +574,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (*abort_flag) break;
         mbar_arrive_expect_tx(&k_full[s], L::TILE);
-        tma_load_3d(smem + L::K_OFF + s * L::TILE, &tmK, &k_full[s], 0,
-                    (int32_t)((tile0 + i) * kTile), (int32_t)bh);
+        tma_load_tok<FLAT>(smem + L::K_OFF + s * L::TILE, &tmK, &k_full[s],
+                     (int32_t)((tile0 + i) * kTile), bh, H);
         issued = i + 1;
       }
       for (int64_t i = (issued > kDecStages ? issued - kDecStages : 0); i < issued; ++i)
@@ -711,7 +711,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&s_empty[w]);
       if (tok < N) {
         const float inv = 1.f / ((sf[0] + sf[1]) + (sf[2] + sf[3]));
-        uint4* dst = reinterpret_cast<uint4*>(Y + (bh * N + tok) * D);
+        uint4* dst = reinterpret_cast<uint4*>(Y + yhead + tok * ty.sn);
 #pragma unroll
         for (int v = 0; v < D / 8; ++v) {
           uint4 u;
@@ -778,9 +778,41 @@ cudaError_t make_map(CUtensorMap* m, const void* base, int D, int64_t rows, int6
   return cudaSuccess;
 }
 
+cudaError_t make_tok_map(CUtensorMap* m, const void* base, const Dims& d, const Tok& t,
+                         int box_rows, bool flat) {
+  auto enc = tensor_map_encoder();
+  if (!enc) {
+    note_error("cuTensorMapEncodeTiled entry point unavailable");
+    return cudaErrorNotSupported;
+  }
+  const int64_t fs = flat_stride(t, d);
+  if (flat && fs <= 0) return cudaErrorInvalidValue;
+  const cuuint32_t rank = flat ? 3 : 4;
+  cuuint64_t dims[4] = {(cuuint64_t)d.D, (cuuint64_t)d.N, (cuuint64_t)d.H, (cuuint64_t)d.B};
+  cuuint64_t strides[3] = {(cuuint64_t)t.sn * 2, (cuuint64_t)t.sh * 2, (cuuint64_t)t.sb * 2};
+  if (flat) {
+    dims[2] = (cuuint64_t)(d.B * d.H);
+    strides[1] = (cuuint64_t)fs * 2;
+  }
+  cuuint32_t box[4] = {(cuuint32_t)d.D, (cuuint32_t)box_rows, 1, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  const CUtensorMapSwizzle sw = (d.D == 32) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
+                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    note_error("cuTensorMapEncodeTiled failed (CUresult %d): token map D=%lld N=%lld H=%lld "
+               "B=%lld strides %lld/%lld/%lld box=%d",
+               (int)r, (long long)d.D, (long long)d.N, (long long)d.H, (long long)d.B,
+               (long long)t.sb, (long long)t.sh, (long long)t.sn, box_rows);
+    return cudaErrorInvalidValue;
+  }
+  return cudaSuccess;
+}
+
 namespace {
 
-template <int D, int M>
+template <int D, int M, bool FLAT>
 cudaError_t tc_encode_t(const void* Q, int64_t qbs, const void* K, const void* V, const Dims& d,
                         float scale, const ChunkPlan& plan, float* pml, float* pacc,
                         uint32_t* err, cudaStream_t st) {
@@ -788,21 +820,21 @@ cudaError_t tc_encode_t(const void* Q, int64_t qbs, const void* K, const void* V
   const int q_per_batch = qbs != 0;
   cudaError_t e;
   if ((e = make_map(&mq, Q, D, M, q_per_batch ? d.BH() : d.H, 128)) != cudaSuccess) return e;
-  if ((e = make_map(&mk, K, D, d.N, d.BH(), kEncTile)) != cudaSuccess) return e;
-  if ((e = make_map(&mv, V, D, d.N, d.BH(), kEncTile)) != cudaSuccess) return e;
+  if ((e = make_tok_map(&mk, K, d, d.k, kEncTile, FLAT)) != cudaSuccess) return e;
+  if ((e = make_tok_map(&mv, V, d, d.v, kEncTile, FLAT)) != cudaSuccess) return e;
   // two CTAs per SM: their TMEM (2 x 256 columns) fits exactly
   const int smem = EncLayout<D, M>::BYTES + 1024;
-  e = cudaFuncSetAttribute(tc_encode_kernel<D, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(tc_encode_kernel<D, M, FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem);
   if (e != cudaSuccess) return e;
   dim3 grid(plan.chunks, (unsigned)d.BH());
-  tc_encode_kernel<D, M><<<grid, kThreads, smem, st>>>(
-      mq, mk, mv, (int)d.H, d.N, q_per_batch, scale * kLog2e, plan.tiles_per_bh, plan.chunk_tiles,
-      plan.slots_per_bh(), pml, pacc, err);
+  tc_encode_kernel<D, M, FLAT><<<grid, kThreads, smem, st>>>(
+      mq, mk, mv, (int)d.H, d.N, q_per_batch, scale * kLog2e, plan.tiles_per_bh,
+      plan.chunk_tiles, plan.slots_per_bh(), pml, pacc, err);
   return cudaPeekAtLastError();
 }
 
-template <int D, int M>
+template <int D, int M, bool FLAT>
 cudaError_t tc_decode_t(const void* Q, int64_t qbs, const void* K, const __nv_bfloat16* Zb,
                         void* Y, const Dims& d, float scale, const ChunkPlan& plan, uint32_t* err,
                         cudaStream_t st) {
@@ -810,17 +842,18 @@ cudaError_t tc_decode_t(const void* Q, int64_t qbs, const void* K, const __nv_bf
   const int q_per_batch = qbs != 0;
   cudaError_t e;
   if ((e = make_map(&mq, Q, D, M, q_per_batch ? d.BH() : d.H, M)) != cudaSuccess) return e;
-  if ((e = make_map(&mk, K, D, d.N, d.BH(), kTile)) != cudaSuccess) return e;
+  if ((e = make_tok_map(&mk, K, d, d.k, kTile, FLAT)) != cudaSuccess) return e;
   if ((e = make_map(&mz, Zb, D, M, d.BH(), M)) != cudaSuccess) return e;
   const int smem = (DecLayout<D, M>::BYTES + 1024 > kMinSmemBytes) ? DecLayout<D, M>::BYTES + 1024
                                                                    : kMinSmemBytes;
-  e = cudaFuncSetAttribute(tc_decode_kernel<D, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(tc_decode_kernel<D, M, FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem);
   if (e != cudaSuccess) return e;
   dim3 grid(plan.chunks, (unsigned)d.BH());
-  tc_decode_kernel<D, M><<<grid, kThreads, smem, st>>>(mq, mk, mz, (int)d.H, d.N, q_per_batch,
+  tc_decode_kernel<D, M, FLAT><<<grid, kThreads, smem, st>>>(mq, mk, mz, (int)d.H, d.N, q_per_batch,
                                                        scale * kLog2e, plan.tiles_per_bh,
-                                                       plan.chunk_tiles, (__nv_bfloat16*)Y, err);
+                                                       plan.chunk_tiles, (__nv_bfloat16*)Y, d.y,
+                                                       err);
   return cudaPeekAtLastError();
 }
 
@@ -829,20 +862,31 @@ cudaError_t tc_decode_t(const void* Q, int64_t qbs, const void* K, const __nv_bf
 cudaError_t launch_tc_encode(const void* Q, int64_t qbs, const void* K, const void* V,
                              const Dims& d, float scale, const ChunkPlan& plan, float* pml,
                              float* pacc, uint32_t* err, cudaStream_t st) {
-  if (d.D == 32 && d.M == 256) return tc_encode_t<32, 256>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
-  if (d.D == 32 && d.M == 128) return tc_encode_t<32, 128>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
-  if (d.D == 16 && d.M == 256) return tc_encode_t<16, 256>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
-  if (d.D == 16 && d.M == 128) return tc_encode_t<16, 128>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
+  const bool flat = tok_flat(d);
+  if (d.D == 32 && d.M == 256)
+    return flat ? tc_encode_t<32, 256, true>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st)
+                : tc_encode_t<32, 256, false>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
+  if (d.D == 32 && d.M == 128)
+    return flat ? tc_encode_t<32, 128, true>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st)
+                : tc_encode_t<32, 128, false>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
+  if (d.D == 16 && d.M == 256)
+    return flat ? tc_encode_t<16, 256, true>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st)
+                : tc_encode_t<16, 256, false>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
+  if (d.D == 16 && d.M == 128)
+    return flat ? tc_encode_t<16, 128, true>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st)
+                : tc_encode_t<16, 128, false>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
   return cudaErrorNotSupported;
 }
 
 cudaError_t launch_tc_decode(const void* Q, int64_t qbs, const void* K, const __nv_bfloat16* Zb,
                              void* Y, const Dims& d, float scale, const ChunkPlan& plan,
                              uint32_t* err, cudaStream_t st) {
-  if (d.D == 32 && d.M == 256) return tc_decode_t<32, 256>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
-  if (d.D == 32 && d.M == 128) return tc_decode_t<32, 128>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
-  if (d.D == 16 && d.M == 256) return tc_decode_t<16, 256>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
-  if (d.D == 16 && d.M == 128) return tc_decode_t<16, 128>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
+  // The decode takes 4-D maps for every layout: its 3-D variant measured no
+  // faster and needs more registers.
+  if (d.D == 32 && d.M == 256) return tc_decode_t<32, 256, false>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
+  if (d.D == 32 && d.M == 128) return tc_decode_t<32, 128, false>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
+  if (d.D == 16 && d.M == 256) return tc_decode_t<16, 256, false>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
+  if (d.D == 16 && d.M == 128) return tc_decode_t<16, 128, false>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
   return cudaErrorNotSupported;
 }
 

@@ -131,7 +131,7 @@ struct ALayout {
 // tile j + 1 while Y = P [Z | e0] of tile j runs on the tensor cores, and
 // then finishes tile j (delta_d, dY', dY'', statistics).  Each warpgroup has
 // two Y accumulators in TMEM for that overlap.
-template <int D>
+template <int D, bool FLAT>
 __global__ void __launch_bounds__(kThr, 1)
     tc_bwd_a_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmdY, const __grid_constant__ CUtensorMap tmZ,
@@ -249,7 +249,8 @@ __global__ void __launch_bounds__(kThr, 1)
           }
           if (*abort_flag) break;
           mbar_arrive_expect_tx(&full[s], L::TILE);
-          tma_load_3d(ring + s * L::TILE, map, &full[s], 0, (int32_t)((tile0 + i) * kT), (int32_t)bh);
+          tma_load_tok<FLAT>(ring + s * L::TILE, map, &full[s], (int32_t)((tile0 + i) * kT), bh,
+                             H);
           issued = i + 1;
         }
         // let every load still in flight land before the CTA can exit
@@ -671,7 +672,7 @@ struct BLayout {
   static constexpr int BYTES = MISC_OFF + 16;
 };
 
-template <int D>
+template <int D, bool FLAT>
 __global__ void __launch_bounds__(kThr, 1)
     tc_bwd_b_exact_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdY,
@@ -680,7 +681,7 @@ __global__ void __launch_bounds__(kThr, 1)
                     float c, float s, int64_t tiles_per_bh, int64_t chunk_tiles,
                     const float4* __restrict__ stats, const float2* __restrict__ params,
                     const float* __restrict__ lse2, int enc_only, __nv_bfloat16* __restrict__ dK,
-                    __nv_bfloat16* __restrict__ dV, float* __restrict__ dq_part,
+                    __nv_bfloat16* __restrict__ dV, Tok tdk, Tok tdv, float* __restrict__ dq_part,
                     uint32_t* __restrict__ err) {
   using L = BLayout<D>;
   constexpr int M = L::M;
@@ -714,6 +715,7 @@ __global__ void __launch_bounds__(kThr, 1)
   const int chunk = blockIdx.x, chunks = gridDim.x;
   const int64_t bh = blockIdx.y;
   const int64_t h = bh % H;
+  const int64_t dk_head = tdk.head(bh, H), dv_head = tdv.head(bh, H);   // row 0 of the head
   const int64_t tile0 = (int64_t)chunk * chunk_tiles;
   const int64_t ntiles = imin64(chunk_tiles, tiles_per_bh - tile0);
   const int64_t KQ = ntiles * NQ;   // quarters of this chunk
@@ -790,9 +792,9 @@ __global__ void __launch_bounds__(kThr, 1)
           uint8_t* dst = smem + L::ST_OFF + k * 3 * L::TILE;
           mbar_arrive_expect_tx(&st_full[k], 3 * L::TILE);
           const int32_t tok = (int32_t)((tile0 + t) * kT);
-          tma_load_3d(dst, &tmK, &st_full[k], 0, tok, (int32_t)bh);
-          tma_load_3d(dst + L::TILE, &tmV, &st_full[k], 0, tok, (int32_t)bh);
-          tma_load_3d(dst + 2 * L::TILE, &tmdY, &st_full[k], 0, tok, (int32_t)bh);
+          tma_load_tok<FLAT>(dst, &tmK, &st_full[k], tok, bh, H);
+          tma_load_tok<FLAT>(dst + L::TILE, &tmV, &st_full[k], tok, bh, H);
+          tma_load_tok<FLAT>(dst + 2 * L::TILE, &tmdY, &st_full[k], tok, bh, H);
           issued = t + 1;
         }
         for (int64_t t = (issued > kBStages ? issued - kBStages : 0); t < issued; ++t)
@@ -933,7 +935,8 @@ __global__ void __launch_bounds__(kThr, 1)
       const int64_t tok = (tile0 + tt) * kT + r;
       if (tok < N) {
         const float f = (w == 0) ? s : gv;
-        uint4* dst = reinterpret_cast<uint4*>((w == 0 ? dK : dV) + (bh * N + tok) * D);
+        uint4* dst = reinterpret_cast<uint4*>(w == 0 ? dK + dk_head + tok * tdk.sn
+                                                     : dV + dv_head + tok * tdv.sn);
         if (enc_only) {   // added to the gradient already in the rows
 #pragma unroll
           for (int v = 0; v < D / 8; ++v) {
@@ -1118,7 +1121,7 @@ struct BFLayout {
   static constexpr int BYTES = MISC_OFF + 16;
 };
 
-template <int D>
+template <int D, bool FLAT>
 __global__ void __launch_bounds__(kThr, 1)
     tc_bwd_b_fast_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdY2,
@@ -1127,8 +1130,8 @@ __global__ void __launch_bounds__(kThr, 1)
                          float c, float s, int64_t tiles_per_bh, int64_t chunk_tiles,
                          const float4* __restrict__ stats, const float2* __restrict__ params,
                          int enc_only, __nv_bfloat16* __restrict__ dK,
-                         __nv_bfloat16* __restrict__ dV, float* __restrict__ dq_part,
-                         uint32_t* __restrict__ err) {
+                         __nv_bfloat16* __restrict__ dV, Tok tdk, Tok tdv,
+                         float* __restrict__ dq_part, uint32_t* __restrict__ err) {
   using L = BFLayout<D>;
   constexpr int M = L::M;
   constexpr int NS = L::NSLOT;
@@ -1166,6 +1169,7 @@ __global__ void __launch_bounds__(kThr, 1)
   const int chunk = blockIdx.x, chunks = gridDim.x;
   const int64_t bh = blockIdx.y;
   const int64_t h = bh % H;
+  const int64_t dk_head = tdk.head(bh, H), dv_head = tdv.head(bh, H);   // row 0 of the head
   const int64_t tile0 = (int64_t)chunk * chunk_tiles;
   const int nt = (int)imin64(chunk_tiles, tiles_per_bh - tile0);
   const float2 prm = params[bh];
@@ -1236,7 +1240,7 @@ __global__ void __launch_bounds__(kThr, 1)
           }
           if (*abort_flag) break;
           mbar_arrive_expect_tx(&k_full[kb], L::TILE);
-          tma_load_3d(smem + L::K_OFF + kb * L::TILE, &tmK, &k_full[kb], 0, tok, (int32_t)bh);
+          tma_load_tok<FLAT>(smem + L::K_OFF + kb * L::TILE, &tmK, &k_full[kb], tok, bh, H);
           if (t >= VST && !mbar_wait_sleep(&v_empty[vb], (uint32_t)(((t / VST) & 1) ^ 1))) {
             record_error(err, kErrBwdBTmaWait);
             *abort_flag = 1;
@@ -1245,7 +1249,7 @@ __global__ void __launch_bounds__(kThr, 1)
           }
           uint8_t* dst = smem + L::VD_OFF + vb * 2 * L::TILE;
           mbar_arrive_expect_tx(&v_full[vb], (enc_only ? 1 : 2) * L::TILE);
-          tma_load_3d(dst, &tmV, &v_full[vb], 0, tok, (int32_t)bh);
+          tma_load_tok<FLAT>(dst, &tmV, &v_full[vb], tok, bh, H);
           if (!enc_only) tma_load_3d(dst + L::TILE, &tmdY2, &v_full[vb], 0, tok, (int32_t)bh);
           issued = t + 1;
         }
@@ -1414,7 +1418,8 @@ __global__ void __launch_bounds__(kThr, 1)
       const int64_t tok = (tile0 + tt) * kT + r;
       if (tok < N) {
         const float f = (w == 0) ? s : 1.f;
-        uint4* dst = reinterpret_cast<uint4*>((w == 0 ? dK : dV) + (bh * N + tok) * D);
+        uint4* dst = reinterpret_cast<uint4*>(w == 0 ? dK + dk_head + tok * tdk.sn
+                                                     : dV + dv_head + tok * tdv.sn);
         if (enc_only) {   // added to the gradient already in the rows
 #pragma unroll
           for (int v = 0; v < D / 8; ++v) {
@@ -1591,7 +1596,7 @@ __global__ void bwd_dq_sum_kernel(const float4* __restrict__ dq_part, int B, int
   *reinterpret_cast<uint2*>(dQ + i * 4) = make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
 }
 
-template <int D>
+template <int D, bool FLAT>
 cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, const void* dY,
                      const float* Z, const float* lse, void* dQ, void* dK, void* dV, const Dims& d,
                      float scale, const WsLayout& L, char* ws, cudaStream_t st) {
@@ -1618,9 +1623,9 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
 
   CUtensorMap mq, mk, mv, mdy, mdy2, mz, mdz, maug;
   if ((e = make_map(&mq, Q, D, kM, q_per_batch ? BH : d.H, kM)) != cudaSuccess) return e;
-  if ((e = make_map(&mk, K, D, d.N, BH, kT)) != cudaSuccess) return e;
-  if ((e = make_map(&mv, V, D, d.N, BH, kT)) != cudaSuccess) return e;
-  if ((e = make_map(&mdy, dY, D, d.N, BH, kT)) != cudaSuccess) return e;
+  if ((e = make_tok_map(&mk, K, d, d.k, kT, FLAT)) != cudaSuccess) return e;
+  if ((e = make_tok_map(&mv, V, d, d.v, kT, FLAT)) != cudaSuccess) return e;
+  if ((e = make_tok_map(&mdy, dY, d, d.dy, kT, FLAT)) != cudaSuccess) return e;
   if ((e = make_map(&mdy2, dy2, D, d.N, BH, kT)) != cudaSuccess) return e;
   if ((e = make_map(&mz, zb, D, kM, BH, kM)) != cudaSuccess) return e;
   if ((e = make_map(&mdz, dzs, D, kM, BH, kM)) != cudaSuccess) return e;
@@ -1628,9 +1633,9 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
 
   dim3 grid(p.chunks, (unsigned)BH);
   const int smemA = ALayout<D>::BYTES + 1024;
-  e = cudaFuncSetAttribute(tc_bwd_a_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemA);
+  e = cudaFuncSetAttribute(tc_bwd_a_kernel<D, FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemA);
   if (e != cudaSuccess) return e;
-  tc_bwd_a_kernel<D><<<grid, kThr, smemA, st>>>(mq, mk, mdy, mz, (int)d.H, d.N, q_per_batch, c,
+  tc_bwd_a_kernel<D, FLAT><<<grid, kThr, smemA, st>>>(mq, mk, mdy, mz, (int)d.H, d.N, q_per_batch, c,
                                                 p.tiles_per_bh, p.chunk_tiles, rref, stats, dy2,
                                                 flags, dzp, err);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
@@ -1641,20 +1646,22 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
 
   // each head runs in exactly one of the two pass-B kernels (params.y)
   const int smemF = BFLayout<D>::BYTES + 1024;
-  e = cudaFuncSetAttribute(tc_bwd_b_fast_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(tc_bwd_b_fast_kernel<D, FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smemF);
   if (e != cudaSuccess) return e;
-  tc_bwd_b_fast_kernel<D><<<grid, kThr, smemF, st>>>(
-      mq, mk, mv, mdy2, mz, mdz, maug, (int)d.H, d.N, q_per_batch, c, scale, p.tiles_per_bh,
-      p.chunk_tiles, stats, params, 0, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, dqp, err);
+  tc_bwd_b_fast_kernel<D, FLAT><<<grid, kThr, smemF, st>>>(
+      mq, mk, mv, mdy2, mz, mdz, maug, (int)d.H, d.N, q_per_batch, c, scale,
+      p.tiles_per_bh,
+      p.chunk_tiles, stats, params, 0, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, d.dk, d.dv, dqp, err);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   const int smemB = BLayout<D>::BYTES + 1024;
-  e = cudaFuncSetAttribute(tc_bwd_b_exact_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(tc_bwd_b_exact_kernel<D, FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smemB);
   if (e != cudaSuccess) return e;
-  tc_bwd_b_exact_kernel<D><<<grid, kThr, smemB, st>>>(
-      mq, mk, mv, mdy, mz, mdz, maug, (int)d.H, d.N, q_per_batch, c, scale, p.tiles_per_bh,
-      p.chunk_tiles, stats, params, lse2, 0, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, dqp, err);
+  tc_bwd_b_exact_kernel<D, FLAT><<<grid, kThr, smemB, st>>>(
+      mq, mk, mv, mdy, mz, mdz, maug, (int)d.H, d.N, q_per_batch, c, scale,
+      p.tiles_per_bh,
+      p.chunk_tiles, stats, params, lse2, 0, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, d.dk, d.dv, dqp, err);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
   const bool shared_q = (qbs == 0);
@@ -1671,7 +1678,7 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
 // FLARE's backward wrote), then dQ = sum over b of (dQ_dyn + the encode's
 // partials).  Runs after FLARE's backward on the same stream and reuses its
 // workspace.
-template <int D>
+template <int D, bool FLAT>
 cudaError_t tc_enc_bwd_t(const void* Q, const void* K, const void* V, const float* Z1,
                          const float* lse1, const void* dZ1, void* dQ, void* dK, void* dV,
                          const Dims& d, float scale, const WsLayout& L, char* ws, cudaStream_t st) {
@@ -1700,28 +1707,30 @@ cudaError_t tc_enc_bwd_t(const void* Q, const void* K, const void* V, const floa
   // the decode operands' maps point at V: valid tiles that are never used
   CUtensorMap mq, mk, mv, mz, mdz, maug;
   if ((e = make_map(&mq, Q, D, kM, d.H, kM)) != cudaSuccess) return e;
-  if ((e = make_map(&mk, K, D, d.N, BH, kT)) != cudaSuccess) return e;
-  if ((e = make_map(&mv, V, D, d.N, BH, kT)) != cudaSuccess) return e;
+  if ((e = make_tok_map(&mk, K, d, d.k, kT, FLAT)) != cudaSuccess) return e;
+  if ((e = make_tok_map(&mv, V, d, d.v, kT, FLAT)) != cudaSuccess) return e;
   if ((e = make_map(&mz, zb, D, kM, BH, kM)) != cudaSuccess) return e;
   if ((e = make_map(&mdz, dzs, D, kM, BH, kM)) != cudaSuccess) return e;
   if ((e = make_map(&maug, aug, 16, kM, BH, kM)) != cudaSuccess) return e;
 
   dim3 grid(p.chunks, (unsigned)BH);
   const int smemF = BFLayout<D>::BYTES + 1024;
-  e = cudaFuncSetAttribute(tc_bwd_b_fast_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(tc_bwd_b_fast_kernel<D, FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smemF);
   if (e != cudaSuccess) return e;
-  tc_bwd_b_fast_kernel<D><<<grid, kThr, smemF, st>>>(
-      mq, mk, mv, mv, mz, mdz, maug, (int)d.H, d.N, 0, c, scale, p.tiles_per_bh, p.chunk_tiles,
-      stats, params, 1, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, dqp, err);
+  tc_bwd_b_fast_kernel<D, FLAT><<<grid, kThr, smemF, st>>>(
+      mq, mk, mv, mv, mz, mdz, maug, (int)d.H, d.N, 0, c, scale, p.tiles_per_bh,
+      p.chunk_tiles,
+      stats, params, 1, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, d.dk, d.dv, dqp, err);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   const int smemB = BLayout<D>::BYTES + 1024;
-  e = cudaFuncSetAttribute(tc_bwd_b_exact_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(tc_bwd_b_exact_kernel<D, FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smemB);
   if (e != cudaSuccess) return e;
-  tc_bwd_b_exact_kernel<D><<<grid, kThr, smemB, st>>>(
-      mq, mk, mv, mv, mz, mdz, maug, (int)d.H, d.N, 0, c, scale, p.tiles_per_bh, p.chunk_tiles,
-      stats, params, lse2, 1, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, dqp, err);
+  tc_bwd_b_exact_kernel<D, FLAT><<<grid, kThr, smemB, st>>>(
+      mq, mk, mv, mv, mz, mdz, maug, (int)d.H, d.N, 0, c, scale, p.tiles_per_bh,
+      p.chunk_tiles,
+      stats, params, lse2, 1, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, d.dk, d.dv, dqp, err);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
   const int64_t total = d.H * kM * D;
@@ -1738,8 +1747,13 @@ cudaError_t launch_tc_bwd(const void* Q, int64_t qbs, const void* K, const void*
                           void* dV, const Dims& d, float scale, const WsLayout& L, char* ws,
                           cudaStream_t st) {
   if (d.M != kM) return cudaErrorNotSupported;
-  if (d.D == 32) return tc_bwd_t<32>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
-  if (d.D == 16) return tc_bwd_t<16>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
+  const bool flat = tok_flat(d);
+  if (d.D == 32)
+    return flat ? tc_bwd_t<32, true>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st)
+                : tc_bwd_t<32, false>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
+  if (d.D == 16)
+    return flat ? tc_bwd_t<16, true>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st)
+                : tc_bwd_t<16, false>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
   return cudaErrorNotSupported;
 }
 
@@ -1748,8 +1762,13 @@ cudaError_t launch_tc_enc_bwd(const void* Q, const void* K, const void* V, const
                               const Dims& d, float scale, const WsLayout& L, char* ws,
                               cudaStream_t st) {
   if (d.M != kM) return cudaErrorNotSupported;
-  if (d.D == 32) return tc_enc_bwd_t<32>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st);
-  if (d.D == 16) return tc_enc_bwd_t<16>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st);
+  const bool flat = tok_flat(d);
+  if (d.D == 32)
+    return flat ? tc_enc_bwd_t<32, true>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st)
+                : tc_enc_bwd_t<32, false>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st);
+  if (d.D == 16)
+    return flat ? tc_enc_bwd_t<16, true>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st)
+                : tc_enc_bwd_t<16, false>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st);
   return cudaErrorNotSupported;
 }
 

@@ -131,6 +131,27 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t c0, int32_t c1, int32_t c2, int32_t c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];"
+      ::"r"(smem_u32(dst)), "l"((uint64_t)map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
+        "r"(c3)
+      : "memory");
+}
+
+// One box of a token tensor: tokens [tok, tok + box) of head bh = b H + h,
+// through a 3-D map {D, N, B*H} (FLAT) or a 4-D map {D, N, H, B}.
+template <bool FLAT>
+__device__ __forceinline__ void tma_load_tok(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                             int32_t tok, int64_t bh, int H) {
+  if constexpr (FLAT)
+    tma_load_3d(dst, map, bar, 0, tok, (int32_t)bh);
+  else
+    tma_load_4d(dst, map, bar, 0, tok, (int32_t)(bh % H), (int32_t)(bh / H));
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)map) : "memory");
 }

@@ -35,6 +35,38 @@ def _need_cuda(*ts):
             raise ValueError("FLARE tensors must be contiguous")
 
 
+def _need_tokens(*ts):
+    """Token tensors [B,H,N,D]: on the device, D contiguous, any other strides."""
+    shape = None
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("FLARE tensors must live on a CUDA device")
+        if t.dim() != 4 or t.stride(-1) != 1:
+            raise ValueError("token tensors must be [B,H,N,D] views with D contiguous")
+        if shape is not None and t.shape != shape:
+            raise ValueError(f"token tensors differ in shape: {tuple(t.shape)} vs {tuple(shape)}")
+        shape = t.shape
+
+
+def _strides(*ts):
+    """None when every token tensor is contiguous, else the flare_strides_t
+    array (one entry per tensor, in the C entry point's order)."""
+    if all(t.is_contiguous() for t in ts):
+        return None
+    arr = (_lib.FlareStrides * len(ts))()
+    for i, t in enumerate(ts):
+        arr[i] = _lib.FlareStrides(t.stride(0), t.stride(1), t.stride(2))
+    return arr
+
+
+def _like(t: torch.Tensor) -> torch.Tensor:
+    """An output with t's layout (empty_like keeps the strides of a dense
+    tensor); a contiguous one where t's layout has gaps or overlaps."""
+    return torch.empty_like(t)
+
+
 def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -99,18 +131,29 @@ def device_status(workspace: torch.Tensor, stream=None) -> int:
 def flare_fwd(Q, K, V, scale: Optional[float] = None, *, save: bool = False,
               workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
               stream=None):
-    """FLARE forward.  Returns Y, or (Y, Z, lse) when ``save``."""
-    _need_cuda(Q, K, V, workspace, out)
+    """FLARE forward.  Returns Y, or (Y, Z, lse) when ``save``.
+
+    K, V (and ``out``) may be any [B,H,N,D] views with D contiguous, e.g.
+    ``x.transpose(1, 2)`` of a [B,N,H,D] projection output; Y then takes K's
+    layout."""
+    _need_cuda(Q, workspace)
+    _need_tokens(K, V, out)
     B, H, N, M, D, qbs = _dims(Q, K)
     dt = _dtype_code(K)
     s = default_scale(D) if scale is None else float(scale)
-    Y = torch.empty_like(K) if out is None else out
+    Y = _like(K) if out is None else out
     Z = torch.empty((B, H, M, D), dtype=torch.float32, device=K.device) if save else None
     lse = torch.empty((B, H, M), dtype=torch.float32, device=K.device) if save else None
     ws = workspace if workspace is not None else alloc_workspace(
         _lib.FLARE_OP_FWD, B, H, N, M, D, K.dtype, K.device)
-    st = _lib.load().flare_fwd(_ptr(Q), qbs, _ptr(K), _ptr(V), _ptr(Y), B, H, N, M, D, dt, s,
-                               _ptr(Z), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream))
+    strides = _strides(K, V, Y)
+    if strides is None:
+        st = _lib.load().flare_fwd(_ptr(Q), qbs, _ptr(K), _ptr(V), _ptr(Y), B, H, N, M, D, dt, s,
+                                   _ptr(Z), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream))
+    else:
+        st = _lib.load().flare_fwd_strided(_ptr(Q), qbs, _ptr(K), _ptr(V), _ptr(Y), strides, B, H,
+                                           N, M, D, dt, s, _ptr(Z), _ptr(lse), _ptr(ws),
+                                           ws.numel(), _stream(stream))
     _lib.check(st, "flare_fwd")
     return (Y, Z, lse) if save else Y
 
@@ -119,40 +162,56 @@ def flare_pp_fwd(Q, K, V, scale: Optional[float] = None, *, save: bool = False,
                  workspace: Optional[torch.Tensor] = None, stream=None):
     """FLARE++ forward with learned Q [H,M,D].  Returns (Y, Q_dyn) or
     (Y, Q_dyn, Z, lse) when ``save``."""
-    _need_cuda(Q, K, V, workspace)
+    _need_cuda(Q, workspace)
+    _need_tokens(K, V)
     B, H, N, M, D, qbs = _dims(Q, K)
     if qbs != 0:
         raise ValueError("FLARE++ takes learned latents Q of shape [H,M,D]")
     dt = _dtype_code(K)
     s = default_scale(D) if scale is None else float(scale)
-    Y = torch.empty_like(K)
+    Y = _like(K)
     Qd = torch.empty((B, H, M, D), dtype=K.dtype, device=K.device)
     Z = torch.empty((B, H, M, D), dtype=torch.float32, device=K.device) if save else None
     lse = torch.empty((B, H, M), dtype=torch.float32, device=K.device) if save else None
     ws = workspace if workspace is not None else alloc_workspace(
         _lib.FLARE_OP_PP_FWD, B, H, N, M, D, K.dtype, K.device)
-    st = _lib.load().flare_pp_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(Y), _ptr(Qd), B, H, N, M, D,
-                                  dt, s, _ptr(Z), _ptr(lse), _ptr(ws), ws.numel(),
-                                  _stream(stream))
+    strides = _strides(K, V, Y)
+    if strides is None:
+        st = _lib.load().flare_pp_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(Y), _ptr(Qd), B, H, N, M,
+                                      D, dt, s, _ptr(Z), _ptr(lse), _ptr(ws), ws.numel(),
+                                      _stream(stream))
+    else:
+        st = _lib.load().flare_pp_fwd_strided(_ptr(Q), _ptr(K), _ptr(V), _ptr(Y), _ptr(Qd),
+                                              strides, B, H, N, M, D, dt, s, _ptr(Z), _ptr(lse),
+                                              _ptr(ws), ws.numel(), _stream(stream))
     _lib.check(st, "flare_pp_fwd")
     return (Y, Qd, Z, lse) if save else (Y, Qd)
 
 
 def flare_bwd(Q, K, V, dY, Z, lse, scale: Optional[float] = None, *,
               workspace: Optional[torch.Tensor] = None, stream=None):
-    """FLARE backward.  Returns (dQ, dK, dV)."""
-    _need_cuda(Q, K, V, dY, Z, lse, workspace)
+    """FLARE backward.  Returns (dQ, dK, dV); dK and dV take K's and V's
+    layouts (token tensors may be strided as in flare_fwd)."""
+    _need_cuda(Q, Z, lse, workspace)
+    _need_tokens(K, V, dY)
     B, H, N, M, D, qbs = _dims(Q, K)
     dt = _dtype_code(K)
     s = default_scale(D) if scale is None else float(scale)
     dQ = torch.empty_like(Q)
-    dK = torch.empty_like(K)
-    dV = torch.empty_like(V)
+    dK = _like(K)
+    dV = _like(V)
     ws = workspace if workspace is not None else alloc_workspace(
         _lib.FLARE_OP_BWD, B, H, N, M, D, K.dtype, K.device)
-    st = _lib.load().flare_bwd(_ptr(Q), qbs, _ptr(K), _ptr(V), _ptr(dY), _ptr(Z), _ptr(lse),
-                               _ptr(dQ), _ptr(dK), _ptr(dV), B, H, N, M, D, dt, s, _ptr(ws),
-                               ws.numel(), _stream(stream))
+    strides = _strides(K, V, dY, dK, dV)
+    if strides is None:
+        st = _lib.load().flare_bwd(_ptr(Q), qbs, _ptr(K), _ptr(V), _ptr(dY), _ptr(Z), _ptr(lse),
+                                   _ptr(dQ), _ptr(dK), _ptr(dV), B, H, N, M, D, dt, s, _ptr(ws),
+                                   ws.numel(), _stream(stream))
+    else:
+        st = _lib.load().flare_bwd_strided(_ptr(Q), qbs, _ptr(K), _ptr(V), _ptr(dY), _ptr(Z),
+                                           _ptr(lse), _ptr(dQ), _ptr(dK), _ptr(dV), strides, B,
+                                           H, N, M, D, dt, s, _ptr(ws), ws.numel(),
+                                           _stream(stream))
     _lib.check(st, "flare_bwd")
     return dQ, dK, dV
 
@@ -161,20 +220,28 @@ def flare_pp_bwd(Q, K, V, dY, Q_dyn, Z, lse, scale: Optional[float] = None, *,
                  workspace: Optional[torch.Tensor] = None, stream=None):
     """FLARE++ backward with learned Q [H,M,D] (Q_dyn, Z, lse from
     flare_pp_fwd(..., save=True)).  Returns (dQ [H,M,D], dK, dV)."""
-    _need_cuda(Q, K, V, dY, Q_dyn, Z, lse, workspace)
+    _need_cuda(Q, Q_dyn, Z, lse, workspace)
+    _need_tokens(K, V, dY)
     B, H, N, M, D, qbs = _dims(Q, K)
     if qbs != 0:
         raise ValueError("FLARE++ takes learned latents Q of shape [H,M,D]")
     dt = _dtype_code(K)
     s = default_scale(D) if scale is None else float(scale)
     dQ = torch.empty_like(Q)
-    dK = torch.empty_like(K)
-    dV = torch.empty_like(V)
+    dK = _like(K)
+    dV = _like(V)
     ws = workspace if workspace is not None else alloc_workspace(
         _lib.FLARE_OP_PP_BWD, B, H, N, M, D, K.dtype, K.device)
-    st = _lib.load().flare_pp_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(dY), _ptr(Q_dyn), _ptr(Z),
-                                  _ptr(lse), _ptr(dQ), _ptr(dK), _ptr(dV), B, H, N, M, D, dt, s,
-                                  _ptr(ws), ws.numel(), _stream(stream))
+    strides = _strides(K, V, dY, dK, dV)
+    if strides is None:
+        st = _lib.load().flare_pp_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(dY), _ptr(Q_dyn), _ptr(Z),
+                                      _ptr(lse), _ptr(dQ), _ptr(dK), _ptr(dV), B, H, N, M, D, dt,
+                                      s, _ptr(ws), ws.numel(), _stream(stream))
+    else:
+        st = _lib.load().flare_pp_bwd_strided(_ptr(Q), _ptr(K), _ptr(V), _ptr(dY), _ptr(Q_dyn),
+                                              _ptr(Z), _ptr(lse), _ptr(dQ), _ptr(dK), _ptr(dV),
+                                              strides, B, H, N, M, D, dt, s, _ptr(ws),
+                                              ws.numel(), _stream(stream))
     _lib.check(st, "flare_pp_bwd")
     return dQ, dK, dV
 

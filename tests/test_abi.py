@@ -206,3 +206,61 @@ def test_binding_fails_loudly_without_cuda_tensors():
     x = torch.zeros(1, 2, 8, 16)
     with pytest.raises(ValueError):
         fl.flare_fwd(torch.zeros(2, 16, 16), x, x)
+
+
+def _st(*triples):
+    arr = (_lib.FlareStrides * len(triples))()
+    for i, t in enumerate(triples):
+        arr[i] = _lib.FlareStrides(*t)
+    return arr
+
+
+@no_gpu_only
+def test_strided_entry_points_validate_strides(lib):
+    # B2 H2 N100 M32 D16 float32: rows must start on 16 bytes (4 elements)
+    B, H, N, M, D = 2, 2, 100, 32, 16
+    F = FAKE
+    ws = lib.flare_workspace_size(0, B, H, N, M, D, 0)
+    contig = (H * N * D, N * D, D)
+    bnhd = (N * H * D, D, H * D)
+
+    def fwd(*triples):
+        st = _st(*triples) if triples else None
+        return lib.flare_fwd_strided(_p(F), 0, _p(F), _p(F), _p(F), st, B, H, N, M, D, 0, 0.25,
+                                     None, None, _p(F), ws, None)
+
+    # valid layouts pass validation and fail only at the first enqueue
+    assert fwd() == CUDA
+    assert fwd(contig, contig, contig) == CUDA
+    assert fwd(bnhd, bnhd, bnhd) == CUDA
+    assert fwd(contig, bnhd, (N * H * D, D, H * D)) == CUDA
+    # an input may overlap itself (rows 8 elements apart); an output may not
+    assert fwd((H * N * 8, N * 8, 8), contig, contig) == CUDA
+    assert fwd(contig, contig, (H * N * 8, N * 8, 8)) == INVALID
+    assert fwd(contig, contig, (N * D, N * D, D)) == INVALID   # b and h rows coincide
+    # strides must be positive multiples of 16 bytes
+    assert fwd((0, N * D, D), contig, contig) == INVALID
+    assert fwd(contig, (H * N * D, N * D, -D), contig) == INVALID
+    assert fwd(contig, contig, (H * N * 18, N * 18, 18)) == UNSUPPORTED
+    assert fwd((1 << 40, N * D, D), contig, contig) == INVALID
+    # the backward's outputs dK, dV are the 4th and 5th entries
+    wsb = lib.flare_workspace_size(2, B, H, N, M, D, 0)
+
+    def bwd(*triples):
+        return lib.flare_bwd_strided(_p(F), 0, _p(F), _p(F), _p(F), _p(F), _p(F), _p(F), _p(F),
+                                     _p(F), _st(*triples), B, H, N, M, D, 0, 0.25, _p(F), wsb,
+                                     None)
+
+    assert bwd(bnhd, bnhd, bnhd, bnhd, bnhd) == CUDA
+    assert bwd(bnhd, bnhd, bnhd, bnhd, (N * H * D, D, 8)) == INVALID
+    assert bwd(bnhd, bnhd, (N * H * D, D, 8), bnhd, bnhd) == CUDA
+    wsp = lib.flare_workspace_size(1, B, H, N, M, D, 0)
+    assert lib.flare_pp_fwd_strided(_p(F), _p(F), _p(F), _p(F), None, _st(bnhd, bnhd, bnhd), B,
+                                    H, N, M, D, 0, 0.25, None, None, _p(F), wsp, None) == CUDA
+    assert lib.flare_pp_fwd_strided(_p(F), _p(F), _p(F), _p(F), None,
+                                    _st(bnhd, bnhd, (N * D, N * D, D)), B, H, N, M, D, 0, 0.25,
+                                    None, None, _p(F), wsp, None) == INVALID
+    wspb = lib.flare_workspace_size(3, B, H, N, M, D, 0)
+    assert lib.flare_pp_bwd_strided(_p(F), _p(F), _p(F), _p(F), _p(F), _p(F), _p(F), _p(F),
+                                    _p(F), _p(F), _st(bnhd, bnhd, bnhd, (0, D, H * D), bnhd), B,
+                                    H, N, M, D, 0, 0.25, _p(F), wspb, None) == INVALID
