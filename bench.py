@@ -419,7 +419,8 @@ def _row_roofline(t_ms: float, exps: float, flops: float, hbm_bytes: float, peak
 
 
 def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0,
-                    which=("flare_pp_fwd", "flare_fwd_bwd", "flare_pp_fwd_bwd")):
+                    which=("flare_pp_fwd", "flare_fwd_bwd", "flare_pp_fwd_bwd",
+                           "flare_strided")):
     """Times the FLARE++ forward (B=2 H=8 N=262,144 M=256 D=32) and the
     forward + backward of B=8 H=8 N=16,384 M=128 D=32, both bf16, on the
     same device with CUDA events (median of `iters` launches after 3
@@ -453,6 +454,8 @@ def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0,
         rows.update(_time_fwd_bwd(dev, peaks, peak_kind, timed, seed))
     if "flare_pp_fwd_bwd" in which:
         rows.update(_time_pp_fwd_bwd(dev, peaks, peak_kind, timed, seed))
+    if "flare_strided" in which:
+        rows.update(_time_strided(dev, peaks, peak_kind, timed, seed))
     del flush_buf
     torch.cuda.empty_cache()
     return rows
@@ -507,6 +510,69 @@ def _time_fwd_bwd(dev, peaks, peak_kind, timed, seed):
         "bwd_roofline": _row_roofline(ms_b, 2.0 * u * w.M, 20.0 * u * w.M * w.D,
                                       5.0 * u * w.D * 2, peaks, peak_kind)}
     return rows
+
+
+def _time_strided(dev, peaks, peak_kind, timed, seed):
+    """Token tensors stored [B,N,H,D] (a fused projection's layout) and read
+    in place: the headline forward (B=1: batch and head flatten, 3-D maps)
+    and the forward + backward workload (B=8: 4-D maps), each beside the
+    same call on contiguous [B,H,N,D] tensors.  Algorithmic work as in the
+    contiguous rows."""
+    import torch
+
+    import rank_latent_attention_flare_b200 as fl
+
+    def bnhd(t):
+        return t.transpose(1, 2).contiguous().transpose(1, 2)
+
+    out = {}
+    w = WORKLOAD
+    x = make_inputs(w.B, w.H, w.N, w.M, w.D, dtype=w.torch_dtype, seed=seed)
+    Q = x["Q"].to(dev)
+    Kt, Vt = bnhd(x["K"].to(dev)), bnhd(x["V"].to(dev))
+    Yt = torch.empty_like(Kt)
+    ws = fl.alloc_workspace(fl.FLARE_OP_FWD, w.B, w.H, w.N, w.M, w.D, w.torch_dtype, dev)
+    ms_t = timed(lambda: fl.flare_fwd(Q, Kt, Vt, w.scale, workspace=ws, out=Yt))
+    del Kt, Vt, Yt
+    K, V = x["K"].to(dev), x["V"].to(dev)
+    Y = torch.empty_like(K)
+    ms_c = timed(lambda: fl.flare_fwd(Q, K, V, w.scale, workspace=ws, out=Y))
+    if fl.device_status(ws) != 0:
+        raise RuntimeError("device wait ran out in the strided forward")
+    del K, V, Y, ws
+    u = w.B * w.H * w.N
+    out["fwd_headline_bnhd"] = {
+        "workload": f"FLARE fwd B={w.B} H={w.H} N={w.N} M={w.M} D={w.D} bf16, K/V/Y [B,N,H,D]",
+        "ms": round(ms_t, 4), "contiguous_ms": round(ms_c, 4),
+        "tokens_per_s": w.B * w.N / (ms_t / 1e3),
+        "roofline": _row_roofline(ms_t, 2.0 * u * w.M, 8.0 * u * w.M * w.D, 4.0 * u * w.D * 2,
+                                  peaks, peak_kind)}
+    w = WORKLOADS["c5_fwdbwd_bf16_16k"]
+    x = make_inputs(w.B, w.H, w.N, w.M, w.D, dtype=w.torch_dtype, seed=seed, with_dy=True)
+    Q = x["Q"].to(dev)
+    t = {k: bnhd(x[k].to(dev)) for k in ("K", "V", "dY")}
+    wsf = fl.alloc_workspace(fl.FLARE_OP_FWD, w.B, w.H, w.N, w.M, w.D, w.torch_dtype, dev)
+    wsb = fl.alloc_workspace(fl.FLARE_OP_BWD, w.B, w.H, w.N, w.M, w.D, w.torch_dtype, dev)
+    saved = {}
+
+    def fwd():
+        saved["out"] = fl.flare_fwd(Q, t["K"], t["V"], w.scale, save=True, workspace=wsf)
+
+    ms_f = timed(fwd)
+    _, Z, lse = saved["out"]
+    ms_b = timed(lambda: fl.flare_bwd(Q, t["K"], t["V"], t["dY"], Z, lse, w.scale, workspace=wsb))
+    if fl.device_status(wsf) != 0 or fl.device_status(wsb) != 0:
+        raise RuntimeError("device wait ran out in the strided forward + backward")
+    u = w.B * w.H * w.N
+    ms = ms_f + ms_b
+    out["fwd_bwd_bnhd"] = {
+        "workload": f"FLARE fwd+bwd B={w.B} H={w.H} N={w.N} M={w.M} D={w.D} bf16, "
+                    "K/V/dY/Y/dK/dV [B,N,H,D]",
+        "ms": round(ms, 4), "fwd_ms": round(ms_f, 4), "bwd_ms": round(ms_b, 4),
+        "tokens_per_s": w.B * w.N / (ms / 1e3),
+        "roofline": _row_roofline(ms, 4.0 * u * w.M, 28.0 * u * w.M * w.D,
+                                  9.0 * u * w.D * 2, peaks, peak_kind)}
+    return {"flare_strided": out}
 
 
 def time_sdpa_context(dev, w=WORKLOAD, iters: int = 5, seed: int = 0):
@@ -641,7 +707,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true",
                     help="skip the FLARE++ and forward+backward timings")
-    ap.add_argument("--row", choices=["flare_pp_fwd", "flare_fwd_bwd", "flare_pp_fwd_bwd"],
+    ap.add_argument("--row", choices=["flare_pp_fwd", "flare_fwd_bwd", "flare_pp_fwd_bwd",
+                                      "flare_strided"],
                     default=None,
                     help="time only this workload (one JSON line with its timing and roofline)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
