@@ -40,6 +40,14 @@
  * [B,H,M,D] when q_bstride == H*M*D; K, V, Y, dY are [B,H,N,D]; Z is
  * [B,H,M,D]; lse is [B,H,M].  All arrays are contiguous, row-major double.
  *
+ * Sequence lengths (key-padding mask; the skill page's module accepts an
+ * attention mask): lens, when not NULL, gives each batch element's number of
+ * valid tokens L_b (clamped to [0, N]); tokens n >= L_b are padding.  The
+ * encode's softmax runs over n < L_b only, the decode produces Y[n] for
+ * n < L_b and Y[n] = 0 for padding, and padding gets zero dK and dV and
+ * contributes nothing to any other gradient.  A sequence with no tokens
+ * encodes to Z = 0 (an empty weighted sum) with lse = -inf.
+ *
  * Parity status: every function here is pinned by CPU tests (brute-force
  * mixing matrix, closed forms, hard-max limit, permutation equivariance,
  * float64 SDPA cross-check, central finite differences for the gradient,
@@ -59,6 +67,12 @@ static double dotd(const double* a, const double* b, int64_t D) {
   return s;
 }
 
+static int64_t seq_len(const int32_t* lens, int64_t b, int64_t N) {
+  if (!lens) return N;
+  int64_t L = lens[b];
+  return L < 0 ? 0 : (L > N ? N : L);
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();
@@ -76,29 +90,35 @@ int oracle_num_threads(void) {
  * lse may be NULL.
  */
 void oracle_encode(const double* Q, int64_t q_bstride, const double* K,
-                   const double* V, int64_t B, int64_t H, int64_t N,
-                   int64_t M, int64_t D, double scale, double* Z,
+                   const double* V, const int32_t* lens, int64_t B, int64_t H,
+                   int64_t N, int64_t M, int64_t D, double scale, double* Z,
                    double* lse) {
 #pragma omp parallel for collapse(3) schedule(dynamic, 1)
   for (int64_t b = 0; b < B; ++b)
     for (int64_t h = 0; h < H; ++h)
       for (int64_t m = 0; m < M; ++m) {
+        const int64_t Nb = seq_len(lens, b, N);
         const double* q = Q + b * q_bstride + (h * M + m) * D;
         const double* Kb = K + (b * H + h) * N * D;
         const double* Vb = V + (b * H + h) * N * D;
+        double* z = Z + ((b * H + h) * M + m) * D;
+        if (Nb == 0) {   /* no tokens: an empty weighted sum */
+          for (int64_t d = 0; d < D; ++d) z[d] = 0.0;
+          if (lse) lse[(b * H + h) * M + m] = -INFINITY;
+          continue;
+        }
         double mu = -INFINITY;
-        for (int64_t n = 0; n < N; ++n) {
+        for (int64_t n = 0; n < Nb; ++n) {
           double l = scale * dotd(q, Kb + n * D, D);
           if (l > mu) mu = l;
         }
         double* acc = (double*)calloc((size_t)D, sizeof(double));
         double den = 0.0;
-        for (int64_t n = 0; n < N; ++n) {
+        for (int64_t n = 0; n < Nb; ++n) {
           double w = exp(scale * dotd(q, Kb + n * D, D) - mu);
           den += w;
           for (int64_t d = 0; d < D; ++d) acc[d] += w * Vb[n * D + d];
         }
-        double* z = Z + ((b * H + h) * M + m) * D;
         for (int64_t d = 0; d < D; ++d) z[d] = acc[d] / den;
         if (lse) lse[(b * H + h) * M + m] = mu + log(den);
         free(acc);
@@ -125,8 +145,8 @@ static void decode_row(const double* q_bh, const double* k, const double* z_bh,
 
 /* Decode [P4]: Y[b,h,n] = softmax_M(s K[b,h,n] Q[h]^T) Z[b,h]. */
 void oracle_decode(const double* Q, int64_t q_bstride, const double* K,
-                   const double* Z, int64_t B, int64_t H, int64_t N,
-                   int64_t M, int64_t D, double scale, double* Y) {
+                   const double* Z, const int32_t* lens, int64_t B, int64_t H,
+                   int64_t N, int64_t M, int64_t D, double scale, double* Y) {
 #pragma omp parallel for collapse(3) schedule(static)
   for (int64_t b = 0; b < B; ++b)
     for (int64_t h = 0; h < H; ++h)
@@ -134,7 +154,12 @@ void oracle_decode(const double* Q, int64_t q_bstride, const double* K,
         const double* q_bh = Q + b * q_bstride + h * M * D;
         const double* z_bh = Z + (b * H + h) * M * D;
         const double* k = K + ((b * H + h) * N + n) * D;
-        decode_row(q_bh, k, z_bh, M, D, scale, Y + ((b * H + h) * N + n) * D);
+        double* y = Y + ((b * H + h) * N + n) * D;
+        if (n >= seq_len(lens, b, N)) {   /* padding */
+          for (int64_t d = 0; d < D; ++d) y[d] = 0.0;
+          continue;
+        }
+        decode_row(q_bh, k, z_bh, M, D, scale, y);
       }
 }
 
@@ -160,11 +185,11 @@ void oracle_decode_rows(const double* Q, int64_t q_bstride, const double* K,
 
 /* FLARE forward [P1 s4, P4]: Z = encode(Q,K,V); Y = decode(Q,K,Z). */
 void oracle_flare_fwd(const double* Q, int64_t q_bstride, const double* K,
-                      const double* V, int64_t B, int64_t H, int64_t N,
-                      int64_t M, int64_t D, double scale, double* Y,
-                      double* Z, double* lse) {
-  oracle_encode(Q, q_bstride, K, V, B, H, N, M, D, scale, Z, lse);
-  oracle_decode(Q, q_bstride, K, Z, B, H, N, M, D, scale, Y);
+                      const double* V, const int32_t* lens, int64_t B,
+                      int64_t H, int64_t N, int64_t M, int64_t D, double scale,
+                      double* Y, double* Z, double* lse) {
+  oracle_encode(Q, q_bstride, K, V, lens, B, H, N, M, D, scale, Z, lse);
+  oracle_decode(Q, q_bstride, K, Z, lens, B, H, N, M, D, scale, Y);
 }
 
 /*
@@ -176,17 +201,17 @@ void oracle_flare_fwd(const double* Q, int64_t q_bstride, const double* K,
  * Qdyn, Z and lse are outputs (lse may be NULL).
  */
 void oracle_flare_pp_fwd(const double* Q, const double* K, const double* V,
-                         int64_t B, int64_t H, int64_t N, int64_t M,
-                         int64_t D, double scale, double* Y, double* Qdyn,
-                         double* Z, double* lse) {
+                         const int32_t* lens, int64_t B, int64_t H, int64_t N,
+                         int64_t M, int64_t D, double scale, double* Y,
+                         double* Qdyn, double* Z, double* lse) {
   int64_t per_b = H * M * D;
   double* Z1 = (double*)malloc((size_t)(B * per_b) * sizeof(double));
-  oracle_encode(Q, 0, K, V, B, H, N, M, D, scale, Z1, NULL);
+  oracle_encode(Q, 0, K, V, lens, B, H, N, M, D, scale, Z1, NULL);
   for (int64_t b = 0; b < B; ++b)
     for (int64_t i = 0; i < per_b; ++i) Qdyn[b * per_b + i] = Q[i] + Z1[b * per_b + i];
   free(Z1);
-  oracle_encode(Qdyn, per_b, K, V, B, H, N, M, D, scale, Z, lse);
-  oracle_decode(Qdyn, per_b, K, Z, B, H, N, M, D, scale, Y);
+  oracle_encode(Qdyn, per_b, K, V, lens, B, H, N, M, D, scale, Z, lse);
+  oracle_decode(Qdyn, per_b, K, Z, lens, B, H, N, M, D, scale, Y);
 }
 
 /*
@@ -203,14 +228,15 @@ void oracle_flare_pp_fwd(const double* Q, const double* K, const double* V,
  * dQ is [H,M,D] summed over b when q_bstride == 0, else [B,H,M,D].
  */
 void oracle_flare_bwd(const double* Q, int64_t q_bstride, const double* K,
-                      const double* V, const double* dY, int64_t B, int64_t H,
-                      int64_t N, int64_t M, int64_t D, double scale,
-                      double* dQ, double* dK, double* dV) {
+                      const double* V, const double* dY, const int32_t* lens,
+                      int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
+                      double scale, double* dQ, double* dK, double* dV) {
   int64_t BH = B * H;
   double* dQbh = (double*)calloc((size_t)(BH * M * D), sizeof(double));
 #pragma omp parallel for schedule(dynamic, 1)
   for (int64_t bh = 0; bh < BH; ++bh) {
     int64_t b = bh / H, h = bh % H;
+    const int64_t Nb = seq_len(lens, b, N);   /* tokens n >= Nb are padding */
     const double* q = Q + b * q_bstride + h * M * D;
     const double* k = K + bh * N * D;
     const double* v = V + bh * N * D;
@@ -225,23 +251,23 @@ void oracle_flare_bwd(const double* Q, int64_t q_bstride, const double* K,
     /* forward recompute: P_e rows (softmax over n) and Z */
     for (int64_t m = 0; m < M; ++m) {
       double mu = -INFINITY;
-      for (int64_t n = 0; n < N; ++n) {
+      for (int64_t n = 0; n < Nb; ++n) {
         double a = scale * dotd(q + m * D, k + n * D, D);
         Pe[m * N + n] = a;
         if (a > mu) mu = a;
       }
       double den = 0.0;
-      for (int64_t n = 0; n < N; ++n) {
+      for (int64_t n = 0; n < Nb; ++n) {
         Pe[m * N + n] = exp(Pe[m * N + n] - mu);
         den += Pe[m * N + n];
       }
-      for (int64_t n = 0; n < N; ++n) {
+      for (int64_t n = 0; n < Nb; ++n) {
         Pe[m * N + n] /= den;
         for (int64_t d = 0; d < D; ++d) Z[m * D + d] += Pe[m * N + n] * v[n * D + d];
       }
     }
     /* forward recompute: P_d rows (softmax over m) */
-    for (int64_t n = 0; n < N; ++n) {
+    for (int64_t n = 0; n < Nb; ++n) {
       double mu = -INFINITY;
       for (int64_t m = 0; m < M; ++m) {
         double a = scale * dotd(k + n * D, q + m * D, D);
@@ -256,7 +282,7 @@ void oracle_flare_bwd(const double* Q, int64_t q_bstride, const double* K,
       for (int64_t m = 0; m < M; ++m) Pd[n * M + m] /= den;
     }
     /* decode stage */
-    for (int64_t n = 0; n < N; ++n) {
+    for (int64_t n = 0; n < Nb; ++n) {
       double delta = 0.0;
       for (int64_t m = 0; m < M; ++m)
         delta += Pd[n * M + m] * dotd(dy + n * D, Z + m * D, D);
@@ -272,16 +298,16 @@ void oracle_flare_bwd(const double* Q, int64_t q_bstride, const double* K,
       }
     }
     /* encode stage */
-    for (int64_t n = 0; n < N; ++n) {
+    for (int64_t n = 0; n < Nb; ++n) {
       for (int64_t d = 0; d < D; ++d) dv[n * D + d] = 0.0;
       for (int64_t m = 0; m < M; ++m)
         for (int64_t d = 0; d < D; ++d) dv[n * D + d] += Pe[m * N + n] * dZ[m * D + d];
     }
     for (int64_t m = 0; m < M; ++m) {
       double delta = 0.0;
-      for (int64_t n = 0; n < N; ++n)
+      for (int64_t n = 0; n < Nb; ++n)
         delta += Pe[m * N + n] * dotd(dZ + m * D, v + n * D, D);
-      for (int64_t n = 0; n < N; ++n) {
+      for (int64_t n = 0; n < Nb; ++n) {
         double dA = Pe[m * N + n] * (dotd(dZ + m * D, v + n * D, D) - delta);
         for (int64_t d = 0; d < D; ++d) {
           dq[m * D + d] += scale * dA * k[n * D + d];
@@ -289,6 +315,8 @@ void oracle_flare_bwd(const double* Q, int64_t q_bstride, const double* K,
         }
       }
     }
+    for (int64_t n = Nb; n < N; ++n)   /* padding: zero gradient */
+      for (int64_t d = 0; d < D; ++d) dk[n * D + d] = dv[n * D + d] = 0.0;
     free(Pe);
     free(Pd);
     free(Z);
@@ -313,14 +341,15 @@ void oracle_flare_bwd(const double* Q, int64_t q_bstride, const double* K,
  *   dV += P^T dZ1,   dK += s dA^T Q,   dQ += s dA K (summed over b).
  */
 static void encode_bwd_add(const double* Q, const double* K, const double* V,
-                           const double* dZ1, int64_t B, int64_t H, int64_t N,
-                           int64_t M, int64_t D, double scale, double* dQ,
-                           double* dK, double* dV) {
+                           const double* dZ1, const int32_t* lens, int64_t B,
+                           int64_t H, int64_t N, int64_t M, int64_t D,
+                           double scale, double* dQ, double* dK, double* dV) {
   int64_t BH = B * H;
   double* dQbh = (double*)calloc((size_t)(BH * M * D), sizeof(double));
 #pragma omp parallel for schedule(dynamic, 1)
   for (int64_t bh = 0; bh < BH; ++bh) {
     int64_t h = bh % H;
+    const int64_t Nb = seq_len(lens, bh / H, N);   /* tokens n >= Nb are padding */
     const double* q = Q + h * M * D;
     const double* k = K + bh * N * D;
     const double* v = V + bh * N * D;
@@ -331,21 +360,21 @@ static void encode_bwd_add(const double* Q, const double* K, const double* V,
     double* P = (double*)malloc((size_t)N * sizeof(double));
     for (int64_t m = 0; m < M; ++m) {
       double mu = -INFINITY;
-      for (int64_t n = 0; n < N; ++n) {
+      for (int64_t n = 0; n < Nb; ++n) {
         P[n] = scale * dotd(q + m * D, k + n * D, D);
         if (P[n] > mu) mu = P[n];
       }
       double den = 0.0;
-      for (int64_t n = 0; n < N; ++n) {
+      for (int64_t n = 0; n < Nb; ++n) {
         P[n] = exp(P[n] - mu);
         den += P[n];
       }
       double delta = 0.0;
-      for (int64_t n = 0; n < N; ++n) {
+      for (int64_t n = 0; n < Nb; ++n) {
         P[n] /= den;
         delta += P[n] * dotd(dz + m * D, v + n * D, D);
       }
-      for (int64_t n = 0; n < N; ++n) {
+      for (int64_t n = 0; n < Nb; ++n) {
         double dA = P[n] * (dotd(dz + m * D, v + n * D, D) - delta);
         for (int64_t d = 0; d < D; ++d) {
           dv[n * D + d] += P[n] * dz[m * D + d];
@@ -364,13 +393,13 @@ static void encode_bwd_add(const double* Q, const double* K, const double* V,
 /* The encode's gradient alone (outputs overwritten): dQ [H,M,D] summed over
  * the batch, dK, dV [B,H,N,D]. */
 void oracle_encode_bwd(const double* Q, const double* K, const double* V,
-                       const double* dZ1, int64_t B, int64_t H, int64_t N,
-                       int64_t M, int64_t D, double scale, double* dQ,
-                       double* dK, double* dV) {
+                       const double* dZ1, const int32_t* lens, int64_t B,
+                       int64_t H, int64_t N, int64_t M, int64_t D,
+                       double scale, double* dQ, double* dK, double* dV) {
   memset(dQ, 0, (size_t)(H * M * D) * sizeof(double));
   memset(dK, 0, (size_t)(B * H * N * D) * sizeof(double));
   memset(dV, 0, (size_t)(B * H * N * D) * sizeof(double));
-  encode_bwd_add(Q, K, V, dZ1, B, H, N, M, D, scale, dQ, dK, dV);
+  encode_bwd_add(Q, K, V, dZ1, lens, B, H, N, M, D, scale, dQ, dK, dV);
 }
 
 /*
@@ -382,21 +411,21 @@ void oracle_encode_bwd(const double* Q, const double* K, const double* V,
  * encode's gradient with upstream dZ1 = dQ_dyn), which also adds to dK, dV.
  */
 void oracle_flare_pp_bwd(const double* Q, const double* K, const double* V,
-                         const double* dY, int64_t B, int64_t H, int64_t N,
-                         int64_t M, int64_t D, double scale, double* dQ,
-                         double* dK, double* dV) {
+                         const double* dY, const int32_t* lens, int64_t B,
+                         int64_t H, int64_t N, int64_t M, int64_t D,
+                         double scale, double* dQ, double* dK, double* dV) {
   int64_t per_b = H * M * D;
   double* Z1 = (double*)malloc((size_t)(B * per_b) * sizeof(double));
   double* Qdyn = (double*)malloc((size_t)(B * per_b) * sizeof(double));
   double* dQd = (double*)malloc((size_t)(B * per_b) * sizeof(double));
-  oracle_encode(Q, 0, K, V, B, H, N, M, D, scale, Z1, NULL);
+  oracle_encode(Q, 0, K, V, lens, B, H, N, M, D, scale, Z1, NULL);
   for (int64_t b = 0; b < B; ++b)
     for (int64_t i = 0; i < per_b; ++i) Qdyn[b * per_b + i] = Q[i] + Z1[b * per_b + i];
-  oracle_flare_bwd(Qdyn, per_b, K, V, dY, B, H, N, M, D, scale, dQd, dK, dV);
+  oracle_flare_bwd(Qdyn, per_b, K, V, dY, lens, B, H, N, M, D, scale, dQd, dK, dV);
   memset(dQ, 0, (size_t)per_b * sizeof(double));
   for (int64_t b = 0; b < B; ++b)
     for (int64_t i = 0; i < per_b; ++i) dQ[i] += dQd[b * per_b + i];
-  encode_bwd_add(Q, K, V, dQd, B, H, N, M, D, scale, dQ, dK, dV);
+  encode_bwd_add(Q, K, V, dQd, lens, B, H, N, M, D, scale, dQ, dK, dV);
   free(Z1);
   free(Qdyn);
   free(dQd);

@@ -405,3 +405,122 @@ def test_encode_bwd_is_the_part_of_the_flare_pp_gradient_through_z1():
     np.testing.assert_allclose(dK, dKa + dKe, rtol=1e-11, atol=1e-13)
     np.testing.assert_allclose(dV, dVa + dVe, rtol=1e-11, atol=1e-13)
     np.testing.assert_allclose(dQ, dQd.sum(0) + dQe, rtol=1e-11, atol=1e-13)
+
+
+# -------------------------------------------- sequence lengths (padding) ---
+
+def _trunc(x, b, L):
+    return {k: (v[b:b + 1, :, :L] if k in ("K", "V", "dY") else v) for k, v in x.items()}
+
+
+def test_varlen_equals_each_sequence_alone():
+    # seq_lens = [N, 7, 1, 0]: every batch element's outputs must equal the
+    # unmasked oracle on its first L_b tokens alone (already pinned above);
+    # padding rows of Y, dK, dV are zero; shared dQ is the sum over b.
+    B, H, N, M, D = 4, 2, 30, 6, 4
+    lens = [N, 7, 1, 0]
+    x = _x(B, H, N, M, D, seed=31, with_dy=True)
+    s = 0.6
+    Y, Z, lse = oracle.flare_fwd(x["Q"], x["K"], x["V"], s, seq_lens=lens)
+    dQ, dK, dV = oracle.flare_bwd(x["Q"], x["K"], x["V"], x["dY"], s, seq_lens=lens)
+    Ypp, Qd, Zpp, _ = oracle.flare_pp_fwd(x["Q"], x["K"], x["V"], s, seq_lens=lens)
+    pQ, pK, pV = oracle.flare_pp_bwd(x["Q"], x["K"], x["V"], x["dY"], s, seq_lens=lens)
+    dQsum = np.zeros_like(dQ)
+    pQsum = np.zeros_like(pQ)
+    for b, L in enumerate(lens):
+        assert not Y[b, :, L:].any() and not dK[b, :, L:].any() and not dV[b, :, L:].any()
+        assert not Ypp[b, :, L:].any() and not pK[b, :, L:].any() and not pV[b, :, L:].any()
+        if L == 0:
+            assert not Z[b].any() and np.all(lse[b] == -np.inf)
+            np.testing.assert_array_equal(Qd[b], x["Q"])      # Z1 = 0
+            continue
+        t = _trunc(x, b, L)
+        Yt, Zt, lt = oracle.flare_fwd(t["Q"], t["K"], t["V"], s)
+        np.testing.assert_allclose(Y[b:b + 1, :, :L], Yt, rtol=0, atol=1e-14)
+        np.testing.assert_allclose(Z[b:b + 1], Zt, rtol=0, atol=1e-14)
+        np.testing.assert_allclose(lse[b:b + 1], lt, rtol=0, atol=1e-13)
+        tQ, tK, tV = oracle.flare_bwd(t["Q"], t["K"], t["V"], t["dY"], s)
+        np.testing.assert_allclose(dK[b:b + 1, :, :L], tK, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(dV[b:b + 1, :, :L], tV, rtol=0, atol=1e-13)
+        dQsum += tQ
+        Yt, Qdt, _, _ = oracle.flare_pp_fwd(t["Q"], t["K"], t["V"], s)
+        np.testing.assert_allclose(Ypp[b:b + 1, :, :L], Yt, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(Qd[b:b + 1], Qdt, rtol=0, atol=1e-14)
+        tQ, tK, tV = oracle.flare_pp_bwd(t["Q"], t["K"], t["V"], t["dY"], s)
+        np.testing.assert_allclose(pK[b:b + 1, :, :L], tK, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(pV[b:b + 1, :, :L], tV, rtol=0, atol=1e-12)
+        pQsum += tQ
+    np.testing.assert_allclose(dQ, dQsum, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(pQ, pQsum, rtol=0, atol=1e-12)
+
+
+def test_varlen_sdpa_key_mask_crosscheck():
+    # torch float64 SDPA with a boolean key-padding mask for the encode, the
+    # decode's SDPA per token, padded outputs multiplied by zero; autograd of
+    # that composition for the gradient.
+    B, H, N, M, D = 3, 2, 40, 8, 4
+    lens = [40, 13, 1]
+    x = _x(B, H, N, M, D, seed=32, with_dy=True)
+    s = 0.45
+    Y, Z, _ = oracle.flare_fwd(x["Q"], x["K"], x["V"], s, seq_lens=lens)
+    dQ, dK, dV = oracle.flare_bwd(x["Q"], x["K"], x["V"], x["dY"], s, seq_lens=lens)
+    t = {k: torch.from_numpy(v.copy()).requires_grad_(k != "dY") for k, v in x.items()}
+    keep = torch.arange(N)[None, :] < torch.tensor(lens)[:, None]          # [B, N]
+    Qb = t["Q"].unsqueeze(0).expand(B, -1, -1, -1)
+    Zt = F.scaled_dot_product_attention(Qb, t["K"], t["V"], attn_mask=keep[:, None, None, :],
+                                        scale=s)
+    Yt = F.scaled_dot_product_attention(t["K"], Qb, Zt, scale=s) * keep[:, None, :, None]
+    np.testing.assert_allclose(Y, Yt.detach().numpy(), rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(Z, Zt.detach().numpy(), rtol=1e-11, atol=1e-13)
+    (Yt * t["dY"]).sum().backward()
+    np.testing.assert_allclose(dQ, t["Q"].grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dK, t["K"].grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dV, t["V"].grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_varlen_padding_is_never_read():
+    # NaN in every padded K, V, dY element changes nothing.
+    B, H, N, M, D = 2, 2, 25, 8, 4
+    lens = [9, 25]
+    x = _x(B, H, N, M, D, seed=33, with_dy=True)
+    y = {k: v.copy() for k, v in x.items()}
+    for k in ("K", "V", "dY"):
+        y[k][0, :, 9:] = np.nan
+    s = 0.5
+    for f in (oracle.flare_fwd, oracle.flare_pp_fwd):
+        for a, b in zip(f(x["Q"], x["K"], x["V"], s, seq_lens=lens),
+                        f(y["Q"], y["K"], y["V"], s, seq_lens=lens)):
+            np.testing.assert_array_equal(a, b)
+    for f in (oracle.flare_bwd, oracle.flare_pp_bwd):
+        for a, b in zip(f(x["Q"], x["K"], x["V"], x["dY"], s, seq_lens=lens),
+                        f(y["Q"], y["K"], y["V"], y["dY"], s, seq_lens=lens)):
+            np.testing.assert_array_equal(a, b)
+
+
+def test_varlen_gradient_central_finite_differences():
+    B, H, N, M, D = 2, 1, 12, 3, 4
+    lens = [5, 12]
+    x = _x(B, H, N, M, D, seed=34, with_dy=True)
+    s = 0.8
+    for fwd, bwd in ((oracle.flare_fwd, oracle.flare_bwd),
+                     (oracle.flare_pp_fwd, oracle.flare_pp_bwd)):
+        grads = dict(zip(("Q", "K", "V"), bwd(x["Q"], x["K"], x["V"], x["dY"], s,
+                                              seq_lens=lens)))
+
+        def loss():
+            return float((fwd(x["Q"], x["K"], x["V"], s, seq_lens=lens)[0] * x["dY"]).sum())
+
+        eps = 1e-5
+        for name in ("Q", "K", "V"):
+            flat = x[name].reshape(-1)
+            fd = np.empty(flat.size)
+            for i in range(flat.size):
+                old = flat[i]
+                flat[i] = old + eps
+                lp = loss()
+                flat[i] = old - eps
+                lm = loss()
+                flat[i] = old
+                fd[i] = (lp - lm) / (2 * eps)
+            g = grads[name].reshape(-1)
+            assert np.abs(g - fd).max() <= 1e-7 * max(np.abs(fd).max(), 1.0), name
