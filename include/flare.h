@@ -18,7 +18,7 @@
  *
  * Conventions shared by every entry point
  *   - Every tensor pointer is a DEVICE pointer to contiguous row-major data
- *     (token tensors may instead be strided: the *_strided calls), 16-byte
+ *     (token tensors may instead be strided: the *_ex calls), 16-byte
  *     aligned.  Shapes:
  *       Q        [H,M,D] when q_batch_stride == 0 (learned latents shared by
  *                the batch) or [B,H,M,D] when q_batch_stride == H*M*D;
@@ -88,8 +88,8 @@ typedef enum {
  * [B,H,N,D] whose head dimension D is contiguous: element (b, h, n, d) sits
  * at element offset b*b_stride + h*h_stride + n*n_stride + d from the base
  * pointer.  Contiguous [B,H,N,D] is {H*N*D, N*D, D}; the layout of a fused
- * projection's output [B,N,H,D] is {N*H*D, D, H*D}.  Used by the *_strided
- * entry points.  Every stride must be >= 1, a multiple of 16 bytes and
+ * projection's output [B,N,H,D] is {N*H*D, D, H*D}.  Used by the *_ex entry
+ * points.  Every stride must be >= 1, a multiple of 16 bytes and
  * below 2^40 bytes (else FLARE_ERR_INVALID_ARG, or FLARE_ERR_UNSUPPORTED for
  * a stride that is not a multiple of 16 bytes).  The rows of an output
  * tensor must not overlap (checked: in order of stride, each dimension with
@@ -184,46 +184,57 @@ FLARE_API flare_status_t flare_pp_bwd(const void* Q, const void* K, const void* 
                             void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * The four entry points above with token tensors in any layout that
- * flare_strides_t describes (for example [B,N,H,D] straight from a fused
- * QKV projection, with no transpose).  `strides` points to one
- * flare_strides_t per token tensor, in this order:
- *   flare_fwd_strided, flare_pp_fwd_strided:  K, V, Y;
- *   flare_bwd_strided, flare_pp_bwd_strided:  K, V, dY, dK, dV.
- * NULL means every token tensor is contiguous [B,H,N,D] (the plain entry
- * points are these calls with NULL).  Latent tensors (Q, Q_dyn, dQ, Z_save,
- * lse_save) stay contiguous.  Results are identical to the plain calls on
- * the same values; outputs must not alias inputs.
+ * The four entry points above, extended:
+ *
+ * `strides` -- token tensors in any layout that flare_strides_t describes
+ * (for example [B,N,H,D] straight from a fused QKV projection, with no
+ * transpose).  It points to one flare_strides_t per token tensor, in this
+ * order:  *_fwd_ex: K, V, Y;   *_bwd_ex: K, V, dY, dK, dV.  NULL means
+ * every token tensor is contiguous [B,H,N,D].  Latent tensors (Q, Q_dyn,
+ * dQ, Z_save, lse_save) stay contiguous; outputs must not alias inputs.
+ *
+ * `seq_lens` -- variable sequence lengths (a key-padding mask for
+ * right-padded batches; the FLARE skill page's module takes an attention
+ * mask): a DEVICE array of B int32 values, 4-byte aligned.  Batch element b
+ * has seq_lens[b] valid tokens; tokens n >= seq_lens[b] are padding, whose
+ * values are never read.  The encode's softmax runs over the valid tokens
+ * only; Y is 0 at padding; dK and dV are 0 at padding and padding adds
+ * nothing to dQ.  A sequence with no tokens encodes to Z = 0 with
+ * lse = -inf (Z_save, lse_save), Y = 0.  Values outside [0, N] are clamped
+ * to it and reported: flare_device_status then returns
+ * FLARE_ERR_INVALID_ARG with detail 0x601.  NULL means every sequence has
+ * N tokens.  flare_pp_bwd_ex / flare_bwd_ex must get the lengths their
+ * forward used.
+ *
+ * With strides == NULL and seq_lens == NULL each call is the plain entry
+ * point (which is implemented that way).
  */
-FLARE_API flare_status_t flare_fwd_strided(const void* Q, int64_t q_batch_stride, const void* K,
-                                           const void* V, void* Y,
-                                           const flare_strides_t* strides, int64_t B, int64_t H,
-                                           int64_t N, int64_t M, int64_t D, flare_dtype_t dtype,
-                                           float scale, float* Z_save, float* lse_save,
-                                           void* workspace, size_t workspace_bytes,
-                                           void* stream);
-FLARE_API flare_status_t flare_pp_fwd_strided(const void* Q, const void* K, const void* V,
-                                              void* Y, void* Q_dyn_out,
-                                              const flare_strides_t* strides, int64_t B,
-                                              int64_t H, int64_t N, int64_t M, int64_t D,
-                                              flare_dtype_t dtype, float scale, float* Z_save,
-                                              float* lse_save, void* workspace,
-                                              size_t workspace_bytes, void* stream);
-FLARE_API flare_status_t flare_bwd_strided(const void* Q, int64_t q_batch_stride, const void* K,
-                                           const void* V, const void* dY, const float* Z_save,
-                                           const float* lse_save, void* dQ, void* dK, void* dV,
-                                           const flare_strides_t* strides, int64_t B, int64_t H,
-                                           int64_t N, int64_t M, int64_t D, flare_dtype_t dtype,
-                                           float scale, void* workspace, size_t workspace_bytes,
-                                           void* stream);
-FLARE_API flare_status_t flare_pp_bwd_strided(const void* Q, const void* K, const void* V,
-                                              const void* dY, const void* Q_dyn,
-                                              const float* Z_save, const float* lse_save,
-                                              void* dQ, void* dK, void* dV,
-                                              const flare_strides_t* strides, int64_t B,
-                                              int64_t H, int64_t N, int64_t M, int64_t D,
-                                              flare_dtype_t dtype, float scale, void* workspace,
-                                              size_t workspace_bytes, void* stream);
+FLARE_API flare_status_t flare_fwd_ex(const void* Q, int64_t q_batch_stride, const void* K,
+                                      const void* V, void* Y, const flare_strides_t* strides,
+                                      const int32_t* seq_lens, int64_t B, int64_t H, int64_t N,
+                                      int64_t M, int64_t D, flare_dtype_t dtype, float scale,
+                                      float* Z_save, float* lse_save, void* workspace,
+                                      size_t workspace_bytes, void* stream);
+FLARE_API flare_status_t flare_pp_fwd_ex(const void* Q, const void* K, const void* V, void* Y,
+                                         void* Q_dyn_out, const flare_strides_t* strides,
+                                         const int32_t* seq_lens, int64_t B, int64_t H,
+                                         int64_t N, int64_t M, int64_t D, flare_dtype_t dtype,
+                                         float scale, float* Z_save, float* lse_save,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+FLARE_API flare_status_t flare_bwd_ex(const void* Q, int64_t q_batch_stride, const void* K,
+                                      const void* V, const void* dY, const float* Z_save,
+                                      const float* lse_save, void* dQ, void* dK, void* dV,
+                                      const flare_strides_t* strides, const int32_t* seq_lens,
+                                      int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
+                                      flare_dtype_t dtype, float scale, void* workspace,
+                                      size_t workspace_bytes, void* stream);
+FLARE_API flare_status_t flare_pp_bwd_ex(const void* Q, const void* K, const void* V,
+                                         const void* dY, const void* Q_dyn, const float* Z_save,
+                                         const float* lse_save, void* dQ, void* dK, void* dV,
+                                         const flare_strides_t* strides, const int32_t* seq_lens,
+                                         int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
+                                         flare_dtype_t dtype, float scale, void* workspace,
+                                         size_t workspace_bytes, void* stream);
 
 /*
  * Stage 1 of the forward -- encode partials.  For each (b, h) and each
@@ -292,8 +303,9 @@ FLARE_API flare_status_t flare_fwd_noalloc(const void* Q, int64_t q_batch_stride
 /*
  * Reads and clears the device error word in the workspace header.  This
  * call SYNCHRONISES `stream`.  Returns FLARE_OK, FLARE_ERR_DEVICE_TIMEOUT
- * (a bounded wait ran out; *detail receives the site code) or
- * FLARE_ERR_CUDA.  detail may be NULL.
+ * (a bounded wait ran out; *detail receives the site code),
+ * FLARE_ERR_INVALID_ARG (a seq_lens value outside [0, N] was clamped;
+ * detail 0x601) or FLARE_ERR_CUDA.  detail may be NULL.
  */
 FLARE_API flare_status_t flare_device_status(void* workspace, size_t workspace_bytes, uint32_t* detail,
                                    void* stream);

@@ -61,13 +61,13 @@ SIGNATURES = {
                          _i64, _i64, _i32, _f32, _vp, _sz, _vp]),
     "flare_pp_bwd": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
                             _i64, _i64, _i32, _f32, _vp, _sz, _vp]),
-    "flare_fwd_strided": (_i32, [_vp, _i64, _vp, _vp, _vp, _stp, _i64, _i64, _i64, _i64, _i64,
+    "flare_fwd_ex": (_i32, [_vp, _i64, _vp, _vp, _vp, _stp, _vp, _i64, _i64, _i64, _i64, _i64,
                                  _i32, _f32, _vp, _vp, _vp, _sz, _vp]),
-    "flare_pp_fwd_strided": (_i32, [_vp, _vp, _vp, _vp, _vp, _stp, _i64, _i64, _i64, _i64, _i64,
+    "flare_pp_fwd_ex": (_i32, [_vp, _vp, _vp, _vp, _vp, _stp, _vp, _i64, _i64, _i64, _i64, _i64,
                                     _i32, _f32, _vp, _vp, _vp, _sz, _vp]),
-    "flare_bwd_strided": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _stp, _i64,
+    "flare_bwd_ex": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _stp, _vp, _i64,
                                  _i64, _i64, _i64, _i64, _i32, _f32, _vp, _sz, _vp]),
-    "flare_pp_bwd_strided": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _stp, _i64,
+    "flare_pp_bwd_ex": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _stp, _vp, _i64,
                                     _i64, _i64, _i64, _i64, _i32, _f32, _vp, _sz, _vp]),
     "flare_encode": (_i32, [_vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i32, _f32, _vp,
                             _sz, _vp]),

@@ -119,6 +119,10 @@ flare_status_t apply_strides(const flare_strides_t* st, Tok Dims::* const* which
   return FLARE_OK;
 }
 
+flare_status_t check_opt_lens(const int32_t* lens) {
+  return (lens == nullptr || ((uintptr_t)lens & 3u) == 0) ? FLARE_OK : FLARE_ERR_INVALID_ARG;
+}
+
 flare_status_t check_ws(const void* ws, size_t bytes, size_t need) {
   if (ws == nullptr || ((uintptr_t)ws & 255u) != 0) return FLARE_ERR_WORKSPACE;
   return bytes >= need ? FLARE_OK : FLARE_ERR_WORKSPACE;
@@ -267,8 +271,9 @@ flare_status_t flare_decode(const void* Q, int64_t qbs, const void* K, void* Y, 
                     (cudaStream_t)stream, sms);
 }
 
-flare_status_t flare_fwd_strided(const void* Q, int64_t qbs, const void* K, const void* V,
-                                 void* Y, const flare_strides_t* strides, int64_t B, int64_t H,
+flare_status_t flare_fwd_ex(const void* Q, int64_t qbs, const void* K, const void* V,
+                                 void* Y, const flare_strides_t* strides,
+                                 const int32_t* seq_lens, int64_t B, int64_t H,
                                  int64_t N, int64_t M, int64_t D, flare_dtype_t dt, float scale,
                                  float* Z_save, float* lse_save, void* workspace,
                                  size_t workspace_bytes, void* stream) {
@@ -284,18 +289,24 @@ flare_status_t flare_fwd_strided(const void* Q, int64_t qbs, const void* K, cons
   const int sms = current_sm_count();
   const WsLayout L = ws_layout(FLARE_OP_FWD, B, H, N, M, D, dt, sms);
   FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  FLARE_TRY(check_opt_lens(seq_lens));
   Dims d{B, H, N, M, D};
   FLARE_TRY(apply_strides(strides, kFwdTensors, 3, 1, dt, &d));
+  d.lens = seq_lens;
   char* ws = (char*)workspace;
   cudaStream_t st = (cudaStream_t)stream;
   FLARE_TRY(reset_error_word(ws, st));
+  FLARE_CUDA(launch_check_lens(d, (uint32_t*)(ws + L.hdr), st));
   FLARE_TRY(run_encode(Q, qbs, K, V, d, dt, scale, L, ws, st));
   FLARE_TRY(run_combine(d, dt, Z_save, lse_save, nullptr, nullptr, L, ws, st));
-  return run_decode(Q, qbs, K, Y, d, dt, scale, L, ws, st, sms);
+  FLARE_TRY(run_decode(Q, qbs, K, Y, d, dt, scale, L, ws, st, sms));
+  FLARE_CUDA(launch_zero_padding(Y, d.y, d, dt, st));   // Y = 0 at padding
+  return FLARE_OK;
 }
 
-flare_status_t flare_pp_fwd_strided(const void* Q, const void* K, const void* V, void* Y,
-                                    void* Q_dyn_out, const flare_strides_t* strides, int64_t B,
+flare_status_t flare_pp_fwd_ex(const void* Q, const void* K, const void* V, void* Y,
+                                    void* Q_dyn_out, const flare_strides_t* strides,
+                                 const int32_t* seq_lens, int64_t B,
                                     int64_t H, int64_t N, int64_t M, int64_t D, flare_dtype_t dt,
                                     float scale, float* Z_save, float* lse_save, void* workspace,
                                     size_t workspace_bytes, void* stream) {
@@ -311,25 +322,31 @@ flare_status_t flare_pp_fwd_strided(const void* Q, const void* K, const void* V,
   const int sms = current_sm_count();
   const WsLayout L = ws_layout(FLARE_OP_PP_FWD, B, H, N, M, D, dt, sms);
   FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  FLARE_TRY(check_opt_lens(seq_lens));
   Dims d{B, H, N, M, D};
   FLARE_TRY(apply_strides(strides, kFwdTensors, 3, 1, dt, &d));
+  d.lens = seq_lens;
   char* ws = (char*)workspace;
   cudaStream_t st = (cudaStream_t)stream;
   void* qdyn = Q_dyn_out ? Q_dyn_out : (void*)(ws + L.qdyn);
   const int64_t qdyn_bs = H * M * D;
   FLARE_TRY(reset_error_word(ws, st));
+  FLARE_CUDA(launch_check_lens(d, (uint32_t*)(ws + L.hdr), st));
   // Z1 = encode(Q, K, V); Q_dyn = Q + Z1 (written by the combine)
   FLARE_TRY(run_encode(Q, 0, K, V, d, dt, scale, L, ws, st));
   FLARE_TRY(run_combine(d, dt, nullptr, nullptr, Q, qdyn, L, ws, st));
   // Z = encode(Q_dyn, K, V); Y = decode(Q_dyn, K, Z)
   FLARE_TRY(run_encode(qdyn, qdyn_bs, K, V, d, dt, scale, L, ws, st));
   FLARE_TRY(run_combine(d, dt, Z_save, lse_save, nullptr, nullptr, L, ws, st));
-  return run_decode(qdyn, qdyn_bs, K, Y, d, dt, scale, L, ws, st, sms);
+  FLARE_TRY(run_decode(qdyn, qdyn_bs, K, Y, d, dt, scale, L, ws, st, sms));
+  FLARE_CUDA(launch_zero_padding(Y, d.y, d, dt, st));   // Y = 0 at padding
+  return FLARE_OK;
 }
 
-flare_status_t flare_bwd_strided(const void* Q, int64_t qbs, const void* K, const void* V,
+flare_status_t flare_bwd_ex(const void* Q, int64_t qbs, const void* K, const void* V,
                                  const void* dY, const float* Z_save, const float* lse_save,
                                  void* dQ, void* dK, void* dV, const flare_strides_t* strides,
+                                 const int32_t* seq_lens,
                                  int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
                                  flare_dtype_t dt, float scale, void* workspace,
                                  size_t workspace_bytes, void* stream) {
@@ -347,18 +364,24 @@ flare_status_t flare_bwd_strided(const void* Q, int64_t qbs, const void* K, cons
   FLARE_TRY(check_qbs(qbs, H, M, D));
   const WsLayout L = ws_layout(FLARE_OP_BWD, B, H, N, M, D, dt, current_sm_count());
   FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  FLARE_TRY(check_opt_lens(seq_lens));
   Dims d{B, H, N, M, D};
   FLARE_TRY(apply_strides(strides, kBwdTensors, 5, 2, dt, &d));
+  d.lens = seq_lens;
   char* ws = (char*)workspace;
   cudaStream_t st = (cudaStream_t)stream;
   FLARE_TRY(reset_error_word(ws, st));
+  FLARE_CUDA(launch_check_lens(d, (uint32_t*)(ws + L.hdr), st));
   FLARE_CUDA(launch_bwd(Q, qbs, K, V, dY, Z_save, lse_save, dQ, dK, dV, d, dt, scale, L, ws, st));
+  FLARE_CUDA(launch_zero_padding(dK, d.dk, d, dt, st));   // no gradient at padding
+  FLARE_CUDA(launch_zero_padding(dV, d.dv, d, dt, st));
   return FLARE_OK;
 }
 
-flare_status_t flare_pp_bwd_strided(const void* Q, const void* K, const void* V, const void* dY,
+flare_status_t flare_pp_bwd_ex(const void* Q, const void* K, const void* V, const void* dY,
                                     const void* Q_dyn, const float* Z_save, const float* lse_save,
                                     void* dQ, void* dK, void* dV, const flare_strides_t* strides,
+                                 const int32_t* seq_lens,
                                     int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
                                     flare_dtype_t dt, float scale, void* workspace,
                                     size_t workspace_bytes, void* stream) {
@@ -376,13 +399,16 @@ flare_status_t flare_pp_bwd_strided(const void* Q, const void* K, const void* V,
   FLARE_TRY(check_ptr(dV));
   const WsLayout L = ws_layout(FLARE_OP_PP_BWD, B, H, N, M, D, dt, current_sm_count());
   FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  FLARE_TRY(check_opt_lens(seq_lens));
   Dims d{B, H, N, M, D};
   FLARE_TRY(apply_strides(strides, kBwdTensors, 5, 2, dt, &d));
+  d.lens = seq_lens;
   char* ws = (char*)workspace;
   cudaStream_t st = (cudaStream_t)stream;
   float* z1 = (float*)(ws + L.z1);
   float* lse1 = (float*)(ws + L.lse1);
   FLARE_TRY(reset_error_word(ws, st));
+  FLARE_CUDA(launch_check_lens(d, (uint32_t*)(ws + L.hdr), st));
   // the first encode, recomputed: Z1 and its lse
   FLARE_TRY(run_encode(Q, 0, K, V, d, dt, scale, L, ws, st));
   FLARE_TRY(run_combine(d, dt, z1, lse1, nullptr, nullptr, L, ws, st));
@@ -391,6 +417,8 @@ flare_status_t flare_pp_bwd_strided(const void* Q, const void* K, const void* V,
                         scale, L, ws, st));
   // the first encode's gradient with upstream dQ_dyn, and dQ
   FLARE_CUDA(launch_pp_bwd_tail(Q, K, V, z1, lse1, ws + L.dqd, dQ, dK, dV, d, dt, scale, L, ws, st));
+  FLARE_CUDA(launch_zero_padding(dK, d.dk, d, dt, st));   // no gradient at padding
+  FLARE_CUDA(launch_zero_padding(dV, d.dv, d, dt, st));
   return FLARE_OK;
 }
 
@@ -398,7 +426,7 @@ flare_status_t flare_fwd(const void* Q, int64_t qbs, const void* K, const void* 
                          int64_t B, int64_t H, int64_t N, int64_t M, int64_t D, flare_dtype_t dt,
                          float scale, float* Z_save, float* lse_save, void* workspace,
                          size_t workspace_bytes, void* stream) {
-  return flare_fwd_strided(Q, qbs, K, V, Y, nullptr, B, H, N, M, D, dt, scale, Z_save, lse_save,
+  return flare_fwd_ex(Q, qbs, K, V, Y, nullptr, nullptr, B, H, N, M, D, dt, scale, Z_save, lse_save,
                            workspace, workspace_bytes, stream);
 }
 
@@ -407,7 +435,7 @@ flare_status_t flare_pp_fwd(const void* Q, const void* K, const void* V, void* Y
                             int64_t D, flare_dtype_t dt, float scale, float* Z_save,
                             float* lse_save, void* workspace, size_t workspace_bytes,
                             void* stream) {
-  return flare_pp_fwd_strided(Q, K, V, Y, Q_dyn_out, nullptr, B, H, N, M, D, dt, scale, Z_save,
+  return flare_pp_fwd_ex(Q, K, V, Y, Q_dyn_out, nullptr, nullptr, B, H, N, M, D, dt, scale, Z_save,
                               lse_save, workspace, workspace_bytes, stream);
 }
 
@@ -416,7 +444,7 @@ flare_status_t flare_bwd(const void* Q, int64_t qbs, const void* K, const void* 
                          void* dK, void* dV, int64_t B, int64_t H, int64_t N, int64_t M,
                          int64_t D, flare_dtype_t dt, float scale, void* workspace,
                          size_t workspace_bytes, void* stream) {
-  return flare_bwd_strided(Q, qbs, K, V, dY, Z_save, lse_save, dQ, dK, dV, nullptr, B, H, N, M,
+  return flare_bwd_ex(Q, qbs, K, V, dY, Z_save, lse_save, dQ, dK, dV, nullptr, nullptr, B, H, N, M,
                            D, dt, scale, workspace, workspace_bytes, stream);
 }
 
@@ -425,7 +453,7 @@ flare_status_t flare_pp_bwd(const void* Q, const void* K, const void* V, const v
                             void* dQ, void* dK, void* dV, int64_t B, int64_t H, int64_t N,
                             int64_t M, int64_t D, flare_dtype_t dt, float scale, void* workspace,
                             size_t workspace_bytes, void* stream) {
-  return flare_pp_bwd_strided(Q, K, V, dY, Q_dyn, Z_save, lse_save, dQ, dK, dV, nullptr, B, H, N,
+  return flare_pp_bwd_ex(Q, K, V, dY, Q_dyn, Z_save, lse_save, dQ, dK, dV, nullptr, nullptr, B, H, N,
                               M, D, dt, scale, workspace, workspace_bytes, stream);
 }
 
@@ -440,7 +468,8 @@ flare_status_t flare_device_status(void* workspace, size_t workspace_bytes, uint
   if (cudaStreamSynchronize(st) != cudaSuccess) return FLARE_ERR_CUDA;
   if (cudaMemsetAsync(workspace, 0, 4, st) != cudaSuccess) return FLARE_ERR_CUDA;
   if (detail) *detail = word;
-  return word == 0 ? FLARE_OK : FLARE_ERR_DEVICE_TIMEOUT;
+  if (word == 0) return FLARE_OK;
+  return word == kErrSeqLen ? FLARE_ERR_INVALID_ARG : FLARE_ERR_DEVICE_TIMEOUT;
 }
 
 }  // extern "C"

@@ -24,9 +24,9 @@ constexpr int kT = kBwdTile;  // tokens per tile (= threads per CTA)
 template <typename T, int D>
 __global__ void __launch_bounds__(kT)
     bwd_decode_kernel(const T* __restrict__ Q, int64_t q_bstride, const T* __restrict__ K,
-                      const T* __restrict__ dY, Tok tk, Tok tdy, const float* __restrict__ Z,
-                      int H, int64_t N, int M, float c, float s, int64_t chunk_tokens,
-                      float* __restrict__ dkf,
+                      const T* __restrict__ dY, Tok tk, Tok tdy, const int32_t* __restrict__ lens,
+                      const float* __restrict__ Z, int H, int64_t N, int M, float c, float s,
+                      int64_t chunk_tokens, float* __restrict__ dkf,
                       float* __restrict__ dq_part, float* __restrict__ dz_part) {
   extern __shared__ float sm[];
   float* qs = sm;                 // [M][D] raw latents
@@ -38,7 +38,8 @@ __global__ void __launch_bounds__(kT)
   float* tdel = tinv + kT;        // [kT] delta_d
   const int chunk = blockIdx.x, chunks = gridDim.x;
   const int64_t bh = blockIdx.y, b = bh / H, h = bh % H;
-  const int64_t n0 = (int64_t)chunk * chunk_tokens, n1 = min(N, n0 + chunk_tokens);
+  const int64_t n0 = (int64_t)chunk * chunk_tokens;
+  const int64_t n1 = min(seq_len(lens, bh / H, N), n0 + chunk_tokens);   // padding: none
   const int64_t kh = tk.head(bh, H), dyh = tdy.head(bh, H);
   for (int i = threadIdx.x; i < M * D; i += blockDim.x) {
     qs[i] = to_f(Q[b * q_bstride + h * (int64_t)M * D + i]);
@@ -169,8 +170,9 @@ __global__ void __launch_bounds__(kT)
     bwd_encode_kernel(const T* __restrict__ Q, int64_t q_bstride, const T* __restrict__ K,
                       const T* __restrict__ V, const float* __restrict__ dkf,
                       const float* __restrict__ lse, const float* __restrict__ dzg,
-                      const float* __restrict__ delta, Tok tk, Tok tv, Tok tdk, Tok tdv, int H,
-                      int64_t N, int M, float c, float s, int64_t chunk_tokens,
+                      const float* __restrict__ delta, Tok tk, Tok tv, Tok tdk, Tok tdv,
+                      const int32_t* __restrict__ lens, int H, int64_t N, int M, float c, float s,
+                      int64_t chunk_tokens,
                       T* __restrict__ dK, T* __restrict__ dV, float* __restrict__ dq_part) {
   extern __shared__ float sm[];
   float* qs = sm;                 // [M][D]
@@ -181,7 +183,8 @@ __global__ void __launch_bounds__(kT)
   float* vs = ks + kT * D;        // [kT][D]
   const int chunk = blockIdx.x, chunks = gridDim.x;
   const int64_t bh = blockIdx.y, b = bh / H, h = bh % H;
-  const int64_t n0 = (int64_t)chunk * chunk_tokens, n1 = min(N, n0 + chunk_tokens);
+  const int64_t n0 = (int64_t)chunk * chunk_tokens;
+  const int64_t n1 = min(seq_len(lens, bh / H, N), n0 + chunk_tokens);   // padding: none
   const int64_t kh = tk.head(bh, H), vh = tv.head(bh, H);
   const int64_t dkh = tdk.head(bh, H), dvh = tdv.head(bh, H);
   for (int i = threadIdx.x; i < M * D; i += blockDim.x) {
@@ -317,7 +320,7 @@ cudaError_t bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, cons
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemA);
   if (e != cudaSuccess) return e;
   bwd_decode_kernel<T, D><<<grid, kT, smemA, st>>>((const T*)Q, qbs, (const T*)K, (const T*)dY, d.k,
-                                                   d.dy, Z, (int)d.H, d.N, M, c, scale,
+                                                   d.dy, d.lens, Z, (int)d.H, d.N, M, c, scale,
                                                    p.chunk_tokens(), dkf, dq_dec, dzp);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
@@ -331,9 +334,9 @@ cudaError_t bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, cons
                            (int)smemB);
   if (e != cudaSuccess) return e;
   bwd_encode_kernel<T, D><<<grid, kT, smemB, st>>>((const T*)Q, qbs, (const T*)K, (const T*)V, dkf,
-                                                   lse, dz, delta, d.k, d.v, d.dk, d.dv, (int)d.H,
-                                                   d.N, M, c, scale, p.chunk_tokens(), (T*)dK,
-                                                   (T*)dV, dq_enc);
+                                                   lse, dz, delta, d.k, d.v, d.dk, d.dv, d.lens,
+                                                   (int)d.H, d.N, M, c, scale, p.chunk_tokens(),
+                                                   (T*)dK, (T*)dV, dq_enc);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
   const bool shared_q = (qbs == 0);
@@ -401,8 +404,8 @@ __global__ void __launch_bounds__(kT)
     pp_encode_bwd_kernel(const T* __restrict__ Q, const T* __restrict__ K,
                          const T* __restrict__ V, const float* __restrict__ lse1,
                          const float* __restrict__ dz1, const float* __restrict__ delta1, Tok tk,
-                         Tok tv, Tok tdk, Tok tdv, int H, int64_t N, int M, float c, float s,
-                         int64_t chunk_tokens,
+                         Tok tv, Tok tdk, Tok tdv, const int32_t* __restrict__ lens, int H,
+                         int64_t N, int M, float c, float s, int64_t chunk_tokens,
                          T* __restrict__ dK, T* __restrict__ dV, float* __restrict__ dq_part) {
   extern __shared__ float sm[];
   float* qs = sm;                 // [M][D]
@@ -413,7 +416,8 @@ __global__ void __launch_bounds__(kT)
   float* vs = ks + kT * D;        // [kT][D]
   const int chunk = blockIdx.x, chunks = gridDim.x;
   const int64_t bh = blockIdx.y, h = bh % H;
-  const int64_t n0 = (int64_t)chunk * chunk_tokens, n1 = min(N, n0 + chunk_tokens);
+  const int64_t n0 = (int64_t)chunk * chunk_tokens;
+  const int64_t n1 = min(seq_len(lens, bh / H, N), n0 + chunk_tokens);   // padding: none
   const int64_t kh = tk.head(bh, H), vh = tv.head(bh, H);
   const int64_t dkh = tdk.head(bh, H), dvh = tdv.head(bh, H);
   for (int i = threadIdx.x; i < M * D; i += blockDim.x) {
@@ -541,8 +545,8 @@ cudaError_t pp_tail_t(const void* Q, const void* K, const void* V, const float* 
   if (e != cudaSuccess) return e;
   dim3 grid(p.chunks, (unsigned)BH);
   pp_encode_bwd_kernel<T, D><<<grid, kT, smem, st>>>(
-      (const T*)Q, (const T*)K, (const T*)V, lse1, dz1, delta1, d.k, d.v, d.dk, d.dv, (int)d.H,
-      d.N, M, scale * kLog2e, scale, p.chunk_tokens(), (T*)dK, (T*)dV, dqe);
+      (const T*)Q, (const T*)K, (const T*)V, lse1, dz1, delta1, d.k, d.v, d.dk, d.dv, d.lens,
+      (int)d.H, d.N, M, scale * kLog2e, scale, p.chunk_tokens(), (T*)dK, (T*)dV, dqe);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   const int64_t per = d.H * M * D;
   pp_dq_kernel<T><<<(unsigned)((per + 255) / 256), 256, 0, st>>>((const T*)dqd, dqe, (int)d.B,

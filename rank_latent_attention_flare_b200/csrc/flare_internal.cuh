@@ -32,6 +32,7 @@ enum ErrorSite : uint32_t {
   kErrBwdBTmaWait = 0x501,
   kErrBwdBMmaWait = 0x502,
   kErrBwdBRowWait = 0x503,
+  kErrSeqLen = 0x601,   // a sequence length outside [0, N] (clamped)
 };
 
 // ------------------------------------------------------------------ planning
@@ -269,8 +270,57 @@ struct Dims {
   int64_t B, H, N, M, D;
   Tok k = contig(), v = contig(), y = contig();     // K, V, the forward's Y
   Tok dy = contig(), dk = contig(), dv = contig();  // dY, dK, dV
+  const int32_t* lens = nullptr;   // device [B]: valid tokens per batch element (NULL: N)
   int64_t BH() const { return B * H; }
   Tok contig() const { return Tok{H * N * D, N * D, D}; }
+};
+
+// Valid tokens of batch element b: lens[b] clamped to [0, N] (N when lens is
+// NULL).  Tokens n >= that count are padding: never read, outputs zero.
+__device__ __forceinline__ int64_t seq_len(const int32_t* __restrict__ lens, int64_t b,
+                                           int64_t N) {
+  if (lens == nullptr) return N;
+  const int64_t L = __ldg(lens + b);
+  return L < 0 ? 0 : (L > N ? N : L);
+}
+
+// Tiles of T tokens over a head with nb valid tokens: tile t starts at t T,
+// except that a partial last tile is right-aligned to end at nb.  It then
+// re-reads rows of the tile before it (or rows before 0, which TMA fills with
+// zeros) instead of rows past nb; a row r of tile t belongs to the tile iff
+// tile_row0(t) + r >= t T.
+__host__ __device__ __forceinline__ int64_t tile_row0(int64_t t, int64_t nb, int T) {
+  const int64_t s = t * T;
+  return (s + T > nb) ? nb - T : s;
+}
+__host__ __device__ __forceinline__ int64_t tiles_of(int64_t nb, int T) { return (nb + T - 1) / T; }
+
+// Token tiles of one head, T tokens each.  Without lengths (VAR false) the
+// head has all N tokens: tile t covers rows [tT, tT + T) and TMA fills the
+// rows past N with zeros.  With lengths it has nb <= N tokens and a partial
+// last tile is right-aligned to end at nb, so no padding row is ever read.
+// Both are compile-time variants: the N-token code is unchanged by lengths.
+template <bool VAR>
+struct HeadTiles {
+  int64_t nb;   // the head's tokens
+  __device__ __forceinline__ HeadTiles(const int32_t* __restrict__ lens, int64_t b, int64_t N)
+      : nb(VAR ? seq_len(lens, b, N) : N) {}
+  __device__ __forceinline__ int64_t count(int T) const { return tiles_of(nb, T); }
+  // token of row 0 of tile t (negative rows read as zeros)
+  __device__ __forceinline__ int64_t row0(int64_t t, int T) const {
+    return VAR ? tile_row0(t, nb, T) : t * T;
+  }
+  // row r of tile t is one of the tile's own tokens
+  __device__ __forceinline__ bool own(int64_t t, int T, int r) const {
+    return VAR ? row0(t, T) + r >= t * T : t * T + r < nb;
+  }
+  // the tile's own tokens are its columns [lo, hi)
+  __device__ __forceinline__ int lo(int64_t t, int T) const {
+    return VAR ? (int)max((t + 1) * T - nb, (int64_t)0) : 0;
+  }
+  __device__ __forceinline__ int hi(int64_t t, int T) const {
+    return VAR ? T : (int)imin64(T, nb - t * T);
+  }
 };
 
 cudaError_t launch_simt_encode(const void* Q, int64_t qbs, const void* K, const void* V,
@@ -280,6 +330,12 @@ cudaError_t launch_simt_encode(const void* Q, int64_t qbs, const void* K, const 
 cudaError_t launch_simt_decode(const void* Q, int64_t qbs, const void* K, const float* Zf,
                                void* Y, const Dims& d, flare_dtype_t dt, float scale,
                                cudaStream_t st);
+// Records kErrSeqLen when a length lies outside [0, N] (lens non-NULL).
+cudaError_t launch_check_lens(const Dims& d, uint32_t* err, cudaStream_t st);
+// Zeroes the padding rows (n >= the batch element's length) of a token
+// tensor with strides t (no-op when d.lens is NULL).
+cudaError_t launch_zero_padding(void* X, const Tok& t, const Dims& d, flare_dtype_t dt,
+                                cudaStream_t st);
 cudaError_t launch_combine(const Dims& d, flare_dtype_t dt, int slots_per_bh,
                            const float* part_ml, const float* part_acc, float* Zf,
                            __nv_bfloat16* Zb, float* Z_save, float* lse_save, const void* Qpp,

@@ -17,8 +17,9 @@ namespace {
 template <typename T, int D>
 __global__ void __launch_bounds__(kSimtEncThreads)
     simt_encode_kernel(const T* __restrict__ Q, int64_t q_bstride, const T* __restrict__ K,
-                       const T* __restrict__ V, Tok tk, Tok tv, int H, int64_t N, int M,
-                       float c, int64_t chunk_tokens, float* __restrict__ part_ml,
+                       const T* __restrict__ V, Tok tk, Tok tv, const int32_t* __restrict__ lens,
+                       int H, int64_t N, int M, float c, int64_t chunk_tokens,
+                       float* __restrict__ part_ml,
                        float* __restrict__ part_acc) {
   __shared__ float ks[kSimtEncTile][D];
   __shared__ float vs[kSimtEncTile][D];
@@ -27,7 +28,7 @@ __global__ void __launch_bounds__(kSimtEncThreads)
   const int64_t bh = blockIdx.y;
   const int64_t b = bh / H, h = bh % H;
   const int64_t n0 = (int64_t)chunk * chunk_tokens;
-  const int64_t n1 = min(N, n0 + chunk_tokens);
+  const int64_t n1 = min(seq_len(lens, b, N), n0 + chunk_tokens);   // empty past the length
   const T* Kb = K + tk.head(bh, H);
   const T* Vb = V + tv.head(bh, H);
   const int m = threadIdx.x;
@@ -96,8 +97,8 @@ __global__ void __launch_bounds__(kSimtEncThreads)
 template <typename T, int D>
 __global__ void __launch_bounds__(kSimtDecThreads)
     simt_decode_kernel(const T* __restrict__ Q, int64_t q_bstride, const T* __restrict__ K,
-                       const float* __restrict__ Zf, T* __restrict__ Y, Tok tk, Tok ty, int H,
-                       int64_t N, int M, float c) {
+                       const float* __restrict__ Zf, T* __restrict__ Y, Tok tk, Tok ty,
+                       const int32_t* __restrict__ lens, int H, int64_t N, int M, float c) {
   extern __shared__ float sm[];
   float* qs = sm;
   float* zs = sm + M * D;
@@ -109,7 +110,7 @@ __global__ void __launch_bounds__(kSimtDecThreads)
   }
   __syncthreads();
   const int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= N) return;
+  if (n >= seq_len(lens, b, N)) return;   // padding rows are zeroed separately
   const T* kr = K + tk.head(bh, H) + n * tk.sn;
   float k[D];
 #pragma unroll
@@ -167,7 +168,7 @@ __global__ void combine_kernel(const float* __restrict__ part_ml,
     if (lane < D) acc = fmaf(f, part_acc[row * D + lane], acc);
   }
   if (lane < D) {
-    const float z = acc / l;
+    const float z = (l > 0.f) ? acc / l : 0.f;   // no tokens: an empty weighted sum
     const int64_t o = w * D + lane;
     Zf[o] = z;
     Zb[o] = __float2bfloat16_rn(z);
@@ -177,7 +178,28 @@ __global__ void combine_kernel(const float* __restrict__ part_ml,
       Qdyn[o] = from_f<T>(to_f(Qpp[(h * M + m) * D + lane]) + z);
     }
   }
-  if (lane == 0 && lse_save) lse_save[w] = (mstar + log2f(l)) * kLn2;
+  if (lane == 0 && lse_save) lse_save[w] = (l > 0.f) ? (mstar + log2f(l)) * kLn2 : -INFINITY;
+}
+
+__global__ void check_lens_kernel(const int32_t* __restrict__ lens, int64_t B, int64_t N,
+                                  uint32_t* __restrict__ err) {
+  const int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B && (lens[b] < 0 || (int64_t)lens[b] > N)) record_error(err, kErrSeqLen);
+}
+
+// One thread per 16 bytes of a padding row: grid.y = b * H + h, x over the
+// row bytes of tokens [L_b, N).
+__global__ void zero_padding_kernel(uint8_t* __restrict__ X, Tok t, int esz,
+                                    const int32_t* __restrict__ lens, int H, int64_t N, int D) {
+  const int64_t bh = blockIdx.y;
+  const int64_t b = bh / H;
+  const int64_t L = seq_len(lens, b, N);
+  const int per_row = D * esz / 16;   // 16-byte pieces per row
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t n = L + i / per_row;
+  if (n >= N) return;
+  uint8_t* row = X + (t.head(bh, H) + n * t.sn) * esz;
+  reinterpret_cast<uint4*>(row)[i % per_row] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 template <typename T, int D>
@@ -186,7 +208,7 @@ cudaError_t simt_encode_t(const void* Q, int64_t qbs, const void* K, const void*
                           float* part_acc, cudaStream_t st) {
   dim3 grid(plan.chunks, (unsigned)d.BH());
   simt_encode_kernel<T, D><<<grid, kSimtEncThreads, 0, st>>>(
-      (const T*)Q, qbs, (const T*)K, (const T*)V, d.k, d.v, (int)d.H, d.N, (int)d.M,
+      (const T*)Q, qbs, (const T*)K, (const T*)V, d.k, d.v, d.lens, (int)d.H, d.N, (int)d.M,
       scale * kLog2e, plan.chunk_tokens(), part_ml, part_acc);
   return cudaPeekAtLastError();
 }
@@ -200,7 +222,7 @@ cudaError_t simt_decode_t(const void* Q, int64_t qbs, const void* K, const float
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((d.N + kSimtDecThreads - 1) / kSimtDecThreads), (unsigned)d.BH());
   simt_decode_kernel<T, D><<<grid, kSimtDecThreads, smem, st>>>(
-      (const T*)Q, qbs, (const T*)K, Zf, (T*)Y, d.k, d.y, (int)d.H, d.N, (int)d.M,
+      (const T*)Q, qbs, (const T*)K, Zf, (T*)Y, d.k, d.y, d.lens, (int)d.H, d.N, (int)d.M,
       scale * kLog2e);
   return cudaPeekAtLastError();
 }
@@ -227,6 +249,23 @@ cudaError_t launch_simt_decode(const void* Q, int64_t qbs, const void* K, const 
                      : simt_decode_t<float, 32>(Q, qbs, K, Zf, Y, d, scale, st);
   return d.D == 16 ? simt_decode_t<__nv_bfloat16, 16>(Q, qbs, K, Zf, Y, d, scale, st)
                    : simt_decode_t<__nv_bfloat16, 32>(Q, qbs, K, Zf, Y, d, scale, st);
+}
+
+cudaError_t launch_check_lens(const Dims& d, uint32_t* err, cudaStream_t st) {
+  if (d.lens == nullptr) return cudaSuccess;
+  check_lens_kernel<<<(unsigned)((d.B + 255) / 256), 256, 0, st>>>(d.lens, d.B, d.N, err);
+  return cudaPeekAtLastError();
+}
+
+cudaError_t launch_zero_padding(void* X, const Tok& t, const Dims& d, flare_dtype_t dt,
+                                cudaStream_t st) {
+  if (d.lens == nullptr) return cudaSuccess;
+  const int esz = (dt == FLARE_F32) ? 4 : 2;
+  const int64_t pieces = d.N * d.D * esz / 16;   // at most (16-byte pieces per head)
+  dim3 grid((unsigned)((pieces + 255) / 256), (unsigned)d.BH());
+  zero_padding_kernel<<<grid, 256, 0, st>>>((uint8_t*)X, t, esz, d.lens, (int)d.H, d.N,
+                                            (int)d.D);
+  return cudaPeekAtLastError();
 }
 
 cudaError_t launch_combine(const Dims& d, flare_dtype_t dt, int slots_per_bh,

@@ -109,13 +109,13 @@ struct EncLayout {
   static constexpr int BYTES = MISC_OFF + 16;
 };
 
-template <int D, int M, bool FLAT>
+template <int D, int M, bool FLAT, bool VAR>
 __global__ void __launch_bounds__(kThreads, 2)
     tc_encode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, int H, int64_t N, int q_per_batch,
                      float c, int64_t tiles_per_bh, int64_t chunk_tiles, int slots_per_bh,
                      float* __restrict__ part_ml, float* __restrict__ part_acc,
-                     uint32_t* __restrict__ err) {
+                     const int32_t* __restrict__ lens, uint32_t* __restrict__ err) {
   using L = EncLayout<D, M>;
   constexpr int NH = M / 128;        // latent halves; M=128 -> the two warpgroups split tiles
   constexpr int SUB = (NH == 1) ? 2 : 1;
@@ -143,7 +143,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int64_t bh = blockIdx.y;
   const int64_t h = bh % H;
   const int64_t tile0 = (int64_t)chunk * chunk_tiles;
-  const int64_t ntiles = imin64(chunk_tiles, tiles_per_bh - tile0);
+  // with lengths, tokens past the batch element's length are padding: their tiles are skipped
+  const HeadTiles<VAR> ht(lens, bh / H, N);
+  const int64_t ntiles = VAR ? max(imin64(chunk_tiles, ht.count(kEncTile) - tile0), (int64_t)0)
+                             : imin64(chunk_tiles, tiles_per_bh - tile0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kEncStages; ++s) {
@@ -190,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           if (*abort_flag) break;
           uint8_t* kt = smem + L::KV_OFF + s * 2 * L::TILE;
           mbar_arrive_expect_tx(&kv_full[s], 2 * L::TILE);
-          const int32_t tok = (int32_t)((tile0 + i) * kEncTile);
+          const int32_t tok = (int32_t)ht.row0(tile0 + i, kEncTile);
           tma_load_tok<FLAT>(kt, &tmK, &kv_full[s], tok, bh, H);
           tma_load_tok<FLAT>(kt + L::TILE, &tmV, &kv_full[s], tok, bh, H);
           issued = i + 1;
@@ -301,8 +304,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int j = 0; j < nW; ++j) {
       const int64_t i = first + (int64_t)stride * j;
       const int b = j & 1;
-      const int nvalid = (int)imin64(kEncTile, N - (tile0 + i) * kEncTile);
-      const bool full = (nvalid == kEncTile);   // warp-uniform: only a head's last tile is partial
+      // the tile's own tokens are its columns [lo, hi); the rest get weight 0
+      const int lo = ht.lo(tile0 + i, kEncTile), hi = ht.hi(tile0 + i, kEncTile);
+      const bool full = (lo == 0 && hi == kEncTile);   // warp-uniform: only a head's last tile is partial
       const uint32_t tS = tW + 48 * b;
       if (!warp_all(mbar_wait(&s_full[2 * w + b], (uint32_t)((j >> 1) & 1)) && !*abort_flag)) {
         ok = false;
@@ -326,10 +330,10 @@ __global__ void __launch_bounds__(kThreads, 2)
           uint32_t a[32];
           tmem_ld32(tS, a);
           tmem_wait_ld_dep(a);
-          if (!full) {   // tokens past the end of the head get weight 0
+          if (!full) {   // masked columns get weight 0
 #pragma unroll
             for (int t = 0; t < 32; ++t)
-              if (t >= nvalid) a[t] = __float_as_uint(-INFINITY);
+              if (t < lo || t >= hi) a[t] = __float_as_uint(-INFINITY);
           }
           max_fold32(a, mf);
           exp_pack32<kEncPolyEvery>(a, c, neg, pa, sf);
@@ -341,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           if (!full) {
 #pragma unroll
             for (int t = 0; t < 16; ++t)
-              if (32 + t >= nvalid) a[t] = __float_as_uint(-INFINITY);
+              if (32 + t < lo || 32 + t >= hi) a[t] = __float_as_uint(-INFINITY);
           }
           max_fold16(a, mf);
           exp_pack16(a, c, neg, pb, sf);
@@ -368,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
       if (exact) {
-        // pass 1: exact tile max of the raw logits (masked past the end of the head)
+        // pass 1: exact tile max of the raw logits (masked columns excluded)
         float mf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         {
           uint32_t a[32];
@@ -376,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           tmem_wait_ld_dep(a);
 #pragma unroll
           for (int t = 0; t < 32; ++t)
-            if (t < nvalid) mf[t & 3] = fmaxf(mf[t & 3], __uint_as_float(a[t]));
+            if (t >= lo && t < hi) mf[t & 3] = fmaxf(mf[t & 3], __uint_as_float(a[t]));
         }
         {
           uint32_t a[16];
@@ -384,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           tmem_wait_ld_dep16(a);
 #pragma unroll
           for (int t = 0; t < 16; ++t)
-            if (32 + t < nvalid) mf[t & 3] = fmaxf(mf[t & 3], __uint_as_float(a[t]));
+            if (32 + t >= lo && 32 + t < hi) mf[t & 3] = fmaxf(mf[t & 3], __uint_as_float(a[t]));
         }
         const float mx2 = fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3])) * c;
         float f = 1.f;   // rescale of this row's earlier tiles (1 when the max did not move)
@@ -410,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           if (!full) {
 #pragma unroll
             for (int t = 0; t < 32; ++t)
-              if (t >= nvalid) a[t] = __float_as_uint(-INFINITY);
+              if (t < lo || t >= hi) a[t] = __float_as_uint(-INFINITY);
           }
           uint32_t pk[16];
           exp_pack32<kEncPolyEvery>(a, c, neg, pk, sf);
@@ -423,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           if (!full) {
 #pragma unroll
             for (int t = 0; t < 16; ++t)
-              if (32 + t >= nvalid) a[t] = __float_as_uint(-INFINITY);
+              if (32 + t < lo || 32 + t >= hi) a[t] = __float_as_uint(-INFINITY);
           }
           uint32_t pk[8];
           exp_pack16(a, c, neg, pk, sf);
@@ -494,12 +498,13 @@ struct DecLayout {
   static constexpr int BYTES = MISC_OFF + 16;
 };
 
-template <int D, int M, bool FLAT>
+template <int D, int M, bool FLAT, bool VAR>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmZ, int H, int64_t N, int q_per_batch,
                      float c, int64_t tiles_per_bh, int64_t chunk_tiles,
-                     __nv_bfloat16* __restrict__ Y, Tok ty, uint32_t* __restrict__ err) {
+                     __nv_bfloat16* __restrict__ Y, Tok ty, const int32_t* __restrict__ lens,
+                     uint32_t* __restrict__ err) {
   using L = DecLayout<D, M>;
   constexpr int RB = L::RB;
   constexpr uint32_t SW = umma_swizzle_code(RB);
@@ -529,7 +534,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t h = bh % H;
   const int64_t yhead = ty.head(bh, H);   // row 0 of this head in Y
   const int64_t tile0 = (int64_t)chunk * chunk_tiles;
-  const int64_t ntiles = imin64(chunk_tiles, tiles_per_bh - tile0);
+  // with lengths, tokens past the batch element's length are padding: their tiles are skipped
+  const HeadTiles<VAR> ht(lens, bh / H, N);
+  const int64_t ntiles = VAR ? max(imin64(chunk_tiles, ht.count(kTile) - tile0), (int64_t)0)
+                             : imin64(chunk_tiles, tiles_per_bh - tile0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDecStages; ++s) {
@@ -575,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (*abort_flag) break;
         mbar_arrive_expect_tx(&k_full[s], L::TILE);
         tma_load_tok<FLAT>(smem + L::K_OFF + s * L::TILE, &tmK, &k_full[s],
-                     (int32_t)((tile0 + i) * kTile), bh, H);
+                           (int32_t)ht.row0(tile0 + i, kTile), bh, H);
         issued = i + 1;
       }
       for (int64_t i = (issued > kDecStages ? issued - kDecStages : 0); i < issued; ++i)
@@ -644,7 +652,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int64_t j = 0; j < nW; ++j) {
       const int64_t i = 2 * j + w;
-      const int64_t tok = (tile0 + i) * kTile + r;
+      const int64_t tok = ht.row0(tile0 + i, kTile) + r;
+      const bool mine = ht.own(tile0 + i, kTile, r);
       if (!warp_all(mbar_wait(&s_full[w], (uint32_t)(j & 1)) && !*abort_flag)) {
         ok = false;
         break;
@@ -709,7 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(&s_empty[w]);
-      if (tok < N) {
+      if (mine) {
         const float inv = 1.f / ((sf[0] + sf[1]) + (sf[2] + sf[3]));
         uint4* dst = reinterpret_cast<uint4*>(Y + yhead + tok * ty.sn);
 #pragma unroll
@@ -812,7 +821,7 @@ cudaError_t make_tok_map(CUtensorMap* m, const void* base, const Dims& d, const 
 
 namespace {
 
-template <int D, int M, bool FLAT>
+template <int D, int M, bool FLAT, bool VAR>
 cudaError_t tc_encode_t(const void* Q, int64_t qbs, const void* K, const void* V, const Dims& d,
                         float scale, const ChunkPlan& plan, float* pml, float* pacc,
                         uint32_t* err, cudaStream_t st) {
@@ -824,17 +833,17 @@ cudaError_t tc_encode_t(const void* Q, int64_t qbs, const void* K, const void* V
   if ((e = make_tok_map(&mv, V, d, d.v, kEncTile, FLAT)) != cudaSuccess) return e;
   // two CTAs per SM: their TMEM (2 x 256 columns) fits exactly
   const int smem = EncLayout<D, M>::BYTES + 1024;
-  e = cudaFuncSetAttribute(tc_encode_kernel<D, M, FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(tc_encode_kernel<D, M, FLAT, VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem);
   if (e != cudaSuccess) return e;
   dim3 grid(plan.chunks, (unsigned)d.BH());
-  tc_encode_kernel<D, M, FLAT><<<grid, kThreads, smem, st>>>(
+  tc_encode_kernel<D, M, FLAT, VAR><<<grid, kThreads, smem, st>>>(
       mq, mk, mv, (int)d.H, d.N, q_per_batch, scale * kLog2e, plan.tiles_per_bh,
-      plan.chunk_tiles, plan.slots_per_bh(), pml, pacc, err);
+      plan.chunk_tiles, plan.slots_per_bh(), pml, pacc, d.lens, err);
   return cudaPeekAtLastError();
 }
 
-template <int D, int M, bool FLAT>
+template <int D, int M, bool FLAT, bool VAR>
 cudaError_t tc_decode_t(const void* Q, int64_t qbs, const void* K, const __nv_bfloat16* Zb,
                         void* Y, const Dims& d, float scale, const ChunkPlan& plan, uint32_t* err,
                         cudaStream_t st) {
@@ -846,47 +855,59 @@ cudaError_t tc_decode_t(const void* Q, int64_t qbs, const void* K, const __nv_bf
   if ((e = make_map(&mz, Zb, D, M, d.BH(), M)) != cudaSuccess) return e;
   const int smem = (DecLayout<D, M>::BYTES + 1024 > kMinSmemBytes) ? DecLayout<D, M>::BYTES + 1024
                                                                    : kMinSmemBytes;
-  e = cudaFuncSetAttribute(tc_decode_kernel<D, M, FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(tc_decode_kernel<D, M, FLAT, VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem);
   if (e != cudaSuccess) return e;
   dim3 grid(plan.chunks, (unsigned)d.BH());
-  tc_decode_kernel<D, M, FLAT><<<grid, kThreads, smem, st>>>(mq, mk, mz, (int)d.H, d.N, q_per_batch,
+  tc_decode_kernel<D, M, FLAT, VAR><<<grid, kThreads, smem, st>>>(mq, mk, mz, (int)d.H, d.N, q_per_batch,
                                                        scale * kLog2e, plan.tiles_per_bh,
                                                        plan.chunk_tiles, (__nv_bfloat16*)Y, d.y,
-                                                       err);
+                                                       d.lens, err);
   return cudaPeekAtLastError();
 }
 
 }  // namespace
 
+template <int D, int M>
+cudaError_t tc_encode_dispatch(const void* Q, int64_t qbs, const void* K, const void* V,
+                               const Dims& d, float scale, const ChunkPlan& plan, float* pml,
+                               float* pacc, uint32_t* err, cudaStream_t st) {
+  const bool flat = tok_flat(d), var = d.lens != nullptr;
+  if (flat)
+    return var ? tc_encode_t<D, M, true, true>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st)
+               : tc_encode_t<D, M, true, false>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
+  return var ? tc_encode_t<D, M, false, true>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st)
+             : tc_encode_t<D, M, false, false>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
+}
+
 cudaError_t launch_tc_encode(const void* Q, int64_t qbs, const void* K, const void* V,
                              const Dims& d, float scale, const ChunkPlan& plan, float* pml,
                              float* pacc, uint32_t* err, cudaStream_t st) {
-  const bool flat = tok_flat(d);
-  if (d.D == 32 && d.M == 256)
-    return flat ? tc_encode_t<32, 256, true>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st)
-                : tc_encode_t<32, 256, false>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
-  if (d.D == 32 && d.M == 128)
-    return flat ? tc_encode_t<32, 128, true>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st)
-                : tc_encode_t<32, 128, false>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
-  if (d.D == 16 && d.M == 256)
-    return flat ? tc_encode_t<16, 256, true>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st)
-                : tc_encode_t<16, 256, false>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
-  if (d.D == 16 && d.M == 128)
-    return flat ? tc_encode_t<16, 128, true>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st)
-                : tc_encode_t<16, 128, false>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
+  if (d.D == 32 && d.M == 256) return tc_encode_dispatch<32, 256>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
+  if (d.D == 32 && d.M == 128) return tc_encode_dispatch<32, 128>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
+  if (d.D == 16 && d.M == 256) return tc_encode_dispatch<16, 256>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
+  if (d.D == 16 && d.M == 128) return tc_encode_dispatch<16, 128>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
   return cudaErrorNotSupported;
+}
+
+template <int D, int M>
+cudaError_t tc_decode_dispatch(const void* Q, int64_t qbs, const void* K,
+                               const __nv_bfloat16* Zb, void* Y, const Dims& d, float scale,
+                               const ChunkPlan& plan, uint32_t* err, cudaStream_t st) {
+  // The decode takes 4-D maps for every layout: its 3-D variant measured no
+  // faster and needs more registers.
+  return d.lens != nullptr
+             ? tc_decode_t<D, M, false, true>(Q, qbs, K, Zb, Y, d, scale, plan, err, st)
+             : tc_decode_t<D, M, false, false>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
 }
 
 cudaError_t launch_tc_decode(const void* Q, int64_t qbs, const void* K, const __nv_bfloat16* Zb,
                              void* Y, const Dims& d, float scale, const ChunkPlan& plan,
                              uint32_t* err, cudaStream_t st) {
-  // The decode takes 4-D maps for every layout: its 3-D variant measured no
-  // faster and needs more registers.
-  if (d.D == 32 && d.M == 256) return tc_decode_t<32, 256, false>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
-  if (d.D == 32 && d.M == 128) return tc_decode_t<32, 128, false>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
-  if (d.D == 16 && d.M == 256) return tc_decode_t<16, 256, false>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
-  if (d.D == 16 && d.M == 128) return tc_decode_t<16, 128, false>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
+  if (d.D == 32 && d.M == 256) return tc_decode_dispatch<32, 256>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
+  if (d.D == 32 && d.M == 128) return tc_decode_dispatch<32, 128>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
+  if (d.D == 16 && d.M == 256) return tc_decode_dispatch<16, 256>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
+  if (d.D == 16 && d.M == 128) return tc_decode_dispatch<16, 128>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
   return cudaErrorNotSupported;
 }
 

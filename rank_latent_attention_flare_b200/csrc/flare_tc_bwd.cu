@@ -131,7 +131,7 @@ struct ALayout {
 // tile j + 1 while Y = P [Z | e0] of tile j runs on the tensor cores, and
 // then finishes tile j (delta_d, dY', dY'', statistics).  Each warpgroup has
 // two Y accumulators in TMEM for that overlap.
-template <int D, bool FLAT>
+template <int D, bool FLAT, bool VAR>
 __global__ void __launch_bounds__(kThr, 1)
     tc_bwd_a_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmdY, const __grid_constant__ CUtensorMap tmZ,
@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(kThr, 1)
                     int64_t chunk_tiles, const float* __restrict__ rref,
                     float4* __restrict__ stats, __nv_bfloat16* __restrict__ dy2,
                     uint32_t* __restrict__ flags, float* __restrict__ dz_part,
-                    uint32_t* __restrict__ err) {
+                    const int32_t* __restrict__ lens, uint32_t* __restrict__ err) {
   using L = ALayout<D>;
   constexpr int M = L::M;
   constexpr int RB = L::RB;
@@ -176,7 +176,10 @@ __global__ void __launch_bounds__(kThr, 1)
   const int64_t bh = blockIdx.y;
   const int64_t h = bh % H;
   const int64_t tile0 = (int64_t)chunk * chunk_tiles;
-  const int nt = (int)imin64(chunk_tiles, tiles_per_bh - tile0);
+  // with lengths, tokens past the batch element's length are padding: their tiles are skipped
+  const HeadTiles<VAR> ht(lens, bh / H, N);
+  const int nt = VAR ? (int)max(imin64(chunk_tiles, ht.count(kT) - tile0), (int64_t)0)
+                     : (int)imin64(chunk_tiles, tiles_per_bh - tile0);
 
   // Y = P [Z | e0]: the second N block of the B operand holds a one in
   // column 0 of every latent row (same swizzled layout as the Z rows), so
@@ -249,8 +252,8 @@ __global__ void __launch_bounds__(kThr, 1)
           }
           if (*abort_flag) break;
           mbar_arrive_expect_tx(&full[s], L::TILE);
-          tma_load_tok<FLAT>(ring + s * L::TILE, map, &full[s], (int32_t)((tile0 + i) * kT), bh,
-                             H);
+          tma_load_tok<FLAT>(ring + s * L::TILE, map, &full[s], (int32_t)ht.row0(tile0 + i, kT),
+                             bh, H);
           issued = i + 1;
         }
         // let every load still in flight land before the CTA can exit
@@ -368,7 +371,9 @@ __global__ void __launch_bounds__(kThr, 1)
     auto finish = [&](int j, float mx, float l) -> bool {
       const int i = 2 * j + w;
       const int s = i % DST;
-      const int64_t tok = (tile0 + i) * kT + r;
+      // rows that are not the tile's own tokens add nothing
+      const int64_t tok = ht.row0(tile0 + i, kT) + r;
+      const bool mine = ht.own(tile0 + i, kT, r);
       if (!warp_all(mbar_wait(&y_full[2 * w + (j & 1)], (uint32_t)((j >> 1) & 1)) &&
                     mbar_wait(&d_full[s], (uint32_t)((i / DST) & 1)) && !*abort_flag))
         return false;
@@ -415,19 +420,21 @@ __global__ void __launch_bounds__(kThr, 1)
           dot = fmaf(a0, y0, fmaf(a1, y1, dot));
           w2[jj] = pack_bf16(a0 * ginv, a1 * ginv);           // dY'' = dY / g
           dot2 = fmaf(bf_lo(w2[jj]), y0, fmaf(bf_hi(w2[jj]), y1, dot2));
-          wv[jj] = pack_bf16(a0 * inv, a1 * inv);             // dY' = dY / rowsum
+          // dY' = dY / rowsum (rows past N are zero already; with lengths
+          // a right-aligned tile's earlier rows hold real dY)
+          wv[jj] = (!VAR || mine) ? pack_bf16(a0 * inv, a1 * inv) : 0u;
         }
         *p = make_uint4(wv[0], wv[1], wv[2], wv[3]);
         o2v[ch] = make_uint4(w2[0], w2[1], w2[2], w2[3]);
       }
-      if (tok < N) {
+      if (mine) {
         // delta_d = dY . Y and its counterpart with the rounded dY'' (= delta_d / g)
         stats[bh * N + tok] = make_float4(mxp, dot * inv, dot2 * inv, 0.f);
         uint4* dst = reinterpret_cast<uint4*>(dy2 + (bh * N + tok) * D);
 #pragma unroll
         for (int ch = 0; ch < D / 8; ++ch) dst[ch] = o2v[ch];
       }
-      if (warp_any(bad && tok < N) && lane == 0) atomicOr(flags + bh, 1u);
+      if (warp_any(bad && mine) && lane == 0) atomicOr(flags + bh, 1u);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&a_done[w]);
@@ -672,7 +679,7 @@ struct BLayout {
   static constexpr int BYTES = MISC_OFF + 16;
 };
 
-template <int D, bool FLAT>
+template <int D, bool FLAT, bool VAR>
 __global__ void __launch_bounds__(kThr, 1)
     tc_bwd_b_exact_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdY,
@@ -682,7 +689,7 @@ __global__ void __launch_bounds__(kThr, 1)
                     const float4* __restrict__ stats, const float2* __restrict__ params,
                     const float* __restrict__ lse2, int enc_only, __nv_bfloat16* __restrict__ dK,
                     __nv_bfloat16* __restrict__ dV, Tok tdk, Tok tdv, float* __restrict__ dq_part,
-                    uint32_t* __restrict__ err) {
+                    const int32_t* __restrict__ lens, uint32_t* __restrict__ err) {
   using L = BLayout<D>;
   constexpr int M = L::M;
   constexpr int NQ = L::NQ;
@@ -717,7 +724,10 @@ __global__ void __launch_bounds__(kThr, 1)
   const int64_t h = bh % H;
   const int64_t dk_head = tdk.head(bh, H), dv_head = tdv.head(bh, H);   // row 0 of the head
   const int64_t tile0 = (int64_t)chunk * chunk_tiles;
-  const int64_t ntiles = imin64(chunk_tiles, tiles_per_bh - tile0);
+  // with lengths, tokens past the batch element's length are padding: their tiles are skipped
+  const HeadTiles<VAR> ht(lens, bh / H, N);
+  const int64_t ntiles = VAR ? max(imin64(chunk_tiles, ht.count(kT) - tile0), (int64_t)0)
+                             : imin64(chunk_tiles, tiles_per_bh - tile0);
   const int64_t KQ = ntiles * NQ;   // quarters of this chunk
   if (params[bh].y != 0.f) return;  // head served by tc_bwd_b_fast_kernel
 
@@ -791,7 +801,7 @@ __global__ void __launch_bounds__(kThr, 1)
           if (*abort_flag) break;
           uint8_t* dst = smem + L::ST_OFF + k * 3 * L::TILE;
           mbar_arrive_expect_tx(&st_full[k], 3 * L::TILE);
-          const int32_t tok = (int32_t)((tile0 + t) * kT);
+          const int32_t tok = (int32_t)ht.row0(tile0 + t, kT);
           tma_load_tok<FLAT>(dst, &tmK, &st_full[k], tok, bh, H);
           tma_load_tok<FLAT>(dst + L::TILE, &tmV, &st_full[k], tok, bh, H);
           tma_load_tok<FLAT>(dst + 2 * L::TILE, &tmdY, &st_full[k], tok, bh, H);
@@ -932,8 +942,8 @@ __global__ void __launch_bounds__(kThr, 1)
       }
       tc_fence_before();
       mbar_arrive(acc_empty);
-      const int64_t tok = (tile0 + tt) * kT + r;
-      if (tok < N) {
+      const int64_t tok = ht.row0(tile0 + tt, kT) + r;
+      if (ht.own(tile0 + tt, kT, r)) {
         const float f = (w == 0) ? s : gv;
         uint4* dst = reinterpret_cast<uint4*>(w == 0 ? dK + dk_head + tok * tdk.sn
                                                      : dV + dv_head + tok * tdv.sn);
@@ -967,8 +977,9 @@ __global__ void __launch_bounds__(kThr, 1)
       const int slot = slot_of(k);
       if (qq == w) {   // this warpgroup's first quarter of tile t: the row's statistics
         gprev = g;
-        const int64_t tok = (tile0 + t) * kT + r;
-        valid = tok < N;
+        // rows that are not the tile's own tokens get G = 0
+        const int64_t tok = ht.row0(tile0 + t, kT) + r;
+        valid = ht.own(tile0 + t, kT, r);
         if (valid) {
           const float4 st = enc_only ? make_float4(0.f, 0.f, 0.f, 0.f) : stats[bh * N + tok];
           mxp = st.x;
@@ -1008,7 +1019,10 @@ __global__ void __launch_bounds__(kThr, 1)
           float x0, x1;
           split_f32x2(fma_f32x2(S2, c2, nm2), x0, x1);
           // an encode-only gradient has no decode term: P_d = 0
-          const float p0 = enc_only ? 0.f : ex2(x0), p1 = enc_only ? 0.f : ex2(x1);
+          // (rows past N have zero K and dY; with lengths a right-aligned
+          // tile's earlier rows hold real ones)
+          const float p0 = (enc_only || (VAR && !valid)) ? 0.f : ex2(x0);
+          const float p1 = (enc_only || (VAR && !valid)) ? 0.f : ex2(x1);
           // exact form: P_e = 2^(c S - lse2[m]); G = P_d (dPd - delta_d) + P_e dPe'
           float s0, s1, e0, e1;
           split_f32x2(S2, s0, s1);
@@ -1121,7 +1135,7 @@ struct BFLayout {
   static constexpr int BYTES = MISC_OFF + 16;
 };
 
-template <int D, bool FLAT>
+template <int D, bool FLAT, bool VAR>
 __global__ void __launch_bounds__(kThr, 1)
     tc_bwd_b_fast_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdY2,
@@ -1131,7 +1145,8 @@ __global__ void __launch_bounds__(kThr, 1)
                          const float4* __restrict__ stats, const float2* __restrict__ params,
                          int enc_only, __nv_bfloat16* __restrict__ dK,
                          __nv_bfloat16* __restrict__ dV, Tok tdk, Tok tdv,
-                         float* __restrict__ dq_part, uint32_t* __restrict__ err) {
+                         float* __restrict__ dq_part, const int32_t* __restrict__ lens,
+                         uint32_t* __restrict__ err) {
   using L = BFLayout<D>;
   constexpr int M = L::M;
   constexpr int NS = L::NSLOT;
@@ -1171,7 +1186,10 @@ __global__ void __launch_bounds__(kThr, 1)
   const int64_t h = bh % H;
   const int64_t dk_head = tdk.head(bh, H), dv_head = tdv.head(bh, H);   // row 0 of the head
   const int64_t tile0 = (int64_t)chunk * chunk_tiles;
-  const int nt = (int)imin64(chunk_tiles, tiles_per_bh - tile0);
+  // with lengths, tokens past the batch element's length are padding: their tiles are skipped
+  const HeadTiles<VAR> ht(lens, bh / H, N);
+  const int nt = VAR ? (int)max(imin64(chunk_tiles, ht.count(kT) - tile0), (int64_t)0)
+                     : (int)imin64(chunk_tiles, tiles_per_bh - tile0);
   const float2 prm = params[bh];
   if (prm.y == 0.f) return;   // head served by tc_bwd_b_exact_kernel
 
@@ -1231,7 +1249,7 @@ __global__ void __launch_bounds__(kThr, 1)
         tma_load_3d(smem + L::AUG_OFF, &tmAug, c_full, 0, 0, (int32_t)bh);
         int issued = 0;
         for (int t = 0; t < nt; ++t) {
-          const int32_t tok = (int32_t)((tile0 + t) * kT);
+          const int32_t tok = (int32_t)ht.row0(tile0 + t, kT);
           const int kb = t % KST, vb = t % VST;
           if (t >= KST && !mbar_wait_sleep(&k_empty[kb], (uint32_t)(((t / KST) & 1) ^ 1))) {
             record_error(err, kErrBwdBTmaWait);
@@ -1385,10 +1403,13 @@ __global__ void __launch_bounds__(kThr, 1)
     const float Rh = prm.x;
     const uint64_t c2 = f32x2(c, c);
     bool ok = true;
+    // This thread's token in tile tt, and whether it is one of the tile's
+    // own tokens (else e = 0, G = 0 and no store).
+    auto row_tok = [&](int tt) -> int64_t { return ht.row0(tile0 + tt, kT) + r; };
+    auto own_row = [&](int tt) -> bool { return ht.own(tile0 + tt, kT, r); };
     // delta'' of this thread's row in tile tt, loaded one tile ahead of use
     auto load_dpp = [&](int tt) -> float {
-      const int64_t tok = (tile0 + tt) * kT + r;
-      return (!enc_only && tt < nt && tok < N) ? stats[bh * N + tok].z : 0.f;
+      return (!enc_only && tt < nt && own_row(tt)) ? stats[bh * N + row_tok(tt)].z : 0.f;
     };
     float dpp_next = load_dpp(0);
 
@@ -1415,8 +1436,8 @@ __global__ void __launch_bounds__(kThr, 1)
       }
       tc_fence_before();
       mbar_arrive(acc_empty);
-      const int64_t tok = (tile0 + tt) * kT + r;
-      if (tok < N) {
+      const int64_t tok = row_tok(tt);
+      if (own_row(tt)) {
         const float f = (w == 0) ? s : 1.f;
         uint4* dst = reinterpret_cast<uint4*>(w == 0 ? dK + dk_head + tok * tdk.sn
                                                      : dV + dv_head + tok * tdv.sn);
@@ -1447,9 +1468,8 @@ __global__ void __launch_bounds__(kThr, 1)
     for (int t = 0; t < nt; ++t) {
       const int k = 2 * t + w;          // this warpgroup's half of tile t
       const int slot = k % NS;
-      const int64_t tok = (tile0 + t) * kT + r;
       const float ndd = -dpp_next;
-      const float nR = (tok < N) ? -Rh : -INFINITY;   // past the end of the head: e = 0, G = 0
+      const float nR = own_row(t) ? -Rh : -INFINITY;   // not this tile's token: e = 0, G = 0
       dpp_next = load_dpp(t + 1);
       if (!warp_all(mbar_wait_sleep(&h_full[slot], (uint32_t)((k / NS) & 1)) && !*abort_flag)) {
         ok = false;
@@ -1596,7 +1616,7 @@ __global__ void bwd_dq_sum_kernel(const float4* __restrict__ dq_part, int B, int
   *reinterpret_cast<uint2*>(dQ + i * 4) = make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
 }
 
-template <int D, bool FLAT>
+template <int D, bool FLAT, bool VAR>
 cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, const void* dY,
                      const float* Z, const float* lse, void* dQ, void* dK, void* dV, const Dims& d,
                      float scale, const WsLayout& L, char* ws, cudaStream_t st) {
@@ -1633,11 +1653,11 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
 
   dim3 grid(p.chunks, (unsigned)BH);
   const int smemA = ALayout<D>::BYTES + 1024;
-  e = cudaFuncSetAttribute(tc_bwd_a_kernel<D, FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemA);
+  e = cudaFuncSetAttribute(tc_bwd_a_kernel<D, FLAT, VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemA);
   if (e != cudaSuccess) return e;
-  tc_bwd_a_kernel<D, FLAT><<<grid, kThr, smemA, st>>>(mq, mk, mdy, mz, (int)d.H, d.N, q_per_batch, c,
+  tc_bwd_a_kernel<D, FLAT, VAR><<<grid, kThr, smemA, st>>>(mq, mk, mdy, mz, (int)d.H, d.N, q_per_batch, c,
                                                 p.tiles_per_bh, p.chunk_tiles, rref, stats, dy2,
-                                                flags, dzp, err);
+                                                flags, dzp, d.lens, err);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
   bwd_mid_kernel<D><<<(unsigned)BH, kM, 0, st>>>(dzp, p.chunks, nullptr, Z, lse, dzs,
@@ -1646,22 +1666,24 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
 
   // each head runs in exactly one of the two pass-B kernels (params.y)
   const int smemF = BFLayout<D>::BYTES + 1024;
-  e = cudaFuncSetAttribute(tc_bwd_b_fast_kernel<D, FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(tc_bwd_b_fast_kernel<D, FLAT, VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smemF);
   if (e != cudaSuccess) return e;
-  tc_bwd_b_fast_kernel<D, FLAT><<<grid, kThr, smemF, st>>>(
+  tc_bwd_b_fast_kernel<D, FLAT, VAR><<<grid, kThr, smemF, st>>>(
       mq, mk, mv, mdy2, mz, mdz, maug, (int)d.H, d.N, q_per_batch, c, scale,
       p.tiles_per_bh,
-      p.chunk_tiles, stats, params, 0, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, d.dk, d.dv, dqp, err);
+      p.chunk_tiles, stats, params, 0, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, d.dk, d.dv, dqp, d.lens,
+      err);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   const int smemB = BLayout<D>::BYTES + 1024;
-  e = cudaFuncSetAttribute(tc_bwd_b_exact_kernel<D, FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(tc_bwd_b_exact_kernel<D, FLAT, VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smemB);
   if (e != cudaSuccess) return e;
-  tc_bwd_b_exact_kernel<D, FLAT><<<grid, kThr, smemB, st>>>(
+  tc_bwd_b_exact_kernel<D, FLAT, VAR><<<grid, kThr, smemB, st>>>(
       mq, mk, mv, mdy, mz, mdz, maug, (int)d.H, d.N, q_per_batch, c, scale,
       p.tiles_per_bh,
-      p.chunk_tiles, stats, params, lse2, 0, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, d.dk, d.dv, dqp, err);
+      p.chunk_tiles, stats, params, lse2, 0, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, d.dk, d.dv, dqp, d.lens,
+      err);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
   const bool shared_q = (qbs == 0);
@@ -1678,7 +1700,7 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
 // FLARE's backward wrote), then dQ = sum over b of (dQ_dyn + the encode's
 // partials).  Runs after FLARE's backward on the same stream and reuses its
 // workspace.
-template <int D, bool FLAT>
+template <int D, bool FLAT, bool VAR>
 cudaError_t tc_enc_bwd_t(const void* Q, const void* K, const void* V, const float* Z1,
                          const float* lse1, const void* dZ1, void* dQ, void* dK, void* dV,
                          const Dims& d, float scale, const WsLayout& L, char* ws, cudaStream_t st) {
@@ -1715,22 +1737,24 @@ cudaError_t tc_enc_bwd_t(const void* Q, const void* K, const void* V, const floa
 
   dim3 grid(p.chunks, (unsigned)BH);
   const int smemF = BFLayout<D>::BYTES + 1024;
-  e = cudaFuncSetAttribute(tc_bwd_b_fast_kernel<D, FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(tc_bwd_b_fast_kernel<D, FLAT, VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smemF);
   if (e != cudaSuccess) return e;
-  tc_bwd_b_fast_kernel<D, FLAT><<<grid, kThr, smemF, st>>>(
+  tc_bwd_b_fast_kernel<D, FLAT, VAR><<<grid, kThr, smemF, st>>>(
       mq, mk, mv, mv, mz, mdz, maug, (int)d.H, d.N, 0, c, scale, p.tiles_per_bh,
       p.chunk_tiles,
-      stats, params, 1, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, d.dk, d.dv, dqp, err);
+      stats, params, 1, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, d.dk, d.dv, dqp, d.lens,
+      err);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   const int smemB = BLayout<D>::BYTES + 1024;
-  e = cudaFuncSetAttribute(tc_bwd_b_exact_kernel<D, FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(tc_bwd_b_exact_kernel<D, FLAT, VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smemB);
   if (e != cudaSuccess) return e;
-  tc_bwd_b_exact_kernel<D, FLAT><<<grid, kThr, smemB, st>>>(
+  tc_bwd_b_exact_kernel<D, FLAT, VAR><<<grid, kThr, smemB, st>>>(
       mq, mk, mv, mv, mz, mdz, maug, (int)d.H, d.N, 0, c, scale, p.tiles_per_bh,
       p.chunk_tiles,
-      stats, params, lse2, 1, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, d.dk, d.dv, dqp, err);
+      stats, params, lse2, 1, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, d.dk, d.dv, dqp, d.lens,
+      err);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
   const int64_t total = d.H * kM * D;
@@ -1740,6 +1764,32 @@ cudaError_t tc_enc_bwd_t(const void* Q, const void* K, const void* V, const floa
   return cudaPeekAtLastError();
 }
 
+template <int D>
+cudaError_t tc_bwd_dispatch(const void* Q, int64_t qbs, const void* K, const void* V,
+                            const void* dY, const float* Z, const float* lse, void* dQ, void* dK,
+                            void* dV, const Dims& d, float scale, const WsLayout& L, char* ws,
+                            cudaStream_t st) {
+  const bool flat = tok_flat(d), var = d.lens != nullptr;
+  if (flat)
+    return var ? tc_bwd_t<D, true, true>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st)
+               : tc_bwd_t<D, true, false>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
+  return var ? tc_bwd_t<D, false, true>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st)
+             : tc_bwd_t<D, false, false>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
+}
+
+template <int D>
+cudaError_t tc_enc_bwd_dispatch(const void* Q, const void* K, const void* V, const float* Z1,
+                                const float* lse1, const void* dZ1, void* dQ, void* dK, void* dV,
+                                const Dims& d, float scale, const WsLayout& L, char* ws,
+                                cudaStream_t st) {
+  const bool flat = tok_flat(d), var = d.lens != nullptr;
+  if (flat)
+    return var ? tc_enc_bwd_t<D, true, true>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st)
+               : tc_enc_bwd_t<D, true, false>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st);
+  return var ? tc_enc_bwd_t<D, false, true>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st)
+             : tc_enc_bwd_t<D, false, false>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st);
+}
+
 }  // namespace
 
 cudaError_t launch_tc_bwd(const void* Q, int64_t qbs, const void* K, const void* V,
@@ -1747,13 +1797,8 @@ cudaError_t launch_tc_bwd(const void* Q, int64_t qbs, const void* K, const void*
                           void* dV, const Dims& d, float scale, const WsLayout& L, char* ws,
                           cudaStream_t st) {
   if (d.M != kM) return cudaErrorNotSupported;
-  const bool flat = tok_flat(d);
-  if (d.D == 32)
-    return flat ? tc_bwd_t<32, true>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st)
-                : tc_bwd_t<32, false>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
-  if (d.D == 16)
-    return flat ? tc_bwd_t<16, true>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st)
-                : tc_bwd_t<16, false>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
+  if (d.D == 32) return tc_bwd_dispatch<32>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
+  if (d.D == 16) return tc_bwd_dispatch<16>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
   return cudaErrorNotSupported;
 }
 
@@ -1762,13 +1807,8 @@ cudaError_t launch_tc_enc_bwd(const void* Q, const void* K, const void* V, const
                               const Dims& d, float scale, const WsLayout& L, char* ws,
                               cudaStream_t st) {
   if (d.M != kM) return cudaErrorNotSupported;
-  const bool flat = tok_flat(d);
-  if (d.D == 32)
-    return flat ? tc_enc_bwd_t<32, true>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st)
-                : tc_enc_bwd_t<32, false>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st);
-  if (d.D == 16)
-    return flat ? tc_enc_bwd_t<16, true>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st)
-                : tc_enc_bwd_t<16, false>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st);
+  if (d.D == 32) return tc_enc_bwd_dispatch<32>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st);
+  if (d.D == 16) return tc_enc_bwd_dispatch<16>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st);
   return cudaErrorNotSupported;
 }
 

@@ -61,6 +61,18 @@ def _strides(*ts):
     return arr
 
 
+def _seq_lens(seq_lens, B: int, device):
+    """Device int32 [B] lengths (or None), checked for shape, dtype and device."""
+    if seq_lens is None:
+        return None
+    if (not isinstance(seq_lens, torch.Tensor) or seq_lens.dtype != torch.int32
+            or seq_lens.shape != (B,) or seq_lens.device != device
+            or not seq_lens.is_contiguous()):
+        raise ValueError("seq_lens must be a contiguous int32 tensor of shape [B] on the "
+                         "tensors' device")
+    return seq_lens
+
+
 def _like(t: torch.Tensor) -> torch.Tensor:
     """An output with t's layout (empty_like keeps the strides of a dense
     tensor); a contiguous one where t's layout has gaps or overlaps."""
@@ -130,12 +142,13 @@ def device_status(workspace: torch.Tensor, stream=None) -> int:
 
 def flare_fwd(Q, K, V, scale: Optional[float] = None, *, save: bool = False,
               workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-              stream=None):
+              seq_lens: Optional[torch.Tensor] = None, stream=None):
     """FLARE forward.  Returns Y, or (Y, Z, lse) when ``save``.
 
     K, V (and ``out``) may be any [B,H,N,D] views with D contiguous, e.g.
     ``x.transpose(1, 2)`` of a [B,N,H,D] projection output; Y then takes K's
-    layout."""
+    layout.  ``seq_lens`` (int32 [B] on the device): valid tokens per batch
+    element; padding is never read, and Y is 0 there."""
     _need_cuda(Q, workspace)
     _need_tokens(K, V, out)
     B, H, N, M, D, qbs = _dims(Q, K)
@@ -147,19 +160,21 @@ def flare_fwd(Q, K, V, scale: Optional[float] = None, *, save: bool = False,
     ws = workspace if workspace is not None else alloc_workspace(
         _lib.FLARE_OP_FWD, B, H, N, M, D, K.dtype, K.device)
     strides = _strides(K, V, Y)
-    if strides is None:
+    lens = _seq_lens(seq_lens, B, K.device)
+    if strides is None and lens is None:
         st = _lib.load().flare_fwd(_ptr(Q), qbs, _ptr(K), _ptr(V), _ptr(Y), B, H, N, M, D, dt, s,
                                    _ptr(Z), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream))
     else:
-        st = _lib.load().flare_fwd_strided(_ptr(Q), qbs, _ptr(K), _ptr(V), _ptr(Y), strides, B, H,
-                                           N, M, D, dt, s, _ptr(Z), _ptr(lse), _ptr(ws),
-                                           ws.numel(), _stream(stream))
+        st = _lib.load().flare_fwd_ex(_ptr(Q), qbs, _ptr(K), _ptr(V), _ptr(Y), strides,
+                                      _ptr(lens), B, H, N, M, D, dt, s, _ptr(Z), _ptr(lse),
+                                      _ptr(ws), ws.numel(), _stream(stream))
     _lib.check(st, "flare_fwd")
     return (Y, Z, lse) if save else Y
 
 
 def flare_pp_fwd(Q, K, V, scale: Optional[float] = None, *, save: bool = False,
-                 workspace: Optional[torch.Tensor] = None, stream=None):
+                 workspace: Optional[torch.Tensor] = None,
+                 seq_lens: Optional[torch.Tensor] = None, stream=None):
     """FLARE++ forward with learned Q [H,M,D].  Returns (Y, Q_dyn) or
     (Y, Q_dyn, Z, lse) when ``save``."""
     _need_cuda(Q, workspace)
@@ -176,20 +191,22 @@ def flare_pp_fwd(Q, K, V, scale: Optional[float] = None, *, save: bool = False,
     ws = workspace if workspace is not None else alloc_workspace(
         _lib.FLARE_OP_PP_FWD, B, H, N, M, D, K.dtype, K.device)
     strides = _strides(K, V, Y)
-    if strides is None:
+    lens = _seq_lens(seq_lens, B, K.device)
+    if strides is None and lens is None:
         st = _lib.load().flare_pp_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(Y), _ptr(Qd), B, H, N, M,
                                       D, dt, s, _ptr(Z), _ptr(lse), _ptr(ws), ws.numel(),
                                       _stream(stream))
     else:
-        st = _lib.load().flare_pp_fwd_strided(_ptr(Q), _ptr(K), _ptr(V), _ptr(Y), _ptr(Qd),
-                                              strides, B, H, N, M, D, dt, s, _ptr(Z), _ptr(lse),
-                                              _ptr(ws), ws.numel(), _stream(stream))
+        st = _lib.load().flare_pp_fwd_ex(_ptr(Q), _ptr(K), _ptr(V), _ptr(Y), _ptr(Qd), strides,
+                                         _ptr(lens), B, H, N, M, D, dt, s, _ptr(Z), _ptr(lse),
+                                         _ptr(ws), ws.numel(), _stream(stream))
     _lib.check(st, "flare_pp_fwd")
     return (Y, Qd, Z, lse) if save else (Y, Qd)
 
 
 def flare_bwd(Q, K, V, dY, Z, lse, scale: Optional[float] = None, *,
-              workspace: Optional[torch.Tensor] = None, stream=None):
+              workspace: Optional[torch.Tensor] = None,
+              seq_lens: Optional[torch.Tensor] = None, stream=None):
     """FLARE backward.  Returns (dQ, dK, dV); dK and dV take K's and V's
     layouts (token tensors may be strided as in flare_fwd)."""
     _need_cuda(Q, Z, lse, workspace)
@@ -203,21 +220,23 @@ def flare_bwd(Q, K, V, dY, Z, lse, scale: Optional[float] = None, *,
     ws = workspace if workspace is not None else alloc_workspace(
         _lib.FLARE_OP_BWD, B, H, N, M, D, K.dtype, K.device)
     strides = _strides(K, V, dY, dK, dV)
-    if strides is None:
+    lens = _seq_lens(seq_lens, B, K.device)
+    if strides is None and lens is None:
         st = _lib.load().flare_bwd(_ptr(Q), qbs, _ptr(K), _ptr(V), _ptr(dY), _ptr(Z), _ptr(lse),
                                    _ptr(dQ), _ptr(dK), _ptr(dV), B, H, N, M, D, dt, s, _ptr(ws),
                                    ws.numel(), _stream(stream))
     else:
-        st = _lib.load().flare_bwd_strided(_ptr(Q), qbs, _ptr(K), _ptr(V), _ptr(dY), _ptr(Z),
-                                           _ptr(lse), _ptr(dQ), _ptr(dK), _ptr(dV), strides, B,
-                                           H, N, M, D, dt, s, _ptr(ws), ws.numel(),
-                                           _stream(stream))
+        st = _lib.load().flare_bwd_ex(_ptr(Q), qbs, _ptr(K), _ptr(V), _ptr(dY), _ptr(Z),
+                                      _ptr(lse), _ptr(dQ), _ptr(dK), _ptr(dV), strides,
+                                      _ptr(lens), B, H, N, M, D, dt, s, _ptr(ws), ws.numel(),
+                                      _stream(stream))
     _lib.check(st, "flare_bwd")
     return dQ, dK, dV
 
 
 def flare_pp_bwd(Q, K, V, dY, Q_dyn, Z, lse, scale: Optional[float] = None, *,
-                 workspace: Optional[torch.Tensor] = None, stream=None):
+                 workspace: Optional[torch.Tensor] = None,
+                 seq_lens: Optional[torch.Tensor] = None, stream=None):
     """FLARE++ backward with learned Q [H,M,D] (Q_dyn, Z, lse from
     flare_pp_fwd(..., save=True)).  Returns (dQ [H,M,D], dK, dV)."""
     _need_cuda(Q, Q_dyn, Z, lse, workspace)
@@ -233,15 +252,16 @@ def flare_pp_bwd(Q, K, V, dY, Q_dyn, Z, lse, scale: Optional[float] = None, *,
     ws = workspace if workspace is not None else alloc_workspace(
         _lib.FLARE_OP_PP_BWD, B, H, N, M, D, K.dtype, K.device)
     strides = _strides(K, V, dY, dK, dV)
-    if strides is None:
+    lens = _seq_lens(seq_lens, B, K.device)
+    if strides is None and lens is None:
         st = _lib.load().flare_pp_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(dY), _ptr(Q_dyn), _ptr(Z),
                                       _ptr(lse), _ptr(dQ), _ptr(dK), _ptr(dV), B, H, N, M, D, dt,
                                       s, _ptr(ws), ws.numel(), _stream(stream))
     else:
-        st = _lib.load().flare_pp_bwd_strided(_ptr(Q), _ptr(K), _ptr(V), _ptr(dY), _ptr(Q_dyn),
-                                              _ptr(Z), _ptr(lse), _ptr(dQ), _ptr(dK), _ptr(dV),
-                                              strides, B, H, N, M, D, dt, s, _ptr(ws),
-                                              ws.numel(), _stream(stream))
+        st = _lib.load().flare_pp_bwd_ex(_ptr(Q), _ptr(K), _ptr(V), _ptr(dY), _ptr(Q_dyn),
+                                         _ptr(Z), _ptr(lse), _ptr(dQ), _ptr(dK), _ptr(dV),
+                                         strides, _ptr(lens), B, H, N, M, D, dt, s, _ptr(ws),
+                                         ws.numel(), _stream(stream))
     _lib.check(st, "flare_pp_bwd")
     return dQ, dK, dV
 

@@ -226,7 +226,7 @@ def test_strided_entry_points_validate_strides(lib):
 
     def fwd(*triples):
         st = _st(*triples) if triples else None
-        return lib.flare_fwd_strided(_p(F), 0, _p(F), _p(F), _p(F), st, B, H, N, M, D, 0, 0.25,
+        return lib.flare_fwd_ex(_p(F), 0, _p(F), _p(F), _p(F), st, None, B, H, N, M, D, 0, 0.25,
                                      None, None, _p(F), ws, None)
 
     # valid layouts pass validation and fail only at the first enqueue
@@ -247,20 +247,25 @@ def test_strided_entry_points_validate_strides(lib):
     wsb = lib.flare_workspace_size(2, B, H, N, M, D, 0)
 
     def bwd(*triples):
-        return lib.flare_bwd_strided(_p(F), 0, _p(F), _p(F), _p(F), _p(F), _p(F), _p(F), _p(F),
-                                     _p(F), _st(*triples), B, H, N, M, D, 0, 0.25, _p(F), wsb,
-                                     None)
+        return lib.flare_bwd_ex(_p(F), 0, _p(F), _p(F), _p(F), _p(F), _p(F), _p(F), _p(F),
+                                _p(F), _st(*triples), None, B, H, N, M, D, 0, 0.25, _p(F), wsb,
+                                None)
 
     assert bwd(bnhd, bnhd, bnhd, bnhd, bnhd) == CUDA
     assert bwd(bnhd, bnhd, bnhd, bnhd, (N * H * D, D, 8)) == INVALID
     assert bwd(bnhd, bnhd, (N * H * D, D, 8), bnhd, bnhd) == CUDA
     wsp = lib.flare_workspace_size(1, B, H, N, M, D, 0)
-    assert lib.flare_pp_fwd_strided(_p(F), _p(F), _p(F), _p(F), None, _st(bnhd, bnhd, bnhd), B,
-                                    H, N, M, D, 0, 0.25, None, None, _p(F), wsp, None) == CUDA
-    assert lib.flare_pp_fwd_strided(_p(F), _p(F), _p(F), _p(F), None,
-                                    _st(bnhd, bnhd, (N * D, N * D, D)), B, H, N, M, D, 0, 0.25,
-                                    None, None, _p(F), wsp, None) == INVALID
+    assert lib.flare_pp_fwd_ex(_p(F), _p(F), _p(F), _p(F), None, _st(bnhd, bnhd, bnhd), None, B,
+                               H, N, M, D, 0, 0.25, None, None, _p(F), wsp, None) == CUDA
+    assert lib.flare_pp_fwd_ex(_p(F), _p(F), _p(F), _p(F), None,
+                               _st(bnhd, bnhd, (N * D, N * D, D)), None, B, H, N, M, D, 0, 0.25,
+                               None, None, _p(F), wsp, None) == INVALID
     wspb = lib.flare_workspace_size(3, B, H, N, M, D, 0)
-    assert lib.flare_pp_bwd_strided(_p(F), _p(F), _p(F), _p(F), _p(F), _p(F), _p(F), _p(F),
-                                    _p(F), _p(F), _st(bnhd, bnhd, bnhd, (0, D, H * D), bnhd), B,
-                                    H, N, M, D, 0, 0.25, _p(F), wspb, None) == INVALID
+    assert lib.flare_pp_bwd_ex(_p(F), _p(F), _p(F), _p(F), _p(F), _p(F), _p(F), _p(F),
+                               _p(F), _p(F), _st(bnhd, bnhd, bnhd, (0, D, H * D), bnhd), None, B,
+                               H, N, M, D, 0, 0.25, _p(F), wspb, None) == INVALID
+    # seq_lens: a device array of int32, 4-byte aligned
+    assert lib.flare_fwd_ex(_p(F), 0, _p(F), _p(F), _p(F), None, _p(F + 0x600002), B, H, N, M,
+                            D, 0, 0.25, None, None, _p(F), ws, None) == INVALID
+    assert lib.flare_fwd_ex(_p(F), 0, _p(F), _p(F), _p(F), None, _p(F + 0x600004), B, H, N, M,
+                            D, 0, 0.25, None, None, _p(F), ws, None) == CUDA

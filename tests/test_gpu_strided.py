@@ -1,7 +1,7 @@
 """Token tensors in other layouts than contiguous [B,H,N,D].
 
 A fused projection produces K and V as [B,N,H,D] (or interleaved
-[B,N,3,H,D]); the *_strided entry points read and write such layouts in
+[B,N,3,H,D]); the *_ex entry points read and write such layouts in
 place.  The arithmetic is the same as for contiguous tensors, so the results
 must equal the contiguous call's bit for bit, and the contiguous call is
 compared with the oracle elsewhere; one case per op is also compared with the
