@@ -420,7 +420,7 @@ def _row_roofline(t_ms: float, exps: float, flops: float, hbm_bytes: float, peak
 
 def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0,
                     which=("flare_pp_fwd", "flare_fwd_bwd", "flare_pp_fwd_bwd",
-                           "flare_strided")):
+                           "flare_strided", "flare_varlen")):
     """Times the FLARE++ forward (B=2 H=8 N=262,144 M=256 D=32) and the
     forward + backward of B=8 H=8 N=16,384 M=128 D=32, both bf16, on the
     same device with CUDA events (median of `iters` launches after 3
@@ -456,6 +456,8 @@ def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0,
         rows.update(_time_pp_fwd_bwd(dev, peaks, peak_kind, timed, seed))
     if "flare_strided" in which:
         rows.update(_time_strided(dev, peaks, peak_kind, timed, seed))
+    if "flare_varlen" in which:
+        rows.update(_time_varlen(dev, peaks, peak_kind, timed, seed))
     del flush_buf
     torch.cuda.empty_cache()
     return rows
@@ -573,6 +575,45 @@ def _time_strided(dev, peaks, peak_kind, timed, seed):
         "roofline": _row_roofline(ms, 4.0 * u * w.M, 28.0 * u * w.M * w.D,
                                   9.0 * u * w.D * 2, peaks, peak_kind)}
     return {"flare_strided": out}
+
+
+def _time_varlen(dev, peaks, peak_kind, timed, seed):
+    """Right-padded batches: the forward + backward workload (B=8 H=8
+    N=16,384 M=128 D=32 bf16) with sequence lengths N - b N/16 (16,384 down
+    to 9,216, 78% of the tokens valid), beside the same call at full length.
+    Throughput counts valid tokens; the roofline is that of the valid work."""
+    import torch
+
+    import rank_latent_attention_flare_b200 as fl
+    w = WORKLOADS["c5_fwdbwd_bf16_16k"]
+    lens_l = [w.N - b * (w.N // 16) for b in range(w.B)]
+    lens = torch.tensor(lens_l, dtype=torch.int32, device=dev)
+    x = make_inputs(w.B, w.H, w.N, w.M, w.D, dtype=w.torch_dtype, seed=seed, with_dy=True)
+    g = {k: v.to(dev) for k, v in x.items()}
+    wsf = fl.alloc_workspace(fl.FLARE_OP_FWD, w.B, w.H, w.N, w.M, w.D, w.torch_dtype, dev)
+    wsb = fl.alloc_workspace(fl.FLARE_OP_BWD, w.B, w.H, w.N, w.M, w.D, w.torch_dtype, dev)
+    saved = {}
+
+    def fwd():
+        saved["out"] = fl.flare_fwd(g["Q"], g["K"], g["V"], w.scale, save=True, workspace=wsf,
+                                    seq_lens=lens)
+
+    ms_f = timed(fwd)
+    _, Z, lse = saved["out"]
+    ms_b = timed(lambda: fl.flare_bwd(g["Q"], g["K"], g["V"], g["dY"], Z, lse, w.scale,
+                                      workspace=wsb, seq_lens=lens))
+    if fl.device_status(wsf) != 0 or fl.device_status(wsb) != 0:
+        raise RuntimeError("device wait ran out in the variable-length forward + backward")
+    valid = sum(lens_l)
+    u = w.H * valid
+    ms = ms_f + ms_b
+    return {"flare_varlen": {
+        "workload": f"FLARE fwd+bwd B={w.B} H={w.H} N={w.N} M={w.M} D={w.D} bf16, "
+                    f"seq_lens {lens_l[0]}..{lens_l[-1]} ({100 * valid / (w.B * w.N):.0f}% valid)",
+        "ms": round(ms, 4), "fwd_ms": round(ms_f, 4), "bwd_ms": round(ms_b, 4),
+        "valid_tokens_per_s": valid / (ms / 1e3),
+        "roofline": _row_roofline(ms, 4.0 * u * w.M, 28.0 * u * w.M * w.D,
+                                  9.0 * u * w.D * 2, peaks, peak_kind)}}
 
 
 def time_sdpa_context(dev, w=WORKLOAD, iters: int = 5, seed: int = 0):
@@ -708,7 +749,7 @@ def main():
     ap.add_argument("--no-rows", action="store_true",
                     help="skip the FLARE++ and forward+backward timings")
     ap.add_argument("--row", choices=["flare_pp_fwd", "flare_fwd_bwd", "flare_pp_fwd_bwd",
-                                      "flare_strided"],
+                                      "flare_strided", "flare_varlen"],
                     default=None,
                     help="time only this workload (one JSON line with its timing and roofline)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -300,7 +300,7 @@ flare_status_t flare_fwd_ex(const void* Q, int64_t qbs, const void* K, const voi
   FLARE_TRY(run_encode(Q, qbs, K, V, d, dt, scale, L, ws, st));
   FLARE_TRY(run_combine(d, dt, Z_save, lse_save, nullptr, nullptr, L, ws, st));
   FLARE_TRY(run_decode(Q, qbs, K, Y, d, dt, scale, L, ws, st, sms));
-  FLARE_CUDA(launch_zero_padding(Y, d.y, d, dt, st));   // Y = 0 at padding
+  FLARE_CUDA(launch_zero_padding(Y, d.y, nullptr, d.y, d, dt, st));   // Y = 0 at padding
   return FLARE_OK;
 }
 
@@ -339,7 +339,7 @@ flare_status_t flare_pp_fwd_ex(const void* Q, const void* K, const void* V, void
   FLARE_TRY(run_encode(qdyn, qdyn_bs, K, V, d, dt, scale, L, ws, st));
   FLARE_TRY(run_combine(d, dt, Z_save, lse_save, nullptr, nullptr, L, ws, st));
   FLARE_TRY(run_decode(qdyn, qdyn_bs, K, Y, d, dt, scale, L, ws, st, sms));
-  FLARE_CUDA(launch_zero_padding(Y, d.y, d, dt, st));   // Y = 0 at padding
+  FLARE_CUDA(launch_zero_padding(Y, d.y, nullptr, d.y, d, dt, st));   // Y = 0 at padding
   return FLARE_OK;
 }
 
@@ -373,8 +373,7 @@ flare_status_t flare_bwd_ex(const void* Q, int64_t qbs, const void* K, const voi
   FLARE_TRY(reset_error_word(ws, st));
   FLARE_CUDA(launch_check_lens(d, (uint32_t*)(ws + L.hdr), st));
   FLARE_CUDA(launch_bwd(Q, qbs, K, V, dY, Z_save, lse_save, dQ, dK, dV, d, dt, scale, L, ws, st));
-  FLARE_CUDA(launch_zero_padding(dK, d.dk, d, dt, st));   // no gradient at padding
-  FLARE_CUDA(launch_zero_padding(dV, d.dv, d, dt, st));
+  FLARE_CUDA(launch_zero_padding(dK, d.dk, dV, d.dv, d, dt, st));   // no gradient at padding
   return FLARE_OK;
 }
 
@@ -417,8 +416,7 @@ flare_status_t flare_pp_bwd_ex(const void* Q, const void* K, const void* V, cons
                         scale, L, ws, st));
   // the first encode's gradient with upstream dQ_dyn, and dQ
   FLARE_CUDA(launch_pp_bwd_tail(Q, K, V, z1, lse1, ws + L.dqd, dQ, dK, dV, d, dt, scale, L, ws, st));
-  FLARE_CUDA(launch_zero_padding(dK, d.dk, d, dt, st));   // no gradient at padding
-  FLARE_CUDA(launch_zero_padding(dV, d.dv, d, dt, st));
+  FLARE_CUDA(launch_zero_padding(dK, d.dk, dV, d.dv, d, dt, st));   // no gradient at padding
   return FLARE_OK;
 }
 

@@ -284,43 +284,53 @@ __device__ __forceinline__ int64_t seq_len(const int32_t* __restrict__ lens, int
   return L < 0 ? 0 : (L > N ? N : L);
 }
 
-// Tiles of T tokens over a head with nb valid tokens: tile t starts at t T,
-// except that a partial last tile is right-aligned to end at nb.  It then
-// re-reads rows of the tile before it (or rows before 0, which TMA fills with
-// zeros) instead of rows past nb; a row r of tile t belongs to the tile iff
-// tile_row0(t) + r >= t T.
-__host__ __device__ __forceinline__ int64_t tile_row0(int64_t t, int64_t nb, int T) {
-  const int64_t s = t * T;
-  return (s + T > nb) ? nb - T : s;
-}
 __host__ __device__ __forceinline__ int64_t tiles_of(int64_t nb, int T) { return (nb + T - 1) / T; }
 
 // Token tiles of one head, T tokens each.  Without lengths (VAR false) the
 // head has all N tokens: tile t covers rows [tT, tT + T) and TMA fills the
 // rows past N with zeros.  With lengths it has nb <= N tokens and a partial
 // last tile is right-aligned to end at nb, so no padding row is ever read.
-// Both are compile-time variants: the N-token code is unchanged by lengths.
+// Both are compile-time variants: the N-token code is unchanged by lengths,
+// and the length-aware one works in 32 bits (the tensor-core kernels take
+// N < 2^31) to keep register pressure down.
 template <bool VAR>
-struct HeadTiles {
-  int64_t nb;   // the head's tokens
-  __device__ __forceinline__ HeadTiles(const int32_t* __restrict__ lens, int64_t b, int64_t N)
-      : nb(VAR ? seq_len(lens, b, N) : N) {}
+struct HeadTiles;
+
+template <>
+struct HeadTiles<false> {
+  int64_t nb;   // the head's tokens (N)
+  __device__ __forceinline__ HeadTiles(const int32_t* __restrict__, int64_t, int64_t N) : nb(N) {}
   __device__ __forceinline__ int64_t count(int T) const { return tiles_of(nb, T); }
-  // token of row 0 of tile t (negative rows read as zeros)
-  __device__ __forceinline__ int64_t row0(int64_t t, int T) const {
-    return VAR ? tile_row0(t, nb, T) : t * T;
-  }
+  // token of row 0 of tile t
+  __device__ __forceinline__ int64_t row0(int64_t t, int T) const { return t * T; }
   // row r of tile t is one of the tile's own tokens
-  __device__ __forceinline__ bool own(int64_t t, int T, int r) const {
-    return VAR ? row0(t, T) + r >= t * T : t * T + r < nb;
-  }
+  __device__ __forceinline__ bool own(int64_t t, int T, int r) const { return t * T + r < nb; }
   // the tile's own tokens are its columns [lo, hi)
+  __device__ __forceinline__ int lo(int64_t, int) const { return 0; }
+  __device__ __forceinline__ int hi(int64_t t, int T) const { return (int)imin64(T, nb - t * T); }
+};
+
+template <>
+struct HeadTiles<true> {
+  int nb;   // the batch element's length, clamped to [0, N]
+  __device__ __forceinline__ HeadTiles(const int32_t* __restrict__ lens, int64_t b, int64_t N)
+      : nb((int)seq_len(lens, b, N)) {}
+  __device__ __forceinline__ int64_t count(int T) const { return (nb + T - 1) / T; }
+  // token of row 0 of tile t: a partial last tile ends at nb (rows before
+  // token 0 read as zeros)
+  __device__ __forceinline__ int64_t row0(int64_t t, int T) const {
+    const int s = (int)t * T;
+    return s + T > nb ? nb - T : s;
+  }
+  __device__ __forceinline__ bool own(int64_t t, int T, int r) const {
+    const int s = (int)t * T;
+    return (s + T > nb ? nb - T : s) + r >= s;
+  }
   __device__ __forceinline__ int lo(int64_t t, int T) const {
-    return VAR ? (int)max((t + 1) * T - nb, (int64_t)0) : 0;
+    const int x = ((int)t + 1) * T - nb;
+    return x > 0 ? x : 0;
   }
-  __device__ __forceinline__ int hi(int64_t t, int T) const {
-    return VAR ? T : (int)imin64(T, nb - t * T);
-  }
+  __device__ __forceinline__ int hi(int64_t, int T) const { return T; }
 };
 
 cudaError_t launch_simt_encode(const void* Q, int64_t qbs, const void* K, const void* V,
@@ -332,10 +342,11 @@ cudaError_t launch_simt_decode(const void* Q, int64_t qbs, const void* K, const 
                                cudaStream_t st);
 // Records kErrSeqLen when a length lies outside [0, N] (lens non-NULL).
 cudaError_t launch_check_lens(const Dims& d, uint32_t* err, cudaStream_t st);
-// Zeroes the padding rows (n >= the batch element's length) of a token
-// tensor with strides t (no-op when d.lens is NULL).
-cudaError_t launch_zero_padding(void* X, const Tok& t, const Dims& d, flare_dtype_t dt,
-                                cudaStream_t st);
+// Zeroes the padding rows (n >= the batch element's length) of the token
+// tensor X0 with strides t0 and, when X1 is not NULL, of X1 (no-op when
+// d.lens is NULL).
+cudaError_t launch_zero_padding(void* X0, const Tok& t0, void* X1, const Tok& t1, const Dims& d,
+                                flare_dtype_t dt, cudaStream_t st);
 cudaError_t launch_combine(const Dims& d, flare_dtype_t dt, int slots_per_bh,
                            const float* part_ml, const float* part_acc, float* Zf,
                            __nv_bfloat16* Zb, float* Z_save, float* lse_save, const void* Qpp,

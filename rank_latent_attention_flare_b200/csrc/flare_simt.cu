@@ -187,19 +187,24 @@ __global__ void check_lens_kernel(const int32_t* __restrict__ lens, int64_t B, i
   if (b < B && (lens[b] < 0 || (int64_t)lens[b] > N)) record_error(err, kErrSeqLen);
 }
 
-// One thread per 16 bytes of a padding row: grid.y = b * H + h, x over the
-// row bytes of tokens [L_b, N).
-__global__ void zero_padding_kernel(uint8_t* __restrict__ X, Tok t, int esz,
-                                    const int32_t* __restrict__ lens, int H, int64_t N, int D) {
+// Zeroes the padding rows (tokens [L_b, N)) of up to two token tensors of
+// the same shape: blockIdx.y = b * H + h, a grid-stride loop over the head's
+// padding in 16-byte pieces.
+__global__ void zero_padding_kernel(uint8_t* __restrict__ X0, Tok t0, uint8_t* __restrict__ X1,
+                                    Tok t1, int esz, const int32_t* __restrict__ lens, int H,
+                                    int64_t N, int D) {
   const int64_t bh = blockIdx.y;
-  const int64_t b = bh / H;
-  const int64_t L = seq_len(lens, b, N);
+  const int64_t L = seq_len(lens, bh / H, N);
   const int per_row = D * esz / 16;   // 16-byte pieces per row
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t n = L + i / per_row;
-  if (n >= N) return;
-  uint8_t* row = X + (t.head(bh, H) + n * t.sn) * esz;
-  reinterpret_cast<uint4*>(row)[i % per_row] = make_uint4(0u, 0u, 0u, 0u);
+  const int64_t total = (N - L) * per_row;
+  const int64_t h0 = t0.head(bh, H), h1 = X1 ? t1.head(bh, H) : 0;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t n = L + i / per_row;
+    const int piece = (int)(i % per_row);
+    reinterpret_cast<uint4*>(X0 + (h0 + n * t0.sn) * esz)[piece] = make_uint4(0u, 0u, 0u, 0u);
+    if (X1) reinterpret_cast<uint4*>(X1 + (h1 + n * t1.sn) * esz)[piece] = make_uint4(0u, 0u, 0u, 0u);
+  }
 }
 
 template <typename T, int D>
@@ -257,14 +262,15 @@ cudaError_t launch_check_lens(const Dims& d, uint32_t* err, cudaStream_t st) {
   return cudaPeekAtLastError();
 }
 
-cudaError_t launch_zero_padding(void* X, const Tok& t, const Dims& d, flare_dtype_t dt,
-                                cudaStream_t st) {
+cudaError_t launch_zero_padding(void* X0, const Tok& t0, void* X1, const Tok& t1, const Dims& d,
+                                flare_dtype_t dt, cudaStream_t st) {
   if (d.lens == nullptr) return cudaSuccess;
   const int esz = (dt == FLARE_F32) ? 4 : 2;
-  const int64_t pieces = d.N * d.D * esz / 16;   // at most (16-byte pieces per head)
-  dim3 grid((unsigned)((pieces + 255) / 256), (unsigned)d.BH());
-  zero_padding_kernel<<<grid, 256, 0, st>>>((uint8_t*)X, t, esz, d.lens, (int)d.H, d.N,
-                                            (int)d.D);
+  // a few blocks per head: padding is usually a fraction of N
+  const int64_t pieces = d.N * d.D * esz / 16;
+  const unsigned bx = (unsigned)imin64((pieces + 255) / 256, 8);
+  zero_padding_kernel<<<dim3(bx, (unsigned)d.BH()), 256, 0, st>>>(
+      (uint8_t*)X0, t0, (uint8_t*)X1, t1, esz, d.lens, (int)d.H, d.N, (int)d.D);
   return cudaPeekAtLastError();
 }
 
