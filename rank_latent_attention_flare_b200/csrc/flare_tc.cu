@@ -38,6 +38,12 @@ constexpr int kRegsSoftmax = 200;
 constexpr int kRegsProducer = 104;
 constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
+constexpr int kWarpNorm = 10;   // decode: warps 10 and 11 bound the row max of alternate K tiles
+// Slots of the decode's bound ring.  The norm warp fills tile i's slot only
+// after the TMA load of tile i, which waits for the S product of tile i - 6,
+// which waits for the row warps to finish tile i - 8's S; so 16 slots are
+// never refilled before the row warps have read them.
+constexpr int kDecBoundSlots = 16;
 constexpr int kEncStages = 8;
 constexpr int kDecStages = 6;
 constexpr float kRescaleTau = 8.0f;   // log2 units: rescale only when the max grows by > 2^8
@@ -51,6 +57,12 @@ constexpr float kRedoTau = 64.0f;     // log2 units: past 2^64 above m_ref a til
 // or 12th pair is slower).
 constexpr int kEncPolyEvery = 4;
 constexpr int kDecPolyEvery = 16;
+// Decode reference of a token row (M = 256): the max of the first 32-logit
+// chunk read, used when c |k| max_m |q_m| (Cauchy-Schwarz: at least every
+// logit) lies at most this far (log2 units) above it, so no weight exceeds
+// 2^kDecRefTau; else the exact row max (a second pass over the row).  With
+// M = 128 the second pass is short and the exact max is always taken.
+constexpr float kDecRefTau = 64.f;
 constexpr int kMinSmemBytes = 120 * 1024;  // keeps one CTA (and its TMEM) per SM
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -493,9 +505,11 @@ struct DecLayout {
   static constexpr int Z_OFF = M * RB;
   static constexpr int K_OFF = 2 * M * RB;
   static constexpr int BAR_OFF = K_OFF + kDecStages * TILE;
-  static constexpr int NBARS = 2 * kDecStages + 1 + 4 * 2 + 1;
+  static constexpr int NBARS = 2 * kDecStages + 1 + 4 * 2 + 1 + kDecBoundSlots;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
-  static constexpr int BYTES = MISC_OFF + 16;
+  static constexpr int QN_OFF = MISC_OFF + 16;              // [M] float: |q_m|^2
+  static constexpr int KN_OFF = QN_OFF + M * 4;             // [slot][kTile] float: bound U
+  static constexpr int BYTES = KN_OFF + kDecBoundSlots * kTile * 4;
 };
 
 template <int D, int M, bool FLAT, bool VAR>
@@ -503,11 +517,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmZ, int H, int64_t N, int q_per_batch,
                      float c, int64_t tiles_per_bh, int64_t chunk_tiles,
-                     __nv_bfloat16* __restrict__ Y, Tok ty, const int32_t* __restrict__ lens,
-                     uint32_t* __restrict__ err) {
+                     __nv_bfloat16* __restrict__ Y, Tok ty, const __nv_bfloat16* __restrict__ Qg,
+                     const int32_t* __restrict__ lens, uint32_t* __restrict__ err) {
   using L = DecLayout<D, M>;
   constexpr int RB = L::RB;
   constexpr uint32_t SW = umma_swizzle_code(RB);
+  constexpr bool kBound = (M == 256);  // first-chunk reference under the row-max bound
   constexpr int R = M;                 // TMEM columns per warpgroup
   constexpr uint32_t NCOLS = 2 * R;    // 256 or 512
   constexpr int TY = M / 2;            // Y accumulator column inside a warpgroup's region
@@ -525,6 +540,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_full = s_empty + 2;
   uint64_t* y_full = p_full + 2;
   uint64_t* drain = y_full + 2;
+  uint64_t* kn_full = drain + 1;   // [slot]: the tile's row bounds written
+  float* kn = (float*)(smem + L::KN_OFF);
   uint32_t* tmem_slot = (uint32_t*)(smem + L::MISC_OFF);
   volatile int* abort_flag = (volatile int*)(smem + L::MISC_OFF + 4);
 
@@ -542,7 +559,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDecStages; ++s) {
       mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
+      // released by the S product's commit (and the bound warp, done reading)
+      mbar_init(&k_empty[s], kBound ? 2 : 1);
+    }
+    for (int s = 0; s < kDecBoundSlots; ++s) {
+      mbar_init(&kn_full[s], 32);
     }
     mbar_init(qz_full, 1);
     for (int w = 0; w < 2; ++w) {
@@ -554,6 +575,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
+  }
+  if (kBound) {
+    // |q_m|^2 of this head's latents, for the bound on each token's row max
+    const __nv_bfloat16* qh = Qg + (q_per_batch ? bh : h) * (int64_t)M * D;
+    float* qn2 = (float*)(smem + L::QN_OFF);
+    for (int m = threadIdx.x; m < M; m += blockDim.x) {
+      float acc = 0.f;
+#pragma unroll
+      for (int v = 0; v < D / 8; ++v) {
+        const uint4 u = reinterpret_cast<const uint4*>(qh + (int64_t)m * D)[v];
+        const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+          acc = fmaf(bf_lo(uu[jj]), bf_lo(uu[jj]), fmaf(bf_hi(uu[jj]), bf_hi(uu[jj]), acc));
+      }
+      qn2[m] = acc;
+    }
   }
   if (warp == kWarpMma) tmem_alloc(tmem_slot, NCOLS);
   tc_fence_before();
@@ -641,6 +679,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(drain);
       mbar_wait_sleep(drain, 0);
     }
+    } else if (kBound && (warp == kWarpNorm || warp == kWarpNorm + 1)) {
+      // The bound U = c |k| max_m |q_m| >= c S[m] on every row of each K tile
+      // (the swizzle only permutes a row's 16-byte pieces; rows outside the
+      // head's tokens were filled with zeros).
+      float qmax2 = 0.f;
+      {
+        const float4* qn2 = (const float4*)(smem + L::QN_OFF);
+        for (int m = 0; m < M / 4; ++m) {
+          const float4 v = qn2[m];
+          qmax2 = fmaxf(qmax2, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+        }
+      }
+      bool ok = true;
+      for (int64_t i = warp - kWarpNorm; i < ntiles; i += 2) {
+        const int s = (int)(i % kDecStages);
+        const int slot = (int)(i % kDecBoundSlots);
+        if (!warp_all(mbar_wait_sleep(&k_full[s], (uint32_t)((i / kDecStages) & 1)) &&
+                      !*abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* kt = smem + L::K_OFF + s * L::TILE;
+#pragma unroll
+        for (int rr = lane; rr < kTile; rr += 32) {
+          uint64_t kq[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
+#pragma unroll
+          for (int v = 0; v < D / 8; ++v) {
+            const uint4 u = reinterpret_cast<const uint4*>(kt + rr * RB)[v];
+            const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              const uint64_t p = f32x2(bf_lo(uu[jj]), bf_hi(uu[jj]));
+              kq[jj & 1] = fma_f32x2(p, p, kq[jj & 1]);
+            }
+          }
+          float q0, q1, q2, q3;
+          split_f32x2(kq[0], q0, q1);
+          split_f32x2(kq[1], q2, q3);
+          kn[slot * kTile + rr] = c * sqrtf(((q0 + q1) + (q2 + q3)) * qmax2);
+        }
+        mbar_arrive(&kn_full[slot]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&k_empty[s]);
+      }
+      if (!ok) {
+        record_error(err, kErrDecTmaWait);
+        *abort_flag = 1;
+      }
     }
   } else {
     regs_acquire<kRegsSoftmax>();
@@ -654,40 +740,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t i = 2 * j + w;
       const int64_t tok = ht.row0(tile0 + i, kTile) + r;
       const bool mine = ht.own(tile0 + i, kTile, r);
-      if (!warp_all(mbar_wait(&s_full[w], (uint32_t)(j & 1)) && !*abort_flag)) {
+      const int slot = (int)(i % kDecBoundSlots);
+      if (!warp_all(mbar_wait(&s_full[w], (uint32_t)(j & 1)) &&
+                    (!kBound || mbar_wait(&kn_full[slot], (uint32_t)((i / kDecBoundSlots) & 1))) &&
+                    !*abort_flag)) {
         ok = false;
         break;
       }
       __syncwarp();
       tc_fence_after();
-      // pass 1: row max over all M logits
-      // Chunks of 32 columns are double-buffered: the load of the next chunk
-      // is in flight while the current one is processed.
+      // Chunks of 32 columns, double-buffered: the load of the next chunk is
+      // in flight while the current one is processed.  Pass 2 below visits
+      // them in the order: upper half last chunk first, then lower half
+      // first chunk first.  The P of upper chunk u (S columns [M/2 + 32u,
+      // +32)) goes to columns [3M/4 + 16u, +16), inside upper chunks already
+      // read; the P of lower chunk u goes to [16u, +16), inside lower chunks
+      // already read.  No store touches a chunk that is still to be loaded.
       constexpr int NC = M / 32;
+      auto chunk_col = [](int k) { return k < NC / 2 ? M / 2 + 32 * (NC / 2 - 1 - k) : 32 * (k - NC / 2); };
+      auto p_col = [](int k) { return k < NC / 2 ? 3 * M / 4 + 16 * (NC / 2 - 1 - k) : 16 * (k - NC / 2); };
       uint32_t a[2][32];
       float mf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      tmem_ld32(tR, a[0]);
+      if constexpr (kBound) {
+        tmem_ld32(tR + chunk_col(0), a[0]);
+        const float U = kn[slot * kTile + r];   // >= c S[m] for every latent (bound warps)
+        tmem_wait_ld_dep(a[0]);
+        max_fold32(a[0], mf);
+        // reference: the first chunk's max, unless the bound allows a logit
+        // more than 2^kDecRefTau above it somewhere in the warp's rows; then
+        // the exact row max (pass 1 over the other chunks)
+        if (warp_any(U - c * fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3])) > kDecRefTau)) {
+          for (int cc = 1; cc < NC; ++cc) {
+            tmem_ld32(tR + chunk_col(cc), a[1]);
+            tmem_wait_ld_dep(a[1]);
+            max_fold32(a[1], mf);
+          }
+        }
+      } else {
+        // pass 1: the exact row max over all M logits
+        tmem_ld32(tR, a[0]);
 #pragma unroll
-      for (int cc = 0; cc < NC; ++cc) {
-        tmem_wait_ld_dep(a[cc & 1]);
-        if (cc + 1 < NC) tmem_ld32(tR + 32 * (cc + 1), a[(cc + 1) & 1]);
-        max_fold32(a[cc & 1], mf);
+        for (int cc = 0; cc < NC; ++cc) {
+          tmem_wait_ld_dep(a[cc & 1]);
+          if (cc + 1 < NC) tmem_ld32(tR + 32 * (cc + 1), a[(cc + 1) & 1]);
+          max_fold32(a[cc & 1], mf);
+        }
+        tmem_ld32(tR + chunk_col(0), a[0]);
       }
       const float mx = fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3]));
       const float neg = -mx * c;
       float sf[4] = {0.f, 0.f, 0.f, 0.f};
-      // pass 2 visits the chunks in the order: upper half last chunk first,
-      // then lower half first chunk first.  The P of upper chunk u (S columns
-      // [M/2 + 32u, +32)) goes to columns [3M/4 + 16u, +16), inside upper
-      // chunks already read; the P of lower chunk u goes to [16u, +16),
-      // inside lower chunks already read.  No store touches a chunk that is
-      // still to be loaded.
-      auto chunk_col = [](int k) { return k < NC / 2 ? M / 2 + 32 * (NC / 2 - 1 - k) : 32 * (k - NC / 2); };
-      auto p_col = [](int k) { return k < NC / 2 ? 3 * M / 4 + 16 * (NC / 2 - 1 - k) : 16 * (k - NC / 2); };
-      tmem_ld32(tR + chunk_col(0), a[0]);
+      // pass 2 (chunk 0 is in, or on its way to, a[0])
 #pragma unroll
       for (int k = 0; k < NC; ++k) {
-        tmem_wait_ld_dep(a[k & 1]);
+        if (k > 0 || !kBound) tmem_wait_ld_dep(a[k & 1]);
         if (k + 1 < NC) tmem_ld32(tR + chunk_col(k + 1), a[(k + 1) & 1]);
         uint32_t pk[16];
         exp_pack32<kDecPolyEvery>(a[k & 1], c, neg, pk, sf);
@@ -862,7 +968,7 @@ cudaError_t tc_decode_t(const void* Q, int64_t qbs, const void* K, const __nv_bf
   tc_decode_kernel<D, M, FLAT, VAR><<<grid, kThreads, smem, st>>>(mq, mk, mz, (int)d.H, d.N, q_per_batch,
                                                        scale * kLog2e, plan.tiles_per_bh,
                                                        plan.chunk_tiles, (__nv_bfloat16*)Y, d.y,
-                                                       d.lens, err);
+                                                       (const __nv_bfloat16*)Q, d.lens, err);
   return cudaPeekAtLastError();
 }
 

@@ -376,6 +376,10 @@ __device__ __forceinline__ void max_fold32(const uint32_t (&a)[32], float (&m)[4
   }
 }
 
+// The two bf16 halves of a packed pair, widened exactly to float.
+__device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
 // 2^x on the FMA pipe, leaving the MUFU free for other exponentials.
 // Single-split range reduction x = j + f with j = round(x) (the 1.5 * 2^23
 // add puts round(x) in the low mantissa bits), f in [-1/2, 1/2]; 2^f by a

@@ -165,3 +165,22 @@ def test_encode_running_max_over_many_tiles(M, regime):
         assert_close(Z, Zo, torch.bfloat16, "Z")
         assert_close(lse, lo, torch.bfloat16, "lse")
         assert_close(Y.float().cpu().reshape(-1, D)[rows], Yo, torch.bfloat16, "Y")
+
+
+def test_decode_row_reference_mixed_within_warps():
+    # M = 256: each token row takes the first 32-logit chunk's max as its
+    # reference when c |k| max |q| is within 2^64 of it, else the warp
+    # computes the exact max.  Every 7th key scaled x40 puts rows of both
+    # kinds in every warp of a tile.
+    B, H, N, M, D = 1, 2, 3000, 256, 32
+    s = 1.0 / math.sqrt(D)
+    x = make_inputs(B, H, N, M, D, dtype=torch.bfloat16, seed=27)
+    x["K"][:, :, ::7] = (x["K"][:, :, ::7].float() * 40.0).to(torch.bfloat16)
+    g = {k: v.to(DEV) for k, v in x.items()}
+    ws = fl.alloc_workspace(fl.FLARE_OP_FWD, B, H, N, M, D, torch.bfloat16, DEV)
+    Y, Z, lse = fl.flare_fwd(g["Q"], g["K"], g["V"], s, save=True, workspace=ws)
+    assert fl.device_status(ws) == 0
+    Yo, Zo, _ = oracle.flare_fwd(x["Q"], x["K"], x["V"], s)
+    assert torch.isfinite(Y.float()).all()
+    for sel, what in ((slice(0, None, 7), "scaled rows"), (slice(1, None, 7), "plain rows")):
+        assert rel_fro(Y[:, :, sel], Yo[:, :, sel]) <= 1e-2, what
