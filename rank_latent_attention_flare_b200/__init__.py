@@ -7,6 +7,7 @@ tensor-core kernels and CUDA-core kernels) behind the C ABI declared in
 from ._lib import (FLARE_BF16, FLARE_F32, FLARE_OP_BWD, FLARE_OP_FWD, FLARE_OP_PP_BWD,
                    FLARE_OP_PP_FWD,
                    NOALLOC_SCRATCH_BYTES, FlareError, LIB_PATH, SIGNATURES, load)
+from .autograd import FlareFunction, FlarePPFunction, flare, flare_pp
 from .flare import (alloc_workspace, bwd_path, default_scale, device_status, flare_bwd, flare_combine,
                     flare_decode, flare_encode, flare_fwd, flare_fwd_noalloc, flare_pp_bwd, flare_pp_fwd,
                     fwd_path, workspace_size)
@@ -18,4 +19,5 @@ __all__ = [
     "flare_bwd", "flare_combine", "flare_decode", "flare_encode", "flare_fwd", "flare_fwd_noalloc",
     "flare_pp_bwd", "flare_pp_fwd", "NOALLOC_SCRATCH_BYTES",
     "bwd_path", "fwd_path", "workspace_size",
+    "FlareFunction", "FlarePPFunction", "flare", "flare_pp",
 ]
