@@ -269,6 +269,60 @@ FLARE_API flare_status_t flare_decode(const void* Q, int64_t q_batch_stride, con
                             size_t workspace_bytes, void* stream);
 
 /*
+ * Context parallelism: the N tokens of every (b, h) split into equal shards,
+ * one per device (the FLARE++ page: sharding the input tokens across
+ * devices without gathering the sequence).  The encode's chunk records are
+ * the only exchange in the forward; the backward exchanges dZ and dQ.
+ * Every shard passes its own token count as N, the same on every device,
+ * contiguous token tensors and no sequence lengths.
+ *
+ * Forward, per device:
+ *   1. flare_encode on the device's shard (records land in the workspace);
+ *   2. flare_records_layout: where they are -- records_per_bh R, and the
+ *      byte offsets of ml [B*H][R][M][2] and acc [B*H][R][M][D] (float32)
+ *      in the workspace;
+ *   3. the caller gathers every shard's ml and acc, in shard order, into
+ *      [shards][B*H][R][M][2] and [shards][B*H][R][M][D] (e.g. NCCL
+ *      all-gather);
+ *   4. flare_combine_shards merges them (fixed order: shard by shard) into
+ *      the Z of the whole sequence, in the workspace and in Z_save / lse_save;
+ *   5. flare_decode on the device's shard.
+ * Backward, per device (Z_save, lse_save: the whole sequence's, from step 4):
+ *   1. flare_bwd_shard_dz: the decode stage over the shard's tokens; writes
+ *      the shard's part of dZ (float32 [B,H,M,D]);
+ *   2. the caller sums the parts over the shards (e.g. NCCL all-reduce);
+ *   3. flare_bwd_shard_finish on the same workspace: the shard's rows of dK
+ *      and dV, and its part of dQ (float32, [H,M,D] summed over the batch
+ *      when q_batch_stride == 0, else [B,H,M,D]) to be summed over the
+ *      shards.
+ * flare_bwd_shard_finish keeps the device error word of the first half.
+ */
+FLARE_API flare_status_t flare_records_layout(int64_t B, int64_t H, int64_t N, int64_t M,
+                                              int64_t D, flare_dtype_t dtype,
+                                              int64_t* records_per_bh, size_t* ml_offset,
+                                              size_t* acc_offset);
+FLARE_API flare_status_t flare_combine_shards(int64_t shards, const float* ml, const float* acc,
+                                              int64_t records_per_bh, int64_t B, int64_t H,
+                                              int64_t N, int64_t M, int64_t D,
+                                              flare_dtype_t dtype, float* Z_save,
+                                              float* lse_save, void* workspace,
+                                              size_t workspace_bytes, void* stream);
+FLARE_API flare_status_t flare_bwd_shard_dz(const void* Q, int64_t q_batch_stride, const void* K,
+                                            const void* V, const void* dY, const float* Z_save,
+                                            const float* lse_save, float* dZ_part, int64_t B,
+                                            int64_t H, int64_t N, int64_t M, int64_t D,
+                                            flare_dtype_t dtype, float scale, void* workspace,
+                                            size_t workspace_bytes, void* stream);
+FLARE_API flare_status_t flare_bwd_shard_finish(const void* Q, int64_t q_batch_stride,
+                                                const void* K, const void* V, const void* dY,
+                                                const float* Z_save, const float* lse_save,
+                                                const float* dZ, float* dQ_part, void* dK,
+                                                void* dV, int64_t B, int64_t H, int64_t N,
+                                                int64_t M, int64_t D, flare_dtype_t dtype,
+                                                float scale, void* workspace,
+                                                size_t workspace_bytes, void* stream);
+
+/*
  * Size of the fixed scratch array behind flare_fwd_noalloc (32 MiB).  Every
  * GPU that loads this library holds one such array until the process exits.
  */

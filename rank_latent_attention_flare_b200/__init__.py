@@ -8,9 +8,11 @@ from ._lib import (FLARE_BF16, FLARE_F32, FLARE_OP_BWD, FLARE_OP_FWD, FLARE_OP_P
                    FLARE_OP_PP_FWD,
                    NOALLOC_SCRATCH_BYTES, FlareError, LIB_PATH, SIGNATURES, load)
 from .autograd import FlareFunction, FlarePPFunction, flare, flare_pp
-from .flare import (alloc_workspace, bwd_path, default_scale, device_status, flare_bwd, flare_combine,
-                    flare_decode, flare_encode, flare_fwd, flare_fwd_noalloc, flare_pp_bwd, flare_pp_fwd,
-                    fwd_path, workspace_size)
+from .flare import (alloc_workspace, bwd_path, default_scale, device_status, encode_records,
+                    flare_bwd, flare_bwd_shard_dz, flare_bwd_shard_finish, flare_combine,
+                    flare_combine_shards, flare_decode, flare_encode, flare_fwd, flare_fwd_noalloc,
+                    flare_pp_bwd, flare_pp_fwd, fwd_path, records_layout, workspace_size)
+from . import parallel
 
 __all__ = [
     "FLARE_BF16", "FLARE_F32", "FLARE_OP_BWD", "FLARE_OP_FWD", "FLARE_OP_PP_BWD",
@@ -20,4 +22,6 @@ __all__ = [
     "flare_pp_bwd", "flare_pp_fwd", "NOALLOC_SCRATCH_BYTES",
     "bwd_path", "fwd_path", "workspace_size",
     "FlareFunction", "FlarePPFunction", "flare", "flare_pp",
+    "encode_records", "flare_bwd_shard_dz", "flare_bwd_shard_finish", "flare_combine_shards",
+    "records_layout", "parallel",
 ]

@@ -38,6 +38,8 @@ _i32 = ctypes.c_int
 _f32 = ctypes.c_float
 _sz = ctypes.c_size_t
 _u32p = ctypes.POINTER(ctypes.c_uint32)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+_szp = ctypes.POINTER(ctypes.c_size_t)
 
 
 class FlareStrides(ctypes.Structure):
@@ -69,6 +71,13 @@ SIGNATURES = {
                                  _i64, _i64, _i64, _i64, _i32, _f32, _vp, _sz, _vp]),
     "flare_pp_bwd_ex": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _stp, _vp, _i64,
                                     _i64, _i64, _i64, _i64, _i32, _f32, _vp, _sz, _vp]),
+    "flare_records_layout": (_i32, [_i64, _i64, _i64, _i64, _i64, _i32, _i64p, _szp, _szp]),
+    "flare_combine_shards": (_i32, [_i64, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _i32, _vp,
+                                    _vp, _vp, _sz, _vp]),
+    "flare_bwd_shard_dz": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
+                                  _i64, _i32, _f32, _vp, _sz, _vp]),
+    "flare_bwd_shard_finish": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
+                                      _i64, _i64, _i64, _i64, _i32, _f32, _vp, _sz, _vp]),
     "flare_encode": (_i32, [_vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i32, _f32, _vp,
                             _sz, _vp]),
     "flare_combine": (_i32, [_i64, _i64, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _sz, _vp]),

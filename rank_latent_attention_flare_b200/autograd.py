@@ -6,11 +6,13 @@ flare_pp_bwd.  Both directions run in libflare.so.
 """
 from __future__ import annotations
 
+import importlib
 from typing import Optional
 
 import torch
 
-from . import flare as _f
+# the binding module (the package's `flare` attribute is the autograd function)
+_f = importlib.import_module(__package__ + ".flare")
 
 
 def _token_grad(t: torch.Tensor) -> torch.Tensor:

@@ -163,7 +163,7 @@ flare_status_t run_encode(const void* Q, int64_t qbs, const void* K, const void*
 flare_status_t run_combine(const Dims& d, flare_dtype_t dt, float* Z_save, float* lse_save,
                            const void* Qpp, void* Qdyn, const WsLayout& L, char* ws,
                            cudaStream_t st) {
-  FLARE_CUDA(launch_combine(d, dt, L.enc.slots_per_bh(), (const float*)(ws + L.part_ml),
+  FLARE_CUDA(launch_combine(d, dt, L.enc.slots_per_bh(), 1, (const float*)(ws + L.part_ml),
                             (const float*)(ws + L.part_acc), (float*)(ws + L.zf),
                             (__nv_bfloat16*)(ws + L.zb), Z_save, lse_save, Qpp, Qdyn, st));
   return FLARE_OK;
@@ -179,6 +179,25 @@ flare_status_t run_decode(const void* Q, int64_t qbs, const void* K, void* Y, co
   else
     FLARE_CUDA(launch_simt_decode(Q, qbs, K, (const float*)(ws + L.zf), Y, d, dt, scale, st));
   return FLARE_OK;
+}
+
+// Validation shared by the two halves of a sharded backward.
+flare_status_t check_bwd_shard(const void* Q, int64_t qbs, const void* K, const void* V,
+                                      const void* dY, const float* Z_save, const float* lse_save,
+                                      int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
+                                      flare_dtype_t dt, float scale, void* workspace,
+                                      size_t workspace_bytes, WsLayout* L) {
+  FLARE_TRY(check_sizes(B, H, N, M, D, dt));
+  FLARE_TRY(check_scale(scale));
+  FLARE_TRY(check_ptr(Q));
+  FLARE_TRY(check_ptr(K));
+  FLARE_TRY(check_ptr(V));
+  FLARE_TRY(check_ptr(dY));
+  FLARE_TRY(check_ptr(Z_save));
+  FLARE_TRY(check_ptr(lse_save));
+  FLARE_TRY(check_qbs(qbs, H, M, D));
+  *L = ws_layout(FLARE_OP_BWD, B, H, N, M, D, dt, current_sm_count());
+  return check_ws(workspace, workspace_bytes, L->total);
 }
 
 // Order of the flare_strides_t entries: forward K, V, Y; backward K, V,
@@ -453,6 +472,78 @@ flare_status_t flare_pp_bwd(const void* Q, const void* K, const void* V, const v
                             size_t workspace_bytes, void* stream) {
   return flare_pp_bwd_ex(Q, K, V, dY, Q_dyn, Z_save, lse_save, dQ, dK, dV, nullptr, nullptr, B, H, N,
                               M, D, dt, scale, workspace, workspace_bytes, stream);
+}
+
+flare_status_t flare_records_layout(int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
+                                    flare_dtype_t dt, int64_t* records_per_bh, size_t* ml_offset,
+                                    size_t* acc_offset) {
+  FLARE_TRY(check_sizes(B, H, N, M, D, dt));
+  if (!records_per_bh || !ml_offset || !acc_offset) return FLARE_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(FLARE_OP_FWD, B, H, N, M, D, dt, current_sm_count());
+  *records_per_bh = L.enc.slots_per_bh();
+  *ml_offset = L.part_ml;
+  *acc_offset = L.part_acc;
+  return FLARE_OK;
+}
+
+flare_status_t flare_combine_shards(int64_t shards, const float* ml, const float* acc,
+                                    int64_t records_per_bh, int64_t B, int64_t H, int64_t N,
+                                    int64_t M, int64_t D, flare_dtype_t dt, float* Z_save,
+                                    float* lse_save, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  FLARE_TRY(check_sizes(B, H, N, M, D, dt));
+  if (shards < 1 || shards > 65536 || records_per_bh < 1 || records_per_bh > (1 << 20))
+    return FLARE_ERR_INVALID_ARG;
+  FLARE_TRY(check_ptr(ml));
+  FLARE_TRY(check_ptr(acc));
+  FLARE_TRY(check_opt_ptr(Z_save));
+  FLARE_TRY(check_opt_ptr(lse_save));
+  const WsLayout L = ws_layout(FLARE_OP_FWD, B, H, N, M, D, dt, current_sm_count());
+  FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  g_error_detail[0] = 0;
+  char* ws = (char*)workspace;
+  FLARE_CUDA(launch_combine(Dims{B, H, N, M, D}, dt, (int)records_per_bh, (int)shards, ml, acc,
+                            (float*)(ws + L.zf), (__nv_bfloat16*)(ws + L.zb), Z_save, lse_save,
+                            nullptr, nullptr, (cudaStream_t)stream));
+  return FLARE_OK;
+}
+
+flare_status_t flare_bwd_shard_dz(const void* Q, int64_t qbs, const void* K, const void* V,
+                                  const void* dY, const float* Z_save, const float* lse_save,
+                                  float* dZ_part, int64_t B, int64_t H, int64_t N, int64_t M,
+                                  int64_t D, flare_dtype_t dt, float scale, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  WsLayout L;
+  FLARE_TRY(check_bwd_shard(Q, qbs, K, V, dY, Z_save, lse_save, B, H, N, M, D, dt, scale,
+                            workspace, workspace_bytes, &L));
+  FLARE_TRY(check_ptr(dZ_part));
+  char* ws = (char*)workspace;
+  cudaStream_t st = (cudaStream_t)stream;
+  FLARE_TRY(reset_error_word(ws, st));
+  FLARE_CUDA(launch_bwd(Q, qbs, K, V, dY, Z_save, lse_save, nullptr, nullptr, nullptr,
+                        Dims{B, H, N, M, D}, dt, scale, L, ws, st, BwdPhase::DZ, dZ_part,
+                        nullptr));
+  return FLARE_OK;
+}
+
+flare_status_t flare_bwd_shard_finish(const void* Q, int64_t qbs, const void* K, const void* V,
+                                      const void* dY, const float* Z_save, const float* lse_save,
+                                      const float* dZ, float* dQ_part, void* dK, void* dV,
+                                      int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
+                                      flare_dtype_t dt, float scale, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  WsLayout L;
+  FLARE_TRY(check_bwd_shard(Q, qbs, K, V, dY, Z_save, lse_save, B, H, N, M, D, dt, scale,
+                            workspace, workspace_bytes, &L));
+  FLARE_TRY(check_ptr(dZ));
+  FLARE_TRY(check_ptr(dQ_part));
+  FLARE_TRY(check_ptr(dK));
+  FLARE_TRY(check_ptr(dV));
+  g_error_detail[0] = 0;   // the error word keeps what the first half recorded
+  FLARE_CUDA(launch_bwd(Q, qbs, K, V, dY, Z_save, lse_save, nullptr, dK, dV, Dims{B, H, N, M, D},
+                        dt, scale, L, (char*)workspace, (cudaStream_t)stream, BwdPhase::FINISH,
+                        const_cast<float*>(dZ), dQ_part));
+  return FLARE_OK;
 }
 
 flare_status_t flare_device_status(void* workspace, size_t workspace_bytes, uint32_t* detail,

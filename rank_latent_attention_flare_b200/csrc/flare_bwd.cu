@@ -302,7 +302,8 @@ __global__ void reduce_dq_kernel(const float* __restrict__ dq_dec, const float* 
 template <typename T, int D>
 cudaError_t bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, const void* dY,
                   const float* Z, const float* lse, void* dQ, void* dK, void* dV, const Dims& d,
-                  float scale, const WsLayout& L, char* ws, cudaStream_t st) {
+                  float scale, const WsLayout& L, char* ws, cudaStream_t st, BwdPhase phase,
+                  float* dz_io, float* dq32) {
   const ChunkPlan& p = L.bwd;
   const int M = (int)d.M;
   const float c = scale * kLog2e;
@@ -314,20 +315,29 @@ cudaError_t bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, cons
   float* dz = (float*)(ws + L.dz);
   float* delta = (float*)(ws + L.delta);
   dim3 grid(p.chunks, (unsigned)d.BH());
-
-  const size_t smemA = (size_t)(2 * M * D + 2 * kT * D + 3 * kT) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(bwd_decode_kernel<T, D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemA);
-  if (e != cudaSuccess) return e;
-  bwd_decode_kernel<T, D><<<grid, kT, smemA, st>>>((const T*)Q, qbs, (const T*)K, (const T*)dY, d.k,
-                                                   d.dy, d.lens, Z, (int)d.H, d.N, M, c, scale,
-                                                   p.chunk_tokens(), dkf, dq_dec, dzp);
-  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
-
+  cudaError_t e;
   const int64_t warps = d.BH() * M;
-  reduce_dz_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(dzp, Z, d.BH(), M, D,
-                                                                          p.chunks, dz, delta);
-  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+
+  if (phase != BwdPhase::FINISH) {
+    const size_t smemA = (size_t)(2 * M * D + 2 * kT * D + 3 * kT) * sizeof(float);
+    e = cudaFuncSetAttribute(bwd_decode_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smemA);
+    if (e != cudaSuccess) return e;
+    bwd_decode_kernel<T, D><<<grid, kT, smemA, st>>>((const T*)Q, qbs, (const T*)K, (const T*)dY,
+                                                     d.k, d.dy, d.lens, Z, (int)d.H, d.N, M, c,
+                                                     scale, p.chunk_tokens(), dkf, dq_dec, dzp);
+    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+    // dZ (this device's tokens) and delta_e = rowsum(dZ * Z)
+    reduce_dz_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(
+        dzp, Z, d.BH(), M, D, p.chunks, phase == BwdPhase::DZ ? dz_io : dz, delta);
+    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+    if (phase == BwdPhase::DZ) return cudaSuccess;
+  } else {
+    // dZ summed over the shards: delta_e from it
+    reduce_dz_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(
+        dz_io, Z, d.BH(), M, D, 1, dz, delta);
+    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+  }
 
   const size_t smemB = (size_t)(2 * M * D + 2 * M + 2 * kT * D) * sizeof(float);
   e = cudaFuncSetAttribute(bwd_encode_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -341,8 +351,12 @@ cudaError_t bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, cons
 
   const bool shared_q = (qbs == 0);
   const int64_t total = shared_q ? d.H * M * D : d.BH() * M * D;
-  reduce_dq_kernel<T><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
-      dq_dec, dq_enc, (int)d.B, (int)d.H, M, D, p.chunks, shared_q, (T*)dQ);
+  if (dq32)
+    reduce_dq_kernel<float><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
+        dq_dec, dq_enc, (int)d.B, (int)d.H, M, D, p.chunks, shared_q, dq32);
+  else
+    reduce_dq_kernel<T><<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
+        dq_dec, dq_enc, (int)d.B, (int)d.H, M, D, p.chunks, shared_q, (T*)dQ);
   return cudaPeekAtLastError();
 }
 
@@ -351,15 +365,15 @@ cudaError_t bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, cons
 cudaError_t launch_bwd(const void* Q, int64_t qbs, const void* K, const void* V, const void* dY,
                        const float* Z, const float* lse, void* dQ, void* dK, void* dV,
                        const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,
-                       char* ws, cudaStream_t st) {
+                       char* ws, cudaStream_t st, BwdPhase phase, float* dz, float* dq32) {
   if (choose_path(d.N, d.M, d.D, dt).tc_bwd)
-    return launch_tc_bwd(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
-  if (dt == FLARE_F32)
-    return d.D == 16 ? bwd_t<float, 16>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st)
-                     : bwd_t<float, 32>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
-  return d.D == 16
-             ? bwd_t<__nv_bfloat16, 16>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st)
-             : bwd_t<__nv_bfloat16, 32>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
+    return launch_tc_bwd(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st, phase, dz,
+                         dq32);
+#define FLARE_BWD_T(T, DD) \
+  bwd_t<T, DD>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st, phase, dz, dq32)
+  if (dt == FLARE_F32) return d.D == 16 ? FLARE_BWD_T(float, 16) : FLARE_BWD_T(float, 32);
+  return d.D == 16 ? FLARE_BWD_T(__nv_bfloat16, 16) : FLARE_BWD_T(__nv_bfloat16, 32);
+#undef FLARE_BWD_T
 }
 
 }  // namespace flare

@@ -347,7 +347,7 @@ cudaError_t launch_check_lens(const Dims& d, uint32_t* err, cudaStream_t st);
 // d.lens is NULL).
 cudaError_t launch_zero_padding(void* X0, const Tok& t0, void* X1, const Tok& t1, const Dims& d,
                                 flare_dtype_t dt, cudaStream_t st);
-cudaError_t launch_combine(const Dims& d, flare_dtype_t dt, int slots_per_bh,
+cudaError_t launch_combine(const Dims& d, flare_dtype_t dt, int slots_per_bh, int groups,
                            const float* part_ml, const float* part_acc, float* Zf,
                            __nv_bfloat16* Zb, float* Z_save, float* lse_save, const void* Qpp,
                            void* Qdyn, cudaStream_t st);
@@ -380,10 +380,19 @@ inline bool tok_flat(const Dims& d) {
 cudaError_t make_tok_map(CUtensorMap* m, const void* base, const Dims& d, const Tok& t,
                          int box_rows, bool flat);
 
+// Which part of the backward a call runs.  With the tokens sharded (context
+// parallelism) each shard runs DZ (the decode stage over its tokens, then
+// its part of dZ, written to `dz`), the shards' parts are summed, and each
+// runs FINISH (the encode stage over its tokens given the summed dZ in `dz`:
+// its rows of dK, dV and its fp32 part of dQ in `dq32`) on the same
+// workspace.  ALL is the whole backward on one device.
+enum class BwdPhase { ALL, DZ, FINISH };
+
 cudaError_t launch_tc_bwd(const void* Q, int64_t qbs, const void* K, const void* V,
                           const void* dY, const float* Z, const float* lse, void* dQ, void* dK,
                           void* dV, const Dims& d, float scale, const WsLayout& L, char* ws,
-                          cudaStream_t st);
+                          cudaStream_t st, BwdPhase phase = BwdPhase::ALL, float* dz = nullptr,
+                          float* dq32 = nullptr);
 // FLARE++'s first-encode gradient on the tensor cores (bf16, M = 128,
 // D in {16, 32}): adds into dK, dV and writes dQ (sum over the batch of dZ1
 // and the encode's dQ); reuses the tensor-core backward's workspace.
@@ -398,6 +407,7 @@ cudaError_t launch_pp_bwd_tail(const void* Q, const void* K, const void* V, cons
 cudaError_t launch_bwd(const void* Q, int64_t qbs, const void* K, const void* V, const void* dY,
                        const float* Z, const float* lse, void* dQ, void* dK, void* dV,
                        const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,
-                       char* ws, cudaStream_t st);
+                       char* ws, cudaStream_t st, BwdPhase phase = BwdPhase::ALL,
+                       float* dz = nullptr, float* dq32 = nullptr);
 
 }  // namespace flare

@@ -142,11 +142,13 @@ __global__ void __launch_bounds__(kSimtDecThreads)
 
 // One warp per (b, h, m); lane d < D owns Z[m][d].  Merges the per-chunk
 // (max, sum, acc) records with the log-sum-exp rule and, for FLARE++,
-// writes Q_dyn = Q + Z in the input dtype.
+// writes Q_dyn = Q + Z in the input dtype.  The records are `groups` blocks
+// of [BH][slots] (one block per token shard when the tokens were encoded in
+// shards), merged in a fixed order: block by block, slot by slot.
 template <typename T>
 __global__ void combine_kernel(const float* __restrict__ part_ml,
                                const float* __restrict__ part_acc, int64_t BH, int H, int M,
-                               int D, int slots, float* __restrict__ Zf,
+                               int D, int slots, int groups, float* __restrict__ Zf,
                                __nv_bfloat16* __restrict__ Zb, float* __restrict__ Z_save,
                                float* __restrict__ lse_save, const T* __restrict__ Qpp,
                                T* __restrict__ Qdyn) {
@@ -156,17 +158,19 @@ __global__ void combine_kernel(const float* __restrict__ part_ml,
   const int64_t bh = w / M;
   const int m = (int)(w % M);
   float mstar = -INFINITY;
-  for (int s = 0; s < slots; ++s)
-    mstar = fmaxf(mstar, part_ml[((bh * slots + s) * M + m) * 2]);
+  for (int g = 0; g < groups; ++g)
+    for (int s = 0; s < slots; ++s)
+      mstar = fmaxf(mstar, part_ml[(((g * BH + bh) * slots + s) * M + m) * 2]);
   float l = 0.f, acc = 0.f;
-  for (int s = 0; s < slots; ++s) {
-    const int64_t row = (bh * slots + s) * M + m;
-    const float ms = part_ml[row * 2];
-    if (ms == -INFINITY) continue;  // empty record
-    const float f = exp2f(ms - mstar);
-    l = fmaf(f, part_ml[row * 2 + 1], l);
-    if (lane < D) acc = fmaf(f, part_acc[row * D + lane], acc);
-  }
+  for (int g = 0; g < groups; ++g)
+    for (int s = 0; s < slots; ++s) {
+      const int64_t row = ((g * BH + bh) * slots + s) * M + m;
+      const float ms = part_ml[row * 2];
+      if (ms == -INFINITY) continue;  // empty record
+      const float f = exp2f(ms - mstar);
+      l = fmaf(f, part_ml[row * 2 + 1], l);
+      if (lane < D) acc = fmaf(f, part_acc[row * D + lane], acc);
+    }
   if (lane < D) {
     const float z = (l > 0.f) ? acc / l : 0.f;   // no tokens: an empty weighted sum
     const int64_t o = w * D + lane;
@@ -274,7 +278,7 @@ cudaError_t launch_zero_padding(void* X0, const Tok& t0, void* X1, const Tok& t1
   return cudaPeekAtLastError();
 }
 
-cudaError_t launch_combine(const Dims& d, flare_dtype_t dt, int slots_per_bh,
+cudaError_t launch_combine(const Dims& d, flare_dtype_t dt, int slots_per_bh, int groups,
                            const float* part_ml, const float* part_acc, float* Zf,
                            __nv_bfloat16* Zb, float* Z_save, float* lse_save, const void* Qpp,
                            void* Qdyn, cudaStream_t st) {
@@ -283,11 +287,11 @@ cudaError_t launch_combine(const Dims& d, flare_dtype_t dt, int slots_per_bh,
   const unsigned blocks = (unsigned)((warps * 32 + threads - 1) / threads);
   if (dt == FLARE_F32)
     combine_kernel<float><<<blocks, threads, 0, st>>>(
-        part_ml, part_acc, d.BH(), (int)d.H, (int)d.M, (int)d.D, slots_per_bh, Zf, Zb, Z_save,
+        part_ml, part_acc, d.BH(), (int)d.H, (int)d.M, (int)d.D, slots_per_bh, groups, Zf, Zb, Z_save,
         lse_save, (const float*)Qpp, (float*)Qdyn);
   else
     combine_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(
-        part_ml, part_acc, d.BH(), (int)d.H, (int)d.M, (int)d.D, slots_per_bh, Zf, Zb, Z_save,
+        part_ml, part_acc, d.BH(), (int)d.H, (int)d.M, (int)d.D, slots_per_bh, groups, Zf, Zb, Z_save,
         lse_save, (const __nv_bfloat16*)Qpp, (__nv_bfloat16*)Qdyn);
   return cudaPeekAtLastError();
 }

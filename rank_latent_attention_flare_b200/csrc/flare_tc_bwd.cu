@@ -1570,7 +1570,7 @@ __global__ void __launch_bounds__(kThr, 1)
 // [B][H][M][D] bf16) is summed over the batch first: FLARE++'s dQ_dyn.
 __global__ void bwd_dq_sum_kernel(const float4* __restrict__ dq_part, int B, int H, int M, int D,
                                   int chunks, bool shared_q, const __nv_bfloat16* __restrict__ extra,
-                                  __nv_bfloat16* __restrict__ dQ) {
+                                  __nv_bfloat16* __restrict__ dQ, float4* __restrict__ dQ32) {
   const int64_t md4 = (int64_t)M * D / 4;
   const int64_t per4 = (int64_t)H * md4;
   const int64_t total4 = shared_q ? per4 : (int64_t)B * per4;
@@ -1611,13 +1611,36 @@ __global__ void bwd_dq_sum_kernel(const float4* __restrict__ dq_part, int B, int
       }
     }
   }
-  *reinterpret_cast<uint2*>(dQ + i * 4) = make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
+  if (dQ32)
+    dQ32[i] = acc;
+  else
+    *reinterpret_cast<uint2*>(dQ + i * 4) = make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
+}
+
+// This device's dZ: the fixed-order sum over chunks of pass A's partials,
+// [BH][chunks][M][D] -> [BH][M][D].  One thread per 4 elements.
+__global__ void bwd_dz_sum_kernel(const float4* __restrict__ dz_part, int64_t BH, int M, int D,
+                                  int chunks, float4* __restrict__ dz) {
+  const int64_t md4 = (int64_t)M * D / 4;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= BH * md4) return;
+  const int64_t bh = i / md4, e = i % md4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k = 0; k < chunks; ++k) {
+    const float4 v = dz_part[(bh * chunks + k) * md4 + e];
+    acc.x += v.x;
+    acc.y += v.y;
+    acc.z += v.z;
+    acc.w += v.w;
+  }
+  dz[i] = acc;
 }
 
 template <int D, bool FLAT, bool VAR>
 cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, const void* dY,
                      const float* Z, const float* lse, void* dQ, void* dK, void* dV, const Dims& d,
-                     float scale, const WsLayout& L, char* ws, cudaStream_t st) {
+                     float scale, const WsLayout& L, char* ws, cudaStream_t st, BwdPhase phase,
+                     float* dz_io, float* dq32) {
   const ChunkPlan& p = L.bwd;
   const int64_t BH = d.BH();
   const int q_per_batch = qbs != 0;
@@ -1636,8 +1659,10 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
   float* dqp = (float*)(ws + L.dqp);
   cudaError_t e;
 
-  bwd_prep_kernel<D><<<(unsigned)BH, kM, 0, st>>>(Z, lse, zb, rref, flags);
-  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+  if (phase != BwdPhase::FINISH) {
+    bwd_prep_kernel<D><<<(unsigned)BH, kM, 0, st>>>(Z, lse, zb, rref, flags);
+    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+  }
 
   CUtensorMap mq, mk, mv, mdy, mdy2, mz, mdz, maug;
   if ((e = make_map(&mq, Q, D, kM, q_per_batch ? BH : d.H, kM)) != cudaSuccess) return e;
@@ -1650,16 +1675,27 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
   if ((e = make_map(&maug, aug, 16, kM, BH, kM)) != cudaSuccess) return e;
 
   dim3 grid(p.chunks, (unsigned)BH);
-  const int smemA = ALayout<D>::BYTES + 1024;
-  e = cudaFuncSetAttribute(tc_bwd_a_kernel<D, FLAT, VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, smemA);
-  if (e != cudaSuccess) return e;
-  tc_bwd_a_kernel<D, FLAT, VAR><<<grid, kThr, smemA, st>>>(mq, mk, mdy, mz, (int)d.H, d.N, q_per_batch, c,
-                                                p.tiles_per_bh, p.chunk_tiles, rref, stats, dy2,
-                                                flags, dzp, d.lens, err);
-  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+  if (phase != BwdPhase::FINISH) {
+    const int smemA = ALayout<D>::BYTES + 1024;
+    e = cudaFuncSetAttribute(tc_bwd_a_kernel<D, FLAT, VAR>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smemA);
+    if (e != cudaSuccess) return e;
+    tc_bwd_a_kernel<D, FLAT, VAR><<<grid, kThr, smemA, st>>>(
+        mq, mk, mdy, mz, (int)d.H, d.N, q_per_batch, c, p.tiles_per_bh, p.chunk_tiles, rref,
+        stats, dy2, flags, dzp, d.lens, err);
+    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+    if (phase == BwdPhase::DZ) {   // this device's part of dZ
+      const int64_t n4 = BH * kM * D / 4;
+      bwd_dz_sum_kernel<<<(unsigned)((n4 + 127) / 128), 128, 0, st>>>(
+          (const float4*)dzp, BH, kM, D, p.chunks, (float4*)dz_io);
+      return cudaPeekAtLastError();
+    }
+  }
 
-  bwd_mid_kernel<D><<<(unsigned)BH, kM, 0, st>>>(dzp, p.chunks, nullptr, Z, lse, dzs,
-                                                 (uint32_t*)aug, flags, params, lse2);
+  // dZ: the chunk partials, or (FINISH) the sum over the shards as one partial
+  bwd_mid_kernel<D><<<(unsigned)BH, kM, 0, st>>>(phase == BwdPhase::FINISH ? dz_io : dzp,
+                                                 phase == BwdPhase::FINISH ? 1 : p.chunks, nullptr,
+                                                 Z, lse, dzs, (uint32_t*)aug, flags, params, lse2);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
   // each head runs in exactly one of the two pass-B kernels (params.y)
@@ -1688,7 +1724,7 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
   const int64_t total = shared_q ? d.H * kM * D : BH * kM * D;
   bwd_dq_sum_kernel<<<(unsigned)((total / 4 + 127) / 128), 128, 0, st>>>(
       (const float4*)dqp, (int)d.B, (int)d.H, kM, D, p.chunks, shared_q, nullptr,
-      (__nv_bfloat16*)dQ);
+      (__nv_bfloat16*)dQ, (float4*)dq32);
   return cudaPeekAtLastError();
 }
 
@@ -1758,7 +1794,7 @@ cudaError_t tc_enc_bwd_t(const void* Q, const void* K, const void* V, const floa
   const int64_t total = d.H * kM * D;
   bwd_dq_sum_kernel<<<(unsigned)((total / 4 + 127) / 128), 128, 0, st>>>(
       (const float4*)dqp, (int)d.B, (int)d.H, kM, D, p.chunks, true,
-      (const __nv_bfloat16*)dZ1, (__nv_bfloat16*)dQ);
+      (const __nv_bfloat16*)dZ1, (__nv_bfloat16*)dQ, nullptr);
   return cudaPeekAtLastError();
 }
 
@@ -1766,13 +1802,13 @@ template <int D>
 cudaError_t tc_bwd_dispatch(const void* Q, int64_t qbs, const void* K, const void* V,
                             const void* dY, const float* Z, const float* lse, void* dQ, void* dK,
                             void* dV, const Dims& d, float scale, const WsLayout& L, char* ws,
-                            cudaStream_t st) {
+                            cudaStream_t st, BwdPhase ph, float* dz, float* dq32) {
   const bool flat = tok_flat(d), var = d.lens != nullptr;
-  if (flat)
-    return var ? tc_bwd_t<D, true, true>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st)
-               : tc_bwd_t<D, true, false>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
-  return var ? tc_bwd_t<D, false, true>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st)
-             : tc_bwd_t<D, false, false>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
+#define FLARE_TC_BWD_T(F, V_) \
+  tc_bwd_t<D, F, V_>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st, ph, dz, dq32)
+  if (flat) return var ? FLARE_TC_BWD_T(true, true) : FLARE_TC_BWD_T(true, false);
+  return var ? FLARE_TC_BWD_T(false, true) : FLARE_TC_BWD_T(false, false);
+#undef FLARE_TC_BWD_T
 }
 
 template <int D>
@@ -1793,10 +1829,14 @@ cudaError_t tc_enc_bwd_dispatch(const void* Q, const void* K, const void* V, con
 cudaError_t launch_tc_bwd(const void* Q, int64_t qbs, const void* K, const void* V,
                           const void* dY, const float* Z, const float* lse, void* dQ, void* dK,
                           void* dV, const Dims& d, float scale, const WsLayout& L, char* ws,
-                          cudaStream_t st) {
+                          cudaStream_t st, BwdPhase phase, float* dz, float* dq32) {
   if (d.M != kM) return cudaErrorNotSupported;
-  if (d.D == 32) return tc_bwd_dispatch<32>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
-  if (d.D == 16) return tc_bwd_dispatch<16>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st);
+  if (d.D == 32)
+    return tc_bwd_dispatch<32>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st, phase,
+                               dz, dq32);
+  if (d.D == 16)
+    return tc_bwd_dispatch<16>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st, phase,
+                               dz, dq32);
   return cudaErrorNotSupported;
 }
 

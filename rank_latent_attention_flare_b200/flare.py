@@ -326,3 +326,79 @@ def flare_fwd_noalloc(Q, K, V, scale: Optional[float] = None, *, save: bool = Fa
         raise FlareError(st, "flare_fwd_noalloc" + (f" [{detail}]" if detail else ""))
     _lib.check(st, "flare_fwd_noalloc")
     return (Y, Z, lse) if save else Y
+
+
+# ------------------------------------------------- context parallelism (stages)
+
+def records_layout(B: int, H: int, N: int, M: int, D: int, dtype: torch.dtype):
+    """(records_per_bh, ml_offset, acc_offset): where flare_encode leaves its
+    chunk records in a FLARE_OP_FWD workspace."""
+    code = _lib.FLARE_F32 if dtype == torch.float32 else _lib.FLARE_BF16
+    r, mo, ao = ctypes.c_int64(0), ctypes.c_size_t(0), ctypes.c_size_t(0)
+    st = _lib.load().flare_records_layout(B, H, N, M, D, code, ctypes.byref(r),
+                                          ctypes.byref(mo), ctypes.byref(ao))
+    _lib.check(st, "flare_records_layout")
+    return int(r.value), int(mo.value), int(ao.value)
+
+
+def encode_records(workspace: torch.Tensor, B: int, H: int, N: int, M: int, D: int,
+                   dtype: torch.dtype):
+    """Views of the records flare_encode left in ``workspace``: ml
+    [B*H, R, M, 2] (running max in log2 units, sum) and acc [B*H, R, M, D],
+    float32."""
+    R, mo, ao = records_layout(B, H, N, M, D, dtype)
+    n_ml, n_acc = B * H * R * M * 2 * 4, B * H * R * M * D * 4
+    ml = workspace[mo:mo + n_ml].view(torch.float32).view(B * H, R, M, 2)
+    acc = workspace[ao:ao + n_acc].view(torch.float32).view(B * H, R, M, D)
+    return ml, acc
+
+
+def flare_combine_shards(ml: torch.Tensor, acc: torch.Tensor, B: int, H: int, N: int, M: int,
+                         D: int, dtype: torch.dtype, *, workspace: torch.Tensor,
+                         Z_save: Optional[torch.Tensor] = None,
+                         lse_save: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Merges the gathered records of every shard (ml [shards, B*H, R, M, 2],
+    acc [shards, B*H, R, M, D]) into the whole sequence's Z, left in
+    ``workspace`` for flare_decode (and written to Z_save / lse_save)."""
+    _need_cuda(ml, acc, workspace, Z_save, lse_save)
+    if ml.dim() != 5 or acc.dim() != 5 or ml.shape[:4] != acc.shape[:4]:
+        raise ValueError("ml must be [shards, B*H, R, M, 2] and acc [shards, B*H, R, M, D]")
+    code = _lib.FLARE_F32 if dtype == torch.float32 else _lib.FLARE_BF16
+    st = _lib.load().flare_combine_shards(ml.shape[0], _ptr(ml), _ptr(acc), ml.shape[2], B, H, N,
+                                          M, D, code, _ptr(Z_save), _ptr(lse_save),
+                                          _ptr(workspace), workspace.numel(), _stream(stream))
+    _lib.check(st, "flare_combine_shards")
+
+
+def flare_bwd_shard_dz(Q, K, V, dY, Z, lse, scale: Optional[float] = None, *,
+                       workspace: torch.Tensor, stream=None) -> torch.Tensor:
+    """First half of a sharded backward: the decode stage over this shard's
+    tokens.  Returns the shard's part of dZ (float32 [B,H,M,D]); keep
+    ``workspace`` (FLARE_OP_BWD size) for flare_bwd_shard_finish."""
+    _need_cuda(Q, K, V, dY, Z, lse, workspace)
+    B, H, N, M, D, qbs = _dims(Q, K)
+    s = default_scale(D) if scale is None else float(scale)
+    dZ = torch.empty((B, H, M, D), dtype=torch.float32, device=K.device)
+    st = _lib.load().flare_bwd_shard_dz(_ptr(Q), qbs, _ptr(K), _ptr(V), _ptr(dY), _ptr(Z),
+                                        _ptr(lse), _ptr(dZ), B, H, N, M, D, _dtype_code(K), s,
+                                        _ptr(workspace), workspace.numel(), _stream(stream))
+    _lib.check(st, "flare_bwd_shard_dz")
+    return dZ
+
+
+def flare_bwd_shard_finish(Q, K, V, dY, Z, lse, dZ, scale: Optional[float] = None, *,
+                           workspace: torch.Tensor, stream=None):
+    """Second half, given dZ summed over the shards: returns (the shard's
+    float32 part of dQ, its rows of dK, dV)."""
+    _need_cuda(Q, K, V, dY, Z, lse, dZ, workspace)
+    B, H, N, M, D, qbs = _dims(Q, K)
+    s = default_scale(D) if scale is None else float(scale)
+    dQ = torch.empty(Q.shape, dtype=torch.float32, device=K.device)
+    dK = torch.empty_like(K)
+    dV = torch.empty_like(V)
+    st = _lib.load().flare_bwd_shard_finish(_ptr(Q), qbs, _ptr(K), _ptr(V), _ptr(dY), _ptr(Z),
+                                            _ptr(lse), _ptr(dZ), _ptr(dQ), _ptr(dK), _ptr(dV), B,
+                                            H, N, M, D, _dtype_code(K), s, _ptr(workspace),
+                                            workspace.numel(), _stream(stream))
+    _lib.check(st, "flare_bwd_shard_finish")
+    return dQ, dK, dV

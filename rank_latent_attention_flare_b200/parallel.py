@@ -1,0 +1,63 @@
+"""Context parallelism over torch.distributed: every rank holds an equal
+shard of each sequence's tokens (the FLARE++ page: the input tokens sharded
+across devices, never gathered).
+
+Forward: each rank encodes its shard into chunk records, the records are
+all-gathered (the only exchange), every rank merges them into the whole
+sequence's Z and decodes its own tokens.  Backward: each rank's part of dZ
+is all-reduced between the decode and the encode stage, and the parts of dQ
+at the end.  Argument marshalling and collectives only: the math runs in
+libflare.so.  ``ops`` defaults to this package's stage calls; the
+multi-process CPU tests pass stand-ins with the same signatures.
+"""
+from __future__ import annotations
+
+import importlib
+from typing import Optional
+
+import torch
+import torch.distributed as dist
+
+# the binding module (the package's `flare` attribute is the autograd function)
+_f = importlib.import_module(__package__ + ".flare")
+
+
+def cp_flare_fwd(Q, K, V, scale: Optional[float] = None, *, group=None, save: bool = False,
+                 ops=_f):
+    """K, V: this rank's shard [B,H,N_r,D] of every sequence (the same N_r on
+    every rank; shards in rank order).  Returns this rank's Y shard, or
+    (Y, Z, lse) of the whole sequence when ``save``."""
+    B, H, N, M, D, _ = _f._dims(Q, K)
+    s = _f.default_scale(D) if scale is None else float(scale)
+    ws = ops.alloc_workspace(_f._lib.FLARE_OP_FWD, B, H, N, M, D, K.dtype, K.device)
+    ops.flare_encode(Q, K, V, s, workspace=ws)
+    ml, acc = ops.encode_records(ws, B, H, N, M, D, K.dtype)
+    G = dist.get_world_size(group)
+    # gathered along the first dimension (rank order), then viewed as [shards, ...]
+    gml = torch.empty((G * ml.shape[0],) + tuple(ml.shape[1:]), dtype=ml.dtype, device=ml.device)
+    gacc = torch.empty((G * acc.shape[0],) + tuple(acc.shape[1:]), dtype=acc.dtype,
+                       device=acc.device)
+    dist.all_gather_into_tensor(gml, ml.contiguous(), group=group)
+    dist.all_gather_into_tensor(gacc, acc.contiguous(), group=group)
+    gml = gml.view((G,) + tuple(ml.shape))
+    gacc = gacc.view((G,) + tuple(acc.shape))
+    Z = torch.empty((B, H, M, D), dtype=torch.float32, device=K.device)
+    lse = torch.empty((B, H, M), dtype=torch.float32, device=K.device)
+    ops.flare_combine_shards(gml, gacc, B, H, N, M, D, K.dtype, workspace=ws, Z_save=Z,
+                             lse_save=lse)
+    Y = ops.flare_decode(Q, K, s, workspace=ws)
+    return (Y, Z, lse) if save else Y
+
+
+def cp_flare_bwd(Q, K, V, dY, Z, lse, scale: Optional[float] = None, *, group=None, ops=_f):
+    """Gradients for this rank's shard (Z, lse: the whole sequence's, from
+    cp_flare_fwd(save=True)).  Returns (dQ summed over the shards, in Q's
+    dtype; this shard's dK, dV)."""
+    B, H, N, M, D, _ = _f._dims(Q, K)
+    s = _f.default_scale(D) if scale is None else float(scale)
+    ws = ops.alloc_workspace(_f._lib.FLARE_OP_BWD, B, H, N, M, D, K.dtype, K.device)
+    dZ = ops.flare_bwd_shard_dz(Q, K, V, dY, Z, lse, s, workspace=ws)
+    dist.all_reduce(dZ, group=group)
+    dQ, dK, dV = ops.flare_bwd_shard_finish(Q, K, V, dY, Z, lse, dZ, s, workspace=ws)
+    dist.all_reduce(dQ, group=group)
+    return dQ.to(Q.dtype), dK, dV
