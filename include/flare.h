@@ -296,6 +296,20 @@ FLARE_API flare_status_t flare_decode(const void* Q, int64_t q_batch_stride, con
  *      when q_batch_stride == 0, else [B,H,M,D]) to be summed over the
  *      shards.
  * flare_bwd_shard_finish keeps the device error word of the first half.
+ *
+ * FLARE++ (learned latents Q [H,M,D]):
+ *   forward: the steps above for the first encode, with Q_learned = Q and
+ *   Q_dyn_out given to flare_combine_shards (which then also writes
+ *   Q_dyn = Q + Z1, [B,H,M,D] in the input dtype), then the steps above with
+ *   Q_dyn as per-batch latents;
+ *   backward: the first encode recomputed as in the forward (its Z1, lse1 of
+ *   the whole sequence into Z_save / lse_save); the backward steps above with
+ *   Q_dyn, on a FLARE_OP_PP_BWD workspace, giving dQ_dyn after the sum over
+ *   the shards; then flare_pp_bwd_shard_tail with that dQ_dyn (input dtype)
+ *   on the same workspace: the first encode's gradient over the shard, added
+ *   to the shard's dK and dV, and its float32 part of dQ [H,M,D] (summed
+ *   over the batch).  dQ = the sum over the shards of those parts + the sum
+ *   over the batch of dQ_dyn.
  */
 FLARE_API flare_status_t flare_records_layout(int64_t B, int64_t H, int64_t N, int64_t M,
                                               int64_t D, flare_dtype_t dtype,
@@ -305,7 +319,8 @@ FLARE_API flare_status_t flare_combine_shards(int64_t shards, const float* ml, c
                                               int64_t records_per_bh, int64_t B, int64_t H,
                                               int64_t N, int64_t M, int64_t D,
                                               flare_dtype_t dtype, float* Z_save,
-                                              float* lse_save, void* workspace,
+                                              float* lse_save, const void* Q_learned,
+                                              void* Q_dyn_out, void* workspace,
                                               size_t workspace_bytes, void* stream);
 FLARE_API flare_status_t flare_bwd_shard_dz(const void* Q, int64_t q_batch_stride, const void* K,
                                             const void* V, const void* dY, const float* Z_save,
@@ -313,6 +328,13 @@ FLARE_API flare_status_t flare_bwd_shard_dz(const void* Q, int64_t q_batch_strid
                                             int64_t H, int64_t N, int64_t M, int64_t D,
                                             flare_dtype_t dtype, float scale, void* workspace,
                                             size_t workspace_bytes, void* stream);
+FLARE_API flare_status_t flare_pp_bwd_shard_tail(const void* Q, const void* K, const void* V,
+                                                 const float* Z1, const float* lse1,
+                                                 const void* dQ_dyn, float* dQ_part, void* dK,
+                                                 void* dV, int64_t B, int64_t H, int64_t N,
+                                                 int64_t M, int64_t D, flare_dtype_t dtype,
+                                                 float scale, void* workspace,
+                                                 size_t workspace_bytes, void* stream);
 FLARE_API flare_status_t flare_bwd_shard_finish(const void* Q, int64_t q_batch_stride,
                                                 const void* K, const void* V, const void* dY,
                                                 const float* Z_save, const float* lse_save,

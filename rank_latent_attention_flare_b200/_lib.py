@@ -73,7 +73,9 @@ SIGNATURES = {
                                     _i64, _i64, _i64, _i64, _i32, _f32, _vp, _sz, _vp]),
     "flare_records_layout": (_i32, [_i64, _i64, _i64, _i64, _i64, _i32, _i64p, _szp, _szp]),
     "flare_combine_shards": (_i32, [_i64, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _i32, _vp,
-                                    _vp, _vp, _sz, _vp]),
+                                    _vp, _vp, _vp, _vp, _sz, _vp]),
+    "flare_pp_bwd_shard_tail": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
+                                       _i64, _i64, _i64, _i32, _f32, _vp, _sz, _vp]),
     "flare_bwd_shard_dz": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
                                   _i64, _i32, _f32, _vp, _sz, _vp]),
     "flare_bwd_shard_finish": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,

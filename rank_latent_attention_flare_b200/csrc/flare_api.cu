@@ -489,8 +489,8 @@ flare_status_t flare_records_layout(int64_t B, int64_t H, int64_t N, int64_t M, 
 flare_status_t flare_combine_shards(int64_t shards, const float* ml, const float* acc,
                                     int64_t records_per_bh, int64_t B, int64_t H, int64_t N,
                                     int64_t M, int64_t D, flare_dtype_t dt, float* Z_save,
-                                    float* lse_save, void* workspace, size_t workspace_bytes,
-                                    void* stream) {
+                                    float* lse_save, const void* Q_learned, void* Q_dyn_out,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
   FLARE_TRY(check_sizes(B, H, N, M, D, dt));
   if (shards < 1 || shards > 65536 || records_per_bh < 1 || records_per_bh > (1 << 20))
     return FLARE_ERR_INVALID_ARG;
@@ -498,13 +498,15 @@ flare_status_t flare_combine_shards(int64_t shards, const float* ml, const float
   FLARE_TRY(check_ptr(acc));
   FLARE_TRY(check_opt_ptr(Z_save));
   FLARE_TRY(check_opt_ptr(lse_save));
+  FLARE_TRY(check_opt_ptr(Q_dyn_out));
+  if (Q_dyn_out) FLARE_TRY(check_ptr(Q_learned));
   const WsLayout L = ws_layout(FLARE_OP_FWD, B, H, N, M, D, dt, current_sm_count());
   FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
   g_error_detail[0] = 0;
   char* ws = (char*)workspace;
   FLARE_CUDA(launch_combine(Dims{B, H, N, M, D}, dt, (int)records_per_bh, (int)shards, ml, acc,
                             (float*)(ws + L.zf), (__nv_bfloat16*)(ws + L.zb), Z_save, lse_save,
-                            nullptr, nullptr, (cudaStream_t)stream));
+                            Q_dyn_out ? Q_learned : nullptr, Q_dyn_out, (cudaStream_t)stream));
   return FLARE_OK;
 }
 
@@ -543,6 +545,31 @@ flare_status_t flare_bwd_shard_finish(const void* Q, int64_t qbs, const void* K,
   FLARE_CUDA(launch_bwd(Q, qbs, K, V, dY, Z_save, lse_save, nullptr, dK, dV, Dims{B, H, N, M, D},
                         dt, scale, L, (char*)workspace, (cudaStream_t)stream, BwdPhase::FINISH,
                         const_cast<float*>(dZ), dQ_part));
+  return FLARE_OK;
+}
+
+flare_status_t flare_pp_bwd_shard_tail(const void* Q, const void* K, const void* V,
+                                       const float* Z1, const float* lse1, const void* dQ_dyn,
+                                       float* dQ_part, void* dK, void* dV, int64_t B, int64_t H,
+                                       int64_t N, int64_t M, int64_t D, flare_dtype_t dt,
+                                       float scale, void* workspace, size_t workspace_bytes,
+                                       void* stream) {
+  FLARE_TRY(check_sizes(B, H, N, M, D, dt));
+  FLARE_TRY(check_scale(scale));
+  FLARE_TRY(check_ptr(Q));
+  FLARE_TRY(check_ptr(K));
+  FLARE_TRY(check_ptr(V));
+  FLARE_TRY(check_ptr(Z1));
+  FLARE_TRY(check_ptr(lse1));
+  FLARE_TRY(check_ptr(dQ_dyn));
+  FLARE_TRY(check_ptr(dQ_part));
+  FLARE_TRY(check_ptr(dK));
+  FLARE_TRY(check_ptr(dV));
+  const WsLayout L = ws_layout(FLARE_OP_PP_BWD, B, H, N, M, D, dt, current_sm_count());
+  FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  g_error_detail[0] = 0;
+  FLARE_CUDA(launch_pp_bwd_tail(Q, K, V, Z1, lse1, dQ_dyn, nullptr, dK, dV, Dims{B, H, N, M, D}, dt,
+                                scale, L, (char*)workspace, (cudaStream_t)stream, dQ_part));
   return FLARE_OK;
 }
 

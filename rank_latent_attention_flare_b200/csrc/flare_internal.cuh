@@ -396,14 +396,16 @@ cudaError_t launch_tc_bwd(const void* Q, int64_t qbs, const void* K, const void*
 // FLARE++'s first-encode gradient on the tensor cores (bf16, M = 128,
 // D in {16, 32}): adds into dK, dV and writes dQ (sum over the batch of dZ1
 // and the encode's dQ); reuses the tensor-core backward's workspace.
+// With dq32 (a shard of a context-parallel backward) only the encode's part
+// of dQ is written, in float32, and dZ1 is not added to it.
 cudaError_t launch_tc_enc_bwd(const void* Q, const void* K, const void* V, const float* Z1,
                               const float* lse1, const void* dZ1, void* dQ, void* dK, void* dV,
                               const Dims& d, float scale, const WsLayout& L, char* ws,
-                              cudaStream_t st);
+                              cudaStream_t st, float* dq32 = nullptr);
 cudaError_t launch_pp_bwd_tail(const void* Q, const void* K, const void* V, const float* z1,
                                const float* lse1, const void* dqd, void* dQ, void* dK, void* dV,
                                const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,
-                               char* ws, cudaStream_t st);
+                               char* ws, cudaStream_t st, float* dq32 = nullptr);
 cudaError_t launch_bwd(const void* Q, int64_t qbs, const void* K, const void* V, const void* dY,
                        const float* Z, const float* lse, void* dQ, void* dK, void* dV,
                        const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,

@@ -1737,7 +1737,8 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
 template <int D, bool FLAT, bool VAR>
 cudaError_t tc_enc_bwd_t(const void* Q, const void* K, const void* V, const float* Z1,
                          const float* lse1, const void* dZ1, void* dQ, void* dK, void* dV,
-                         const Dims& d, float scale, const WsLayout& L, char* ws, cudaStream_t st) {
+                         const Dims& d, float scale, const WsLayout& L, char* ws, cudaStream_t st,
+                         float* dq32) {
   const ChunkPlan& p = L.bwd;
   const int64_t BH = d.BH();
   const float c = scale * kLog2e;
@@ -1794,7 +1795,7 @@ cudaError_t tc_enc_bwd_t(const void* Q, const void* K, const void* V, const floa
   const int64_t total = d.H * kM * D;
   bwd_dq_sum_kernel<<<(unsigned)((total / 4 + 127) / 128), 128, 0, st>>>(
       (const float4*)dqp, (int)d.B, (int)d.H, kM, D, p.chunks, true,
-      (const __nv_bfloat16*)dZ1, (__nv_bfloat16*)dQ, nullptr);
+      dq32 ? nullptr : (const __nv_bfloat16*)dZ1, (__nv_bfloat16*)dQ, (float4*)dq32);
   return cudaPeekAtLastError();
 }
 
@@ -1815,13 +1816,13 @@ template <int D>
 cudaError_t tc_enc_bwd_dispatch(const void* Q, const void* K, const void* V, const float* Z1,
                                 const float* lse1, const void* dZ1, void* dQ, void* dK, void* dV,
                                 const Dims& d, float scale, const WsLayout& L, char* ws,
-                                cudaStream_t st) {
+                                cudaStream_t st, float* dq32) {
   const bool flat = tok_flat(d), var = d.lens != nullptr;
-  if (flat)
-    return var ? tc_enc_bwd_t<D, true, true>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st)
-               : tc_enc_bwd_t<D, true, false>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st);
-  return var ? tc_enc_bwd_t<D, false, true>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st)
-             : tc_enc_bwd_t<D, false, false>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st);
+#define FLARE_TC_ENC_T(F, V_) \
+  tc_enc_bwd_t<D, F, V_>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st, dq32)
+  if (flat) return var ? FLARE_TC_ENC_T(true, true) : FLARE_TC_ENC_T(true, false);
+  return var ? FLARE_TC_ENC_T(false, true) : FLARE_TC_ENC_T(false, false);
+#undef FLARE_TC_ENC_T
 }
 
 }  // namespace
@@ -1843,10 +1844,12 @@ cudaError_t launch_tc_bwd(const void* Q, int64_t qbs, const void* K, const void*
 cudaError_t launch_tc_enc_bwd(const void* Q, const void* K, const void* V, const float* Z1,
                               const float* lse1, const void* dZ1, void* dQ, void* dK, void* dV,
                               const Dims& d, float scale, const WsLayout& L, char* ws,
-                              cudaStream_t st) {
+                              cudaStream_t st, float* dq32) {
   if (d.M != kM) return cudaErrorNotSupported;
-  if (d.D == 32) return tc_enc_bwd_dispatch<32>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st);
-  if (d.D == 16) return tc_enc_bwd_dispatch<16>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st);
+  if (d.D == 32)
+    return tc_enc_bwd_dispatch<32>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st, dq32);
+  if (d.D == 16)
+    return tc_enc_bwd_dispatch<16>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st, dq32);
   return cudaErrorNotSupported;
 }
 

@@ -356,17 +356,21 @@ def encode_records(workspace: torch.Tensor, B: int, H: int, N: int, M: int, D: i
 def flare_combine_shards(ml: torch.Tensor, acc: torch.Tensor, B: int, H: int, N: int, M: int,
                          D: int, dtype: torch.dtype, *, workspace: torch.Tensor,
                          Z_save: Optional[torch.Tensor] = None,
-                         lse_save: Optional[torch.Tensor] = None, stream=None) -> None:
+                         lse_save: Optional[torch.Tensor] = None,
+                         Q_learned: Optional[torch.Tensor] = None,
+                         Q_dyn_out: Optional[torch.Tensor] = None, stream=None) -> None:
     """Merges the gathered records of every shard (ml [shards, B*H, R, M, 2],
     acc [shards, B*H, R, M, D]) into the whole sequence's Z, left in
-    ``workspace`` for flare_decode (and written to Z_save / lse_save)."""
-    _need_cuda(ml, acc, workspace, Z_save, lse_save)
+    ``workspace`` for flare_decode (and written to Z_save / lse_save).  With
+    Q_dyn_out (FLARE++'s first encode) also Q_dyn = Q_learned + Z."""
+    _need_cuda(ml, acc, workspace, Z_save, lse_save, Q_learned, Q_dyn_out)
     if ml.dim() != 5 or acc.dim() != 5 or ml.shape[:4] != acc.shape[:4]:
         raise ValueError("ml must be [shards, B*H, R, M, 2] and acc [shards, B*H, R, M, D]")
     code = _lib.FLARE_F32 if dtype == torch.float32 else _lib.FLARE_BF16
     st = _lib.load().flare_combine_shards(ml.shape[0], _ptr(ml), _ptr(acc), ml.shape[2], B, H, N,
                                           M, D, code, _ptr(Z_save), _ptr(lse_save),
-                                          _ptr(workspace), workspace.numel(), _stream(stream))
+                                          _ptr(Q_learned), _ptr(Q_dyn_out), _ptr(workspace),
+                                          workspace.numel(), _stream(stream))
     _lib.check(st, "flare_combine_shards")
 
 
@@ -402,3 +406,23 @@ def flare_bwd_shard_finish(Q, K, V, dY, Z, lse, dZ, scale: Optional[float] = Non
                                             workspace.numel(), _stream(stream))
     _lib.check(st, "flare_bwd_shard_finish")
     return dQ, dK, dV
+
+
+def flare_pp_bwd_shard_tail(Q, K, V, Z1, lse1, dQ_dyn, dK, dV, scale: Optional[float] = None, *,
+                            workspace: torch.Tensor, stream=None) -> torch.Tensor:
+    """FLARE++'s first-encode gradient over this shard, given dQ_dyn summed
+    over the shards (input dtype) and the first encode's Z1, lse1 of the
+    whole sequence: adds into dK, dV (in place) and returns the shard's
+    float32 part of dQ [H,M,D].  ``workspace``: FLARE_OP_PP_BWD size."""
+    _need_cuda(Q, K, V, Z1, lse1, dQ_dyn, dK, dV, workspace)
+    B, H, N, M, D, qbs = _dims(Q, K)
+    if qbs != 0:
+        raise ValueError("FLARE++ takes learned latents Q of shape [H,M,D]")
+    s = default_scale(D) if scale is None else float(scale)
+    dQ = torch.empty(Q.shape, dtype=torch.float32, device=K.device)
+    st = _lib.load().flare_pp_bwd_shard_tail(_ptr(Q), _ptr(K), _ptr(V), _ptr(Z1), _ptr(lse1),
+                                             _ptr(dQ_dyn), _ptr(dQ), _ptr(dK), _ptr(dV), B, H, N,
+                                             M, D, _dtype_code(K), s, _ptr(workspace),
+                                             workspace.numel(), _stream(stream))
+    _lib.check(st, "flare_pp_bwd_shard_tail")
+    return dQ

@@ -22,14 +22,10 @@ import torch.distributed as dist
 _f = importlib.import_module(__package__ + ".flare")
 
 
-def cp_flare_fwd(Q, K, V, scale: Optional[float] = None, *, group=None, save: bool = False,
-                 ops=_f):
-    """K, V: this rank's shard [B,H,N_r,D] of every sequence (the same N_r on
-    every rank; shards in rank order).  Returns this rank's Y shard, or
-    (Y, Z, lse) of the whole sequence when ``save``."""
+def _encode_and_merge(ops, Q, K, V, s, ws, group, **outs):
+    """Encodes this rank's shard, all-gathers every rank's records (rank
+    order) and merges them into the whole sequence's Z in ``ws``."""
     B, H, N, M, D, _ = _f._dims(Q, K)
-    s = _f.default_scale(D) if scale is None else float(scale)
-    ws = ops.alloc_workspace(_f._lib.FLARE_OP_FWD, B, H, N, M, D, K.dtype, K.device)
     ops.flare_encode(Q, K, V, s, workspace=ws)
     ml, acc = ops.encode_records(ws, B, H, N, M, D, K.dtype)
     G = dist.get_world_size(group)
@@ -39,25 +35,81 @@ def cp_flare_fwd(Q, K, V, scale: Optional[float] = None, *, group=None, save: bo
                        device=acc.device)
     dist.all_gather_into_tensor(gml, ml.contiguous(), group=group)
     dist.all_gather_into_tensor(gacc, acc.contiguous(), group=group)
-    gml = gml.view((G,) + tuple(ml.shape))
-    gacc = gacc.view((G,) + tuple(acc.shape))
+    ops.flare_combine_shards(gml.view((G,) + tuple(ml.shape)), gacc.view((G,) + tuple(acc.shape)),
+                             B, H, N, M, D, K.dtype, workspace=ws, **outs)
+
+
+def cp_flare_fwd(Q, K, V, scale: Optional[float] = None, *, group=None, save: bool = False,
+                 ops=_f):
+    """K, V: this rank's shard [B,H,N_r,D] of every sequence (the same N_r on
+    every rank; shards in rank order).  Returns this rank's Y shard, or
+    (Y, Z, lse) of the whole sequence when ``save``."""
+    B, H, N, M, D, _ = _f._dims(Q, K)
+    s = _f.default_scale(D) if scale is None else float(scale)
+    ws = ops.alloc_workspace(_f._lib.FLARE_OP_FWD, B, H, N, M, D, K.dtype, K.device)
     Z = torch.empty((B, H, M, D), dtype=torch.float32, device=K.device)
     lse = torch.empty((B, H, M), dtype=torch.float32, device=K.device)
-    ops.flare_combine_shards(gml, gacc, B, H, N, M, D, K.dtype, workspace=ws, Z_save=Z,
-                             lse_save=lse)
+    _encode_and_merge(ops, Q, K, V, s, ws, group, Z_save=Z, lse_save=lse)
     Y = ops.flare_decode(Q, K, s, workspace=ws)
     return (Y, Z, lse) if save else Y
 
 
-def cp_flare_bwd(Q, K, V, dY, Z, lse, scale: Optional[float] = None, *, group=None, ops=_f):
+def cp_flare_bwd(Q, K, V, dY, Z, lse, scale: Optional[float] = None, *, group=None, ops=_f,
+                 workspace=None):
     """Gradients for this rank's shard (Z, lse: the whole sequence's, from
     cp_flare_fwd(save=True)).  Returns (dQ summed over the shards, in Q's
     dtype; this shard's dK, dV)."""
+    dQ, dK, dV = _cp_bwd32(Q, K, V, dY, Z, lse, scale, group, ops, workspace)
+    return dQ.to(Q.dtype), dK, dV
+
+
+def _cp_bwd32(Q, K, V, dY, Z, lse, scale, group, ops, ws):
     B, H, N, M, D, _ = _f._dims(Q, K)
     s = _f.default_scale(D) if scale is None else float(scale)
-    ws = ops.alloc_workspace(_f._lib.FLARE_OP_BWD, B, H, N, M, D, K.dtype, K.device)
+    if ws is None:
+        ws = ops.alloc_workspace(_f._lib.FLARE_OP_BWD, B, H, N, M, D, K.dtype, K.device)
     dZ = ops.flare_bwd_shard_dz(Q, K, V, dY, Z, lse, s, workspace=ws)
     dist.all_reduce(dZ, group=group)
     dQ, dK, dV = ops.flare_bwd_shard_finish(Q, K, V, dY, Z, lse, dZ, s, workspace=ws)
     dist.all_reduce(dQ, group=group)
-    return dQ.to(Q.dtype), dK, dV
+    return dQ, dK, dV
+
+
+def cp_flare_pp_fwd(Q, K, V, scale: Optional[float] = None, *, group=None, save: bool = False,
+                    ops=_f):
+    """FLARE++ with learned latents Q [H,M,D] over token shards: two record
+    exchanges (the first encode, which gives Q_dyn = Q + Z1, and the second
+    with Q_dyn).  Returns (Y shard, Q_dyn), or (Y, Q_dyn, Z, lse) when
+    ``save`` (Z, lse: the second encode's, whole sequence)."""
+    B, H, N, M, D, qbs = _f._dims(Q, K)
+    if qbs != 0:
+        raise ValueError("FLARE++ takes learned latents Q of shape [H,M,D]")
+    s = _f.default_scale(D) if scale is None else float(scale)
+    ws = ops.alloc_workspace(_f._lib.FLARE_OP_FWD, B, H, N, M, D, K.dtype, K.device)
+    Qd = torch.empty((B, H, M, D), dtype=K.dtype, device=K.device)
+    _encode_and_merge(ops, Q, K, V, s, ws, group, Q_learned=Q, Q_dyn_out=Qd)
+    Z = torch.empty((B, H, M, D), dtype=torch.float32, device=K.device)
+    lse = torch.empty((B, H, M), dtype=torch.float32, device=K.device)
+    _encode_and_merge(ops, Qd, K, V, s, ws, group, Z_save=Z, lse_save=lse)
+    Y = ops.flare_decode(Qd, K, s, workspace=ws)
+    return (Y, Qd, Z, lse) if save else (Y, Qd)
+
+
+def cp_flare_pp_bwd(Q, K, V, dY, Q_dyn, Z, lse, scale: Optional[float] = None, *, group=None,
+                    ops=_f):
+    """FLARE++ gradients for this rank's shard (Q_dyn, Z, lse from
+    cp_flare_pp_fwd(save=True)).  Returns (dQ [H,M,D] in Q's dtype; this
+    shard's dK, dV)."""
+    B, H, N, M, D, _ = _f._dims(Q, K)
+    s = _f.default_scale(D) if scale is None else float(scale)
+    # the first encode, recomputed: Z1, lse1 of the whole sequence
+    wsf = ops.alloc_workspace(_f._lib.FLARE_OP_FWD, B, H, N, M, D, K.dtype, K.device)
+    Z1 = torch.empty((B, H, M, D), dtype=torch.float32, device=K.device)
+    lse1 = torch.empty((B, H, M), dtype=torch.float32, device=K.device)
+    _encode_and_merge(ops, Q, K, V, s, wsf, group, Z_save=Z1, lse_save=lse1)
+    # FLARE's backward with the per-batch latents Q_dyn, then the first encode's
+    ws = ops.alloc_workspace(_f._lib.FLARE_OP_PP_BWD, B, H, N, M, D, K.dtype, K.device)
+    dQd, dK, dV = _cp_bwd32(Q_dyn, K, V, dY, Z, lse, s, group, ops, ws)
+    dQe = ops.flare_pp_bwd_shard_tail(Q, K, V, Z1, lse1, dQd.to(K.dtype), dK, dV, s, workspace=ws)
+    dist.all_reduce(dQe, group=group)
+    return (dQd.sum(0) + dQe).to(Q.dtype), dK, dV

@@ -1,4 +1,5 @@
-"""Context parallelism's host logic on CPU (gloo, world size 2 and 3).
+"""Context parallelism's host logic on CPU (gloo, world size 2 and 3), for
+FLARE and FLARE++.
 
 rank_latent_attention_flare_b200.parallel runs the collectives: the
 all-gather of the encode records and the all-reduces of dZ and dQ.  Here its
@@ -55,15 +56,19 @@ class _Stand:
         return ml, acc.reshape(B * H, 1, M, D)
 
     @staticmethod
-    def flare_combine_shards(gml, gacc, B, H, N, M, D, dtype, *, workspace, Z_save, lse_save):
+    def flare_combine_shards(gml, gacc, B, H, N, M, D, dtype, *, workspace, Z_save=None,
+                             lse_save=None, Q_learned=None, Q_dyn_out=None):
         m, l = gml[..., 0], gml[..., 1]                        # [G, BH, R, M]
         mstar = m.amax(dim=(0, 2))                             # [BH, M]
         f = torch.exp2(m - mstar[None, :, None, :])
         L = (f * l).sum(dim=(0, 2))
         Z = (f[..., None] * gacc).sum(dim=(0, 2)) / L[..., None]
         workspace["Z"] = Z.reshape(B, H, M, D)
-        Z_save.copy_(workspace["Z"])
-        lse_save.copy_(((mstar + torch.log2(L)) / LOG2E).reshape(B, H, M))
+        if Z_save is not None:
+            Z_save.copy_(workspace["Z"])
+            lse_save.copy_(((mstar + torch.log2(L)) / LOG2E).reshape(B, H, M))
+        if Q_dyn_out is not None:   # FLARE++: Q_dyn = Q + Z1
+            Q_dyn_out.copy_(Q_learned.double().unsqueeze(0) + workspace["Z"])
 
     @staticmethod
     def _pd(Q, K, s):
@@ -94,6 +99,17 @@ class _Stand:
         dq = workspace["dq"] + s * torch.einsum("bhmn,bhnd->bhmd", dAe, K.double())
         return (dq.sum(0) if Q.dim() == 3 else dq), dK, dV
 
+    @staticmethod
+    def flare_pp_bwd_shard_tail(Q, K, V, Z1, lse1, dQd, dK, dV, s, *, workspace):
+        # the first encode's gradient with upstream dZ1 = dQ_dyn, over the shard
+        Qb = _Stand._q(Q, K.shape[0])
+        P = torch.exp(s * torch.einsum("bhmd,bhnd->bhmn", Qb, K.double()) - lse1.double()[..., None])
+        dP = torch.einsum("bhmd,bhnd->bhmn", dQd.double(), V.double())
+        dA = P * (dP - (dQd.double() * Z1.double()).sum(-1)[..., None])
+        dV += torch.einsum("bhmn,bhmd->bhnd", P, dQd.double())
+        dK += s * torch.einsum("bhmn,bhmd->bhnd", dA, Qb)
+        return (s * torch.einsum("bhmn,bhnd->bhmd", dA, K.double())).sum(0)
+
 
 def _free_port() -> int:
     with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
@@ -101,7 +117,7 @@ def _free_port() -> int:
         return s.getsockname()[1]
 
 
-def _worker(rank, world, port, batch_q, out):
+def _worker(rank, world, port, batch_q, pp, out):
     os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
     sys.path.insert(0, ROOT)
     sys.path.insert(0, os.path.join(ROOT, "tests"))
@@ -116,25 +132,35 @@ def _worker(rank, world, port, batch_q, out):
         x = make_inputs(B, H, N, M, D, dtype=torch.float64, seed=7, per_batch_q=batch_q,
                         with_dy=True)
         sh = {k: x[k].chunk(world, dim=2)[rank].contiguous() for k in ("K", "V", "dY")}
-        Y, Z, lse = parallel.cp_flare_fwd(x["Q"], sh["K"], sh["V"], s, save=True, ops=_Stand)
-        dQ, dK, dV = parallel.cp_flare_bwd(x["Q"], sh["K"], sh["V"], sh["dY"], Z, lse, s,
-                                           ops=_Stand)
+        if pp:
+            Y, Qd, Z, lse = parallel.cp_flare_pp_fwd(x["Q"], sh["K"], sh["V"], s, save=True,
+                                                     ops=_Stand)
+            dQ, dK, dV = parallel.cp_flare_pp_bwd(x["Q"], sh["K"], sh["V"], sh["dY"], Qd, Z, lse,
+                                                  s, ops=_Stand)
+        else:
+            Y, Z, lse = parallel.cp_flare_fwd(x["Q"], sh["K"], sh["V"], s, save=True, ops=_Stand)
+            dQ, dK, dV = parallel.cp_flare_bwd(x["Q"], sh["K"], sh["V"], sh["dY"], Z, lse, s,
+                                               ops=_Stand)
         out[rank] = (Y.numpy(), Z.numpy(), dQ.numpy(), dK.numpy(), dV.numpy())
     finally:
         dist.destroy_process_group()
 
 
-def _run(world, batch_q):
+def _run(world, batch_q, pp=False):
     import oracle
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     from flare_inputs import make_inputs
     out = mp.Manager().dict()
-    mp.start_processes(_worker, args=(world, _free_port(), batch_q, out), nprocs=world,
+    mp.start_processes(_worker, args=(world, _free_port(), batch_q, pp, out), nprocs=world,
                        join=True, start_method="spawn")
     B, H, N, M, D = 2, 2, 24 * world, 5, 4
     x = make_inputs(B, H, N, M, D, dtype=torch.float64, seed=7, per_batch_q=batch_q, with_dy=True)
-    Yo, Zo, _ = oracle.flare_fwd(x["Q"], x["K"], x["V"], 0.5)
-    dQo, dKo, dVo = oracle.flare_bwd(x["Q"], x["K"], x["V"], x["dY"], 0.5)
+    if pp:
+        Yo, _, Zo, _ = oracle.flare_pp_fwd(x["Q"], x["K"], x["V"], 0.5)
+        dQo, dKo, dVo = oracle.flare_pp_bwd(x["Q"], x["K"], x["V"], x["dY"], 0.5)
+    else:
+        Yo, Zo, _ = oracle.flare_fwd(x["Q"], x["K"], x["V"], 0.5)
+        dQo, dKo, dVo = oracle.flare_bwd(x["Q"], x["K"], x["V"], x["dY"], 0.5)
     n = N // world
     for r in range(world):
         Y, Z, dQ, dK, dV = out[r]
@@ -154,3 +180,7 @@ def test_two_ranks_shared_latents():
 
 def test_three_ranks_per_batch_latents():
     _run(3, True)
+
+
+def test_flare_pp_two_ranks():
+    _run(2, False, pp=True)

@@ -105,3 +105,71 @@ def test_parallel_module_with_one_rank():
     assert torch.equal(Y, Y1) and torch.equal(Z, Z1)
     assert torch.equal(dK, r1[1]) and torch.equal(dV, r1[2])
     assert_close(dQ, r1[0].float(), torch.bfloat16, "dQ")
+
+
+def _merge(Qx, Ks, Vs, s, wss, dims, dtype, **outs_per_shard):
+    """Encode every shard, stack the records, merge them on every shard's
+    workspace; outs_per_shard(r) gives the output tensors of shard r."""
+    B, H, Nr, M, D = dims
+    recs = []
+    for r, (K, V) in enumerate(zip(Ks, Vs)):
+        fl.flare_encode(Qx, K, V, s, workspace=wss[r])
+        recs.append([t.clone() for t in fl.encode_records(wss[r], B, H, Nr, M, D, dtype)])
+    gml = torch.stack([a for a, _ in recs])
+    gacc = torch.stack([b for _, b in recs])
+    for r in range(len(Ks)):
+        fl.flare_combine_shards(gml, gacc, B, H, Nr, M, D, dtype, workspace=wss[r],
+                                **{k: f(r) for k, f in outs_per_shard.items()})
+
+
+@pytest.mark.parametrize("B,H,N,M,D,dtype,G", [(2, 2, 1536, 128, 32, torch.bfloat16, 2),
+                                               (2, 2, 600, 32, 16, torch.float32, 3)],
+                         ids=["tc_2", "simt_f32_3"])
+def test_sharded_flare_pp(B, H, N, M, D, dtype, G):
+    s = 1.0 / math.sqrt(D)
+    x = make_inputs(B, H, N, M, D, dtype=dtype, seed=111 + G, with_dy=True)
+    g = {k: v.to(DEV) for k, v in x.items()}
+    Q = g["Q"]
+    Ks, Vs, dYs = _shards(g["K"], G), _shards(g["V"], G), _shards(g["dY"], G)
+    Nr = N // G
+    dims = (B, H, Nr, M, D)
+    new = lambda *shape, dt=torch.float32: torch.empty(shape, dtype=dt, device=DEV)
+    wss = [fl.alloc_workspace(fl.FLARE_OP_FWD, B, H, Nr, M, D, dtype, DEV) for _ in range(G)]
+    # first encode: Q_dyn = Q + Z1 (and Z1, lse1 for the backward)
+    Qds = [new(B, H, M, D, dt=dtype) for _ in range(G)]
+    Z1s = [new(B, H, M, D) for _ in range(G)]
+    l1s = [new(B, H, M) for _ in range(G)]
+    _merge(Q, Ks, Vs, s, wss, dims, dtype, Q_learned=lambda r: Q, Q_dyn_out=lambda r: Qds[r],
+           Z_save=lambda r: Z1s[r], lse_save=lambda r: l1s[r])
+    for r in range(1, G):
+        assert torch.equal(Qds[r], Qds[0])
+    Qd, Z1, lse1 = Qds[0], Z1s[0], l1s[0]
+    # second encode with Q_dyn, then each shard's decode
+    Zs = [new(B, H, M, D) for _ in range(G)]
+    ls = [new(B, H, M) for _ in range(G)]
+    _merge(Qd, Ks, Vs, s, wss, dims, dtype, Z_save=lambda r: Zs[r], lse_save=lambda r: ls[r])
+    Z, lse = Zs[0], ls[0]
+    Y = torch.cat([fl.flare_decode(Qd, Ks[r], s, workspace=wss[r]) for r in range(G)], dim=2)
+    Y1, Qd1, Zo1, _ = fl.flare_pp_fwd(Q, g["K"], g["V"], s, save=True)
+    Yo, Qdo, _, _ = oracle.flare_pp_fwd(x["Q"], x["K"], x["V"], s)
+    assert_close(Qd, Qdo, dtype, "Q_dyn (sharded)")
+    assert_close(Y, Yo, dtype, "Y (sharded)")
+    # backward: FLARE's with Q_dyn, then the first encode's, shard by shard
+    wsb = [fl.alloc_workspace(fl.FLARE_OP_PP_BWD, B, H, Nr, M, D, dtype, DEV) for _ in range(G)]
+    dZ = sum(fl.flare_bwd_shard_dz(Qd, Ks[r], Vs[r], dYs[r], Z, lse, s, workspace=wsb[r])
+             for r in range(G))
+    parts = [fl.flare_bwd_shard_finish(Qd, Ks[r], Vs[r], dYs[r], Z, lse, dZ, s, workspace=wsb[r])
+             for r in range(G)]
+    dQd = sum(p[0] for p in parts)
+    dQ = dQd.sum(0)
+    for r in range(G):
+        dQ += fl.flare_pp_bwd_shard_tail(Q, Ks[r], Vs[r], Z1, lse1, dQd.to(dtype), parts[r][1],
+                                         parts[r][2], s, workspace=wsb[r])
+    for w in wss + wsb:
+        assert fl.device_status(w) == 0
+    dK = torch.cat([p[1] for p in parts], dim=2)
+    dV = torch.cat([p[2] for p in parts], dim=2)
+    dQo, dKo, dVo = oracle.flare_pp_bwd(x["Q"], x["K"], x["V"], x["dY"], s)
+    assert_close(dV, dVo, dtype, "dV (sharded)", rel_f32=TOL_F32_GRAD_REL)
+    assert_close(dK, dKo, dtype, "dK (sharded)", rel_f32=TOL_F32_GRAD_REL)
+    assert_close(dQ, dQo, dtype, "dQ (sharded)", rel_f32=TOL_F32_GRAD_REL)
