@@ -3,7 +3,7 @@ rejects invalid arguments with status codes before touching the device.
 
 These run without a GPU.  The argument-validation tests pass fake
 (never dereferenced) device addresses, so they are skipped when a CUDA
-device is present: on a GPU machine the same checks run in the gpu tests with
+device is present: with a GPU the same checks run in the gpu tests with
 real buffers.
 """
 import ctypes
