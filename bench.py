@@ -419,8 +419,8 @@ def _row_roofline(t_ms: float, exps: float, flops: float, hbm_bytes: float, peak
 
 
 def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0,
-                    which=("flare_pp_fwd", "flare_fwd_bwd", "flare_pp_fwd_bwd",
-                           "flare_strided", "flare_varlen")):
+                    which=("flare_pp_fwd", "flare_fwd_bwd", "flare_fwd_bwd_m256",
+                           "flare_pp_fwd_bwd", "flare_strided", "flare_varlen")):
     """Times the FLARE++ forward (B=2 H=8 N=262,144 M=256 D=32) and the
     forward + backward of B=8 H=8 N=16,384 M=128 D=32, both bf16, on the
     same device with CUDA events (median of `iters` launches after 3
@@ -452,6 +452,9 @@ def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0,
         rows.update(_time_pp(dev, peaks, peak_kind, timed, seed))
     if "flare_fwd_bwd" in which:
         rows.update(_time_fwd_bwd(dev, peaks, peak_kind, timed, seed))
+    if "flare_fwd_bwd_m256" in which:
+        rows.update(_time_fwd_bwd(dev, peaks, peak_kind, timed, seed, M=256,
+                                  row="flare_fwd_bwd_m256"))
     if "flare_pp_fwd_bwd" in which:
         rows.update(_time_pp_fwd_bwd(dev, peaks, peak_kind, timed, seed))
     if "flare_strided" in which:
@@ -482,10 +485,16 @@ def _time_pp(dev, peaks, peak_kind, timed, seed):
     return rows
 
 
-def _time_fwd_bwd(dev, peaks, peak_kind, timed, seed):
+def _time_fwd_bwd(dev, peaks, peak_kind, timed, seed, M=None, row="flare_fwd_bwd"):
+    """FLARE forward + backward, B=8 H=8 N=16,384 D=32 bf16; M = 128 (the
+    workload's) or, for the M = 256 row, the headline's latent count."""
+    import dataclasses
+
     import rank_latent_attention_flare_b200 as fl
     rows = {}
     w = WORKLOADS["c5_fwdbwd_bf16_16k"]
+    if M is not None:
+        w = dataclasses.replace(w, M=M)
     x = make_inputs(w.B, w.H, w.N, w.M, w.D, dtype=w.torch_dtype, seed=seed, with_dy=True)
     g = {k: v.to(dev) for k, v in x.items()}
     wsf = fl.alloc_workspace(fl.FLARE_OP_FWD, w.B, w.H, w.N, w.M, w.D, w.torch_dtype, dev)
@@ -503,7 +512,7 @@ def _time_fwd_bwd(dev, peaks, peak_kind, timed, seed):
         raise RuntimeError("device wait ran out in the forward + backward")
     u = w.B * w.H * w.N
     ms = ms_f + ms_b
-    rows["flare_fwd_bwd"] = {
+    rows[row] = {
         "workload": f"FLARE fwd+bwd B={w.B} H={w.H} N={w.N} M={w.M} D={w.D} bf16",
         "ms": round(ms, 4), "fwd_ms": round(ms_f, 4), "bwd_ms": round(ms_b, 4),
         "tokens_per_s": w.B * w.N / (ms / 1e3),
@@ -748,7 +757,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true",
                     help="skip the FLARE++ and forward+backward timings")
-    ap.add_argument("--row", choices=["flare_pp_fwd", "flare_fwd_bwd", "flare_pp_fwd_bwd",
+    ap.add_argument("--row", choices=["flare_pp_fwd", "flare_fwd_bwd", "flare_fwd_bwd_m256",
+                                      "flare_pp_fwd_bwd",
                                       "flare_strided", "flare_varlen"],
                     default=None,
                     help="time only this workload (one JSON line with its timing and roofline)")

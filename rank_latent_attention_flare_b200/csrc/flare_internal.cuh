@@ -15,6 +15,10 @@ namespace flare {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+// Tensor-core backward: a token whose decode log-sum-exp lies more than
+// this far (log2 units) below its head's R = max_m lse2[m] flags the head,
+// which then takes the exact form of the encode weights.
+constexpr float kBwdRowRange = 100.f;
 
 // Error sites recorded in the workspace header when a bounded wait runs out.
 enum ErrorSite : uint32_t {
@@ -90,7 +94,7 @@ inline Path choose_path(int64_t N, int64_t M, int64_t D, flare_dtype_t dt) {
   Path p;
   p.tc_fwd = (dt == FLARE_BF16) && (M == 128 || M == 256) && (D == 16 || D == 32) &&
              (N < (1LL << 31) - 256);
-  p.tc_bwd = (dt == FLARE_BF16) && (M == 128) && (D == 16 || D == 32) &&
+  p.tc_bwd = (dt == FLARE_BF16) && (M == 128 || M == 256) && (D == 16 || D == 32) &&
              (N < (1LL << 31) - 256);
   return p;
 }
@@ -159,6 +163,7 @@ struct WsLayout {
   size_t dqe = 0;       // [BH*chunks][M][D] float  first encode's dQ partials
   size_t total = 0;
   ChunkPlan enc, bwd, ppe;
+  ChunkPlan dec;        // tensor-core backward, M = 256: its decode-statistics pass
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -186,11 +191,14 @@ inline WsLayout ws_layout(flare_op_t op, int64_t B, int64_t H, int64_t N, int64_
   if (bwd_like && choose_path(N, M, D, dt).tc_bwd) {
     L.bwd = tc_bwd_plan(BH, N, sms);
     const int64_t bslots = BH * L.bwd.chunks;
+    // with M = 256 the dZ partials come from the encode pipeline (its chunks)
+    const int64_t zslots = (M == 256) ? BH * L.enc.slots_per_bh() : bslots;
+    if (M == 256) L.dec = decode_plan(BH, N, sms);
     L.stats = take((size_t)BH * N * 16);
     L.dy2 = take((size_t)BH * N * D * 2);
     L.rref = take((size_t)BH * 4);
     L.flags = take((size_t)BH * 4);
-    L.dzp = take((size_t)bslots * M * D * 4);
+    L.dzp = take((size_t)zslots * M * D * 4);
     L.dqp = take((size_t)bslots * M * D * 4);
     L.dzs = take((size_t)BH * M * D * 2);
     L.aug = take((size_t)BH * M * 16 * 2);
@@ -357,6 +365,18 @@ cudaError_t launch_tc_encode(const void* Q, int64_t qbs, const void* K, const vo
 cudaError_t launch_tc_decode(const void* Q, int64_t qbs, const void* K,
                              const __nv_bfloat16* Zb, void* Y, const Dims& d, float scale,
                              const ChunkPlan& plan, uint32_t* err, cudaStream_t st);
+// Tensor-core backward with M = 256, decode stage.  launch_tc_bwd_stats: the
+// decode pipeline with the backward's per-token statistics in place of Y
+// (stats, dY'' = dY / g, the head's range flag).  launch_tc_dz: the encode
+// pipeline with dY as V and the weights P_d = 2^(c S - mx'[n]), giving the
+// chunk partials of dZ = P_d^T dY ([BH][slots][M][D], plan = the encode's).
+cudaError_t launch_tc_bwd_stats(const void* Q, int64_t qbs, const void* K, const __nv_bfloat16* Zb,
+                                const void* dY, const Dims& d, float scale, const ChunkPlan& plan,
+                                const float* rref, float4* stats, __nv_bfloat16* dy2,
+                                uint32_t* flags, uint32_t* err, cudaStream_t st);
+cudaError_t launch_tc_dz(const void* Q, int64_t qbs, const void* K, const void* dY, const Dims& d,
+                         float scale, const ChunkPlan& plan, const float4* stats, float* dz_part,
+                         uint32_t* err, cudaStream_t st);
 // 3-D TMA map over a bf16 tensor [depth][rows][D] (D in {16, 32}) with
 // boxes of box_rows whole rows, swizzled to match the UMMA descriptors
 // (64-byte swizzle for 64-byte rows, 32-byte for 32-byte rows).

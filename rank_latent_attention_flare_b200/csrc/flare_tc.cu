@@ -109,7 +109,7 @@ __device__ __forceinline__ void scale_tmem_row(uint32_t taddr, float f) {
 constexpr int kEncTile = 48;
 constexpr int kEncRegsSoftmax = 88, kEncRegsProducer = 56;   // 256 x 88 + 128 x 56 <= 384 x 80
 
-template <int D, int M>
+template <int D, int M, bool DZ = false>
 struct EncLayout {
   static constexpr int RB = 2 * D;                  // bytes per row (one token or latent)
   static constexpr int TILE = kEncTile * RB;        // one K or V tile
@@ -118,17 +118,43 @@ struct EncLayout {
   static constexpr int BAR_OFF = KV_OFF + kEncStages * 2 * TILE;
   static constexpr int NBARS = 2 * kEncStages + 1 + 4 + 4 + 4 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
-  static constexpr int BYTES = MISC_OFF + 16;
+  // dZ form: per stage, the tile's column offsets (kEncTile floats)
+  static constexpr int NB_OFF = MISC_OFF + 16;
+  static constexpr int BYTES = DZ ? NB_OFF + kEncStages * kEncTile * 4 : MISC_OFF + 16;
 };
 
-template <int D, int M, bool FLAT, bool VAR>
+// p = 2^(c a + nb) for NP consecutive pairs of logits, nb per column (a
+// float pair from shared memory): bf16 pairs into pk.  With POLY_EVERY = k
+// > 0, every k-th pair on the FMA pipe.
+template <int NP, int POLY_EVERY>
+__device__ __forceinline__ void exp_bias_pairs(const uint32_t* a, float c, const float* nb,
+                                               uint32_t* pk) {
+  const uint64_t c2 = f32x2(c, c);
+#pragma unroll
+  for (int t = 0; t < NP; ++t) {
+    const uint64_t b2 = *reinterpret_cast<const uint64_t*>(nb + 2 * t);
+    float x0, x1;
+    split_f32x2(fma_f32x2(f32x2(__uint_as_float(a[2 * t]), __uint_as_float(a[2 * t + 1])), c2, b2),
+                x0, x1);
+    const bool poly = POLY_EVERY > 0 && (t % (POLY_EVERY > 0 ? POLY_EVERY : 1)) == POLY_EVERY - 1;
+    pk[t] = pack_bf16(poly ? exp2_fma(x0) : ex2(x0), poly ? exp2_fma(x1) : ex2(x1));
+  }
+}
+
+// DZ = true: the same pipeline computes the decode stage's dZ = P_d^T dY of
+// the backward (latents as rows, tV := dY): the weights of token n are
+// P_d[n,m] = 2^(c S[m,n] - mx'[n]), mx'[n] the decode log-sum-exp (log2
+// units) in stats[n].x, so no running max, rescale or row sum is needed
+// (P_d <= 1); the record is the accumulator alone.
+template <int D, int M, bool FLAT, bool VAR, bool DZ>
 __global__ void __launch_bounds__(kThreads, 2)
     tc_encode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, int H, int64_t N, int q_per_batch,
                      float c, int64_t tiles_per_bh, int64_t chunk_tiles, int slots_per_bh,
                      float* __restrict__ part_ml, float* __restrict__ part_acc,
-                     const int32_t* __restrict__ lens, uint32_t* __restrict__ err) {
-  using L = EncLayout<D, M>;
+                     const int32_t* __restrict__ lens, const float4* __restrict__ stats,
+                     uint32_t* __restrict__ err) {
+  using L = EncLayout<D, M, DZ>;
   constexpr int NH = M / 128;        // latent halves; M=128 -> the two warpgroups split tiles
   constexpr int SUB = (NH == 1) ? 2 : 1;
   constexpr int RB = L::RB;
@@ -183,7 +209,54 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   if (warp >= 8) {
     regs_release<kEncRegsProducer>();
-    if (warp == kWarpTma) {
+    if (DZ && warp == kWarpTma) {
+      // ------------------------------------ TMA producer, dZ form (whole warp)
+      // Each stage also carries the tile's column offsets -mx'[n] (-inf for
+      // columns that are not the tile's own tokens), stored by the warp's
+      // lanes before lane 0 arms the stage's barrier.
+      float* nb_ring = (float*)(smem + L::NB_OFF);
+      if (lane == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        mbar_arrive_expect_tx(q_full, M * RB);
+        const int32_t qz = (int32_t)(q_per_batch ? bh : h);
+        for (int half = 0; half < NH; ++half)
+          tma_load_3d(Qs + half * 128 * RB, &tmQ, q_full, 0, half * 128, qz);
+      }
+      int issued = 0;
+      for (int i = 0; i < (int)ntiles; ++i) {
+        const int s = i % kEncStages;
+        const uint32_t ph = (uint32_t)((i / kEncStages) & 1);
+        int stop = 0;
+        if (lane == 0) {
+          if (i >= kEncStages && !mbar_wait_sleep(&kv_empty[s], ph ^ 1)) {
+            record_error(err, kErrEncTmaWait);
+            *abort_flag = 1;
+          }
+          stop = *abort_flag;
+        }
+        if (__shfl_sync(0xffffffffu, stop, 0)) break;
+        const int64_t tok = ht.row0(tile0 + i, kEncTile);
+        const int lo = ht.lo(tile0 + i, kEncTile), hi = ht.hi(tile0 + i, kEncTile);
+        float* nb = nb_ring + s * kEncTile;
+        for (int t = lane; t < kEncTile; t += 32)
+          nb[t] = (t >= lo && t < hi) ? -stats[bh * N + tok + t].x : -INFINITY;
+        __syncwarp();
+        if (lane == 0) {
+          uint8_t* kt = smem + L::KV_OFF + s * 2 * L::TILE;
+          mbar_arrive_expect_tx(&kv_full[s], 2 * L::TILE);
+          tma_load_tok<FLAT>(kt, &tmK, &kv_full[s], (int32_t)tok, bh, H);
+          tma_load_tok<FLAT>(kt + L::TILE, &tmV, &kv_full[s], (int32_t)tok, bh, H);
+        }
+        issued = i + 1;
+      }
+      if (lane == 0) {
+        for (int i = (issued > kEncStages ? issued - kEncStages : 0); i < issued; ++i)
+          mbar_wait_sleep(&kv_full[i % kEncStages], (uint32_t)((i / kEncStages) & 1));
+        mbar_wait_sleep(q_full, 0);
+      }
+    } else if (warp == kWarpTma) {
       // ---------------------------------------------------- TMA producer
       if (lane == 0) {
         prefetch_tmap(&tmQ);
@@ -313,7 +386,42 @@ __global__ void __launch_bounds__(kThreads, 2)
       scale_tmem_row<D>(tO, g);   // rows without a rescale multiply by 1
       return true;
     };
-    for (int j = 0; j < nW; ++j) {
+    if constexpr (DZ) {
+      const float* nb_ring = (const float*)(smem + L::NB_OFF);
+      for (int j = 0; j < nW; ++j) {
+        const int64_t i = first + (int64_t)stride * j;
+        const int b = j & 1;
+        const int s = (int)(i % kEncStages);
+        const uint32_t tS = tW + 48 * b;
+        // the tile's S in TMEM, and its stage (with the column offsets) landed
+        if (!warp_all(mbar_wait(&s_full[2 * w + b], (uint32_t)((j >> 1) & 1)) &&
+                      mbar_wait(&kv_full[s], (uint32_t)((i / kEncStages) & 1)) && !*abort_flag)) {
+          ok = false;
+          break;
+        }
+        __syncwarp();
+        tc_fence_after();
+        const float* nb = nb_ring + s * kEncTile;
+        {
+          uint32_t a[32], pk[16];
+          tmem_ld32(tS, a);
+          tmem_wait_ld_dep(a);
+          exp_bias_pairs<16, kEncPolyEvery>(a, c, nb, pk);
+          tmem_st16(tS, pk);
+        }
+        {
+          uint32_t a[16], pk[8];
+          tmem_ld16(tS + 32, a);
+          tmem_wait_ld_dep16(a);
+          exp_bias_pairs<8, 0>(a, c, nb + 32, pk);
+          tmem_st8(tS + 16, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&sp_done[2 * w + b]);
+      }
+    }
+    for (int j = 0; !DZ && j < nW; ++j) {
       const int64_t i = first + (int64_t)stride * j;
       const int b = j & 1;
       // the tile's own tokens are its columns [lo, hi); the rest get weight 0
@@ -480,8 +588,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     } else {
       const int64_t slot = bh * slots_per_bh + (int64_t)chunk * SUB + (NH == 1 ? w : 0);
       const int64_t row = slot * M + (NH == 2 ? w * 128 : 0) + r;
-      part_ml[row * 2 + 0] = (nW > 0) ? mref : -INFINITY;
-      part_ml[row * 2 + 1] = l;
+      if (!DZ) {
+        part_ml[row * 2 + 0] = (nW > 0) ? mref : -INFINITY;
+        part_ml[row * 2 + 1] = l;
+      }
       float4* dst = reinterpret_cast<float4*>(part_acc + row * D);
 #pragma unroll
       for (int d = 0; d < D / 4; ++d)
@@ -512,13 +622,28 @@ struct DecLayout {
   static constexpr int BYTES = KN_OFF + kDecBoundSlots * kTile * 4;
 };
 
-template <int D, int M, bool FLAT, bool VAR>
+// The backward's decode statistics (ST = true): in place of Y, every token
+// row gets its decode log-sum-exp mx' (log2 units), delta_d = dY . Y and
+// delta'' = dY'' . Y with dY'' = bf16(dY / g), g = 2^(mx' - R) (R per
+// head), and dY'' itself; a row with g below 2^-kBwdRowRange flags its head
+// (the head then takes the backward's exact form).
+struct DecStats {
+  const __nv_bfloat16* dY;
+  Tok tdy;
+  const float* rref;     // [BH] R
+  float4* stats;         // [BH][N] (mx', delta_d, delta'', 0)
+  __nv_bfloat16* dy2;    // [BH][N][D] dY''
+  uint32_t* flags;       // [BH]
+};
+
+template <int D, int M, bool FLAT, bool VAR, bool ST>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmZ, int H, int64_t N, int q_per_batch,
                      float c, int64_t tiles_per_bh, int64_t chunk_tiles,
                      __nv_bfloat16* __restrict__ Y, Tok ty, const __nv_bfloat16* __restrict__ Qg,
-                     const int32_t* __restrict__ lens, uint32_t* __restrict__ err) {
+                     const int32_t* __restrict__ lens, const DecStats bs,
+                     uint32_t* __restrict__ err) {
   using L = DecLayout<D, M>;
   constexpr int RB = L::RB;
   constexpr uint32_t SW = umma_swizzle_code(RB);
@@ -736,6 +861,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tR = tmem + lb + w * R;
     const int64_t nW = (ntiles - w + 1) / 2;
     bool ok = true;
+    const float Rh = ST ? bs.rref[bh] : 0.f;
+    const int64_t dyhead = ST ? bs.tdy.head(bh, H) : 0;
     for (int64_t j = 0; j < nW; ++j) {
       const int64_t i = 2 * j + w;
       const int64_t tok = ht.row0(tile0 + i, kTile) + r;
@@ -824,7 +951,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(&s_empty[w]);
-      if (mine) {
+      if constexpr (ST) {
+        const float l = (sf[0] + sf[1]) + (sf[2] + sf[3]);
+        const float inv = 1.f / l;
+        const float mxp = fmaf(mx, c, log2f(l));   // the row's log-sum-exp, log2 units
+        const float lg = mxp - Rh;                  // log2 of g
+        const bool bad = mine && lg < -kBwdRowRange;
+        if (mine) {
+          const float ginv = bad ? 0.f : ex2(-lg);
+          const uint4* src = reinterpret_cast<const uint4*>(bs.dY + dyhead + tok * bs.tdy.sn);
+          uint4* dst = reinterpret_cast<uint4*>(bs.dy2 + (bh * N + tok) * D);
+          float dot = 0.f, dot2 = 0.f;
+#pragma unroll
+          for (int v = 0; v < D / 8; ++v) {
+            const uint4 u = src[v];
+            const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
+            uint32_t w2[4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              const float a0 = bf_lo(uu[jj]), a1 = bf_hi(uu[jj]);
+              const float y0 = y[8 * v + 2 * jj], y1 = y[8 * v + 2 * jj + 1];
+              dot = fmaf(a0, y0, fmaf(a1, y1, dot));
+              w2[jj] = pack_bf16(a0 * ginv, a1 * ginv);
+              dot2 = fmaf(bf_lo(w2[jj]), y0, fmaf(bf_hi(w2[jj]), y1, dot2));
+            }
+            dst[v] = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+          }
+          bs.stats[bh * N + tok] = make_float4(mxp, dot * inv, dot2 * inv, 0.f);
+        }
+        if (warp_any(bad) && lane == 0) atomicOr(bs.flags + bh, 1u);
+      } else if (mine) {
         const float inv = 1.f / ((sf[0] + sf[1]) + (sf[2] + sf[3]));
         uint4* dst = reinterpret_cast<uint4*>(Y + yhead + tok * ty.sn);
 #pragma unroll
@@ -927,32 +1083,33 @@ cudaError_t make_tok_map(CUtensorMap* m, const void* base, const Dims& d, const 
 
 namespace {
 
-template <int D, int M, bool FLAT, bool VAR>
+// DZ: V is dY (token strides d.dy), stats the decode statistics, pml unused.
+template <int D, int M, bool FLAT, bool VAR, bool DZ>
 cudaError_t tc_encode_t(const void* Q, int64_t qbs, const void* K, const void* V, const Dims& d,
                         float scale, const ChunkPlan& plan, float* pml, float* pacc,
-                        uint32_t* err, cudaStream_t st) {
+                        const float4* stats, uint32_t* err, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   const int q_per_batch = qbs != 0;
   cudaError_t e;
   if ((e = make_map(&mq, Q, D, M, q_per_batch ? d.BH() : d.H, 128)) != cudaSuccess) return e;
   if ((e = make_tok_map(&mk, K, d, d.k, kEncTile, FLAT)) != cudaSuccess) return e;
-  if ((e = make_tok_map(&mv, V, d, d.v, kEncTile, FLAT)) != cudaSuccess) return e;
+  if ((e = make_tok_map(&mv, V, d, DZ ? d.dy : d.v, kEncTile, FLAT)) != cudaSuccess) return e;
   // two CTAs per SM: their TMEM (2 x 256 columns) fits exactly
-  const int smem = EncLayout<D, M>::BYTES + 1024;
-  e = cudaFuncSetAttribute(tc_encode_kernel<D, M, FLAT, VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           smem);
+  const int smem = EncLayout<D, M, DZ>::BYTES + 1024;
+  e = cudaFuncSetAttribute(tc_encode_kernel<D, M, FLAT, VAR, DZ>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(plan.chunks, (unsigned)d.BH());
-  tc_encode_kernel<D, M, FLAT, VAR><<<grid, kThreads, smem, st>>>(
+  tc_encode_kernel<D, M, FLAT, VAR, DZ><<<grid, kThreads, smem, st>>>(
       mq, mk, mv, (int)d.H, d.N, q_per_batch, scale * kLog2e, plan.tiles_per_bh,
-      plan.chunk_tiles, plan.slots_per_bh(), pml, pacc, d.lens, err);
+      plan.chunk_tiles, plan.slots_per_bh(), pml, pacc, d.lens, stats, err);
   return cudaPeekAtLastError();
 }
 
-template <int D, int M, bool FLAT, bool VAR>
+template <int D, int M, bool FLAT, bool VAR, bool ST>
 cudaError_t tc_decode_t(const void* Q, int64_t qbs, const void* K, const __nv_bfloat16* Zb,
-                        void* Y, const Dims& d, float scale, const ChunkPlan& plan, uint32_t* err,
-                        cudaStream_t st) {
+                        void* Y, const Dims& d, float scale, const ChunkPlan& plan,
+                        const DecStats& bs, uint32_t* err, cudaStream_t st) {
   CUtensorMap mq, mk, mz;
   const int q_per_batch = qbs != 0;
   cudaError_t e;
@@ -961,38 +1118,52 @@ cudaError_t tc_decode_t(const void* Q, int64_t qbs, const void* K, const __nv_bf
   if ((e = make_map(&mz, Zb, D, M, d.BH(), M)) != cudaSuccess) return e;
   const int smem = (DecLayout<D, M>::BYTES + 1024 > kMinSmemBytes) ? DecLayout<D, M>::BYTES + 1024
                                                                    : kMinSmemBytes;
-  e = cudaFuncSetAttribute(tc_decode_kernel<D, M, FLAT, VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           smem);
+  e = cudaFuncSetAttribute(tc_decode_kernel<D, M, FLAT, VAR, ST>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(plan.chunks, (unsigned)d.BH());
-  tc_decode_kernel<D, M, FLAT, VAR><<<grid, kThreads, smem, st>>>(mq, mk, mz, (int)d.H, d.N, q_per_batch,
-                                                       scale * kLog2e, plan.tiles_per_bh,
-                                                       plan.chunk_tiles, (__nv_bfloat16*)Y, d.y,
-                                                       (const __nv_bfloat16*)Q, d.lens, err);
+  tc_decode_kernel<D, M, FLAT, VAR, ST><<<grid, kThreads, smem, st>>>(
+      mq, mk, mz, (int)d.H, d.N, q_per_batch, scale * kLog2e, plan.tiles_per_bh, plan.chunk_tiles,
+      (__nv_bfloat16*)Y, d.y, (const __nv_bfloat16*)Q, d.lens, bs, err);
   return cudaPeekAtLastError();
 }
 
 }  // namespace
 
-template <int D, int M>
+template <int D, int M, bool DZ>
 cudaError_t tc_encode_dispatch(const void* Q, int64_t qbs, const void* K, const void* V,
                                const Dims& d, float scale, const ChunkPlan& plan, float* pml,
-                               float* pacc, uint32_t* err, cudaStream_t st) {
+                               float* pacc, const float4* stats, uint32_t* err, cudaStream_t st) {
   const bool flat = tok_flat(d), var = d.lens != nullptr;
-  if (flat)
-    return var ? tc_encode_t<D, M, true, true>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st)
-               : tc_encode_t<D, M, true, false>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
-  return var ? tc_encode_t<D, M, false, true>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st)
-             : tc_encode_t<D, M, false, false>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
+#define FLARE_TC_ENC(F, V_) \
+  tc_encode_t<D, M, F, V_, DZ>(Q, qbs, K, V, d, scale, plan, pml, pacc, stats, err, st)
+  if (flat) return var ? FLARE_TC_ENC(true, true) : FLARE_TC_ENC(true, false);
+  return var ? FLARE_TC_ENC(false, true) : FLARE_TC_ENC(false, false);
+#undef FLARE_TC_ENC
 }
 
 cudaError_t launch_tc_encode(const void* Q, int64_t qbs, const void* K, const void* V,
                              const Dims& d, float scale, const ChunkPlan& plan, float* pml,
                              float* pacc, uint32_t* err, cudaStream_t st) {
-  if (d.D == 32 && d.M == 256) return tc_encode_dispatch<32, 256>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
-  if (d.D == 32 && d.M == 128) return tc_encode_dispatch<32, 128>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
-  if (d.D == 16 && d.M == 256) return tc_encode_dispatch<16, 256>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
-  if (d.D == 16 && d.M == 128) return tc_encode_dispatch<16, 128>(Q, qbs, K, V, d, scale, plan, pml, pacc, err, st);
+#define FLARE_ENC_ARGS Q, qbs, K, V, d, scale, plan, pml, pacc, nullptr, err, st
+  if (d.D == 32 && d.M == 256) return tc_encode_dispatch<32, 256, false>(FLARE_ENC_ARGS);
+  if (d.D == 32 && d.M == 128) return tc_encode_dispatch<32, 128, false>(FLARE_ENC_ARGS);
+  if (d.D == 16 && d.M == 256) return tc_encode_dispatch<16, 256, false>(FLARE_ENC_ARGS);
+  if (d.D == 16 && d.M == 128) return tc_encode_dispatch<16, 128, false>(FLARE_ENC_ARGS);
+#undef FLARE_ENC_ARGS
+  return cudaErrorNotSupported;
+}
+
+cudaError_t launch_tc_dz(const void* Q, int64_t qbs, const void* K, const void* dY, const Dims& d,
+                         float scale, const ChunkPlan& plan, const float4* stats, float* dz_part,
+                         uint32_t* err, cudaStream_t st) {
+  if (d.M != 256) return cudaErrorNotSupported;
+  if (d.D == 32)
+    return tc_encode_dispatch<32, 256, true>(Q, qbs, K, dY, d, scale, plan, nullptr, dz_part,
+                                             stats, err, st);
+  if (d.D == 16)
+    return tc_encode_dispatch<16, 256, true>(Q, qbs, K, dY, d, scale, plan, nullptr, dz_part,
+                                             stats, err, st);
   return cudaErrorNotSupported;
 }
 
@@ -1002,9 +1173,10 @@ cudaError_t tc_decode_dispatch(const void* Q, int64_t qbs, const void* K,
                                const ChunkPlan& plan, uint32_t* err, cudaStream_t st) {
   // The decode takes 4-D maps for every layout: its 3-D variant measured no
   // faster and needs more registers.
+  const DecStats none{};
   return d.lens != nullptr
-             ? tc_decode_t<D, M, false, true>(Q, qbs, K, Zb, Y, d, scale, plan, err, st)
-             : tc_decode_t<D, M, false, false>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
+             ? tc_decode_t<D, M, false, true, false>(Q, qbs, K, Zb, Y, d, scale, plan, none, err, st)
+             : tc_decode_t<D, M, false, false, false>(Q, qbs, K, Zb, Y, d, scale, plan, none, err, st);
 }
 
 cudaError_t launch_tc_decode(const void* Q, int64_t qbs, const void* K, const __nv_bfloat16* Zb,
@@ -1014,6 +1186,21 @@ cudaError_t launch_tc_decode(const void* Q, int64_t qbs, const void* K, const __
   if (d.D == 32 && d.M == 128) return tc_decode_dispatch<32, 128>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
   if (d.D == 16 && d.M == 256) return tc_decode_dispatch<16, 256>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
   if (d.D == 16 && d.M == 128) return tc_decode_dispatch<16, 128>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
+  return cudaErrorNotSupported;
+}
+
+cudaError_t launch_tc_bwd_stats(const void* Q, int64_t qbs, const void* K, const __nv_bfloat16* Zb,
+                                const void* dY, const Dims& d, float scale, const ChunkPlan& plan,
+                                const float* rref, float4* stats, __nv_bfloat16* dy2,
+                                uint32_t* flags, uint32_t* err, cudaStream_t st) {
+  if (d.M != 256) return cudaErrorNotSupported;
+  const DecStats bs{(const __nv_bfloat16*)dY, d.dy, rref, stats, dy2, flags};
+#define FLARE_TC_ST(D_, V_) \
+  tc_decode_t<D_, 256, false, V_, true>(Q, qbs, K, Zb, nullptr, d, scale, plan, bs, err, st)
+  const bool var = d.lens != nullptr;
+  if (d.D == 32) return var ? FLARE_TC_ST(32, true) : FLARE_TC_ST(32, false);
+  if (d.D == 16) return var ? FLARE_TC_ST(16, true) : FLARE_TC_ST(16, false);
+#undef FLARE_TC_ST
   return cudaErrorNotSupported;
 }
 

@@ -67,7 +67,10 @@ constexpr int kBStages = 3;
 constexpr uint32_t kSw128 = 2u;  // UMMA descriptor code of the 128-byte swizzle
 constexpr uint32_t kSw32 = 6u;   // ... and of the 32-byte swizzle
 constexpr float kSpreadMax = 64.f;     // log2 units: lse spread beyond which a head takes the exact form
-constexpr float kRowRangeMax = 100.f;  // log2 units: a token this far below R flags its head
+constexpr float kRowRangeMax = kBwdRowRange;
+// mode bits of the pass-B kernels
+constexpr int kModeEncOnly = 1;   // the encode's gradient only (no decode term)
+constexpr int kModeAccum = 2;     // dK, dV added to the values already in their rows
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return (uint8_t*)(((uintptr_t)p + 1023) & ~(uintptr_t)1023);
@@ -537,15 +540,15 @@ __global__ void __launch_bounds__(kThr, 1)
 // One block per (b, h), one thread per latent m: the bf16 copy of Z (the
 // operand of Y = P Z and of dY'' Z^T) and R = max_m lse2[m], the reference
 // of the split of the encode weights; clears the head's range flag.
-template <int D>
-__global__ void __launch_bounds__(kM)
+template <int D, int M>
+__global__ void __launch_bounds__(M)
     bwd_prep_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
                     __nv_bfloat16* __restrict__ zb, float* __restrict__ rref,
                     uint32_t* __restrict__ flags) {
-  __shared__ float red[kM / 32];
+  __shared__ float red[M / 32];
   const int64_t bh = blockIdx.x;
   const int m = threadIdx.x;
-  const int64_t row = bh * kM + m;
+  const int64_t row = bh * M + m;
 #pragma unroll
   for (int d = 0; d < D; d += 4) {
     const float4 v = *reinterpret_cast<const float4*>(Z + row * D + d);
@@ -559,7 +562,7 @@ __global__ void __launch_bounds__(kM)
   if (m == 0) {
     float R = red[0];
 #pragma unroll
-    for (int k = 1; k < kM / 32; ++k) R = fmaxf(R, red[k]);
+    for (int k = 1; k < M / 32; ++k) R = fmaxf(R, red[k]);
     rref[bh] = R;
     flags[bh] = 0u;
   }
@@ -571,17 +574,17 @@ __global__ void __launch_bounds__(kM)
 // token of it lies more than kRowRangeMax below R (else f = 1 and the exact
 // form); the bf16 operand dZ'' = f dZ; the extra K-step row: -dZ'' . Z
 // (= -f delta_e) as three bf16 terms, then zeros.
-template <int D>
-__global__ void __launch_bounds__(kM)
+template <int D, int M>
+__global__ void __launch_bounds__(M)
     bwd_mid_kernel(const float* __restrict__ dz_part, int chunks,
                    const __nv_bfloat16* __restrict__ dz_direct, const float* __restrict__ Z,
                    const float* __restrict__ lse, __nv_bfloat16* __restrict__ dzs,
                    uint32_t* __restrict__ aug, const uint32_t* __restrict__ flags,
                    float2* __restrict__ params, float* __restrict__ lse2_out) {
-  __shared__ float red_max[kM / 32], red_min[kM / 32];
+  __shared__ float red_max[M / 32], red_min[M / 32];
   const int64_t bh = blockIdx.x;
   const int m = threadIdx.x;
-  const int64_t row = bh * kM + m;
+  const int64_t row = bh * M + m;
   float dz[D];
 #pragma unroll
   for (int d = 0; d < D; ++d) dz[d] = 0.f;
@@ -590,7 +593,7 @@ __global__ void __launch_bounds__(kM)
     for (int d = 0; d < D; ++d) dz[d] = __bfloat162float(dz_direct[row * D + d]);
   }
   for (int k = 0; k < chunks; ++k) {
-    const float4* p = reinterpret_cast<const float4*>(dz_part + ((bh * chunks + k) * kM + m) * D);
+    const float4* p = reinterpret_cast<const float4*>(dz_part + ((bh * chunks + k) * M + m) * D);
 #pragma unroll
     for (int d = 0; d < D / 4; ++d) {
       const float4 v = p[d];
@@ -614,7 +617,7 @@ __global__ void __launch_bounds__(kM)
   __syncthreads();
   float R = red_max[0], lo = red_min[0];
 #pragma unroll
-  for (int k = 1; k < kM / 32; ++k) {
+  for (int k = 1; k < M / 32; ++k) {
     R = fmaxf(R, red_max[k]);
     lo = fminf(lo, red_min[k]);
   }
@@ -685,7 +688,8 @@ __global__ void __launch_bounds__(kThr, 1)
                     const __grid_constant__ CUtensorMap tmAug, int H, int64_t N, int q_per_batch,
                     float c, float s, int64_t tiles_per_bh, int64_t chunk_tiles,
                     const float4* __restrict__ stats, const float2* __restrict__ params,
-                    const float* __restrict__ lse2, int enc_only, __nv_bfloat16* __restrict__ dK,
+                    const float* __restrict__ lse2, int mode, int m0, int Mt,
+                    __nv_bfloat16* __restrict__ dK,
                     __nv_bfloat16* __restrict__ dV, Tok tdk, Tok tdv, float* __restrict__ dq_part,
                     const int32_t* __restrict__ lens, uint32_t* __restrict__ err) {
   using L = BLayout<D>;
@@ -727,6 +731,8 @@ __global__ void __launch_bounds__(kThr, 1)
   const int64_t ntiles = VAR ? max(imin64(chunk_tiles, ht.count(kT) - tile0), (int64_t)0)
                              : imin64(chunk_tiles, tiles_per_bh - tile0);
   const int64_t KQ = ntiles * NQ;   // quarters of this chunk
+  const bool enc_only = (mode & kModeEncOnly) != 0;   // no decode term
+  const bool accum = (mode & kModeAccum) != 0;        // dK, dV added to the rows' values
   if (params[bh].y != 0.f) return;  // head served by tc_bwd_b_fast_kernel
 
   // the constant A operand of the extra K-step: ones in columns 0-2 of
@@ -741,7 +747,7 @@ __global__ void __launch_bounds__(kThr, 1)
       *reinterpret_cast<uint4*>(ones + t * 32 + x1 * 16) = zero;
     }
     float* ls = (float*)(smem + L::LSE_OFF);
-    for (int m = threadIdx.x; m < M; m += blockDim.x) ls[m] = lse2[bh * M + m];
+    for (int m = threadIdx.x; m < M; m += blockDim.x) ls[m] = lse2[bh * Mt + m0 + m];
   }
   fence_proxy_async_smem();
   if (threadIdx.x == 0) {
@@ -783,10 +789,10 @@ __global__ void __launch_bounds__(kThr, 1)
         prefetch_tmap(&tmDZ);
         prefetch_tmap(&tmAug);
         mbar_arrive_expect_tx(c_full, 3 * M * RB + M * 32);
-        tma_load_3d(smem + L::Q_OFF, &tmQ, c_full, 0, 0, (int32_t)(q_per_batch ? bh : h));
-        tma_load_3d(smem + L::Z_OFF, &tmZ, c_full, 0, 0, (int32_t)bh);
-        tma_load_3d(smem + L::DZ_OFF, &tmDZ, c_full, 0, 0, (int32_t)bh);
-        tma_load_3d(smem + L::AUG_OFF, &tmAug, c_full, 0, 0, (int32_t)bh);
+        tma_load_3d(smem + L::Q_OFF, &tmQ, c_full, 0, m0, (int32_t)(q_per_batch ? bh : h));
+        tma_load_3d(smem + L::Z_OFF, &tmZ, c_full, 0, m0, (int32_t)bh);
+        tma_load_3d(smem + L::DZ_OFF, &tmDZ, c_full, 0, m0, (int32_t)bh);
+        tma_load_3d(smem + L::AUG_OFF, &tmAug, c_full, 0, m0, (int32_t)bh);
         int64_t issued = 0;
         for (int64_t t = 0; t < ntiles; ++t) {
           const int k = (int)(t % kBStages);
@@ -945,7 +951,7 @@ __global__ void __launch_bounds__(kThr, 1)
         const float f = (w == 0) ? s : gv;
         uint4* dst = reinterpret_cast<uint4*>(w == 0 ? dK + dk_head + tok * tdk.sn
                                                      : dV + dv_head + tok * tdv.sn);
-        if (enc_only) {   // added to the gradient already in the rows
+        if (accum) {   // added to the gradient already in the rows
 #pragma unroll
           for (int v = 0; v < D / 8; ++v) {
             const uint4 q4 = dst[v];
@@ -1079,7 +1085,7 @@ __global__ void __launch_bounds__(kThr, 1)
           *abort_flag = 1;
         }
       }
-      float4* dst = reinterpret_cast<float4*>(dq_part + (((int64_t)bh * chunks + chunk) * M + r) * D);
+      float4* dst = reinterpret_cast<float4*>(dq_part + (((int64_t)bh * chunks + chunk) * Mt + m0 + r) * D);
 #pragma unroll
       for (int d = 0; d < D / 4; ++d)
         dst[d] = make_float4(acc[4 * d], acc[4 * d + 1], acc[4 * d + 2], acc[4 * d + 3]);
@@ -1141,7 +1147,7 @@ __global__ void __launch_bounds__(kThr, 1)
                          const __grid_constant__ CUtensorMap tmAug, int H, int64_t N, int q_per_batch,
                          float c, float s, int64_t tiles_per_bh, int64_t chunk_tiles,
                          const float4* __restrict__ stats, const float2* __restrict__ params,
-                         int enc_only, __nv_bfloat16* __restrict__ dK,
+                         int mode, int m0, int Mt, __nv_bfloat16* __restrict__ dK,
                          __nv_bfloat16* __restrict__ dV, Tok tdk, Tok tdv,
                          float* __restrict__ dq_part, const int32_t* __restrict__ lens,
                          uint32_t* __restrict__ err) {
@@ -1190,6 +1196,8 @@ __global__ void __launch_bounds__(kThr, 1)
                      : (int)imin64(chunk_tiles, tiles_per_bh - tile0);
   const float2 prm = params[bh];
   if (prm.y == 0.f) return;   // head served by tc_bwd_b_exact_kernel
+  const bool enc_only = (mode & kModeEncOnly) != 0;   // no decode term
+  const bool accum = (mode & kModeAccum) != 0;        // dK, dV added to the rows' values
 
   if (threadIdx.x == 0) {
     for (int k = 0; k < KST; ++k) {
@@ -1241,10 +1249,10 @@ __global__ void __launch_bounds__(kThr, 1)
         prefetch_tmap(&tmDZ);
         prefetch_tmap(&tmAug);
         mbar_arrive_expect_tx(c_full, 3 * M * RB + M * 32);
-        tma_load_3d(smem + L::Q_OFF, &tmQ, c_full, 0, 0, (int32_t)(q_per_batch ? bh : h));
-        tma_load_3d(smem + L::Z_OFF, &tmZ, c_full, 0, 0, (int32_t)bh);
-        tma_load_3d(smem + L::DZ_OFF, &tmDZ, c_full, 0, 0, (int32_t)bh);
-        tma_load_3d(smem + L::AUG_OFF, &tmAug, c_full, 0, 0, (int32_t)bh);
+        tma_load_3d(smem + L::Q_OFF, &tmQ, c_full, 0, m0, (int32_t)(q_per_batch ? bh : h));
+        tma_load_3d(smem + L::Z_OFF, &tmZ, c_full, 0, m0, (int32_t)bh);
+        tma_load_3d(smem + L::DZ_OFF, &tmDZ, c_full, 0, m0, (int32_t)bh);
+        tma_load_3d(smem + L::AUG_OFF, &tmAug, c_full, 0, m0, (int32_t)bh);
         int issued = 0;
         for (int t = 0; t < nt; ++t) {
           const int32_t tok = (int32_t)ht.row0(tile0 + t, kT);
@@ -1439,7 +1447,7 @@ __global__ void __launch_bounds__(kThr, 1)
         const float f = (w == 0) ? s : 1.f;
         uint4* dst = reinterpret_cast<uint4*>(w == 0 ? dK + dk_head + tok * tdk.sn
                                                      : dV + dv_head + tok * tdv.sn);
-        if (enc_only) {   // added to the gradient already in the rows
+        if (accum) {   // added to the gradient already in the rows
 #pragma unroll
           for (int v = 0; v < D / 8; ++v) {
             const uint4 q4 = dst[v];
@@ -1550,7 +1558,7 @@ __global__ void __launch_bounds__(kThr, 1)
           *abort_flag = 1;
         }
       }
-      float4* dst = reinterpret_cast<float4*>(dq_part + (((int64_t)bh * chunks + chunk) * M + r) * D);
+      float4* dst = reinterpret_cast<float4*>(dq_part + (((int64_t)bh * chunks + chunk) * Mt + m0 + r) * D);
 #pragma unroll
       for (int d = 0; d < D / 4; ++d)
         dst[d] = make_float4(acc[4 * d], acc[4 * d + 1], acc[4 * d + 2], acc[4 * d + 3]);
@@ -1636,7 +1644,15 @@ __global__ void bwd_dz_sum_kernel(const float4* __restrict__ dz_part, int64_t BH
   dz[i] = acc;
 }
 
-template <int D, bool FLAT, bool VAR>
+// M = 128: pass A (tc_bwd_a_kernel) gives the per-token statistics and the
+// dZ partials in one pass.  M = 256: an S row of 256 latents per token does
+// not fit pass A's TMEM and shared-memory layout, so the decode stage runs
+// as two passes of the forward's pipelines -- the decode kernel with the
+// statistics in place of Y, then the encode kernel with dY as V and the
+// per-token weights P_d = 2^(c S - mx') -- and pass B runs once per half of
+// the latents (the encode weights and G of a latent depend on it and on the
+// per-token statistics alone), the second half adding into dK and dV.
+template <int D, int M, bool FLAT, bool VAR>
 cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, const void* dY,
                      const float* Z, const float* lse, void* dQ, void* dK, void* dV, const Dims& d,
                      float scale, const WsLayout& L, char* ws, cudaStream_t st, BwdPhase phase,
@@ -1657,45 +1673,55 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
   float2* params = (float2*)(ws + L.params);
   float* lse2 = (float*)(ws + L.lse2);
   float* dqp = (float*)(ws + L.dqp);
+  const int zchunks = (M == kM) ? p.chunks : L.enc.slots_per_bh();   // dZ partials per head
   cudaError_t e;
 
   if (phase != BwdPhase::FINISH) {
-    bwd_prep_kernel<D><<<(unsigned)BH, kM, 0, st>>>(Z, lse, zb, rref, flags);
+    bwd_prep_kernel<D, M><<<(unsigned)BH, M, 0, st>>>(Z, lse, zb, rref, flags);
     if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   }
 
+  // latent operands: M rows per head, loaded 128 rows at a time
   CUtensorMap mq, mk, mv, mdy, mdy2, mz, mdz, maug;
-  if ((e = make_map(&mq, Q, D, kM, q_per_batch ? BH : d.H, kM)) != cudaSuccess) return e;
+  if ((e = make_map(&mq, Q, D, M, q_per_batch ? BH : d.H, kM)) != cudaSuccess) return e;
   if ((e = make_tok_map(&mk, K, d, d.k, kT, FLAT)) != cudaSuccess) return e;
   if ((e = make_tok_map(&mv, V, d, d.v, kT, FLAT)) != cudaSuccess) return e;
   if ((e = make_tok_map(&mdy, dY, d, d.dy, kT, FLAT)) != cudaSuccess) return e;
   if ((e = make_map(&mdy2, dy2, D, d.N, BH, kT)) != cudaSuccess) return e;
-  if ((e = make_map(&mz, zb, D, kM, BH, kM)) != cudaSuccess) return e;
-  if ((e = make_map(&mdz, dzs, D, kM, BH, kM)) != cudaSuccess) return e;
-  if ((e = make_map(&maug, aug, 16, kM, BH, kM)) != cudaSuccess) return e;
+  if ((e = make_map(&mz, zb, D, M, BH, kM)) != cudaSuccess) return e;
+  if ((e = make_map(&mdz, dzs, D, M, BH, kM)) != cudaSuccess) return e;
+  if ((e = make_map(&maug, aug, 16, M, BH, kM)) != cudaSuccess) return e;
 
   dim3 grid(p.chunks, (unsigned)BH);
   if (phase != BwdPhase::FINISH) {
-    const int smemA = ALayout<D>::BYTES + 1024;
-    e = cudaFuncSetAttribute(tc_bwd_a_kernel<D, FLAT, VAR>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, smemA);
-    if (e != cudaSuccess) return e;
-    tc_bwd_a_kernel<D, FLAT, VAR><<<grid, kThr, smemA, st>>>(
-        mq, mk, mdy, mz, (int)d.H, d.N, q_per_batch, c, p.tiles_per_bh, p.chunk_tiles, rref,
-        stats, dy2, flags, dzp, d.lens, err);
-    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+    if constexpr (M == kM) {
+      const int smemA = ALayout<D>::BYTES + 1024;
+      e = cudaFuncSetAttribute(tc_bwd_a_kernel<D, FLAT, VAR>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, smemA);
+      if (e != cudaSuccess) return e;
+      tc_bwd_a_kernel<D, FLAT, VAR><<<grid, kThr, smemA, st>>>(
+          mq, mk, mdy, mz, (int)d.H, d.N, q_per_batch, c, p.tiles_per_bh, p.chunk_tiles, rref,
+          stats, dy2, flags, dzp, d.lens, err);
+      if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+    } else {
+      if ((e = launch_tc_bwd_stats(Q, qbs, K, zb, dY, d, scale, L.dec, rref, stats, dy2, flags,
+                                   err, st)) != cudaSuccess)
+        return e;
+      if ((e = launch_tc_dz(Q, qbs, K, dY, d, scale, L.enc, stats, dzp, err, st)) != cudaSuccess)
+        return e;
+    }
     if (phase == BwdPhase::DZ) {   // this device's part of dZ
-      const int64_t n4 = BH * kM * D / 4;
+      const int64_t n4 = BH * M * D / 4;
       bwd_dz_sum_kernel<<<(unsigned)((n4 + 127) / 128), 128, 0, st>>>(
-          (const float4*)dzp, BH, kM, D, p.chunks, (float4*)dz_io);
+          (const float4*)dzp, BH, M, D, zchunks, (float4*)dz_io);
       return cudaPeekAtLastError();
     }
   }
 
   // dZ: the chunk partials, or (FINISH) the sum over the shards as one partial
-  bwd_mid_kernel<D><<<(unsigned)BH, kM, 0, st>>>(phase == BwdPhase::FINISH ? dz_io : dzp,
-                                                 phase == BwdPhase::FINISH ? 1 : p.chunks, nullptr,
-                                                 Z, lse, dzs, (uint32_t*)aug, flags, params, lse2);
+  bwd_mid_kernel<D, M><<<(unsigned)BH, M, 0, st>>>(phase == BwdPhase::FINISH ? dz_io : dzp,
+                                                   phase == BwdPhase::FINISH ? 1 : zchunks, nullptr,
+                                                   Z, lse, dzs, (uint32_t*)aug, flags, params, lse2);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
   // each head runs in exactly one of the two pass-B kernels (params.y)
@@ -1703,27 +1729,28 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
   e = cudaFuncSetAttribute(tc_bwd_b_fast_kernel<D, FLAT, VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smemF);
   if (e != cudaSuccess) return e;
-  tc_bwd_b_fast_kernel<D, FLAT, VAR><<<grid, kThr, smemF, st>>>(
-      mq, mk, mv, mdy2, mz, mdz, maug, (int)d.H, d.N, q_per_batch, c, scale,
-      p.tiles_per_bh,
-      p.chunk_tiles, stats, params, 0, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, d.dk, d.dv, dqp, d.lens,
-      err);
-  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   const int smemB = BLayout<D>::BYTES + 1024;
   e = cudaFuncSetAttribute(tc_bwd_b_exact_kernel<D, FLAT, VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smemB);
   if (e != cudaSuccess) return e;
-  tc_bwd_b_exact_kernel<D, FLAT, VAR><<<grid, kThr, smemB, st>>>(
-      mq, mk, mv, mdy, mz, mdz, maug, (int)d.H, d.N, q_per_batch, c, scale,
-      p.tiles_per_bh,
-      p.chunk_tiles, stats, params, lse2, 0, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, d.dk, d.dv, dqp, d.lens,
-      err);
-  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+  for (int m0 = 0; m0 < M; m0 += kM) {
+    const int mode = (m0 > 0) ? kModeAccum : 0;
+    tc_bwd_b_fast_kernel<D, FLAT, VAR><<<grid, kThr, smemF, st>>>(
+        mq, mk, mv, mdy2, mz, mdz, maug, (int)d.H, d.N, q_per_batch, c, scale, p.tiles_per_bh,
+        p.chunk_tiles, stats, params, mode, m0, M, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, d.dk,
+        d.dv, dqp, d.lens, err);
+    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+    tc_bwd_b_exact_kernel<D, FLAT, VAR><<<grid, kThr, smemB, st>>>(
+        mq, mk, mv, mdy, mz, mdz, maug, (int)d.H, d.N, q_per_batch, c, scale, p.tiles_per_bh,
+        p.chunk_tiles, stats, params, lse2, mode, m0, M, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV,
+        d.dk, d.dv, dqp, d.lens, err);
+    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+  }
 
   const bool shared_q = (qbs == 0);
-  const int64_t total = shared_q ? d.H * kM * D : BH * kM * D;
+  const int64_t total = shared_q ? d.H * M * D : BH * M * D;
   bwd_dq_sum_kernel<<<(unsigned)((total / 4 + 127) / 128), 128, 0, st>>>(
-      (const float4*)dqp, (int)d.B, (int)d.H, kM, D, p.chunks, shared_q, nullptr,
+      (const float4*)dqp, (int)d.B, (int)d.H, M, D, p.chunks, shared_q, nullptr,
       (__nv_bfloat16*)dQ, (float4*)dq32);
   return cudaPeekAtLastError();
 }
@@ -1731,10 +1758,10 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
 // FLARE++'s first encode, Z1 = softmax_N(s Q K^T) V with Q shared over the
 // batch, differentiated with upstream dZ1 = dQ_dyn: the pass-B kernels in
 // their encode-only form (no decode term; dK, dV added to the rows that
-// FLARE's backward wrote), then dQ = sum over b of (dQ_dyn + the encode's
-// partials).  Runs after FLARE's backward on the same stream and reuses its
-// workspace.
-template <int D, bool FLAT, bool VAR>
+// FLARE's backward wrote), once per half of the latents with M = 256, then
+// dQ = sum over b of (dQ_dyn + the encode's partials).  Runs after FLARE's
+// backward on the same stream and reuses its workspace.
+template <int D, int M, bool FLAT, bool VAR>
 cudaError_t tc_enc_bwd_t(const void* Q, const void* K, const void* V, const float* Z1,
                          const float* lse1, const void* dZ1, void* dQ, void* dK, void* dV,
                          const Dims& d, float scale, const WsLayout& L, char* ws, cudaStream_t st,
@@ -1755,71 +1782,71 @@ cudaError_t tc_enc_bwd_t(const void* Q, const void* K, const void* V, const floa
   cudaError_t e;
 
   // bf16 Z1 and a cleared range flag (no decode, so no token can raise it)
-  bwd_prep_kernel<D><<<(unsigned)BH, kM, 0, st>>>(Z1, lse1, zb, rref, flags);
+  bwd_prep_kernel<D, M><<<(unsigned)BH, M, 0, st>>>(Z1, lse1, zb, rref, flags);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
-  bwd_mid_kernel<D><<<(unsigned)BH, kM, 0, st>>>(nullptr, 0, (const __nv_bfloat16*)dZ1, Z1, lse1,
-                                                 dzs, (uint32_t*)aug, flags, params, lse2);
+  bwd_mid_kernel<D, M><<<(unsigned)BH, M, 0, st>>>(nullptr, 0, (const __nv_bfloat16*)dZ1, Z1, lse1,
+                                                   dzs, (uint32_t*)aug, flags, params, lse2);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
   // the decode operands' maps point at V: valid tiles that are never used
   CUtensorMap mq, mk, mv, mz, mdz, maug;
-  if ((e = make_map(&mq, Q, D, kM, d.H, kM)) != cudaSuccess) return e;
+  if ((e = make_map(&mq, Q, D, M, d.H, kM)) != cudaSuccess) return e;
   if ((e = make_tok_map(&mk, K, d, d.k, kT, FLAT)) != cudaSuccess) return e;
   if ((e = make_tok_map(&mv, V, d, d.v, kT, FLAT)) != cudaSuccess) return e;
-  if ((e = make_map(&mz, zb, D, kM, BH, kM)) != cudaSuccess) return e;
-  if ((e = make_map(&mdz, dzs, D, kM, BH, kM)) != cudaSuccess) return e;
-  if ((e = make_map(&maug, aug, 16, kM, BH, kM)) != cudaSuccess) return e;
+  if ((e = make_map(&mz, zb, D, M, BH, kM)) != cudaSuccess) return e;
+  if ((e = make_map(&mdz, dzs, D, M, BH, kM)) != cudaSuccess) return e;
+  if ((e = make_map(&maug, aug, 16, M, BH, kM)) != cudaSuccess) return e;
 
   dim3 grid(p.chunks, (unsigned)BH);
   const int smemF = BFLayout<D>::BYTES + 1024;
   e = cudaFuncSetAttribute(tc_bwd_b_fast_kernel<D, FLAT, VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smemF);
   if (e != cudaSuccess) return e;
-  tc_bwd_b_fast_kernel<D, FLAT, VAR><<<grid, kThr, smemF, st>>>(
-      mq, mk, mv, mv, mz, mdz, maug, (int)d.H, d.N, 0, c, scale, p.tiles_per_bh,
-      p.chunk_tiles,
-      stats, params, 1, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, d.dk, d.dv, dqp, d.lens,
-      err);
-  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   const int smemB = BLayout<D>::BYTES + 1024;
   e = cudaFuncSetAttribute(tc_bwd_b_exact_kernel<D, FLAT, VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smemB);
   if (e != cudaSuccess) return e;
-  tc_bwd_b_exact_kernel<D, FLAT, VAR><<<grid, kThr, smemB, st>>>(
-      mq, mk, mv, mv, mz, mdz, maug, (int)d.H, d.N, 0, c, scale, p.tiles_per_bh,
-      p.chunk_tiles,
-      stats, params, lse2, 1, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, d.dk, d.dv, dqp, d.lens,
-      err);
-  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+  for (int m0 = 0; m0 < M; m0 += kM) {
+    tc_bwd_b_fast_kernel<D, FLAT, VAR><<<grid, kThr, smemF, st>>>(
+        mq, mk, mv, mv, mz, mdz, maug, (int)d.H, d.N, 0, c, scale, p.tiles_per_bh, p.chunk_tiles,
+        stats, params, kModeEncOnly | kModeAccum, m0, M, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV,
+        d.dk, d.dv, dqp, d.lens, err);
+    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+    tc_bwd_b_exact_kernel<D, FLAT, VAR><<<grid, kThr, smemB, st>>>(
+        mq, mk, mv, mv, mz, mdz, maug, (int)d.H, d.N, 0, c, scale, p.tiles_per_bh, p.chunk_tiles,
+        stats, params, lse2, kModeEncOnly | kModeAccum, m0, M, (__nv_bfloat16*)dK,
+        (__nv_bfloat16*)dV, d.dk, d.dv, dqp, d.lens, err);
+    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+  }
 
-  const int64_t total = d.H * kM * D;
+  const int64_t total = d.H * M * D;
   bwd_dq_sum_kernel<<<(unsigned)((total / 4 + 127) / 128), 128, 0, st>>>(
-      (const float4*)dqp, (int)d.B, (int)d.H, kM, D, p.chunks, true,
+      (const float4*)dqp, (int)d.B, (int)d.H, M, D, p.chunks, true,
       dq32 ? nullptr : (const __nv_bfloat16*)dZ1, (__nv_bfloat16*)dQ, (float4*)dq32);
   return cudaPeekAtLastError();
 }
 
-template <int D>
+template <int D, int M>
 cudaError_t tc_bwd_dispatch(const void* Q, int64_t qbs, const void* K, const void* V,
                             const void* dY, const float* Z, const float* lse, void* dQ, void* dK,
                             void* dV, const Dims& d, float scale, const WsLayout& L, char* ws,
                             cudaStream_t st, BwdPhase ph, float* dz, float* dq32) {
   const bool flat = tok_flat(d), var = d.lens != nullptr;
 #define FLARE_TC_BWD_T(F, V_) \
-  tc_bwd_t<D, F, V_>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st, ph, dz, dq32)
+  tc_bwd_t<D, M, F, V_>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st, ph, dz, dq32)
   if (flat) return var ? FLARE_TC_BWD_T(true, true) : FLARE_TC_BWD_T(true, false);
   return var ? FLARE_TC_BWD_T(false, true) : FLARE_TC_BWD_T(false, false);
 #undef FLARE_TC_BWD_T
 }
 
-template <int D>
+template <int D, int M>
 cudaError_t tc_enc_bwd_dispatch(const void* Q, const void* K, const void* V, const float* Z1,
                                 const float* lse1, const void* dZ1, void* dQ, void* dK, void* dV,
                                 const Dims& d, float scale, const WsLayout& L, char* ws,
                                 cudaStream_t st, float* dq32) {
   const bool flat = tok_flat(d), var = d.lens != nullptr;
 #define FLARE_TC_ENC_T(F, V_) \
-  tc_enc_bwd_t<D, F, V_>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st, dq32)
+  tc_enc_bwd_t<D, M, F, V_>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st, dq32)
   if (flat) return var ? FLARE_TC_ENC_T(true, true) : FLARE_TC_ENC_T(true, false);
   return var ? FLARE_TC_ENC_T(false, true) : FLARE_TC_ENC_T(false, false);
 #undef FLARE_TC_ENC_T
@@ -1831,13 +1858,14 @@ cudaError_t launch_tc_bwd(const void* Q, int64_t qbs, const void* K, const void*
                           const void* dY, const float* Z, const float* lse, void* dQ, void* dK,
                           void* dV, const Dims& d, float scale, const WsLayout& L, char* ws,
                           cudaStream_t st, BwdPhase phase, float* dz, float* dq32) {
-  if (d.M != kM) return cudaErrorNotSupported;
-  if (d.D == 32)
-    return tc_bwd_dispatch<32>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st, phase,
-                               dz, dq32);
-  if (d.D == 16)
-    return tc_bwd_dispatch<16>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st, phase,
-                               dz, dq32);
+#define FLARE_TC_BWD(D_, M_)                                                                  \
+  tc_bwd_dispatch<D_, M_>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st, phase, dz, \
+                          dq32)
+  if (d.D == 32 && d.M == 128) return FLARE_TC_BWD(32, 128);
+  if (d.D == 32 && d.M == 256) return FLARE_TC_BWD(32, 256);
+  if (d.D == 16 && d.M == 128) return FLARE_TC_BWD(16, 128);
+  if (d.D == 16 && d.M == 256) return FLARE_TC_BWD(16, 256);
+#undef FLARE_TC_BWD
   return cudaErrorNotSupported;
 }
 
@@ -1845,11 +1873,13 @@ cudaError_t launch_tc_enc_bwd(const void* Q, const void* K, const void* V, const
                               const float* lse1, const void* dZ1, void* dQ, void* dK, void* dV,
                               const Dims& d, float scale, const WsLayout& L, char* ws,
                               cudaStream_t st, float* dq32) {
-  if (d.M != kM) return cudaErrorNotSupported;
-  if (d.D == 32)
-    return tc_enc_bwd_dispatch<32>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st, dq32);
-  if (d.D == 16)
-    return tc_enc_bwd_dispatch<16>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st, dq32);
+#define FLARE_TC_ENC(D_, M_) \
+  tc_enc_bwd_dispatch<D_, M_>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st, dq32)
+  if (d.D == 32 && d.M == 128) return FLARE_TC_ENC(32, 128);
+  if (d.D == 32 && d.M == 256) return FLARE_TC_ENC(32, 256);
+  if (d.D == 16 && d.M == 128) return FLARE_TC_ENC(16, 128);
+  if (d.D == 16 && d.M == 256) return FLARE_TC_ENC(16, 256);
+#undef FLARE_TC_ENC
   return cudaErrorNotSupported;
 }
 

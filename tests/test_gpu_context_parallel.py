@@ -19,7 +19,7 @@ DEV = "cuda"
 
 CASES = [
     (2, 2, 1536, 128, 32, torch.bfloat16, 2, False),   # tensor-core fwd and bwd, 2 shards
-    (1, 2, 1536, 256, 32, torch.bfloat16, 3, False),   # tc fwd (M = 256), CUDA-core bwd
+    (1, 2, 1536, 256, 32, torch.bfloat16, 3, False),   # tensor cores, M = 256
     (2, 2, 1536, 128, 16, torch.bfloat16, 4, True),    # per-batch latents
     (2, 2, 600, 32, 16, torch.float32, 3, False),      # CUDA-core fp32
 ]

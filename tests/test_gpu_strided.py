@@ -23,7 +23,7 @@ DEV = "cuda"
 # (B, H, N, M, D, dtype): tensor-core and CUDA-core forward / backward shapes
 CASES = [
     (2, 3, 1000, 128, 32, torch.bfloat16),    # tensor-core fwd and bwd
-    (1, 2, 777, 256, 16, torch.bfloat16),     # tensor-core fwd, CUDA-core bwd
+    (1, 2, 777, 256, 16, torch.bfloat16),     # tensor cores, M = 256
     (2, 2, 300, 64, 32, torch.bfloat16),      # CUDA-core fwd and bwd
     (2, 2, 257, 32, 16, torch.float32),       # CUDA-core, fp32
 ]

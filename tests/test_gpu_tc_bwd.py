@@ -1,5 +1,7 @@
-"""GPU parity of the tensor-core backward (bf16, M = 128, D in {16, 32})
-against the double-precision oracle.
+"""GPU parity of the tensor-core backward (bf16, M in {128, 256}, D in
+{16, 32}) against the double-precision oracle.  With M = 256 the decode
+stage runs as the statistics pass (decode pipeline) and the dZ pass (encode
+pipeline, 48-token tiles), and pass B once per half of the latents.
 
 Covers single tokens, one tile, ragged tails, many tiles and several chunks
 per (b, h), shared and per-batch latents, both forms of the encode weights
@@ -53,12 +55,21 @@ def test_tc_bwd_sizes(N, D):
 
 
 @pytest.mark.parametrize("D", [32, 16])
-def test_tc_bwd_single_token_closed_form(D):
+@pytest.mark.parametrize("N", [2, 47, 48, 49, 129, 1000])
+def test_tc_bwd_sizes_m256(N, D):
+    # both tile sizes of the M = 256 path: 48 tokens (dZ pass), 128 (the
+    # rest); one token (dK = 0 exactly) is the closed-form test below
+    _run(2, 2, N, 256, D, seed=200 + N)
+
+
+@pytest.mark.parametrize("M", [128, 256])
+@pytest.mark.parametrize("D", [32, 16])
+def test_tc_bwd_single_token_closed_form(D, M):
     # One token: every latent encodes Z[m] = V[0] and the decode returns
     # Y[0] = V[0] whatever K and Q are, so dQ = dK = 0 and dV = dY.  The
     # kernels take every derived sum with the bf16 operands the tensor cores
     # use, so the zeros come out at float32 rounding level.
-    B, H, N, M = 2, 2, 1, 128
+    B, H, N = 2, 2, 1
     s = 1.0 / math.sqrt(D)
     x = make_inputs(B, H, N, M, D, dtype=BF16, seed=4, with_dy=True)
     g = {k: v.to(DEV) for k, v in x.items()}
@@ -70,34 +81,40 @@ def test_tc_bwd_single_token_closed_form(D):
     assert float((dV.float() - g["dY"].float()).abs().max()) <= 3e-2
 
 
+@pytest.mark.parametrize("M", [128, 256])
 @pytest.mark.parametrize("D", [32, 16])
-def test_tc_bwd_per_batch_latents(D):
-    _run(3, 2, 700, 128, D, seed=7, per_batch_q=True)
+def test_tc_bwd_per_batch_latents(D, M):
+    _run(3, 2, 700, M, D, seed=7, per_batch_q=True)
 
 
+@pytest.mark.parametrize("M", [128, 256])
 @pytest.mark.parametrize("D", [32, 16])
-def test_tc_bwd_many_tiles_and_chunks(D):
+def test_tc_bwd_many_tiles_and_chunks(D, M):
     # 40,000 tokens per head: 313 tiles, split over several CTAs per head
-    _run(1, 2, 40000, 128, D, seed=9)
+    _run(1, 2, 40000, M, D, seed=9)
 
 
+@pytest.mark.parametrize("M", [128, 256])
 @pytest.mark.parametrize("scale_mul", [4.0, 100.0])
-def test_tc_bwd_sharp_softmax_exact_form(scale_mul):
+def test_tc_bwd_sharp_softmax_exact_form(scale_mul, M):
     # Large logits spread the lse over more than 64 (log2 units) on some heads:
     # those heads take the exact form of the encode weights.
-    _run(2, 2, 900, 128, 32, seed=11, scale_mul=scale_mul)
+    _run(2, 2, 900, M, 32, seed=11, scale_mul=scale_mul)
 
 
-def test_tc_bwd_near_uniform_softmax():
-    _run(2, 2, 3000, 128, 32, seed=12, q_std=0.02)
+@pytest.mark.parametrize("M", [128, 256])
+def test_tc_bwd_near_uniform_softmax(M):
+    _run(2, 2, 3000, M, 32, seed=12, q_std=0.02)
 
 
-def test_tc_bwd_poisoned_workspace():
-    _run(1, 3, 517, 128, 32, seed=13, poison=True)
+@pytest.mark.parametrize("M", [128, 256])
+def test_tc_bwd_poisoned_workspace(M):
+    _run(1, 3, 517, M, 32, seed=13, poison=True)
 
 
-def test_tc_bwd_bitwise_reproducible():
-    B, H, N, M, D = 2, 2, 5000, 128, 32
+@pytest.mark.parametrize("M", [128, 256])
+def test_tc_bwd_bitwise_reproducible(M):
+    B, H, N, D = 2, 2, 5000, 32
     s = 1.0 / math.sqrt(D)
     x = make_inputs(B, H, N, M, D, dtype=BF16, seed=14, with_dy=True)
     g = {k: v.to(DEV) for k, v in x.items()}
@@ -109,11 +126,12 @@ def test_tc_bwd_bitwise_reproducible():
         assert torch.equal(u, v)
 
 
-def test_tc_bwd_mixed_heads_fast_and_exact():
+@pytest.mark.parametrize("M", [128, 256])
+def test_tc_bwd_mixed_heads_fast_and_exact(M):
     # Head 1's latents are scaled up so its lse spreads far beyond 64 (log2
     # units) and it takes the exact form, while head 0 takes the
     # one-exponential form, in the same launch.
-    B, H, N, M, D = 2, 2, 1500, 128, 32
+    B, H, N, D = 2, 2, 1500, 32
     s = 1.0 / math.sqrt(D)
     x = make_inputs(B, H, N, M, D, dtype=BF16, seed=15, with_dy=True)
     x["Q"][1] = (x["Q"][1].float() * 40.0).to(BF16)

@@ -23,7 +23,7 @@ DEV = "cuda"
 CASES = [
     (6, 2, 400, 128, 32, torch.bfloat16, [400, 0, 1, 47, 129, 256]),   # tensor-core fwd + bwd
     (4, 2, 300, 128, 16, torch.bfloat16, [49, 128, 127, 300]),         # tensor-core, D = 16
-    (3, 2, 500, 256, 32, torch.bfloat16, [96, 500, 5]),                # tc fwd (M = 256), CUDA-core bwd
+    (3, 2, 500, 256, 32, torch.bfloat16, [96, 500, 5]),                # tensor cores, M = 256
     (3, 2, 200, 64, 16, torch.bfloat16, [0, 65, 200]),                 # CUDA-core bf16
     (3, 2, 150, 32, 16, torch.float32, [1, 150, 64]),                  # CUDA-core fp32
 ]
