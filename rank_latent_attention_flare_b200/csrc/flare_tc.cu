@@ -15,6 +15,11 @@
 //   Y = (P Z) / rowsum(P)     (A = P from TMEM, B = Z from smem)
 // so the N x M logits never leave the SM.
 //
+// The tensor-core backward with M = 256 reuses both pipelines (template
+// flags): the decode with the backward's per-token statistics in place of Y
+// (ST), and the encode with dY in place of V and fixed per-token weights in
+// place of the online softmax (DZ), which gives dZ = P_d^T dY.
+//
 // Roles per CTA (384 threads, three warpgroups): warps 0-3 and 4-7 are two
 // softmax warpgroups, warp 8 issues TMA loads, warp 9 owns TMEM and issues
 // the MMAs, warps 10-11 only lend their registers.  The CTA launches at 168

@@ -1,5 +1,5 @@
-// Tensor-core FLARE backward for sm_100a: bf16 inputs, M = 128 latents,
-// D in {16, 32}.  Gradients of sum(Y * dY) with respect to Q, K and V with
+// Tensor-core FLARE backward for sm_100a: bf16 inputs, M in {128, 256}
+// latents, D in {16, 32}.  Gradients of sum(Y * dY) with respect to Q, K and V with
 // the logits of both stages recomputed on the tensor cores (tcgen05.mma,
 // TMEM accumulators, TMA-fed operands).  The pages give no backward; this is
 // the chain rule through the encode (skill page section 2: softmax over the
@@ -43,6 +43,9 @@
 // chunk's tiles).  dK and dV are final per tile; dQ partials per chunk are
 // summed in a fixed order afterwards, so results are reproducible bitwise.
 //
+// With M = 256 the decode stage runs as two passes of the forward's
+// pipelines instead of pass A (tc_bwd_t), and pass B once per latent half.
+//
 // Roles per CTA (384 threads): warps 0-3 and 4-7 are the row warpgroups,
 // warp 8 issues TMA loads, warp 9 issues the MMAs, warps 10-11 only lend
 // registers (as in the forward's decode kernel).
@@ -57,7 +60,7 @@ namespace {
 using namespace tc;
 
 constexpr int kT = 128;          // tokens per tile
-constexpr int kM = 128;          // latents
+constexpr int kM = 128;          // latents of one pass-A / pass-B launch (M, or half of it)
 constexpr int kThr = 384;
 constexpr int kRegsRow = 200;
 constexpr int kRegsPro = 104;
