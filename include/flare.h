@@ -152,10 +152,11 @@ FLARE_API flare_status_t flare_pp_fwd(const void* Q, const void* K, const void* 
  * Outputs in the input dtype: dQ ([H,M,D] summed over the batch when
  * q_batch_stride == 0, else [B,H,M,D]), dK, dV.  The logits of both stages
  * are recomputed; every reduction is in a fixed order, so results are
- * bitwise reproducible run to run.  With bf16, M = 128 and D in {16, 32}
- * the work runs on the tensor cores in two passes over the tokens (the
- * decode-stage softmax and dZ, then dK, dV and dQ with one exponential per
- * token-latent pair); other sizes use CUDA-core kernels.
+ * bitwise reproducible run to run.  With bf16, M in {128, 256} and D in
+ * {16, 32} the work runs on the tensor cores: the decode-stage softmax and
+ * dZ (one pass over the tokens with M = 128; with M = 256 a statistics pass
+ * and a dZ pass), then dK, dV and dQ with one exponential per token-latent
+ * pair (once per 128-latent half); other sizes use CUDA-core kernels.
  */
 FLARE_API flare_status_t flare_bwd(const void* Q, int64_t q_batch_stride, const void* K, const void* V,
                          const void* dY, const float* Z_save, const float* lse_save, void* dQ,
@@ -394,8 +395,8 @@ FLARE_API flare_status_t flare_device_status(void* workspace, size_t workspace_b
 FLARE_API int flare_fwd_path(int64_t B, int64_t H, int64_t N, int64_t M, int64_t D, flare_dtype_t dtype);
 
 /*
- * Which kernel family flare_bwd uses for these sizes: 1 = the two-pass
- * tcgen05 backward (bf16, M = 128, D in {16, 32}), 0 = CUDA-core kernels.
+ * Which kernel family flare_bwd uses for these sizes: 1 = the tcgen05
+ * backward (bf16, M in {128, 256}, D in {16, 32}), 0 = CUDA-core kernels.
  * Returns -1 for invalid or unsupported sizes.
  */
 FLARE_API int flare_bwd_path(int64_t B, int64_t H, int64_t N, int64_t M, int64_t D, flare_dtype_t dtype);
