@@ -872,6 +872,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t i = 2 * j + w;
       const int64_t tok = ht.row0(tile0 + i, kTile) + r;
       const bool mine = ht.own(tile0 + i, kTile, r);
+      // statistics: the row's dY is read after the softmax; start its load now
+      if (ST && mine) prefetch_l1(bs.dY + dyhead + tok * bs.tdy.sn);
       const int slot = (int)(i % kDecBoundSlots);
       if (!warp_all(mbar_wait(&s_full[w], (uint32_t)(j & 1)) &&
                     (!kBound || mbar_wait(&kn_full[slot], (uint32_t)((i / kDecBoundSlots) & 1))) &&

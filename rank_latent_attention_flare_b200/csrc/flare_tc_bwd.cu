@@ -1480,6 +1480,10 @@ __global__ void __launch_bounds__(kThr, 1)
       const float ndd = -dpp_next;
       const float nR = own_row(t) ? -Rh : -INFINITY;   // not this tile's token: e = 0, G = 0
       dpp_next = load_dpp(t + 1);
+      // the row finish(t - 1) adds into: start its load now
+      if (accum && t > 0 && own_row(t - 1))
+        prefetch_l1(w == 0 ? dK + dk_head + row_tok(t - 1) * tdk.sn
+                           : dV + dv_head + row_tok(t - 1) * tdv.sn);
       if (!warp_all(mbar_wait_sleep(&h_full[slot], (uint32_t)((k / NS) & 1)) && !*abort_flag)) {
         ok = false;
         break;

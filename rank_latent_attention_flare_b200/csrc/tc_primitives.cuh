@@ -156,6 +156,12 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)map) : "memory");
 }
 
+// Starts moving the 128-byte line holding p into this SM's L1 (a hint: no
+// register waits on it), so a load of it issued later finds it there.
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
 // ------------------------------------------------------ register split
 
 // Warpgroup-wide: lower / raise this warpgroup's per-thread register limit.
