@@ -23,11 +23,12 @@ DEV = "cuda"
 # (B, H, N, M, D, dtype): tensor-core and CUDA-core forward / backward shapes
 CASES = [
     (2, 3, 1000, 128, 32, torch.bfloat16),    # tensor-core fwd and bwd
-    (1, 2, 777, 256, 16, torch.bfloat16),     # tensor cores, M = 256
+    (1, 2, 777, 256, 16, torch.bfloat16),     # tensor cores, M = 256 (B = 1: 3-D maps)
+    (2, 2, 1000, 256, 32, torch.bfloat16),    # tensor cores, M = 256, 4-D maps
     (2, 2, 300, 64, 32, torch.bfloat16),      # CUDA-core fwd and bwd
     (2, 2, 257, 32, 16, torch.float32),       # CUDA-core, fp32
 ]
-IDS = ["tc", "tc_fwd_M256", "simt_bf16", "simt_f32"]
+IDS = ["tc", "tc_M256", "tc_M256_4d", "simt_bf16", "simt_f32"]
 
 
 def _bnhd(x: torch.Tensor) -> torch.Tensor:
@@ -97,7 +98,8 @@ def test_bwd_strided_equals_contiguous(B, H, N, M, D, dtype):
         assert_close(r1[0], dQo, dtype, "dQ", rel_f32=TOL_F32_GRAD_REL)
 
 
-@pytest.mark.parametrize("B,H,N,M,D,dtype", [CASES[0], CASES[2]], ids=["tc", "simt_bf16"])
+@pytest.mark.parametrize("B,H,N,M,D,dtype", [CASES[0], CASES[2], CASES[3]],
+                         ids=["tc", "tc_M256_4d", "simt_bf16"])
 def test_pp_fwd_bwd_strided_equals_contiguous(B, H, N, M, D, dtype):
     s = 1.0 / math.sqrt(D)
     x, g = _inputs(B, H, N, M, D, dtype, seed=73 + N, with_dy=True)
