@@ -29,7 +29,9 @@
  *   - dtype: FLARE_F32 or FLARE_BF16 for Q, K, V, Y, dY, dQ, dK, dV.  All
  *     arithmetic accumulates in float32; bf16 operands feed the tensor cores.
  *   - Supported sizes: B, H >= 1; N >= 1; D in {16, 32}; M a multiple of 16
- *     in [16, 256]; B*H*N*D < 2^40.  scale must be finite and > 0.
+ *     in [16, 256]; B*H*N*D < 2^40; B*H <= 65535 (one grid row per head;
+ *     larger products return FLARE_ERR_UNSUPPORTED).  scale must be finite
+ *     and > 0.
  *   - The caller owns every buffer.  The library never allocates or frees
  *     memory and never synchronises the device (flare_device_status is the
  *     one exception and says so).  Work is enqueued on `stream` (a
@@ -47,7 +49,10 @@
  *   - Every wait inside a kernel is bounded.  A wait that runs out sets an
  *     error word in the workspace header instead of hanging; read it with
  *     flare_device_status after the stream has been synchronised.
- *   - The library holds no mutable global state and is thread-safe.
+ *   - The library is thread-safe and holds no mutable global state, with
+ *     one exception: flare_fwd_noalloc's fixed device scratch array (one per
+ *     device) and the cache of its per-device address, described with that
+ *     call below.
  */
 #ifndef FLARE_H_
 #define FLARE_H_
@@ -366,16 +371,27 @@ FLARE_API flare_status_t flare_bwd_shard_finish(const void* Q, int64_t q_batch_s
  * (flare_last_error_detail says why); use flare_fwd for them.
  *
  * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current) and caches it; make that
- * first call before any stream capture.  All calls on a device share the
- * array: calls whose work overlaps on the GPU (other streams or host
- * threads, same device) race on it and must be serialised by the caller.
+ * (cudaGetSymbolAddress, with that device current) and caches it per device
+ * and context (a context made after cudaDeviceReset is looked up again);
+ * make that first call before any stream capture.  All calls on a device
+ * share the array: calls whose work overlaps on the GPU (other streams or
+ * host threads, same device) race on it and must be serialised by the
+ * caller.  A bounded wait that runs out inside one of these calls sets the
+ * error word at the start of the array; read it with
+ * flare_noalloc_device_status.
  */
 FLARE_API flare_status_t flare_fwd_noalloc(const void* Q, int64_t q_batch_stride, const void* K,
                                            const void* V, void* Y, int64_t B, int64_t H,
                                            int64_t N, int64_t M, int64_t D, flare_dtype_t dtype,
                                            float scale, float* Z_save, float* lse_save,
                                            void* stream);
+
+/*
+ * flare_device_status for flare_fwd_noalloc's scratch array on the current
+ * device: reads and clears its error word (SYNCHRONISES `stream`).  Same
+ * return values and detail codes as flare_device_status.
+ */
+FLARE_API flare_status_t flare_noalloc_device_status(uint32_t* detail, void* stream);
 
 /*
  * Reads and clears the device error word in the workspace header.  This
@@ -400,6 +416,72 @@ FLARE_API int flare_fwd_path(int64_t B, int64_t H, int64_t N, int64_t M, int64_t
  * Returns -1 for invalid or unsupported sizes.
  */
 FLARE_API int flare_bwd_path(int64_t B, int64_t H, int64_t N, int64_t M, int64_t D, flare_dtype_t dtype);
+
+/*
+ * Measurement and self-test support.  Not part of the method: these calls
+ * exist so that the roofline the library is measured against, the
+ * hand-written exponential and the bounded waits can be checked on the
+ * device itself.  Unlike the calls above, flare_probe_unit_rates
+ * synchronises the device.
+ */
+
+/* Throughputs measured by flare_probe_unit_rates, per SM and per SM clock. */
+typedef struct {
+  int sms;                    /* multiprocessors of the current device          */
+  double sm_mhz;              /* SM clock during the probes (clock64 against the
+                                 global timer, mean over the probe kernels)     */
+  double ex2_per_clk_sm;      /* ex2.approx.ftz.f32 results                     */
+  double fma_per_clk_sm;      /* fp32 FMAs issued as fma.rn.f32                 */
+  double fma2_per_clk_sm;     /* fp32 FMAs issued as packed fma.rn.f32x2 (2 each) */
+  double mix_ex2_per_clk_sm;  /* ex2 results while 6 FMAs per ex2 also issue    */
+  double mix_fma_per_clk_sm;  /* the FMAs of that mix                           */
+  double ex2_ms, fma_ms, fma2_ms, mix_ms;  /* CUDA-event time of each probe     */
+} flare_unit_rates_t;
+
+/* Bytes of device scratch flare_probe_unit_rates needs (0 without a device). */
+FLARE_API size_t flare_probe_scratch_bytes(void);
+
+/*
+ * Times four probe kernels on the current device (about 4 SM-resident CTAs
+ * of 256 threads per SM, independent dependency chains): MUFU exponentials,
+ * scalar FMAs, packed FMAs, and exponentials mixed with six FMAs each.
+ * Rates are results per SM per SM clock, from CUDA-event times and the
+ * clock the kernels saw.  scratch: device memory of at least
+ * flare_probe_scratch_bytes() bytes, 16-byte aligned (the kernels' clock
+ * records).  Runs on `stream` and SYNCHRONISES it.  Returns FLARE_OK,
+ * FLARE_ERR_INVALID_ARG (NULL pointer), FLARE_ERR_WORKSPACE (scratch too
+ * small or misaligned) or FLARE_ERR_CUDA.
+ */
+FLARE_API flare_status_t flare_probe_unit_rates(void* scratch, size_t scratch_bytes,
+                                                flare_unit_rates_t* out, void* stream);
+
+/*
+ * y[i] = 2^x[i] for n floats (device pointers), with the exponential the
+ * kernels use: form 0 = the MUFU instruction (ex2.approx.ftz.f32), form 1 =
+ * the FMA-pipe polynomial evaluated one value at a time, form 2 = the same
+ * polynomial in packed fp32x2 arithmetic, two values at a time (the form
+ * the softmax loops use).  The polynomial: round-to-nearest range
+ * reduction x = j + f, a degree-3 minimax fit of 2^f on [-1/2, 1/2]
+ * (relative error 7.5e-5), j added to the exponent field; valid for
+ * x <= 126, inputs below -125 are clamped to -125.  Enqueued on `stream`.
+ */
+FLARE_API flare_status_t flare_eval_exp2(const float* x, float* y, int64_t n, int form,
+                                         void* stream);
+
+/*
+ * Launches one CTA that waits, with the kernels' bounded wait, on an
+ * mbarrier that nothing arrives on, for limit_ns nanoseconds (at most the
+ * kernels' own limit of 1 s, else FLARE_ERR_INVALID_ARG); around the wait
+ * it holds TMEM and a bulk copy of workspace bytes [256, 512) in flight,
+ * as the FLARE kernels do.  When the wait runs out the kernel records site
+ * 0x701 in the workspace error word, lets the copy land, frees TMEM and
+ * returns: flare_device_status on the same workspace then returns
+ * FLARE_ERR_DEVICE_TIMEOUT with detail 0x701, and the device stays usable.
+ * workspace: device memory of at least 512 bytes, 256-byte aligned (the
+ * error word is cleared first).  Enqueued on `stream`.
+ */
+FLARE_API flare_status_t flare_selftest_wait_timeout(void* workspace, size_t workspace_bytes,
+                                                     uint64_t limit_ns, void* stream);
 
 #ifdef __cplusplus
 }

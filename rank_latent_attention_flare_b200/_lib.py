@@ -50,6 +50,16 @@ class FlareStrides(ctypes.Structure):
 
 _stp = ctypes.POINTER(FlareStrides)
 
+
+class UnitRates(ctypes.Structure):
+    """flare_unit_rates_t: probe throughputs per SM per SM clock."""
+    _fields_ = [("sms", ctypes.c_int), ("sm_mhz", ctypes.c_double),
+                ("ex2_per_clk_sm", ctypes.c_double), ("fma_per_clk_sm", ctypes.c_double),
+                ("fma2_per_clk_sm", ctypes.c_double), ("mix_ex2_per_clk_sm", ctypes.c_double),
+                ("mix_fma_per_clk_sm", ctypes.c_double), ("ex2_ms", ctypes.c_double),
+                ("fma_ms", ctypes.c_double), ("fma2_ms", ctypes.c_double),
+                ("mix_ms", ctypes.c_double)]
+
 SIGNATURES = {
     "flare_version": (_i32, []),
     "flare_last_error_detail": (ctypes.c_char_p, []),
@@ -90,6 +100,11 @@ SIGNATURES = {
     "flare_bwd_path": (_i32, [_i64, _i64, _i64, _i64, _i64, _i32]),
     "flare_fwd_noalloc": (_i32, [_vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i32,
                                  _f32, _vp, _vp, _vp]),
+    "flare_noalloc_device_status": (_i32, [_u32p, _vp]),
+    "flare_probe_scratch_bytes": (_sz, []),
+    "flare_probe_unit_rates": (_i32, [_vp, _sz, ctypes.POINTER(UnitRates), _vp]),
+    "flare_eval_exp2": (_i32, [_vp, _vp, _i64, _i32, _vp]),
+    "flare_selftest_wait_timeout": (_i32, [_vp, _sz, ctypes.c_uint64, _vp]),
 }
 
 _lib = None

@@ -1,7 +1,8 @@
 // C ABI of the FLARE library: argument validation, workspace carving and
 // launch orchestration on the caller's stream.  No allocation, no
 // synchronisation (except flare_device_status, documented as such), no
-// global mutable state.
+// global mutable state (the one exception, flare_fwd_noalloc's fixed scratch
+// array and its address cache, lives in flare_noalloc.cu).
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>

@@ -53,6 +53,8 @@ constexpr int kEncStages = 8;
 constexpr int kDecStages = 6;
 constexpr float kRescaleTau = 8.0f;   // log2 units: rescale only when the max grows by > 2^8
 constexpr float kRedoTau = 64.0f;     // log2 units: past 2^64 above m_ref a tile is recomputed
+constexpr float kRescaleLimit = 256.0f;                  // 2^kRescaleTau
+constexpr float kRedoLimit = 18446744073709551616.0f;   // 2^kRedoTau
 // Every k-th pair of exponentials is computed on the FMA pipe (exp2_fma)
 // instead of the MUFU, which is the unit that bounds both kernels.  The
 // encode (four softmax warps per SM sub-partition) gains from moving every
@@ -60,8 +62,21 @@ constexpr float kRedoTau = 64.0f;     // log2 units: past 2^64 above m_ref a til
 // (two per sub-partition, close to its register budget) gains only from the
 // last pair of each 32-column chunk (1.40 -> 1.38 ms; every 4th, 8th, 10th
 // or 12th pair is slower).
-constexpr int kEncPolyEvery = 4;
-constexpr int kDecPolyEvery = 16;
+#ifndef FLARE_ENC_POLY32
+#define FLARE_ENC_POLY32 4
+#endif
+#ifndef FLARE_ENC_POLY16
+#define FLARE_ENC_POLY16 0
+#endif
+#ifndef FLARE_DEC_POLY
+#define FLARE_DEC_POLY 16
+#endif
+#ifndef FLARE_ENC_MAXLESS
+#define FLARE_ENC_MAXLESS 1
+#endif
+constexpr int kEncPolyEvery = FLARE_ENC_POLY32;
+constexpr int kEncPolyEvery16 = FLARE_ENC_POLY16;
+constexpr int kDecPolyEvery = FLARE_DEC_POLY;
 // Decode reference of a token row (M = 256): the max of the first 32-logit
 // chunk read, used when c |k| max_m |q_m| (Cauchy-Schwarz: at least every
 // logit) lies at most this far (log2 units) above it, so no weight exceeds
@@ -142,7 +157,13 @@ __device__ __forceinline__ void exp_bias_pairs(const uint32_t* a, float c, const
     split_f32x2(fma_f32x2(f32x2(__uint_as_float(a[2 * t]), __uint_as_float(a[2 * t + 1])), c2, b2),
                 x0, x1);
     const bool poly = POLY_EVERY > 0 && (t % (POLY_EVERY > 0 ? POLY_EVERY : 1)) == POLY_EVERY - 1;
-    pk[t] = pack_bf16(poly ? exp2_fma(x0) : ex2(x0), poly ? exp2_fma(x1) : ex2(x1));
+    if (poly) {
+      float p0, p1;
+      exp2_fma_pair(f32x2(x0, x1), p0, p1);
+      pk[t] = pack_bf16(p0, p1);
+    } else {
+      pk[t] = pack_bf16(ex2(x0), ex2(x1));
+    }
   }
 }
 
@@ -418,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           uint32_t a[16], pk[8];
           tmem_ld16(tS + 32, a);
           tmem_wait_ld_dep16(a);
-          exp_bias_pairs<8, 0>(a, c, nb + 32, pk);
+          exp_bias_pairs<8, kEncPolyEvery16>(a, c, nb + 32, pk);
           tmem_st8(tS + 16, pk);
         }
         tmem_wait_st();
@@ -448,7 +469,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       bool exact = warp_any(mref == -INFINITY);
       if (!exact) {
         const float neg = -mref;
+#if !FLARE_ENC_MAXLESS
         float mf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#endif
         float sf[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t pa[16], pb[8];
         {
@@ -460,7 +483,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int t = 0; t < 32; ++t)
               if (t < lo || t >= hi) a[t] = __float_as_uint(-INFINITY);
           }
+#if !FLARE_ENC_MAXLESS
           max_fold32(a, mf);
+#endif
           exp_pack32<kEncPolyEvery>(a, c, neg, pa, sf);
         }
         {
@@ -472,9 +497,38 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int t = 0; t < 16; ++t)
               if (32 + t < lo || 32 + t >= hi) a[t] = __float_as_uint(-INFINITY);
           }
+#if !FLARE_ENC_MAXLESS
           max_fold16(a, mf);
-          exp_pack16(a, c, neg, pb, sf);
+#endif
+          exp_pack16<kEncPolyEvery16>(a, c, neg, pb, sf);
         }
+        const float sum = (sf[0] + sf[1]) + (sf[2] + sf[3]);
+#if FLARE_ENC_MAXLESS
+        // Every weight of the tile is at most the tile's row sum, so the sum
+        // stands in for the max: above 2^kRedoTau (or not finite) a weight
+        // may have overflowed and the tile is recomputed with the exact max;
+        // above 2^kRescaleTau the reference moves up by log2(sum), which
+        // keeps it within log2(tile) of the running max.
+        if (warp_any(!(sum <= kRedoLimit))) {
+          exact = true;
+        } else {
+          if (!scale_O(j, pend)) {   // a rescale decided after the previous tile
+            ok = false;
+            break;
+          }
+          pend = 1.f;
+          tmem_st16(tS, pa);          // P over S columns already read
+          tmem_st8(tS + 16, pb);
+          if (sum > kRescaleLimit) {
+            const float mx2 = mref + lg2(sum);
+            pend = ex2(mref - mx2);
+            l = (l + sum) * pend;
+            mref = mx2;
+          } else {
+            l += sum;
+          }
+        }
+#else
         const float mx2 = fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3])) * c;
         if (warp_any(mx2 > mref + kRedoTau)) {
           exact = true;
@@ -486,7 +540,6 @@ __global__ void __launch_bounds__(kThreads, 2)
           pend = 1.f;
           tmem_st16(tS, pa);          // P over S columns already read
           tmem_st8(tS + 16, pb);
-          const float sum = (sf[0] + sf[1]) + (sf[2] + sf[3]);
           if (mx2 > mref + kRescaleTau) {
             pend = ex2(mref - mx2);
             l = (l + sum) * pend;
@@ -495,6 +548,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             l += sum;
           }
         }
+#endif
       }
       if (exact) {
         // pass 1: exact tile max of the raw logits (masked columns excluded)
@@ -555,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, 2)
               if (32 + t < lo || 32 + t >= hi) a[t] = __float_as_uint(-INFINITY);
           }
           uint32_t pk[8];
-          exp_pack16(a, c, neg, pk, sf);
+          exp_pack16<kEncPolyEvery16>(a, c, neg, pk, sf);
           tmem_st8(tS + 16, pk);
         }
         l += (sf[0] + sf[1]) + (sf[2] + sf[3]);

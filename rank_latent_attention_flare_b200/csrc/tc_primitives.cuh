@@ -13,6 +13,10 @@
 namespace flare {
 namespace tc {
 
+#ifndef FLARE_POLY_PACKED
+#define FLARE_POLY_PACKED 1
+#endif
+
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
 constexpr uint32_t kSuspendHintNs = 100000u;       // per poll; far below the bound
 
@@ -89,26 +93,29 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 // As mbar_wait, but suspended between polls: for waits whose spinning would
 // take issue slots from the exponential-bound softmax warps on the same SM
 // sub-partition.  Same bound; false on timeout.
-__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity,
+                                                uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait_sleep(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait_sleep(bar, parity)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) return false;
+    if (globaltimer() - t0 > limit_ns) return false;
   }
 }
 
-// Waits for the phase with the given parity to complete; false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Waits for the phase with the given parity to complete; false once
+// limit_ns have passed without it.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) return false;
+    if (globaltimer() - t0 > limit_ns) return false;
   }
 }
 
@@ -358,6 +365,12 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Warp votes.  Every branch that guards a warp-collective tcgen05 instruction
 // (.sync.aligned loads, stores and waits) must be taken by all 32 lanes, so
 // per-lane decisions in front of one go through these.
@@ -454,6 +467,37 @@ __device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
+__device__ __forceinline__ uint64_t sub_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// 2^x for a pair of values (x.lo, x.hi) on the FMA pipe, as exp2_fma but
+// with the range reduction and the polynomial in packed fp32x2 arithmetic
+// (one instruction for both values): two clamps, three packed adds, three
+// packed FMAs and two exponent-field adds per pair.  The same
+// coefficients, hence the same error bound (7.5e-5 relative) and domain
+// (x <= 126; x below -125 gives 2^-125 times the polynomial).
+__device__ __forceinline__ void exp2_fma_pair(uint64_t x, float& r0, float& r1) {
+  constexpr float kE0 = 0.9999280571937561f, kE1 = 0.6932609677314758f;
+  constexpr float kE2 = 0.2426111251115799f, kE3 = 0.0551716685295105f;
+  constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
+  float x0, x1;
+  split_f32x2(x, x0, x1);
+  const uint64_t xc = f32x2(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t rr = f32x2(kRound, kRound);
+  const uint64_t t = add_f32x2(xc, rr);
+  const uint64_t f = sub_f32x2(xc, sub_f32x2(t, rr));
+  uint64_t p = fma_f32x2(f32x2(kE3, kE3), f, f32x2(kE2, kE2));
+  p = fma_f32x2(p, f, f32x2(kE1, kE1));
+  p = fma_f32x2(p, f, f32x2(kE0, kE0));
+  float t0, t1, p0, p1;
+  split_f32x2(t, t0, t1);
+  split_f32x2(p, p0, p1);
+  r0 = __uint_as_float((__float_as_uint(t0) << 23) + __float_as_uint(p0));
+  r1 = __uint_as_float((__float_as_uint(t1) << 23) + __float_as_uint(p1));
+}
 
 // 2^(a*c + neg) for NP consecutive pairs of logits: bf16 pairs into pk, the
 // values summed into s (s[0], s[2] collect even lanes, s[1], s[3] odd ones).
@@ -464,12 +508,25 @@ __device__ __forceinline__ void exp_pack_pairs(const uint32_t* a, float c, float
   uint64_t acc[2] = {f32x2(s[0], s[1]), f32x2(s[2], s[3])};
 #pragma unroll
   for (int t = 0; t < NP; ++t) {
-    float x0, x1;
-    split_f32x2(fma_f32x2(f32x2(__uint_as_float(a[2 * t]), __uint_as_float(a[2 * t + 1])), c2, n2),
-                x0, x1);
+    const uint64_t x =
+        fma_f32x2(f32x2(__uint_as_float(a[2 * t]), __uint_as_float(a[2 * t + 1])), c2, n2);
     const bool poly = POLY_EVERY > 0 && (t % (POLY_EVERY > 0 ? POLY_EVERY : 1)) == POLY_EVERY - 1;
-    const float p0 = poly ? exp2_fma(x0) : ex2(x0);
-    const float p1 = poly ? exp2_fma(x1) : ex2(x1);
+    float p0, p1;
+    if (poly) {
+#if FLARE_POLY_PACKED
+      exp2_fma_pair(x, p0, p1);
+#else
+      float x0, x1;
+      split_f32x2(x, x0, x1);
+      p0 = exp2_fma(x0);
+      p1 = exp2_fma(x1);
+#endif
+    } else {
+      float x0, x1;
+      split_f32x2(x, x0, x1);
+      p0 = ex2(x0);
+      p1 = ex2(x1);
+    }
     acc[t & 1] = add_f32x2(acc[t & 1], f32x2(p0, p1));
     pk[t] = pack_bf16(p0, p1);
   }
@@ -484,9 +541,10 @@ __device__ __forceinline__ void exp_pack32(const uint32_t (&a)[32], float c, flo
 }
 
 // p = 2^(a*c + neg) for 16 logits: 8 bf16 pairs, sums into four accumulators.
+template <int POLY_EVERY = 0>
 __device__ __forceinline__ void exp_pack16(const uint32_t (&a)[16], float c, float neg,
                                            uint32_t (&pk)[8], float (&s)[4]) {
-  exp_pack_pairs<8, 0>(a, c, neg, pk, s);
+  exp_pack_pairs<8, POLY_EVERY>(a, c, neg, pk, s);
 }
 
 }  // namespace tc

@@ -330,6 +330,54 @@ def flare_fwd_noalloc(Q, K, V, scale: Optional[float] = None, *, save: bool = Fa
 
 # ------------------------------------------------- context parallelism (stages)
 
+def noalloc_device_status(stream=None) -> int:
+    """Reads and clears the device error word of flare_fwd_noalloc's scratch
+    array on the current device (synchronises the stream); returns its
+    detail code (0: no bounded wait ran out)."""
+    detail = ctypes.c_uint32(0)
+    st = _lib.load().flare_noalloc_device_status(ctypes.byref(detail), _stream(stream))
+    if st not in (0, 5):
+        _lib.check(st, "flare_noalloc_device_status")
+    return int(detail.value)
+
+
+def probe_unit_rates(device=None, stream=None) -> dict:
+    """Measured throughputs of the units the kernels are bound by
+    (flare_probe_unit_rates): MUFU exponentials, scalar and packed fp32 FMAs
+    and their mix, per SM per SM clock, with the SM clock seen by the probe
+    kernels.  Synchronises the device."""
+    lib = _lib.load()
+    n = int(lib.flare_probe_scratch_bytes())
+    if n == 0:
+        raise RuntimeError("flare_probe_scratch_bytes: no CUDA device")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    scratch = torch.empty(n, dtype=torch.uint8, device=dev)
+    out = _lib.UnitRates()
+    _lib.check(lib.flare_probe_unit_rates(_ptr(scratch), n, ctypes.byref(out), _stream(stream)),
+               "flare_probe_unit_rates")
+    return {name: getattr(out, name) for name, _ in _lib.UnitRates._fields_}
+
+
+def eval_exp2(x: torch.Tensor, form: int, stream=None) -> torch.Tensor:
+    """2^x with one of the kernels' exponentials (flare_eval_exp2): form 0 =
+    MUFU ex2.approx, 1 = FMA-pipe polynomial, 2 = the packed polynomial."""
+    _need_cuda(x)
+    if x.dtype != torch.float32:
+        raise TypeError("eval_exp2 takes float32")
+    y = torch.empty_like(x)
+    _lib.check(_lib.load().flare_eval_exp2(_ptr(x), _ptr(y), x.numel(), form, _stream(stream)),
+               "flare_eval_exp2")
+    return y
+
+
+def selftest_wait_timeout(workspace: torch.Tensor, limit_ns: int, stream=None) -> None:
+    """Launches the bounded-wait self-test (flare_selftest_wait_timeout) on
+    a workspace of at least 512 bytes; read the result with device_status."""
+    _lib.check(_lib.load().flare_selftest_wait_timeout(_ptr(workspace), workspace.numel(),
+                                                       int(limit_ns), _stream(stream)),
+               "flare_selftest_wait_timeout")
+
+
 def records_layout(B: int, H: int, N: int, M: int, D: int, dtype: torch.dtype):
     """(records_per_bh, ml_offset, acc_offset): where flare_encode leaves its
     chunk records in a FLARE_OP_FWD workspace."""

@@ -50,6 +50,25 @@ def test_noalloc_matches_workspace_entry_point(dtype, B, H, N, M, D, per_batch_q
         torch.cuda.synchronize()
         assert not torch.isnan(Y.float()).any()
         assert_close(Y, ref.float().cpu().double().numpy(), dtype, f"Y seed {seed}")
+    assert fl.noalloc_device_status() == 0   # no bounded wait ran out
+
+
+def test_noalloc_large_then_small_call():
+    # A large call fills more of the shared scratch array (more chunk
+    # records, other offsets) than a small one reads: the small call after
+    # it must not pick up the large call's leftovers.
+    cases = [(torch.bfloat16, 1, 2, 5000, 256, 32), (torch.bfloat16, 1, 1, 777, 128, 32),
+             (torch.bfloat16, 1, 2, 5000, 256, 32), (torch.bfloat16, 2, 1, 300, 128, 16)]
+    for i, (dtype, B, H, N, M, D) in enumerate(cases):
+        s = 1.0 / math.sqrt(D)
+        x = make_inputs(B, H, N, M, D, dtype=dtype, seed=30 + i)
+        g = {k: v.cuda() for k, v in x.items()}
+        ref = fl.flare_fwd(g["Q"], g["K"], g["V"], s)
+        Y = torch.full_like(g["K"], float("nan"))
+        assert _noalloc_c_call(g, Y, s) == 0
+        torch.cuda.synchronize()
+        assert_close(Y, ref.float().cpu().double().numpy(), dtype, f"Y case {i}")
+    assert fl.noalloc_device_status() == 0
 
 
 def test_noalloc_rejects_sizes_beyond_the_scratch_array():
