@@ -34,12 +34,22 @@ from flare_inputs import WORKLOADS, make_inputs  # noqa: E402
 WORKLOAD = WORKLOADS["c3_fwd_bf16_1M"]
 METRIC = "FLARE fwd tokens/s at N=1M, M=256, H=16, D=32 bf16; % of roofline"
 
-# Nominal B200 unit counts used to derive the exp (MUFU) ceiling: 148 SMs,
-# 16 ex2 results per clock per SM (4 per SM sub-partition), max SM clock
-# 1965 MHz.  The HBM and tensor ceilings come from MEASURED_PEAKS.json.
-SMS = 148
-MUFU_PER_CLK_SM = 16
+# The exponential ceilings come from the unit-rate probe the library carries
+# (flare_probe_unit_rates, run at the start of every bench): MUFU ex2 results
+# and packed fp32 FMAs per SM per clock, times the SM count and the max SM
+# clock.  Nominal B200 figures (148 SMs, 16 ex2 and 128 FMAs per clock per
+# SM) stand in only if the probe cannot run.  The HBM and tensor ceilings
+# come from MEASURED_PEAKS.json.
+NOMINAL_RATES = {"sms": 148, "ex2_per_clk_sm": 16.0, "fma_per_clk_sm": 128.0,
+                 "fma2_per_clk_sm": 128.0}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0}
+# fp32 FMA-pipe operations per softmax weight, counted from the kernels'
+# softmax loops: the scale-and-shift FMA and the row-sum add of every
+# weight; a weight computed by the polynomial adds the three adds of its
+# range reduction and the three FMAs of its Horner steps.  (The clamp, the
+# exponent-field add and the bf16 packing run on the integer/ALU pipe.)
+FMA_OPS_BASE = 2.0
+FMA_OPS_POLY = 6.0
 
 THROTTLE_BAD = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 
@@ -197,31 +207,78 @@ def workload_from_args(args):
     return w
 
 
-def roofline_entry(kernel_ms: dict, peaks: dict, peak_kind: str, w=WORKLOAD):
-    """Roofline of the dominant kernel (largest average duration).
+def measure_unit_rates():
+    """The library's unit-rate probe on the current device, or the nominal
+    B200 figures (marked as such) if it fails."""
+    import rank_latent_attention_flare_b200 as fl
+    try:
+        r = fl.probe_unit_rates()
+        r["source"] = "flare_probe_unit_rates, this run"
+        return r
+    except Exception as e:   # noqa: BLE001 -- reported, nominal figures used instead
+        r = dict(NOMINAL_RATES)
+        r["source"] = f"nominal (probe failed: {str(e)[:120]})"
+        return r
 
-    Both forward kernels are bound by exponentials (MUFU ex2): each computes
-    B*H*N*M of them per launch (encode: softmax over tokens of every latent
-    row; decode: softmax over latents of every token).  Their other ceilings
-    (tensor-pipe FLOPs, HBM bytes) are reported alongside.
+
+def exp_ceiling(exps: float, poly: float, rates: dict, clk_hz: float):
+    """Time floor of `exps` softmax weights of which a share `poly` runs as
+    the FMA-pipe polynomial and the rest on the MUFU: the slower of the two
+    units at its measured rate.  Returns (seconds, binding unit)."""
+    sms = rates["sms"]
+    mufu = rates["ex2_per_clk_sm"] * sms * clk_hz
+    fma = max(rates["fma_per_clk_sm"], rates["fma2_per_clk_sm"]) * sms * clk_hz
+    t_mufu = exps * (1.0 - poly) / mufu
+    t_fma = exps * (FMA_OPS_BASE + FMA_OPS_POLY * poly) / fma
+    return (t_mufu, "mufu") if t_mufu >= t_fma else (t_fma, "fma")
+
+
+def roofline_entry(kernel_ms: dict, peaks: dict, peak_kind: str, rates: dict, w=WORKLOAD):
+    """Roofline of the dominant kernel (largest average duration), and of
+    the whole forward.
+
+    Both forward kernels are bound by exponentials: each computes B*H*N*M
+    of them per launch (encode: softmax over tokens of every latent row;
+    decode: softmax over latents of every token), a fixed share of them as
+    a polynomial on the FMA pipe (flare_exp_split).  The ceiling is the
+    combined MUFU + FMA one for that share (exp_ceiling), so moving
+    exponentials to the polynomial cannot lift the fraction past 1; the
+    MUFU-only figure and the tensor-pipe and HBM fractions are reported
+    alongside.
     """
+    import rank_latent_attention_flare_b200 as fl
     name = max(("encode", "decode"), key=lambda k: kernel_ms[k])
-    t = kernel_ms[name] / 1e3
     exps = w.B * w.H * w.N * w.M
     clk = float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
-    mufu_peak = SMS * MUFU_PER_CLK_SM * clk / 1e9  # Gexp/s
+    mufu_peak = rates["ex2_per_clk_sm"] * rates["sms"] * clk / 1e9   # Gexp/s
+    ceil = {}
+    for k, kid in (("encode", 0), ("decode", 1)):
+        poly = fl.exp_split(kid, w.M, w.D, w.torch_dtype)
+        t_c, unit = exp_ceiling(exps, poly, rates, clk)
+        ceil[k] = {"poly_share": round(poly, 4), "t_ceiling_ms": round(t_c * 1e3, 4),
+                   "binding_unit": unit, "peak_gexps": round(exps / t_c / 1e9, 1)}
+    t = kernel_ms[name] / 1e3
     achieved = exps / t / 1e9
+    peak = ceil[name]["peak_gexps"]
     flops = 4 * w.B * w.H * w.N * w.M * w.D
-    if name == "encode":
-        hbm_bytes = 2 * w.B * w.H * w.N * w.D * 2          # K and V read once
-    else:
-        hbm_bytes = 2 * w.B * w.H * w.N * w.D * 2          # K read, Y written
-    traffic = read_traffic(name)
+    hbm_bytes = 2 * w.B * w.H * w.N * w.D * 2   # encode: K and V read; decode: K read, Y written
+    t_fwd = sum(kernel_ms.values()) / 1e3
+    t_fwd_ceil = sum(c["t_ceiling_ms"] for c in ceil.values()) / 1e3
     entry = {
         "bound": "alu", "kernel": f"flare_{name}", "achieved": round(achieved, 1),
-        "peak": round(mufu_peak, 1), "unit": "Gexp/s", "frac": round(achieved / mufu_peak, 4),
-        "traffic": traffic,
-        "peak_basis": f"MUFU ex2: {MUFU_PER_CLK_SM}/clk/SM x {SMS} SMs x {clk / 1e6:.0f} MHz",
+        "peak": peak, "unit": "Gexp/s", "frac": round(achieved / peak, 4),
+        "traffic": read_traffic(name),
+        "peak_basis": (f"combined MUFU + FMA exponential ceiling at the kernel's polynomial share "
+                       f"{ceil[name]['poly_share']:.4f}: max((1-share)/MUFU, "
+                       f"({FMA_OPS_BASE:g} + {FMA_OPS_POLY:g} share)/FMA) per weight; MUFU "
+                       f"{rates['ex2_per_clk_sm']:.2f} ex2/clk/SM, FMA "
+                       f"{max(rates['fma_per_clk_sm'], rates['fma2_per_clk_sm']):.1f}/clk/SM "
+                       f"({rates['source']}) x {rates['sms']} SMs x {clk / 1e6:.0f} MHz"),
+        "mufu_only": {"peak": round(mufu_peak, 1), "frac": round(achieved / mufu_peak, 4)},
+        "kernels": ceil,
+        "forward": {"t_ms": round(t_fwd * 1e3, 4), "t_ceiling_ms": round(t_fwd_ceil * 1e3, 4),
+                    "frac": round(t_fwd_ceil / t_fwd, 4)},
+        "unit_rates": {k: (round(v, 3) if isinstance(v, float) else v) for k, v in rates.items()},
         "algorithmic": {"exps": exps, "tensor_flops": flops, "hbm_bytes": hbm_bytes},
         "other_ceilings": {
             "tensor_frac": round(flops / t / 1e12 / float(peaks["bf16_tflops"]), 4),
@@ -262,6 +319,7 @@ def run_ours(args, rank, world, local):
     w = workload_from_args(args)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    rates = measure_unit_rates()
     x = make_inputs(w.B, w.H, w.N, w.M, w.D, dtype=w.torch_dtype, seed=rank)
     g = {k: v.to(dev) for k, v in x.items()}
     ws = fl.alloc_workspace(fl.FLARE_OP_FWD, w.B, w.H, w.N, w.M, w.D, w.torch_dtype, dev)
@@ -352,7 +410,7 @@ def run_ours(args, rank, world, local):
         del hx, hY, dX
 
     peaks, peak_kind = load_peaks()
-    roof = roofline_entry(kernel_ms, peaks, peak_kind, w)
+    roof = roofline_entry(kernel_ms, peaks, peak_kind, rates, w)
 
     rows = None
     context = None
@@ -360,7 +418,7 @@ def run_ours(args, rank, world, local):
         del Y, ws
         g.clear()
         torch.cuda.empty_cache()
-        rows = time_other_rows(dev, peaks, peak_kind, seed=rank)
+        rows = time_other_rows(dev, peaks, peak_kind, seed=rank, rates=rates)
         try:
             context = time_sdpa_context(dev, seed=rank)
         except (RuntimeError, ValueError) as e:   # a torch build without a kernel for this shape
@@ -399,12 +457,16 @@ def run_ours(args, rank, world, local):
 
 # ------------------------------------------------------- the other rows
 
+_ROW_RATES = dict(NOMINAL_RATES, source="nominal")
+
+
 def _row_roofline(t_ms: float, exps: float, flops: float, hbm_bytes: float, peaks: dict,
                   peak_kind: str):
     """Roofline of a whole row: the slowest of the exponential, tensor and
-    HBM limits (each at its peak) over the measured time."""
+    HBM limits (each at its peak) over the measured time.  The exponential
+    limit takes every weight on the MUFU at the probe's measured rate."""
     clk = float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
-    mufu = SMS * MUFU_PER_CLK_SM * clk            # exp/s
+    mufu = _ROW_RATES["ex2_per_clk_sm"] * _ROW_RATES["sms"] * clk   # exp/s
     lim = {"exp": exps / mufu, "tensor": flops / (float(peaks["bf16_tflops"]) * 1e12),
            "hbm": hbm_bytes / (float(peaks["hbm_gbs"]) * 1e9)}
     bound = max(lim, key=lim.get)
@@ -414,13 +476,13 @@ def _row_roofline(t_ms: float, exps: float, flops: float, hbm_bytes: float, peak
             "exp_frac": round(lim["exp"] / t, 4), "tensor_frac": round(lim["tensor"] / t, 4),
             "hbm_frac": round(lim["hbm"] / t, 4),
             "algorithmic": {"exps": exps, "tensor_flops": flops, "hbm_bytes": hbm_bytes},
-            "peaks": f"MUFU {mufu / 1e9:.0f} Gexp/s (derived), {peak_kind} bf16 "
+            "peaks": f"MUFU {mufu / 1e9:.0f} Gexp/s ({_ROW_RATES['source']}), {peak_kind} bf16 "
                      f"{peaks['bf16_tflops']} TFLOP/s, {peak_kind} HBM {peaks['hbm_gbs']} GB/s"}
 
 
 def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0,
-                    which=("flare_pp_fwd", "flare_fwd_bwd", "flare_fwd_bwd_m256",
-                           "flare_pp_fwd_bwd", "flare_strided", "flare_varlen")):
+                    which=("flare_fwd_c2", "flare_pp_fwd", "flare_fwd_bwd", "flare_fwd_bwd_m256",
+                           "flare_pp_fwd_bwd", "flare_strided", "flare_varlen"), rates=None):
     """Times the FLARE++ forward (B=2 H=8 N=262,144 M=256 D=32) and the
     forward + backward of B=8 H=8 N=16,384 M=128 D=32, both bf16, on the
     same device with CUDA events (median of `iters` launches after 3
@@ -431,6 +493,8 @@ def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0,
 
     st = torch.cuda.current_stream()
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    if rates is not None:
+        _ROW_RATES.update(rates)
 
     def timed(fn):
         for _ in range(3):
@@ -448,6 +512,8 @@ def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0,
         return statistics.median(a.elapsed_time(b) for a, b in pairs)
 
     rows = {}
+    if "flare_fwd_c2" in which:
+        rows.update(_time_c2(dev, peaks, peak_kind, timed, seed))
     if "flare_pp_fwd" in which:
         rows.update(_time_pp(dev, peaks, peak_kind, timed, seed))
     if "flare_fwd_bwd" in which:
@@ -464,6 +530,39 @@ def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0,
     del flush_buf
     torch.cuda.empty_cache()
     return rows
+
+
+def _time_c2(dev, peaks, peak_kind, timed, seed):
+    """FLARE forward on the 256x256-mesh workload: B=4 H=8 N=65,536 M=128
+    D=16 bf16 (64 MiB per token tensor, so the L2 is flushed before each
+    launch).  Roofline as the headline's: the combined exponential ceilings
+    of its encode and decode at their polynomial shares, beside the tensor
+    and HBM fractions."""
+    import torch
+
+    import rank_latent_attention_flare_b200 as fl
+    w = WORKLOADS["c2_fwd_bf16_mesh256"]
+    x = make_inputs(w.B, w.H, w.N, w.M, w.D, dtype=w.torch_dtype, seed=seed)
+    g = {k: v.to(dev) for k, v in x.items()}
+    ws = fl.alloc_workspace(fl.FLARE_OP_FWD, w.B, w.H, w.N, w.M, w.D, w.torch_dtype, dev)
+    Y = torch.empty_like(g["K"])
+    ms = timed(lambda: fl.flare_fwd(g["Q"], g["K"], g["V"], w.scale, workspace=ws, out=Y))
+    if fl.device_status(ws) != 0:
+        raise RuntimeError("device wait ran out in the mesh-sized forward")
+    u = w.B * w.H * w.N
+    exps = u * w.M
+    clk = float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
+    t_ceil = sum(exp_ceiling(exps, fl.exp_split(k, w.M, w.D, w.torch_dtype), _ROW_RATES, clk)[0]
+                 for k in (0, 1))
+    roof = _row_roofline(ms, 2.0 * exps, 8.0 * u * w.M * w.D, 4.0 * u * w.D * 2, peaks,
+                         peak_kind)
+    roof["combined_exp_ceiling_ms"] = round(t_ceil * 1e3, 4)
+    roof["frac"] = round(t_ceil / (ms / 1e3), 4)
+    roof["bound"] = "exp (combined MUFU + FMA)"
+    return {"flare_fwd_c2": {
+        "workload": f"FLARE fwd B={w.B} H={w.H} N={w.N} M={w.M} D={w.D} bf16 (mesh 256x256)",
+        "ms": round(ms, 4), "tokens_per_s": w.B * w.N / (ms / 1e3), "l2": "flushed (256 MB)",
+        "roofline": roof}}
 
 
 def _time_pp(dev, peaks, peak_kind, timed, seed):
@@ -703,7 +802,7 @@ def run_row(args, rank, local):
     torch.cuda.set_device(dev)
     peaks, peak_kind = load_peaks()
     rows = time_other_rows(dev, peaks, peak_kind, iters=max(1, args.steps), seed=rank,
-                           which=(args.row,))
+                           which=(args.row,), rates=measure_unit_rates())
     if rank == 0:
         print(json.dumps({"row": args.row, **rows[args.row]}), flush=True)
 
@@ -757,7 +856,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true",
                     help="skip the FLARE++ and forward+backward timings")
-    ap.add_argument("--row", choices=["flare_pp_fwd", "flare_fwd_bwd", "flare_fwd_bwd_m256",
+    ap.add_argument("--row", choices=["flare_fwd_c2", "flare_pp_fwd", "flare_fwd_bwd",
+                                      "flare_fwd_bwd_m256",
                                       "flare_pp_fwd_bwd",
                                       "flare_strided", "flare_varlen"],
                     default=None,

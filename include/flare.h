@@ -314,8 +314,9 @@ FLARE_API flare_status_t flare_decode(const void* Q, int64_t q_batch_stride, con
  *   the shards; then flare_pp_bwd_shard_tail with that dQ_dyn (input dtype)
  *   on the same workspace: the first encode's gradient over the shard, added
  *   to the shard's dK and dV, and its float32 part of dQ [H,M,D] (summed
- *   over the batch).  dQ = the sum over the shards of those parts + the sum
- *   over the batch of dQ_dyn.
+ *   over the batch).  Exactly one shard passes add_dq_dyn = 1, which adds
+ *   the sum over the batch of dQ_dyn to its part (the others pass 0), so
+ *   that dQ = the sum over the shards of the parts.
  */
 FLARE_API flare_status_t flare_records_layout(int64_t B, int64_t H, int64_t N, int64_t M,
                                               int64_t D, flare_dtype_t dtype,
@@ -336,7 +337,8 @@ FLARE_API flare_status_t flare_bwd_shard_dz(const void* Q, int64_t q_batch_strid
                                             size_t workspace_bytes, void* stream);
 FLARE_API flare_status_t flare_pp_bwd_shard_tail(const void* Q, const void* K, const void* V,
                                                  const float* Z1, const float* lse1,
-                                                 const void* dQ_dyn, float* dQ_part, void* dK,
+                                                 const void* dQ_dyn, int add_dq_dyn,
+                                                 float* dQ_part, void* dK,
                                                  void* dV, int64_t B, int64_t H, int64_t N,
                                                  int64_t M, int64_t D, flare_dtype_t dtype,
                                                  float scale, void* workspace,
@@ -456,14 +458,28 @@ FLARE_API flare_status_t flare_probe_unit_rates(void* scratch, size_t scratch_by
                                                 flare_unit_rates_t* out, void* stream);
 
 /*
+ * Share of the exponentials of the forward's encode (kernel 0) or decode
+ * (kernel 1) that runs as the FMA-pipe polynomial instead of the MUFU, for
+ * a forward call with these M, D and dtype (0 for the CUDA-core kernels,
+ * which use exp2f).  The roofline of an exponential-bound kernel depends on
+ * it: the MUFU then computes (1 - share) of the exponentials.
+ */
+FLARE_API flare_status_t flare_exp_split(int kernel, int64_t M, int64_t D, flare_dtype_t dtype,
+                                         double* poly_fraction);
+
+/*
  * y[i] = 2^x[i] for n floats (device pointers), with the exponential the
  * kernels use: form 0 = the MUFU instruction (ex2.approx.ftz.f32), form 1 =
  * the FMA-pipe polynomial evaluated one value at a time, form 2 = the same
- * polynomial in packed fp32x2 arithmetic, two values at a time (the form
- * the softmax loops use).  The polynomial: round-to-nearest range
- * reduction x = j + f, a degree-3 minimax fit of 2^f on [-1/2, 1/2]
- * (relative error 7.5e-5), j added to the exponent field; valid for
- * x <= 126, inputs below -125 are clamped to -125.  Enqueued on `stream`.
+ * polynomial in packed fp32x2 arithmetic, two values at a time (the form of
+ * the backward's fixed-weight pass), form 3 = the packed polynomial with
+ * the exponent clamped by a saturating FMA (the form the forward's softmax
+ * loops use).  The polynomial: round-to-nearest range reduction x = j + f,
+ * a degree-3 minimax fit of 2^f on [-1/2, 1/2] (relative error 7.5e-5), j
+ * added to the exponent field.  Forms 1 and 2 are valid for x <= 126 and
+ * clamp inputs below -125 to -125; form 3 clamps x to [-125, 126] and adds
+ * at most 5.2e-6 relative error (the rounding of (x + 125) / 251).
+ * Enqueued on `stream`.
  */
 FLARE_API flare_status_t flare_eval_exp2(const float* x, float* y, int64_t n, int form,
                                          void* stream);

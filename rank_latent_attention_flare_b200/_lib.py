@@ -84,7 +84,7 @@ SIGNATURES = {
     "flare_records_layout": (_i32, [_i64, _i64, _i64, _i64, _i64, _i32, _i64p, _szp, _szp]),
     "flare_combine_shards": (_i32, [_i64, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _i32, _vp,
                                     _vp, _vp, _vp, _vp, _sz, _vp]),
-    "flare_pp_bwd_shard_tail": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
+    "flare_pp_bwd_shard_tail": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _i64, _i64,
                                        _i64, _i64, _i64, _i32, _f32, _vp, _sz, _vp]),
     "flare_bwd_shard_dz": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
                                   _i64, _i32, _f32, _vp, _sz, _vp]),
@@ -104,6 +104,7 @@ SIGNATURES = {
     "flare_probe_scratch_bytes": (_sz, []),
     "flare_probe_unit_rates": (_i32, [_vp, _sz, ctypes.POINTER(UnitRates), _vp]),
     "flare_eval_exp2": (_i32, [_vp, _vp, _i64, _i32, _vp]),
+    "flare_exp_split": (_i32, [_i32, _i64, _i64, _i32, ctypes.POINTER(ctypes.c_double)]),
     "flare_selftest_wait_timeout": (_i32, [_vp, _sz, ctypes.c_uint64, _vp]),
 }
 

@@ -551,7 +551,8 @@ flare_status_t flare_bwd_shard_finish(const void* Q, int64_t qbs, const void* K,
 
 flare_status_t flare_pp_bwd_shard_tail(const void* Q, const void* K, const void* V,
                                        const float* Z1, const float* lse1, const void* dQ_dyn,
-                                       float* dQ_part, void* dK, void* dV, int64_t B, int64_t H,
+                                       int add_dq_dyn, float* dQ_part, void* dK, void* dV,
+                                       int64_t B, int64_t H,
                                        int64_t N, int64_t M, int64_t D, flare_dtype_t dt,
                                        float scale, void* workspace, size_t workspace_bytes,
                                        void* stream) {
@@ -570,7 +571,8 @@ flare_status_t flare_pp_bwd_shard_tail(const void* Q, const void* K, const void*
   FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
   g_error_detail[0] = 0;
   FLARE_CUDA(launch_pp_bwd_tail(Q, K, V, Z1, lse1, dQ_dyn, nullptr, dK, dV, Dims{B, H, N, M, D}, dt,
-                                scale, L, (char*)workspace, (cudaStream_t)stream, dQ_part));
+                                scale, L, (char*)workspace, (cudaStream_t)stream, dQ_part,
+                                add_dq_dyn != 0));
   return FLARE_OK;
 }
 

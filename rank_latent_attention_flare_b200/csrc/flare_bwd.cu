@@ -521,12 +521,12 @@ __global__ void __launch_bounds__(kT)
 
 // dQ[h] = sum over b of (dQ_dyn[b, h] + sum over chunks of the encode
 // partials), in a fixed order.  One thread per output element.  With dq32
-// (a shard of a context-parallel backward) only the encode partials are
-// summed, into float32.
+// (a shard of a context-parallel backward) the sum goes to float32 and
+// includes dQ_dyn only when add_dqd.
 template <typename T>
 __global__ void pp_dq_kernel(const T* __restrict__ dqd, const float* __restrict__ dq_part, int B,
                              int H, int M, int D, int chunks, T* __restrict__ dQ,
-                             float* __restrict__ dq32) {
+                             float* __restrict__ dq32, bool add_dqd) {
   const int64_t per = (int64_t)H * M * D;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= per) return;
@@ -535,7 +535,7 @@ __global__ void pp_dq_kernel(const T* __restrict__ dqd, const float* __restrict_
   float acc = 0.f;
   for (int b = 0; b < B; ++b) {
     const int64_t bh = (int64_t)b * H + h;
-    if (!dq32) acc += to_f(dqd[(int64_t)b * per + i]);
+    if (add_dqd) acc += to_f(dqd[(int64_t)b * per + i]);
     for (int k = 0; k < chunks; ++k) acc += dq_part[(bh * chunks + k) * (int64_t)M * D + md];
   }
   if (dq32)
@@ -548,7 +548,7 @@ template <typename T, int D>
 cudaError_t pp_tail_t(const void* Q, const void* K, const void* V, const float* z1,
                       const float* lse1, const void* dqd, void* dQ, void* dK, void* dV,
                       const Dims& d, float scale, const WsLayout& L, char* ws, cudaStream_t st,
-                      float* dq32) {
+                      float* dq32, bool add_dqd) {
   const ChunkPlan& p = L.ppe;
   const int M = (int)d.M;
   const int64_t BH = d.BH();
@@ -572,7 +572,8 @@ cudaError_t pp_tail_t(const void* Q, const void* K, const void* V, const float* 
   const int64_t per = d.H * M * D;
   pp_dq_kernel<T><<<(unsigned)((per + 255) / 256), 256, 0, st>>>((const T*)dqd, dqe, (int)d.B,
                                                                  (int)d.H, M, D, p.chunks,
-                                                                 (T*)dQ, dq32);
+                                                                 (T*)dQ, dq32,
+                                                                 dq32 == nullptr || add_dqd);
   return cudaPeekAtLastError();
 }
 
@@ -581,11 +582,12 @@ cudaError_t pp_tail_t(const void* Q, const void* K, const void* V, const float* 
 cudaError_t launch_pp_bwd_tail(const void* Q, const void* K, const void* V, const float* z1,
                                const float* lse1, const void* dqd, void* dQ, void* dK, void* dV,
                                const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,
-                               char* ws, cudaStream_t st, float* dq32) {
+                               char* ws, cudaStream_t st, float* dq32, bool add_dqd) {
   if (choose_path(d.N, d.M, d.D, dt).tc_bwd)
-    return launch_tc_enc_bwd(Q, K, V, z1, lse1, dqd, dQ, dK, dV, d, scale, L, ws, st, dq32);
+    return launch_tc_enc_bwd(Q, K, V, z1, lse1, dqd, dQ, dK, dV, d, scale, L, ws, st, dq32,
+                             add_dqd);
 #define FLARE_PP_TAIL_T(T, DD) \
-  pp_tail_t<T, DD>(Q, K, V, z1, lse1, dqd, dQ, dK, dV, d, scale, L, ws, st, dq32)
+  pp_tail_t<T, DD>(Q, K, V, z1, lse1, dqd, dQ, dK, dV, d, scale, L, ws, st, dq32, add_dqd)
   if (dt == FLARE_F32) return d.D == 16 ? FLARE_PP_TAIL_T(float, 16) : FLARE_PP_TAIL_T(float, 32);
   return d.D == 16 ? FLARE_PP_TAIL_T(__nv_bfloat16, 16) : FLARE_PP_TAIL_T(__nv_bfloat16, 32);
 #undef FLARE_PP_TAIL_T

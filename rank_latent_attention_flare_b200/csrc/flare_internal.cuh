@@ -99,6 +99,31 @@ inline Path choose_path(int64_t N, int64_t M, int64_t D, flare_dtype_t dt) {
   return p;
 }
 
+// Split of the forward's exponentials between the MUFU (ex2.approx) and the
+// FMA-pipe polynomial: in the tensor-core encode, every kEncPolyEvery-th
+// pair of each 48-logit row tile's first 32 logits and every
+// kEncPolyEvery16-th pair of its last 16 runs as the polynomial (0 = none);
+// in the decode, every kDecPolyEvery-th pair of each 32-logit chunk.
+#ifndef FLARE_ENC_POLY32
+#define FLARE_ENC_POLY32 4
+#endif
+#ifndef FLARE_ENC_POLY16
+#define FLARE_ENC_POLY16 4
+#endif
+#ifndef FLARE_DEC_POLY
+#define FLARE_DEC_POLY 16
+#endif
+constexpr int kEncPolyEvery = FLARE_ENC_POLY32;
+constexpr int kEncPolyEvery16 = FLARE_ENC_POLY16;
+constexpr int kDecPolyEvery = FLARE_DEC_POLY;
+
+// Share of a tensor-core kernel's exponentials computed by the polynomial.
+constexpr double enc_poly_fraction() {
+  return ((kEncPolyEvery > 0 ? 16 / kEncPolyEvery : 0) +
+          (kEncPolyEvery16 > 0 ? 8 / kEncPolyEvery16 : 0)) / 24.0;
+}
+constexpr double dec_poly_fraction() { return (kDecPolyEvery > 0 ? 16 / kDecPolyEvery : 0) / 16.0; }
+
 constexpr int kSimtEncTile = 64;
 constexpr int kSimtEncThreads = 256;
 constexpr int kSimtDecThreads = 128;
@@ -416,16 +441,18 @@ cudaError_t launch_tc_bwd(const void* Q, int64_t qbs, const void* K, const void*
 // FLARE++'s first-encode gradient on the tensor cores (bf16, M = 128,
 // D in {16, 32}): adds into dK, dV and writes dQ (sum over the batch of dZ1
 // and the encode's dQ); reuses the tensor-core backward's workspace.
-// With dq32 (a shard of a context-parallel backward) only the encode's part
-// of dQ is written, in float32, and dZ1 is not added to it.
+// With dq32 (a shard of a context-parallel backward) dQ is written in
+// float32 and holds the encode's part, plus the sum over the batch of dZ1
+// only when add_dz1 (one shard of the context-parallel group adds it).
 cudaError_t launch_tc_enc_bwd(const void* Q, const void* K, const void* V, const float* Z1,
                               const float* lse1, const void* dZ1, void* dQ, void* dK, void* dV,
                               const Dims& d, float scale, const WsLayout& L, char* ws,
-                              cudaStream_t st, float* dq32 = nullptr);
+                              cudaStream_t st, float* dq32 = nullptr, bool add_dz1 = false);
 cudaError_t launch_pp_bwd_tail(const void* Q, const void* K, const void* V, const float* z1,
                                const float* lse1, const void* dqd, void* dQ, void* dK, void* dV,
                                const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,
-                               char* ws, cudaStream_t st, float* dq32 = nullptr);
+                               char* ws, cudaStream_t st, float* dq32 = nullptr,
+                               bool add_dqd = false);
 cudaError_t launch_bwd(const void* Q, int64_t qbs, const void* K, const void* V, const void* dY,
                        const float* Z, const float* lse, void* dQ, void* dK, void* dV,
                        const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,

@@ -186,8 +186,11 @@ __global__ void eval_exp2_kernel(const float* __restrict__ x, float* __restrict_
   } else if (form == 1) {
     r0 = exp2_fma(x0);
     r1 = exp2_fma(x1);
-  } else {
+  } else if (form == 2) {
     exp2_fma_pair(f32x2(x0, x1), r0, r1);
+  } else {
+    // the form the softmax loops use: 2^(c a + neg) with c = 1, neg = 0
+    exp2_fma_pair_logits(x0, x1, 1.0f / 251.0f, 125.0f / 251.0f, r0, r1);
   }
   y[2 * i] = r0;
   if (2 * i + 1 < n) y[2 * i + 1] = r1;
@@ -338,9 +341,21 @@ extern "C" flare_status_t flare_probe_unit_rates(void* scratch, size_t scratch_b
   return status;
 }
 
+extern "C" flare_status_t flare_exp_split(int kernel, int64_t M, int64_t D, flare_dtype_t dtype,
+                                          double* poly_fraction) {
+  if (poly_fraction == nullptr || (kernel != 0 && kernel != 1)) return FLARE_ERR_INVALID_ARG;
+  if ((D != 16 && D != 32) || M < 16 || M > 256 || (M % 16) != 0 ||
+      (dtype != FLARE_F32 && dtype != FLARE_BF16))
+    return FLARE_ERR_UNSUPPORTED;
+  const flare::Path p = flare::choose_path(1, M, D, dtype);
+  *poly_fraction =
+      !p.tc_fwd ? 0.0 : (kernel == 0 ? flare::enc_poly_fraction() : flare::dec_poly_fraction());
+  return FLARE_OK;
+}
+
 extern "C" flare_status_t flare_eval_exp2(const float* x, float* y, int64_t n, int form,
                                           void* stream) {
-  if (n < 0 || form < 0 || form > 2) return FLARE_ERR_INVALID_ARG;
+  if (n < 0 || form < 0 || form > 3) return FLARE_ERR_INVALID_ARG;
   if (n == 0) return FLARE_OK;
   if (x == nullptr || y == nullptr) return FLARE_ERR_INVALID_ARG;
   const int64_t pairs = (n + 1) / 2;

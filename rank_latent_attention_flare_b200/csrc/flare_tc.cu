@@ -3,30 +3,36 @@
 // TMEM lane (one row) per thread.
 //
 // Encode, per (b, h) and chunk of tokens ("Flare Fast Low Rank Attention"
-// skill page, section 2, latents as queries): for every 128-token tile
-//   S = Q K_tile^T            (tcgen05, M=128 latents x N=128 tokens x K=D)
-//   P = 2^(c S - m_ref)       (row = latent, online max with lazy rescale)
+// skill page, section 2, latents as queries), for every 48-token tile:
+//   S = Q K_tile^T            (tcgen05, M=128 latents x N=48 tokens x K=D)
+//   P = 2^(c S - m_ref)       (row = latent, running reference with lazy rescale)
 //   O += P V_tile             (tcgen05, A = P from TMEM, B = V from smem)
 // and at the end of the chunk the record (m_ref, l = row sum of P, O) goes to
-// the workspace for the log-sum-exp combine.
-// Decode (FLARE arXiv abstract, second SDPA call): for every 128-token tile
+// the workspace for the log-sum-exp combine.  Two CTAs share an SM.
+// Decode (FLARE arXiv abstract, second SDPA call), for every 128-token tile:
 //   S = K_tile Q^T            (M=128 tokens x N=M latents x K=D)
-//   P = 2^(c S - rowmax)      (row = token, whole row in one thread)
+//   P = 2^(c S - ref)         (row = token, whole row in one thread)
 //   Y = (P Z) / rowsum(P)     (A = P from TMEM, B = Z from smem)
-// so the N x M logits never leave the SM.
+// so the N x M logits never leave the SM.  One CTA per SM.
 //
 // The tensor-core backward with M = 256 reuses both pipelines (template
 // flags): the decode with the backward's per-token statistics in place of Y
 // (ST), and the encode with dY in place of V and fixed per-token weights in
 // place of the online softmax (DZ), which gives dZ = P_d^T dY.
 //
-// Roles per CTA (384 threads, three warpgroups): warps 0-3 and 4-7 are two
-// softmax warpgroups, warp 8 issues TMA loads, warp 9 owns TMEM and issues
-// the MMAs, warps 10-11 only lend their registers.  The CTA launches at 168
-// registers per thread; the producer warpgroup moves to 104 and the softmax
-// warpgroups to 200 (2 x 128 x 200 + 128 x 104 = 384 x 168, and each SM
-// sub-partition holds 2 x 200 + 104 <= 512 registers per lane).
-// Exponentials use ex2.approx (MUFU); c = scale * log2(e) is folded in.
+// Roles per CTA (384 threads, twelve warps):
+//   encode -- warps 0-3 and 4-7 are two softmax warpgroups; warp 8 issues the
+//     TMA loads; warps 9 and 10 issue the MMAs of softmax warpgroup 0 and 1
+//     (one elected lane each; warp 9 also owns TMEM); warp 11 only lends its
+//     registers.  Launched at 80 registers per thread, the producer
+//     warpgroup moves to 56 and the softmax warpgroups to 88
+//     (2 x 128 x 88 + 128 x 56 <= 384 x 80).
+//   decode -- the same softmax warpgroups (alternate tiles), warp 8 TMA,
+//     warp 9 TMEM and MMAs, warps 10-11 bound each K tile's row maxima
+//     (M = 256).  Launched at 168 registers per thread: the producer
+//     warpgroup moves to 104 and the softmax warpgroups to 200.
+// Exponentials use ex2.approx (MUFU) with c = scale * log2(e) folded in;
+// a fixed share of them runs as a polynomial on the FMA pipe instead.
 #include <cudaTypedefs.h>
 
 #include "flare_internal.cuh"
@@ -62,21 +68,12 @@ constexpr float kRedoLimit = 18446744073709551616.0f;   // 2^kRedoTau
 // (two per sub-partition, close to its register budget) gains only from the
 // last pair of each 32-column chunk (1.40 -> 1.38 ms; every 4th, 8th, 10th
 // or 12th pair is slower).
-#ifndef FLARE_ENC_POLY32
-#define FLARE_ENC_POLY32 4
-#endif
-#ifndef FLARE_ENC_POLY16
-#define FLARE_ENC_POLY16 0
-#endif
-#ifndef FLARE_DEC_POLY
-#define FLARE_DEC_POLY 16
-#endif
 #ifndef FLARE_ENC_MAXLESS
 #define FLARE_ENC_MAXLESS 1
 #endif
-constexpr int kEncPolyEvery = FLARE_ENC_POLY32;
-constexpr int kEncPolyEvery16 = FLARE_ENC_POLY16;
-constexpr int kDecPolyEvery = FLARE_DEC_POLY;
+#ifndef FLARE_ENC_ONEWAIT
+#define FLARE_ENC_ONEWAIT 0
+#endif
 // Decode reference of a token row (M = 256): the max of the first 32-logit
 // chunk read, used when c |k| max_m |q_m| (Cauchy-Schwarz: at least every
 // logit) lies at most this far (log2 units) above it, so no weight exceeds
@@ -474,6 +471,25 @@ __global__ void __launch_bounds__(kThreads, 2)
 #endif
         float sf[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t pa[16], pb[8];
+#if FLARE_ENC_ONEWAIT
+        {
+          // the tile's 48 logits as two loads in flight together, one wait
+          uint32_t a[32], a2[16];
+          tmem_ld32(tS, a);
+          tmem_ld16(tS + 32, a2);
+          tmem_wait_ld_dep48(a, a2);
+          if (!full) {   // masked columns get weight 0
+#pragma unroll
+            for (int t = 0; t < 32; ++t)
+              if (t < lo || t >= hi) a[t] = __float_as_uint(-INFINITY);
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+              if (32 + t < lo || 32 + t >= hi) a2[t] = __float_as_uint(-INFINITY);
+          }
+          exp_pack32<kEncPolyEvery>(a, c, neg, pa, sf);
+          exp_pack16<kEncPolyEvery16>(a2, c, neg, pb, sf);
+        }
+#else
         {
           uint32_t a[32];
           tmem_ld32(tS, a);
@@ -502,6 +518,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #endif
           exp_pack16<kEncPolyEvery16>(a, c, neg, pb, sf);
         }
+#endif
         const float sum = (sf[0] + sf[1]) + (sf[2] + sf[3]);
 #if FLARE_ENC_MAXLESS
         // Every weight of the tile is at most the tile's row sum, so the sum

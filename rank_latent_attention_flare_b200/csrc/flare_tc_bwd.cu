@@ -1772,7 +1772,7 @@ template <int D, int M, bool FLAT, bool VAR>
 cudaError_t tc_enc_bwd_t(const void* Q, const void* K, const void* V, const float* Z1,
                          const float* lse1, const void* dZ1, void* dQ, void* dK, void* dV,
                          const Dims& d, float scale, const WsLayout& L, char* ws, cudaStream_t st,
-                         float* dq32) {
+                         float* dq32, bool add_dz1) {
   const ChunkPlan& p = L.bwd;
   const int64_t BH = d.BH();
   const float c = scale * kLog2e;
@@ -1829,7 +1829,8 @@ cudaError_t tc_enc_bwd_t(const void* Q, const void* K, const void* V, const floa
   const int64_t total = d.H * M * D;
   bwd_dq_sum_kernel<<<(unsigned)((total / 4 + 127) / 128), 128, 0, st>>>(
       (const float4*)dqp, (int)d.B, (int)d.H, M, D, p.chunks, true,
-      dq32 ? nullptr : (const __nv_bfloat16*)dZ1, (__nv_bfloat16*)dQ, (float4*)dq32);
+      (dq32 && !add_dz1) ? nullptr : (const __nv_bfloat16*)dZ1, (__nv_bfloat16*)dQ,
+      (float4*)dq32);
   return cudaPeekAtLastError();
 }
 
@@ -1850,10 +1851,10 @@ template <int D, int M>
 cudaError_t tc_enc_bwd_dispatch(const void* Q, const void* K, const void* V, const float* Z1,
                                 const float* lse1, const void* dZ1, void* dQ, void* dK, void* dV,
                                 const Dims& d, float scale, const WsLayout& L, char* ws,
-                                cudaStream_t st, float* dq32) {
+                                cudaStream_t st, float* dq32, bool add_dz1) {
   const bool flat = tok_flat(d), var = d.lens != nullptr;
 #define FLARE_TC_ENC_T(F, V_) \
-  tc_enc_bwd_t<D, M, F, V_>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st, dq32)
+  tc_enc_bwd_t<D, M, F, V_>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st, dq32, add_dz1)
   if (flat) return var ? FLARE_TC_ENC_T(true, true) : FLARE_TC_ENC_T(true, false);
   return var ? FLARE_TC_ENC_T(false, true) : FLARE_TC_ENC_T(false, false);
 #undef FLARE_TC_ENC_T
@@ -1879,9 +1880,9 @@ cudaError_t launch_tc_bwd(const void* Q, int64_t qbs, const void* K, const void*
 cudaError_t launch_tc_enc_bwd(const void* Q, const void* K, const void* V, const float* Z1,
                               const float* lse1, const void* dZ1, void* dQ, void* dK, void* dV,
                               const Dims& d, float scale, const WsLayout& L, char* ws,
-                              cudaStream_t st, float* dq32) {
+                              cudaStream_t st, float* dq32, bool add_dz1) {
 #define FLARE_TC_ENC(D_, M_) \
-  tc_enc_bwd_dispatch<D_, M_>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st, dq32)
+  tc_enc_bwd_dispatch<D_, M_>(Q, K, V, Z1, lse1, dZ1, dQ, dK, dV, d, scale, L, ws, st, dq32, add_dz1)
   if (d.D == 32 && d.M == 128) return FLARE_TC_ENC(32, 128);
   if (d.D == 32 && d.M == 256) return FLARE_TC_ENC(32, 256);
   if (d.D == 16 && d.M == 128) return FLARE_TC_ENC(16, 128);

@@ -13,10 +13,6 @@
 namespace flare {
 namespace tc {
 
-#ifndef FLARE_POLY_PACKED
-#define FLARE_POLY_PACKED 1
-#endif
-
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
 constexpr uint32_t kSuspendHintNs = 100000u;       // per poll; far below the bound
 
@@ -247,6 +243,22 @@ __device__ __forceinline__ void tmem_wait_ld_dep16(uint32_t (&r)[16]) {
                : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
                  "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
                  "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
+}
+
+// tcgen05.wait::ld that names two loads' registers (32 + 16) as in/out
+// operands, for a 48-column row read as two loads in flight together.
+__device__ __forceinline__ void tmem_wait_ld_dep48(uint32_t (&r)[32], uint32_t (&q)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                 "+r"(r[30]), "+r"(r[31]), "+r"(q[0]), "+r"(q[1]), "+r"(q[2]), "+r"(q[3]),
+                 "+r"(q[4]), "+r"(q[5]), "+r"(q[6]), "+r"(q[7]), "+r"(q[8]), "+r"(q[9]),
+                 "+r"(q[10]), "+r"(q[11]), "+r"(q[12]), "+r"(q[13]), "+r"(q[14]), "+r"(q[15])
                :
                : "memory");
 }
@@ -499,29 +511,56 @@ __device__ __forceinline__ void exp2_fma_pair(uint64_t x, float& r0, float& r1) 
   r1 = __uint_as_float((__float_as_uint(t1) << 23) + __float_as_uint(p1));
 }
 
+// 2^(c a + neg) for a pair of raw logits (a0, a1) on the FMA pipe, with the
+// exponent x = c a + neg clamped to [-125, 126] for free: the saturating FMA
+// that computes y = (x + 125) / 251 = a cs + ns (cs = c / 251,
+// ns = (neg + 125) / 251) clamps y to [0, 1].  Then x = 251 y - 125, its
+// integer part j by round-to-nearest (t = 251 y + (1.5 * 2^23 - 125)) and
+// f = 251 y - 125 - j in packed FMAs, 2^f by the Horner steps of
+// exp2_fma, j added to the exponent field.  Error: the polynomial's
+// 7.5e-5 plus the rounding of y (at most 251 * 2^-25 in x, 5.2e-6
+// relative).  A clamped exponent keeps a large positive x finite (2^126),
+// so a sum of such weights still exposes it.
+__device__ __forceinline__ void exp2_fma_pair_logits(float a0, float a1, float cs, float ns,
+                                                     float& r0, float& r1) {
+  constexpr float kE0 = 0.9999280571937561f, kE1 = 0.6932609677314758f;
+  constexpr float kE2 = 0.2426111251115799f, kE3 = 0.0551716685295105f;
+  constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
+  float y0, y1;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(y0) : "f"(a0), "f"(cs), "f"(ns));
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(y1) : "f"(a1), "f"(cs), "f"(ns));
+  const uint64_t y = f32x2(y0, y1);
+  const uint64_t w = f32x2(251.0f, 251.0f), r = f32x2(kRound - 125.0f, kRound - 125.0f);
+  const uint64_t t = fma_f32x2(y, w, r);
+  const uint64_t f = fma_f32x2(y, w, sub_f32x2(r, t));
+  uint64_t p = fma_f32x2(f32x2(kE3, kE3), f, f32x2(kE2, kE2));
+  p = fma_f32x2(p, f, f32x2(kE1, kE1));
+  p = fma_f32x2(p, f, f32x2(kE0, kE0));
+  float t0, t1, p0, p1;
+  split_f32x2(t, t0, t1);
+  split_f32x2(p, p0, p1);
+  r0 = __uint_as_float((__float_as_uint(t0) << 23) + __float_as_uint(p0));
+  r1 = __uint_as_float((__float_as_uint(t1) << 23) + __float_as_uint(p1));
+}
+
 // 2^(a*c + neg) for NP consecutive pairs of logits: bf16 pairs into pk, the
 // values summed into s (s[0], s[2] collect even lanes, s[1], s[3] odd ones).
 template <int NP, int POLY_EVERY>
 __device__ __forceinline__ void exp_pack_pairs(const uint32_t* a, float c, float neg,
                                                uint32_t* pk, float (&s)[4]) {
   const uint64_t c2 = f32x2(c, c), n2 = f32x2(neg, neg);
+  const float cs = c * (1.0f / 251.0f), ns = (neg + 125.0f) * (1.0f / 251.0f);
   uint64_t acc[2] = {f32x2(s[0], s[1]), f32x2(s[2], s[3])};
 #pragma unroll
   for (int t = 0; t < NP; ++t) {
-    const uint64_t x =
-        fma_f32x2(f32x2(__uint_as_float(a[2 * t]), __uint_as_float(a[2 * t + 1])), c2, n2);
     const bool poly = POLY_EVERY > 0 && (t % (POLY_EVERY > 0 ? POLY_EVERY : 1)) == POLY_EVERY - 1;
     float p0, p1;
     if (poly) {
-#if FLARE_POLY_PACKED
-      exp2_fma_pair(x, p0, p1);
-#else
-      float x0, x1;
-      split_f32x2(x, x0, x1);
-      p0 = exp2_fma(x0);
-      p1 = exp2_fma(x1);
-#endif
+      exp2_fma_pair_logits(__uint_as_float(a[2 * t]), __uint_as_float(a[2 * t + 1]), cs, ns, p0,
+                           p1);
     } else {
+      const uint64_t x =
+          fma_f32x2(f32x2(__uint_as_float(a[2 * t]), __uint_as_float(a[2 * t + 1])), c2, n2);
       float x0, x1;
       split_f32x2(x, x0, x1);
       p0 = ex2(x0);

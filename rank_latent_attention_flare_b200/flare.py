@@ -358,9 +358,20 @@ def probe_unit_rates(device=None, stream=None) -> dict:
     return {name: getattr(out, name) for name, _ in _lib.UnitRates._fields_}
 
 
+def exp_split(kernel: int, M: int, D: int, dtype: torch.dtype) -> float:
+    """Share of the forward encode's (kernel 0) or decode's (kernel 1)
+    exponentials computed by the FMA-pipe polynomial (flare_exp_split)."""
+    code = _lib.FLARE_F32 if dtype == torch.float32 else _lib.FLARE_BF16
+    out = ctypes.c_double(0.0)
+    _lib.check(_lib.load().flare_exp_split(int(kernel), M, D, code, ctypes.byref(out)),
+               "flare_exp_split")
+    return float(out.value)
+
+
 def eval_exp2(x: torch.Tensor, form: int, stream=None) -> torch.Tensor:
     """2^x with one of the kernels' exponentials (flare_eval_exp2): form 0 =
-    MUFU ex2.approx, 1 = FMA-pipe polynomial, 2 = the packed polynomial."""
+    MUFU ex2.approx, 1 = FMA-pipe polynomial, 2 = the packed polynomial,
+    3 = the packed polynomial with its exponent clamped to [-125, 126]."""
     _need_cuda(x)
     if x.dtype != torch.float32:
         raise TypeError("eval_exp2 takes float32")
@@ -457,11 +468,14 @@ def flare_bwd_shard_finish(Q, K, V, dY, Z, lse, dZ, scale: Optional[float] = Non
 
 
 def flare_pp_bwd_shard_tail(Q, K, V, Z1, lse1, dQ_dyn, dK, dV, scale: Optional[float] = None, *,
-                            workspace: torch.Tensor, stream=None) -> torch.Tensor:
+                            workspace: torch.Tensor, add_dq_dyn: bool = False,
+                            stream=None) -> torch.Tensor:
     """FLARE++'s first-encode gradient over this shard, given dQ_dyn summed
     over the shards (input dtype) and the first encode's Z1, lse1 of the
     whole sequence: adds into dK, dV (in place) and returns the shard's
-    float32 part of dQ [H,M,D].  ``workspace``: FLARE_OP_PP_BWD size."""
+    float32 part of dQ [H,M,D]; with ``add_dq_dyn`` (on exactly one shard)
+    that part also holds the sum over the batch of dQ_dyn, so that dQ is the
+    sum of the parts.  ``workspace``: FLARE_OP_PP_BWD size."""
     _need_cuda(Q, K, V, Z1, lse1, dQ_dyn, dK, dV, workspace)
     B, H, N, M, D, qbs = _dims(Q, K)
     if qbs != 0:
@@ -469,7 +483,8 @@ def flare_pp_bwd_shard_tail(Q, K, V, Z1, lse1, dQ_dyn, dK, dV, scale: Optional[f
     s = default_scale(D) if scale is None else float(scale)
     dQ = torch.empty(Q.shape, dtype=torch.float32, device=K.device)
     st = _lib.load().flare_pp_bwd_shard_tail(_ptr(Q), _ptr(K), _ptr(V), _ptr(Z1), _ptr(lse1),
-                                             _ptr(dQ_dyn), _ptr(dQ), _ptr(dK), _ptr(dV), B, H, N,
+                                             _ptr(dQ_dyn), int(bool(add_dq_dyn)), _ptr(dQ),
+                                             _ptr(dK), _ptr(dV), B, H, N,
                                              M, D, _dtype_code(K), s, _ptr(workspace),
                                              workspace.numel(), _stream(stream))
     _lib.check(st, "flare_pp_bwd_shard_tail")

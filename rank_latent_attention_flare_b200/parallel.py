@@ -110,6 +110,9 @@ def cp_flare_pp_bwd(Q, K, V, dY, Q_dyn, Z, lse, scale: Optional[float] = None, *
     # FLARE's backward with the per-batch latents Q_dyn, then the first encode's
     ws = ops.alloc_workspace(_f._lib.FLARE_OP_PP_BWD, B, H, N, M, D, K.dtype, K.device)
     dQd, dK, dV = _cp_bwd32(Q_dyn, K, V, dY, Z, lse, s, group, ops, ws)
-    dQe = ops.flare_pp_bwd_shard_tail(Q, K, V, Z1, lse1, dQd.to(K.dtype), dK, dV, s, workspace=ws)
-    dist.all_reduce(dQe, group=group)
-    return (dQd.sum(0) + dQe).to(Q.dtype), dK, dV
+    # rank 0's part also carries the sum over the batch of dQ_dyn, so the
+    # all-reduced parts are the whole dQ
+    dQp = ops.flare_pp_bwd_shard_tail(Q, K, V, Z1, lse1, dQd.to(K.dtype), dK, dV, s, workspace=ws,
+                                      add_dq_dyn=dist.get_rank(group) == 0)
+    dist.all_reduce(dQp, group=group)
+    return dQp.to(Q.dtype), dK, dV

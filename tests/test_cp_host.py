@@ -100,7 +100,7 @@ class _Stand:
         return (dq.sum(0) if Q.dim() == 3 else dq), dK, dV
 
     @staticmethod
-    def flare_pp_bwd_shard_tail(Q, K, V, Z1, lse1, dQd, dK, dV, s, *, workspace):
+    def flare_pp_bwd_shard_tail(Q, K, V, Z1, lse1, dQd, dK, dV, s, *, workspace, add_dq_dyn=False):
         # the first encode's gradient with upstream dZ1 = dQ_dyn, over the shard
         Qb = _Stand._q(Q, K.shape[0])
         P = torch.exp(s * torch.einsum("bhmd,bhnd->bhmn", Qb, K.double()) - lse1.double()[..., None])
@@ -108,7 +108,8 @@ class _Stand:
         dA = P * (dP - (dQd.double() * Z1.double()).sum(-1)[..., None])
         dV += torch.einsum("bhmn,bhmd->bhnd", P, dQd.double())
         dK += s * torch.einsum("bhmn,bhmd->bhnd", dA, Qb)
-        return (s * torch.einsum("bhmn,bhnd->bhmd", dA, K.double())).sum(0)
+        part = (s * torch.einsum("bhmn,bhnd->bhmd", dA, K.double())).sum(0)
+        return part + dQd.double().sum(0) if add_dq_dyn else part
 
 
 def _free_port() -> int:

@@ -161,10 +161,9 @@ def test_sharded_flare_pp(B, H, N, M, D, dtype, G):
     parts = [fl.flare_bwd_shard_finish(Qd, Ks[r], Vs[r], dYs[r], Z, lse, dZ, s, workspace=wsb[r])
              for r in range(G)]
     dQd = sum(p[0] for p in parts)
-    dQ = dQd.sum(0)
-    for r in range(G):
-        dQ += fl.flare_pp_bwd_shard_tail(Q, Ks[r], Vs[r], Z1, lse1, dQd.to(dtype), parts[r][1],
-                                         parts[r][2], s, workspace=wsb[r])
+    dQ = sum(fl.flare_pp_bwd_shard_tail(Q, Ks[r], Vs[r], Z1, lse1, dQd.to(dtype), parts[r][1],
+                                        parts[r][2], s, workspace=wsb[r], add_dq_dyn=(r == 0))
+             for r in range(G))
     for w in wss + wsb:
         assert fl.device_status(w) == 0
     dK = torch.cat([p[1] for p in parts], dim=2)
