@@ -26,7 +26,7 @@ def test_header_coefficients_are_the_fit():
     c, err = fit_exp2_poly.remez_exp2()
     c32 = [float(np.float32(v)) for v in c]
     sets = _header_coeffs()
-    assert len(sets) == 2, "expected the scalar and the packed polynomial"
+    assert len(sets) == 3, "expected the scalar, packed and clamped packed polynomials"
     for s in sets:
         assert [float(np.float32(v)) for v in s] == c32
     assert err <= 7.5e-5
