@@ -481,7 +481,8 @@ def _row_roofline(t_ms: float, exps: float, flops: float, hbm_bytes: float, peak
 
 
 def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0,
-                    which=("flare_fwd_c2", "flare_pp_fwd", "flare_fwd_bwd", "flare_fwd_bwd_m256",
+                    which=("flare_fwd_c2", "flare_fwd_m64", "flare_pp_fwd", "flare_fwd_bwd",
+                           "flare_fwd_bwd_m256",
                            "flare_pp_fwd_bwd", "flare_strided", "flare_varlen"), rates=None):
     """Times the FLARE++ forward (B=2 H=8 N=262,144 M=256 D=32) and the
     forward + backward of B=8 H=8 N=16,384 M=128 D=32, both bf16, on the
@@ -514,6 +515,8 @@ def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0,
     rows = {}
     if "flare_fwd_c2" in which:
         rows.update(_time_c2(dev, peaks, peak_kind, timed, seed))
+    if "flare_fwd_m64" in which:
+        rows.update(_time_c2(dev, peaks, peak_kind, timed, seed, M=64, row="flare_fwd_m64"))
     if "flare_pp_fwd" in which:
         rows.update(_time_pp(dev, peaks, peak_kind, timed, seed))
     if "flare_fwd_bwd" in which:
@@ -532,16 +535,22 @@ def time_other_rows(dev, peaks, peak_kind, iters: int = 20, seed: int = 0,
     return rows
 
 
-def _time_c2(dev, peaks, peak_kind, timed, seed):
+def _time_c2(dev, peaks, peak_kind, timed, seed, M=None, row="flare_fwd_c2"):
     """FLARE forward on the 256x256-mesh workload: B=4 H=8 N=65,536 M=128
     D=16 bf16 (64 MiB per token tensor, so the L2 is flushed before each
-    launch).  Roofline as the headline's: the combined exponential ceilings
-    of its encode and decode at their polynomial shares, beside the tensor
-    and HBM fractions."""
+    launch), or the same with another latent count M (the flare_fwd_m64
+    row: 64 latents, padded to the kernels' 128-row latent tile).  Roofline
+    as the headline's: the combined exponential ceilings of its encode and
+    decode at their polynomial shares for the M latents of the workload,
+    beside the tensor and HBM fractions."""
+    import dataclasses
+
     import torch
 
     import rank_latent_attention_flare_b200 as fl
     w = WORKLOADS["c2_fwd_bf16_mesh256"]
+    if M is not None:
+        w = dataclasses.replace(w, M=M)
     x = make_inputs(w.B, w.H, w.N, w.M, w.D, dtype=w.torch_dtype, seed=seed)
     g = {k: v.to(dev) for k, v in x.items()}
     ws = fl.alloc_workspace(fl.FLARE_OP_FWD, w.B, w.H, w.N, w.M, w.D, w.torch_dtype, dev)
@@ -559,8 +568,9 @@ def _time_c2(dev, peaks, peak_kind, timed, seed):
     roof["combined_exp_ceiling_ms"] = round(t_ceil * 1e3, 4)
     roof["frac"] = round(t_ceil / (ms / 1e3), 4)
     roof["bound"] = "exp (combined MUFU + FMA)"
-    return {"flare_fwd_c2": {
+    return {row: {
         "workload": f"FLARE fwd B={w.B} H={w.H} N={w.N} M={w.M} D={w.D} bf16 (mesh 256x256)",
+        "fwd_path": fl.fwd_path(w.B, w.H, w.N, w.M, w.D, w.torch_dtype),
         "ms": round(ms, 4), "tokens_per_s": w.B * w.N / (ms / 1e3), "l2": "flushed (256 MB)",
         "roofline": roof}}
 
@@ -856,7 +866,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true",
                     help="skip the FLARE++ and forward+backward timings")
-    ap.add_argument("--row", choices=["flare_fwd_c2", "flare_pp_fwd", "flare_fwd_bwd",
+    ap.add_argument("--row", choices=["flare_fwd_c2", "flare_fwd_m64", "flare_pp_fwd", "flare_fwd_bwd",
                                       "flare_fwd_bwd_m256",
                                       "flare_pp_fwd_bwd",
                                       "flare_strided", "flare_varlen"],

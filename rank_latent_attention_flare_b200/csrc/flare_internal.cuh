@@ -88,11 +88,17 @@ struct Path {
   bool tc_bwd = false;  // tcgen05 backward (two passes over the tokens)
 };
 
-// The tcgen05 kernels cover bf16 with M in {128, 256} (one or two 128-row
-// MMA tiles of latents), D in {16, 32} and N addressable by a TMA coordinate.
+// Latent rows the tensor-core forward computes for M latents: one 128-row
+// MMA tile (M <= 128) or two (M <= 256); rows past M are zero latents that
+// are never stored (encode) or never weighted (decode).
+inline int tc_latent_tile(int64_t M) { return M <= 128 ? 128 : 256; }
+
+// The tcgen05 forward covers bf16 with any supported M (a multiple of 16 in
+// [16, 256], padded to tc_latent_tile), D in {16, 32} and N addressable by a
+// TMA coordinate; the tcgen05 backward covers M in {128, 256}.
 inline Path choose_path(int64_t N, int64_t M, int64_t D, flare_dtype_t dt) {
   Path p;
-  p.tc_fwd = (dt == FLARE_BF16) && (M == 128 || M == 256) && (D == 16 || D == 32) &&
+  p.tc_fwd = (dt == FLARE_BF16) && (M % 16 == 0) && M >= 16 && M <= 256 && (D == 16 || D == 32) &&
              (N < (1LL << 31) - 256);
   p.tc_bwd = (dt == FLARE_BF16) && (M == 128 || M == 256) && (D == 16 || D == 32) &&
              (N < (1LL << 31) - 256);
@@ -137,7 +143,7 @@ inline ChunkPlan encode_plan(int64_t BH, int64_t N, int64_t M, int64_t D, flare_
   if (path.tc_fwd) {
     // two encode CTAs are resident per SM
     ChunkPlan p = plan_chunks(BH, N, kTcEncTile, 2LL * sms, 12.0, 32 * (int64_t)sms);
-    p.sub = (M == 128) ? 2 : 1;
+    p.sub = (tc_latent_tile(M) == 128) ? 2 : 1;   // one 128-row tile: the warpgroups split tiles
     return p;
   }
   return plan_chunks(BH, N, kSimtEncTile, 4LL * sms, 2.0, 64 * (int64_t)sms);

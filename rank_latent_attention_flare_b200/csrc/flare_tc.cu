@@ -74,6 +74,12 @@ constexpr float kRedoLimit = 18446744073709551616.0f;   // 2^kRedoTau
 #ifndef FLARE_ENC_ONEWAIT
 #define FLARE_ENC_ONEWAIT 0
 #endif
+#ifndef FLARE_DEC_LD64
+#define FLARE_DEC_LD64 0
+#endif
+#ifndef FLARE_ENC_SLEEPWAIT
+#define FLARE_ENC_SLEEPWAIT 0
+#endif
 // Decode reference of a token row (M = 256): the max of the first 32-logit
 // chunk read, used when c |k| max_m |q_m| (Cauchy-Schwarz: at least every
 // logit) lies at most this far (log2 units) above it, so no weight exceeds
@@ -173,7 +179,7 @@ template <int D, int M, bool FLAT, bool VAR, bool DZ>
 __global__ void __launch_bounds__(kThreads, 2)
     tc_encode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, int H, int64_t N, int q_per_batch,
-                     float c, int64_t tiles_per_bh, int64_t chunk_tiles, int slots_per_bh,
+                     int Mv, float c, int64_t tiles_per_bh, int64_t chunk_tiles, int slots_per_bh,
                      float* __restrict__ part_ml, float* __restrict__ part_acc,
                      const int32_t* __restrict__ lens, const float4* __restrict__ stats,
                      uint32_t* __restrict__ err) {
@@ -451,7 +457,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int lo = ht.lo(tile0 + i, kEncTile), hi = ht.hi(tile0 + i, kEncTile);
       const bool full = (lo == 0 && hi == kEncTile);   // warp-uniform: only a head's last tile is partial
       const uint32_t tS = tW + 48 * b;
+#if FLARE_ENC_SLEEPWAIT
+      if (!warp_all(mbar_wait_sleep(&s_full[2 * w + b], (uint32_t)((j >> 1) & 1)) && !*abort_flag)) {
+#else
       if (!warp_all(mbar_wait(&s_full[2 * w + b], (uint32_t)((j >> 1) & 1)) && !*abort_flag)) {
+#endif
         ok = false;
         break;
       }
@@ -486,8 +496,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int t = 0; t < 16; ++t)
               if (32 + t < lo || 32 + t >= hi) a2[t] = __float_as_uint(-INFINITY);
           }
-          exp_pack32<kEncPolyEvery>(a, c, neg, pa, sf);
-          exp_pack16<kEncPolyEvery16>(a2, c, neg, pb, sf);
+          exp_pack32<kEncPolyEvery, true>(a, c, neg, pa, sf);
+          exp_pack16<kEncPolyEvery16, true>(a2, c, neg, pb, sf);
         }
 #else
         {
@@ -502,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #if !FLARE_ENC_MAXLESS
           max_fold32(a, mf);
 #endif
-          exp_pack32<kEncPolyEvery>(a, c, neg, pa, sf);
+          exp_pack32<kEncPolyEvery, true>(a, c, neg, pa, sf);
         }
         {
           uint32_t a[16];
@@ -516,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #if !FLARE_ENC_MAXLESS
           max_fold16(a, mf);
 #endif
-          exp_pack16<kEncPolyEvery16>(a, c, neg, pb, sf);
+          exp_pack16<kEncPolyEvery16, true>(a, c, neg, pb, sf);
         }
 #endif
         const float sum = (sf[0] + sf[1]) + (sf[2] + sf[3]);
@@ -662,16 +672,21 @@ __global__ void __launch_bounds__(kThreads, 2)
       record_error(err, kErrEncSoftmaxWait);
       *abort_flag = 1;
     } else {
-      const int64_t slot = bh * slots_per_bh + (int64_t)chunk * SUB + (NH == 1 ? w : 0);
-      const int64_t row = slot * M + (NH == 2 ? w * 128 : 0) + r;
-      if (!DZ) {
-        part_ml[row * 2 + 0] = (nW > 0) ? mref : -INFINITY;
-        part_ml[row * 2 + 1] = l;
-      }
-      float4* dst = reinterpret_cast<float4*>(part_acc + row * D);
+      // latent rows past Mv are the zero rows that pad the latents to the
+      // MMA's 128-row tiles: computed alongside, never stored
+      const int lat = (NH == 2 ? w * 128 : 0) + r;
+      if (lat < Mv) {
+        const int64_t slot = bh * slots_per_bh + (int64_t)chunk * SUB + (NH == 1 ? w : 0);
+        const int64_t row = slot * Mv + lat;
+        if (!DZ) {
+          part_ml[row * 2 + 0] = (nW > 0) ? mref : -INFINITY;
+          part_ml[row * 2 + 1] = l;
+        }
+        float4* dst = reinterpret_cast<float4*>(part_acc + row * D);
 #pragma unroll
-      for (int d = 0; d < D / 4; ++d)
-        dst[d] = make_float4(acc[4 * d], acc[4 * d + 1], acc[4 * d + 2], acc[4 * d + 3]);
+        for (int d = 0; d < D / 4; ++d)
+          dst[d] = make_float4(acc[4 * d], acc[4 * d + 1], acc[4 * d + 2], acc[4 * d + 3]);
+      }
     }
   }
 
@@ -712,18 +727,23 @@ struct DecStats {
   uint32_t* flags;       // [BH]
 };
 
-template <int D, int M, bool FLAT, bool VAR, bool ST>
+// PAD = true: the latent count Mv (a multiple of 16) is below the kernel's
+// M (128 or 256); the Q and Z tiles past row Mv are the TMA's zero fill,
+// their logit columns are skipped (never exponentiated, no MMA K-step), and
+// every row takes the exact max over its Mv logits.
+template <int D, int M, bool FLAT, bool VAR, bool ST, bool PAD = false>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmZ, int H, int64_t N, int q_per_batch,
-                     float c, int64_t tiles_per_bh, int64_t chunk_tiles,
+                     int Mv, float c, int64_t tiles_per_bh, int64_t chunk_tiles,
                      __nv_bfloat16* __restrict__ Y, Tok ty, const __nv_bfloat16* __restrict__ Qg,
                      const int32_t* __restrict__ lens, const DecStats bs,
                      uint32_t* __restrict__ err) {
   using L = DecLayout<D, M>;
   constexpr int RB = L::RB;
   constexpr uint32_t SW = umma_swizzle_code(RB);
-  constexpr bool kBound = (M == 256);  // first-chunk reference under the row-max bound
+  // first-chunk reference under the row-max bound
+  constexpr bool kBound = (M == 256) && !PAD;
   constexpr int R = M;                 // TMEM columns per warpgroup
   constexpr uint32_t NCOLS = 2 * R;    // 256 or 512
   constexpr int TY = M / 2;            // Y accumulator column inside a warpgroup's region
@@ -859,6 +879,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < M / 16; ++kk) {
+          if (PAD && 16 * kk >= Mv) break;   // latents past Mv: no K-step
           const uint32_t acol = (kk < M / 32) ? 8 * kk : M / 2 + 8 * kk;
           mma_ts(tmem + w * R + TY, tmem + w * R + acol,
                  smem_desc(z_addr + kk * 16 * RB, M * RB, 8 * RB, SW), idY, kk > 0);
@@ -964,45 +985,113 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr int NC = M / 32;
       auto chunk_col = [](int k) { return k < NC / 2 ? M / 2 + 32 * (NC / 2 - 1 - k) : 32 * (k - NC / 2); };
       auto p_col = [](int k) { return k < NC / 2 ? 3 * M / 4 + 16 * (NC / 2 - 1 - k) : 16 * (k - NC / 2); };
-      uint32_t a[2][32];
-      float mf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if constexpr (kBound) {
-        tmem_ld32(tR + chunk_col(0), a[0]);
-        const float U = kn[slot * kTile + r];   // >= c S[m] for every latent (bound warps)
-        tmem_wait_ld_dep(a[0]);
-        max_fold32(a[0], mf);
-        // reference: the first chunk's max, unless the bound allows a logit
-        // more than 2^kDecRefTau above it somewhere in the warp's rows; then
-        // the exact row max (pass 1 over the other chunks)
-        if (warp_any(U - c * fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3])) > kDecRefTau)) {
-          for (int cc = 1; cc < NC; ++cc) {
-            tmem_ld32(tR + chunk_col(cc), a[1]);
-            tmem_wait_ld_dep(a[1]);
-            max_fold32(a[1], mf);
+      float sf[4] = {0.f, 0.f, 0.f, 0.f};
+      float rmx;   // the row's reference logit (its max, or the first chunk's)
+      if constexpr (PAD) {
+        // Columns [0, Mv) only, in whole or half (16-column) chunks: pass 1
+        // the exact row max, pass 2 the weights in the placement order above
+        // (a skipped chunk's columns are never read, so the P of an upper
+        // chunk may land on them).
+        float mf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int cc = 0; cc < NC; ++cc) {
+          if (32 * cc >= Mv) break;
+          if (32 * cc + 32 <= Mv) {
+            uint32_t a[32];
+            tmem_ld32(tR + 32 * cc, a);
+            tmem_wait_ld_dep(a);
+            max_fold32(a, mf);
+          } else {
+            uint32_t a[16];
+            tmem_ld16(tR + 32 * cc, a);
+            tmem_wait_ld_dep16(a);
+            max_fold16(a, mf);
+          }
+        }
+        rmx = fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3]));
+        const float neg = -rmx * c;
+#pragma unroll
+        for (int k = 0; k < NC; ++k) {
+          const int col = chunk_col(k);
+          if (col >= Mv) continue;
+          if (col + 32 <= Mv) {
+            uint32_t a[32], pk[16];
+            tmem_ld32(tR + col, a);
+            tmem_wait_ld_dep(a);
+            exp_pack32<kDecPolyEvery>(a, c, neg, pk, sf);
+            tmem_st16(tR + p_col(k), pk);
+          } else {
+            uint32_t a[16], pk[8];
+            tmem_ld16(tR + col, a);
+            tmem_wait_ld_dep16(a);
+            exp_pack16<0>(a, c, neg, pk, sf);
+            tmem_st8(tR + p_col(k), pk);
           }
         }
       } else {
-        // pass 1: the exact row max over all M logits
-        tmem_ld32(tR, a[0]);
+        uint32_t a[2][32];
+        float mf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if constexpr (kBound) {
+          tmem_ld32(tR + chunk_col(0), a[0]);
+          const float U = kn[slot * kTile + r];   // >= c S[m] for every latent (bound warps)
+          tmem_wait_ld_dep(a[0]);
+          max_fold32(a[0], mf);
+          // reference: the first chunk's max, unless the bound allows a logit
+          // more than 2^kDecRefTau above it somewhere in the warp's rows; then
+          // the exact row max (pass 1 over the other chunks)
+          if (warp_any(U - c * fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3])) > kDecRefTau)) {
+            for (int cc = 1; cc < NC; ++cc) {
+              tmem_ld32(tR + chunk_col(cc), a[1]);
+              tmem_wait_ld_dep(a[1]);
+              max_fold32(a[1], mf);
+            }
+          }
+        } else {
+          // pass 1: the exact row max over all M logits
+          tmem_ld32(tR, a[0]);
 #pragma unroll
-        for (int cc = 0; cc < NC; ++cc) {
-          tmem_wait_ld_dep(a[cc & 1]);
-          if (cc + 1 < NC) tmem_ld32(tR + 32 * (cc + 1), a[(cc + 1) & 1]);
-          max_fold32(a[cc & 1], mf);
+          for (int cc = 0; cc < NC; ++cc) {
+            tmem_wait_ld_dep(a[cc & 1]);
+            if (cc + 1 < NC) tmem_ld32(tR + 32 * (cc + 1), a[(cc + 1) & 1]);
+            max_fold32(a[cc & 1], mf);
+          }
+          tmem_ld32(tR + chunk_col(0), a[0]);
         }
-        tmem_ld32(tR + chunk_col(0), a[0]);
-      }
-      const float mx = fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3]));
-      const float neg = -mx * c;
-      float sf[4] = {0.f, 0.f, 0.f, 0.f};
-      // pass 2 (chunk 0 is in, or on its way to, a[0])
+        const float mx = fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3]));
+        const float neg = -mx * c;
+#if FLARE_DEC_LD64
+        if (!kBound) tmem_wait_ld_dep(a[0]);
+        // pass 2 in 64-column loads: chunks k and k + 1 of the placement order
+        // are adjacent (descending in the upper half, ascending in the lower)
 #pragma unroll
-      for (int k = 0; k < NC; ++k) {
-        if (k > 0 || !kBound) tmem_wait_ld_dep(a[k & 1]);
-        if (k + 1 < NC) tmem_ld32(tR + chunk_col(k + 1), a[(k + 1) & 1]);
-        uint32_t pk[16];
-        exp_pack32<kDecPolyEvery>(a[k & 1], c, neg, pk, sf);
-        tmem_st16(tR + p_col(k), pk);
+        for (int k = 0; k < NC; k += 2) {
+          const int c0 = chunk_col(k), c1 = chunk_col(k + 1);
+          const int lo = c0 < c1 ? c0 : c1;
+          uint32_t b[64], pk[32];
+          tmem_ld64(tR + lo, b);
+          tmem_wait_ld_dep64(b);
+          exp_pack_pairs<32, kDecPolyEvery>(b, c, neg, pk, sf);
+          uint32_t p0[16], p1[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            p0[t] = pk[t];
+            p1[t] = pk[16 + t];
+          }
+          tmem_st16(tR + (lo == c0 ? p_col(k) : p_col(k + 1)), p0);
+          tmem_st16(tR + (lo == c0 ? p_col(k + 1) : p_col(k)), p1);
+        }
+#else
+        // pass 2 (chunk 0 is in, or on its way to, a[0])
+#pragma unroll
+        for (int k = 0; k < NC; ++k) {
+          if (k > 0 || !kBound) tmem_wait_ld_dep(a[k & 1]);
+          if (k + 1 < NC) tmem_ld32(tR + chunk_col(k + 1), a[(k + 1) & 1]);
+          uint32_t pk[16];
+          exp_pack32<kDecPolyEvery>(a[k & 1], c, neg, pk, sf);
+          tmem_st16(tR + p_col(k), pk);
+        }
+#endif
+        rmx = mx;
       }
       tmem_wait_st();
       tc_fence_before();
@@ -1032,7 +1121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (ST) {
         const float l = (sf[0] + sf[1]) + (sf[2] + sf[3]);
         const float inv = 1.f / l;
-        const float mxp = fmaf(mx, c, log2f(l));   // the row's log-sum-exp, log2 units
+        const float mxp = fmaf(rmx, c, log2f(l));   // the row's log-sum-exp, log2 units
         const float lg = mxp - Rh;                  // log2 of g
         const bool bad = mine && lg < -kBwdRowRange;
         if (mine) {
@@ -1169,7 +1258,8 @@ cudaError_t tc_encode_t(const void* Q, int64_t qbs, const void* K, const void* V
   CUtensorMap mq, mk, mv;
   const int q_per_batch = qbs != 0;
   cudaError_t e;
-  if ((e = make_map(&mq, Q, D, M, q_per_batch ? d.BH() : d.H, 128)) != cudaSuccess) return e;
+  // Q [.., Mv, D]: rows past Mv of the 128-row boxes are the TMA's zero fill
+  if ((e = make_map(&mq, Q, D, d.M, q_per_batch ? d.BH() : d.H, 128)) != cudaSuccess) return e;
   if ((e = make_tok_map(&mk, K, d, d.k, kEncTile, FLAT)) != cudaSuccess) return e;
   if ((e = make_tok_map(&mv, V, d, DZ ? d.dy : d.v, kEncTile, FLAT)) != cudaSuccess) return e;
   // two CTAs per SM: their TMEM (2 x 256 columns) fits exactly
@@ -1179,29 +1269,31 @@ cudaError_t tc_encode_t(const void* Q, int64_t qbs, const void* K, const void* V
   if (e != cudaSuccess) return e;
   dim3 grid(plan.chunks, (unsigned)d.BH());
   tc_encode_kernel<D, M, FLAT, VAR, DZ><<<grid, kThreads, smem, st>>>(
-      mq, mk, mv, (int)d.H, d.N, q_per_batch, scale * kLog2e, plan.tiles_per_bh,
+      mq, mk, mv, (int)d.H, d.N, q_per_batch, (int)d.M, scale * kLog2e, plan.tiles_per_bh,
       plan.chunk_tiles, plan.slots_per_bh(), pml, pacc, d.lens, stats, err);
   return cudaPeekAtLastError();
 }
 
-template <int D, int M, bool FLAT, bool VAR, bool ST>
+template <int D, int M, bool FLAT, bool VAR, bool ST, bool PAD = false>
 cudaError_t tc_decode_t(const void* Q, int64_t qbs, const void* K, const __nv_bfloat16* Zb,
                         void* Y, const Dims& d, float scale, const ChunkPlan& plan,
                         const DecStats& bs, uint32_t* err, cudaStream_t st) {
   CUtensorMap mq, mk, mz;
   const int q_per_batch = qbs != 0;
   cudaError_t e;
-  if ((e = make_map(&mq, Q, D, M, q_per_batch ? d.BH() : d.H, M)) != cudaSuccess) return e;
+  // Q and Z [.., Mv, D] in boxes of M rows: rows past Mv are the TMA's zero fill
+  if ((e = make_map(&mq, Q, D, d.M, q_per_batch ? d.BH() : d.H, M)) != cudaSuccess) return e;
   if ((e = make_tok_map(&mk, K, d, d.k, kTile, FLAT)) != cudaSuccess) return e;
-  if ((e = make_map(&mz, Zb, D, M, d.BH(), M)) != cudaSuccess) return e;
+  if ((e = make_map(&mz, Zb, D, d.M, d.BH(), M)) != cudaSuccess) return e;
   const int smem = (DecLayout<D, M>::BYTES + 1024 > kMinSmemBytes) ? DecLayout<D, M>::BYTES + 1024
                                                                    : kMinSmemBytes;
-  e = cudaFuncSetAttribute(tc_decode_kernel<D, M, FLAT, VAR, ST>,
+  e = cudaFuncSetAttribute(tc_decode_kernel<D, M, FLAT, VAR, ST, PAD>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(plan.chunks, (unsigned)d.BH());
-  tc_decode_kernel<D, M, FLAT, VAR, ST><<<grid, kThreads, smem, st>>>(
-      mq, mk, mz, (int)d.H, d.N, q_per_batch, scale * kLog2e, plan.tiles_per_bh, plan.chunk_tiles,
+  tc_decode_kernel<D, M, FLAT, VAR, ST, PAD><<<grid, kThreads, smem, st>>>(
+      mq, mk, mz, (int)d.H, d.N, q_per_batch, (int)d.M, scale * kLog2e, plan.tiles_per_bh,
+      plan.chunk_tiles,
       (__nv_bfloat16*)Y, d.y, (const __nv_bfloat16*)Q, d.lens, bs, err);
   return cudaPeekAtLastError();
 }
@@ -1224,10 +1316,13 @@ cudaError_t launch_tc_encode(const void* Q, int64_t qbs, const void* K, const vo
                              const Dims& d, float scale, const ChunkPlan& plan, float* pml,
                              float* pacc, uint32_t* err, cudaStream_t st) {
 #define FLARE_ENC_ARGS Q, qbs, K, V, d, scale, plan, pml, pacc, nullptr, err, st
-  if (d.D == 32 && d.M == 256) return tc_encode_dispatch<32, 256, false>(FLARE_ENC_ARGS);
-  if (d.D == 32 && d.M == 128) return tc_encode_dispatch<32, 128, false>(FLARE_ENC_ARGS);
-  if (d.D == 16 && d.M == 256) return tc_encode_dispatch<16, 256, false>(FLARE_ENC_ARGS);
-  if (d.D == 16 && d.M == 128) return tc_encode_dispatch<16, 128, false>(FLARE_ENC_ARGS);
+  // latent counts below 128 (or between 128 and 256) run on the 128-row
+  // (256-row) kernel with zero latents past d.M that are never stored
+  const int Mp = tc_latent_tile(d.M);
+  if (d.D == 32 && Mp == 256) return tc_encode_dispatch<32, 256, false>(FLARE_ENC_ARGS);
+  if (d.D == 32 && Mp == 128) return tc_encode_dispatch<32, 128, false>(FLARE_ENC_ARGS);
+  if (d.D == 16 && Mp == 256) return tc_encode_dispatch<16, 256, false>(FLARE_ENC_ARGS);
+  if (d.D == 16 && Mp == 128) return tc_encode_dispatch<16, 128, false>(FLARE_ENC_ARGS);
 #undef FLARE_ENC_ARGS
   return cudaErrorNotSupported;
 }
@@ -1252,6 +1347,12 @@ cudaError_t tc_decode_dispatch(const void* Q, int64_t qbs, const void* K,
   // The decode takes 4-D maps for every layout: its 3-D variant measured no
   // faster and needs more registers.
   const DecStats none{};
+  if (d.M != M)   // latents padded to the kernel's M
+    return d.lens != nullptr
+               ? tc_decode_t<D, M, false, true, false, true>(Q, qbs, K, Zb, Y, d, scale, plan, none,
+                                                             err, st)
+               : tc_decode_t<D, M, false, false, false, true>(Q, qbs, K, Zb, Y, d, scale, plan,
+                                                              none, err, st);
   return d.lens != nullptr
              ? tc_decode_t<D, M, false, true, false>(Q, qbs, K, Zb, Y, d, scale, plan, none, err, st)
              : tc_decode_t<D, M, false, false, false>(Q, qbs, K, Zb, Y, d, scale, plan, none, err, st);
@@ -1260,10 +1361,11 @@ cudaError_t tc_decode_dispatch(const void* Q, int64_t qbs, const void* K,
 cudaError_t launch_tc_decode(const void* Q, int64_t qbs, const void* K, const __nv_bfloat16* Zb,
                              void* Y, const Dims& d, float scale, const ChunkPlan& plan,
                              uint32_t* err, cudaStream_t st) {
-  if (d.D == 32 && d.M == 256) return tc_decode_dispatch<32, 256>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
-  if (d.D == 32 && d.M == 128) return tc_decode_dispatch<32, 128>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
-  if (d.D == 16 && d.M == 256) return tc_decode_dispatch<16, 256>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
-  if (d.D == 16 && d.M == 128) return tc_decode_dispatch<16, 128>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
+  const int Mp = tc_latent_tile(d.M);
+  if (d.D == 32 && Mp == 256) return tc_decode_dispatch<32, 256>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
+  if (d.D == 32 && Mp == 128) return tc_decode_dispatch<32, 128>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
+  if (d.D == 16 && Mp == 256) return tc_decode_dispatch<16, 256>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
+  if (d.D == 16 && Mp == 128) return tc_decode_dispatch<16, 128>(Q, qbs, K, Zb, Y, d, scale, plan, err, st);
   return cudaErrorNotSupported;
 }
 

@@ -445,7 +445,7 @@ __device__ __forceinline__ void max_fold16(const uint32_t (&a)[16], float (&m)[4
 // p = 2^(a*c + neg) for 32 logits: packed into 16 bf16 pairs, sums folded
 // into four independent accumulators.  With POLY_EVERY = k > 0, every k-th
 // pair is computed on the FMA pipe (exp2_fma) instead of the MUFU.
-template <int POLY_EVERY = 0>
+template <int POLY_EVERY = 0, bool CLAMP_HI = false>
 __device__ __forceinline__ void exp_pack32(const uint32_t (&a)[32], float c, float neg,
                                            uint32_t (&pk)[16], float (&s)[4]);
 
@@ -545,7 +545,11 @@ __device__ __forceinline__ void exp2_fma_pair_logits(float a0, float a1, float c
 
 // 2^(a*c + neg) for NP consecutive pairs of logits: bf16 pairs into pk, the
 // values summed into s (s[0], s[2] collect even lanes, s[1], s[3] odd ones).
-template <int NP, int POLY_EVERY>
+// CLAMP_HI: the polynomial pairs clamp their exponent to [-125, 126]
+// (exp2_fma_pair_logits), for callers whose exponents can be large and
+// positive; otherwise they use exp2_fma_pair (exponents known to be at most
+// 126).
+template <int NP, int POLY_EVERY, bool CLAMP_HI = false>
 __device__ __forceinline__ void exp_pack_pairs(const uint32_t* a, float c, float neg,
                                                uint32_t* pk, float (&s)[4]) {
   const uint64_t c2 = f32x2(c, c), n2 = f32x2(neg, neg);
@@ -555,9 +559,13 @@ __device__ __forceinline__ void exp_pack_pairs(const uint32_t* a, float c, float
   for (int t = 0; t < NP; ++t) {
     const bool poly = POLY_EVERY > 0 && (t % (POLY_EVERY > 0 ? POLY_EVERY : 1)) == POLY_EVERY - 1;
     float p0, p1;
-    if (poly) {
+    if (poly && CLAMP_HI) {
       exp2_fma_pair_logits(__uint_as_float(a[2 * t]), __uint_as_float(a[2 * t + 1]), cs, ns, p0,
                            p1);
+    } else if (poly) {
+      exp2_fma_pair(
+          fma_f32x2(f32x2(__uint_as_float(a[2 * t]), __uint_as_float(a[2 * t + 1])), c2, n2), p0,
+          p1);
     } else {
       const uint64_t x =
           fma_f32x2(f32x2(__uint_as_float(a[2 * t]), __uint_as_float(a[2 * t + 1])), c2, n2);
@@ -573,17 +581,17 @@ __device__ __forceinline__ void exp_pack_pairs(const uint32_t* a, float c, float
   split_f32x2(acc[1], s[2], s[3]);
 }
 
-template <int POLY_EVERY>
+template <int POLY_EVERY, bool CLAMP_HI>
 __device__ __forceinline__ void exp_pack32(const uint32_t (&a)[32], float c, float neg,
                                            uint32_t (&pk)[16], float (&s)[4]) {
-  exp_pack_pairs<16, POLY_EVERY>(a, c, neg, pk, s);
+  exp_pack_pairs<16, POLY_EVERY, CLAMP_HI>(a, c, neg, pk, s);
 }
 
 // p = 2^(a*c + neg) for 16 logits: 8 bf16 pairs, sums into four accumulators.
-template <int POLY_EVERY = 0>
+template <int POLY_EVERY = 0, bool CLAMP_HI = false>
 __device__ __forceinline__ void exp_pack16(const uint32_t (&a)[16], float c, float neg,
                                            uint32_t (&pk)[8], float (&s)[4]) {
-  exp_pack_pairs<8, POLY_EVERY>(a, c, neg, pk, s);
+  exp_pack_pairs<8, POLY_EVERY, CLAMP_HI>(a, c, neg, pk, s);
 }
 
 }  // namespace tc

@@ -97,7 +97,10 @@ def test_fwd_path_selection(lib):
     assert lib.flare_fwd_path(1, 4, 1024, 32, 16, 0) == 0        # fp32 -> CUDA cores
     assert lib.flare_fwd_path(1, 16, 1 << 20, 256, 32, 1) == 1     # bf16 headline -> tcgen05
     assert lib.flare_fwd_path(4, 8, 1 << 16, 128, 16, 1) == 1
-    assert lib.flare_fwd_path(1, 4, 1000, 64, 32, 1) == 0         # bf16, M=64 -> CUDA cores
+    assert lib.flare_fwd_path(1, 4, 1000, 64, 32, 1) == 1         # bf16, M=64 -> tcgen05 (padded)
+    assert lib.flare_fwd_path(1, 4, 1000, 16, 16, 1) == 1
+    assert lib.flare_fwd_path(1, 4, 1000, 192, 32, 1) == 1
+    assert lib.flare_fwd_path(1, 4, 1000, 64, 32, 0) == 0         # fp32, M=64 -> CUDA cores
     assert lib.flare_fwd_path(1, 4, 1024, 40, 16, 1) == -1
     assert lib.flare_bwd_path(8, 8, 16384, 128, 32, 1) == 1      # bf16, M=128 -> tcgen05
     assert lib.flare_bwd_path(1, 2, 300, 128, 16, 1) == 1

@@ -188,3 +188,44 @@ def test_decode_row_reference_mixed_within_warps():
         assert_close(Y[:, :, sel], Yo[:, :, sel], torch.bfloat16, what)
     assert_close(Y, Yo, torch.bfloat16, "Y")
     assert_close(Z, Zo, torch.bfloat16, "Z")
+
+
+@pytest.mark.parametrize("M", [16, 48, 64, 80, 112, 144, 192, 240])
+@pytest.mark.parametrize("D", [16, 32])
+def test_fwd_tensor_core_padded_latents(M, D):
+    # Latent counts other than 128 and 256 run on the tensor-core kernels
+    # with the latent tile padded by zero rows: never stored by the encode,
+    # never weighted by the decode.
+    B, H, N = 2, 2, 1000
+    s = 1.0 / math.sqrt(D)
+    assert fl.fwd_path(B, H, N, M, D, torch.bfloat16) == 1
+    x = make_inputs(B, H, N, M, D, dtype=torch.bfloat16, seed=100 + M + D)
+    g = {k: v.to(DEV) for k, v in x.items()}
+    ws = fl.alloc_workspace(fl.FLARE_OP_FWD, B, H, N, M, D, torch.bfloat16, DEV)
+    ws.fill_(0xFF)
+    Y, Z, lse = fl.flare_fwd(g["Q"], g["K"], g["V"], s, save=True, workspace=ws)
+    assert fl.device_status(ws) == 0
+    Yo, Zo, lo = oracle.flare_fwd(x["Q"], x["K"], x["V"], s)
+    assert_close(Z, Zo, torch.bfloat16, f"Z M={M}")
+    assert_close(lse, lo, torch.bfloat16, f"lse M={M}")
+    assert_close(Y, Yo, torch.bfloat16, f"Y M={M}")
+
+
+@pytest.mark.parametrize("M", [64, 192])
+def test_padded_latents_per_batch_flare_pp_and_backward(M):
+    # per-batch latents (FLARE++'s Q_dyn path) and the backward (CUDA cores
+    # for these M) from the tensor-core forward's saved Z and lse
+    B, H, N, D = 2, 2, 777, 32
+    s = 1.0 / math.sqrt(D)
+    x = make_inputs(B, H, N, M, D, dtype=torch.bfloat16, seed=200 + M, with_dy=True)
+    g = {k: v.to(DEV) for k, v in x.items()}
+    Y, Qd = fl.flare_pp_fwd(g["Q"], g["K"], g["V"], s)
+    Yo, Qdo, _, _ = oracle.flare_pp_fwd(x["Q"], x["K"], x["V"], s)
+    assert_close(Qd, Qdo, torch.bfloat16, "Q_dyn")
+    assert_close(Y, Yo, torch.bfloat16, "Y (FLARE++)")
+    Y, Z, lse = fl.flare_fwd(g["Q"], g["K"], g["V"], s, save=True)
+    dQ, dK, dV = fl.flare_bwd(g["Q"], g["K"], g["V"], g["dY"], Z, lse, s)
+    dQo, dKo, dVo = oracle.flare_bwd(x["Q"], x["K"], x["V"], x["dY"], s)
+    assert_close(dV, dVo, torch.bfloat16, "dV")
+    assert_close(dK, dKo, torch.bfloat16, "dK")
+    assert_close(dQ, dQo, torch.bfloat16, "dQ")
