@@ -25,8 +25,8 @@
 //     TMA loads; warps 9 and 10 issue the MMAs of softmax warpgroup 0 and 1
 //     (one elected lane each; warp 9 also owns TMEM); warp 11 only lends its
 //     registers.  Launched at 80 registers per thread, the producer
-//     warpgroup moves to 40 and the softmax warpgroups to 96
-//     (2 x 128 x 96 + 128 x 40 <= 384 x 80).
+//     warpgroup moves to 56 and the softmax warpgroups to 88
+//     (2 x 128 x 88 + 128 x 56 <= 384 x 80).
 //   decode -- the same softmax warpgroups (alternate tiles), warp 8 TMA,
 //     warp 9 TMEM and MMAs, warps 10-11 bound each K tile's row maxima
 //     (M = 256).  Launched at 168 registers per thread: the producer
@@ -42,6 +42,15 @@ namespace flare {
 namespace {
 
 using namespace tc;
+
+#ifndef FLARE_MMA_SPIN
+#define FLARE_MMA_SPIN 0
+#endif
+#if FLARE_MMA_SPIN
+#define MMA_WAIT mbar_wait
+#else
+#define MMA_WAIT mbar_wait_sleep
+#endif
 
 constexpr int kTile = 128;        // tokens per tile (MMA M or N)
 constexpr int kThreads = 384;
@@ -68,9 +77,6 @@ constexpr float kRedoLimit = 18446744073709551616.0f;   // 2^kRedoTau
 // (two per sub-partition, close to its register budget) gains only from the
 // last pair of each 32-column chunk (1.40 -> 1.38 ms; every 4th, 8th, 10th
 // or 12th pair is slower).
-#ifndef FLARE_ENC_SLEEPWAIT
-#define FLARE_ENC_SLEEPWAIT 0
-#endif
 // Decode reference of a token row (M = 256): the max of the first 32-logit
 // chunk read, used when c |k| max_m |q_m| (Cauchy-Schwarz: at least every
 // logit) lies at most this far (log2 units) above it, so no weight exceeds
@@ -113,52 +119,29 @@ __device__ __forceinline__ void scale_tmem_row(uint32_t taddr, float f) {
 // Tiles of kEncTile = 48 tokens; two CTAs share an SM (256 TMEM columns and
 // an 80-register launch each), so four softmax warpgroups per SM hide each
 // other's latencies.  Softmax warpgroup w owns TMEM columns
-// [128w, 128w + 128): two 48-column S buffers at 128w + 48b (b = 0, 1) and
-// the O accumulator at 128w + 96.  The softmax reads a tile's S, releases
-// the buffer (the MMA then computes the logits of the warpgroup's tile after
-// next into it) and writes the tile's P to one of its two shared-memory P
-// buffers, from which P.V reads it; so a buffer's next S never waits for
-// the P.V of the tile before.  (The backward's dZ form instead writes P over
-// the S columns, and refills the buffer after that P.V.)  With M = 256
+// [128w, 128w + 128): two 48-column S buffers at 128w + 48b (b = 0, 1), whose
+// first 24 columns receive the tile's P (bf16 pairs) once S has been read,
+// and the O accumulator at 128w + 96.  While the softmax works on one
+// buffer, the MMA fills the other with the next tile's logits.  With M = 256
 // warpgroup w owns latent rows [128w, 128w + 128) of every tile; with M = 128
 // the warpgroups take alternate tiles, each with its own running record.
 
 constexpr int kEncTile = 48;
-// 256 x 96 + 128 x 40 <= 384 x 80 (the launch); the TMA and MMA warps need few
-constexpr int kEncRegsSoftmax = 96, kEncRegsProducer = 40;
-
-// The softmax form keeps each tile's P in shared memory (four buffers: two
-// per warpgroup), so that an S buffer in TMEM can take the next tile's
-// logits as soon as they have been read, without waiting for the P.V that
-// reads P; the dZ form writes P over the S columns in TMEM.  P buffer layout:
-// the K-major A operand of P.V with the 32-byte swizzle, 128 latent rows x
-// 48 tokens as three 16-token atom columns of 4 KB, rows 32 bytes apart in
-// an atom column, the two 16-byte halves of a row swapped on rows 4-7 of
-// every 8.
-constexpr int kEncPAtomCol = 128 * 32;   // one 16-token atom column of a P buffer
+constexpr int kEncRegsSoftmax = 88, kEncRegsProducer = 56;   // 256 x 88 + 128 x 56 <= 384 x 80
 
 template <int D, int M, bool DZ = false>
 struct EncLayout {
-  static constexpr int STAGES = DZ ? 8 : 6;         // K/V ring
   static constexpr int RB = 2 * D;                  // bytes per row (one token or latent)
   static constexpr int TILE = kEncTile * RB;        // one K or V tile
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = M * RB;
-  static constexpr int PBUF = (kEncTile / 16) * kEncPAtomCol;
-  static constexpr int P_OFF = ((KV_OFF + STAGES * 2 * TILE + 1023) / 1024) * 1024;
-  static constexpr int BAR_OFF = DZ ? KV_OFF + STAGES * 2 * TILE : P_OFF + 4 * PBUF;
-  static constexpr int NBARS = 2 * STAGES + 1 + 4 + 4 + 4 + 2 + 4;
+  static constexpr int BAR_OFF = KV_OFF + kEncStages * 2 * TILE;
+  static constexpr int NBARS = 2 * kEncStages + 1 + 4 + 4 + 4 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   // dZ form: per stage, the tile's column offsets (kEncTile floats)
   static constexpr int NB_OFF = MISC_OFF + 16;
-  static constexpr int BYTES = DZ ? NB_OFF + STAGES * kEncTile * 4 : MISC_OFF + 16;
+  static constexpr int BYTES = DZ ? NB_OFF + kEncStages * kEncTile * 4 : MISC_OFF + 16;
 };
-
-// Byte offset of the 16-byte group of tokens [8 g, 8 g + 8) of latent row r
-// in a P buffer.
-__device__ __forceinline__ uint32_t enc_p_off(int r, int g) {
-  return (uint32_t)((g >> 1) * kEncPAtomCol + r * 32 + (((g & 1) ^ ((r >> 2) & 1)) << 4));
-}
 
 // p = 2^(c a + nb) for NP consecutive pairs of logits, nb per column (a
 // float pair from shared memory): bf16 pairs into pk.  With POLY_EVERY = k
@@ -210,13 +193,12 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint8_t* Qs = smem + L::Q_OFF;
   uint64_t* bars = (uint64_t*)(smem + L::BAR_OFF);
   uint64_t* kv_full = bars;
-  uint64_t* kv_empty = bars + L::STAGES;
-  uint64_t* q_full = bars + 2 * L::STAGES;
+  uint64_t* kv_empty = bars + kEncStages;
+  uint64_t* q_full = bars + 2 * kEncStages;
   uint64_t* s_full = q_full + 1;      // [2w + b]: S written by the MMA
-  uint64_t* sp_done = s_full + 4;     // [2w + b]: the tile's P written (shared memory / TMEM)
+  uint64_t* sp_done = s_full + 4;     // [2w + b]: S read and P written by the softmax
   uint64_t* pv_done = sp_done + 4;    // [2w + b]: P.V of a tile from buffer b complete
   uint64_t* drain = pv_done + 4;      // [w]
-  uint64_t* s_read = drain + 2;       // [2w + b]: S read from buffer b (softmax form)
   uint32_t* tmem_slot = (uint32_t*)(smem + L::MISC_OFF);
   volatile int* abort_flag = (volatile int*)(smem + L::MISC_OFF + 4);
 
@@ -231,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                              : imin64(chunk_tiles, tiles_per_bh - tile0);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < L::STAGES; ++s) {
+    for (int s = 0; s < kEncStages; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], NH == 2 ? 2 : 1);   // one release per warpgroup reading the tile
     }
@@ -240,7 +222,6 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&s_full[k], 1);
       mbar_init(&sp_done[k], 128);
       mbar_init(&pv_done[k], 1);
-      mbar_init(&s_read[k], 128);
     }
     for (int k = 0; k < 2; ++k) mbar_init(&drain[k], 1);
     *abort_flag = 0;
@@ -271,11 +252,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       int issued = 0;
       for (int i = 0; i < (int)ntiles; ++i) {
-        const int s = i % L::STAGES;
-        const uint32_t ph = (uint32_t)((i / L::STAGES) & 1);
+        const int s = i % kEncStages;
+        const uint32_t ph = (uint32_t)((i / kEncStages) & 1);
         int stop = 0;
         if (lane == 0) {
-          if (i >= L::STAGES && !mbar_wait_sleep(&kv_empty[s], ph ^ 1)) {
+          if (i >= kEncStages && !mbar_wait_sleep(&kv_empty[s], ph ^ 1)) {
             record_error(err, kErrEncTmaWait);
             *abort_flag = 1;
           }
@@ -297,8 +278,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         issued = i + 1;
       }
       if (lane == 0) {
-        for (int i = (issued > L::STAGES ? issued - L::STAGES : 0); i < issued; ++i)
-          mbar_wait_sleep(&kv_full[i % L::STAGES], (uint32_t)((i / L::STAGES) & 1));
+        for (int i = (issued > kEncStages ? issued - kEncStages : 0); i < issued; ++i)
+          mbar_wait_sleep(&kv_full[i % kEncStages], (uint32_t)((i / kEncStages) & 1));
         mbar_wait_sleep(q_full, 0);
       }
     } else if (warp == kWarpTma) {
@@ -313,9 +294,9 @@ __global__ void __launch_bounds__(kThreads, 2)
           tma_load_3d(Qs + half * 128 * RB, &tmQ, q_full, 0, half * 128, qz);
         int issued = 0;
         for (int i = 0; i < (int)ntiles; ++i) {
-          const int s = i % L::STAGES;
-          const uint32_t ph = (uint32_t)((i / L::STAGES) & 1);
-          if (i >= L::STAGES && !mbar_wait_sleep(&kv_empty[s], ph ^ 1)) {
+          const int s = i % kEncStages;
+          const uint32_t ph = (uint32_t)((i / kEncStages) & 1);
+          if (i >= kEncStages && !mbar_wait_sleep(&kv_empty[s], ph ^ 1)) {
             record_error(err, kErrEncTmaWait);
             *abort_flag = 1;
             break;
@@ -329,8 +310,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           issued = i + 1;
         }
         // let every load still in flight land before the CTA can exit
-        for (int i = (issued > L::STAGES ? issued - L::STAGES : 0); i < issued; ++i)
-          mbar_wait_sleep(&kv_full[i % L::STAGES], (uint32_t)((i / L::STAGES) & 1));
+        for (int i = (issued > kEncStages ? issued - kEncStages : 0); i < issued; ++i)
+          mbar_wait_sleep(&kv_full[i % kEncStages], (uint32_t)((i / kEncStages) & 1));
         mbar_wait_sleep(q_full, 0);
       }
     } else if (warp == kWarpMma || warp == kWarpMma + 1) {
@@ -354,8 +335,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         bool ok = mbar_wait_sleep(q_full, 0);
         auto issue_S = [&](int j) -> bool {
           const int i = first + stride * j;
-          const int s = i % L::STAGES;
-          if (!mbar_wait_sleep(&kv_full[s], (uint32_t)((i / L::STAGES) & 1))) return false;
+          const int s = i % kEncStages;
+          if (!mbar_wait_sleep(&kv_full[s], (uint32_t)((i / kEncStages) & 1))) return false;
           tc_fence_after();
           const uint32_t koff = (uint32_t)(s * 2 * L::TILE) >> 4;
           const int b = j & 1;
@@ -366,55 +347,24 @@ __global__ void __launch_bounds__(kThreads, 2)
           return true;
         };
         for (int j = 0; ok && j < 2 && j < nw; ++j) ok = issue_S(j);
-        // P buffers in shared memory (softmax form), K-major with the 32-byte swizzle
-        const uint64_t dP = smem_desc(smem_u32(smem + L::P_OFF), 16, 8 * 32, 6u);
-        for (int j = 0; ok && !DZ && j < nw; ++j) {
+        for (int j = 0; ok && j < nw; ++j) {
           const int b = j & 1;
-          const int i = first + stride * j;
-          // the S of tile j + 2 into buffer b as soon as the softmax has read
-          // tile j's logits from it
-          if (j + 2 < nw) {
-            if (!mbar_wait_sleep(&s_read[2 * w + b], (uint32_t)((j >> 1) & 1))) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            if (!(ok = issue_S(j + 2))) break;
-          }
-          // P.V of tile j once its P is in shared memory
-          if (!mbar_wait_sleep(&sp_done[2 * w + b], (uint32_t)((j >> 1) & 1))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t voff = (uint32_t)((i % L::STAGES) * 2 * L::TILE) >> 4;
-          const uint32_t poff = (uint32_t)((2 * w + b) * L::PBUF) >> 4;
-#pragma unroll
-          for (int kk = 0; kk < kEncTile / 16; ++kk)
-            mma_ss(tW + 96, dP + poff + (uint32_t)(kk * (kEncPAtomCol >> 4)),
-                   dV + voff + ((uint32_t)(kk * 16 * RB) >> 4), idPV, (j > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&pv_done[2 * w + b]);
-          mma_commit(&kv_empty[i % L::STAGES]);
-          if (*abort_flag) ok = false;
-        }
-        for (int j = 0; ok && DZ && j < nw; ++j) {
-          const int b = j & 1;
-          if (!mbar_wait_sleep(&sp_done[2 * w + b], (uint32_t)((j >> 1) & 1))) {
+          if (!MMA_WAIT(&sp_done[2 * w + b], (uint32_t)((j >> 1) & 1))) {
             ok = false;
             break;
           }
           tc_fence_after();
           const int i = first + stride * j;
-          const uint32_t voff = (uint32_t)((i % L::STAGES) * 2 * L::TILE) >> 4;
+          const uint32_t voff = (uint32_t)((i % kEncStages) * 2 * L::TILE) >> 4;
 #pragma unroll
           for (int kk = 0; kk < kEncTile / 16; ++kk)
             mma_ts(tW + 96, tW + 48 * b + 8 * kk, dV + voff + ((uint32_t)(kk * 16 * RB) >> 4),
                    idPV, (j > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&pv_done[2 * w + b]);
-          mma_commit(&kv_empty[i % L::STAGES]);
+          mma_commit(&kv_empty[i % kEncStages]);
           if (j + 2 < nw) {
             // buffer b still holds the P this P.V reads: wait for it to finish
-            if (!mbar_wait_sleep(&pv_done[2 * w + b], (uint32_t)((j >> 1) & 1))) {
+            if (!MMA_WAIT(&pv_done[2 * w + b], (uint32_t)((j >> 1) & 1))) {
               ok = false;
               break;
             }
@@ -467,11 +417,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int j = 0; j < nW; ++j) {
         const int64_t i = first + (int64_t)stride * j;
         const int b = j & 1;
-        const int s = (int)(i % L::STAGES);
+        const int s = (int)(i % kEncStages);
         const uint32_t tS = tW + 48 * b;
         // the tile's S in TMEM, and its stage (with the column offsets) landed
         if (!warp_all(mbar_wait(&s_full[2 * w + b], (uint32_t)((j >> 1) & 1)) &&
-                      mbar_wait(&kv_full[s], (uint32_t)((i / L::STAGES) & 1)) && !*abort_flag)) {
+                      mbar_wait(&kv_full[s], (uint32_t)((i / kEncStages) & 1)) && !*abort_flag)) {
           ok = false;
           break;
         }
@@ -497,11 +447,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_arrive(&sp_done[2 * w + b]);
       }
     }
-    // Softmax form, per tile j of this warpgroup (buffer b = j % 2): read
-    // the tile's logits S from TMEM, compute P in registers, release the S
-    // buffer (s_read: the MMA warp then computes tile j + 2's S into it),
-    // and once tile j - 2's P.V has finished with the P buffer, write P to
-    // shared memory for this tile's P.V (sp_done).
     for (int j = 0; !DZ && j < nW; ++j) {
       const int64_t i = first + (int64_t)stride * j;
       const int b = j & 1;
@@ -509,29 +454,20 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int lo = ht.lo(tile0 + i, kEncTile), hi = ht.hi(tile0 + i, kEncTile);
       const bool full = (lo == 0 && hi == kEncTile);   // warp-uniform: only a head's last tile is partial
       const uint32_t tS = tW + 48 * b;
-#if FLARE_ENC_SLEEPWAIT
-      if (!warp_all(mbar_wait_sleep(&s_full[2 * w + b], (uint32_t)((j >> 1) & 1)) && !*abort_flag)) {
-#else
       if (!warp_all(mbar_wait(&s_full[2 * w + b], (uint32_t)((j >> 1) & 1)) && !*abort_flag)) {
-#endif
         ok = false;
         break;
       }
       __syncwarp();
       tc_fence_after();
-      uint32_t pa[16], pb[8];   // the tile's P as bf16 pairs (columns 0-31, 32-47)
-      float g = 1.f;            // factor O owes before this tile's P.V
       // Optimistic single pass (every tile after a warpgroup's first): P is
-      // taken against the running reference m_ref.  Every weight is at most
-      // the tile's row sum, so the sum stands in for the max: above
-      // 2^kRedoTau (or not finite) a weight may have overflowed and the
-      // whole warp recomputes the tile with the exact max; above
-      // 2^kRescaleTau the reference moves up by log2(sum) after the tile
-      // (l at once, O before the next P.V).
+      // taken against the running reference m_ref and stays in registers
+      // until the overflow check below passes.
       bool exact = warp_any(mref == -INFINITY);
       if (!exact) {
         const float neg = -mref;
         float sf[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t pa[16], pb[8];
         {
           uint32_t a[32];
           tmem_ld32(tS, a);
@@ -555,11 +491,21 @@ __global__ void __launch_bounds__(kThreads, 2)
           exp_pack16<kEncPolyEvery16, true>(a, c, neg, pb, sf);
         }
         const float sum = (sf[0] + sf[1]) + (sf[2] + sf[3]);
+        // Every weight of the tile is at most the tile's row sum, so the sum
+        // stands in for the max: above 2^kRedoTau (or not finite) a weight
+        // may have overflowed and the tile is recomputed with the exact max;
+        // above 2^kRescaleTau the reference moves up by log2(sum), which
+        // keeps it within log2(tile) of the running max.
         if (warp_any(!(sum <= kRedoLimit))) {
           exact = true;
         } else {
-          g = pend;   // a rescale decided after the previous tile
+          if (!scale_O(j, pend)) {   // a rescale decided after the previous tile
+            ok = false;
+            break;
+          }
           pend = 1.f;
+          tmem_st16(tS, pa);          // P over S columns already read
+          tmem_st8(tS + 16, pb);
           if (sum > kRescaleLimit) {
             const float mx2 = mref + lg2(sum);
             pend = ex2(mref - mx2);
@@ -596,9 +542,14 @@ __global__ void __launch_bounds__(kThreads, 2)
           mref = mx2;
         }
         l *= f;
-        g = pend * f;
+        if (!scale_O(j, pend * f)) {
+          ok = false;
+          break;
+        }
         pend = 1.f;
-        // pass 2: P = 2^(c S - m_ref) as bf16 pairs, and its row sum
+        // pass 2: P = 2^(c S - m_ref) as bf16 pairs, and its row sum; chunk
+        // 0's P lands on S columns [0, 16) and chunk 1's on [16, 24), both
+        // already read.
         const float neg = -mref;
         float sf[4] = {0.f, 0.f, 0.f, 0.f};
         {
@@ -610,7 +561,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int t = 0; t < 32; ++t)
               if (t < lo || t >= hi) a[t] = __float_as_uint(-INFINITY);
           }
-          exp_pack32<kEncPolyEvery, true>(a, c, neg, pa, sf);
+          uint32_t pk[16];
+          exp_pack32<kEncPolyEvery, true>(a, c, neg, pk, sf);
+          tmem_st16(tS, pk);
         }
         {
           uint32_t a[16];
@@ -621,34 +574,13 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int t = 0; t < 16; ++t)
               if (32 + t < lo || 32 + t >= hi) a[t] = __float_as_uint(-INFINITY);
           }
-          exp_pack16<kEncPolyEvery16, true>(a, c, neg, pb, sf);
+          uint32_t pk[8];
+          exp_pack16<kEncPolyEvery16, true>(a, c, neg, pk, sf);
+          tmem_st8(tS + 16, pk);
         }
         l += (sf[0] + sf[1]) + (sf[2] + sf[3]);
       }
-      // every load of the tile's S has completed: the buffer is free
-      tc_fence_before();
-      mbar_arrive(&s_read[2 * w + b]);
-      // the P buffer was last read by tile j - 2's P.V
-      if (j >= 2 && !warp_all(pv_wait(j - 2))) {
-        ok = false;
-        break;
-      }
-      uint8_t* pbuf = smem + L::P_OFF + (2 * w + b) * L::PBUF;
-#pragma unroll
-      for (int gq = 0; gq < 4; ++gq)
-        *reinterpret_cast<uint4*>(pbuf + enc_p_off(r, gq)) =
-            make_uint4(pa[4 * gq], pa[4 * gq + 1], pa[4 * gq + 2], pa[4 * gq + 3]);
-#pragma unroll
-      for (int gq = 0; gq < 2; ++gq)
-        *reinterpret_cast<uint4*>(pbuf + enc_p_off(r, 4 + gq)) =
-            make_uint4(pb[4 * gq], pb[4 * gq + 1], pb[4 * gq + 2], pb[4 * gq + 3]);
-      fence_proxy_async_smem();
-      // a rescale of O waits for tile j - 1's P.V (O stable)
-      if (!scale_O(j, g)) {
-        ok = false;
-        break;
-      }
-      tmem_wait_st();   // a rescale's stores to O
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sp_done[2 * w + b]);
     }
@@ -873,7 +805,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t j = i >> 1;
         const int s = (int)(i % kDecStages);
         if (!mbar_wait_sleep(&k_full[s], (uint32_t)((i / kDecStages) & 1))) return false;
-        if (j > 0 && !mbar_wait_sleep(&s_empty[w], (uint32_t)((j - 1) & 1))) return false;
+        if (j > 0 && !MMA_WAIT(&s_empty[w], (uint32_t)((j - 1) & 1))) return false;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(smem + L::K_OFF + s * L::TILE);
 #pragma unroll
@@ -904,19 +836,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int w = (int)(i & 1);
         const uint32_t ph = (uint32_t)((i >> 1) & 1);
         if constexpr (PAD) {
-          if (!mbar_wait_sleep(&p_full[w], ph)) return false;
+          if (!MMA_WAIT(&p_full[w], ph)) return false;
           tc_fence_after();
           y_steps(w, 0, M / 16, 0);
         } else {
-          if (!mbar_wait_sleep(&p_part[2 * w], ph)) return false;
+          if (!MMA_WAIT(&p_part[2 * w], ph)) return false;
           tc_fence_after();
           y_steps(w, M / 32, M / 16, M / 32);
           if (M == 256) {
-            if (!mbar_wait_sleep(&p_part[2 * w + 1], ph)) return false;
+            if (!MMA_WAIT(&p_part[2 * w + 1], ph)) return false;
             tc_fence_after();
             y_steps(w, 0, 4, -1);
           }
-          if (!mbar_wait_sleep(&p_full[w], ph)) return false;
+          if (!MMA_WAIT(&p_full[w], ph)) return false;
           tc_fence_after();
           y_steps(w, M == 256 ? 4 : 0, M / 32, -1);
         }
