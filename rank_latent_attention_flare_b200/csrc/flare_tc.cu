@@ -43,14 +43,10 @@ namespace {
 
 using namespace tc;
 
-#ifndef FLARE_MMA_SPIN
-#define FLARE_MMA_SPIN 1
-#endif
-#if FLARE_MMA_SPIN
+// The MMA-issuing threads poll their barriers instead of sleeping between
+// polls: the decode's tile chain (Y, then the next S) runs through them
+// twice per tile, and a suspended poll added about 8% to its time.
 #define MMA_WAIT mbar_wait
-#else
-#define MMA_WAIT mbar_wait_sleep
-#endif
 
 constexpr int kTile = 128;        // tokens per tile (MMA M or N)
 constexpr int kThreads = 384;
@@ -119,22 +115,15 @@ __device__ __forceinline__ void scale_tmem_row(uint32_t taddr, float f) {
 // Tiles of kEncTile = 48 tokens; two CTAs share an SM (256 TMEM columns and
 // an 80-register launch each), so four softmax warpgroups per SM hide each
 // other's latencies.  Softmax warpgroup w owns TMEM columns
-// [128w, 128w + 128): one 48-column S buffer, two 24-column P buffers (a
-// tile's 48 weights as bf16 pairs) and the O accumulator.  The softmax
-// threads load a tile's logits into registers at the start of the tile and
-// release the S buffer at once, so the MMA computes the next tile's logits
-// while this tile's exponentials run; P goes to P buffer j % 2, which the
-// P.V of tile j - 2 has finished reading.  With M = 256 warpgroup w owns
-// latent rows [128w, 128w + 128) of every tile; with M = 128 the warpgroups
-// take alternate tiles, each with its own running record.
+// [128w, 128w + 128): two 48-column S buffers at 128w + 48b (b = 0, 1), whose
+// first 24 columns receive the tile's P (bf16 pairs) once S has been read,
+// and the O accumulator at 128w + 96.  While the softmax works on one
+// buffer, the MMA fills the other with the next tile's logits.  With M = 256
+// warpgroup w owns latent rows [128w, 128w + 128) of every tile; with M = 128
+// the warpgroups take alternate tiles, each with its own running record.
 
 constexpr int kEncTile = 48;
-// TMEM columns of a softmax warpgroup, from its base 128 w: the S buffer
-// (48 fp32 logits), two P buffers (48 bf16 weights each) and the O
-// accumulator (D fp32).
-constexpr uint32_t kEncS = 0, kEncP = 48, kEncO = 96;
-// 256 x 96 + 128 x 40 <= 384 x 80 (the launch); the TMA and MMA warps need few
-constexpr int kEncRegsSoftmax = 96, kEncRegsProducer = 40;
+constexpr int kEncRegsSoftmax = 88, kEncRegsProducer = 56;   // 256 x 88 + 128 x 56 <= 384 x 80
 
 template <int D, int M, bool DZ = false>
 struct EncLayout {
@@ -143,7 +132,7 @@ struct EncLayout {
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = M * RB;
   static constexpr int BAR_OFF = KV_OFF + kEncStages * 2 * TILE;
-  static constexpr int NBARS = 2 * kEncStages + 1 + 2 + 2 + 4 + 4 + 2;
+  static constexpr int NBARS = 2 * kEncStages + 1 + 4 + 4 + 4 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   // dZ form: per stage, the tile's column offsets (kEncTile floats)
   static constexpr int NB_OFF = MISC_OFF + 16;
@@ -202,10 +191,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = bars + kEncStages;
   uint64_t* q_full = bars + 2 * kEncStages;
-  uint64_t* s_full = q_full + 1;      // [w]: S written by the MMA
-  uint64_t* s_read = s_full + 2;      // [w]: S read by the softmax
-  uint64_t* p_done = s_read + 2;      // [2w + b]: P written into P buffer b
-  uint64_t* pv_done = p_done + 4;     // [2w + b]: P.V of a tile from P buffer b complete
+  uint64_t* s_full = q_full + 1;      // [2w + b]: S written by the MMA
+  uint64_t* sp_done = s_full + 4;     // [2w + b]: S read and P written by the softmax
+  uint64_t* pv_done = sp_done + 4;    // [2w + b]: P.V of a tile from buffer b complete
   uint64_t* drain = pv_done + 4;      // [w]
   uint32_t* tmem_slot = (uint32_t*)(smem + L::MISC_OFF);
   volatile int* abort_flag = (volatile int*)(smem + L::MISC_OFF + 4);
@@ -226,12 +214,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&kv_empty[s], NH == 2 ? 2 : 1);   // one release per warpgroup reading the tile
     }
     mbar_init(q_full, 1);
-    for (int k = 0; k < 2; ++k) {
-      mbar_init(&s_full[k], 1);
-      mbar_init(&s_read[k], 128);
-    }
     for (int k = 0; k < 4; ++k) {
-      mbar_init(&p_done[k], 128);
+      mbar_init(&s_full[k], 1);
+      mbar_init(&sp_done[k], 128);
       mbar_init(&pv_done[k], 1);
     }
     for (int k = 0; k < 2; ++k) mbar_init(&drain[k], 1);
@@ -328,9 +313,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     } else if (warp == kWarpMma || warp == kWarpMma + 1) {
       // -------------------------------------- MMA issuers, one per warpgroup
       // Warp 9 serves softmax warpgroup 0 and warp 10 warpgroup 1.  For the
-      // warpgroup's j-th tile: once the softmax has read tile j's logits out
-      // of the S buffer (s_read), the S of tile j + 1 into it; once it has
-      // written tile j's P into P buffer j % 2 (p_done), P.V.
+      // warpgroup's j-th tile (buffer b = j % 2): P.V once the softmax has
+      // finished it; then, once that P.V has completed (it reads P from
+      // buffer b), the S of tile j + 2 into the same buffer.
       if (lane == 0) {
         const int w = warp - kWarpMma;
         constexpr uint32_t idS = idesc_bf16_f32(128, kEncTile, 0, 0);
@@ -350,24 +335,17 @@ __global__ void __launch_bounds__(kThreads, 2)
           if (!mbar_wait_sleep(&kv_full[s], (uint32_t)((i / kEncStages) & 1))) return false;
           tc_fence_after();
           const uint32_t koff = (uint32_t)(s * 2 * L::TILE) >> 4;
+          const int b = j & 1;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tW + kEncS, dQ + 2 * kk, dK + koff + 2 * kk, idS, kk > 0);
-          mma_commit(&s_full[w]);
+            mma_ss(tW + 48 * b, dQ + 2 * kk, dK + koff + 2 * kk, idS, kk > 0);
+          mma_commit(&s_full[2 * w + b]);
           return true;
         };
-        if (ok && nw > 0) ok = issue_S(0);
+        for (int j = 0; ok && j < 2 && j < nw; ++j) ok = issue_S(j);
         for (int j = 0; ok && j < nw; ++j) {
           const int b = j & 1;
-          if (j + 1 < nw) {
-            if (!MMA_WAIT(&s_read[w], (uint32_t)(j & 1))) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            if (!(ok = issue_S(j + 1))) break;
-          }
-          if (!MMA_WAIT(&p_done[2 * w + b], (uint32_t)((j >> 1) & 1))) {
+          if (!MMA_WAIT(&sp_done[2 * w + b], (uint32_t)((j >> 1) & 1))) {
             ok = false;
             break;
           }
@@ -376,10 +354,19 @@ __global__ void __launch_bounds__(kThreads, 2)
           const uint32_t voff = (uint32_t)((i % kEncStages) * 2 * L::TILE) >> 4;
 #pragma unroll
           for (int kk = 0; kk < kEncTile / 16; ++kk)
-            mma_ts(tW + kEncO, tW + kEncP + 24 * b + 8 * kk,
-                   dV + voff + ((uint32_t)(kk * 16 * RB) >> 4), idPV, (j > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tW + 96, tW + 48 * b + 8 * kk, dV + voff + ((uint32_t)(kk * 16 * RB) >> 4),
+                   idPV, (j > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&pv_done[2 * w + b]);
           mma_commit(&kv_empty[i % kEncStages]);
+          if (j + 2 < nw) {
+            // buffer b still holds the P this P.V reads: wait for it to finish
+            if (!MMA_WAIT(&pv_done[2 * w + b], (uint32_t)((j >> 1) & 1))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            if (!(ok = issue_S(j + 2))) break;
+          }
           if (*abort_flag) ok = false;
         }
         if (!ok) {
@@ -397,103 +384,201 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int r = q * 32 + lane;                     // TMEM lane = latent row in the half
     const uint32_t lb = (uint32_t)(q * 32) << 16;
     const uint32_t tW = tmem + lb + 128 * w;
-    const uint32_t tS = tW + kEncS;
-    const uint32_t tO = tW + kEncO;
+    const uint32_t tO = tW + 96;
     const int nW = (NH == 2) ? (int)ntiles : (int)((ntiles - w + 1) / 2);
     const int first = (NH == 2) ? 0 : w;
     float mref = -INFINITY, l = 0.f;
+    float pend = 1.f;   // factor O still owes to a move of m_ref
     bool ok = true;
     // P.V of this warpgroup's tile jj (and, by issue order, of every earlier
-    // one) has completed.  Each P buffer has its own barrier: with one
+    // one) has completed.  Each S buffer has its own barrier: with one
     // barrier per warpgroup a waiter two phases behind would read the
     // wrong parity as complete.
     auto pv_wait = [&](int jj) -> bool {
       return mbar_wait(&pv_done[2 * w + (jj & 1)], (uint32_t)((jj >> 1) & 1));
     };
-    for (int j = 0; j < nW; ++j) {
+    // Waits for the previous tile's P.V (O stable) and multiplies O by g.
+    auto scale_O = [&](int j, float g) -> bool {
+      if (!warp_any(g != 1.f)) return true;
+      if (j > 0) {
+        if (!warp_all(pv_wait(j - 1))) return false;
+        __syncwarp();
+        tc_fence_after();
+      }
+      scale_tmem_row<D>(tO, g);   // rows without a rescale multiply by 1
+      return true;
+    };
+    if constexpr (DZ) {
+      const float* nb_ring = (const float*)(smem + L::NB_OFF);
+      for (int j = 0; j < nW; ++j) {
+        const int64_t i = first + (int64_t)stride * j;
+        const int b = j & 1;
+        const int s = (int)(i % kEncStages);
+        const uint32_t tS = tW + 48 * b;
+        // the tile's S in TMEM, and its stage (with the column offsets) landed
+        if (!warp_all(mbar_wait(&s_full[2 * w + b], (uint32_t)((j >> 1) & 1)) &&
+                      mbar_wait(&kv_full[s], (uint32_t)((i / kEncStages) & 1)) && !*abort_flag)) {
+          ok = false;
+          break;
+        }
+        __syncwarp();
+        tc_fence_after();
+        const float* nb = nb_ring + s * kEncTile;
+        {
+          uint32_t a[32], pk[16];
+          tmem_ld32(tS, a);
+          tmem_wait_ld_dep(a);
+          exp_bias_pairs<16, kEncPolyEvery>(a, c, nb, pk);
+          tmem_st16(tS, pk);
+        }
+        {
+          uint32_t a[16], pk[8];
+          tmem_ld16(tS + 32, a);
+          tmem_wait_ld_dep16(a);
+          exp_bias_pairs<8, kEncPolyEvery16>(a, c, nb + 32, pk);
+          tmem_st8(tS + 16, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&sp_done[2 * w + b]);
+      }
+    }
+    for (int j = 0; !DZ && j < nW; ++j) {
       const int64_t i = first + (int64_t)stride * j;
       const int b = j & 1;
-      const int s = (int)(i % kEncStages);
       // the tile's own tokens are its columns [lo, hi); the rest get weight 0
       const int lo = ht.lo(tile0 + i, kEncTile), hi = ht.hi(tile0 + i, kEncTile);
       const bool full = (lo == 0 && hi == kEncTile);   // warp-uniform: only a head's last tile is partial
-      // the tile's S in TMEM (and, dZ form, its stage with the column offsets)
-      if (!warp_all(mbar_wait(&s_full[w], (uint32_t)(j & 1)) &&
-                    (!DZ || mbar_wait(&kv_full[s], (uint32_t)((i / kEncStages) & 1))) &&
-                    !*abort_flag)) {
+      const uint32_t tS = tW + 48 * b;
+      if (!warp_all(mbar_wait(&s_full[2 * w + b], (uint32_t)((j >> 1) & 1)) && !*abort_flag)) {
         ok = false;
         break;
       }
       __syncwarp();
       tc_fence_after();
-      // the tile's 48 logits into registers, masked columns at -inf
-      uint32_t a[32], a2[16];
-      tmem_ld32(tS, a);
-      tmem_wait_ld_dep(a);
-      tmem_ld16(tS + 32, a2);
-      tmem_wait_ld_dep16(a2);
-      if (!full) {
-#pragma unroll
-        for (int t = 0; t < 32; ++t)
-          if (t < lo || t >= hi) a[t] = __float_as_uint(-INFINITY);
-#pragma unroll
-        for (int t = 0; t < 16; ++t)
-          if (32 + t < lo || 32 + t >= hi) a2[t] = __float_as_uint(-INFINITY);
-      }
-      float g = 1.f;   // factor O owes before this tile's P.V
-      float mx2 = 0.f;
-      if constexpr (!DZ) {
-        float mf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        max_fold32(a, mf);
-        max_fold16(a2, mf);
-        mx2 = fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3])) * c;
-      }
-      // S has been read: the MMA warp may compute the next tile's into it
-      tc_fence_before();
-      mbar_arrive(&s_read[w]);
-      uint32_t pa[16], pb[8];
-      if constexpr (DZ) {
-        const float* nb = (const float*)(smem + L::NB_OFF) + s * kEncTile;
-        exp_bias_pairs<16, kEncPolyEvery>(a, c, nb, pa);
-        exp_bias_pairs<8, kEncPolyEvery16>(a2, c, nb + 32, pb);
-      } else {
-        // The reference m_ref moves up to the tile max whenever that is more
-        // than 2^kRescaleTau above it (l now, O before this tile's P.V), so
-        // every weight is at most 2^kRescaleTau.
-        if (mx2 > mref + kRescaleTau) {
-          if (mref != -INFINITY) g = ex2(mref - mx2);
-          l *= g;
-          mref = mx2;
-        }
+      // Optimistic single pass (every tile after a warpgroup's first): P is
+      // taken against the running reference m_ref and stays in registers
+      // until the overflow check below passes.
+      bool exact = warp_any(mref == -INFINITY);
+      if (!exact) {
         const float neg = -mref;
         float sf[4] = {0.f, 0.f, 0.f, 0.f};
-        exp_pack32<kEncPolyEvery>(a, c, neg, pa, sf);
-        exp_pack16<kEncPolyEvery16>(a2, c, neg, pb, sf);
-        l += (sf[0] + sf[1]) + (sf[2] + sf[3]);
-      }
-      // P buffer b was last read by tile j - 2's P.V; a rescale of O waits
-      // for tile j - 1's (O stable)
-      if (j >= 2 && !warp_all(pv_wait(j - 2))) {
-        ok = false;
-        break;
-      }
-      const uint32_t tP = tW + kEncP + 24 * b;
-      tmem_st16(tP, pa);
-      tmem_st8(tP + 16, pb);
-      if (!DZ && warp_any(g != 1.f)) {
-        if (j > 0) {
-          if (!warp_all(pv_wait(j - 1))) {
+        uint32_t pa[16], pb[8];
+        {
+          uint32_t a[32];
+          tmem_ld32(tS, a);
+          tmem_wait_ld_dep(a);
+          if (!full) {   // masked columns get weight 0
+#pragma unroll
+            for (int t = 0; t < 32; ++t)
+              if (t < lo || t >= hi) a[t] = __float_as_uint(-INFINITY);
+          }
+          exp_pack32<kEncPolyEvery, true>(a, c, neg, pa, sf);
+        }
+        {
+          uint32_t a[16];
+          tmem_ld16(tS + 32, a);
+          tmem_wait_ld_dep16(a);
+          if (!full) {
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+              if (32 + t < lo || 32 + t >= hi) a[t] = __float_as_uint(-INFINITY);
+          }
+          exp_pack16<kEncPolyEvery16, true>(a, c, neg, pb, sf);
+        }
+        const float sum = (sf[0] + sf[1]) + (sf[2] + sf[3]);
+        // Every weight of the tile is at most the tile's row sum, so the sum
+        // stands in for the max: above 2^kRedoTau (or not finite) a weight
+        // may have overflowed and the tile is recomputed with the exact max;
+        // above 2^kRescaleTau the reference moves up by log2(sum), which
+        // keeps it within log2(tile) of the running max.
+        if (warp_any(!(sum <= kRedoLimit))) {
+          exact = true;
+        } else {
+          if (!scale_O(j, pend)) {   // a rescale decided after the previous tile
             ok = false;
             break;
           }
-          __syncwarp();
-          tc_fence_after();
+          pend = 1.f;
+          tmem_st16(tS, pa);          // P over S columns already read
+          tmem_st8(tS + 16, pb);
+          if (sum > kRescaleLimit) {
+            const float mx2 = mref + lg2(sum);
+            pend = ex2(mref - mx2);
+            l = (l + sum) * pend;
+            mref = mx2;
+          } else {
+            l += sum;
+          }
         }
-        scale_tmem_row<D>(tO, g);   // rows without a rescale multiply by 1
+      }
+      if (exact) {
+        // pass 1: exact tile max of the raw logits (masked columns excluded)
+        float mf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        {
+          uint32_t a[32];
+          tmem_ld32(tS, a);
+          tmem_wait_ld_dep(a);
+#pragma unroll
+          for (int t = 0; t < 32; ++t)
+            if (t >= lo && t < hi) mf[t & 3] = fmaxf(mf[t & 3], __uint_as_float(a[t]));
+        }
+        {
+          uint32_t a[16];
+          tmem_ld16(tS + 32, a);
+          tmem_wait_ld_dep16(a);
+#pragma unroll
+          for (int t = 0; t < 16; ++t)
+            if (32 + t >= lo && 32 + t < hi) mf[t & 3] = fmaxf(mf[t & 3], __uint_as_float(a[t]));
+        }
+        const float mx2 = fmaxf(fmaxf(mf[0], mf[1]), fmaxf(mf[2], mf[3])) * c;
+        float f = 1.f;   // rescale of this row's earlier tiles (1 when the max did not move)
+        if (mx2 > mref) {
+          if (mref != -INFINITY) f = ex2(mref - mx2);
+          mref = mx2;
+        }
+        l *= f;
+        if (!scale_O(j, pend * f)) {
+          ok = false;
+          break;
+        }
+        pend = 1.f;
+        // pass 2: P = 2^(c S - m_ref) as bf16 pairs, and its row sum; chunk
+        // 0's P lands on S columns [0, 16) and chunk 1's on [16, 24), both
+        // already read.
+        const float neg = -mref;
+        float sf[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+          uint32_t a[32];
+          tmem_ld32(tS, a);
+          tmem_wait_ld_dep(a);
+          if (!full) {
+#pragma unroll
+            for (int t = 0; t < 32; ++t)
+              if (t < lo || t >= hi) a[t] = __float_as_uint(-INFINITY);
+          }
+          uint32_t pk[16];
+          exp_pack32<kEncPolyEvery, true>(a, c, neg, pk, sf);
+          tmem_st16(tS, pk);
+        }
+        {
+          uint32_t a[16];
+          tmem_ld16(tS + 32, a);
+          tmem_wait_ld_dep16(a);
+          if (!full) {
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+              if (32 + t < lo || 32 + t >= hi) a[t] = __float_as_uint(-INFINITY);
+          }
+          uint32_t pk[8];
+          exp_pack16<kEncPolyEvery16, true>(a, c, neg, pk, sf);
+          tmem_st8(tS + 16, pk);
+        }
+        l += (sf[0] + sf[1]) + (sf[2] + sf[3]);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_done[2 * w + b]);
+      mbar_arrive(&sp_done[2 * w + b]);
     }
     float acc[D];
 #pragma unroll
@@ -508,13 +593,13 @@ __global__ void __launch_bounds__(kThreads, 2)
           tmem_ld32(tO, o);
           tmem_wait_ld_dep(o);
 #pragma unroll
-          for (int d = 0; d < D; ++d) acc[d] = __uint_as_float(o[d]);
+          for (int d = 0; d < D; ++d) acc[d] = __uint_as_float(o[d]) * pend;
         } else {
           uint32_t o[16];
           tmem_ld16(tO, o);
           tmem_wait_ld_dep16(o);
 #pragma unroll
-          for (int d = 0; d < D; ++d) acc[d] = __uint_as_float(o[d & 15]);
+          for (int d = 0; d < D; ++d) acc[d] = __uint_as_float(o[d & 15]) * pend;
         }
       }
     }
