@@ -460,14 +460,31 @@ def run_ours(args, rank, world, local):
 _ROW_RATES = dict(NOMINAL_RATES, source="nominal")
 
 
+def _fwd_exp_floor(exps_per_stage: float, M: int, D: int, peaks: dict, stages=(0, 1)) -> float:
+    """Seconds the forward's exponentials need at least: each stage (0 =
+    an encode, 1 = the decode) computes exps_per_stage weights, a share of
+    them on the FMA-pipe polynomial (flare_exp_split), at the combined
+    MUFU + FMA ceiling of that share."""
+    import torch
+
+    import rank_latent_attention_flare_b200 as fl
+    clk = float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
+    return sum(exp_ceiling(exps_per_stage, fl.exp_split(k, M, D, torch.bfloat16), _ROW_RATES, clk)[0]
+               for k in stages)
+
+
 def _row_roofline(t_ms: float, exps: float, flops: float, hbm_bytes: float, peaks: dict,
-                  peak_kind: str):
+                  peak_kind: str, fwd_exp_s: float = 0.0, fwd_exps: float = 0.0):
     """Roofline of a whole row: the slowest of the exponential, tensor and
     HBM limits (each at its peak) over the measured time.  The exponential
-    limit takes every weight on the MUFU at the probe's measured rate."""
+    limit takes the forward's fwd_exps weights at their combined MUFU + FMA
+    floor fwd_exp_s (the kernels' polynomial shares) and the remaining
+    exps - fwd_exps (the backward's, all on the MUFU) at the probe's
+    measured MUFU rate."""
     clk = float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
     mufu = _ROW_RATES["ex2_per_clk_sm"] * _ROW_RATES["sms"] * clk   # exp/s
-    lim = {"exp": exps / mufu, "tensor": flops / (float(peaks["bf16_tflops"]) * 1e12),
+    lim = {"exp": fwd_exp_s + (exps - fwd_exps) / mufu,
+           "tensor": flops / (float(peaks["bf16_tflops"]) * 1e12),
            "hbm": hbm_bytes / (float(peaks["hbm_gbs"]) * 1e9)}
     bound = max(lim, key=lim.get)
     t = t_ms / 1e3
@@ -560,14 +577,9 @@ def _time_c2(dev, peaks, peak_kind, timed, seed, M=None, row="flare_fwd_c2"):
         raise RuntimeError("device wait ran out in the mesh-sized forward")
     u = w.B * w.H * w.N
     exps = u * w.M
-    clk = float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
-    t_ceil = sum(exp_ceiling(exps, fl.exp_split(k, w.M, w.D, w.torch_dtype), _ROW_RATES, clk)[0]
-                 for k in (0, 1))
+    t_ceil = _fwd_exp_floor(exps, w.M, w.D, peaks)
     roof = _row_roofline(ms, 2.0 * exps, 8.0 * u * w.M * w.D, 4.0 * u * w.D * 2, peaks,
-                         peak_kind)
-    roof["combined_exp_ceiling_ms"] = round(t_ceil * 1e3, 4)
-    roof["frac"] = round(t_ceil / (ms / 1e3), 4)
-    roof["bound"] = "exp (combined MUFU + FMA)"
+                         peak_kind, t_ceil, 2.0 * exps)
     return {row: {
         "workload": f"FLARE fwd B={w.B} H={w.H} N={w.N} M={w.M} D={w.D} bf16 (mesh 256x256)",
         "fwd_path": fl.fwd_path(w.B, w.H, w.N, w.M, w.D, w.torch_dtype),
@@ -590,7 +602,9 @@ def _time_pp(dev, peaks, peak_kind, timed, seed):
         "workload": f"FLARE++ fwd B={w.B} H={w.H} N={w.N} M={w.M} D={w.D} bf16",
         "ms": round(ms, 4), "tokens_per_s": w.B * w.N / (ms / 1e3),
         "roofline": _row_roofline(ms, 3.0 * u * w.M, 12.0 * u * w.M * w.D,
-                                  6.0 * u * w.D * 2, peaks, peak_kind)}
+                                  6.0 * u * w.D * 2, peaks, peak_kind,
+                                  _fwd_exp_floor(u * w.M, w.M, w.D, peaks, (0, 0, 1)),
+                                  3.0 * u * w.M)}
     return rows
 
 
@@ -626,7 +640,8 @@ def _time_fwd_bwd(dev, peaks, peak_kind, timed, seed, M=None, row="flare_fwd_bwd
         "ms": round(ms, 4), "fwd_ms": round(ms_f, 4), "bwd_ms": round(ms_b, 4),
         "tokens_per_s": w.B * w.N / (ms / 1e3),
         "roofline": _row_roofline(ms, 4.0 * u * w.M, 28.0 * u * w.M * w.D,
-                                  9.0 * u * w.D * 2, peaks, peak_kind),
+                                  9.0 * u * w.D * 2, peaks, peak_kind,
+                                  _fwd_exp_floor(u * w.M, w.M, w.D, peaks), 2.0 * u * w.M),
         "bwd_roofline": _row_roofline(ms_b, 2.0 * u * w.M, 20.0 * u * w.M * w.D,
                                       5.0 * u * w.D * 2, peaks, peak_kind)}
     return rows
@@ -666,7 +681,8 @@ def _time_strided(dev, peaks, peak_kind, timed, seed):
         "ms": round(ms_t, 4), "contiguous_ms": round(ms_c, 4),
         "tokens_per_s": w.B * w.N / (ms_t / 1e3),
         "roofline": _row_roofline(ms_t, 2.0 * u * w.M, 8.0 * u * w.M * w.D, 4.0 * u * w.D * 2,
-                                  peaks, peak_kind)}
+                                  peaks, peak_kind, _fwd_exp_floor(u * w.M, w.M, w.D, peaks),
+                                  2.0 * u * w.M)}
     w = WORKLOADS["c5_fwdbwd_bf16_16k"]
     x = make_inputs(w.B, w.H, w.N, w.M, w.D, dtype=w.torch_dtype, seed=seed, with_dy=True)
     Q = x["Q"].to(dev)
@@ -691,7 +707,8 @@ def _time_strided(dev, peaks, peak_kind, timed, seed):
         "ms": round(ms, 4), "fwd_ms": round(ms_f, 4), "bwd_ms": round(ms_b, 4),
         "tokens_per_s": w.B * w.N / (ms / 1e3),
         "roofline": _row_roofline(ms, 4.0 * u * w.M, 28.0 * u * w.M * w.D,
-                                  9.0 * u * w.D * 2, peaks, peak_kind)}
+                                  9.0 * u * w.D * 2, peaks, peak_kind,
+                                  _fwd_exp_floor(u * w.M, w.M, w.D, peaks), 2.0 * u * w.M)}
     return {"flare_strided": out}
 
 
@@ -731,7 +748,8 @@ def _time_varlen(dev, peaks, peak_kind, timed, seed):
         "ms": round(ms, 4), "fwd_ms": round(ms_f, 4), "bwd_ms": round(ms_b, 4),
         "valid_tokens_per_s": valid / (ms / 1e3),
         "roofline": _row_roofline(ms, 4.0 * u * w.M, 28.0 * u * w.M * w.D,
-                                  9.0 * u * w.D * 2, peaks, peak_kind)}}
+                                  9.0 * u * w.D * 2, peaks, peak_kind,
+                                  _fwd_exp_floor(u * w.M, w.M, w.D, peaks), 2.0 * u * w.M)}}
 
 
 def time_sdpa_context(dev, w=WORKLOAD, iters: int = 5, seed: int = 0):
@@ -799,7 +817,9 @@ def _time_pp_fwd_bwd(dev, peaks, peak_kind, timed, seed):
         "ms": round(ms, 4), "fwd_ms": round(ms_f, 4), "bwd_ms": round(ms_b, 4),
         "tokens_per_s": w.B * w.N / (ms / 1e3),
         "roofline": _row_roofline(ms, 6.0 * u * w.M, 42.0 * u * w.M * w.D,
-                                  11.0 * u * w.D * 2, peaks, peak_kind),
+                                  11.0 * u * w.D * 2, peaks, peak_kind,
+                                  _fwd_exp_floor(u * w.M, w.M, w.D, peaks, (0, 0, 1)),
+                                  3.0 * u * w.M),
         "bwd_roofline": _row_roofline(ms_b, 3.0 * u * w.M, 30.0 * u * w.M * w.D,
                                       5.0 * u * w.D * 2, peaks, peak_kind)}}
 
