@@ -678,7 +678,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int RB = L::RB;
   constexpr uint32_t SW = umma_swizzle_code(RB);
   // first-chunk reference under the row-max bound
-  constexpr bool kBound = (M == 256) && !PAD;
+#ifndef FLARE_DEC_BOUND128
+#define FLARE_DEC_BOUND128 0
+#endif
+  constexpr bool kBound = (M == 256 || (FLARE_DEC_BOUND128 && M == 128)) && !PAD;
   constexpr int R = M;                 // TMEM columns per warpgroup
   constexpr uint32_t NCOLS = 2 * R;    // 256 or 512
   constexpr int TY = M / 2;            // Y accumulator column inside a warpgroup's region
