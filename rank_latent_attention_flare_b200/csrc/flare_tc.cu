@@ -677,11 +677,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   using L = DecLayout<D, M>;
   constexpr int RB = L::RB;
   constexpr uint32_t SW = umma_swizzle_code(RB);
-  // first-chunk reference under the row-max bound
-#ifndef FLARE_DEC_BOUND128
-#define FLARE_DEC_BOUND128 0
-#endif
-  constexpr bool kBound = (M == 256 || (FLARE_DEC_BOUND128 && M == 128)) && !PAD;
+  // first-chunk reference under the row-max bound (measured no faster with
+  // M = 128, whose exact two-pass row is short)
+  constexpr bool kBound = (M == 256) && !PAD;
   constexpr int R = M;                 // TMEM columns per warpgroup
   constexpr uint32_t NCOLS = 2 * R;    // 256 or 512
   constexpr int TY = M / 2;            // Y accumulator column inside a warpgroup's region
