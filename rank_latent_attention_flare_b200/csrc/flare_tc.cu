@@ -639,7 +639,10 @@ struct DecLayout {
   static constexpr int TILE = kTile * RB;
   static constexpr int Q_OFF = 0;
   static constexpr int Z_OFF = M * RB;
-  static constexpr int K_OFF = 2 * M * RB;
+  // bf16 ones in Z's layout, right after Z: the second N-atom of Y's B
+  // operand [Z | 1], so Y's product also gives each row's weight sum
+  static constexpr int ONES_OFF = 2 * M * RB;
+  static constexpr int K_OFF = 3 * M * RB;
   static constexpr int BAR_OFF = K_OFF + kDecStages * TILE;
   static constexpr int NBARS = 2 * kDecStages + 1 + 4 * 2 + 1 + kDecBoundSlots + 4;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
@@ -680,9 +683,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   // first-chunk reference under the row-max bound (measured no faster with
   // M = 128, whose exact two-pass row is short)
   constexpr bool kBound = (M == 256) && !PAD;
-  constexpr int R = M;                 // TMEM columns per warpgroup
-  constexpr uint32_t NCOLS = 2 * R;    // 256 or 512
-  constexpr int TY = M / 2;            // Y accumulator column inside a warpgroup's region
+  // TMEM columns per warpgroup: S (M fp32 columns, P written over the ones
+  // already read) and the accumulator [Y | l] (D + 16 columns, l = the row's
+  // weight sum in its first column): inside S's upper half with M = 256
+  // (columns 128-175, below the upper P at 192), past S with M = 128.
+  constexpr int R = 256;
+  constexpr uint32_t NCOLS = 2 * R;
+  constexpr int TY = (M == 256) ? M / 2 : M;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -755,6 +762,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       qn2[m] = acc;
     }
   }
+  {
+    // the ones of Y's B operand (bf16 1.0, in Z's layout after Z)
+    uint4* ones = reinterpret_cast<uint4*>(smem + L::ONES_OFF);
+    for (int i = threadIdx.x; i < M * RB / 16; i += blockDim.x)
+      ones[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+    fence_proxy_async_smem();
+  }
   if (warp == kWarpMma) tmem_alloc(tmem_slot, NCOLS);
   tc_fence_before();
   __syncthreads();
@@ -793,7 +807,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpMma) {
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, M, 0, 0);
-      constexpr uint32_t idY = idesc_bf16_f32(128, D, 0, 1);
+      constexpr uint32_t idY = idesc_bf16_f32(128, D + 16, 0, 1);   // N = [Z | 1]
       const uint32_t q_addr = smem_u32(Qs);
       const uint32_t z_addr = smem_u32(Zs);
       bool ok = mbar_wait_sleep(qz_full, 0);
@@ -983,13 +997,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t a[32], pk[16];
             tmem_ld32(tR + col, a);
             tmem_wait_ld_dep(a);
-            exp_pack32<kDecPolyEvery>(a, c, neg, pk, sf);
+            exp_pack32<kDecPolyEvery, false, false>(a, c, neg, pk, sf);
             tmem_st16(tR + p_col(k), pk);
           } else {
             uint32_t a[16], pk[8];
             tmem_ld16(tR + col, a);
             tmem_wait_ld_dep16(a);
-            exp_pack16<0>(a, c, neg, pk, sf);
+            exp_pack16<0, false, false>(a, c, neg, pk, sf);
             tmem_st8(tR + p_col(k), pk);
           }
         }
@@ -1032,7 +1046,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (k > 0 || !kBound) tmem_wait_ld_dep(a[k & 1]);
           if (k + 1 < NC) tmem_ld32(tR + chunk_col(k + 1), a[(k + 1) & 1]);
           uint32_t pk[16];
-          exp_pack32<kDecPolyEvery>(a[k & 1], c, neg, pk, sf);
+          exp_pack32<kDecPolyEvery, false, false>(a[k & 1], c, neg, pk, sf);
           tmem_st16(tR + p_col(k), pk);
           if (k == NC / 2 - 1 || (NC == 8 && k == 5)) {
             tmem_wait_st();
@@ -1051,24 +1065,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       tc_fence_after();
-      float y[D];
+      // [Y | l]: l = the row's sum of its bf16 weights (the ones of Z's N-atom)
+      float y[D], l;
       if (D == 32) {
+        uint32_t o[32], o2[16];
+        tmem_ld32(tR + TY, o);
+        tmem_ld16(tR + TY + 32, o2);
+        tmem_wait_ld();
+#pragma unroll
+        for (int d = 0; d < D; ++d) y[d] = __uint_as_float(o[d]);
+        l = __uint_as_float(o2[0]);
+      } else {
         uint32_t o[32];
         tmem_ld32(tR + TY, o);
         tmem_wait_ld();
 #pragma unroll
-        for (int d = 0; d < D; ++d) y[d] = __uint_as_float(o[d]);
-      } else {
-        uint32_t o[16];
-        tmem_ld16(tR + TY, o);
-        tmem_wait_ld();
-#pragma unroll
-        for (int d = 0; d < D; ++d) y[d] = __uint_as_float(o[d & 15]);
+        for (int d = 0; d < D; ++d) y[d] = __uint_as_float(o[d & 31]);
+        l = __uint_as_float(o[16]);
       }
       tc_fence_before();
       mbar_arrive(&s_empty[w]);
       if constexpr (ST) {
-        const float l = (sf[0] + sf[1]) + (sf[2] + sf[3]);
         const float inv = 1.f / l;
         const float mxp = fmaf(rmx, c, log2f(l));   // the row's log-sum-exp, log2 units
         const float lg = mxp - Rh;                  // log2 of g
@@ -1097,7 +1114,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (warp_any(bad) && lane == 0) atomicOr(bs.flags + bh, 1u);
       } else if (mine) {
-        const float inv = 1.f / ((sf[0] + sf[1]) + (sf[2] + sf[3]));
+        const float inv = 1.f / l;
         uint4* dst = reinterpret_cast<uint4*>(Y + yhead + tok * ty.sn);
 #pragma unroll
         for (int v = 0; v < D / 8; ++v) {

@@ -445,7 +445,7 @@ __device__ __forceinline__ void max_fold16(const uint32_t (&a)[16], float (&m)[4
 // p = 2^(a*c + neg) for 32 logits: packed into 16 bf16 pairs, sums folded
 // into four independent accumulators.  With POLY_EVERY = k > 0, every k-th
 // pair is computed on the FMA pipe (exp2_fma) instead of the MUFU.
-template <int POLY_EVERY = 0, bool CLAMP_HI = false>
+template <int POLY_EVERY = 0, bool CLAMP_HI = false, bool SUM = true>
 __device__ __forceinline__ void exp_pack32(const uint32_t (&a)[32], float c, float neg,
                                            uint32_t (&pk)[16], float (&s)[4]);
 
@@ -549,7 +549,7 @@ __device__ __forceinline__ void exp2_fma_pair_logits(float a0, float a1, float c
 // (exp2_fma_pair_logits), for callers whose exponents can be large and
 // positive; otherwise they use exp2_fma_pair (exponents known to be at most
 // 126).
-template <int NP, int POLY_EVERY, bool CLAMP_HI = false>
+template <int NP, int POLY_EVERY, bool CLAMP_HI = false, bool SUM = true>
 __device__ __forceinline__ void exp_pack_pairs(const uint32_t* a, float c, float neg,
                                                uint32_t* pk, float (&s)[4]) {
   const uint64_t c2 = f32x2(c, c), n2 = f32x2(neg, neg);
@@ -574,24 +574,24 @@ __device__ __forceinline__ void exp_pack_pairs(const uint32_t* a, float c, float
       p0 = ex2(x0);
       p1 = ex2(x1);
     }
-    acc[t & 1] = add_f32x2(acc[t & 1], f32x2(p0, p1));
+    if (SUM) acc[t & 1] = add_f32x2(acc[t & 1], f32x2(p0, p1));
     pk[t] = pack_bf16(p0, p1);
   }
   split_f32x2(acc[0], s[0], s[1]);
   split_f32x2(acc[1], s[2], s[3]);
 }
 
-template <int POLY_EVERY, bool CLAMP_HI>
+template <int POLY_EVERY, bool CLAMP_HI, bool SUM>
 __device__ __forceinline__ void exp_pack32(const uint32_t (&a)[32], float c, float neg,
                                            uint32_t (&pk)[16], float (&s)[4]) {
-  exp_pack_pairs<16, POLY_EVERY, CLAMP_HI>(a, c, neg, pk, s);
+  exp_pack_pairs<16, POLY_EVERY, CLAMP_HI, SUM>(a, c, neg, pk, s);
 }
 
 // p = 2^(a*c + neg) for 16 logits: 8 bf16 pairs, sums into four accumulators.
-template <int POLY_EVERY = 0, bool CLAMP_HI = false>
+template <int POLY_EVERY = 0, bool CLAMP_HI = false, bool SUM = true>
 __device__ __forceinline__ void exp_pack16(const uint32_t (&a)[16], float c, float neg,
                                            uint32_t (&pk)[8], float (&s)[4]) {
-  exp_pack_pairs<8, POLY_EVERY, CLAMP_HI>(a, c, neg, pk, s);
+  exp_pack_pairs<8, POLY_EVERY, CLAMP_HI, SUM>(a, c, neg, pk, s);
 }
 
 }  // namespace tc
