@@ -715,8 +715,9 @@ def _time_strided(dev, peaks, peak_kind, timed, seed):
 def _time_varlen(dev, peaks, peak_kind, timed, seed):
     """Right-padded batches: the forward + backward workload (B=8 H=8
     N=16,384 M=128 D=32 bf16) with sequence lengths N - b N/16 (16,384 down
-    to 9,216, 78% of the tokens valid), beside the same call at full length.
-    Throughput counts valid tokens; the roofline is that of the valid work."""
+    to 9,216, 78% of the tokens valid), beside the same call without lengths
+    (`vs_full_length` = the ratio of their times).  Throughput counts valid
+    tokens; the roofline is that of the valid work."""
     import torch
 
     import rank_latent_attention_flare_b200 as fl
@@ -739,6 +740,15 @@ def _time_varlen(dev, peaks, peak_kind, timed, seed):
                                       workspace=wsb, seq_lens=lens))
     if fl.device_status(wsf) != 0 or fl.device_status(wsb) != 0:
         raise RuntimeError("device wait ran out in the variable-length forward + backward")
+
+    # the same call without lengths (every token valid), for the ratio
+    def fwd_full():
+        saved["full"] = fl.flare_fwd(g["Q"], g["K"], g["V"], w.scale, save=True, workspace=wsf)
+
+    ms_ff = timed(fwd_full)
+    _, Zf, lsef = saved["full"]
+    ms_fb = timed(lambda: fl.flare_bwd(g["Q"], g["K"], g["V"], g["dY"], Zf, lsef, w.scale,
+                                       workspace=wsb))
     valid = sum(lens_l)
     u = w.H * valid
     ms = ms_f + ms_b
@@ -746,6 +756,8 @@ def _time_varlen(dev, peaks, peak_kind, timed, seed):
         "workload": f"FLARE fwd+bwd B={w.B} H={w.H} N={w.N} M={w.M} D={w.D} bf16, "
                     f"seq_lens {lens_l[0]}..{lens_l[-1]} ({100 * valid / (w.B * w.N):.0f}% valid)",
         "ms": round(ms, 4), "fwd_ms": round(ms_f, 4), "bwd_ms": round(ms_b, 4),
+        "full_length_ms": round(ms_ff + ms_fb, 4),
+        "vs_full_length": round(ms / (ms_ff + ms_fb), 3),
         "valid_tokens_per_s": valid / (ms / 1e3),
         "roofline": _row_roofline(ms, 4.0 * u * w.M, 28.0 * u * w.M * w.D,
                                   9.0 * u * w.D * 2, peaks, peak_kind,

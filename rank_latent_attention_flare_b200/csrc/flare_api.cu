@@ -163,10 +163,10 @@ flare_status_t run_encode(const void* Q, int64_t qbs, const void* K, const void*
 
 flare_status_t run_combine(const Dims& d, flare_dtype_t dt, float* Z_save, float* lse_save,
                            const void* Qpp, void* Qdyn, const WsLayout& L, char* ws,
-                           cudaStream_t st) {
-  FLARE_CUDA(launch_combine(d, dt, L.enc.slots_per_bh(), 1, (const float*)(ws + L.part_ml),
+                           cudaStream_t st, const PadZero* pz = nullptr) {
+  FLARE_CUDA(launch_combine(d, dt, L.enc.slots_per_bh(), L.enc.sub, 1, (const float*)(ws + L.part_ml),
                             (const float*)(ws + L.part_acc), (float*)(ws + L.zf),
-                            (__nv_bfloat16*)(ws + L.zb), Z_save, lse_save, Qpp, Qdyn, st));
+                            (__nv_bfloat16*)(ws + L.zb), Z_save, lse_save, Qpp, Qdyn, st, pz));
   return FLARE_OK;
 }
 
@@ -316,11 +316,12 @@ flare_status_t flare_fwd_ex(const void* Q, int64_t qbs, const void* K, const voi
   char* ws = (char*)workspace;
   cudaStream_t st = (cudaStream_t)stream;
   FLARE_TRY(reset_error_word(ws, st));
-  FLARE_CUDA(launch_check_lens(d, (uint32_t*)(ws + L.hdr), st));
+  FLARE_CUDA(launch_var_plan(d, L, ws, st, sms));   // lengths: checked, work plans
   FLARE_TRY(run_encode(Q, qbs, K, V, d, dt, scale, L, ws, st));
-  FLARE_TRY(run_combine(d, dt, Z_save, lse_save, nullptr, nullptr, L, ws, st));
+  // Y = 0 at padding, by extra blocks of the combine
+  const PadZero pz = pad_zero(Y, d.y, nullptr, d.y, d, dt, 256);
+  FLARE_TRY(run_combine(d, dt, Z_save, lse_save, nullptr, nullptr, L, ws, st, &pz));
   FLARE_TRY(run_decode(Q, qbs, K, Y, d, dt, scale, L, ws, st, sms));
-  FLARE_CUDA(launch_zero_padding(Y, d.y, nullptr, d.y, d, dt, st));   // Y = 0 at padding
   return FLARE_OK;
 }
 
@@ -351,15 +352,16 @@ flare_status_t flare_pp_fwd_ex(const void* Q, const void* K, const void* V, void
   void* qdyn = Q_dyn_out ? Q_dyn_out : (void*)(ws + L.qdyn);
   const int64_t qdyn_bs = H * M * D;
   FLARE_TRY(reset_error_word(ws, st));
-  FLARE_CUDA(launch_check_lens(d, (uint32_t*)(ws + L.hdr), st));
+  FLARE_CUDA(launch_var_plan(d, L, ws, st, sms));   // lengths: checked, work plans
   // Z1 = encode(Q, K, V); Q_dyn = Q + Z1 (written by the combine)
   FLARE_TRY(run_encode(Q, 0, K, V, d, dt, scale, L, ws, st));
   FLARE_TRY(run_combine(d, dt, nullptr, nullptr, Q, qdyn, L, ws, st));
   // Z = encode(Q_dyn, K, V); Y = decode(Q_dyn, K, Z)
   FLARE_TRY(run_encode(qdyn, qdyn_bs, K, V, d, dt, scale, L, ws, st));
-  FLARE_TRY(run_combine(d, dt, Z_save, lse_save, nullptr, nullptr, L, ws, st));
+  // Y = 0 at padding, by extra blocks of the combine
+  const PadZero pz = pad_zero(Y, d.y, nullptr, d.y, d, dt, 256);
+  FLARE_TRY(run_combine(d, dt, Z_save, lse_save, nullptr, nullptr, L, ws, st, &pz));
   FLARE_TRY(run_decode(qdyn, qdyn_bs, K, Y, d, dt, scale, L, ws, st, sms));
-  FLARE_CUDA(launch_zero_padding(Y, d.y, nullptr, d.y, d, dt, st));   // Y = 0 at padding
   return FLARE_OK;
 }
 
@@ -382,7 +384,8 @@ flare_status_t flare_bwd_ex(const void* Q, int64_t qbs, const void* K, const voi
   FLARE_TRY(check_ptr(dK));
   FLARE_TRY(check_ptr(dV));
   FLARE_TRY(check_qbs(qbs, H, M, D));
-  const WsLayout L = ws_layout(FLARE_OP_BWD, B, H, N, M, D, dt, current_sm_count());
+  const int sms = current_sm_count();
+  const WsLayout L = ws_layout(FLARE_OP_BWD, B, H, N, M, D, dt, sms);
   FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
   FLARE_TRY(check_opt_lens(seq_lens));
   Dims d{B, H, N, M, D};
@@ -391,9 +394,11 @@ flare_status_t flare_bwd_ex(const void* Q, int64_t qbs, const void* K, const voi
   char* ws = (char*)workspace;
   cudaStream_t st = (cudaStream_t)stream;
   FLARE_TRY(reset_error_word(ws, st));
-  FLARE_CUDA(launch_check_lens(d, (uint32_t*)(ws + L.hdr), st));
-  FLARE_CUDA(launch_bwd(Q, qbs, K, V, dY, Z_save, lse_save, dQ, dK, dV, d, dt, scale, L, ws, st));
-  FLARE_CUDA(launch_zero_padding(dK, d.dk, dV, d.dv, d, dt, st));   // no gradient at padding
+  FLARE_CUDA(launch_var_plan(d, L, ws, st, sms));   // lengths: checked, work plans
+  // no gradient at padding: dK = dV = 0 there (zeroed by the backward)
+  const PadZero pz = pad_zero(dK, d.dk, dV, d.dv, d, dt, (int)M);
+  FLARE_CUDA(launch_bwd(Q, qbs, K, V, dY, Z_save, lse_save, dQ, dK, dV, d, dt, scale, L, ws, st,
+                        BwdPhase::ALL, nullptr, nullptr, &pz));
   return FLARE_OK;
 }
 
@@ -416,7 +421,8 @@ flare_status_t flare_pp_bwd_ex(const void* Q, const void* K, const void* V, cons
   FLARE_TRY(check_ptr(dQ));
   FLARE_TRY(check_ptr(dK));
   FLARE_TRY(check_ptr(dV));
-  const WsLayout L = ws_layout(FLARE_OP_PP_BWD, B, H, N, M, D, dt, current_sm_count());
+  const int sms = current_sm_count();
+  const WsLayout L = ws_layout(FLARE_OP_PP_BWD, B, H, N, M, D, dt, sms);
   FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
   FLARE_TRY(check_opt_lens(seq_lens));
   Dims d{B, H, N, M, D};
@@ -427,16 +433,17 @@ flare_status_t flare_pp_bwd_ex(const void* Q, const void* K, const void* V, cons
   float* z1 = (float*)(ws + L.z1);
   float* lse1 = (float*)(ws + L.lse1);
   FLARE_TRY(reset_error_word(ws, st));
-  FLARE_CUDA(launch_check_lens(d, (uint32_t*)(ws + L.hdr), st));
+  FLARE_CUDA(launch_var_plan(d, L, ws, st, sms));   // lengths: checked, work plans
   // the first encode, recomputed: Z1 and its lse
   FLARE_TRY(run_encode(Q, 0, K, V, d, dt, scale, L, ws, st));
   FLARE_TRY(run_combine(d, dt, z1, lse1, nullptr, nullptr, L, ws, st));
   // FLARE's backward with the per-batch latents Q_dyn: dQ_dyn, dK, dV
+  // (no gradient at padding: dK = dV = 0 there, zeroed by this backward)
+  const PadZero pz = pad_zero(dK, d.dk, dV, d.dv, d, dt, (int)M);
   FLARE_CUDA(launch_bwd(Q_dyn, H * M * D, K, V, dY, Z_save, lse_save, ws + L.dqd, dK, dV, d, dt,
-                        scale, L, ws, st));
-  // the first encode's gradient with upstream dQ_dyn, and dQ
+                        scale, L, ws, st, BwdPhase::ALL, nullptr, nullptr, &pz));
+  // the first encode's gradient with upstream dQ_dyn (valid rows only), and dQ
   FLARE_CUDA(launch_pp_bwd_tail(Q, K, V, z1, lse1, ws + L.dqd, dQ, dK, dV, d, dt, scale, L, ws, st));
-  FLARE_CUDA(launch_zero_padding(dK, d.dk, dV, d.dv, d, dt, st));   // no gradient at padding
   return FLARE_OK;
 }
 
@@ -505,7 +512,7 @@ flare_status_t flare_combine_shards(int64_t shards, const float* ml, const float
   FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
   g_error_detail[0] = 0;
   char* ws = (char*)workspace;
-  FLARE_CUDA(launch_combine(Dims{B, H, N, M, D}, dt, (int)records_per_bh, (int)shards, ml, acc,
+  FLARE_CUDA(launch_combine(Dims{B, H, N, M, D}, dt, (int)records_per_bh, 1, (int)shards, ml, acc,
                             (float*)(ws + L.zf), (__nv_bfloat16*)(ws + L.zb), Z_save, lse_save,
                             Q_dyn_out ? Q_learned : nullptr, Q_dyn_out, (cudaStream_t)stream));
   return FLARE_OK;

@@ -365,15 +365,21 @@ cudaError_t bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, cons
 cudaError_t launch_bwd(const void* Q, int64_t qbs, const void* K, const void* V, const void* dY,
                        const float* Z, const float* lse, void* dQ, void* dK, void* dV,
                        const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,
-                       char* ws, cudaStream_t st, BwdPhase phase, float* dz, float* dq32) {
+                       char* ws, cudaStream_t st, BwdPhase phase, float* dz, float* dq32,
+                       const PadZero* pz) {
+  // the tensor-core backward zeroes the padding in its preparation kernel;
+  // the CUDA-core one with the standalone kernel
   if (choose_path(d.N, d.M, d.D, dt).tc_bwd)
     return launch_tc_bwd(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st, phase, dz,
-                         dq32);
+                         dq32, pz);
 #define FLARE_BWD_T(T, DD) \
   bwd_t<T, DD>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st, phase, dz, dq32)
-  if (dt == FLARE_F32) return d.D == 16 ? FLARE_BWD_T(float, 16) : FLARE_BWD_T(float, 32);
-  return d.D == 16 ? FLARE_BWD_T(__nv_bfloat16, 16) : FLARE_BWD_T(__nv_bfloat16, 32);
+  cudaError_t e = (dt == FLARE_F32) ? (d.D == 16 ? FLARE_BWD_T(float, 16) : FLARE_BWD_T(float, 32))
+                                    : (d.D == 16 ? FLARE_BWD_T(__nv_bfloat16, 16)
+                                                 : FLARE_BWD_T(__nv_bfloat16, 32));
 #undef FLARE_BWD_T
+  if (e == cudaSuccess && pz) e = launch_pad_zero(*pz, d.BH(), st);
+  return e;
 }
 
 }  // namespace flare

@@ -41,6 +41,9 @@ enum ErrorSite : uint32_t {
 
 // ------------------------------------------------------------------ planning
 
+__host__ __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int64_t imax64(int64_t a, int64_t b) { return a > b ? a : b; }
+
 // Split of one (b, h) token range into `chunks` contiguous chunks of
 // `chunk_tiles` tiles of `tile` tokens (the last chunk may be shorter).
 struct ChunkPlan {
@@ -153,6 +156,13 @@ inline ChunkPlan decode_plan(int64_t BH, int64_t N, int sms) {
   return plan_chunks(BH, N, kTcTile, sms, 6.0, 16 * (int64_t)sms);
 }
 
+// Units a length-proportional plan may use (calls with lengths): at least
+// the chunk plan's, and up to two waves of `cta_slots` CTAs, but never more
+// than the tiles.
+inline int64_t var_units(int64_t BH, const ChunkPlan& p, int64_t cta_slots) {
+  return imax64(BH * p.chunks, imin64(2 * cta_slots, BH * p.tiles_per_bh));
+}
+
 inline ChunkPlan bwd_plan(int64_t BH, int64_t N, int sms) {
   return plan_chunks(BH, N, kBwdTile, 2LL * sms, 1.0, 16 * (int64_t)sms);
 }
@@ -192,6 +202,12 @@ struct WsLayout {
   size_t dz1 = 0;       // [BH][M][D] float  dQ_dyn widened
   size_t delta1 = 0;    // [BH][M] float  rowsum(dZ1 * Z1)
   size_t dqe = 0;       // [BH*chunks][M][D] float  first encode's dQ partials
+  // the work plans of calls with lengths (tensor-core path)
+  size_t vu_enc = 0;    // [n_enc] int4 units of the encode
+  size_t vh_enc = 0;    // [BH] int2 (first unit, units)
+  size_t vu_tok = 0;    // [n_tok] int4 units of the 128-token kernels
+  size_t vh_tok = 0;    // [BH] int2
+  int64_t n_enc = 0, n_tok = 0;
   size_t total = 0;
   ChunkPlan enc, bwd, ppe;
   ChunkPlan dec;        // tensor-core backward, M = 256: its decode-statistics pass
@@ -211,8 +227,19 @@ inline WsLayout ws_layout(flare_op_t op, int64_t B, int64_t H, int64_t N, int64_
     return o;
   };
   L.enc = encode_plan(BH, N, M, D, dt, sms);
-  const int64_t slots = BH * L.enc.slots_per_bh();
+  const Path path = choose_path(N, M, D, dt);
+  if (path.tc_fwd) {
+    L.n_enc = var_units(BH, L.enc, 2 * sms);
+    L.n_tok = var_units(BH, decode_plan(BH, N, sms), sms);
+  }
+  const int64_t slots = imax64(BH * L.enc.slots_per_bh(), L.n_enc * L.enc.sub);
   L.hdr = take(256);
+  if (path.tc_fwd) {
+    L.vu_enc = take((size_t)L.n_enc * 16);
+    L.vh_enc = take((size_t)BH * 8);
+    L.vu_tok = take((size_t)L.n_tok * 16);
+    L.vh_tok = take((size_t)BH * 8);
+  }
   L.part_ml = take((size_t)slots * M * 2 * 4);
   L.part_acc = take((size_t)slots * M * D * 4);
   L.zf = take((size_t)BH * M * D * 4);
@@ -221,9 +248,9 @@ inline WsLayout ws_layout(flare_op_t op, int64_t B, int64_t H, int64_t N, int64_
   const bool bwd_like = (op == FLARE_OP_BWD || op == FLARE_OP_PP_BWD);
   if (bwd_like && choose_path(N, M, D, dt).tc_bwd) {
     L.bwd = tc_bwd_plan(BH, N, sms);
-    const int64_t bslots = BH * L.bwd.chunks;
+    const int64_t bslots = imax64(BH * L.bwd.chunks, L.n_tok);
     // with M = 256 the dZ partials come from the encode pipeline (its chunks)
-    const int64_t zslots = (M == 256) ? BH * L.enc.slots_per_bh() : bslots;
+    const int64_t zslots = (M == 256) ? slots : bslots;
     if (M == 256) L.dec = decode_plan(BH, N, sms);
     L.stats = take((size_t)BH * N * 16);
     L.dy2 = take((size_t)BH * N * D * 2);
@@ -280,8 +307,6 @@ __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
 }
 
-__host__ __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
-
 __device__ __forceinline__ void record_error(uint32_t* err, uint32_t site) {
   if (err) atomicCAS(err, 0u, site);
 }
@@ -303,6 +328,18 @@ struct Tok {
   }
 };
 
+// A length-proportional work plan.  Unit u of a launch of `n` CTAs is
+// units[u] = (bh, first tile, tiles, 0) -- head bh's tiles split into
+// max(1, ceil(tiles / per)) near-equal units, heads in order, one CTA each;
+// bh < 0 marks a unit the plan leaves empty.  heads[bh] = (first unit, units)
+// locates a head's records, which the CTAs write at their unit's slot.
+struct VarPlan {
+  const int4* units = nullptr;
+  const int2* heads = nullptr;
+  int64_t n = 0;
+  bool on() const { return units != nullptr; }
+};
+
 // Problem sizes and the layouts of the token tensors (contiguous [B,H,N,D]
 // unless the caller gave strides).
 struct Dims {
@@ -310,8 +347,29 @@ struct Dims {
   Tok k = contig(), v = contig(), y = contig();     // K, V, the forward's Y
   Tok dy = contig(), dk = contig(), dv = contig();  // dY, dK, dV
   const int32_t* lens = nullptr;   // device [B]: valid tokens per batch element (NULL: N)
+  // With lengths on the tensor-core path, the length-proportional work plans
+  // that the plan kernel writes into the workspace (NULL otherwise): one for
+  // the 48-token encode, one for the 128-token kernels (decode, backward).
+  VarPlan venc, vtok;
   int64_t BH() const { return B * H; }
   Tok contig() const { return Tok{H * N * D, N * D, D}; }
+};
+
+// The padding rows (tokens [L_b, N)) of up to two token tensors of the same
+// shape, to be zeroed by `nxb` blocks per head: the standalone kernel, or
+// extra blocks of a kernel launched anyway (the combine, the backward's
+// preparation) beside its own.
+struct PadZero {
+  uint8_t* x0 = nullptr;   // NULL: nothing to zero
+  Tok t0{};
+  uint8_t* x1 = nullptr;
+  Tok t1{};
+  const int32_t* lens = nullptr;
+  int64_t N = 0;
+  int H = 1, esz = 2;
+  int lg_row = 2;          // log2 of the 16-byte pieces per row
+  int nxb = 0;             // blocks per head
+  int64_t blocks(int64_t BH) const { return x0 ? (int64_t)nxb * BH : 0; }
 };
 
 // Valid tokens of batch element b: lens[b] clamped to [0, N] (N when lens is
@@ -324,6 +382,24 @@ __device__ __forceinline__ int64_t seq_len(const int32_t* __restrict__ lens, int
 }
 
 __host__ __device__ __forceinline__ int64_t tiles_of(int64_t nb, int T) { return (nb + T - 1) / T; }
+
+// Block xb of a PadZero's nxb blocks for head bh: a stride loop over the
+// head's padding in 16-byte stores.
+__device__ __forceinline__ void zero_padding_part(const PadZero& z, int64_t xb, int64_t bh) {
+  const int64_t L = seq_len(z.lens, bh / z.H, z.N);
+  const int64_t total = (z.N - L) << z.lg_row;
+  if (total == 0) return;
+  const int mask = (1 << z.lg_row) - 1;
+  uint8_t* p0 = z.x0 + (z.t0.head(bh, z.H) + L * z.t0.sn) * z.esz;
+  uint8_t* p1 = z.x1 ? z.x1 + (z.t1.head(bh, z.H) + L * z.t1.sn) * z.esz : nullptr;
+  const int64_t r0 = z.t0.sn * z.esz, r1 = z.t1.sn * z.esz;   // row strides in bytes
+  for (int64_t i = xb * blockDim.x + threadIdx.x; i < total; i += (int64_t)z.nxb * blockDim.x) {
+    const int64_t n = i >> z.lg_row;
+    const int piece = (int)i & mask;
+    reinterpret_cast<uint4*>(p0 + n * r0)[piece] = make_uint4(0u, 0u, 0u, 0u);
+    if (p1) reinterpret_cast<uint4*>(p1 + n * r1)[piece] = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
 
 // Token tiles of one head, T tokens each.  Without lengths (VAR false) the
 // head has all N tokens: tile t covers rows [tT, tT + T) and TMA fills the
@@ -372,6 +448,45 @@ struct HeadTiles<true> {
   __device__ __forceinline__ int hi(int64_t, int T) const { return T; }
 };
 
+// The work of one CTA of a tensor-core kernel: head bh, its tiles [tile0,
+// tile0 + ntiles), and the slot of the records (partials) it writes.
+// Without lengths the grid is (chunks, BH) over the chunk plan; with them it
+// is one CTA per unit of the work plan, and bh < 0 leaves the CTA idle.
+struct CtaWork {
+  int64_t bh, tile0, ntiles, slot;
+};
+
+template <bool VAR>
+__device__ __forceinline__ CtaWork cta_work(const int4* __restrict__ units, int64_t chunk_tiles,
+                                            int64_t tiles_per_bh) {
+  CtaWork w;
+  if constexpr (VAR) {
+    const int4 u = units[blockIdx.x];
+    w.bh = u.x;
+    w.tile0 = u.y;
+    w.ntiles = u.z;
+    w.slot = blockIdx.x;
+  } else {
+    w.bh = blockIdx.y;
+    w.tile0 = (int64_t)blockIdx.x * chunk_tiles;
+    w.ntiles = imin64(chunk_tiles, tiles_per_bh - w.tile0);
+    w.slot = (int64_t)blockIdx.y * gridDim.x + blockIdx.x;
+  }
+  return w;
+}
+
+// The slot of this CTA's records (the same as cta_work's).
+template <bool VAR>
+__device__ __forceinline__ int64_t cta_slot() {
+  return VAR ? (int64_t)blockIdx.x : (int64_t)blockIdx.y * gridDim.x + blockIdx.x;
+}
+
+// Records (partials) of head bh: `count` slots from `first`, by the work
+// plan's head table when there is one, else the chunk plan's `chunks` per head.
+__device__ __forceinline__ int2 head_slots(const int2* __restrict__ heads, int64_t bh, int chunks) {
+  return heads ? heads[bh] : make_int2((int)(bh * chunks), chunks);
+}
+
 cudaError_t launch_simt_encode(const void* Q, int64_t qbs, const void* K, const void* V,
                                const Dims& d, flare_dtype_t dt, float scale,
                                const ChunkPlan& plan, float* part_ml, float* part_acc,
@@ -381,15 +496,23 @@ cudaError_t launch_simt_decode(const void* Q, int64_t qbs, const void* K, const 
                                cudaStream_t st);
 // Records kErrSeqLen when a length lies outside [0, N] (lens non-NULL).
 cudaError_t launch_check_lens(const Dims& d, uint32_t* err, cudaStream_t st);
+// Checks the lengths (as launch_check_lens) and writes the work plans of a
+// tensor-core call with lengths into the workspace; returns d with them attached.
+cudaError_t launch_var_plan(Dims& d, const WsLayout& L, char* ws, cudaStream_t st, int sms);
 // Zeroes the padding rows (n >= the batch element's length) of the token
 // tensor X0 with strides t0 and, when X1 is not NULL, of X1 (no-op when
 // d.lens is NULL).
-cudaError_t launch_zero_padding(void* X0, const Tok& t0, void* X1, const Tok& t1, const Dims& d,
-                                flare_dtype_t dt, cudaStream_t st);
-cudaError_t launch_combine(const Dims& d, flare_dtype_t dt, int slots_per_bh, int groups,
+// The padding of X0 (and X1) for blocks of `threads` threads (x0 NULL
+// without lengths).
+PadZero pad_zero(void* X0, const Tok& t0, void* X1, const Tok& t1, const Dims& d, flare_dtype_t dt,
+                 int threads);
+cudaError_t launch_pad_zero(const PadZero& z, int64_t BH, cudaStream_t st);
+// Records of head bh: slots_per_bh per head in each of `groups` blocks, or,
+// when d carries the encode's work plan, its units of `sub` records.
+cudaError_t launch_combine(const Dims& d, flare_dtype_t dt, int slots_per_bh, int sub, int groups,
                            const float* part_ml, const float* part_acc, float* Zf,
                            __nv_bfloat16* Zb, float* Z_save, float* lse_save, const void* Qpp,
-                           void* Qdyn, cudaStream_t st);
+                           void* Qdyn, cudaStream_t st, const PadZero* pz = nullptr);
 cudaError_t launch_tc_encode(const void* Q, int64_t qbs, const void* K, const void* V,
                              const Dims& d, float scale, const ChunkPlan& plan,
                              float* part_ml, float* part_acc, uint32_t* err, cudaStream_t st);
@@ -443,7 +566,7 @@ cudaError_t launch_tc_bwd(const void* Q, int64_t qbs, const void* K, const void*
                           const void* dY, const float* Z, const float* lse, void* dQ, void* dK,
                           void* dV, const Dims& d, float scale, const WsLayout& L, char* ws,
                           cudaStream_t st, BwdPhase phase = BwdPhase::ALL, float* dz = nullptr,
-                          float* dq32 = nullptr);
+                          float* dq32 = nullptr, const PadZero* pz = nullptr);
 // FLARE++'s first-encode gradient on the tensor cores (bf16, M = 128,
 // D in {16, 32}): adds into dK, dV and writes dQ (sum over the batch of dZ1
 // and the encode's dQ); reuses the tensor-core backward's workspace.
@@ -463,6 +586,6 @@ cudaError_t launch_bwd(const void* Q, int64_t qbs, const void* K, const void* V,
                        const float* Z, const float* lse, void* dQ, void* dK, void* dV,
                        const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,
                        char* ws, cudaStream_t st, BwdPhase phase = BwdPhase::ALL,
-                       float* dz = nullptr, float* dq32 = nullptr);
+                       float* dz = nullptr, float* dq32 = nullptr, const PadZero* pz = nullptr);
 
 }  // namespace flare

@@ -172,10 +172,10 @@ template <int D, int M, bool FLAT, bool VAR, bool DZ>
 __global__ void __launch_bounds__(kThreads, 2)
     tc_encode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, int H, int64_t N, int q_per_batch,
-                     int Mv, float c, int64_t tiles_per_bh, int64_t chunk_tiles, int slots_per_bh,
+                     int Mv, float c, int64_t tiles_per_bh, int64_t chunk_tiles,
                      float* __restrict__ part_ml, float* __restrict__ part_acc,
-                     const int32_t* __restrict__ lens, const float4* __restrict__ stats,
-                     uint32_t* __restrict__ err) {
+                     const int32_t* __restrict__ lens, const int4* __restrict__ units,
+                     const float4* __restrict__ stats, uint32_t* __restrict__ err) {
   using L = EncLayout<D, M, DZ>;
   constexpr int NH = M / 128;        // latent halves; M=128 -> the two warpgroups split tiles
   constexpr int SUB = (NH == 1) ? 2 : 1;
@@ -199,14 +199,14 @@ __global__ void __launch_bounds__(kThreads, 2)
   volatile int* abort_flag = (volatile int*)(smem + L::MISC_OFF + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int chunk = blockIdx.x;
-  const int64_t bh = blockIdx.y;
+  const CtaWork cw = cta_work<VAR>(units, chunk_tiles, tiles_per_bh);
+  if (cw.bh < 0) return;   // a unit the work plan leaves empty
+  const int64_t bh = cw.bh;
   const int64_t h = bh % H;
-  const int64_t tile0 = (int64_t)chunk * chunk_tiles;
-  // with lengths, tokens past the batch element's length are padding: their tiles are skipped
+  const int64_t tile0 = cw.tile0, ntiles = cw.ntiles;
+  // with lengths, tokens past the batch element's length are padding: the
+  // work plan covers the head's own tiles only
   const HeadTiles<VAR> ht(lens, bh / H, N);
-  const int64_t ntiles = VAR ? max(imin64(chunk_tiles, ht.count(kEncTile) - tile0), (int64_t)0)
-                             : imin64(chunk_tiles, tiles_per_bh - tile0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kEncStages; ++s) {
@@ -611,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       // MMA's 128-row tiles: computed alongside, never stored
       const int lat = (NH == 2 ? w * 128 : 0) + r;
       if (lat < Mv) {
-        const int64_t slot = bh * slots_per_bh + (int64_t)chunk * SUB + (NH == 1 ? w : 0);
+        const int64_t slot = cta_slot<VAR>() * SUB + (NH == 1 ? w : 0);
         const int64_t row = slot * Mv + lat;
         if (!DZ) {
           part_ml[row * 2 + 0] = (nW > 0) ? mref : -INFINITY;
@@ -675,8 +675,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap tmZ, int H, int64_t N, int q_per_batch,
                      int Mv, float c, int64_t tiles_per_bh, int64_t chunk_tiles,
                      __nv_bfloat16* __restrict__ Y, Tok ty, const __nv_bfloat16* __restrict__ Qg,
-                     const int32_t* __restrict__ lens, const DecStats bs,
-                     uint32_t* __restrict__ err) {
+                     const int32_t* __restrict__ lens, const int4* __restrict__ units,
+                     const DecStats bs, uint32_t* __restrict__ err) {
   using L = DecLayout<D, M>;
   constexpr int RB = L::RB;
   constexpr uint32_t SW = umma_swizzle_code(RB);
@@ -713,15 +713,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = (volatile int*)(smem + L::MISC_OFF + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int chunk = blockIdx.x;
-  const int64_t bh = blockIdx.y;
+  const CtaWork cw = cta_work<VAR>(units, chunk_tiles, tiles_per_bh);
+  if (cw.bh < 0) return;   // a unit the work plan leaves empty
+  const int64_t bh = cw.bh;
   const int64_t h = bh % H;
   const int64_t yhead = ty.head(bh, H);   // row 0 of this head in Y
-  const int64_t tile0 = (int64_t)chunk * chunk_tiles;
-  // with lengths, tokens past the batch element's length are padding: their tiles are skipped
+  const int64_t tile0 = cw.tile0, ntiles = cw.ntiles;
+  // with lengths, tokens past the batch element's length are padding: the
+  // work plan covers the head's own tiles only
   const HeadTiles<VAR> ht(lens, bh / H, N);
-  const int64_t ntiles = VAR ? max(imin64(chunk_tiles, ht.count(kTile) - tile0), (int64_t)0)
-                             : imin64(chunk_tiles, tiles_per_bh - tile0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDecStages; ++s) {
@@ -1233,10 +1233,11 @@ cudaError_t tc_encode_t(const void* Q, int64_t qbs, const void* K, const void* V
   e = cudaFuncSetAttribute(tc_encode_kernel<D, M, FLAT, VAR, DZ>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(plan.chunks, (unsigned)d.BH());
+  // with lengths: one CTA per unit of the encode's work plan
+  const dim3 grid = VAR ? dim3((unsigned)d.venc.n) : dim3(plan.chunks, (unsigned)d.BH());
   tc_encode_kernel<D, M, FLAT, VAR, DZ><<<grid, kThreads, smem, st>>>(
       mq, mk, mv, (int)d.H, d.N, q_per_batch, (int)d.M, scale * kLog2e, plan.tiles_per_bh,
-      plan.chunk_tiles, plan.slots_per_bh(), pml, pacc, d.lens, stats, err);
+      plan.chunk_tiles, pml, pacc, d.lens, d.venc.units, stats, err);
   return cudaPeekAtLastError();
 }
 
@@ -1256,11 +1257,12 @@ cudaError_t tc_decode_t(const void* Q, int64_t qbs, const void* K, const __nv_bf
   e = cudaFuncSetAttribute(tc_decode_kernel<D, M, FLAT, VAR, ST, PAD>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(plan.chunks, (unsigned)d.BH());
+  // with lengths: one CTA per unit of the 128-token work plan
+  const dim3 grid = VAR ? dim3((unsigned)d.vtok.n) : dim3(plan.chunks, (unsigned)d.BH());
   tc_decode_kernel<D, M, FLAT, VAR, ST, PAD><<<grid, kThreads, smem, st>>>(
       mq, mk, mz, (int)d.H, d.N, q_per_batch, (int)d.M, scale * kLog2e, plan.tiles_per_bh,
-      plan.chunk_tiles,
-      (__nv_bfloat16*)Y, d.y, (const __nv_bfloat16*)Q, d.lens, bs, err);
+      plan.chunk_tiles, (__nv_bfloat16*)Y, d.y, (const __nv_bfloat16*)Q, d.lens, d.vtok.units, bs,
+      err);
   return cudaPeekAtLastError();
 }
 

@@ -143,7 +143,8 @@ __global__ void __launch_bounds__(kThr, 1)
                     int64_t chunk_tiles, const float* __restrict__ rref,
                     float4* __restrict__ stats, __nv_bfloat16* __restrict__ dy2,
                     uint32_t* __restrict__ flags, float* __restrict__ dz_part,
-                    const int32_t* __restrict__ lens, uint32_t* __restrict__ err) {
+                    const int32_t* __restrict__ lens, const int4* __restrict__ units,
+                    uint32_t* __restrict__ err) {
   using L = ALayout<D>;
   constexpr int M = L::M;
   constexpr int RB = L::RB;
@@ -176,14 +177,15 @@ __global__ void __launch_bounds__(kThr, 1)
   volatile int* abort_flag = (volatile int*)(smem + L::MISC_OFF + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int chunk = blockIdx.x, chunks = gridDim.x;
-  const int64_t bh = blockIdx.y;
+  const CtaWork cw = cta_work<VAR>(units, chunk_tiles, tiles_per_bh);
+  if (cw.bh < 0) return;   // a unit the work plan leaves empty
+  const int64_t bh = cw.bh;
   const int64_t h = bh % H;
-  const int64_t tile0 = (int64_t)chunk * chunk_tiles;
-  // with lengths, tokens past the batch element's length are padding: their tiles are skipped
+  const int64_t tile0 = cw.tile0;
+  const int nt = (int)cw.ntiles;
+  // with lengths, tokens past the batch element's length are padding: the
+  // work plan covers the head's own tiles only
   const HeadTiles<VAR> ht(lens, bh / H, N);
-  const int nt = VAR ? (int)max(imin64(chunk_tiles, ht.count(kT) - tile0), (int64_t)0)
-                     : (int)imin64(chunk_tiles, tiles_per_bh - tile0);
 
   // Y = P [Z | e0]: the second N block of the B operand holds a one in
   // column 0 of every latent row (same swizzled layout as the Z rows), so
@@ -525,7 +527,7 @@ __global__ void __launch_bounds__(kThr, 1)
           *abort_flag = 1;
         }
       }
-      float4* dst = reinterpret_cast<float4*>(dz_part + (((int64_t)bh * chunks + chunk) * M + r) * D);
+      float4* dst = reinterpret_cast<float4*>(dz_part + (cta_slot<VAR>() * M + r) * D);
 #pragma unroll
       for (int d = 0; d < D / 4; ++d)
         dst[d] = make_float4(acc[4 * d], acc[4 * d + 1], acc[4 * d + 2], acc[4 * d + 3]);
@@ -547,8 +549,13 @@ template <int D, int M>
 __global__ void __launch_bounds__(M)
     bwd_prep_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
                     __nv_bfloat16* __restrict__ zb, float* __restrict__ rref,
-                    uint32_t* __restrict__ flags) {
+                    uint32_t* __restrict__ flags, int64_t BH, const PadZero z) {
   __shared__ float red[M / 32];
+  if (blockIdx.x >= BH) {   // the padding rows of dK and dV
+    const int64_t x = blockIdx.x - BH;
+    zero_padding_part(z, x % z.nxb, x / z.nxb);
+    return;
+  }
   const int64_t bh = blockIdx.x;
   const int m = threadIdx.x;
   const int64_t row = bh * M + m;
@@ -572,14 +579,14 @@ __global__ void __launch_bounds__(M)
 }
 
 // One block per (b, h), one thread per latent m.  dZ = sum of the chunk
-// partials (fixed order), lse2 = lse log2(e); R = max lse2 over the head;
+// partials (fixed order; the work plan's head table locates them when given), lse2 = lse log2(e); R = max lse2 over the head;
 // f = 2^(R - lse2) when the head's lse2 spread is at most kSpreadMax and no
 // token of it lies more than kRowRangeMax below R (else f = 1 and the exact
 // form); the bf16 operand dZ'' = f dZ; the extra K-step row: -dZ'' . Z
 // (= -f delta_e) as three bf16 terms, then zeros.
 template <int D, int M>
 __global__ void __launch_bounds__(M)
-    bwd_mid_kernel(const float* __restrict__ dz_part, int chunks,
+    bwd_mid_kernel(const float* __restrict__ dz_part, int chunks, const int2* __restrict__ heads,
                    const __nv_bfloat16* __restrict__ dz_direct, const float* __restrict__ Z,
                    const float* __restrict__ lse, __nv_bfloat16* __restrict__ dzs,
                    uint32_t* __restrict__ aug, const uint32_t* __restrict__ flags,
@@ -595,15 +602,33 @@ __global__ void __launch_bounds__(M)
 #pragma unroll
     for (int d = 0; d < D; ++d) dz[d] = __bfloat162float(dz_direct[row * D + d]);
   }
-  for (int k = 0; k < chunks; ++k) {
-    const float4* p = reinterpret_cast<const float4*>(dz_part + ((bh * chunks + k) * M + m) * D);
+  const int2 hs = head_slots(heads, bh, chunks);
+  // two partials' loads in flight at a time, added in partial order
+  for (int k = 0; k < hs.y; k += 2) {
+    const float4* p = reinterpret_cast<const float4*>(dz_part + (((int64_t)hs.x + k) * M + m) * D);
+    const float4* p2 = p + (int64_t)M * D / 4;
+    const bool two = k + 1 < hs.y;
+    float4 v[D / 4], v2[D / 4];
 #pragma unroll
     for (int d = 0; d < D / 4; ++d) {
-      const float4 v = p[d];
-      dz[4 * d] += v.x;
-      dz[4 * d + 1] += v.y;
-      dz[4 * d + 2] += v.z;
-      dz[4 * d + 3] += v.w;
+      v[d] = p[d];
+      if (two) v2[d] = p2[d];
+    }
+#pragma unroll
+    for (int d = 0; d < D / 4; ++d) {
+      dz[4 * d] += v[d].x;
+      dz[4 * d + 1] += v[d].y;
+      dz[4 * d + 2] += v[d].z;
+      dz[4 * d + 3] += v[d].w;
+    }
+    if (two) {
+#pragma unroll
+      for (int d = 0; d < D / 4; ++d) {
+        dz[4 * d] += v2[d].x;
+        dz[4 * d + 1] += v2[d].y;
+        dz[4 * d + 2] += v2[d].z;
+        dz[4 * d + 3] += v2[d].w;
+      }
     }
   }
   const float l2 = lse[row] * kLog2e;
@@ -694,7 +719,8 @@ __global__ void __launch_bounds__(kThr, 1)
                     const float* __restrict__ lse2, int mode, int m0, int Mt,
                     __nv_bfloat16* __restrict__ dK,
                     __nv_bfloat16* __restrict__ dV, Tok tdk, Tok tdv, float* __restrict__ dq_part,
-                    const int32_t* __restrict__ lens, uint32_t* __restrict__ err) {
+                    const int32_t* __restrict__ lens, const int4* __restrict__ units,
+                    uint32_t* __restrict__ err) {
   using L = BLayout<D>;
   constexpr int M = L::M;
   constexpr int NQ = L::NQ;
@@ -724,15 +750,15 @@ __global__ void __launch_bounds__(kThr, 1)
   volatile int* abort_flag = (volatile int*)(smem + L::MISC_OFF + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int chunk = blockIdx.x, chunks = gridDim.x;
-  const int64_t bh = blockIdx.y;
+  const CtaWork cw = cta_work<VAR>(units, chunk_tiles, tiles_per_bh);
+  if (cw.bh < 0) return;   // a unit the work plan leaves empty
+  const int64_t bh = cw.bh;
   const int64_t h = bh % H;
   const int64_t dk_head = tdk.head(bh, H), dv_head = tdv.head(bh, H);   // row 0 of the head
-  const int64_t tile0 = (int64_t)chunk * chunk_tiles;
-  // with lengths, tokens past the batch element's length are padding: their tiles are skipped
+  const int64_t tile0 = cw.tile0, ntiles = cw.ntiles;
+  // with lengths, tokens past the batch element's length are padding: the
+  // work plan covers the head's own tiles only
   const HeadTiles<VAR> ht(lens, bh / H, N);
-  const int64_t ntiles = VAR ? max(imin64(chunk_tiles, ht.count(kT) - tile0), (int64_t)0)
-                             : imin64(chunk_tiles, tiles_per_bh - tile0);
   const int64_t KQ = ntiles * NQ;   // quarters of this chunk
   const bool enc_only = (mode & kModeEncOnly) != 0;   // no decode term
   const bool accum = (mode & kModeAccum) != 0;        // dK, dV added to the rows' values
@@ -1088,7 +1114,7 @@ __global__ void __launch_bounds__(kThr, 1)
           *abort_flag = 1;
         }
       }
-      float4* dst = reinterpret_cast<float4*>(dq_part + (((int64_t)bh * chunks + chunk) * Mt + m0 + r) * D);
+      float4* dst = reinterpret_cast<float4*>(dq_part + (cta_slot<VAR>() * Mt + m0 + r) * D);
 #pragma unroll
       for (int d = 0; d < D / 4; ++d)
         dst[d] = make_float4(acc[4 * d], acc[4 * d + 1], acc[4 * d + 2], acc[4 * d + 3]);
@@ -1153,7 +1179,7 @@ __global__ void __launch_bounds__(kThr, 1)
                          int mode, int m0, int Mt, __nv_bfloat16* __restrict__ dK,
                          __nv_bfloat16* __restrict__ dV, Tok tdk, Tok tdv,
                          float* __restrict__ dq_part, const int32_t* __restrict__ lens,
-                         uint32_t* __restrict__ err) {
+                         const int4* __restrict__ units, uint32_t* __restrict__ err) {
   using L = BFLayout<D>;
   constexpr int M = L::M;
   constexpr int NS = L::NSLOT;
@@ -1188,15 +1214,16 @@ __global__ void __launch_bounds__(kThr, 1)
   volatile int* abort_flag = (volatile int*)(smem + L::MISC_OFF + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int chunk = blockIdx.x, chunks = gridDim.x;
-  const int64_t bh = blockIdx.y;
+  const CtaWork cw = cta_work<VAR>(units, chunk_tiles, tiles_per_bh);
+  if (cw.bh < 0) return;   // a unit the work plan leaves empty
+  const int64_t bh = cw.bh;
   const int64_t h = bh % H;
   const int64_t dk_head = tdk.head(bh, H), dv_head = tdv.head(bh, H);   // row 0 of the head
-  const int64_t tile0 = (int64_t)chunk * chunk_tiles;
-  // with lengths, tokens past the batch element's length are padding: their tiles are skipped
+  const int64_t tile0 = cw.tile0;
+  const int nt = (int)cw.ntiles;
+  // with lengths, tokens past the batch element's length are padding: the
+  // work plan covers the head's own tiles only
   const HeadTiles<VAR> ht(lens, bh / H, N);
-  const int nt = VAR ? (int)max(imin64(chunk_tiles, ht.count(kT) - tile0), (int64_t)0)
-                     : (int)imin64(chunk_tiles, tiles_per_bh - tile0);
   const float2 prm = params[bh];
   if (prm.y == 0.f) return;   // head served by tc_bwd_b_exact_kernel
   const bool enc_only = (mode & kModeEncOnly) != 0;   // no decode term
@@ -1565,7 +1592,7 @@ __global__ void __launch_bounds__(kThr, 1)
           *abort_flag = 1;
         }
       }
-      float4* dst = reinterpret_cast<float4*>(dq_part + (((int64_t)bh * chunks + chunk) * Mt + m0 + r) * D);
+      float4* dst = reinterpret_cast<float4*>(dq_part + (cta_slot<VAR>() * Mt + m0 + r) * D);
 #pragma unroll
       for (int d = 0; d < D / 4; ++d)
         dst[d] = make_float4(acc[4 * d], acc[4 * d + 1], acc[4 * d + 2], acc[4 * d + 3]);
@@ -1579,25 +1606,32 @@ __global__ void __launch_bounds__(kThr, 1)
 }
 
 // dQ = sum over (batch when Q is shared) x chunks of the scaled partials,
-// in a fixed order (batch outer, chunk inner).  One thread per 4 output
-// elements; the partials' loads are issued in groups of 8 before they are
-// added, so their latencies overlap.  With Q shared, `extra` (if given,
-// [B][H][M][D] bf16) is summed over the batch first: FLARE++'s dQ_dyn.
+// in a fixed order.  Eight lanes per 4 output elements: with Q shared, lane
+// s sums the partials of batch elements s, s + 8, ... (batch outer, chunk
+// inner), else those of chunks s, s + 8, ...; the eight sums then combine in
+// a butterfly (the same on every lane).  With Q shared, `extra` (if given,
+// [B][H][M][D] bf16) is summed over the batch first, by lane 0: FLARE++'s
+// dQ_dyn.
+constexpr int kDqLanes = 8;
+
 __global__ void bwd_dq_sum_kernel(const float4* __restrict__ dq_part, int B, int H, int M, int D,
-                                  int chunks, bool shared_q, const __nv_bfloat16* __restrict__ extra,
+                                  int chunks, const int2* __restrict__ heads, bool shared_q,
+                                  const __nv_bfloat16* __restrict__ extra,
                                   __nv_bfloat16* __restrict__ dQ, float4* __restrict__ dQ32) {
   const int64_t md4 = (int64_t)M * D / 4;
   const int64_t per4 = (int64_t)H * md4;
   const int64_t total4 = shared_q ? per4 : (int64_t)B * per4;
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t i = gid / kDqLanes;
+  const int s = (int)(gid % kDqLanes);
+  // whole warps lie inside or outside the output (total4 is a multiple of 4)
   if (i >= total4) return;
   const int64_t b0 = shared_q ? 0 : i / per4;
   const int64_t rr = i % per4;
   const int64_t h = rr / md4;
   const int64_t e = rr % md4;
-  const int n = (shared_q ? B : 1) * chunks;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (extra && shared_q) {
+  if (extra && shared_q && s == 0) {
     for (int b = 0; b < B; ++b) {
       const uint2 x = *reinterpret_cast<const uint2*>(extra + (b * per4 + i) * 4);
       acc.x += bf_lo(x.x);
@@ -1606,26 +1640,40 @@ __global__ void bwd_dq_sum_kernel(const float4* __restrict__ dq_part, int B, int
       acc.w += bf_hi(x.y);
     }
   }
-  for (int q0 = 0; q0 < n; q0 += 8) {
-    float4 v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int q = q0 + u;
-      if (q < n) {
-        const int64_t bh = (b0 + q / chunks) * H + h;
-        v[u] = dq_part[(bh * chunks + q % chunks) * md4 + e];
+  auto add = [&](const float4 v) {
+    acc.x += v.x;
+    acc.y += v.y;
+    acc.z += v.z;
+    acc.w += v.w;
+  };
+  if (shared_q) {
+    for (int64_t b = s; b < B; b += kDqLanes) {
+      const int2 hs = head_slots(heads, b * H + h, chunks);
+      int k = 0;
+      for (; k + 4 <= hs.y; k += 4) {   // four loads in flight
+        const float4 v0 = dq_part[((int64_t)hs.x + k) * md4 + e];
+        const float4 v1 = dq_part[((int64_t)hs.x + k + 1) * md4 + e];
+        const float4 v2 = dq_part[((int64_t)hs.x + k + 2) * md4 + e];
+        const float4 v3 = dq_part[((int64_t)hs.x + k + 3) * md4 + e];
+        add(v0);
+        add(v1);
+        add(v2);
+        add(v3);
       }
+      for (; k < hs.y; ++k) add(dq_part[((int64_t)hs.x + k) * md4 + e]);
     }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (q0 + u < n) {
-        acc.x += v[u].x;
-        acc.y += v[u].y;
-        acc.z += v[u].z;
-        acc.w += v[u].w;
-      }
-    }
+  } else {
+    const int2 hs = head_slots(heads, b0 * H + h, chunks);
+    for (int k = s; k < hs.y; k += kDqLanes) add(dq_part[((int64_t)hs.x + k) * md4 + e]);
   }
+#pragma unroll
+  for (int o = 1; o < kDqLanes; o <<= 1) {
+    acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
+    acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
+    acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
+    acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
+  }
+  if (s != 0) return;
   if (dQ32)
     dQ32[i] = acc;
   else
@@ -1635,14 +1683,16 @@ __global__ void bwd_dq_sum_kernel(const float4* __restrict__ dq_part, int B, int
 // This device's dZ: the fixed-order sum over chunks of pass A's partials,
 // [BH][chunks][M][D] -> [BH][M][D].  One thread per 4 elements.
 __global__ void bwd_dz_sum_kernel(const float4* __restrict__ dz_part, int64_t BH, int M, int D,
-                                  int chunks, float4* __restrict__ dz) {
+                                  int chunks, const int2* __restrict__ heads,
+                                  float4* __restrict__ dz) {
   const int64_t md4 = (int64_t)M * D / 4;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= BH * md4) return;
   const int64_t bh = i / md4, e = i % md4;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int k = 0; k < chunks; ++k) {
-    const float4 v = dz_part[(bh * chunks + k) * md4 + e];
+  const int2 hs = head_slots(heads, bh, chunks);
+  for (int k = 0; k < hs.y; ++k) {
+    const float4 v = dz_part[((int64_t)hs.x + k) * md4 + e];
     acc.x += v.x;
     acc.y += v.y;
     acc.z += v.z;
@@ -1663,7 +1713,7 @@ template <int D, int M, bool FLAT, bool VAR>
 cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, const void* dY,
                      const float* Z, const float* lse, void* dQ, void* dK, void* dV, const Dims& d,
                      float scale, const WsLayout& L, char* ws, cudaStream_t st, BwdPhase phase,
-                     float* dz_io, float* dq32) {
+                     float* dz_io, float* dq32, const PadZero* pz) {
   const ChunkPlan& p = L.bwd;
   const int64_t BH = d.BH();
   const int q_per_batch = qbs != 0;
@@ -1681,10 +1731,15 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
   float* lse2 = (float*)(ws + L.lse2);
   float* dqp = (float*)(ws + L.dqp);
   const int zchunks = (M == kM) ? p.chunks : L.enc.slots_per_bh();   // dZ partials per head
+  // with lengths: the work plans' head tables locate the partials
+  const int2* zheads = VAR ? ((M == kM) ? d.vtok.heads : d.venc.heads) : nullptr;
+  const int2* qheads = VAR ? d.vtok.heads : nullptr;
   cudaError_t e;
 
   if (phase != BwdPhase::FINISH) {
-    bwd_prep_kernel<D, M><<<(unsigned)BH, M, 0, st>>>(Z, lse, zb, rref, flags);
+    const PadZero z = pz ? *pz : PadZero{};
+    bwd_prep_kernel<D, M><<<(unsigned)(BH + z.blocks(BH)), M, 0, st>>>(Z, lse, zb, rref, flags,
+                                                                      BH, z);
     if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   }
 
@@ -1699,7 +1754,8 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
   if ((e = make_map(&mdz, dzs, D, M, BH, kM)) != cudaSuccess) return e;
   if ((e = make_map(&maug, aug, 16, M, BH, kM)) != cudaSuccess) return e;
 
-  dim3 grid(p.chunks, (unsigned)BH);
+  // with lengths: one CTA per unit of the 128-token work plan
+  const dim3 grid = VAR ? dim3((unsigned)d.vtok.n) : dim3(p.chunks, (unsigned)BH);
   if (phase != BwdPhase::FINISH) {
     if constexpr (M == kM) {
       const int smemA = ALayout<D>::BYTES + 1024;
@@ -1708,7 +1764,7 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
       if (e != cudaSuccess) return e;
       tc_bwd_a_kernel<D, FLAT, VAR><<<grid, kThr, smemA, st>>>(
           mq, mk, mdy, mz, (int)d.H, d.N, q_per_batch, c, p.tiles_per_bh, p.chunk_tiles, rref,
-          stats, dy2, flags, dzp, d.lens, err);
+          stats, dy2, flags, dzp, d.lens, d.vtok.units, err);
       if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
     } else {
       if ((e = launch_tc_bwd_stats(Q, qbs, K, zb, dY, d, scale, L.dec, rref, stats, dy2, flags,
@@ -1720,14 +1776,16 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
     if (phase == BwdPhase::DZ) {   // this device's part of dZ
       const int64_t n4 = BH * M * D / 4;
       bwd_dz_sum_kernel<<<(unsigned)((n4 + 127) / 128), 128, 0, st>>>(
-          (const float4*)dzp, BH, M, D, zchunks, (float4*)dz_io);
+          (const float4*)dzp, BH, M, D, zchunks, zheads, (float4*)dz_io);
       return cudaPeekAtLastError();
     }
   }
 
   // dZ: the chunk partials, or (FINISH) the sum over the shards as one partial
   bwd_mid_kernel<D, M><<<(unsigned)BH, M, 0, st>>>(phase == BwdPhase::FINISH ? dz_io : dzp,
-                                                   phase == BwdPhase::FINISH ? 1 : zchunks, nullptr,
+                                                   phase == BwdPhase::FINISH ? 1 : zchunks,
+                                                   phase == BwdPhase::FINISH ? nullptr : zheads,
+                                                   nullptr,
                                                    Z, lse, dzs, (uint32_t*)aug, flags, params, lse2);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
@@ -1745,19 +1803,19 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
     tc_bwd_b_fast_kernel<D, FLAT, VAR><<<grid, kThr, smemF, st>>>(
         mq, mk, mv, mdy2, mz, mdz, maug, (int)d.H, d.N, q_per_batch, c, scale, p.tiles_per_bh,
         p.chunk_tiles, stats, params, mode, m0, M, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, d.dk,
-        d.dv, dqp, d.lens, err);
+        d.dv, dqp, d.lens, d.vtok.units, err);
     if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
     tc_bwd_b_exact_kernel<D, FLAT, VAR><<<grid, kThr, smemB, st>>>(
         mq, mk, mv, mdy, mz, mdz, maug, (int)d.H, d.N, q_per_batch, c, scale, p.tiles_per_bh,
         p.chunk_tiles, stats, params, lse2, mode, m0, M, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV,
-        d.dk, d.dv, dqp, d.lens, err);
+        d.dk, d.dv, dqp, d.lens, d.vtok.units, err);
     if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   }
 
   const bool shared_q = (qbs == 0);
   const int64_t total = shared_q ? d.H * M * D : BH * M * D;
-  bwd_dq_sum_kernel<<<(unsigned)((total / 4 + 127) / 128), 128, 0, st>>>(
-      (const float4*)dqp, (int)d.B, (int)d.H, M, D, p.chunks, shared_q, nullptr,
+  bwd_dq_sum_kernel<<<(unsigned)((total / 4 * kDqLanes + 127) / 128), 128, 0, st>>>(
+      (const float4*)dqp, (int)d.B, (int)d.H, M, D, p.chunks, qheads, shared_q, nullptr,
       (__nv_bfloat16*)dQ, (float4*)dq32);
   return cudaPeekAtLastError();
 }
@@ -1789,10 +1847,11 @@ cudaError_t tc_enc_bwd_t(const void* Q, const void* K, const void* V, const floa
   cudaError_t e;
 
   // bf16 Z1 and a cleared range flag (no decode, so no token can raise it)
-  bwd_prep_kernel<D, M><<<(unsigned)BH, M, 0, st>>>(Z1, lse1, zb, rref, flags);
+  bwd_prep_kernel<D, M><<<(unsigned)BH, M, 0, st>>>(Z1, lse1, zb, rref, flags, BH, PadZero{});
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
-  bwd_mid_kernel<D, M><<<(unsigned)BH, M, 0, st>>>(nullptr, 0, (const __nv_bfloat16*)dZ1, Z1, lse1,
-                                                   dzs, (uint32_t*)aug, flags, params, lse2);
+  bwd_mid_kernel<D, M><<<(unsigned)BH, M, 0, st>>>(nullptr, 0, nullptr, (const __nv_bfloat16*)dZ1,
+                                                   Z1, lse1, dzs, (uint32_t*)aug, flags, params,
+                                                   lse2);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
   // the decode operands' maps point at V: valid tiles that are never used
@@ -1804,7 +1863,8 @@ cudaError_t tc_enc_bwd_t(const void* Q, const void* K, const void* V, const floa
   if ((e = make_map(&mdz, dzs, D, M, BH, kM)) != cudaSuccess) return e;
   if ((e = make_map(&maug, aug, 16, M, BH, kM)) != cudaSuccess) return e;
 
-  dim3 grid(p.chunks, (unsigned)BH);
+  // with lengths: one CTA per unit of the 128-token work plan
+  const dim3 grid = VAR ? dim3((unsigned)d.vtok.n) : dim3(p.chunks, (unsigned)BH);
   const int smemF = BFLayout<D>::BYTES + 1024;
   e = cudaFuncSetAttribute(tc_bwd_b_fast_kernel<D, FLAT, VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smemF);
@@ -1817,18 +1877,18 @@ cudaError_t tc_enc_bwd_t(const void* Q, const void* K, const void* V, const floa
     tc_bwd_b_fast_kernel<D, FLAT, VAR><<<grid, kThr, smemF, st>>>(
         mq, mk, mv, mv, mz, mdz, maug, (int)d.H, d.N, 0, c, scale, p.tiles_per_bh, p.chunk_tiles,
         stats, params, kModeEncOnly | kModeAccum, m0, M, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV,
-        d.dk, d.dv, dqp, d.lens, err);
+        d.dk, d.dv, dqp, d.lens, d.vtok.units, err);
     if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
     tc_bwd_b_exact_kernel<D, FLAT, VAR><<<grid, kThr, smemB, st>>>(
         mq, mk, mv, mv, mz, mdz, maug, (int)d.H, d.N, 0, c, scale, p.tiles_per_bh, p.chunk_tiles,
         stats, params, lse2, kModeEncOnly | kModeAccum, m0, M, (__nv_bfloat16*)dK,
-        (__nv_bfloat16*)dV, d.dk, d.dv, dqp, d.lens, err);
+        (__nv_bfloat16*)dV, d.dk, d.dv, dqp, d.lens, d.vtok.units, err);
     if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   }
 
   const int64_t total = d.H * M * D;
-  bwd_dq_sum_kernel<<<(unsigned)((total / 4 + 127) / 128), 128, 0, st>>>(
-      (const float4*)dqp, (int)d.B, (int)d.H, M, D, p.chunks, true,
+  bwd_dq_sum_kernel<<<(unsigned)((total / 4 * kDqLanes + 127) / 128), 128, 0, st>>>(
+      (const float4*)dqp, (int)d.B, (int)d.H, M, D, p.chunks, VAR ? d.vtok.heads : nullptr, true,
       (dq32 && !add_dz1) ? nullptr : (const __nv_bfloat16*)dZ1, (__nv_bfloat16*)dQ,
       (float4*)dq32);
   return cudaPeekAtLastError();
@@ -1838,10 +1898,11 @@ template <int D, int M>
 cudaError_t tc_bwd_dispatch(const void* Q, int64_t qbs, const void* K, const void* V,
                             const void* dY, const float* Z, const float* lse, void* dQ, void* dK,
                             void* dV, const Dims& d, float scale, const WsLayout& L, char* ws,
-                            cudaStream_t st, BwdPhase ph, float* dz, float* dq32) {
+                            cudaStream_t st, BwdPhase ph, float* dz, float* dq32,
+                            const PadZero* pz) {
   const bool flat = tok_flat(d), var = d.lens != nullptr;
 #define FLARE_TC_BWD_T(F, V_) \
-  tc_bwd_t<D, M, F, V_>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st, ph, dz, dq32)
+  tc_bwd_t<D, M, F, V_>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st, ph, dz, dq32, pz)
   if (flat) return var ? FLARE_TC_BWD_T(true, true) : FLARE_TC_BWD_T(true, false);
   return var ? FLARE_TC_BWD_T(false, true) : FLARE_TC_BWD_T(false, false);
 #undef FLARE_TC_BWD_T
@@ -1865,10 +1926,11 @@ cudaError_t tc_enc_bwd_dispatch(const void* Q, const void* K, const void* V, con
 cudaError_t launch_tc_bwd(const void* Q, int64_t qbs, const void* K, const void* V,
                           const void* dY, const float* Z, const float* lse, void* dQ, void* dK,
                           void* dV, const Dims& d, float scale, const WsLayout& L, char* ws,
-                          cudaStream_t st, BwdPhase phase, float* dz, float* dq32) {
+                          cudaStream_t st, BwdPhase phase, float* dz, float* dq32,
+                          const PadZero* pz) {
 #define FLARE_TC_BWD(D_, M_)                                                                  \
   tc_bwd_dispatch<D_, M_>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st, phase, dz, \
-                          dq32)
+                          dq32, pz)
   if (d.D == 32 && d.M == 128) return FLARE_TC_BWD(32, 128);
   if (d.D == 32 && d.M == 256) return FLARE_TC_BWD(32, 256);
   if (d.D == 16 && d.M == 128) return FLARE_TC_BWD(16, 128);

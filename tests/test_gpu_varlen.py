@@ -14,7 +14,7 @@ import torch
 import oracle
 import rank_latent_attention_flare_b200 as fl
 from flare_inputs import make_inputs
-from gpu_util import TOL_F32_GRAD_REL, assert_close, max_abs
+from gpu_util import TOL_F32_GRAD_REL, assert_close, max_abs, to64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -178,3 +178,57 @@ def test_out_of_range_lengths_are_clamped_and_reported():
                       seq_lens=torch.tensor([N, 0], dtype=torch.int32, device=DEV))
     torch.cuda.synchronize()
     assert torch.equal(Y, Yc)
+
+
+def _plan_lens(B, N, seed):
+    r = np.random.default_rng(seed)
+    lens = r.integers(0, N + 1, size=B)
+    lens[0], lens[-1] = N, 0
+    return [int(v) for v in lens]
+
+
+# Length-proportional work plans: one long sequence among short ones (its
+# tiles split into many units, the short heads into one each), and a batch
+# larger than the plan kernel's thread count (its scan over the batch takes
+# several elements per thread).
+PLAN_CASES = [
+    (4, 8, 20000, 128, 32, [20000, 3000, 0, 17]),
+    (2, 4, 9000, 256, 32, [9000, 1]),
+    (1100, 1, 64, 128, 16, _plan_lens(1100, 64, 87)),
+]
+PLAN_IDS = ["skewed_M128", "skewed_M256", "batch1100"]
+
+
+@pytest.mark.parametrize("B,H,N,M,D,lens", PLAN_CASES, ids=PLAN_IDS)
+def test_varlen_work_plan_matches_oracle(B, H, N, M, D, lens):
+    dtype = torch.bfloat16
+    s = 1.0 / math.sqrt(D)
+    x, g = _inputs(B, H, N, M, D, dtype, lens, seed=88 + B)
+    wsf = fl.alloc_workspace(fl.FLARE_OP_FWD, B, H, N, M, D, dtype, DEV)
+    wsb = fl.alloc_workspace(fl.FLARE_OP_BWD, B, H, N, M, D, dtype, DEV)
+    wsf.fill_(0xFF)
+    wsb.fill_(0xFF)
+    Y, Z, lse = fl.flare_fwd(g["Q"], g["K"], g["V"], s, save=True, seq_lens=g["lens"],
+                             workspace=wsf)
+    dQ, dK, dV = fl.flare_bwd(g["Q"], g["K"], g["V"], g["dY"], Z, lse, s, seq_lens=g["lens"],
+                              workspace=wsb)
+    assert fl.device_status(wsf) == 0 and fl.device_status(wsb) == 0
+    Yo, Zo, _ = oracle.flare_fwd(x["Q"], x["K"], x["V"], s, seq_lens=lens)
+    dQo, dKo, dVo = oracle.flare_bwd(x["Q"], x["K"], x["V"], x["dY"], s, seq_lens=lens)
+    for t in (Y, Z, dQ, dK, dV):
+        assert torch.isfinite(t).all()
+    _check_padding_zero(Y, lens, "Y")
+    _check_padding_zero(dK, lens, "dK")
+    _check_padding_zero(dV, lens, "dV")
+    if B > 64:   # many short heads: compare all valid rows at once
+        mask = np.zeros(tuple(Y.shape), dtype=bool)
+        for b, L in enumerate(lens):
+            mask[b, :, :L] = True
+        for got, ref, what in ((Y, Yo, "Y"), (dK, dKo, "dK"), (dV, dVo, "dV")):
+            assert_close(to64(got)[mask], np.asarray(ref)[mask], dtype, what)
+    else:
+        _close_valid(Y, Yo, lens, dtype, "Y")
+        _close_valid(dK, dKo, lens, dtype, "dK")
+        _close_valid(dV, dVo, lens, dtype, "dV")
+    assert_close(Z, Zo, dtype, "Z")
+    assert_close(dQ, dQo, dtype, "dQ")
