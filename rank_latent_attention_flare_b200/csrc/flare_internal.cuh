@@ -448,6 +448,35 @@ struct HeadTiles<true> {
   __device__ __forceinline__ int hi(int64_t, int T) const { return T; }
 };
 
+// Programmatic dependent launch.  A kernel launched by launch_pdl may be
+// scheduled while the kernel before it in the stream is still running:
+// pdl_wait() returns once that kernel has completed and its writes are
+// visible (at once when there is none), so each such kernel calls it before
+// touching global memory or tensor memory; pdl_trigger() lets the next
+// kernel be scheduled as soon as every CTA of this one has started.  The
+// next kernel's CTAs then wait on the SMs this one frees, and the launch gap
+// between the two disappears.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // The work of one CTA of a tensor-core kernel: head bh, its tiles [tile0,
 // tile0 + ntiles), and the slot of the records (partials) it writes.
 // Without lengths the grid is (chunks, BH) over the chunk plan; with them it

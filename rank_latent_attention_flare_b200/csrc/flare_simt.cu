@@ -153,6 +153,8 @@ __global__ void combine_kernel(const float* __restrict__ part_ml,
                                __nv_bfloat16* __restrict__ Zb, float* __restrict__ Z_save,
                                float* __restrict__ lse_save, const T* __restrict__ Qpp,
                                T* __restrict__ Qdyn) {
+  pdl_wait();   // the previous kernel's results (programmatic dependent launch)
+  pdl_trigger();
   if (blockIdx.x >= own_blocks) {   // the padding rows of Y
     const int64_t x = blockIdx.x - own_blocks;
     zero_padding_part(z, x % z.nxb, x / z.nxb);
@@ -274,6 +276,8 @@ __device__ __forceinline__ void plan_head(const PlanKind& k, int64_t bh, int64_t
 __global__ void __launch_bounds__(kPlanThreads)
     var_plan_kernel(const int32_t* __restrict__ lens, int64_t B, int64_t H, int64_t N,
                     PlanKind k0, PlanKind k1, uint32_t* __restrict__ err) {
+  pdl_wait();   // the previous kernel's results (programmatic dependent launch)
+  pdl_trigger();
   __shared__ double s_cost[2][kPlanCaps];
   __shared__ int64_t s_per[2][kPlanCaps];
   __shared__ int64_t s_scan[2][kPlanThreads / 32];
@@ -497,8 +501,8 @@ PadZero pad_zero(void* X0, const Tok& t0, void* X1, const Tok& t1, const Dims& d
   z.esz = (dt == FLARE_F32) ? 4 : 2;
   const int per_row = (int)d.D * z.esz / 16;   // 16-byte pieces per row: 2, 4 or 8
   z.lg_row = per_row == 2 ? 1 : (per_row == 4 ? 2 : 3);
-  // about four pieces per thread for a head that is all padding, at most 32 blocks
-  z.nxb = (int)imax64(1, imin64((d.N * per_row + 4 * threads - 1) / (4 * threads), 32));
+  // about sixteen pieces per thread for a head that is all padding, at most 32 blocks
+  z.nxb = (int)imax64(1, imin64((d.N * per_row + 16 * threads - 1) / (16 * threads), 32));
   return z;
 }
 
@@ -518,11 +522,11 @@ cudaError_t launch_combine(const Dims& d, flare_dtype_t dt, int slots_per_bh, in
   const PadZero z = pz ? *pz : PadZero{};
   const unsigned blocks = (unsigned)(own + z.blocks(d.BH()));
   if (dt == FLARE_F32)
-    combine_kernel<float><<<blocks, threads, 0, st>>>(
+    launch_pdl(combine_kernel<float>, blocks, threads, 0, st,
         part_ml, part_acc, d.BH(), (int)d.H, (int)d.M, (int)d.D, slots_per_bh, groups,
         d.venc.heads, sub, z, own, Zf, Zb, Z_save, lse_save, (const float*)Qpp, (float*)Qdyn);
   else
-    combine_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(
+    launch_pdl(combine_kernel<__nv_bfloat16>, blocks, threads, 0, st,
         part_ml, part_acc, d.BH(), (int)d.H, (int)d.M, (int)d.D, slots_per_bh, groups,
         d.venc.heads, sub, z, own, Zf, Zb, Z_save, lse_save, (const __nv_bfloat16*)Qpp,
         (__nv_bfloat16*)Qdyn);

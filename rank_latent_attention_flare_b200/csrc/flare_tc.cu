@@ -176,6 +176,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                      float* __restrict__ part_ml, float* __restrict__ part_acc,
                      const int32_t* __restrict__ lens, const int4* __restrict__ units,
                      const float4* __restrict__ stats, uint32_t* __restrict__ err) {
+  pdl_wait();   // the previous kernel's results (programmatic dependent launch)
+  pdl_trigger();
   using L = EncLayout<D, M, DZ>;
   constexpr int NH = M / 128;        // latent halves; M=128 -> the two warpgroups split tiles
   constexpr int SUB = (NH == 1) ? 2 : 1;
@@ -677,6 +679,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                      __nv_bfloat16* __restrict__ Y, Tok ty, const __nv_bfloat16* __restrict__ Qg,
                      const int32_t* __restrict__ lens, const int4* __restrict__ units,
                      const DecStats bs, uint32_t* __restrict__ err) {
+  pdl_wait();   // the previous kernel's results (programmatic dependent launch)
+  pdl_trigger();
   using L = DecLayout<D, M>;
   constexpr int RB = L::RB;
   constexpr uint32_t SW = umma_swizzle_code(RB);
@@ -1235,7 +1239,7 @@ cudaError_t tc_encode_t(const void* Q, int64_t qbs, const void* K, const void* V
   if (e != cudaSuccess) return e;
   // with lengths: one CTA per unit of the encode's work plan
   const dim3 grid = VAR ? dim3((unsigned)d.venc.n) : dim3(plan.chunks, (unsigned)d.BH());
-  tc_encode_kernel<D, M, FLAT, VAR, DZ><<<grid, kThreads, smem, st>>>(
+  launch_pdl(tc_encode_kernel<D, M, FLAT, VAR, DZ>, grid, kThreads, smem, st,
       mq, mk, mv, (int)d.H, d.N, q_per_batch, (int)d.M, scale * kLog2e, plan.tiles_per_bh,
       plan.chunk_tiles, pml, pacc, d.lens, d.venc.units, stats, err);
   return cudaPeekAtLastError();
@@ -1259,7 +1263,7 @@ cudaError_t tc_decode_t(const void* Q, int64_t qbs, const void* K, const __nv_bf
   if (e != cudaSuccess) return e;
   // with lengths: one CTA per unit of the 128-token work plan
   const dim3 grid = VAR ? dim3((unsigned)d.vtok.n) : dim3(plan.chunks, (unsigned)d.BH());
-  tc_decode_kernel<D, M, FLAT, VAR, ST, PAD><<<grid, kThreads, smem, st>>>(
+  launch_pdl(tc_decode_kernel<D, M, FLAT, VAR, ST, PAD>, grid, kThreads, smem, st,
       mq, mk, mz, (int)d.H, d.N, q_per_batch, (int)d.M, scale * kLog2e, plan.tiles_per_bh,
       plan.chunk_tiles, (__nv_bfloat16*)Y, d.y, (const __nv_bfloat16*)Q, d.lens, d.vtok.units, bs,
       err);

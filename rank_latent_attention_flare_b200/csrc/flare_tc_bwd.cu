@@ -145,6 +145,8 @@ __global__ void __launch_bounds__(kThr, 1)
                     uint32_t* __restrict__ flags, float* __restrict__ dz_part,
                     const int32_t* __restrict__ lens, const int4* __restrict__ units,
                     uint32_t* __restrict__ err) {
+  pdl_wait();   // the previous kernel's results (programmatic dependent launch)
+  pdl_trigger();
   using L = ALayout<D>;
   constexpr int M = L::M;
   constexpr int RB = L::RB;
@@ -550,6 +552,8 @@ __global__ void __launch_bounds__(M)
     bwd_prep_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
                     __nv_bfloat16* __restrict__ zb, float* __restrict__ rref,
                     uint32_t* __restrict__ flags, int64_t BH, const PadZero z) {
+  pdl_wait();   // the previous kernel's results (programmatic dependent launch)
+  pdl_trigger();
   __shared__ float red[M / 32];
   if (blockIdx.x >= BH) {   // the padding rows of dK and dV
     const int64_t x = blockIdx.x - BH;
@@ -591,6 +595,8 @@ __global__ void __launch_bounds__(M)
                    const float* __restrict__ lse, __nv_bfloat16* __restrict__ dzs,
                    uint32_t* __restrict__ aug, const uint32_t* __restrict__ flags,
                    float2* __restrict__ params, float* __restrict__ lse2_out) {
+  pdl_wait();   // the previous kernel's results (programmatic dependent launch)
+  pdl_trigger();
   __shared__ float red_max[M / 32], red_min[M / 32];
   const int64_t bh = blockIdx.x;
   const int m = threadIdx.x;
@@ -721,6 +727,8 @@ __global__ void __launch_bounds__(kThr, 1)
                     __nv_bfloat16* __restrict__ dV, Tok tdk, Tok tdv, float* __restrict__ dq_part,
                     const int32_t* __restrict__ lens, const int4* __restrict__ units,
                     uint32_t* __restrict__ err) {
+  pdl_wait();   // the previous kernel's results (programmatic dependent launch)
+  pdl_trigger();
   using L = BLayout<D>;
   constexpr int M = L::M;
   constexpr int NQ = L::NQ;
@@ -1180,6 +1188,8 @@ __global__ void __launch_bounds__(kThr, 1)
                          __nv_bfloat16* __restrict__ dV, Tok tdk, Tok tdv,
                          float* __restrict__ dq_part, const int32_t* __restrict__ lens,
                          const int4* __restrict__ units, uint32_t* __restrict__ err) {
+  pdl_wait();   // the previous kernel's results (programmatic dependent launch)
+  pdl_trigger();
   using L = BFLayout<D>;
   constexpr int M = L::M;
   constexpr int NS = L::NSLOT;
@@ -1618,6 +1628,8 @@ __global__ void bwd_dq_sum_kernel(const float4* __restrict__ dq_part, int B, int
                                   int chunks, const int2* __restrict__ heads, bool shared_q,
                                   const __nv_bfloat16* __restrict__ extra,
                                   __nv_bfloat16* __restrict__ dQ, float4* __restrict__ dQ32) {
+  pdl_wait();   // the previous kernel's results (programmatic dependent launch)
+  pdl_trigger();
   const int64_t md4 = (int64_t)M * D / 4;
   const int64_t per4 = (int64_t)H * md4;
   const int64_t total4 = shared_q ? per4 : (int64_t)B * per4;
@@ -1685,6 +1697,8 @@ __global__ void bwd_dq_sum_kernel(const float4* __restrict__ dq_part, int B, int
 __global__ void bwd_dz_sum_kernel(const float4* __restrict__ dz_part, int64_t BH, int M, int D,
                                   int chunks, const int2* __restrict__ heads,
                                   float4* __restrict__ dz) {
+  pdl_wait();   // the previous kernel's results (programmatic dependent launch)
+  pdl_trigger();
   const int64_t md4 = (int64_t)M * D / 4;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= BH * md4) return;
@@ -1782,11 +1796,10 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
   }
 
   // dZ: the chunk partials, or (FINISH) the sum over the shards as one partial
-  bwd_mid_kernel<D, M><<<(unsigned)BH, M, 0, st>>>(phase == BwdPhase::FINISH ? dz_io : dzp,
-                                                   phase == BwdPhase::FINISH ? 1 : zchunks,
-                                                   phase == BwdPhase::FINISH ? nullptr : zheads,
-                                                   nullptr,
-                                                   Z, lse, dzs, (uint32_t*)aug, flags, params, lse2);
+  const bool fin = phase == BwdPhase::FINISH;
+  bwd_mid_kernel<D, M><<<(unsigned)BH, M, 0, st>>>(fin ? dz_io : dzp, fin ? 1 : zchunks,
+                                                   fin ? nullptr : zheads, nullptr, Z, lse, dzs,
+                                                   (uint32_t*)aug, flags, params, lse2);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
   // each head runs in exactly one of the two pass-B kernels (params.y)
