@@ -264,6 +264,12 @@ def roofline_entry(kernel_ms: dict, peaks: dict, peak_kind: str, rates: dict, w=
     hbm_bytes = 2 * w.B * w.H * w.N * w.D * 2   # encode: K and V read; decode: K read, Y written
     t_fwd = sum(kernel_ms.values()) / 1e3
     t_fwd_ceil = sum(c["t_ceiling_ms"] for c in ceil.values()) / 1e3
+    # context: the share at which the two units bind together, whose floor no
+    # split of the exponentials between them can beat
+    mufu_r = rates["ex2_per_clk_sm"]
+    fma_r = max(rates["fma_per_clk_sm"], rates["fma2_per_clk_sm"])
+    phi_b = (fma_r - FMA_OPS_BASE * mufu_r) / (fma_r + FMA_OPS_POLY * mufu_r)
+    t_b, _ = exp_ceiling(exps, phi_b, rates, clk)
     entry = {
         "bound": "alu", "kernel": f"flare_{name}", "achieved": round(achieved, 1),
         "peak": peak, "unit": "Gexp/s", "frac": round(achieved / peak, 4),
@@ -275,6 +281,9 @@ def roofline_entry(kernel_ms: dict, peaks: dict, peak_kind: str, rates: dict, w=
                        f"{max(rates['fma_per_clk_sm'], rates['fma2_per_clk_sm']):.1f}/clk/SM "
                        f"({rates['source']}) x {rates['sms']} SMs x {clk / 1e6:.0f} MHz"),
         "mufu_only": {"peak": round(mufu_peak, 1), "frac": round(achieved / mufu_peak, 4)},
+        "best_split": {"poly_share": round(phi_b, 4), "t_ceiling_ms": round(t_b * 1e3, 4),
+                       "frac": round(t_b / t, 4),
+                       "forward_frac": round(2 * t_b / t_fwd, 4)},
         "kernels": ceil,
         "forward": {"t_ms": round(t_fwd * 1e3, 4), "t_ceiling_ms": round(t_fwd_ceil * 1e3, 4),
                     "frac": round(t_fwd_ceil / t_fwd, 4)},

@@ -109,29 +109,34 @@ inline Path choose_path(int64_t N, int64_t M, int64_t D, flare_dtype_t dt) {
 }
 
 // Split of the forward's exponentials between the MUFU (ex2.approx) and the
-// FMA-pipe polynomial: in the tensor-core encode, every kEncPolyEvery-th
-// pair of each 48-logit row tile's first 32 logits and every
-// kEncPolyEvery16-th pair of its last 16 runs as the polynomial (0 = none);
-// in the decode, every kDecPolyEvery-th pair of each 32-logit chunk.
+// FMA-pipe polynomial, per latent tile (128 or 256 rows): in the
+// tensor-core encode, every enc_poly_every32-th pair of each 48-logit row
+// tile's first 32 logits and every enc_poly_every16-th pair of its last 16
+// runs as the polynomial (0 = none); in the decode, every dec_poly_every-th
+// pair of each 32-logit chunk.  Measured on the 256-row tile at one million
+// tokens, and on the 128-row tile at 16K-65K tokens (where the larger shares
+// measured slower).
 #ifndef FLARE_ENC_POLY32
-#define FLARE_ENC_POLY32 4
+#define FLARE_ENC_POLY32 3
 #endif
 #ifndef FLARE_ENC_POLY16
-#define FLARE_ENC_POLY16 4
+#define FLARE_ENC_POLY16 3
 #endif
 #ifndef FLARE_DEC_POLY
-#define FLARE_DEC_POLY 16
+#define FLARE_DEC_POLY 8
 #endif
-constexpr int kEncPolyEvery = FLARE_ENC_POLY32;
-constexpr int kEncPolyEvery16 = FLARE_ENC_POLY16;
-constexpr int kDecPolyEvery = FLARE_DEC_POLY;
+constexpr int enc_poly_every32(int Mp) { return Mp == 256 ? FLARE_ENC_POLY32 : 4; }
+constexpr int enc_poly_every16(int Mp) { return Mp == 256 ? FLARE_ENC_POLY16 : 4; }
+constexpr int dec_poly_every(int Mp) { return Mp == 256 ? FLARE_DEC_POLY : 16; }
 
 // Share of a tensor-core kernel's exponentials computed by the polynomial.
-constexpr double enc_poly_fraction() {
-  return ((kEncPolyEvery > 0 ? 16 / kEncPolyEvery : 0) +
-          (kEncPolyEvery16 > 0 ? 8 / kEncPolyEvery16 : 0)) / 24.0;
+constexpr double enc_poly_fraction(int Mp) {
+  return ((enc_poly_every32(Mp) > 0 ? 16 / enc_poly_every32(Mp) : 0) +
+          (enc_poly_every16(Mp) > 0 ? 8 / enc_poly_every16(Mp) : 0)) / 24.0;
 }
-constexpr double dec_poly_fraction() { return (kDecPolyEvery > 0 ? 16 / kDecPolyEvery : 0) / 16.0; }
+constexpr double dec_poly_fraction(int Mp) {
+  return (dec_poly_every(Mp) > 0 ? 16 / dec_poly_every(Mp) : 0) / 16.0;
+}
 
 constexpr int kSimtEncTile = 64;
 constexpr int kSimtEncThreads = 256;

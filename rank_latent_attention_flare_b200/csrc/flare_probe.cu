@@ -348,8 +348,10 @@ extern "C" flare_status_t flare_exp_split(int kernel, int64_t M, int64_t D, flar
       (dtype != FLARE_F32 && dtype != FLARE_BF16))
     return FLARE_ERR_UNSUPPORTED;
   const flare::Path p = flare::choose_path(1, M, D, dtype);
-  *poly_fraction =
-      !p.tc_fwd ? 0.0 : (kernel == 0 ? flare::enc_poly_fraction() : flare::dec_poly_fraction());
+  const int Mp = flare::tc_latent_tile(M);
+  *poly_fraction = !p.tc_fwd ? 0.0
+                             : (kernel == 0 ? flare::enc_poly_fraction(Mp)
+                                            : flare::dec_poly_fraction(Mp));
   return FLARE_OK;
 }
 

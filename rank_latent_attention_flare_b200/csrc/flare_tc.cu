@@ -67,12 +67,15 @@ constexpr float kRedoTau = 64.0f;     // log2 units: past 2^64 above m_ref a til
 constexpr float kRescaleLimit = 256.0f;                  // 2^kRescaleTau
 constexpr float kRedoLimit = 18446744073709551616.0f;   // 2^kRedoTau
 // Every k-th pair of exponentials is computed on the FMA pipe (exp2_fma)
-// instead of the MUFU, which is the unit that bounds both kernels.  The
-// encode (four softmax warps per SM sub-partition) gains from moving every
-// fourth pair (1.44 -> 1.36 ms on the million-token workload); the decode
-// (two per sub-partition, close to its register budget) gains only from the
-// last pair of each 32-column chunk (1.40 -> 1.38 ms; every 4th, 8th, 10th
-// or 12th pair is slower).
+// instead of the MUFU, which is the unit that bounds both kernels.  On the
+// million-token workload the encode (four softmax warps per SM
+// sub-partition) is fastest with every third pair (5 of 16 and 2 of 8 per
+// 48-logit row tile: 1.23 -> 1.21 ms against every fourth; every second is
+// 1.37 ms), the decode with every eighth pair of each 32-logit chunk (1.19 ->
+// 1.16 ms against the last pair only, once its row sums came from Y's
+// product and freed FMA-pipe issue slots; every fifth or fourth pair measured
+// the same within noise, and fewer polynomials keep more weights at the
+// MUFU's accuracy).
 // Decode reference of a token row (M = 256): the max of the first 32-logit
 // chunk read, used when c |k| max_m |q_m| (Cauchy-Schwarz: at least every
 // logit) lies at most this far (log2 units) above it, so no weight exceeds
@@ -430,14 +433,14 @@ __global__ void __launch_bounds__(kThreads, 2)
           uint32_t a[32], pk[16];
           tmem_ld32(tS, a);
           tmem_wait_ld_dep(a);
-          exp_bias_pairs<16, kEncPolyEvery>(a, c, nb, pk);
+          exp_bias_pairs<16, enc_poly_every32(M)>(a, c, nb, pk);
           tmem_st16(tS, pk);
         }
         {
           uint32_t a[16], pk[8];
           tmem_ld16(tS + 32, a);
           tmem_wait_ld_dep16(a);
-          exp_bias_pairs<8, kEncPolyEvery16>(a, c, nb + 32, pk);
+          exp_bias_pairs<8, enc_poly_every16(M)>(a, c, nb + 32, pk);
           tmem_st8(tS + 16, pk);
         }
         tmem_wait_st();
@@ -475,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int t = 0; t < 32; ++t)
               if (t < lo || t >= hi) a[t] = __float_as_uint(-INFINITY);
           }
-          exp_pack32<kEncPolyEvery, true>(a, c, neg, pa, sf);
+          exp_pack32<enc_poly_every32(M), true>(a, c, neg, pa, sf);
         }
         {
           uint32_t a[16];
@@ -486,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int t = 0; t < 16; ++t)
               if (32 + t < lo || 32 + t >= hi) a[t] = __float_as_uint(-INFINITY);
           }
-          exp_pack16<kEncPolyEvery16, true>(a, c, neg, pb, sf);
+          exp_pack16<enc_poly_every16(M), true>(a, c, neg, pb, sf);
         }
         const float sum = (sf[0] + sf[1]) + (sf[2] + sf[3]);
         // Every weight of the tile is at most the tile's row sum, so the sum
@@ -560,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 2)
               if (t < lo || t >= hi) a[t] = __float_as_uint(-INFINITY);
           }
           uint32_t pk[16];
-          exp_pack32<kEncPolyEvery, true>(a, c, neg, pk, sf);
+          exp_pack32<enc_poly_every32(M), true>(a, c, neg, pk, sf);
           tmem_st16(tS, pk);
         }
         {
@@ -573,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 2)
               if (32 + t < lo || 32 + t >= hi) a[t] = __float_as_uint(-INFINITY);
           }
           uint32_t pk[8];
-          exp_pack16<kEncPolyEvery16, true>(a, c, neg, pk, sf);
+          exp_pack16<enc_poly_every16(M), true>(a, c, neg, pk, sf);
           tmem_st8(tS + 16, pk);
         }
         l += (sf[0] + sf[1]) + (sf[2] + sf[3]);
@@ -1001,7 +1004,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t a[32], pk[16];
             tmem_ld32(tR + col, a);
             tmem_wait_ld_dep(a);
-            exp_pack32<kDecPolyEvery, false, false>(a, c, neg, pk, sf);
+            exp_pack32<dec_poly_every(M), false, false>(a, c, neg, pk, sf);
             tmem_st16(tR + p_col(k), pk);
           } else {
             uint32_t a[16], pk[8];
@@ -1050,7 +1053,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (k > 0 || !kBound) tmem_wait_ld_dep(a[k & 1]);
           if (k + 1 < NC) tmem_ld32(tR + chunk_col(k + 1), a[(k + 1) & 1]);
           uint32_t pk[16];
-          exp_pack32<kDecPolyEvery, false, false>(a[k & 1], c, neg, pk, sf);
+          exp_pack32<dec_poly_every(M), false, false>(a[k & 1], c, neg, pk, sf);
           tmem_st16(tR + p_col(k), pk);
           if (k == NC / 2 - 1 || (NC == 8 && k == 5)) {
             tmem_wait_st();
