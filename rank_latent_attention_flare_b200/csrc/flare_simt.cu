@@ -175,19 +175,44 @@ __global__ void combine_kernel(const float* __restrict__ part_ml,
     cnt = hs.y * sub;
   }
   const int64_t gstride = BH * slots;
+  // lane s reads record s of each run of 32: the loads of a run are in
+  // flight together
   float mstar = -INFINITY;
   for (int g = 0; g < groups; ++g)
-    for (int s = 0; s < cnt; ++s)
-      mstar = fmaxf(mstar, part_ml[((g * gstride + r0 + s) * M + m) * 2]);
+    for (int s0 = 0; s0 < cnt; s0 += 32)
+      if (s0 + lane < cnt)
+        mstar = fmaxf(mstar, part_ml[((g * gstride + r0 + s0 + lane) * M + m) * 2]);
+  for (int o = 16; o > 0; o >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, o));
+  // then, record by record in order, l += f l_s and (lane d) acc += f acc_s[d]
   float l = 0.f, acc = 0.f;
   for (int g = 0; g < groups; ++g)
-    for (int s = 0; s < cnt; ++s) {
-      const int64_t row = (g * gstride + r0 + s) * M + m;
-      const float ms = part_ml[row * 2];
-      if (ms == -INFINITY) continue;  // empty record
-      const float f = exp2f(ms - mstar);
-      l = fmaf(f, part_ml[row * 2 + 1], l);
-      if (lane < D) acc = fmaf(f, part_acc[row * D + lane], acc);
+    for (int s0 = 0; s0 < cnt; s0 += 32) {
+      const int n = min(32, cnt - s0);   // warp-uniform
+      float ms = -INFINITY, ls = 0.f;
+      if (lane < n) {
+        const int64_t row = (g * gstride + r0 + s0 + lane) * M + m;
+        ms = part_ml[row * 2];
+        ls = part_ml[row * 2 + 1];
+      }
+      const float f = (ms == -INFINITY) ? 0.f : exp2f(ms - mstar);   // an empty record: none
+      for (int u0 = 0; u0 < n; u0 += 8) {
+        float a[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          a[u] = (u0 + u < n && lane < D)
+                     ? part_acc[((g * gstride + r0 + s0 + u0 + u) * M + m) * D + lane]
+                     : 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (u0 + u >= n) break;
+          const float mu = __shfl_sync(0xffffffffu, ms, u0 + u);
+          const float fu = __shfl_sync(0xffffffffu, f, u0 + u);
+          const float lu = __shfl_sync(0xffffffffu, ls, u0 + u);
+          if (mu == -INFINITY) continue;
+          l = fmaf(fu, lu, l);
+          acc = fmaf(fu, a[u], acc);
+        }
+      }
     }
   if (lane < D) {
     const float z = (l > 0.f) ? acc / l : 0.f;   // no tokens: an empty weighted sum
