@@ -458,6 +458,25 @@ FLARE_API flare_status_t flare_probe_unit_rates(void* scratch, size_t scratch_by
                                                 flare_unit_rates_t* out, void* stream);
 
 /*
+ * SM clocks one tcgen05.mma of the kernels' shapes (kind::f16, bf16
+ * operands, fp32 accumulator, M = 128, K = 16, N = n in {32, 48, 64, 128,
+ * 256}) costs when `issuers` (1 to 4) threads of every SM issue 1024 of them
+ * each, back to back, with the A operand in shared memory (a_in_tmem = 0) or
+ * in TMEM (1): the median over the SMs of the slowest issuer's span divided
+ * by all the SM's products.  With one issuer this is the issue latency of a
+ * thread; with several, the SM's own cost of a product.  scratch: device
+ * memory of at least flare_probe_scratch_bytes() bytes, 16-byte aligned.
+ * Runs on `stream` and SYNCHRONISES it.  Returns FLARE_OK,
+ * FLARE_ERR_INVALID_ARG (NULL pointer, issuers outside [1, 4]),
+ * FLARE_ERR_UNSUPPORTED (another n, or n x issuers > 256),
+ * FLARE_ERR_WORKSPACE, FLARE_ERR_DEVICE_TIMEOUT (a bounded wait ran out) or
+ * FLARE_ERR_CUDA.
+ */
+FLARE_API flare_status_t flare_probe_mma_rate(int n, int a_in_tmem, int issuers, void* scratch,
+                                              size_t scratch_bytes, double* clk_per_mma,
+                                              void* stream);
+
+/*
  * Share of the exponentials of the forward's encode (kernel 0) or decode
  * (kernel 1) that runs as the FMA-pipe polynomial instead of the MUFU, for
  * a forward call with these M, D and dtype (0 for the CUDA-core kernels,

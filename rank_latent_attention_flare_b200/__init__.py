@@ -12,7 +12,7 @@ from .flare import (alloc_workspace, bwd_path, default_scale, device_status, enc
                     flare_bwd, flare_bwd_shard_dz, flare_bwd_shard_finish, flare_combine,
                     flare_combine_shards, flare_decode, flare_encode, flare_fwd, flare_fwd_noalloc,
                     flare_pp_bwd, flare_pp_bwd_shard_tail, flare_pp_fwd, fwd_path, records_layout,
-                    workspace_size, noalloc_device_status, probe_unit_rates, eval_exp2,
+                    workspace_size, noalloc_device_status, probe_unit_rates, probe_mma_rates, eval_exp2,
                     selftest_wait_timeout, exp_split)
 from . import parallel
 
@@ -26,5 +26,5 @@ __all__ = [
     "FlareFunction", "FlarePPFunction", "flare", "flare_pp",
     "encode_records", "flare_bwd_shard_dz", "flare_bwd_shard_finish", "flare_combine_shards",
     "records_layout", "parallel", "flare_pp_bwd_shard_tail", "noalloc_device_status",
-    "probe_unit_rates", "eval_exp2", "selftest_wait_timeout", "exp_split",
+    "probe_unit_rates", "probe_mma_rates", "eval_exp2", "selftest_wait_timeout", "exp_split",
 ]

@@ -105,6 +105,8 @@ SIGNATURES = {
     "flare_probe_unit_rates": (_i32, [_vp, _sz, ctypes.POINTER(UnitRates), _vp]),
     "flare_eval_exp2": (_i32, [_vp, _vp, _i64, _i32, _vp]),
     "flare_exp_split": (_i32, [_i32, _i64, _i64, _i32, ctypes.POINTER(ctypes.c_double)]),
+    "flare_probe_mma_rate": (_i32, [_i32, _i32, _i32, _vp, _sz, ctypes.POINTER(ctypes.c_double),
+                                    _vp]),
     "flare_selftest_wait_timeout": (_i32, [_vp, _sz, ctypes.c_uint64, _vp]),
 }
 

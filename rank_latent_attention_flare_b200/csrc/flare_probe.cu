@@ -8,6 +8,12 @@
 // the launch, with the SM clock read inside the kernels (clock64 against the
 // global nanosecond timer) so that every rate is also given per clock.
 //
+// flare_probe_mma_rate: the time a tcgen05.mma of the kernels' shapes
+// (kind::f16, M = 128, K = 16, N tokens or latents) takes an SM, with its
+// A operand in shared memory or in TMEM and one to four threads of the SM
+// issuing at once, so that the cost of a product can be told apart from the
+// issue latency of one thread.
+//
 // flare_eval_exp2: the kernels' exponentials (the MUFU one and the
 // FMA-pipe polynomial, scalar and packed) evaluated element by element, so
 // that a test can hold them against their stated error bounds.
@@ -20,6 +26,7 @@
 // reports FLARE_ERR_DEVICE_TIMEOUT with the device still usable.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <vector>
 
 #include "flare_internal.cuh"
@@ -258,10 +265,123 @@ int sm_count() {
   return sms;
 }
 
+// One CTA per SM (its shared memory keeps a second one out); warps 0 ..
+// issuers - 1 each issue `reps` products of N columns into their own TMEM
+// columns (A from TMEM: its own 8 columns from column 256) on zeroed
+// operands, then wait for them to complete (bounded).  Each issuer records
+// its clocks from the first issue to the completion.
+struct MmaRec {
+  unsigned long long clk;
+  unsigned ok, pad;
+};
+
+template <int N, bool TS>
+__global__ void __launch_bounds__(128, 1) probe_mma_kernel(int reps, int issuers, MmaRec* out) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  __shared__ __align__(8) uint64_t bar[4];
+  __shared__ uint32_t slot;
+  // A: 128 rows x 64 bytes, B: up to 256 rows x 64 bytes, all zero
+  for (int i = threadIdx.x; i < (128 + 256) * 64 / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(sm)[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < 4; ++k) mbar_init(&bar[k], 1);
+    fence_mbar_init();
+  }
+  if (threadIdx.x < 32) tmem_alloc(&slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = slot;
+  const int w = threadIdx.x >> 5;
+  if (w < issuers && (threadIdx.x & 31) == 0) {
+    const uint64_t da = smem_desc(smem_u32(sm), 16, 8 * 64, umma_swizzle_code(64));
+    const uint64_t db = smem_desc(smem_u32(sm + 128 * 64), 16, 8 * 64, umma_swizzle_code(64));
+    constexpr uint32_t id = idesc_bf16_f32(128, N, 0, 0);
+    const unsigned long long t0 = clock64();
+    for (int i = 0; i < reps; ++i) {
+      if (TS)
+        mma_ts(tmem + N * w, tmem + 256 + 8 * w, db, id, 1u);
+      else
+        mma_ss(tmem + N * w, da, db, id, i > 0 ? 1u : 0u);
+    }
+    mma_commit(&bar[w]);
+    const bool ok = mbar_wait(&bar[w], 0);
+    out[blockIdx.x * 4 + w] = MmaRec{clock64() - t0, ok ? 1u : 0u, 0u};
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x < 32) tmem_dealloc(tmem, 512);
+}
+
+template <int N, bool TS>
+cudaError_t launch_probe_mma(int sms, int reps, int issuers, MmaRec* out, cudaStream_t st) {
+  const int smem = 120 * 1024;   // one CTA per SM
+  cudaError_t e =
+      cudaFuncSetAttribute(probe_mma_kernel<N, TS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  probe_mma_kernel<N, TS><<<sms, 128, smem, st>>>(reps, issuers, out);
+  return cudaPeekAtLastError();
+}
+
 }  // namespace
 }  // namespace flare
 
 using flare::ClockRec;
+
+extern "C" flare_status_t flare_probe_mma_rate(int n, int a_in_tmem, int issuers, void* scratch,
+                                               size_t scratch_bytes, double* clk_per_mma,
+                                               void* stream) {
+  using namespace flare;
+  if (clk_per_mma == nullptr || scratch == nullptr) return FLARE_ERR_INVALID_ARG;
+  if (issuers < 1 || issuers > 4) return FLARE_ERR_INVALID_ARG;
+  if (n != 32 && n != 48 && n != 64 && n != 128 && n != 256) return FLARE_ERR_UNSUPPORTED;
+  if (n * issuers > 256) return FLARE_ERR_UNSUPPORTED;   // each issuer's TMEM columns
+  const int sms = sm_count();
+  if (sms <= 0) return FLARE_ERR_CUDA;
+  if (scratch_bytes < (size_t)sms * 4 * sizeof(MmaRec) || ((uintptr_t)scratch & 15u))
+    return FLARE_ERR_WORKSPACE;
+  MmaRec* rec = (MmaRec*)scratch;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int reps = 1024;
+  cudaError_t e = cudaSuccess;
+  // one untimed launch (code load, clocks), then the measured one
+  for (int rep = 0; rep < 2 && e == cudaSuccess; ++rep) {
+#define FLARE_PROBE_MMA(NN)                                                          \
+  e = a_in_tmem ? launch_probe_mma<NN, true>(sms, reps, issuers, rec, st)            \
+                : launch_probe_mma<NN, false>(sms, reps, issuers, rec, st)
+    if (n == 32) FLARE_PROBE_MMA(32);
+    else if (n == 48) FLARE_PROBE_MMA(48);
+    else if (n == 64) FLARE_PROBE_MMA(64);
+    else if (n == 128) FLARE_PROBE_MMA(128);
+    else FLARE_PROBE_MMA(256);
+#undef FLARE_PROBE_MMA
+  }
+  std::vector<MmaRec> host((size_t)sms * 4);
+  if (e != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess ||
+      cudaMemcpy(host.data(), rec, host.size() * sizeof(MmaRec), cudaMemcpyDeviceToHost) !=
+          cudaSuccess) {
+    note_error("flare_probe_mma_rate: probe kernel failed (%s)", cudaGetErrorName(cudaGetLastError()));
+    return FLARE_ERR_CUDA;
+  }
+  // per SM: the issuers' products share it, so its clocks per product are
+  // the slowest issuer's span over all of them; the median over the SMs
+  std::vector<double> per_sm;
+  for (int b = 0; b < sms; ++b) {
+    unsigned long long span = 0;
+    for (int w = 0; w < issuers; ++w) {
+      const MmaRec& r = host[(size_t)b * 4 + w];
+      if (!r.ok) return FLARE_ERR_DEVICE_TIMEOUT;
+      span = r.clk > span ? r.clk : span;
+    }
+    per_sm.push_back((double)span / ((double)reps * issuers));
+  }
+  std::sort(per_sm.begin(), per_sm.end());
+  *clk_per_mma = per_sm[per_sm.size() / 2];
+  return FLARE_OK;
+}
 
 extern "C" size_t flare_probe_scratch_bytes(void) {
   const int sms = flare::sm_count();

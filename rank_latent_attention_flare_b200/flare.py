@@ -358,6 +358,30 @@ def probe_unit_rates(device=None, stream=None) -> dict:
     return {name: getattr(out, name) for name, _ in _lib.UnitRates._fields_}
 
 
+def probe_mma_rates(cases=None, device=None, stream=None) -> dict:
+    """SM clocks per tcgen05.mma of the kernels' shapes (flare_probe_mma_rate)
+    for each (n, a_in_tmem, issuers) case: with one issuer the issue latency
+    of a thread, with several the SM's own cost of a product.  Synchronises
+    the device."""
+    lib = _lib.load()
+    nbytes = int(lib.flare_probe_scratch_bytes())
+    if nbytes == 0:
+        raise RuntimeError("flare_probe_scratch_bytes: no CUDA device")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    scratch = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    if cases is None:
+        cases = [(n, t, i) for t in (0, 1) for n in (32, 48) for i in (1, 4)] + \
+                [(128, 0, 1), (256, 0, 1)]
+    out = {}
+    for n, tm, iss in cases:
+        v = ctypes.c_double(0.0)
+        _lib.check(lib.flare_probe_mma_rate(int(n), int(tm), int(iss), _ptr(scratch), nbytes,
+                                            ctypes.byref(v), _stream(stream)),
+                   "flare_probe_mma_rate")
+        out[f"{'ts' if tm else 'ss'}_n{n}_x{iss}"] = float(v.value)
+    return out
+
+
 def exp_split(kernel: int, M: int, D: int, dtype: torch.dtype) -> float:
     """Share of the forward encode's (kernel 0) or decode's (kernel 1)
     exponentials computed by the FMA-pipe polynomial (flare_exp_split)."""

@@ -31,6 +31,24 @@ def test_probe_unit_rates_are_plausible():
     assert 4.0 < r["mix_ex2_per_clk_sm"] < 40.0, r
 
 
+def test_probe_mma_rates_are_plausible():
+    # The tensor core's math alone takes 2 M N K / 8192 clocks per product
+    # at B200's dense bf16 rate (~8K flops / clk / SM), so no product is
+    # cheaper than that; a product of N = 256 is math-bound, and an A operand
+    # read from shared memory (4 KB) costs at least 4096 / 128 = 32 clocks
+    # of the shared-memory port once several threads keep the SM busy.
+    r = fl.probe_mma_rates()
+    for k, v in r.items():
+        assert 1.0 < v < 1000.0, (k, v)
+    assert r["ss_n256_x1"] >= 0.9 * 2 * 128 * 256 * 16 / 8192, r
+    assert r["ss_n32_x4"] >= 0.9 * 4096 / 128, r
+    # with A in TMEM, four issuers get more products per clock than with A
+    # in shared memory
+    assert r["ts_n32_x4"] < r["ss_n32_x4"], r
+    with pytest.raises(fl.FlareError):   # 4 issuers x 128 columns do not fit
+        fl.probe_mma_rates(cases=[(128, 0, 4)])
+
+
 def _grid():
     xs = [np.linspace(-130.0, 126.0, 1 << 20)]
     k = np.arange(-130, 127, dtype=np.float64)
