@@ -387,19 +387,25 @@ def run_ours(args, rank, world, local):
     value = world * tokens_per_step * args.steps / (ms_total / 1e3)
 
     # End to end through the public API: pinned host inputs -> device ->
-    # flare_fwd -> result back to pinned host memory, every step.
+    # forward -> result back to pinned host memory, every step, by the
+    # library's host-memory call (flare_fwd_host: the heads' copies in on a
+    # second stream, overlapped with the compute and the copies out).
     e2e = None
     if not args.no_e2e:
         hx = {k: v.pin_memory() for k, v in x.items()}
         hY = torch.empty(Y.shape, dtype=Y.dtype, pin_memory=True)
         dX = {k: torch.empty_like(v) for k, v in g.items()}
+        bufs = {"Q": dX["Q"], "K": dX["K"], "V": dX["V"], "Y": Y}
+        wsh = torch.empty(int(fl.load().flare_fwd_host_workspace_size(
+            w.B, w.H, w.N, w.M, w.D,
+            fl.FLARE_BF16 if w.torch_dtype == torch.bfloat16 else fl.FLARE_F32)),
+            dtype=torch.uint8, device=dev)
+        copy_stream = torch.cuda.Stream(device=dev)
         e2e_steps = max(1, min(args.steps, args.e2e_steps))
 
         def e2e_step():
-            for k in ("Q", "K", "V"):
-                dX[k].copy_(hx[k], non_blocking=True)
-            fl.flare_fwd(dX["Q"], dX["K"], dX["V"], w.scale, workspace=ws, out=Y)
-            hY.copy_(Y, non_blocking=True)
+            fl.flare_fwd_host(hx["Q"], hx["K"], hx["V"], w.scale, out=hY, device_buffers=bufs,
+                              workspace=wsh, device=dev, stream=st, copy_stream=copy_stream)
 
         e2e_step()
         torch.cuda.synchronize()

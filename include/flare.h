@@ -34,7 +34,8 @@
  *     and > 0.
  *   - The caller owns every buffer.  The library never allocates or frees
  *     memory and never synchronises the device (flare_device_status is the
- *     one exception and says so).  Work is enqueued on `stream` (a
+ *     one exception and says so; flare_fwd_host creates and releases CUDA
+ *     events to order its two streams).  Work is enqueued on `stream` (a
  *     cudaStream_t; NULL = legacy default stream).
  *   - `workspace` is caller-allocated device memory of at least
  *     flare_workspace_size(op, ...) bytes, 256-byte aligned.  Its contents
@@ -126,6 +127,33 @@ FLARE_API const char* flare_status_string(flare_status_t status);
  */
 FLARE_API size_t flare_workspace_size(flare_op_t op, int64_t B, int64_t H, int64_t N, int64_t M,
                             int64_t D, flare_dtype_t dtype);
+
+/*
+ * FLARE forward from and to HOST memory: Q, K, V are copied in and Y is
+ * copied out by the library, overlapped with the compute.  The heads go in
+ * about 16 chunks (each inside one batch element): a chunk's K and V are
+ * copied in on `copy_stream` while `stream` runs the previous chunk's
+ * forward and copies its Y out, so the call takes about as long as its
+ * host-to-device copies.  Q_host / K_host / V_host / Y_host: host memory
+ * (page-locked for the copies to overlap), laid out as flare_fwd's device
+ * tensors; Q_dev, K_dev, V_dev, Y_dev: caller-owned device buffers of the
+ * same sizes, overwritten.  workspace: flare_fwd_host_workspace_size bytes.
+ * Everything is ordered after the work already on `stream`, and the call's
+ * results (Y_host) are complete once `stream` is: synchronise `stream`
+ * before reading Y_host.  copy_stream may equal stream (no overlap).
+ * Returns the codes of flare_fwd; the device error word is read with
+ * flare_device_status on the workspace.
+ */
+FLARE_API flare_status_t flare_fwd_host(const void* Q_host, int64_t q_batch_stride,
+                                        const void* K_host, const void* V_host, void* Y_host,
+                                        void* Q_dev, void* K_dev, void* V_dev, void* Y_dev,
+                                        int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
+                                        flare_dtype_t dtype, float scale, void* workspace,
+                                        size_t workspace_bytes, void* stream, void* copy_stream);
+
+/* Bytes of workspace flare_fwd_host needs (0 for invalid sizes). */
+FLARE_API size_t flare_fwd_host_workspace_size(int64_t B, int64_t H, int64_t N, int64_t M,
+                                               int64_t D, flare_dtype_t dtype);
 
 /*
  * FLARE forward: Y = decode(Q, K, encode(Q, K, V)).

@@ -69,6 +69,9 @@ SIGNATURES = {
                          _vp, _vp, _vp, _sz, _vp]),
     "flare_pp_fwd": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i32, _f32,
                             _vp, _vp, _vp, _sz, _vp]),
+    "flare_fwd_host": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
+                              _i64, _i32, _f32, _vp, _sz, _vp, _vp]),
+    "flare_fwd_host_workspace_size": (_sz, [_i64, _i64, _i64, _i64, _i64, _i32]),
     "flare_bwd": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
                          _i64, _i64, _i32, _f32, _vp, _sz, _vp]),
     "flare_pp_bwd": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,

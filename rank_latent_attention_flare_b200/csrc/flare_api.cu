@@ -455,6 +455,107 @@ flare_status_t flare_fwd(const void* Q, int64_t qbs, const void* K, const void* 
                            workspace, workspace_bytes, stream);
 }
 
+// ------------------------------------------------- forward from host memory
+
+}  // extern "C"
+
+namespace {
+
+// Heads per chunk of flare_fwd_host: about 16 chunks, each inside one
+// batch element.
+int64_t host_chunk_heads(int64_t B, int64_t H) {
+  const int64_t hc = (B * H + 15) / 16;
+  return hc < 1 ? 1 : (hc > H ? H : hc);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t flare_fwd_host_workspace_size(int64_t B, int64_t H, int64_t N, int64_t M, int64_t D,
+                                     flare_dtype_t dt) {
+  if (check_sizes(B, H, N, M, D, dt) != FLARE_OK) return 0;
+  return ws_layout(FLARE_OP_FWD, 1, host_chunk_heads(B, H), N, M, D, dt, current_sm_count()).total;
+}
+
+flare_status_t flare_fwd_host(const void* Q_host, int64_t qbs, const void* K_host,
+                              const void* V_host, void* Y_host, void* Q_dev, void* K_dev,
+                              void* V_dev, void* Y_dev, int64_t B, int64_t H, int64_t N, int64_t M,
+                              int64_t D, flare_dtype_t dt, float scale, void* workspace,
+                              size_t workspace_bytes, void* stream, void* copy_stream) {
+  FLARE_TRY(check_sizes(B, H, N, M, D, dt));
+  FLARE_TRY(check_scale(scale));
+  FLARE_TRY(check_qbs(qbs, H, M, D));
+  if (!Q_host || !K_host || !V_host || !Y_host) return FLARE_ERR_INVALID_ARG;
+  FLARE_TRY(check_ptr(Q_dev));
+  FLARE_TRY(check_ptr(K_dev));
+  FLARE_TRY(check_ptr(V_dev));
+  FLARE_TRY(check_ptr(Y_dev));
+  const int sms = current_sm_count();
+  const int64_t hc = host_chunk_heads(B, H);
+  const WsLayout L = ws_layout(FLARE_OP_FWD, 1, hc, N, M, D, dt, sms);
+  FLARE_TRY(check_ws(workspace, workspace_bytes, L.total));
+  char* ws = (char*)workspace;
+  cudaStream_t st = (cudaStream_t)stream, cs = (cudaStream_t)copy_stream;
+  const int64_t esz = (dt == FLARE_F32) ? 4 : 2;
+  const int64_t head_bytes = N * D * esz, lat_bytes = M * D * esz;
+  // the copies start after the work already queued on `stream` (which may
+  // still use the device buffers)
+  cudaEvent_t start = nullptr;
+  FLARE_CUDA(cudaEventCreateWithFlags(&start, cudaEventDisableTiming));
+  flare_status_t status = FLARE_OK;
+  auto fail = [&](cudaError_t e, const char* what) {
+    note_error("flare_fwd_host: %s (%s)", what, cudaGetErrorName(e));
+    status = FLARE_ERR_CUDA;
+  };
+  cudaError_t e;
+  if ((e = cudaEventRecord(start, st)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(cs, start, 0)) != cudaSuccess)
+    fail(e, "stream ordering");
+  if (status == FLARE_OK &&
+      (e = cudaMemcpyAsync(Q_dev, Q_host, (qbs ? B * H : H) * lat_bytes, cudaMemcpyHostToDevice,
+                           cs)) != cudaSuccess)
+    fail(e, "Q copy");
+  if (status == FLARE_OK) status = reset_error_word(ws, st);
+  // chunk k: heads [h0, h1) of batch element b.  Its K and V go in on the
+  // copy stream; `stream` waits for them, runs the forward on the chunk (B =
+  // 1, shared latents at the chunk's offset) and copies its Y out, while
+  // the copy stream already brings in the next chunk.
+  for (int64_t b = 0; b < B && status == FLARE_OK; ++b) {
+    for (int64_t h0 = 0; h0 < H && status == FLARE_OK; h0 += hc) {
+      const int64_t h1 = (h0 + hc < H) ? h0 + hc : H;
+      const int64_t off = (b * H + h0) * head_bytes, bytes = (h1 - h0) * head_bytes;
+      cudaEvent_t in = nullptr;
+      if ((e = cudaEventCreateWithFlags(&in, cudaEventDisableTiming)) != cudaSuccess) {
+        fail(e, "event");
+        break;
+      }
+      if ((e = cudaMemcpyAsync((char*)K_dev + off, (const char*)K_host + off, bytes,
+                               cudaMemcpyHostToDevice, cs)) != cudaSuccess ||
+          (e = cudaMemcpyAsync((char*)V_dev + off, (const char*)V_host + off, bytes,
+                               cudaMemcpyHostToDevice, cs)) != cudaSuccess ||
+          (e = cudaEventRecord(in, cs)) != cudaSuccess ||
+          (e = cudaStreamWaitEvent(st, in, 0)) != cudaSuccess)
+        fail(e, "K / V copy");
+      cudaEventDestroy(in);   // released once recorded work completes
+      if (status != FLARE_OK) break;
+      const char* Qc = (const char*)Q_dev + ((qbs ? b * H : 0) + h0) * lat_bytes;
+      Dims d{1, h1 - h0, N, M, D};
+      if ((status = run_encode(Qc, 0, (const char*)K_dev + off, (const char*)V_dev + off, d, dt,
+                               scale, L, ws, st)) != FLARE_OK ||
+          (status = run_combine(d, dt, nullptr, nullptr, nullptr, nullptr, L, ws, st)) != FLARE_OK ||
+          (status = run_decode(Qc, 0, (const char*)K_dev + off, (char*)Y_dev + off, d, dt, scale, L,
+                               ws, st, sms)) != FLARE_OK)
+        break;
+      if ((e = cudaMemcpyAsync((char*)Y_host + off, (const char*)Y_dev + off, bytes,
+                               cudaMemcpyDeviceToHost, st)) != cudaSuccess)
+        fail(e, "Y copy");
+    }
+  }
+  cudaEventDestroy(start);
+  return status;
+}
+
 flare_status_t flare_pp_fwd(const void* Q, const void* K, const void* V, void* Y,
                             void* Q_dyn_out, int64_t B, int64_t H, int64_t N, int64_t M,
                             int64_t D, flare_dtype_t dt, float scale, float* Z_save,

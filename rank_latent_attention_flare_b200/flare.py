@@ -172,6 +172,46 @@ def flare_fwd(Q, K, V, scale: Optional[float] = None, *, save: bool = False,
     return (Y, Z, lse) if save else Y
 
 
+def flare_fwd_host(Q, K, V, scale: Optional[float] = None, *, out: Optional[torch.Tensor] = None,
+                   device_buffers=None, workspace: Optional[torch.Tensor] = None, device=None,
+                   stream=None, copy_stream=None):
+    """FLARE forward from and to host memory (flare_fwd_host): Q, K, V are
+    contiguous CPU tensors (pinned for the copies to overlap the compute),
+    and Y comes back in ``out`` (a pinned CPU tensor shaped like K, created
+    if not given).  ``device_buffers``: an optional dict of device tensors
+    "Q", "K", "V", "Y" shaped like the host ones, reused across calls.
+    Returns Y once ``stream`` is synchronised (this call does not wait)."""
+    for t in (Q, K, V, out):
+        if t is not None and (t.is_cuda or not t.is_contiguous()):
+            raise ValueError("flare_fwd_host takes contiguous host tensors")
+    if K.dim() != 4:
+        raise ValueError("K must be [B,H,N,D]")
+    B, H, N, D = K.shape
+    M = Q.shape[-2]
+    qbs = 0 if Q.dim() == 3 else H * M * D
+    dt = _dtype_code(K)
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    s = default_scale(D) if scale is None else float(scale)
+    Y = torch.empty(K.shape, dtype=K.dtype, pin_memory=True) if out is None else out
+    buf = device_buffers if device_buffers is not None else {
+        "Q": torch.empty(Q.shape, dtype=Q.dtype, device=dev),
+        **{k: torch.empty(K.shape, dtype=K.dtype, device=dev) for k in ("K", "V", "Y")}}
+    lib = _lib.load()
+    if workspace is None:
+        n = int(lib.flare_fwd_host_workspace_size(B, H, N, M, D, dt))
+        if n == 0:
+            raise FlareError(2, "flare_fwd_host_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=dev)
+    st = _stream(stream)
+    cs = _stream(copy_stream) if copy_stream is not None else st
+    _lib.check(lib.flare_fwd_host(ctypes.c_void_p(Q.data_ptr()), qbs, ctypes.c_void_p(K.data_ptr()),
+                                  ctypes.c_void_p(V.data_ptr()), ctypes.c_void_p(Y.data_ptr()),
+                                  _ptr(buf["Q"]), _ptr(buf["K"]), _ptr(buf["V"]), _ptr(buf["Y"]),
+                                  B, H, N, M, D, dt, s, _ptr(workspace), workspace.numel(), st, cs),
+               "flare_fwd_host")
+    return Y
+
+
 def flare_pp_fwd(Q, K, V, scale: Optional[float] = None, *, save: bool = False,
                  workspace: Optional[torch.Tensor] = None,
                  seq_lens: Optional[torch.Tensor] = None, stream=None):

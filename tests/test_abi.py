@@ -200,6 +200,27 @@ def test_other_entry_points_validate(lib):
 
 
 @no_gpu_only
+def test_fwd_host_validates(lib):
+    F = FAKE
+    host = ctypes.create_string_buffer(64)   # never read: validation fails first
+    hp = ctypes.cast(host, ctypes.c_void_p)
+    need = lib.flare_fwd_host_workspace_size(1, 2, 100, 32, 16, 0)
+    assert need > 0
+    assert lib.flare_fwd_host_workspace_size(1, 2, 100, 40, 16, 0) == 0   # M not a multiple of 16
+    args = dict(B=1, H=2, N=100, M=32, D=16)
+
+    def call(q=hp, y=hp, qd=_p(F), wsb=need, scale=0.25):
+        return lib.flare_fwd_host(q, 0, hp, hp, y, qd, _p(F), _p(F), _p(F), args["B"], args["H"],
+                                  args["N"], args["M"], args["D"], 0, scale, _p(F), wsb, None,
+                                  None)
+    assert call(q=None) == INVALID          # host pointers are required
+    assert call(y=None) == INVALID
+    assert call(qd=None) == INVALID         # and device buffers
+    assert call(scale=-1.0) == INVALID
+    assert call(wsb=need - 1) == WORKSPACE
+
+
+@no_gpu_only
 def test_valid_call_without_device_reports_cuda_error(lib):
     # Arguments pass validation; the first enqueue fails because there is no
     # device, which must surface as FLARE_ERR_CUDA (not a crash).
