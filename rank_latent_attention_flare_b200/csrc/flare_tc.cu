@@ -251,32 +251,59 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int half = 0; half < NH; ++half)
           tma_load_3d(Qs + half * 128 * RB, &tmQ, q_full, 0, half * 128, qz);
       }
-      int issued = 0;
-      for (int i = 0; i < (int)ntiles; ++i) {
-        const int s = i % kEncStages;
-        const uint32_t ph = (uint32_t)((i / kEncStages) & 1);
-        int stop = 0;
-        if (lane == 0) {
-          if (i >= kEncStages && !mbar_wait_sleep(&kv_empty[s], ph ^ 1)) {
-            record_error(err, kErrEncTmaWait);
-            *abort_flag = 1;
-          }
-          stop = *abort_flag;
-        }
-        if (__shfl_sync(0xffffffffu, stop, 0)) break;
+      // The offsets of tile i are loaded kNbAhead tiles before they are
+      // stored (lane l: columns l and l + 32), so the loads' latency is not
+      // on the producer's path; the loop is unrolled by kNbAhead so that
+      // each tile's values stay in fixed registers.
+      constexpr int kNbAhead = 4;
+      auto load_nb = [&](int i, float (&v)[2]) {
+        if (i >= (int)ntiles) return;
         const int64_t tok = ht.row0(tile0 + i, kEncTile);
         const int lo = ht.lo(tile0 + i, kEncTile), hi = ht.hi(tile0 + i, kEncTile);
-        float* nb = nb_ring + s * kEncTile;
-        for (int t = lane; t < kEncTile; t += 32)
-          nb[t] = (t >= lo && t < hi) ? -stats[bh * N + tok + t].x : -INFINITY;
-        __syncwarp();
-        if (lane == 0) {
-          uint8_t* kt = smem + L::KV_OFF + s * 2 * L::TILE;
-          mbar_arrive_expect_tx(&kv_full[s], 2 * L::TILE);
-          tma_load_tok<FLAT>(kt, &tmK, &kv_full[s], (int32_t)tok, bh, H);
-          tma_load_tok<FLAT>(kt + L::TILE, &tmV, &kv_full[s], (int32_t)tok, bh, H);
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int t = lane + 32 * k;
+          v[k] = (t < kEncTile && t >= lo && t < hi) ? -stats[bh * N + tok + t].x : -INFINITY;
         }
-        issued = i + 1;
+      };
+      float pre[kNbAhead][2];
+#pragma unroll
+      for (int u = 0; u < kNbAhead; ++u) load_nb(u, pre[u]);
+      int issued = 0;
+      bool stopped = false;
+      for (int i0 = 0; i0 < (int)ntiles && !stopped; i0 += kNbAhead) {
+#pragma unroll
+        for (int u = 0; u < kNbAhead; ++u) {
+          const int i = i0 + u;
+          if (i >= (int)ntiles) break;
+          const int s = i % kEncStages;
+          const uint32_t ph = (uint32_t)((i / kEncStages) & 1);
+          int stop = 0;
+          if (lane == 0) {
+            if (i >= kEncStages && !mbar_wait_sleep(&kv_empty[s], ph ^ 1)) {
+              record_error(err, kErrEncTmaWait);
+              *abort_flag = 1;
+            }
+            stop = *abort_flag;
+          }
+          if (__shfl_sync(0xffffffffu, stop, 0)) {
+            stopped = true;
+            break;
+          }
+          float* nb = nb_ring + s * kEncTile;
+          nb[lane] = pre[u][0];
+          if (lane + 32 < kEncTile) nb[lane + 32] = pre[u][1];
+          load_nb(i + kNbAhead, pre[u]);
+          __syncwarp();
+          if (lane == 0) {
+            const int64_t tok = ht.row0(tile0 + i, kEncTile);
+            uint8_t* kt = smem + L::KV_OFF + s * 2 * L::TILE;
+            mbar_arrive_expect_tx(&kv_full[s], 2 * L::TILE);
+            tma_load_tok<FLAT>(kt, &tmK, &kv_full[s], (int32_t)tok, bh, H);
+            tma_load_tok<FLAT>(kt + L::TILE, &tmV, &kv_full[s], (int32_t)tok, bh, H);
+          }
+          issued = i + 1;
+        }
       }
       if (lane == 0) {
         for (int i = (issued > kEncStages ? issued - kEncStages : 0); i < issued; ++i)
