@@ -7,7 +7,7 @@
 #include <stdio.h>
 #include <string.h>
 
-#include "flare_internal.cuh"
+#include "flare_plan.cuh"
 
 using namespace flare;
 
@@ -394,11 +394,13 @@ flare_status_t flare_bwd_ex(const void* Q, int64_t qbs, const void* K, const voi
   char* ws = (char*)workspace;
   cudaStream_t st = (cudaStream_t)stream;
   FLARE_TRY(reset_error_word(ws, st));
-  FLARE_CUDA(launch_var_plan(d, L, ws, st, sms));   // lengths: checked, work plans
+  // lengths: checked, work plans (computed inside the backward's first kernel)
+  PlanArgs plan;
+  FLARE_CUDA(launch_var_plan(d, L, ws, st, sms, &plan));
   // no gradient at padding: dK = dV = 0 there (zeroed by the backward)
   const PadZero pz = pad_zero(dK, d.dk, dV, d.dv, d, dt, (int)M);
   FLARE_CUDA(launch_bwd(Q, qbs, K, V, dY, Z_save, lse_save, dQ, dK, dV, d, dt, scale, L, ws, st,
-                        BwdPhase::ALL, nullptr, nullptr, &pz));
+                        BwdPhase::ALL, nullptr, nullptr, &pz, &plan));
   return FLARE_OK;
 }
 

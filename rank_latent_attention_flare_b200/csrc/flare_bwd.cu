@@ -14,7 +14,7 @@
 //     dQ += s dA_e K
 // Every cross-token sum goes through per-chunk partial records that are then
 // added in a fixed order, so the results are bitwise reproducible.
-#include "flare_internal.cuh"
+#include "flare_plan.cuh"
 
 namespace flare {
 namespace {
@@ -366,12 +366,17 @@ cudaError_t launch_bwd(const void* Q, int64_t qbs, const void* K, const void* V,
                        const float* Z, const float* lse, void* dQ, void* dK, void* dV,
                        const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,
                        char* ws, cudaStream_t st, BwdPhase phase, float* dz, float* dq32,
-                       const PadZero* pz) {
-  // the tensor-core backward zeroes the padding in its preparation kernel;
-  // the CUDA-core one with the standalone kernel
+                       const PadZero* pz, const PlanArgs* plan) {
+  // the tensor-core backward zeroes the padding and computes a deferred work
+  // plan in its preparation kernel; the CUDA-core one uses the standalone
+  // kernels
   if (choose_path(d.N, d.M, d.D, dt).tc_bwd)
     return launch_tc_bwd(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st, phase, dz,
-                         dq32, pz);
+                         dq32, pz, plan);
+  if (plan) {
+    const cudaError_t e = launch_plan(*plan, st);
+    if (e != cudaSuccess) return e;
+  }
 #define FLARE_BWD_T(T, DD) \
   bwd_t<T, DD>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st, phase, dz, dq32)
   cudaError_t e = (dt == FLARE_F32) ? (d.D == 16 ? FLARE_BWD_T(float, 16) : FLARE_BWD_T(float, 32))

@@ -530,9 +530,16 @@ cudaError_t launch_simt_decode(const void* Q, int64_t qbs, const void* K, const 
                                cudaStream_t st);
 // Records kErrSeqLen when a length lies outside [0, N] (lens non-NULL).
 cudaError_t launch_check_lens(const Dims& d, uint32_t* err, cudaStream_t st);
+// The arguments of a work-plan block (flare_plan.cuh).
+struct PlanArgs;
 // Checks the lengths (as launch_check_lens) and writes the work plans of a
-// tensor-core call with lengths into the workspace; returns d with them attached.
-cudaError_t launch_var_plan(Dims& d, const WsLayout& L, char* ws, cudaStream_t st, int sms);
+// tensor-core call with lengths into the workspace; returns d with them
+// attached.  With `defer` the plan kernel is not launched: *defer receives
+// its arguments (lens NULL when there is no plan), and the caller has the
+// plan computed before any kernel that reads it (launch_bwd does, by a block
+// of the backward's preparation kernel).
+cudaError_t launch_var_plan(Dims& d, const WsLayout& L, char* ws, cudaStream_t st, int sms,
+                            PlanArgs* defer = nullptr);
 // Zeroes the padding rows (n >= the batch element's length) of the token
 // tensor X0 with strides t0 and, when X1 is not NULL, of X1 (no-op when
 // d.lens is NULL).
@@ -600,7 +607,8 @@ cudaError_t launch_tc_bwd(const void* Q, int64_t qbs, const void* K, const void*
                           const void* dY, const float* Z, const float* lse, void* dQ, void* dK,
                           void* dV, const Dims& d, float scale, const WsLayout& L, char* ws,
                           cudaStream_t st, BwdPhase phase = BwdPhase::ALL, float* dz = nullptr,
-                          float* dq32 = nullptr, const PadZero* pz = nullptr);
+                          float* dq32 = nullptr, const PadZero* pz = nullptr,
+                          const PlanArgs* plan = nullptr);
 // FLARE++'s first-encode gradient on the tensor cores (bf16, M = 128,
 // D in {16, 32}): adds into dK, dV and writes dQ (sum over the batch of dZ1
 // and the encode's dQ); reuses the tensor-core backward's workspace.
@@ -620,6 +628,7 @@ cudaError_t launch_bwd(const void* Q, int64_t qbs, const void* K, const void* V,
                        const float* Z, const float* lse, void* dQ, void* dK, void* dV,
                        const Dims& d, flare_dtype_t dt, float scale, const WsLayout& L,
                        char* ws, cudaStream_t st, BwdPhase phase = BwdPhase::ALL,
-                       float* dz = nullptr, float* dq32 = nullptr, const PadZero* pz = nullptr);
+                       float* dz = nullptr, float* dq32 = nullptr, const PadZero* pz = nullptr,
+                       const PlanArgs* plan = nullptr);
 
 }  // namespace flare

@@ -51,7 +51,7 @@
 // registers (as in the forward's decode kernel).
 #include <cudaTypedefs.h>
 
-#include "flare_internal.cuh"
+#include "flare_plan.cuh"
 #include "tc_primitives.cuh"
 
 namespace flare {
@@ -546,15 +546,22 @@ __global__ void __launch_bounds__(kThr, 1)
 
 // One block per (b, h), one thread per latent m: the bf16 copy of Z (the
 // operand of Y = P Z and of dY'' Z^T) and R = max_m lse2[m], the reference
-// of the split of the encode weights; clears the head's range flag.
+// of the split of the encode weights; clears the head's range flag.  With
+// lengths, blocks past the heads zero the padding rows of dK and dV, and the
+// last block computes the work plan of the passes that follow.
 template <int D, int M>
 __global__ void __launch_bounds__(M)
     bwd_prep_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
                     __nv_bfloat16* __restrict__ zb, float* __restrict__ rref,
-                    uint32_t* __restrict__ flags, int64_t BH, const PadZero z) {
+                    uint32_t* __restrict__ flags, int64_t BH, const PadZero z,
+                    const PlanArgs plan) {
   pdl_wait();   // the previous kernel's results (programmatic dependent launch)
   pdl_trigger();
   __shared__ float red[M / 32];
+  if (plan.on() && blockIdx.x == gridDim.x - 1) {   // the work plan with lengths
+    var_plan_body<M>(plan);
+    return;
+  }
   if (blockIdx.x >= BH) {   // the padding rows of dK and dV
     const int64_t x = blockIdx.x - BH;
     zero_padding_part(z, x % z.nxb, x / z.nxb);
@@ -1727,7 +1734,7 @@ template <int D, int M, bool FLAT, bool VAR>
 cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, const void* dY,
                      const float* Z, const float* lse, void* dQ, void* dK, void* dV, const Dims& d,
                      float scale, const WsLayout& L, char* ws, cudaStream_t st, BwdPhase phase,
-                     float* dz_io, float* dq32, const PadZero* pz) {
+                     float* dz_io, float* dq32, const PadZero* pz, const PlanArgs* plan) {
   const ChunkPlan& p = L.bwd;
   const int64_t BH = d.BH();
   const int q_per_batch = qbs != 0;
@@ -1751,10 +1758,14 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
   cudaError_t e;
 
   if (phase != BwdPhase::FINISH) {
+    // with lengths, the work plan is computed by one more block
     const PadZero z = pz ? *pz : PadZero{};
-    bwd_prep_kernel<D, M><<<(unsigned)(BH + z.blocks(BH)), M, 0, st>>>(Z, lse, zb, rref, flags,
-                                                                      BH, z);
+    const PlanArgs pa = plan ? *plan : PlanArgs{};
+    const int64_t blocks = BH + z.blocks(BH) + (pa.on() ? 1 : 0);
+    bwd_prep_kernel<D, M><<<(unsigned)blocks, M, 0, st>>>(Z, lse, zb, rref, flags, BH, z, pa);
     if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+  } else if (plan) {
+    if ((e = launch_plan(*plan, st)) != cudaSuccess) return e;
   }
 
   // latent operands: M rows per head, loaded 128 rows at a time
@@ -1860,7 +1871,8 @@ cudaError_t tc_enc_bwd_t(const void* Q, const void* K, const void* V, const floa
   cudaError_t e;
 
   // bf16 Z1 and a cleared range flag (no decode, so no token can raise it)
-  bwd_prep_kernel<D, M><<<(unsigned)BH, M, 0, st>>>(Z1, lse1, zb, rref, flags, BH, PadZero{});
+  bwd_prep_kernel<D, M><<<(unsigned)BH, M, 0, st>>>(Z1, lse1, zb, rref, flags, BH, PadZero{},
+                                                    PlanArgs{});
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   bwd_mid_kernel<D, M><<<(unsigned)BH, M, 0, st>>>(nullptr, 0, nullptr, (const __nv_bfloat16*)dZ1,
                                                    Z1, lse1, dzs, (uint32_t*)aug, flags, params,
@@ -1912,10 +1924,11 @@ cudaError_t tc_bwd_dispatch(const void* Q, int64_t qbs, const void* K, const voi
                             const void* dY, const float* Z, const float* lse, void* dQ, void* dK,
                             void* dV, const Dims& d, float scale, const WsLayout& L, char* ws,
                             cudaStream_t st, BwdPhase ph, float* dz, float* dq32,
-                            const PadZero* pz) {
+                            const PadZero* pz, const PlanArgs* plan) {
   const bool flat = tok_flat(d), var = d.lens != nullptr;
-#define FLARE_TC_BWD_T(F, V_) \
-  tc_bwd_t<D, M, F, V_>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st, ph, dz, dq32, pz)
+#define FLARE_TC_BWD_T(F, V_)                                                                   \
+  tc_bwd_t<D, M, F, V_>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st, ph, dz, dq32, \
+                        pz, plan)
   if (flat) return var ? FLARE_TC_BWD_T(true, true) : FLARE_TC_BWD_T(true, false);
   return var ? FLARE_TC_BWD_T(false, true) : FLARE_TC_BWD_T(false, false);
 #undef FLARE_TC_BWD_T
@@ -1940,10 +1953,10 @@ cudaError_t launch_tc_bwd(const void* Q, int64_t qbs, const void* K, const void*
                           const void* dY, const float* Z, const float* lse, void* dQ, void* dK,
                           void* dV, const Dims& d, float scale, const WsLayout& L, char* ws,
                           cudaStream_t st, BwdPhase phase, float* dz, float* dq32,
-                          const PadZero* pz) {
+                          const PadZero* pz, const PlanArgs* plan) {
 #define FLARE_TC_BWD(D_, M_)                                                                  \
   tc_bwd_dispatch<D_, M_>(Q, qbs, K, V, dY, Z, lse, dQ, dK, dV, d, scale, L, ws, st, phase, dz, \
-                          dq32, pz)
+                          dq32, pz, plan)
   if (d.D == 32 && d.M == 128) return FLARE_TC_BWD(32, 128);
   if (d.D == 32 && d.M == 256) return FLARE_TC_BWD(32, 256);
   if (d.D == 16 && d.M == 128) return FLARE_TC_BWD(16, 128);
