@@ -28,7 +28,8 @@ struct PlanKind {
   int2* heads;      // [B H]
 };
 
-// Everything a plan block needs (lens NULL: no plan to compute).
+// Everything a plan block needs (lens NULL: no plan to compute; k0.units
+// NULL: the encode's plan is not needed, only the 128-token one is written).
 struct PlanArgs {
   const int32_t* lens = nullptr;
   int64_t B = 0, H = 0, N = 0;
@@ -97,11 +98,12 @@ __device__ void var_plan_body(const PlanArgs& a) {
   const int64_t B = a.B, H = a.H, N = a.N;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t BH = B * H;
+  const int kind0 = a.k0.units ? 0 : 1;   // the first kind to plan
   for (int64_t b = tid; b < B; b += NT)
     if (lens[b] < 0 || (int64_t)lens[b] > N) record_error(a.err, kErrSeqLen);
 
   // one warp per (kind, cap) at a time: the smallest per whose plan fits the cap
-  for (int wc = warp; wc < 2 * kPlanCaps; wc += NW) {
+  for (int wc = kind0 * kPlanCaps + warp; wc < 2 * kPlanCaps; wc += NW) {
     const int kind = wc / kPlanCaps, ci = wc % kPlanCaps;
     const PlanKind& k = kind ? a.k1 : a.k0;
     const int64_t cap = (ci + 1 < kPlanCaps) ? imin64((int64_t)(ci + 1) * k.slots, k.n) : k.n;
@@ -144,7 +146,7 @@ __device__ void var_plan_body(const PlanArgs& a) {
     }
   }
   __syncthreads();
-  if (tid < 2) {
+  if (tid < 2 && tid >= kind0) {
     int best = 0;
     for (int ci = 1; ci < kPlanCaps; ++ci)
       if (s_cost[tid][ci] < s_cost[tid][best]) best = ci;
@@ -155,7 +157,7 @@ __device__ void var_plan_body(const PlanArgs& a) {
   if (B <= kPlanWarpB) {
     // warp k scans kind k over the batch (lane b: batch element b); then
     // every thread writes heads, one (kind, head) at a time
-    if (warp < 2) {
+    if (warp < 2 && warp >= kind0) {
       const PlanKind& k = warp ? a.k1 : a.k0;
       const uint32_t cnt = lane < B ? (uint32_t)tiles_of(seq_len(lens, lane, N), k.tile) : 0u;
       const uint32_t c = units_of(cnt, (uint32_t)s_best[warp]);
@@ -171,7 +173,7 @@ __device__ void var_plan_body(const PlanArgs& a) {
       if (lane == 31) s_used[warp] = incl;
     }
     __syncthreads();
-    for (int64_t x = tid; x < 2 * BH; x += NT) {
+    for (int64_t x = kind0 * BH + tid; x < 2 * BH; x += NT) {
       const int kind = x >= BH;
       const int64_t bh = x - (kind ? BH : 0), b = bh / H, h = bh % H;
       const uint32_t c = s_c[kind][b];
@@ -182,8 +184,8 @@ __device__ void var_plan_body(const PlanArgs& a) {
     // each thread taking a contiguous run of batch elements
     const int64_t run = (B + NT - 1) / NT;
     const int64_t b0 = imin64((int64_t)tid * run, B), b1 = imin64(b0 + run, B);
-    int64_t mine[2] = {0, 0}, incl[2];
-    for (int kind = 0; kind < 2; ++kind) {
+    int64_t mine[2] = {0, 0}, incl[2] = {0, 0};
+    for (int kind = kind0; kind < 2; ++kind) {
       const PlanKind& k = kind ? a.k1 : a.k0;
       for (int64_t b = b0; b < b1; ++b)
         mine[kind] += H * units_of((uint32_t)tiles_of(seq_len(lens, b, N), k.tile),
@@ -196,7 +198,7 @@ __device__ void var_plan_body(const PlanArgs& a) {
       if (lane == 31) s_scan[kind][warp] = incl[kind];
     }
     __syncthreads();
-    if (warp < 2) {
+    if (warp < 2 && warp >= kind0) {
       const int64_t t = lane < NW ? s_scan[warp][lane] : 0;
       int64_t ti = t;
       for (int o = 1; o < 32; o <<= 1) {
@@ -207,7 +209,7 @@ __device__ void var_plan_body(const PlanArgs& a) {
       if (lane == NW - 1) s_used[warp] = ti;
     }
     __syncthreads();
-    for (int kind = 0; kind < 2; ++kind) {
+    for (int kind = kind0; kind < 2; ++kind) {
       const PlanKind& k = kind ? a.k1 : a.k0;
       const uint32_t per = (uint32_t)s_best[kind];
       int64_t first = s_scan[kind][warp] + incl[kind] - mine[kind];
@@ -221,7 +223,7 @@ __device__ void var_plan_body(const PlanArgs& a) {
   }
   __syncthreads();
   // the units past the plan's stay empty
-  for (int kind = 0; kind < 2; ++kind) {
+  for (int kind = kind0; kind < 2; ++kind) {
     const PlanKind& k = kind ? a.k1 : a.k0;
     for (int64_t u = s_used[kind] + tid; u < k.n; u += NT) k.units[u] = make_int4(-1, 0, 0, 0);
   }

@@ -547,8 +547,8 @@ __global__ void __launch_bounds__(kThr, 1)
 // One block per (b, h), one thread per latent m: the bf16 copy of Z (the
 // operand of Y = P Z and of dY'' Z^T) and R = max_m lse2[m], the reference
 // of the split of the encode weights; clears the head's range flag.  With
-// lengths, blocks past the heads zero the padding rows of dK and dV, and the
-// last block computes the work plan of the passes that follow.
+// lengths, blocks past the heads zero the padding rows of dK and dV, and one
+// more block (block 0) computes the work plan of the passes that follow.
 template <int D, int M>
 __global__ void __launch_bounds__(M)
     bwd_prep_kernel(const float* __restrict__ Z, const float* __restrict__ lse,
@@ -558,16 +558,19 @@ __global__ void __launch_bounds__(M)
   pdl_wait();   // the previous kernel's results (programmatic dependent launch)
   pdl_trigger();
   __shared__ float red[M / 32];
-  if (plan.on() && blockIdx.x == gridDim.x - 1) {   // the work plan with lengths
+  // block 0 computes the work plan with lengths (scheduled first, it runs
+  // beside all the others)
+  if (plan.on() && blockIdx.x == 0) {
     var_plan_body<M>(plan);
     return;
   }
-  if (blockIdx.x >= BH) {   // the padding rows of dK and dV
-    const int64_t x = blockIdx.x - BH;
+  const int64_t bx = (int64_t)blockIdx.x - (plan.on() ? 1 : 0);
+  if (bx >= BH) {   // the padding rows of dK and dV
+    const int64_t x = bx - BH;
     zero_padding_part(z, x % z.nxb, x / z.nxb);
     return;
   }
-  const int64_t bh = blockIdx.x;
+  const int64_t bh = bx;
   const int m = threadIdx.x;
   const int64_t row = bh * M + m;
 #pragma unroll
@@ -1758,9 +1761,11 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
   cudaError_t e;
 
   if (phase != BwdPhase::FINISH) {
-    // with lengths, the work plan is computed by one more block
+    // with lengths, the work plan is computed by one more block (M = 128
+    // reads the 128-token plan only)
     const PadZero z = pz ? *pz : PadZero{};
-    const PlanArgs pa = plan ? *plan : PlanArgs{};
+    PlanArgs pa = plan ? *plan : PlanArgs{};
+    if (M == kM) pa.k0.units = nullptr;
     const int64_t blocks = BH + z.blocks(BH) + (pa.on() ? 1 : 0);
     bwd_prep_kernel<D, M><<<(unsigned)blocks, M, 0, st>>>(Z, lse, zb, rref, flags, BH, z, pa);
     if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
