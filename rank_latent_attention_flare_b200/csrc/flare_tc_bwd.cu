@@ -592,14 +592,18 @@ __global__ void __launch_bounds__(M)
   }
 }
 
-// One block per (b, h), one thread per latent m.  dZ = sum of the chunk
-// partials (fixed order; the work plan's head table locates them when given), lse2 = lse log2(e); R = max lse2 over the head;
-// f = 2^(R - lse2) when the head's lse2 spread is at most kSpreadMax and no
-// token of it lies more than kRowRangeMax below R (else f = 1 and the exact
-// form); the bf16 operand dZ'' = f dZ; the extra K-step row: -dZ'' . Z
-// (= -f delta_e) as three bf16 terms, then zeros.
+// One block per (b, h), kMidLanes(M) threads per latent m, each taking D /
+// lanes of its columns.  dZ = sum of the chunk partials (fixed order; the
+// work plan's head table locates them when given), lse2 = lse log2(e);
+// R = max lse2 over the head; f = 2^(R - lse2) when the head's lse2 spread
+// is at most kSpreadMax and no token of it lies more than kRowRangeMax below
+// R (else f = 1 and the exact form); the bf16 operand dZ'' = f dZ; the extra
+// K-step row: -dZ'' . Z (= -f delta_e) as three bf16 terms, then zeros.
+constexpr int kMidThreads = 512;
+constexpr int mid_lanes(int M) { return kMidThreads / M; }   // 4 (M = 128) or 2 (M = 256)
+
 template <int D, int M>
-__global__ void __launch_bounds__(M)
+__global__ void __launch_bounds__(kMidThreads)
     bwd_mid_kernel(const float* __restrict__ dz_part, int chunks, const int2* __restrict__ heads,
                    const __nv_bfloat16* __restrict__ dz_direct, const float* __restrict__ Z,
                    const float* __restrict__ lse, __nv_bfloat16* __restrict__ dzs,
@@ -607,43 +611,45 @@ __global__ void __launch_bounds__(M)
                    float2* __restrict__ params, float* __restrict__ lse2_out) {
   pdl_wait();   // the previous kernel's results (programmatic dependent launch)
   pdl_trigger();
-  __shared__ float red_max[M / 32], red_min[M / 32];
+  constexpr int LN = mid_lanes(M);
+  constexpr int DL = D / LN;                 // columns of this thread: 4, 8 or 16
+  constexpr int NF = DL <= 8 ? 4 : 2;        // partials whose loads are in flight at once
+  static_assert(DL % 4 == 0 && M * LN == kMidThreads, "float4 columns, whole rows per block");
+  __shared__ float red_max[kMidThreads / 32], red_min[kMidThreads / 32];
   const int64_t bh = blockIdx.x;
-  const int m = threadIdx.x;
+  const int m = threadIdx.x / LN, q = threadIdx.x % LN;
   const int64_t row = bh * M + m;
-  float dz[D];
+  const int d0 = q * DL;
+  float dz[DL];
 #pragma unroll
-  for (int d = 0; d < D; ++d) dz[d] = 0.f;
+  for (int d = 0; d < DL; ++d) dz[d] = 0.f;
   if (dz_direct) {   // FLARE++'s first encode: dZ1 = dQ_dyn
 #pragma unroll
-    for (int d = 0; d < D; ++d) dz[d] = __bfloat162float(dz_direct[row * D + d]);
+    for (int d = 0; d < DL; ++d) dz[d] = __bfloat162float(dz_direct[row * D + d0 + d]);
   }
   const int2 hs = head_slots(heads, bh, chunks);
-  // two partials' loads in flight at a time, added in partial order
-  for (int k = 0; k < hs.y; k += 2) {
-    const float4* p = reinterpret_cast<const float4*>(dz_part + (((int64_t)hs.x + k) * M + m) * D);
-    const float4* p2 = p + (int64_t)M * D / 4;
-    const bool two = k + 1 < hs.y;
-    float4 v[D / 4], v2[D / 4];
+  // NF partials' loads in flight at a time, added in partial order
+  for (int k = 0; k < hs.y; k += NF) {
+    float4 v[NF][DL / 4];
 #pragma unroll
-    for (int d = 0; d < D / 4; ++d) {
-      v[d] = p[d];
-      if (two) v2[d] = p2[d];
+    for (int j = 0; j < NF; ++j) {
+      const float4* p =
+          reinterpret_cast<const float4*>(dz_part + (((int64_t)hs.x + k + j) * M + m) * D + d0);
+      if (k + j < hs.y) {
+#pragma unroll
+        for (int d = 0; d < DL / 4; ++d) v[j][d] = p[d];
+      }
     }
 #pragma unroll
-    for (int d = 0; d < D / 4; ++d) {
-      dz[4 * d] += v[d].x;
-      dz[4 * d + 1] += v[d].y;
-      dz[4 * d + 2] += v[d].z;
-      dz[4 * d + 3] += v[d].w;
-    }
-    if (two) {
+    for (int j = 0; j < NF; ++j) {
+      if (k + j < hs.y) {
 #pragma unroll
-      for (int d = 0; d < D / 4; ++d) {
-        dz[4 * d] += v2[d].x;
-        dz[4 * d + 1] += v2[d].y;
-        dz[4 * d + 2] += v2[d].z;
-        dz[4 * d + 3] += v2[d].w;
+        for (int d = 0; d < DL / 4; ++d) {
+          dz[4 * d] += v[j][d].x;
+          dz[4 * d + 1] += v[j][d].y;
+          dz[4 * d + 2] += v[j][d].z;
+          dz[4 * d + 3] += v[j][d].w;
+        }
       }
     }
   }
@@ -654,14 +660,14 @@ __global__ void __launch_bounds__(M)
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
   }
-  if ((m & 31) == 0) {
-    red_max[m >> 5] = mx;
-    red_min[m >> 5] = mn;
+  if ((threadIdx.x & 31) == 0) {
+    red_max[threadIdx.x >> 5] = mx;
+    red_min[threadIdx.x >> 5] = mn;
   }
   __syncthreads();
   float R = red_max[0], lo = red_min[0];
 #pragma unroll
-  for (int k = 1; k < M / 32; ++k) {
+  for (int k = 1; k < kMidThreads / 32; ++k) {
     R = fmaxf(R, red_max[k]);
     lo = fminf(lo, red_min[k]);
   }
@@ -669,10 +675,10 @@ __global__ void __launch_bounds__(M)
   const float f = fast ? exp2f(R - l2) : 1.f;
   // delta_e is taken with the bf16 operand dZ'' that the tensor cores use,
   // so dPe'' = V dZ''^T - dZ'' . Z vanishes exactly where V = Z.
-  float zr[D];
+  float zr[DL];
 #pragma unroll
-  for (int d = 0; d < D; d += 4) {
-    const float4 zv = *reinterpret_cast<const float4*>(Z + row * D + d);
+  for (int d = 0; d < DL; d += 4) {
+    const float4 zv = *reinterpret_cast<const float4*>(Z + row * D + d0 + d);
     zr[d] = zv.x;
     zr[d + 1] = zv.y;
     zr[d + 2] = zv.z;
@@ -680,25 +686,31 @@ __global__ void __launch_bounds__(M)
   }
   float de = 0.f;
 #pragma unroll
-  for (int d = 0; d < D; d += 2) {
+  for (int d = 0; d < DL; d += 2) {
     const uint32_t pr = pack_bf16(f * dz[d], f * dz[d + 1]);
-    *reinterpret_cast<uint32_t*>(dzs + row * D + d) = pr;
+    *reinterpret_cast<uint32_t*>(dzs + row * D + d0 + d) = pr;
     de = fmaf(bf_lo(pr), zr[d], de);
     de = fmaf(bf_hi(pr), zr[d + 1], de);
   }
-  const float x = -de;
-  const __nv_bfloat16 b0 = __float2bfloat16_rn(x);
-  const float r1 = x - __bfloat162float(b0);
-  const __nv_bfloat16 b1 = __float2bfloat16_rn(r1);
-  const float r2 = r1 - __bfloat162float(b1);
-  const __nv_bfloat16 b2 = __float2bfloat16_rn(r2);
-  uint32_t* a = aug + row * 8;   // 16 bf16
-  a[0] = (uint32_t)__bfloat16_as_ushort(b0) | ((uint32_t)__bfloat16_as_ushort(b1) << 16);
-  a[1] = (uint32_t)__bfloat16_as_ushort(b2);
+  // the row's lanes (adjacent threads) add their parts pairwise: every lane
+  // ends with the same sum
 #pragma unroll
-  for (int k = 2; k < 8; ++k) a[k] = 0u;
-  lse2_out[row] = l2;
-  if (m == 0) params[bh] = make_float2(R, fast ? 1.f : 0.f);
+  for (int o = 1; o < LN; o <<= 1) de += __shfl_xor_sync(0xffffffffu, de, o);
+  if (q == 0) {
+    const float x = -de;
+    const __nv_bfloat16 b0 = __float2bfloat16_rn(x);
+    const float r1 = x - __bfloat162float(b0);
+    const __nv_bfloat16 b1 = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(b1);
+    const __nv_bfloat16 b2 = __float2bfloat16_rn(r2);
+    uint32_t* a = aug + row * 8;   // 16 bf16
+    a[0] = (uint32_t)__bfloat16_as_ushort(b0) | ((uint32_t)__bfloat16_as_ushort(b1) << 16);
+    a[1] = (uint32_t)__bfloat16_as_ushort(b2);
+#pragma unroll
+    for (int k = 2; k < 8; ++k) a[k] = 0u;
+    lse2_out[row] = l2;
+    if (m == 0) params[bh] = make_float2(R, fast ? 1.f : 0.f);
+  }
 }
 
 // ============================================================== pass B
@@ -1813,9 +1825,9 @@ cudaError_t tc_bwd_t(const void* Q, int64_t qbs, const void* K, const void* V, c
 
   // dZ: the chunk partials, or (FINISH) the sum over the shards as one partial
   const bool fin = phase == BwdPhase::FINISH;
-  bwd_mid_kernel<D, M><<<(unsigned)BH, M, 0, st>>>(fin ? dz_io : dzp, fin ? 1 : zchunks,
-                                                   fin ? nullptr : zheads, nullptr, Z, lse, dzs,
-                                                   (uint32_t*)aug, flags, params, lse2);
+  bwd_mid_kernel<D, M><<<(unsigned)BH, kMidThreads, 0, st>>>(
+      fin ? dz_io : dzp, fin ? 1 : zchunks, fin ? nullptr : zheads, nullptr, Z, lse, dzs,
+      (uint32_t*)aug, flags, params, lse2);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
   // each head runs in exactly one of the two pass-B kernels (params.y)
@@ -1879,9 +1891,9 @@ cudaError_t tc_enc_bwd_t(const void* Q, const void* K, const void* V, const floa
   bwd_prep_kernel<D, M><<<(unsigned)BH, M, 0, st>>>(Z1, lse1, zb, rref, flags, BH, PadZero{},
                                                     PlanArgs{});
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
-  bwd_mid_kernel<D, M><<<(unsigned)BH, M, 0, st>>>(nullptr, 0, nullptr, (const __nv_bfloat16*)dZ1,
-                                                   Z1, lse1, dzs, (uint32_t*)aug, flags, params,
-                                                   lse2);
+  bwd_mid_kernel<D, M><<<(unsigned)BH, kMidThreads, 0, st>>>(
+      nullptr, 0, nullptr, (const __nv_bfloat16*)dZ1, Z1, lse1, dzs, (uint32_t*)aug, flags, params,
+      lse2);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
 
   // the decode operands' maps point at V: valid tiles that are never used
