@@ -238,11 +238,12 @@ FLARE_API flare_status_t flare_pp_bwd(const void* Q, const void* K, const void* 
  * to it and reported: flare_device_status then returns
  * FLARE_ERR_INVALID_ARG with detail 0x601.  NULL means every sequence has
  * N tokens.  flare_pp_bwd_ex / flare_bwd_ex must get the lengths their
- * forward used.  On the tensor-core path a call with lengths first runs a
- * one-CTA kernel that reads them and writes a work plan into the
- * workspace: each head's valid tiles split into near-equal units, one CTA
- * each, so that short sequences take less time instead of leaving SMs
- * idle (no host synchronisation; the workspace size already covers it).
+ * forward used.  On the tensor-core path a call with lengths first has one
+ * block read them and write a work plan into the workspace (a kernel of
+ * its own in the forward, a block of the first kernel in the backward):
+ * each head's valid tiles split into near-equal units, one CTA each, so
+ * that short sequences take less time instead of leaving SMs idle (no host
+ * synchronisation; the workspace size already covers it).
  *
  * With strides == NULL and seq_lens == NULL each call is the plain entry
  * point (which is implemented that way).
