@@ -353,7 +353,7 @@ struct Dims {
   Tok dy = contig(), dk = contig(), dv = contig();  // dY, dK, dV
   const int32_t* lens = nullptr;   // device [B]: valid tokens per batch element (NULL: N)
   // With lengths on the tensor-core path, the length-proportional work plans
-  // that the plan kernel writes into the workspace (NULL otherwise): one for
+  // that a plan block writes into the workspace (NULL otherwise): one for
   // the 48-token encode, one for the 128-token kernels (decode, backward).
   VarPlan venc, vtok;
   int64_t BH() const { return B * H; }
